@@ -1,0 +1,235 @@
+"""Seeded synthetic workloads for the CSA / HCA hot path.
+
+This module only draws random inputs and lays them out in the library's buffer formats.
+It holds none of the method's arithmetic (no pooling, normalisation, RoPE, scoring,
+selection or attention); both the CUDA library's tests/benchmarks and the CPU oracle
+consume the tensors it returns.
+
+Distributions follow the workloads the method is specified on: raw per-token KV and gate
+logits ~N(0,1) stored as bf16, positional bias ~N(0, 0.1) fp32, attention-sink logits
+~N(0,1) per head, queries ~N(0,1) bf16, indexer heads in FP8 E4M3 -- either
+integer-valued in [-3, 3] with unit scales (exact-arithmetic runs) or N(0,1) quantised
+with one scale per 1x128 row -- and per-head indexer weights ~U(0,1).
+
+Random numbers come from ``torch.Generator`` seeded per workload, on the device the
+tensors are made on; a given (workload, seed, device) always yields the same tensors.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+E4M3 = torch.float8_e4m3fn
+
+
+@dataclasses.dataclass
+class Workload:
+    """Inputs of one hot-path pass.  Integer offsets are int64, positions int32."""
+    name: str
+    B: int                      # sequences
+    T: torch.Tensor             # [B] int64 context lengths (host tensor)
+    D: int                      # head dim (RoPE on the last 64)
+    H: int                      # query heads
+    m: int                      # compression ratio used for visibility (4 CSA, 128 HCA)
+    span: int                   # tokens pooled per entry (2m CSA, m' HCA)
+    W: int                      # sliding window
+    fmt: int                    # entry storage format: 0 bf16, 1 = 576-dim fp8 + bf16 rope
+    # raw per-token data: position p of sequence b sits in row kv_off[b] + p - kv_pos0[b]
+    kv: torch.Tensor            # [rows, D] bf16
+    gate: torch.Tensor          # [rows, D] bf16
+    kv_off: torch.Tensor        # [B] int64
+    kv_pos0: torch.Tensor       # [B] int64
+    bias: torch.Tensor          # [span, D] fp32
+    # compressed entries: entry i of sequence b is row ent_off[b] + i
+    ent_off: torch.Tensor       # [B] int64
+    n_ent: torch.Tensor         # [B] int64 = floor(T_b / m)
+    # queries
+    q_seq: torch.Tensor         # [Q] int32
+    q_pos: torch.Tensor         # [Q] int32
+    q: torch.Tensor             # [Q, H, D] bf16
+    sink: torch.Tensor          # [H] fp32
+    # lightning indexer (CSA only; None for HCA)
+    H_I: int = 0
+    d_I: int = 0
+    k: int = 0
+    kI: Optional[torch.Tensor] = None   # [ent_rows, d_I] uint8 (e4m3 codes)
+    ks: Optional[torch.Tensor] = None   # [ent_rows] fp32
+    qI: Optional[torch.Tensor] = None   # [Q, H_I, d_I] uint8
+    qs: Optional[torch.Tensor] = None   # [Q, H_I] fp32
+    w: Optional[torch.Tensor] = None    # [Q, H_I] fp32
+    theta: float = 10000.0
+    eps: float = 1e-6
+
+    @property
+    def Q(self) -> int:
+        return int(self.q_seq.numel())
+
+    @property
+    def ent_rows(self) -> int:
+        return int(self.n_ent.sum())
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    def to(self, device) -> "Workload":
+        f = {}
+        for fld in dataclasses.fields(self):
+            v = getattr(self, fld.name)
+            if isinstance(v, torch.Tensor) and fld.name != "T":
+                v = v.to(device)
+            f[fld.name] = v
+        return Workload(**f)
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _bf16_normal(shape, g, device, std=1.0):
+    return (torch.randn(shape, generator=g, device=device) * std).to(torch.bfloat16)
+
+
+def fp8_integer(shape, g, device, lo=-3, hi=3):
+    """E4M3 codes of integers drawn uniformly from [lo, hi] (exact in e4m3)."""
+    x = torch.randint(lo, hi + 1, shape, generator=g, device=device).to(torch.float32)
+    return x.to(E4M3).view(torch.uint8)
+
+
+def fp8_rows_from_normal(rows, cols, g, device):
+    """N(0,1) rows quantised to E4M3 with one fp32 scale per row (amax / 448)."""
+    x = torch.randn((rows, cols), generator=g, device=device)
+    amax = x.abs().amax(dim=1).clamp_min(1e-12)
+    scale = (amax / 448.0).to(torch.float32)
+    codes = (x / scale[:, None]).clamp(-448.0, 448.0).to(E4M3).view(torch.uint8)
+    return codes, scale
+
+
+def random_entries(n, fmt, D, g, device):
+    """Random stored entry rows (used where entries are generated directly, e.g. for
+    neighbour sequences).  fmt 0: bf16 N(0,1).  fmt 1 (D=576): e4m3 codes of N(0,1)
+    quantised per 128 channels, the 4 fp32 scales, then 64 bf16 N(0,1) values."""
+    if fmt == 0:
+        return _bf16_normal((n, D), g, device).view(torch.uint8).reshape(n, 2 * D)
+    assert fmt == 1 and D == 576
+    x = torch.randn((n, 4, 128), generator=g, device=device)
+    amax = x.abs().amax(dim=2).clamp_min(1e-12)
+    scale = (amax / 448.0).to(torch.float32)
+    codes = (x / scale[:, :, None]).clamp(-448.0, 448.0).to(E4M3).view(torch.uint8)
+    rope = _bf16_normal((n, 64), g, device)
+    row = torch.empty((n, 656), dtype=torch.uint8, device=device)
+    row[:, :512] = codes.reshape(n, 512)
+    row[:, 512:528] = scale.view(torch.uint8).reshape(n, 16)
+    row[:, 528:] = rope.view(torch.uint8).reshape(n, 128)
+    return row
+
+
+def _offsets(lengths: torch.Tensor) -> torch.Tensor:
+    off = torch.zeros(lengths.numel(), dtype=torch.int64)
+    if lengths.numel() > 1:
+        off[1:] = torch.cumsum(lengths[:-1], 0)
+    return off
+
+
+def make_workload(name: str, *, B: int, T, D: int, H: int, m: int, span: int, W: int = 128,
+                  fmt: int = 0, H_I: int = 0, d_I: int = 0, k: int = 0,
+                  indexer: str = "int", keep_raw: Optional[int] = None,
+                  queries: str = "decode", n_new: int = 0, seed: int = 0,
+                  device="cpu") -> Workload:
+    """Draw one workload.
+
+    T: int or list of context lengths.  queries="decode": one query per sequence at
+    position T_b - 1.  queries="prefill": the last ``n_new`` positions of every sequence.
+    keep_raw: store only the last ``keep_raw`` raw tokens of each sequence (None = all).
+    indexer: "int" (integers in [-3,3], unit scales) or "fp8" (N(0,1), 1x128 scales).
+    """
+    g = _gen(seed, device)
+    T = torch.as_tensor(T if not isinstance(T, int) else [T] * B, dtype=torch.int64)
+    assert T.numel() == B
+    keep = T.clone() if keep_raw is None else torch.minimum(T, torch.tensor(keep_raw))
+    kv_pos0 = T - keep
+    kv_off = _offsets(keep)
+    rows = int(keep.sum())
+    kv = _bf16_normal((rows, D), g, device)
+    gate = _bf16_normal((rows, D), g, device)
+    bias = torch.randn((span, D), generator=g, device=device) * 0.1
+    n_ent = T // m
+    ent_off = _offsets(n_ent)
+    if queries == "decode":
+        q_seq = torch.arange(B, dtype=torch.int32)
+        q_pos = (T - 1).to(torch.int32)
+    else:
+        q_seq = torch.arange(B, dtype=torch.int32).repeat_interleave(n_new)
+        q_pos = torch.cat([torch.arange(int(t) - n_new, int(t), dtype=torch.int32) for t in T])
+    Q = q_seq.numel()
+    q = _bf16_normal((Q, H, D), g, device)
+    sink = torch.randn((H,), generator=g, device=device)
+    wl = Workload(name=name, B=B, T=T, D=D, H=H, m=m, span=span, W=W, fmt=fmt, kv=kv,
+                  gate=gate, kv_off=kv_off.to(device), kv_pos0=kv_pos0.to(device), bias=bias,
+                  ent_off=ent_off.to(device), n_ent=n_ent.to(device),
+                  q_seq=q_seq.to(device), q_pos=q_pos.to(device), q=q, sink=sink)
+    if H_I:
+        er = int(n_ent.sum())
+        if indexer == "int":
+            kI = fp8_integer((er, d_I), g, device)
+            ks = torch.ones(er, dtype=torch.float32, device=device)
+            qI = fp8_integer((Q, H_I, d_I), g, device)
+            qs = torch.ones((Q, H_I), dtype=torch.float32, device=device)
+        else:
+            kI, ks = fp8_rows_from_normal(er, d_I, g, device)
+            qI, qs = fp8_rows_from_normal(Q * H_I, d_I, g, device)
+            qI = qI.reshape(Q, H_I, d_I)
+            qs = qs.reshape(Q, H_I)
+        w = torch.rand((Q, H_I), generator=g, device=device)
+        wl.H_I, wl.d_I, wl.k = H_I, d_I, k
+        wl.kI, wl.ks, wl.qI, wl.qs, wl.w = kI, ks, qI, qs, w
+    return wl
+
+
+def jittered_lengths(B: int, T: int, jitter: int, seed: int) -> list:
+    g = torch.Generator().manual_seed(int(seed) + 7919)
+    return (T + torch.randint(-jitter, jitter + 1, (B,), generator=g)).tolist()
+
+
+# ---- the named workloads -------------------------------------------------------------
+def csa_decode_4k(device="cpu", seed=0, indexer="int") -> Workload:
+    """CSA single layer, decode, batch 1, 4096 tokens -> 1024 entries; indexer 4 heads x 64,
+    top-64; 16 query heads, head dim 128; window 128."""
+    return make_workload("csa_decode_4k_b1", B=1, T=4096, D=128, H=16, m=4, span=8, W=128,
+                         H_I=4, d_I=64, k=64, indexer=indexer, seed=seed, device=device)
+
+
+def csa_decode_128k(device="cpu", seed=0, indexer="int", B=32, keep_raw=None) -> Workload:
+    """CSA decode, 32 sequences of 131072 +- 1024 tokens; 64 heads, head dim 128; indexer
+    64 heads x 128 FP8; top-512; window 128."""
+    return make_workload("csa_decode_128k_b32", B=B, T=jittered_lengths(B, 131072, 1024, seed),
+                         D=128, H=64, m=4, span=8, W=128, H_I=64, d_I=128, k=512,
+                         indexer=indexer, keep_raw=keep_raw, seed=seed, device=device)
+
+
+def hca_decode_1m(device="cpu", seed=0, B=16, keep_raw=None) -> Workload:
+    """HCA decode, 16 sequences of 1,048,576 tokens -> 8192 entries each; dense attention
+    plus window 128; 64 heads, head dim 128."""
+    return make_workload("hca_decode_1m_b16", B=B, T=1 << 20, D=128, H=64, m=128, span=128,
+                         W=128, keep_raw=keep_raw, seed=seed, device=device)
+
+
+def csa_prefill_64k(device="cpu", seed=0, indexer="int") -> Workload:
+    """CSA prefill chunk: 8192 new query tokens after 65536 prior tokens (18432 entries);
+    indexer 64 x 128 FP8, top-1024; 64 heads, head dim 128; window 128."""
+    return make_workload("csa_prefill_8k_on_64k", B=1, T=65536 + 8192, D=128, H=64, m=4,
+                         span=8, W=128, H_I=64, d_I=128, k=1024, indexer=indexer,
+                         queries="prefill", n_new=8192, seed=seed, device=device)
+
+
+def csa_decode_1m_fp8(device="cpu", seed=0, indexer="int", B=8, keep_raw=None) -> Workload:
+    """CSA decode at 1,048,576 tokens, batch 8, top-1024, 128 query heads, entries of head
+    dim 576 stored as 512 FP8 (1x128 scales) + 64 BF16 RoPE dims; indexer 64 x 128 FP8."""
+    return make_workload("csa_decode_1m_b8_fp8", B=B, T=1 << 20, D=576, H=128, m=4, span=8,
+                         W=128, fmt=1, H_I=64, d_I=128, k=1024, indexer=indexer,
+                         keep_raw=keep_raw, seed=seed, device=device)
