@@ -1,0 +1,385 @@
+"""Benchmark of the CSA / HCA decode hot path on B200.
+
+One step = one pass of the whole hot path over one batch: compress each sequence's newest
+entry, lightning indexer + top-k (CSA), sparse (CSA) or dense (HCA) attention.  The
+default workload is CSA decode with 32 sequences of 131072 +- 1024 tokens, 64 query heads
+of dim 128, a 64 x 128 FP8 indexer and top-512.  Inputs are synthetic and seeded; the
+compressed cache is built with the library itself before timing.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs its own batch (sequences
+shard across GPUs with no data-path collective; weak scaling); the timed region is
+bracketed by barriers and device syncs and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "CSA/HCA decode query-tokens/s at 128K–1M ctx; % of HBM roofline"
+UNIT = "query-tokens/s"
+
+WORKLOADS = {
+    "csa_decode_128k_b32": dict(kind="csa", B=32, T=131072, jitter=1024, D=128, H=64, H_I=64,
+                                d_I=128, k=512, fmt=0),
+    "hca_decode_1m_b16": dict(kind="hca", B=16, T=1 << 20, jitter=0, D=128, H=64, fmt=0),
+    "csa_decode_1m_b8_fp8": dict(kind="csa", B=8, T=1 << 20, jitter=0, D=576, H=128, H_I=64,
+                                 d_I=128, k=1024, fmt=1),
+}
+
+
+def _peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def make_workload(name: str, rank: int, device):
+    from long_context_compressed_04_b200 import synth
+    c = WORKLOADS[name]
+    T = synth.jittered_lengths(c["B"], c["T"], c["jitter"], 1000 + rank) if c["jitter"] else c["T"]
+    if c["kind"] == "csa":
+        return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
+                                   fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
+                                   indexer="fp8", seed=rank, device=device)
+    return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=128, span=128, W=128,
+                               fmt=c["fmt"], seed=rank, device=device)
+
+
+def algorithmic_bytes(wl):
+    """Bytes the method must move per step (each counted once): indexer keys + scales of
+    every visible entry, the selected (or all, for HCA) entry rows, the window's raw rows,
+    q, out and the index sets; plus the newest block's raw rows for compression."""
+    from long_context_compressed_04_b200 import csa_entry_row_bytes
+    n_vis = ((wl.q_pos.cpu().to(torch.int64) + 1) // wl.m)
+    rb = csa_entry_row_bytes(wl.fmt, wl.D)
+    win = torch.clamp(wl.q_pos.cpu().to(torch.int64) + 1, max=wl.W)
+    qo = wl.Q * wl.H * wl.D * 2 * 2
+    comp = wl.B * (wl.span * wl.D * 2 * 2 + rb)
+    if wl.H_I:
+        keys = int(n_vis.sum()) * (wl.d_I + 4) + wl.Q * wl.H_I * (wl.d_I + 8)
+        sel = int(torch.clamp(n_vis, max=wl.k).sum()) * rb + wl.Q * wl.k * 4
+    else:
+        keys = 0
+        sel = int(n_vis.sum()) * rb
+    total = keys + sel + int(win.sum()) * wl.D * 2 + qo + comp
+    return total, keys
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_index_for_smi(dev: int) -> str:
+    try:
+        props = torch.cuda.get_device_properties(dev)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            dom = getattr(props, "pci_domain_id", 0)
+            dv = getattr(props, "pci_device_id", 0)
+            return f"{dom:08x}:{bus:02x}:{dv:02x}.0"
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        return vis.split(",")[dev]
+    return str(dev)
+
+
+CPU_SAMPLE_SEQS = {"csa_decode_128k_b32": 32, "hca_decode_1m_b16": 16, "csa_decode_1m_b8_fp8": 2}
+
+
+def cpu_baseline(name: str, n_seq: int | None = None):
+    """The oracle, as it stands, on a bounded sample of the workload: n_seq sequences of
+    the workload's shape, one decode step each (compress the newest entry, score every
+    visible entry and select, attend).  The sample's cache rows are synthetic stored-format
+    rows (untimed set-up); the timed step recompresses the newest entry itself."""
+    n_seq = n_seq or CPU_SAMPLE_SEQS[name]
+    import numpy as np
+    import oracle
+    from oracle import workload as _orc
+    from long_context_compressed_04_b200 import synth
+
+    c = WORKLOADS[name]
+    T = synth.jittered_lengths(n_seq, c["T"], c["jitter"], 99) if c["jitter"] else [c["T"]] * n_seq
+    if c["kind"] == "csa":
+        wl = synth.make_workload(name, B=n_seq, T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
+                                 fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
+                                 indexer="fp8", keep_raw=256, seed=7)
+    else:
+        wl = synth.make_workload(name, B=n_seq, T=T, D=c["D"], H=c["H"], m=128, span=128, W=128,
+                                 fmt=c["fmt"], keep_raw=256, seed=7)
+    # cache of entries for the sample (the raw store keeps only the tail, so the cache is
+    # filled with stored-format rows drawn directly; the step recompresses the newest one)
+    g = torch.Generator().manual_seed(5)
+    rows = synth.random_entries(max(wl.ent_rows, 1), wl.fmt, wl.D, g, "cpu").numpy().copy()
+    n = _orc.i64(wl.n_ent)
+    item_seq = np.arange(wl.B, dtype=np.int32)
+    item_ent = (n - 1).astype(np.int32)
+    t0 = time.perf_counter()
+    oracle.compress(_orc.u16(wl.kv), _orc.u16(wl.gate), _orc.f32(wl.bias), _orc.i64(wl.kv_off),
+                    _orc.i64(wl.kv_pos0), _orc.i64(wl.ent_off), item_seq, item_ent, m=wl.m,
+                    span=wl.span, D=wl.D, fmt=wl.fmt, entries=rows)
+    idx = _orc.indexer(wl, want_scores=False) if wl.H_I else None
+    _orc.attention(wl, rows, idx)
+    dt = time.perf_counter() - t0
+    return {"value": wl.Q / dt, "unit": UNIT, "cores": min(oracle.num_threads(), wl.Q),
+            "kind": "oracle",
+            "sample": f"{wl.Q} decode queries of {name} (one step each: newest-entry compress, "
+                      f"indexer over all visible entries, top-k, attention), {dt:.2f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    samples = []
+    for _ in range(args.warmup):
+        cpu_baseline(args.workload, n_seq=1)
+    for _ in range(args.steps):
+        samples.append(cpu_baseline(args.workload, n_seq=1))
+    v = sum(s["value"] for s in samples) / len(samples)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, **WORKLOADS[args.workload]},
+            "cpu_baseline": {"value": v, "unit": UNIT, "kind": "oracle",
+                             "cores": samples[0]["cores"], "sample": samples[0]["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="csa_decode_128k_b32", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    import long_context_compressed_04_b200 as L
+    from long_context_compressed_04_b200 import pipeline
+
+    wl = make_workload(args.workload, rank, dev)
+    buf = pipeline.alloc(wl, dev)
+    all_seq, all_ent = pipeline.all_entry_items(wl, dev)
+    pipeline.compress(wl, buf, all_seq, all_ent)          # build the compressed cache
+    new_seq, new_ent = pipeline.newest_entry_items(wl, dev)
+    torch.cuda.synchronize()
+    del all_seq, all_ent
+
+    def step():
+        pipeline.step(wl, buf, new_seq, new_ent)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    launches0 = L.csa_launch_count()
+    with ClockSampler(gpu_index_for_smi(local)) as clk:
+        barrier()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        barrier()
+    launches = L.csa_launch_count() - launches0
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    assert int(buf.dev_status.item()) == 0, "device status flagged during the run"
+
+    # second pass: the same steps with per-kernel CUDA events (roofline of each kernel)
+    L.csa_profile_collect()
+    L.csa_profile_enable(True)
+    for i in range(K):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    L.csa_profile_enable(False)
+    per_kernel = L.csa_profile_collect()
+
+    # e2e: host buffers, h2d of the step's inputs and d2h of its output in the region
+    h_in = {"q": wl.q, "qI": wl.qI, "qs": wl.qs, "w": wl.w}
+    h_in = {k2: v for k2, v in h_in.items() if v is not None}
+    pinned = {k2: torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v.cpu())
+              for k2, v in h_in.items()}
+    last_rows = (wl.kv_off + (wl.T.to(dev) - 1 - wl.kv_pos0)).long()
+    pin_kv = torch.empty((wl.B, wl.D), dtype=wl.kv.dtype, pin_memory=True).copy_(wl.kv[last_rows].cpu())
+    pin_gate = torch.empty((wl.B, wl.D), dtype=wl.gate.dtype, pin_memory=True).copy_(wl.gate[last_rows].cpu())
+    out_host = torch.empty(buf.out.shape, dtype=buf.out.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values()) + 2 * pin_kv.numel() * 2
+    d2h = out_host.numel() * out_host.element_size()
+    E = max(K // 2, 10)
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(E)]
+    barrier()
+    for i in range(E):
+        flush.zero_()
+        ee[i][0].record()
+        for k2, v in pinned.items():
+            h_in[k2].copy_(v, non_blocking=True)
+        wl.kv[last_rows] = pin_kv.to(dev, non_blocking=True)
+        wl.gate[last_rows] = pin_gate.to(dev, non_blocking=True)
+        step()
+        out_host.copy_(buf.out, non_blocking=True)
+        ee[i][1].record()
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
+    te = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+    if dist:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+
+    peak, peak_kind = _peaks()
+    total_bytes, key_bytes = algorithmic_bytes(wl)
+    Qtot = wl.Q * world
+    value = Qtot * K / (ms_max / 1e3)
+    step_s = ms_max / K / 1e3
+    # dominant kernel: the one with the largest share of the profiled device time
+    dom = max(per_kernel.items(), key=lambda kv: kv[1][1]) if per_kernel else None
+    roof = None
+    if dom:
+        name, (n_l, tot_ms) = dom
+        avg_s = tot_ms / n_l / 1e3
+        if name.startswith("indexer"):
+            alg = key_bytes
+        elif name.startswith("attn"):
+            alg = total_bytes - key_bytes
+        else:
+            alg = total_bytes
+        ach = alg / avg_s / 1e9
+        roof = {"bound": "hbm", "kernel": name, "achieved": round(ach, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(ach / peak, 4), "traffic": None,
+                "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                "algorithmic_bytes_per_launch": alg, "avg_launch_us": round(avg_s * 1e6, 2)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, **WORKLOADS[args.workload],
+                   "queries_per_gpu": wl.Q, "l2": "flushed (256 MB write) before every timed step",
+                   "indexer_inputs": "fp8 e4m3 N(0,1), 1x128 scales"},
+        "roofline": roof,
+        "step_roofline": {"algorithmic_bytes": total_bytes,
+                          "achieved_gbs": round(total_bytes / step_s / 1e9, 1),
+                          "frac": round(total_bytes / step_s / 1e9 / peak, 4)},
+        "kernels": {k2: {"launches": v[0], "avg_us": round(v[1] / v[0] * 1e3, 2),
+                         "share": round(v[1] / sum(x[1] for x in per_kernel.values()), 4)}
+                    for k2, v in per_kernel.items()},
+        "e2e": {"value": Qtot * E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,224 @@
+/*
+ * libcsa -- hybrid compressed attention (CSA / HCA) for NVIDIA B200 (sm_100a).
+ *
+ * The method is described on the pages about the DeepSeek-V4 technical report:
+ *   "DeepSeek-V4 深度分析报告" (juejin.cn), section 2.1 "混合注意力架构：CSA + HCA", its
+ *   Figure 2, the list "其他注意力技术细节", section 3.3 (batch-invariant kernels) and
+ *   section 3.5 (state cache / classical KV cache); and the stuffyNLP post 255 on
+ *   DeepSeek-V4 (CSA stride m=4 with 2m tokens per entry, HCA m'=128, partial RoPE on the
+ *   last 64 dims, FP8 with 1x128 blocks).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller.  The library never
+ *    allocates, frees or synchronises; each call only enqueues kernels on `stream`
+ *    (a cudaStream_t passed as void*, NULL = legacy default stream) and returns.
+ *  - Host-side validation happens before any launch.  On failure nothing is launched and
+ *    the call returns a non-zero csa_status_t; csa_last_error() (thread-local) describes it.
+ *  - `dev_status` (nullable device int32) collects CSA_DEV_* bits with atomicOr when a
+ *    kernel meets data it must not use (an index outside the visible entries, a position
+ *    that is not stored, a NaN score, too small a workspace).  The offending access is
+ *    skipped; kernels never trap.  Read it after your own synchronisation.
+ *  - bf16 tensors are passed as raw 16-bit storage, e4m3 as raw bytes ("fn" encoding,
+ *    largest finite 448).  Row-major layouts throughout.
+ *  - Ragged batches.  B sequences; seq_len[b] (int64) is the number of tokens sequence b
+ *    holds so far (positions 0 .. seq_len[b]-1).  Raw per-token data (kv, gate) is a row
+ *    store: position p of sequence b is row kv_off[b] + (p - kv_pos0[b]); only positions
+ *    kv_pos0[b] .. seq_len[b]-1 are stored (a decode state cache keeps just the tail).
+ *    Compressed entries and indexer keys share one entry numbering: entry i of sequence b
+ *    is row ent_off[b] + i, for i < floor(seq_len[b]/m).  seq_len, kv_off, kv_pos0 and
+ *    ent_off are int64 [B]; kernels check every position and index against them.
+ *  - Queries: q_seq[Q] (int32, sequence) and q_pos[Q] (int32, token position
+ *    0 <= t < seq_len[q_seq]; other queries set CSA_DEV_OOB and are skipped).  Entry i is
+ *    visible to a query at t iff its block has ended: (i+1)*m - 1 <= t, so
+ *    n_vis(t) = floor((t+1)/m).  The window is raw tokens max(0, t-W+1) .. t.
+ *  - RoPE: interleaved pairs (D-64+2j, D-64+2j+1), j = 0..31, angle pos*theta^(-2j/64),
+ *    (x, y) -> (x cos a - y sin a, x sin a + y cos a).  Angles are formed in fp64.
+ *  - Batch invariance (section 3.3): every output element of a query is computed by the
+ *    same instructions in the same order whatever the batch, the neighbours or the slot;
+ *    no reduction of one query is split by batch size or SM count.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size or enum */
+    CSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented shape (head dims, heads, k) */
+    CSA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed */
+    CSA_ERR_WORKSPACE = 4      /* workspace missing or smaller than the query says */
+} csa_status_t;
+
+/* Bits OR-ed into *dev_status by kernels. */
+#define CSA_DEV_OOB 1       /* index / position outside the visible or stored range (skipped) */
+#define CSA_DEV_TIMEOUT 2   /* a bounded wait on a barrier gave up; the kernel returned */
+#define CSA_DEV_NAN 4       /* a NaN indexer score */
+#define CSA_DEV_CAPACITY 8  /* n_vis larger than the max_n the workspace was sized for */
+
+/* Entry storage formats.
+ * CSA_KV_BF16: D bf16 values per entry (row of 2*D bytes).
+ * CSA_KV_FP8_576: D = 576 only; row of 656 bytes = 512 e4m3 codes for channels 0..511,
+ *   4 fp32 scales at byte 512 (channel c of block c/128 has value code*scale; the scale is
+ *   the block's absmax / 448), then 64 bf16 values for the RoPE channels 512..575
+ *   ("混合精度存储": RoPE dims in BF16, the rest FP8; stuffyNLP: FP8 1x128 blocks). */
+#define CSA_KV_BF16 0
+#define CSA_KV_FP8_576 1
+
+int csa_version(void);
+const char* csa_last_error(void);
+/* Bytes per stored entry row for (fmt, D), or -1 if unsupported. */
+int32_t csa_entry_row_bytes(int32_t fmt, int32_t D);
+
+/*
+ * csa_compress -- CSA 4:1 overlapped KV compression (step a1).
+ *   "DeepSeek-V4 深度分析报告" 2.1 CSA / Figure 2 "KV Compress 4:1 Overlapped": every
+ *   m=4 tokens make one entry, and each entry pools 2m=8 tokens (its own block and the
+ *   previous one).  For entry i: positions P = (i-1)*4 .. (i+1)*4-1 (positions < 0 are
+ *   dropped, so entry 0 pools tokens 0..3 with bias rows 4..7); per channel c,
+ *   w_j = softmax_j(gate[p_j, c] + pos_bias[j, c]), e_c = sum_j w_j * kv[p_j, c];
+ *   then RMSNorm over all D channels (unit weight, epsilon eps); then RoPE on the last 64
+ *   channels at the block-end position (i+1)*4 - 1; then stored in format fmt.
+ * Arguments:
+ *   kv, gate   bf16 [rows, D] raw KV and gate logits (row addressing as above)
+ *   pos_bias   fp32 [8, D], row j pairs with the j-th pooled position
+ *   item_seq, item_ent  int32 [n_items]: compute entry item_ent[n] of sequence item_seq[n]
+ *   entries    output rows, format fmt; only the listed rows are written
+ *   B          number of sequences (item_seq must be < B; the entry's last pooled
+ *              position (i+1)*4-1 must be < seq_len[b], else CSA_DEV_OOB and no write)
+ *   D          128 (fmt CSA_KV_BF16) or 576 (either format)
+ * Pointers kv/gate/entries must be 16-byte aligned.  n_items = 0 is a no-op.
+ * Errors: CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA; an entry whose tokens are
+ * not stored sets CSA_DEV_OOB and is left unwritten.
+ */
+csa_status_t csa_compress(const void* kv, const void* gate, const float* pos_bias,
+                          const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
+                          const int64_t* ent_off,
+                          const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
+                          int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
+                          void* entries, int32_t* dev_status, void* stream);
+
+/*
+ * hca_compress -- HCA 128:1 compression (step a2).
+ *   "DeepSeek-V4 深度分析报告" 2.1 HCA / Figure 2 "KV Compress 128:1 Single Block": every
+ *   m'=128 tokens make one entry, no overlap.  Entry i pools positions 128i .. 128i+127
+ *   with the same per-channel softmax pooling, RMSNorm, and RoPE at position 128i+127.
+ *   pos_bias is fp32 [128, D].  Other arguments as csa_compress.
+ */
+csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bias,
+                          const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
+                          const int64_t* ent_off,
+                          const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
+                          int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
+                          void* entries, int32_t* dev_status, void* stream);
+
+/*
+ * lightning_indexer_topk -- lightning-indexer scores and top-k selection (steps a3, a4).
+ *   "DeepSeek-V4 深度分析报告" 2.1 CSA "稀疏选择": a lightning indexer scores the compressed
+ *   entries and keeps the top-k (k = 1024 for V4-Pro, 512 for V4-Flash); Figure 2.
+ * For query q at t and every visible entry i < n_vis(t) of its sequence:
+ *   d_h = sum_c qI[q,h,c] * kI[i,c]          (e4m3 products, fp32 accumulation)
+ *   acc = +0; for h = 0..H_I-1: acc = fmaf(w[q,h] * qI_scale[q,h], max(d_h, 0), acc)
+ *   s_i = acc * kI_scale[i]                  (all fp32, in this order)
+ * idx_out[q, :] holds the k entries with the largest s_i (ties: lower i first), in
+ * ascending entry order, padded with -1 when n_vis < k.
+ * Arguments:
+ *   qI e4m3 [Q, H_I, d_I]; qI_scale, w fp32 [Q, H_I]; kI e4m3 [ent_rows, d_I];
+ *   kI_scale fp32 [ent_rows]; seq_len, ent_off int64 [B]; q_seq, q_pos int32 [Q]
+ *   H_I in 1..64, d_I in {64, 128}, m >= 1 (4 for CSA), 1 <= k <= 2048
+ *   max_n: upper bound of n_vis over the batch (sizes the workspace)
+ *   idx_out int32 [Q, k]
+ *   scores_out: nullable fp32 [Q, ld_scores] receiving s_i for i < n_vis (ld_scores >= max_n)
+ *   workspace: device buffer of at least csa_indexer_workspace_size(Q, max_n, k) bytes,
+ *   256-byte aligned; contents on entry are ignored.
+ * kI and qI must be 16-byte aligned.  Errors as above; CSA_DEV_NAN, CSA_DEV_CAPACITY.
+ */
+size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k);
+csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, const float* w,
+                                    const uint8_t* kI, const float* kI_scale,
+                                    const int64_t* seq_len, const int64_t* ent_off,
+                                    const int32_t* q_seq,
+                                    const int32_t* q_pos, int32_t Q, int32_t B, int32_t H_I,
+                                    int32_t d_I, int32_t m, int32_t k, int32_t max_n,
+                                    int32_t* idx_out, float* scores_out, int64_t ld_scores,
+                                    void* workspace, size_t workspace_bytes,
+                                    int32_t* dev_status, void* stream);
+
+/*
+ * sparse_mqa_attn -- CSA shared-KV MQA over the selected entries and the window (a5).
+ *   "DeepSeek-V4 深度分析报告" 2.1 CSA (top-k entries plus a 128-token sliding window);
+ *   "其他注意力技术细节": Shared Key-Value MQA (an entry is both key and value, all heads
+ *   share it), Partial RoPE with inverse RoPE on the output, Attention Sink (learnable
+ *   per-head logit, weights may sum to less than 1).
+ * For query q (sequence b, position t) and head h:
+ *   keys K = { entry idx[q,j] : idx >= 0 }  U  { window rows p = max(0,t-W+1) .. t },
+ *   window row p = RoPE_p(RMSNorm(kv[p])) computed on the fly in fp32 (never stored);
+ *   l_j = softmax_scale * < RoPE_t(q[q,h]), k_j >,  M = max(sink[h], max_j l_j),
+ *   o = sum_j e^(l_j-M) k_j / (e^(sink[h]-M) + sum_j e^(l_j-M)),  out = RoPE_{-t}(o) (bf16).
+ * Arguments:
+ *   q bf16 [Q, H, D]; entries in format fmt; kv bf16 raw rows for the window;
+ *   idx int32 [Q, k] (entries < n_vis(t) for ratio m, or -1 = skip); sink fp32 [H]
+ *   H in {16, 64, 128}; D 128 (bf16) or 576 (either format); 0 <= W <= 128
+ *   out bf16 [Q, H, D]
+ * Pointers q/kv/entries/out must be 16-byte aligned.  Out-of-range indices set CSA_DEV_OOB
+ * and are skipped.
+ */
+csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt,
+                             const int64_t* seq_len, const int64_t* ent_off, const void* kv,
+                             const int64_t* kv_off,
+                             const int64_t* kv_pos0, const int32_t* q_seq,
+                             const int32_t* q_pos, const int32_t* idx, int32_t k, int32_t m,
+                             const float* sink, int32_t Q, int32_t B, int32_t H, int32_t D,
+                             int32_t W, float softmax_scale, float rope_theta, float eps,
+                             void* out, int32_t* dev_status, void* stream);
+
+/*
+ * dense_hca_attn -- HCA dense MQA over every visible entry plus the window (a6).
+ *   "DeepSeek-V4 深度分析报告" 2.1 HCA: dense attention over all compressed entries, with
+ *   the same sliding-window branch; Figure 2 "Dense Attention on All Compressed KV
+ *   Entries".  As sparse_mqa_attn with K = { entries 0 .. n_vis(t)-1 } U window, where
+ *   n_vis(t) = floor((t+1)/m) (m = 128 for HCA).
+ *   max_n: upper bound of n_vis over the batch; workspace: at least
+ *   dense_hca_workspace_size(Q, H, D, max_n) bytes, 256-byte aligned (partial softmax
+ *   states of the fixed entry chunks one query is split into; the chunking depends only
+ *   on the query's own n_vis and the shape, so results do not depend on the batch).
+ */
+size_t dense_hca_workspace_size(int32_t Q, int32_t H, int32_t D, int32_t max_n);
+csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
+                            const int64_t* seq_len, const int64_t* ent_off, const void* kv,
+                            const int64_t* kv_off,
+                            const int64_t* kv_pos0, const int32_t* q_seq, const int32_t* q_pos,
+                            int32_t m, const float* sink, int32_t Q, int32_t B, int32_t H,
+                            int32_t D, int32_t W, float softmax_scale, float rope_theta,
+                            float eps, int32_t max_n, void* out, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Launch accounting and kernel timing (no counterpart on the pages; instrumentation).
+ *   csa_launch_count: kernels this library has launched in the process so far.
+ *   csa_profile_enable(1): from now on every launch is bracketed by a CUDA event pair
+ *     recorded on its own stream (adds two event records per launch); 0 turns it off.
+ *   csa_profile_collect: waits for the recorded events, writes one record per kernel
+ *     kind timed since the last collect (launch count and total device milliseconds) to
+ *     out[0 .. max_entries), returns how many it wrote, and resets the totals.
+ * Thread-safe.  Uses the CUDA device that was current at each launch.
+ */
+typedef struct {
+    char name[40];
+    long long launches;
+    double total_ms;
+} csa_kernel_time_t;
+long long csa_launch_count(void);
+void csa_profile_enable(int on);
+int csa_profile_collect(csa_kernel_time_t* out, int max_entries);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H */

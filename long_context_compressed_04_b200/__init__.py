@@ -1,0 +1,176 @@
+"""Hybrid compressed attention (CSA / HCA) on B200: Python binding of libcsa.
+
+Argument marshalling only: every function here passes tensor pointers, sizes and the
+current CUDA stream to the C ABI of ``libcsa.so`` (declared in ``include/csa.h``) and raises
+``CSAError`` when it returns a non-zero status.  All computation happens in the CUDA
+kernels.  There is no CPU fallback: importing this package fails if ``libcsa.so`` has not
+been built (``python -m long_context_compressed_04_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_KV_BF16 = 0
+CSA_KV_FP8_576 = 1
+CSA_DEV_OOB = 1
+CSA_DEV_TIMEOUT = 2
+CSA_DEV_NAN = 4
+CSA_DEV_CAPACITY = 8
+
+STATUS_NAMES = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED",
+                3: "CSA_ERR_CUDA", 4: "CSA_ERR_WORKSPACE"}
+
+
+class CSAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with "
+                      "`python -m long_context_compressed_04_b200.build` (needs nvcc)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P, _I32, _I64, _F32, _SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+_SIGS = {
+    "csa_version": (ctypes.c_int, []),
+    "csa_last_error": (ctypes.c_char_p, []),
+    "csa_entry_row_bytes": (_I32, [_I32, _I32]),
+    "csa_compress": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32,
+                                    _F32, _F32, _P, _P, _P]),
+    "hca_compress": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32,
+                                    _F32, _F32, _P, _P, _P]),
+    "csa_indexer_workspace_size": (_SZ, [_I32, _I32, _I32]),
+    "lightning_indexer_topk": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32,
+                                              _I32, _I32, _I32, _I32, _P, _P, _I64, _P, _SZ, _P,
+                                              _P]),
+    "sparse_mqa_attn": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P,
+                                       _I32, _I32, _I32, _I32, _I32, _F32, _F32, _F32, _P, _P,
+                                       _P]),
+    "dense_hca_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
+    "dense_hca_attn": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32,
+                                      _I32, _I32, _I32, _F32, _F32, _F32, _I32, _P, _P, _SZ, _P,
+                                      _P]),
+    "csa_launch_count": (ctypes.c_longlong, []),
+    "csa_profile_enable": (None, [ctypes.c_int]),
+    "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+EXPORTED = tuple(_SIGS)
+
+
+def _p(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int):
+    if status != 0:
+        raise CSAError(status, _lib.csa_last_error().decode())
+
+
+class _KernelTime(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 40), ("launches", ctypes.c_longlong),
+                ("total_ms", ctypes.c_double)]
+
+
+def csa_launch_count() -> int:
+    return _lib.csa_launch_count()
+
+
+def csa_profile_enable(on: bool = True):
+    _lib.csa_profile_enable(1 if on else 0)
+
+
+def csa_profile_collect() -> dict:
+    """{kernel name: (timed launches, total device ms)} since the last collect."""
+    arr = (_KernelTime * 32)()
+    n = _lib.csa_profile_collect(ctypes.cast(arr, ctypes.c_void_p), 32)
+    return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}
+
+
+def csa_version() -> int:
+    return _lib.csa_version()
+
+
+def csa_entry_row_bytes(fmt: int, D: int) -> int:
+    return _lib.csa_entry_row_bytes(fmt, D)
+
+
+def csa_indexer_workspace_size(Q: int, max_n: int, k: int) -> int:
+    return _lib.csa_indexer_workspace_size(Q, max_n, k)
+
+
+def dense_hca_workspace_size(Q: int, H: int, D: int, max_n: int) -> int:
+    return _lib.dense_hca_workspace_size(Q, H, D, max_n)
+
+
+def csa_compress(kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq, item_ent,
+                 entries, *,
+                 B: int, D: int, fmt: int = CSA_KV_BF16, rope_theta: float = 10000.0,
+                 eps: float = 1e-6, dev_status=None, stream=None):
+    _check(_lib.csa_compress(_p(kv), _p(gate), _p(pos_bias), _p(seq_len), _p(kv_off), _p(kv_pos0),
+                             _p(ent_off), _p(item_seq), _p(item_ent), item_seq.numel(), B, D, fmt,
+                             rope_theta, eps, _p(entries), _p(dev_status), _s(stream)))
+
+
+def hca_compress(kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq, item_ent,
+                 entries, *,
+                 B: int, D: int, fmt: int = CSA_KV_BF16, rope_theta: float = 10000.0,
+                 eps: float = 1e-6, dev_status=None, stream=None):
+    _check(_lib.hca_compress(_p(kv), _p(gate), _p(pos_bias), _p(seq_len), _p(kv_off), _p(kv_pos0),
+                             _p(ent_off), _p(item_seq), _p(item_ent), item_seq.numel(), B, D, fmt,
+                             rope_theta, eps, _p(entries), _p(dev_status), _s(stream)))
+
+
+def lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_seq, q_pos, idx_out,
+                           workspace, *, B: int, H_I: int, d_I: int, m: int, k: int, max_n: int,
+                           scores_out=None, ld_scores: int = 0, dev_status=None, stream=None):
+    _check(_lib.lightning_indexer_topk(
+        _p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), _p(seq_len), _p(ent_off), _p(q_seq),
+        _p(q_pos),
+        q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out), ld_scores,
+        _p(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _p(dev_status), _s(stream)))
+
+
+def sparse_mqa_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos, idx, sink,
+                    out, *,
+                    fmt: int, B: int, H: int, D: int, W: int, m: int, k: int,
+                    softmax_scale: float, rope_theta: float = 10000.0, eps: float = 1e-6,
+                    dev_status=None, stream=None):
+    _check(_lib.sparse_mqa_attn(
+        _p(q), _p(entries), fmt, _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
+        _p(q_pos), _p(idx), k, m, _p(sink), q_seq.numel(), B, H, D, W, softmax_scale,
+        rope_theta, eps, _p(out), _p(dev_status), _s(stream)))
+
+
+def dense_hca_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos, sink, out,
+                   workspace, *, fmt: int, B: int, H: int, D: int, W: int, m: int, max_n: int,
+                   softmax_scale: float, rope_theta: float = 10000.0, eps: float = 1e-6,
+                   dev_status=None, stream=None):
+    _check(_lib.dense_hca_attn(
+        _p(q), _p(entries), fmt, _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
+        _p(q_pos), m, _p(sink), q_seq.numel(), B, H, D, W, softmax_scale, rope_theta, eps,
+        max_n, _p(out), _p(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _p(dev_status), _s(stream)))

@@ -1,0 +1,217 @@
+// The C ABI of libcsa: host-side validation, workspace layout and kernel dispatch.
+// Declarations and the contract of every call are in include/csa.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "launchers.cuh"
+
+
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+csa_status_t fail(csa_status_t s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+csa_status_t ok() {
+    g_err[0] = '\0';
+    return CSA_OK;
+}
+
+csa_status_t cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return ok();
+    return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+#define REQUIRE(cond, ...)                                      \
+    do {                                                        \
+        if (!(cond)) return fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); \
+    } while (0)
+#define SUPPORT(cond, ...)                                      \
+    do {                                                        \
+        if (!(cond)) return fail(CSA_ERR_UNSUPPORTED, __VA_ARGS__); \
+    } while (0)
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+csa_status_t compress_common(int m, int span, const void* kv, const void* gate,
+                             const float* bias, const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
+                             const int64_t* ent_off, const int32_t* item_seq,
+                             const int32_t* item_ent, int64_t n_items, int32_t B, int32_t D,
+                             int32_t fmt, float theta, float eps, void* entries,
+                             int32_t* dev_status, void* stream) {
+    REQUIRE(n_items >= 0 && n_items < (1ll << 31), "n_items out of range: %lld", (long long)n_items);
+    if (n_items == 0) return ok();
+    REQUIRE(kv && gate && bias && seq_len && kv_off && kv_pos0 && ent_off && item_seq && item_ent &&
+                entries,
+            "null pointer argument");
+    REQUIRE(aligned(kv, 16) && aligned(gate, 16) && aligned(entries, 16) && aligned(bias, 16),
+            "kv, gate, pos_bias and entries must be 16-byte aligned");
+    REQUIRE(B >= 1, "B must be >= 1");
+    REQUIRE(fmt == CSA_KV_BF16 || fmt == CSA_KV_FP8_576, "unknown entry format %d", fmt);
+    SUPPORT(D == 128 || D == 576, "head dim %d not supported (128 or 576)", D);
+    SUPPORT(fmt == CSA_KV_BF16 || D == 576, "fp8 entry format needs D = 576");
+    REQUIRE(theta > 1.f && eps >= 0.f, "rope_theta must be > 1 and eps >= 0");
+    cudaError_t e = csa::launch_compress(span, kv, gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
+                                         item_ent, n_items, B, m, D, fmt, theta, eps, entries,
+                                         dev_status, (cudaStream_t)stream);
+    return cuda_status(e, "compress launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int csa_version(void) { return 100; }
+
+const char* csa_last_error(void) { return g_err; }
+
+int32_t csa_entry_row_bytes(int32_t fmt, int32_t D) {
+    if (fmt == CSA_KV_BF16 && (D == 128 || D == 576)) return 2 * D;
+    if (fmt == CSA_KV_FP8_576 && D == 576) return 656;
+    return -1;
+}
+
+csa_status_t csa_compress(const void* kv, const void* gate, const float* pos_bias,
+                          const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
+                          const int64_t* ent_off,
+                          const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
+                          int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
+                          void* entries, int32_t* dev_status, void* stream) {
+    return compress_common(4, 8, kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq, item_ent,
+                           n_items, B, D, fmt, rope_theta, eps, entries, dev_status, stream);
+}
+
+csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bias,
+                          const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
+                          const int64_t* ent_off,
+                          const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
+                          int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
+                          void* entries, int32_t* dev_status, void* stream) {
+    return compress_common(128, 128, kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
+                           item_ent, n_items, B, D, fmt, rope_theta, eps, entries, dev_status,
+                           stream);
+}
+
+size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k) {
+    if (Q <= 0 || max_n < 0 || k <= 0) return 0;
+    (void)k;
+    return round_up((size_t)Q * round_up((size_t)max_n, 32) * sizeof(float), 256) + 256;
+}
+
+csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, const float* w,
+                                    const uint8_t* kI, const float* kI_scale,
+                                    const int64_t* seq_len, const int64_t* ent_off,
+                                    const int32_t* q_seq,
+                                    const int32_t* q_pos, int32_t Q, int32_t B, int32_t H_I,
+                                    int32_t d_I, int32_t m, int32_t k, int32_t max_n,
+                                    int32_t* idx_out, float* scores_out, int64_t ld_scores,
+                                    void* workspace, size_t workspace_bytes,
+                                    int32_t* dev_status, void* stream) {
+    REQUIRE(Q >= 0, "Q must be >= 0");
+    if (Q == 0) return ok();
+    REQUIRE(qI && qI_scale && w && seq_len && ent_off && q_seq && q_pos && idx_out,
+            "null pointer argument");
+    REQUIRE(max_n >= 0, "max_n must be >= 0");
+    REQUIRE(max_n == 0 || (kI && kI_scale), "null key pointer");
+    REQUIRE(aligned(qI, 16) && (kI == nullptr || aligned(kI, 16)), "qI and kI must be 16-byte aligned");
+    REQUIRE(B >= 1 && m >= 1, "B and m must be >= 1");
+    SUPPORT(H_I >= 1 && H_I <= 64, "indexer heads %d not supported (1..64)", H_I);
+    SUPPORT(d_I == 64 || d_I == 128, "indexer dim %d not supported (64 or 128)", d_I);
+    SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
+    REQUIRE(scores_out == nullptr || ld_scores >= max_n, "ld_scores must be >= max_n");
+    const size_t need = csa_indexer_workspace_size(Q, max_n, k);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+        return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", need);
+    float* scores = scores_out ? scores_out : (float*)workspace;
+    const int64_t ld = scores_out ? ld_scores : (int64_t)round_up((size_t)max_n, 32);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = csa::launch_indexer_simt(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_seq, q_pos,
+                                             Q, B, H_I, d_I, m, max_n, scores, ld, dev_status, s);
+    if (e != cudaSuccess) return cuda_status(e, "indexer launch");
+    e = csa::launch_topk(scores, ld, q_seq, q_pos, seq_len, Q, B, m, max_n, k, idx_out, dev_status,
+                         s);
+    return cuda_status(e, "top-k launch");
+}
+
+static csa_status_t attn_validate(const void* q, const void* entries, int32_t fmt,
+                                  const int64_t* seq_len, const int64_t* ent_off, const void* kv, const int64_t* kv_off,
+                                  const int64_t* kv_pos0, const int32_t* q_seq,
+                                  const int32_t* q_pos, const float* sink, int32_t B,
+                                  int32_t H, int32_t D, int32_t W, int32_t m, float scale,
+                                  float theta, float eps, void* out) {
+    REQUIRE(q && entries && seq_len && ent_off && kv && kv_off && kv_pos0 && q_seq && q_pos && sink &&
+                out,
+            "null pointer argument");
+    REQUIRE(aligned(q, 16) && aligned(entries, 16) && aligned(kv, 16) && aligned(out, 16),
+            "q, entries, kv and out must be 16-byte aligned");
+    REQUIRE(fmt == CSA_KV_BF16 || fmt == CSA_KV_FP8_576, "unknown entry format %d", fmt);
+    SUPPORT(D == 128 || D == 576, "head dim %d not supported (128 or 576)", D);
+    SUPPORT(fmt == CSA_KV_BF16 || D == 576, "fp8 entry format needs D = 576");
+    SUPPORT(H == 16 || H == 64 || H == 128, "query heads %d not supported (16, 64, 128)", H);
+    REQUIRE(W >= 0 && W <= 128, "window %d outside 0..128", W);
+    REQUIRE(B >= 1 && m >= 1, "B and m must be >= 1");
+    REQUIRE(scale > 0.f && theta > 1.f && eps >= 0.f, "bad softmax_scale / rope_theta / eps");
+    return ok();
+}
+
+csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt,
+                             const int64_t* seq_len, const int64_t* ent_off, const void* kv, const int64_t* kv_off,
+                             const int64_t* kv_pos0, const int32_t* q_seq,
+                             const int32_t* q_pos, const int32_t* idx, int32_t k, int32_t m,
+                             const float* sink, int32_t Q, int32_t B, int32_t H, int32_t D,
+                             int32_t W, float softmax_scale, float rope_theta, float eps,
+                             void* out, int32_t* dev_status, void* stream) {
+    REQUIRE(Q >= 0, "Q must be >= 0");
+    if (Q == 0) return ok();
+    csa_status_t v = attn_validate(q, entries, fmt, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
+                                   sink, B, H, D, W, m, softmax_scale, rope_theta, eps, out);
+    if (v != CSA_OK) return v;
+    REQUIRE(idx != nullptr, "idx must not be null");
+    SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
+    csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, ent_off, (const uint16_t*)kv,
+                    kv_off, kv_pos0, q_seq, q_pos, seq_len, idx, sink, (uint16_t*)out, dev_status,
+                    k, m, B, H, W, fmt, softmax_scale, eps, log2((double)rope_theta)};
+    return cuda_status(csa::launch_attn_simt(a, Q, D, (cudaStream_t)stream), "attention launch");
+}
+
+size_t dense_hca_workspace_size(int32_t Q, int32_t H, int32_t D, int32_t max_n) {
+    (void)Q;
+    (void)H;
+    (void)D;
+    (void)max_n;
+    return 256;
+}
+
+csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
+                            const int64_t* seq_len, const int64_t* ent_off, const void* kv, const int64_t* kv_off,
+                            const int64_t* kv_pos0, const int32_t* q_seq, const int32_t* q_pos,
+                            int32_t m, const float* sink, int32_t Q, int32_t B, int32_t H,
+                            int32_t D, int32_t W, float softmax_scale, float rope_theta,
+                            float eps, int32_t max_n, void* out, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    REQUIRE(Q >= 0, "Q must be >= 0");
+    if (Q == 0) return ok();
+    csa_status_t v = attn_validate(q, entries, fmt, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
+                                   sink, B, H, D, W, m, softmax_scale, rope_theta, eps, out);
+    if (v != CSA_OK) return v;
+    REQUIRE(max_n >= 0, "max_n must be >= 0");
+    const size_t need = dense_hca_workspace_size(Q, H, D, max_n);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+        return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", need);
+    csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, ent_off, (const uint16_t*)kv,
+                    kv_off, kv_pos0, q_seq, q_pos, seq_len, nullptr, sink, (uint16_t*)out, dev_status,
+                    0, m, B, H, W, fmt, softmax_scale, eps, log2((double)rope_theta)};
+    return cuda_status(csa::launch_attn_simt(a, Q, D, (cudaStream_t)stream), "attention launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// Device helpers shared by the libcsa kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+constexpr int kRopeDims = 64;
+
+__device__ __forceinline__ void flag(int32_t* st, int bits) {
+    if (st) atomicOr(st, bits);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
+    return __uint_as_float(bits16 << 16);
+}
+
+// Two packed bf16 (low half = first element) -> two floats.
+__device__ __forceinline__ float2 bf16x2_to_f32(uint32_t packed) {
+    return make_float2(__uint_as_float(packed << 16), __uint_as_float(packed & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float x) {
+    __nv_bfloat16 h = __float2bfloat16_rn(x);
+    return (uint32_t)(*reinterpret_cast<uint16_t*>(&h));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    return f32_to_bf16_bits(lo) | (f32_to_bf16_bits(hi) << 16);
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    __nv_fp8_e4m3 v;
+    v.__x = (__nv_fp8_storage_t)code;
+    return float(v);
+}
+
+__device__ __forceinline__ uint32_t f32_to_e4m3_satfinite(float x) {
+    return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+
+// RoPE rotation of pair j (of the last 64 dims) at position pos: cos/sin of
+// pos * theta^(-2j/64).  The angle is formed and reduced to [-pi, pi] in fp64 so that
+// positions up to 2^20 keep ~1e-7 rad accuracy; the reduced angle then goes to sincosf.
+__device__ __forceinline__ void rope_cos_sin(double pos, int j, double log2_theta, float& c,
+                                             float& s) {
+    const double kTwoPi = 6.283185307179586476925;
+    const double kInvTwoPi = 0.159154943091895335769;
+    double inv_freq = exp2(-(double)(2 * j) * (1.0 / 64.0) * log2_theta);
+    double a = pos * inv_freq;
+    double r = a - kTwoPi * rint(a * kInvTwoPi);
+    sincosf((float)r, &s, &c);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+}  // namespace csa

@@ -1,0 +1,160 @@
+// Steps a1/a2: CSA (m=4, 8 pooled tokens) and HCA (m'=128, 128 pooled tokens) compression.
+//
+// "DeepSeek-V4 深度分析报告" 2.1: CSA turns every 4 tokens into one entry drawing on 8
+// tokens (its block and the previous one); HCA turns every 128 tokens into one entry.
+// Per channel: softmax over the pooled tokens of (gate logit + positional bias row),
+// weighted sum of the raw KV, then RMSNorm over the head dim and RoPE on the last 64
+// channels at the block-end position, then bf16 or fp8(1x128)+bf16 storage.
+//
+// One CTA per entry; each thread owns 4 consecutive channels (8-byte bf16x4 loads, so a
+// warp reads 256 contiguous bytes of a token row).  The softmax runs online over the
+// pooled tokens in fp32; RMSNorm reduces over the CTA; the RoPE pairs of a thread's 4
+// channels are local to it.  HBM-bound: every raw token row is read once per entry that
+// pools it (twice for CSA's overlap; the second read mostly hits L2).
+#include "launchers.cuh"
+
+namespace csa {
+
+template <int SPAN>
+__global__ void __launch_bounds__(160) compress_kernel(
+    const uint16_t* __restrict__ kv, const uint16_t* __restrict__ gate,
+    const float* __restrict__ bias, const int64_t* __restrict__ seq_len,
+    const int64_t* __restrict__ kv_off,
+    const int64_t* __restrict__ kv_pos0, const int64_t* __restrict__ ent_off,
+    const int32_t* __restrict__ item_seq, const int32_t* __restrict__ item_ent, int B, int m,
+    int D, int fmt, double log2_theta, float eps, uint8_t* __restrict__ entries,
+    int32_t* __restrict__ dev_status) {
+    __shared__ float red[8];
+    const int64_t it = blockIdx.x;
+    const int b = item_seq[it];
+    const int64_t i = item_ent[it];
+    if (b < 0 || b >= B || i < 0) {
+        if (threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
+        return;
+    }
+    const int64_t first = (i + 1) * (int64_t)m - SPAN;
+    const int64_t pos0 = kv_pos0[b];
+    const int64_t row0 = kv_off[b];
+    // every pooled token must be stored: positions max(first, 0) .. (i+1)m-1
+    if ((first > 0 ? first : 0) < pos0 || (i + 1) * (int64_t)m > seq_len[b]) {
+        if (threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
+        return;
+    }
+    const int tid = threadIdx.x;
+    const int c0 = tid * 4;
+    const bool active = c0 < D;
+
+    float e[4] = {0.f, 0.f, 0.f, 0.f};
+    if (active) {
+        float mx[4], den[4], acc[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            mx[u] = -INFINITY;
+            den[u] = 0.f;
+            acc[u] = 0.f;
+        }
+        const int j0 = first < 0 ? (int)(-first) : 0;
+#pragma unroll 4
+        for (int j = j0; j < SPAN; j++) {
+            const int64_t row = row0 + (first + j) - pos0;
+            const uint2 zz = *reinterpret_cast<const uint2*>(gate + row * D + c0);
+            const uint2 vv = *reinterpret_cast<const uint2*>(kv + row * D + c0);
+            const float4 bb = *reinterpret_cast<const float4*>(bias + (int64_t)j * D + c0);
+            const float2 z01 = bf16x2_to_f32(zz.x), z23 = bf16x2_to_f32(zz.y);
+            const float2 v01 = bf16x2_to_f32(vv.x), v23 = bf16x2_to_f32(vv.y);
+            const float l[4] = {z01.x + bb.x, z01.y + bb.y, z23.x + bb.z, z23.y + bb.w};
+            const float v[4] = {v01.x, v01.y, v23.x, v23.y};
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                if (l[u] > mx[u]) {
+                    const float sc = expf(mx[u] - l[u]);
+                    den[u] = den[u] * sc + 1.f;
+                    acc[u] = acc[u] * sc + v[u];
+                    mx[u] = l[u];
+                } else {
+                    const float p = expf(l[u] - mx[u]);
+                    den[u] += p;
+                    acc[u] = fmaf(p, v[u], acc[u]);
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; u++) e[u] = acc[u] / den[u];
+    }
+
+    // RMSNorm over all D channels (unit weight).
+    float ss = e[0] * e[0] + e[1] * e[1] + e[2] * e[2] + e[3] * e[3];
+    ss = warp_sum(ss);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); w++) tot += red[w];
+    const float r = rsqrtf(tot / (float)D + eps);
+#pragma unroll
+    for (int u = 0; u < 4; u++) e[u] *= r;
+
+    // RoPE on the last 64 channels at the block-end position.
+    if (active && c0 >= D - kRopeDims) {
+        const double pos = (double)((i + 1) * (int64_t)m - 1);
+        const int pair = (c0 - (D - kRopeDims)) >> 1;
+#pragma unroll
+        for (int u = 0; u < 2; u++) {
+            float cs, sn;
+            rope_cos_sin(pos, pair + u, log2_theta, cs, sn);
+            const float x = e[2 * u], y = e[2 * u + 1];
+            e[2 * u] = x * cs - y * sn;
+            e[2 * u + 1] = x * sn + y * cs;
+        }
+    }
+
+    // Store.
+    const int64_t erow = ent_off[b] + i;
+    if (fmt == CSA_KV_BF16) {
+        if (active) {
+            uint8_t* dst = entries + erow * (int64_t)(2 * D) + 2 * c0;
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]));
+        }
+    } else {  // CSA_KV_FP8_576: warps 0..3 hold channels 0..511 (one 1x128 block per warp)
+        uint8_t* dst = entries + erow * 656;
+        const int warp = tid >> 5, lane = tid & 31;
+        if (warp < 4) {
+            float amax = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
+            amax = warp_max(amax);
+            float scale = amax / 448.0f;
+            if (!(scale > 0.f)) scale = 1.f;
+            uint32_t codes = 0;
+#pragma unroll
+            for (int u = 0; u < 4; u++) codes |= f32_to_e4m3_satfinite(e[u] / scale) << (8 * u);
+            *reinterpret_cast<uint32_t*>(dst + c0) = codes;
+            if (lane == 0) *reinterpret_cast<float*>(dst + 512 + 4 * warp) = scale;
+        } else if (active) {
+            *reinterpret_cast<uint2*>(dst + 528 + 2 * (c0 - 512)) =
+                make_uint2(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]));
+        }
+    }
+}
+
+cudaError_t launch_compress(int span, const void* kv, const void* gate, const float* bias,
+                            const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
+                            const int64_t* ent_off, const int32_t* item_seq,
+                            const int32_t* item_ent, int64_t n_items, int B, int m, int D,
+                            int fmt, float theta, float eps, void* entries, int32_t* st,
+                            cudaStream_t stream) {
+    if (n_items == 0) return cudaSuccess;
+    const int threads = 32 * ((D / 4 + 31) / 32);
+    const double log2_theta = log2((double)theta);
+    const dim3 grid((unsigned)n_items);
+    LaunchScope scope(kKCompress, stream);
+    if (span == 8) {
+        compress_kernel<8><<<grid, threads, 0, stream>>>(
+            (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
+            item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
+    } else {
+        compress_kernel<128><<<grid, threads, 0, stream>>>(
+            (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
+            item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -1,0 +1,60 @@
+// Internal launcher declarations shared by the kernel files and the C ABI layer.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa {
+
+// Kernel kinds for launch accounting (names in prof.cu).
+enum KernelKind { kKCompress = 0, kKIndexerSimt, kKTopk, kKAttnSimt, kKernelKinds };
+
+// Counts one kernel launch; with timing enabled, brackets it with CUDA events on `stream`.
+class LaunchScope {
+  public:
+    LaunchScope(int kind, cudaStream_t stream);
+    ~LaunchScope();
+    LaunchScope(const LaunchScope&) = delete;
+    LaunchScope& operator=(const LaunchScope&) = delete;
+
+  private:
+    int kind_;
+    cudaStream_t stream_;
+    cudaEvent_t start_ = nullptr, stop_ = nullptr;
+};
+
+struct AttnArgs {
+    const uint16_t* q;
+    const uint8_t* entries;
+    const int64_t* ent_off;
+    const uint16_t* kv;
+    const int64_t* kv_off;
+    const int64_t* kv_pos0;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    const int64_t* seq_len;
+    const int32_t* idx;  // nullptr = dense over all visible entries
+    const float* sink;
+    uint16_t* out;
+    int32_t* st;
+    int k, m, B, H, W, fmt;
+    float scale, eps;
+    double log2_theta;
+};
+
+cudaError_t launch_compress(int span, const void* kv, const void* gate, const float* bias,
+                            const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
+                            const int64_t* ent_off, const int32_t* item_seq,
+                            const int32_t* item_ent, int64_t n_items, int B, int m, int D,
+                            int fmt, float theta, float eps, void* entries, int32_t* st,
+                            cudaStream_t stream);
+cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float* w,
+                                const uint8_t* kI, const float* ks, const int64_t* seq_len,
+                                const int64_t* ent_off, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
+                                int HI, int dI, int m, int max_n, float* scores, int64_t ld,
+                                int32_t* st, cudaStream_t stream);
+cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
+                        const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
+                        int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream);
+cudaError_t launch_attn_simt(const AttnArgs& a, int Q, int D, cudaStream_t stream);
+
+}  // namespace csa

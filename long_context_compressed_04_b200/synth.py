@@ -64,6 +64,13 @@ class Workload:
     eps: float = 1e-6
 
     @property
+    def seq_len(self) -> torch.Tensor:
+        """[B] int64 context lengths on the workload's device."""
+        if getattr(self, "_seq_len", None) is None or self._seq_len.device != self.kv.device:
+            self._seq_len = self.T.to(self.kv.device)
+        return self._seq_len
+
+    @property
     def Q(self) -> int:
         return int(self.q_seq.numel())
 
@@ -233,3 +240,60 @@ def csa_decode_1m_fp8(device="cpu", seed=0, indexer="int", B=8, keep_raw=None) -
     return make_workload("csa_decode_1m_b8_fp8", B=B, T=1 << 20, D=576, H=128, m=4, span=8,
                          W=128, fmt=1, H_I=64, d_I=128, k=1024, indexer=indexer,
                          keep_raw=keep_raw, seed=seed, device=device)
+
+
+# ---- re-batching (for batch-invariance runs) -----------------------------------------
+def split(wl: Workload) -> list:
+    """One single-sequence workload per sequence of ``wl`` (same tensors, re-based)."""
+    out = []
+    T = wl.T.cpu()
+    kv_off, kv_pos0 = wl.kv_off.cpu(), wl.kv_pos0.cpu()
+    ent_off, n_ent = wl.ent_off.cpu(), wl.n_ent.cpu()
+    q_seq = wl.q_seq.cpu()
+    for b in range(wl.B):
+        r0, nr = int(kv_off[b]), int(T[b] - kv_pos0[b])
+        e0, ne = int(ent_off[b]), int(n_ent[b])
+        qsel = torch.nonzero(q_seq == b).flatten().to(wl.q.device)
+        z = torch.zeros(1, dtype=torch.int64, device=wl.kv_off.device)
+        f = dict(name=wl.name, B=1, T=T[b:b + 1].clone(), D=wl.D, H=wl.H, m=wl.m, span=wl.span,
+                 W=wl.W, fmt=wl.fmt, kv=wl.kv[r0:r0 + nr], gate=wl.gate[r0:r0 + nr],
+                 kv_off=z.clone(), kv_pos0=wl.kv_pos0[b:b + 1].clone(), bias=wl.bias,
+                 ent_off=z.clone(), n_ent=wl.n_ent[b:b + 1].clone(),
+                 q_seq=torch.zeros(qsel.numel(), dtype=torch.int32, device=wl.q_seq.device),
+                 q_pos=wl.q_pos[qsel], q=wl.q[qsel], sink=wl.sink, H_I=wl.H_I, d_I=wl.d_I,
+                 k=wl.k, theta=wl.theta, eps=wl.eps)
+        if wl.H_I:
+            f.update(kI=wl.kI[e0:e0 + ne], ks=wl.ks[e0:e0 + ne], qI=wl.qI[qsel], qs=wl.qs[qsel],
+                     w=wl.w[qsel])
+        out.append(Workload(**f))
+    return out
+
+
+def merge(parts: list) -> Workload:
+    """Concatenate single- or multi-sequence workloads (same shapes) into one batch."""
+    p0 = parts[0]
+    dev = p0.kv.device
+    Ts, kv_off, kv_pos0, ent_off, n_ent, q_seq = [], [], [], [], [], []
+    rows = ents = seqs = 0
+    for p in parts:
+        for b in range(p.B):
+            Ts.append(int(p.T[b]))
+            kv_off.append(rows + int(p.kv_off[b]))
+            kv_pos0.append(int(p.kv_pos0[b]))
+            ent_off.append(ents + int(p.ent_off[b]))
+            n_ent.append(int(p.n_ent[b]))
+        q_seq.append(p.q_seq.to(torch.int64) + seqs)
+        rows += p.kv.shape[0]
+        ents += int(p.n_ent.sum())
+        seqs += p.B
+    cat = lambda name: torch.cat([getattr(p, name) for p in parts])  # noqa: E731
+    as_dev = lambda v: torch.tensor(v, dtype=torch.int64, device=dev)  # noqa: E731
+    f = dict(name=p0.name, B=seqs, T=torch.tensor(Ts, dtype=torch.int64), D=p0.D, H=p0.H,
+             m=p0.m, span=p0.span, W=p0.W, fmt=p0.fmt, kv=cat("kv"), gate=cat("gate"),
+             kv_off=as_dev(kv_off), kv_pos0=as_dev(kv_pos0), bias=p0.bias,
+             ent_off=as_dev(ent_off), n_ent=as_dev(n_ent),
+             q_seq=torch.cat(q_seq).to(torch.int32), q_pos=cat("q_pos"), q=cat("q"),
+             sink=p0.sink, H_I=p0.H_I, d_I=p0.d_I, k=p0.k, theta=p0.theta, eps=p0.eps)
+    if p0.H_I:
+        f.update(kI=cat("kI"), ks=cat("ks"), qI=cat("qI"), qs=cat("qs"), w=cat("w"))
+    return Workload(**f)

@@ -1,0 +1,120 @@
+"""GPU parity of lightning_indexer_topk against the oracle.
+
+Integer-valued e4m3 inputs make every dot product exact, so scores and index sets must be
+bit-identical (the fp32 head accumulation order is part of the definition).  With real
+FP8 inputs the dot products round differently, so selections may differ only among
+entries whose oracle score lies within the rounding bound of the k-th score."""
+import numpy as np
+import pytest
+import torch
+
+import _orc
+from long_context_compressed_04_b200 import CSA_DEV_CAPACITY, pipeline, synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(wl, scores=True):
+    buf = pipeline.alloc(wl, DEV)
+    sc = None
+    if scores:
+        sc = torch.full((wl.Q, max(buf.max_n, 1)), float("nan"), device=DEV)
+    pipeline.indexer_topk(wl, buf, scores_out=sc)
+    torch.cuda.synchronize()
+    return buf, sc
+
+
+def _exact(wl):
+    buf, sc = _run(wl)
+    assert int(buf.dev_status.item()) == 0
+    idx_o, s_o = _orc.indexer(wl.to("cpu"))
+    s_g = sc.cpu().numpy()
+    n = (_orc.i64(wl.q_pos) + 1) // wl.m
+    for q in range(wl.Q):
+        assert np.array_equal(s_g[q, :n[q]].view(np.uint32), s_o[q, :n[q]].view(np.uint32)), q
+    assert np.array_equal(buf.idx.cpu().numpy(), idx_o)
+    return buf.idx.cpu().numpy()
+
+
+def test_decode_4k_shape_bit_exact():
+    # CSA decode, 1 sequence of 4096 tokens: 1024 entries, 4 indexer heads x 64, top-64
+    _exact(synth.csa_decode_4k(device=DEV))
+
+
+@pytest.mark.parametrize("HI,dI,k", [(64, 128, 512), (4, 64, 64), (16, 128, 100)])
+def test_ragged_batch_bit_exact(HI, dI, k):
+    # visible counts 1500, 4000, 300 (< k for some shapes: padded with -1), 7
+    wl = synth.make_workload("t", B=4, T=[6003, 16000, 1201, 29], D=128, H=16, m=4, span=8,
+                             H_I=HI, d_I=dI, k=k, seed=21, device=DEV)
+    idx = _exact(wl)
+    assert np.all(idx[3, 7:] == -1) and idx[3, :7].tolist() == list(range(7))
+
+
+def test_ties_break_toward_lower_index():
+    wl = synth.make_workload("t", B=2, T=[8192, 5000], D=128, H=16, m=4, span=8, H_I=8,
+                             d_I=128, k=256, seed=22, device=DEV)
+    # only 5 distinct key rows -> massive ties at the k-th score
+    g = torch.Generator(device=DEV).manual_seed(0)
+    rows = wl.kI[torch.randint(0, 5, (wl.kI.shape[0],), device=DEV, generator=g)]
+    wl.kI.copy_(rows)
+    wl.w.fill_(1.0)
+    _exact(wl)
+
+
+def _abs_bound(wl, q):
+    """fp32 rounding bound of one query's scores: the dot products accumulate 128 e4m3
+    products in fp32 (error <= 2^-17 of the sum of |products| each, doubled for margin)
+    and the head chain adds <= 2^-18 of |s| per step."""
+    cw = wl.to("cpu")
+    qv = torch.from_numpy(_orc.u8(cw.qI[q])).view(torch.float8_e4m3fn).double().abs()
+    kv = torch.from_numpy(_orc.u8(cw.kI)).view(torch.float8_e4m3fn).double().abs()
+    b = int(cw.q_seq[q])
+    e0, n = int(cw.ent_off[b]), (int(cw.q_pos[q]) + 1) // wl.m
+    ws = (cw.w[q].double() * cw.qs[q].double())
+    mag = (kv[e0:e0 + n] @ qv.T) @ ws * cw.ks[e0:e0 + n].double()
+    return (2.0 ** -16 * mag).numpy()
+
+
+def test_real_fp8_inputs_select_within_rounding():
+    wl = synth.make_workload("t", B=3, T=[40000, 9000, 20001], D=128, H=16, m=4, span=8,
+                             H_I=64, d_I=128, k=512, indexer="fp8", seed=23, device=DEV)
+    buf, sc = _run(wl)
+    idx_o, s_o = _orc.indexer(wl.to("cpu"))
+    idx_g = buf.idx.cpu().numpy()
+    s_g = sc.cpu().numpy()
+    n = (_orc.i64(wl.q_pos) + 1) // wl.m
+    for q in range(wl.Q):
+        bound = _abs_bound(wl, q) + 2.0 ** -18 * 64 * np.abs(s_o[q, :n[q]])
+        assert np.all(np.abs(s_g[q, :n[q]] - s_o[q, :n[q]]) <= bound)
+        order = np.argsort(-s_o[q, :n[q]], kind="stable")
+        kth = s_o[q, order[wl.k - 1]]
+        diff = set(idx_g[q].tolist()) ^ set(idx_o[q].tolist())
+        for i in diff:
+            assert abs(s_o[q, i] - kth) <= 2 * (bound[i] + bound[order[wl.k - 1]]), (q, i)
+
+
+def test_batch_invariance_bitwise():
+    base = synth.make_workload("t", B=7, T=[3001, 60000, 777, 12345, 4096, 50, 99999], D=128,
+                               H=16, m=4, span=8, H_I=64, d_I=128, k=512, indexer="fp8",
+                               seed=24, device=DEV)
+    parts = synth.split(base)
+    target = 3
+    ref_buf, ref_sc = _run(synth.merge([parts[target]]))
+    for order in ([1, 3, 0], [6, 5, 4, 3, 2, 1, 0], [3] + [i for i in range(7) if i != 3]):
+        wl = synth.merge([parts[i] for i in order])
+        buf, sc = _run(wl)
+        slot = order.index(target)
+        n = int(parts[target].n_ent[0])
+        assert torch.equal(buf.idx[slot], ref_buf.idx[0])
+        assert torch.equal(sc[slot, :n].view(torch.int32), ref_sc[0, :n].view(torch.int32))
+
+
+def test_capacity_flag_when_max_n_too_small():
+    wl = synth.make_workload("t", B=1, T=[4000], D=128, H=16, m=4, span=8, H_I=4, d_I=64, k=8,
+                             seed=25, device=DEV)
+    buf = pipeline.alloc(wl, DEV)
+    buf.max_n = 500
+    pipeline.indexer_topk(wl, buf)
+    torch.cuda.synchronize()
+    assert int(buf.dev_status.item()) & CSA_DEV_CAPACITY
