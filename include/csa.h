@@ -200,6 +200,37 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
                             size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * lightning_indexer_topk_noalloc -- the same scores and selection as
+ * lightning_indexer_topk, for callers that cannot allocate device memory (no counterpart
+ * on the pages: it is a deployment variant of this library).
+ *   Some callers cannot call cudaMalloc or provide a workspace: a plugin inside a host
+ *   framework that owns the whole device-memory pool and gives plugins no scratch, or a
+ *   latency-critical loop where a cudaMalloc (which may synchronise the device) is not
+ *   allowed.  This call takes the same inputs and outputs minus the workspace and keeps
+ *   its scratch (the per-query score rows) in a device array inside the library of
+ *   CSA_NOALLOC_SCRATCH_BYTES bytes; it allocates nothing.
+ *   - A call needing more than that (csa_indexer_workspace_size(Q, max_n, k) > the size)
+ *     returns CSA_ERR_WORKSPACE with a message and launches nothing.  16 MiB covers, e.g.,
+ *     32 queries of up to 131040 visible entries.
+ *   - Every GPU that loads the library holds the array until the process exits.
+ *   - All calls on a device share the array, which keeps the last call's contents;
+ *     nothing in it has to start at zero.  Calls whose kernels overlap on the GPU (e.g.
+ *     on two unordered streams) race on it: order them on one stream.
+ *   - The first call on each device resolves the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it: make that first
+ *     call before any stream capture.
+ */
+#define CSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+csa_status_t lightning_indexer_topk_noalloc(const uint8_t* qI, const float* qI_scale,
+                                            const float* w, const uint8_t* kI,
+                                            const float* kI_scale, const int64_t* seq_len,
+                                            const int64_t* ent_off, const int32_t* q_seq,
+                                            const int32_t* q_pos, int32_t Q, int32_t B,
+                                            int32_t H_I, int32_t d_I, int32_t m, int32_t k,
+                                            int32_t max_n, int32_t* idx_out, float* scores_out,
+                                            int64_t ld_scores, int32_t* dev_status, void* stream);
+
+/*
  * Launch accounting and kernel timing (no counterpart on the pages; instrumentation).
  *   csa_launch_count: kernels this library has launched in the process so far.
  *   csa_profile_enable(1): from now on every launch is bracketed by a CUDA event pair

@@ -59,6 +59,9 @@ _SIGS = {
     "dense_hca_attn": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32,
                                       _I32, _I32, _I32, _F32, _F32, _F32, _I32, _P, _P, _SZ, _P,
                                       _P]),
+    "lightning_indexer_topk_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32,
+                                                      _I32, _I32, _I32, _I32, _I32, _I32, _P, _P,
+                                                      _I64, _P, _P]),
     "csa_launch_count": (ctypes.c_longlong, []),
     "csa_profile_enable": (None, [ctypes.c_int]),
     "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int]),
@@ -151,6 +154,22 @@ def lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_se
         q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out), ld_scores,
         _p(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
         _p(dev_status), _s(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def lightning_indexer_topk_noalloc(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_seq, q_pos,
+                                   idx_out, *, B: int, H_I: int, d_I: int, m: int, k: int,
+                                   max_n: int, scores_out=None, ld_scores: int = 0,
+                                   dev_status=None, stream=None):
+    """lightning_indexer_topk without a workspace, for callers that cannot allocate device
+    memory: the scratch lives in a fixed 16 MiB device array inside libcsa, shared by all
+    calls on a device (calls that overlap on the GPU race on it)."""
+    _check(_lib.lightning_indexer_topk_noalloc(
+        _p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), _p(seq_len), _p(ent_off), _p(q_seq),
+        _p(q_pos), q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out),
+        ld_scores, _p(dev_status), _s(stream)))
 
 
 def sparse_mqa_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos, idx, sink,

@@ -69,6 +69,15 @@ csa_status_t compress_common(int m, int span, const void* kv, const void* gate,
 
 }  // namespace
 
+namespace csa {
+void set_error_message(const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+}  // namespace csa
+
 extern "C" {
 
 int csa_version(void) { return 100; }

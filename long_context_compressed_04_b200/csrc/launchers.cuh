@@ -57,4 +57,7 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream);
 cudaError_t launch_attn_simt(const AttnArgs& a, int Q, int D, cudaStream_t stream);
 
+// Sets the thread-local message csa_last_error() returns (printf-style).
+void set_error_message(const char* fmt, ...);
+
 }  // namespace csa
