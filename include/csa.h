@@ -130,7 +130,8 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
  * ascending entry order, padded with -1 when n_vis < k.
  * Arguments:
  *   qI e4m3 [Q, H_I, d_I]; qI_scale, w fp32 [Q, H_I]; kI e4m3 [ent_rows, d_I];
- *   kI_scale fp32 [ent_rows]; seq_len, ent_off int64 [B]; q_seq, q_pos int32 [Q]
+ *   kI_scale fp32 [ent_rows] (ent_rows: rows in kI / kI_scale; every visible entry's row
+ *   ent_off[b] + i must be < ent_rows, else CSA_DEV_OOB and the rest are skipped); seq_len, ent_off int64 [B]; q_seq, q_pos int32 [Q]
  *   H_I in 1..64, d_I in {64, 128}, m >= 1 (4 for CSA), 1 <= k <= 2048
  *   max_n: upper bound of n_vis over the batch (sizes the workspace)
  *   idx_out int32 [Q, k]
@@ -141,7 +142,7 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
  */
 size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k);
 csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, const float* w,
-                                    const uint8_t* kI, const float* kI_scale,
+                                    const uint8_t* kI, const float* kI_scale, int64_t ent_rows,
                                     const int64_t* seq_len, const int64_t* ent_off,
                                     const int32_t* q_seq,
                                     const int32_t* q_pos, int32_t Q, int32_t B, int32_t H_I,
@@ -223,7 +224,8 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
 #define CSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 csa_status_t lightning_indexer_topk_noalloc(const uint8_t* qI, const float* qI_scale,
                                             const float* w, const uint8_t* kI,
-                                            const float* kI_scale, const int64_t* seq_len,
+                                            const float* kI_scale, int64_t ent_rows,
+                                            const int64_t* seq_len,
                                             const int64_t* ent_off, const int32_t* q_seq,
                                             const int32_t* q_pos, int32_t Q, int32_t B,
                                             int32_t H_I, int32_t d_I, int32_t m, int32_t k,

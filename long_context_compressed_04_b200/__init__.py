@@ -49,7 +49,7 @@ _SIGS = {
     "hca_compress": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32,
                                     _F32, _F32, _P, _P, _P]),
     "csa_indexer_workspace_size": (_SZ, [_I32, _I32, _I32]),
-    "lightning_indexer_topk": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32,
+    "lightning_indexer_topk": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32,
                                               _I32, _I32, _I32, _I32, _P, _P, _I64, _P, _SZ, _P,
                                               _P]),
     "sparse_mqa_attn": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P,
@@ -59,7 +59,8 @@ _SIGS = {
     "dense_hca_attn": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32,
                                       _I32, _I32, _I32, _F32, _F32, _F32, _I32, _P, _P, _SZ, _P,
                                       _P]),
-    "lightning_indexer_topk_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I32,
+    "lightning_indexer_topk_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P,
+                                                      _I32,
                                                       _I32, _I32, _I32, _I32, _I32, _I32, _P, _P,
                                                       _I64, _P, _P]),
     "csa_launch_count": (ctypes.c_longlong, []),
@@ -149,7 +150,8 @@ def lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_se
                            workspace, *, B: int, H_I: int, d_I: int, m: int, k: int, max_n: int,
                            scores_out=None, ld_scores: int = 0, dev_status=None, stream=None):
     _check(_lib.lightning_indexer_topk(
-        _p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), _p(seq_len), _p(ent_off), _p(q_seq),
+        _p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), kI_scale.numel(), _p(seq_len),
+        _p(ent_off), _p(q_seq),
         _p(q_pos),
         q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out), ld_scores,
         _p(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
@@ -167,7 +169,8 @@ def lightning_indexer_topk_noalloc(qI, qI_scale, w, kI, kI_scale, seq_len, ent_o
     memory: the scratch lives in a fixed 16 MiB device array inside libcsa, shared by all
     calls on a device (calls that overlap on the GPU race on it)."""
     _check(_lib.lightning_indexer_topk_noalloc(
-        _p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), _p(seq_len), _p(ent_off), _p(q_seq),
+        _p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), kI_scale.numel(), _p(seq_len),
+        _p(ent_off), _p(q_seq),
         _p(q_pos), q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out),
         ld_scores, _p(dev_status), _s(stream)))
 

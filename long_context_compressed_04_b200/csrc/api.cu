@@ -118,7 +118,7 @@ size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k) {
 }
 
 csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, const float* w,
-                                    const uint8_t* kI, const float* kI_scale,
+                                    const uint8_t* kI, const float* kI_scale, int64_t ent_rows,
                                     const int64_t* seq_len, const int64_t* ent_off,
                                     const int32_t* q_seq,
                                     const int32_t* q_pos, int32_t Q, int32_t B, int32_t H_I,
@@ -131,7 +131,8 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     REQUIRE(qI && qI_scale && w && seq_len && ent_off && q_seq && q_pos && idx_out,
             "null pointer argument");
     REQUIRE(max_n >= 0, "max_n must be >= 0");
-    REQUIRE(max_n == 0 || (kI && kI_scale), "null key pointer");
+    REQUIRE(ent_rows >= 0 && ent_rows < (1ll << 31), "ent_rows out of range");
+    REQUIRE(max_n == 0 || ent_rows == 0 || (kI && kI_scale), "null key pointer");
     REQUIRE(aligned(qI, 16) && (kI == nullptr || aligned(kI, 16)), "qI and kI must be 16-byte aligned");
     REQUIRE(B >= 1 && m >= 1, "B and m must be >= 1");
     SUPPORT(H_I >= 1 && H_I <= 64, "indexer heads %d not supported (1..64)", H_I);
@@ -144,8 +145,14 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     float* scores = scores_out ? scores_out : (float*)workspace;
     const int64_t ld = scores_out ? ld_scores : (int64_t)round_up((size_t)max_n, 32);
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = csa::launch_indexer_simt(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_seq, q_pos,
-                                             Q, B, H_I, d_I, m, max_n, scores, ld, dev_status, s);
+    cudaError_t e;
+    if (csa::indexer_tc_supported(H_I, d_I))
+        e = csa::launch_indexer_tc(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
+                                   q_seq, q_pos, Q, B, H_I, m, max_n, scores, ld, dev_status, s);
+    else
+        e = csa::launch_indexer_simt(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
+                                     q_seq, q_pos, Q, B, H_I, d_I, m, max_n, scores, ld,
+                                     dev_status, s);
     if (e != cudaSuccess) return cuda_status(e, "indexer launch");
     e = csa::launch_topk(scores, ld, q_seq, q_pos, seq_len, Q, B, m, max_n, k, idx_out, dev_status,
                          s);

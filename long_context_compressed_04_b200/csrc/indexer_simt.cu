@@ -15,7 +15,7 @@ namespace csa {
 template <int DI>
 __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
     const uint8_t* __restrict__ qI, const float* __restrict__ qs, const float* __restrict__ w,
-    const uint8_t* __restrict__ kI, const float* __restrict__ ks,
+    const uint8_t* __restrict__ kI, const float* __restrict__ ks, int64_t ent_rows,
     const int64_t* __restrict__ seq_len, const int64_t* __restrict__ ent_off, const int32_t* __restrict__ q_seq,
     const int32_t* __restrict__ q_pos, int B, int HI, int m, int max_n,
     float* __restrict__ scores, int64_t ld, int32_t* __restrict__ dev_status) {
@@ -33,6 +33,11 @@ __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
     if (n > max_n) {
         if (blockIdx.x == 0 && threadIdx.x == 0) flag(dev_status, CSA_DEV_CAPACITY);
         n = max_n;
+    }
+    const int64_t avail = ent_rows - ent_off[b];
+    if ((int64_t)n > avail) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
+        n = avail > 0 ? (int)avail : 0;
     }
     if ((int64_t)blockIdx.x * blockDim.x >= n) return;
     for (int x = threadIdx.x; x < HI * DI; x += blockDim.x)
@@ -67,7 +72,8 @@ __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
 }
 
 cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float* w,
-                                const uint8_t* kI, const float* ks, const int64_t* seq_len,
+                                const uint8_t* kI, const float* ks, int64_t ent_rows,
+                                const int64_t* seq_len,
                                 const int64_t* ent_off, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
                                 int HI, int dI, int m, int max_n, float* scores, int64_t ld,
                                 int32_t* st, cudaStream_t stream) {
@@ -77,12 +83,12 @@ cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float*
     LaunchScope scope(kKIndexerSimt, stream);
     if (dI == 64) {
         indexer_score_simt_kernel<64><<<grid, 128, smem, stream>>>(
-            qI, qs, w, kI, ks, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n, scores, ld, st);
+            qI, qs, w, kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n, scores, ld, st);
     } else {
         cudaFuncSetAttribute(indexer_score_simt_kernel<128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         indexer_score_simt_kernel<128><<<grid, 128, smem, stream>>>(
-            qI, qs, w, kI, ks, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n, scores, ld, st);
+            qI, qs, w, kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n, scores, ld, st);
     }
     return cudaGetLastError();
 }

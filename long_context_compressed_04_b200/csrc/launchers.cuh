@@ -6,7 +6,7 @@
 namespace csa {
 
 // Kernel kinds for launch accounting (names in prof.cu).
-enum KernelKind { kKCompress = 0, kKIndexerSimt, kKTopk, kKAttnSimt, kKernelKinds };
+enum KernelKind { kKCompress = 0, kKIndexerSimt, kKTopk, kKAttnSimt, kKIndexerTc, kKernelKinds };
 
 // Counts one kernel launch; with timing enabled, brackets it with CUDA events on `stream`.
 class LaunchScope {
@@ -48,10 +48,18 @@ cudaError_t launch_compress(int span, const void* kv, const void* gate, const fl
                             int fmt, float theta, float eps, void* entries, int32_t* st,
                             cudaStream_t stream);
 cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float* w,
-                                const uint8_t* kI, const float* ks, const int64_t* seq_len,
+                                const uint8_t* kI, const float* ks, int64_t ent_rows,
+                                const int64_t* seq_len,
                                 const int64_t* ent_off, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
                                 int HI, int dI, int m, int max_n, float* scores, int64_t ld,
                                 int32_t* st, cudaStream_t stream);
+bool indexer_tc_supported(int HI, int dI);
+cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w,
+                              const uint8_t* kI, const float* ks, int64_t ent_rows,
+                              const int64_t* seq_len, const int64_t* ent_off,
+                              const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
+                              int m, int max_n, float* scores, int64_t ld, int32_t* st,
+                              cudaStream_t stream);
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream);

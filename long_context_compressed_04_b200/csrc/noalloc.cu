@@ -37,11 +37,11 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 extern "C" csa_status_t lightning_indexer_topk_noalloc(
     const uint8_t* qI, const float* qI_scale, const float* w, const uint8_t* kI,
-    const float* kI_scale, const int64_t* seq_len, const int64_t* ent_off, const int32_t* q_seq,
+    const float* kI_scale, int64_t ent_rows, const int64_t* seq_len, const int64_t* ent_off, const int32_t* q_seq,
     const int32_t* q_pos, int32_t Q, int32_t B, int32_t H_I, int32_t d_I, int32_t m, int32_t k,
     int32_t max_n, int32_t* idx_out, float* scores_out, int64_t ld_scores, int32_t* dev_status,
     void* stream) {
-    if (Q == 0) return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off,
+    if (Q == 0) return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
                                               q_seq, q_pos, Q, B, H_I, d_I, m, k, max_n, idx_out,
                                               scores_out, ld_scores, nullptr, 0, dev_status,
                                               stream);
@@ -75,7 +75,7 @@ extern "C" csa_status_t lightning_indexer_topk_noalloc(
         }
         scratch = g_scratch_ptr[dev];
     }
-    return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_seq, q_pos,
+    return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off, q_seq, q_pos,
                                   Q, B, H_I, d_I, m, k, max_n, idx_out, scores_out, ld_scores,
                                   scratch, (size_t)CSA_NOALLOC_SCRATCH_BYTES, dev_status, stream);
 }

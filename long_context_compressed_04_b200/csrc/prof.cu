@@ -40,7 +40,7 @@ cudaEvent_t take_event() {
 
 const char* kernel_name(int kind) {
     static const char* names[kKernelKinds] = {"compress", "indexer_score_simt", "topk_radix",
-                                              "attn_simt"};
+                                              "attn_simt", "indexer_score_tc"};
     return (kind >= 0 && kind < kKernelKinds) ? names[kind] : "?";
 }
 

@@ -83,12 +83,12 @@ def test_workspace_is_checked_on_host():
     P = ctypes.c_void_p
     fake = P(4096)
     need = lib.csa_indexer_workspace_size(2, 1000, 64)
-    st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, fake, fake, fake, fake, 2, 2, 4, 64,
+    st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, 100, fake, fake, fake, fake, 2, 2, 4, 64,
                                     4, 64, 1000, fake, None, 0, fake, need - 1, None, None)
     assert st == 4 and b"workspace" in lib.csa_last_error()
-    st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, fake, fake, fake, fake, 2, 2, 4, 64,
+    st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, 100, fake, fake, fake, fake, 2, 2, 4, 64,
                                     4, 4096, 1000, fake, None, 0, fake, need, None, None)
     assert st == 2 and b"k =" in lib.csa_last_error()
-    st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, fake, fake, fake, fake, 2, 2, 80, 64,
+    st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, 100, fake, fake, fake, fake, 2, 2, 80, 64,
                                     4, 64, 1000, fake, None, 0, fake, need, None, None)
     assert st == 2

@@ -51,8 +51,15 @@ def test_ragged_batch_bit_exact(HI, dI, k):
     assert np.all(idx[3, 7:] == -1) and idx[3, :7].tolist() == list(range(7))
 
 
+def test_long_sequences_many_work_items_bit_exact():
+    # 130K + 25K + 750 entries: many 1024-entry work items per query on the tensor-core path
+    wl = synth.make_workload("t", B=3, T=[520003, 100000, 3001], D=128, H=16, m=4, span=8,
+                             H_I=64, d_I=128, k=1024, seed=26, device=DEV)
+    _exact(wl)
+
+
 def test_ties_break_toward_lower_index():
-    wl = synth.make_workload("t", B=2, T=[8192, 5000], D=128, H=16, m=4, span=8, H_I=8,
+    wl = synth.make_workload("t", B=2, T=[8192, 5000], D=128, H=16, m=4, span=8, H_I=16,
                              d_I=128, k=256, seed=22, device=DEV)
     # only 5 distinct key rows -> massive ties at the k-th score
     g = torch.Generator(device=DEV).manual_seed(0)
