@@ -227,6 +227,7 @@ def main():
     ap.add_argument("--workload", default="csa_decode_128k_b32", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -255,8 +256,29 @@ def main():
     torch.cuda.synchronize()
     del all_seq, all_ent
 
-    def step():
+    def step_eager():
         pipeline.step(wl, buf, new_seq, new_ent)
+
+    # the step's launches are captured once into a CUDA graph and replayed, so the timed
+    # region measures device work rather than Python/ctypes launch overhead
+    for _ in range(args.warmup):
+        step_eager()
+    torch.cuda.synchronize()
+    graph = None
+    kernels_per_step = 0
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        c0 = L.csa_launch_count()
+        with torch.cuda.graph(graph):
+            step_eager()
+        kernels_per_step = L.csa_launch_count() - c0   # libcsa kernels in the graph
+        torch.cuda.synchronize()
+
+    def step():
+        if graph is not None:
+            graph.replay()
+        else:
+            step_eager()
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
 
@@ -281,7 +303,7 @@ def main():
             step()
             ev[i][1].record()
         barrier()
-    launches = L.csa_launch_count() - launches0
+    launches = L.csa_launch_count() - launches0 + kernels_per_step * K
     ms = sum(a.elapsed_time(b) for a, b in ev)
     t = torch.tensor([ms], device=dev, dtype=torch.float64)
     if dist:
@@ -289,12 +311,13 @@ def main():
     ms_max = float(t.item())
     assert int(buf.dev_status.item()) == 0, "device status flagged during the run"
 
-    # second pass: the same steps with per-kernel CUDA events (roofline of each kernel)
+    # second pass: the same steps, launched eagerly, with per-kernel CUDA events recorded on
+    # the launching stream (roofline of each kernel)
     L.csa_profile_collect()
     L.csa_profile_enable(True)
     for i in range(K):
         flush.zero_()
-        step()
+        step_eager()
     torch.cuda.synchronize()
     L.csa_profile_enable(False)
     per_kernel = L.csa_profile_collect()
@@ -319,8 +342,8 @@ def main():
         ee[i][0].record()
         for k2, v in pinned.items():
             h_in[k2].copy_(v, non_blocking=True)
-        wl.kv[last_rows] = pin_kv.to(dev, non_blocking=True)
-        wl.gate[last_rows] = pin_gate.to(dev, non_blocking=True)
+        wl.kv.index_copy_(0, last_rows, pin_kv.to(dev, non_blocking=True))
+        wl.gate.index_copy_(0, last_rows, pin_gate.to(dev, non_blocking=True))
         step()
         out_host.copy_(buf.out, non_blocking=True)
         ee[i][1].record()
@@ -370,6 +393,7 @@ def main():
         "e2e": {"value": Qtot * E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
+        "launch": "cuda graph replay" if graph is not None else "eager",
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

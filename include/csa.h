@@ -163,14 +163,15 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
  *   l_j = softmax_scale * < RoPE_t(q[q,h]), k_j >,  M = max(sink[h], max_j l_j),
  *   o = sum_j e^(l_j-M) k_j / (e^(sink[h]-M) + sum_j e^(l_j-M)),  out = RoPE_{-t}(o) (bf16).
  * Arguments:
- *   q bf16 [Q, H, D]; entries in format fmt; kv bf16 raw rows for the window;
+ *   q bf16 [Q, H, D]; entries in format fmt, ent_rows rows (an entry row ent_off[b] + i at or
+ *   past ent_rows sets CSA_DEV_OOB and is skipped); kv bf16 raw rows for the window;
  *   idx int32 [Q, k] (entries < n_vis(t) for ratio m, or -1 = skip); sink fp32 [H]
  *   H in {16, 64, 128}; D 128 (bf16) or 576 (either format); 0 <= W <= 128
  *   out bf16 [Q, H, D]
  * Pointers q/kv/entries/out must be 16-byte aligned.  Out-of-range indices set CSA_DEV_OOB
  * and are skipped.
  */
-csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt,
+csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,
                              const int64_t* seq_len, const int64_t* ent_off, const void* kv,
                              const int64_t* kv_off,
                              const int64_t* kv_pos0, const int32_t* q_seq,
@@ -191,7 +192,7 @@ csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt,
  *   on the query's own n_vis and the shape, so results do not depend on the batch).
  */
 size_t dense_hca_workspace_size(int32_t Q, int32_t H, int32_t D, int32_t max_n);
-csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
+csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,
                             const int64_t* seq_len, const int64_t* ent_off, const void* kv,
                             const int64_t* kv_off,
                             const int64_t* kv_pos0, const int32_t* q_seq, const int32_t* q_pos,

@@ -52,11 +52,11 @@ _SIGS = {
     "lightning_indexer_topk": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32,
                                               _I32, _I32, _I32, _I32, _P, _P, _I64, _P, _SZ, _P,
                                               _P]),
-    "sparse_mqa_attn": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P,
+    "sparse_mqa_attn": (ctypes.c_int, [_P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P,
                                        _I32, _I32, _I32, _I32, _I32, _F32, _F32, _F32, _P, _P,
                                        _P]),
     "dense_hca_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
-    "dense_hca_attn": (ctypes.c_int, [_P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32,
+    "dense_hca_attn": (ctypes.c_int, [_P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32,
                                       _I32, _I32, _I32, _F32, _F32, _F32, _I32, _P, _P, _SZ, _P,
                                       _P]),
     "lightning_indexer_topk_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P,
@@ -181,7 +181,7 @@ def sparse_mqa_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_
                     softmax_scale: float, rope_theta: float = 10000.0, eps: float = 1e-6,
                     dev_status=None, stream=None):
     _check(_lib.sparse_mqa_attn(
-        _p(q), _p(entries), fmt, _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
+        _p(q), _p(entries), fmt, entries.shape[0], _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
         _p(q_pos), _p(idx), k, m, _p(sink), q_seq.numel(), B, H, D, W, softmax_scale,
         rope_theta, eps, _p(out), _p(dev_status), _s(stream)))
 
@@ -191,7 +191,7 @@ def dense_hca_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_p
                    softmax_scale: float, rope_theta: float = 10000.0, eps: float = 1e-6,
                    dev_status=None, stream=None):
     _check(_lib.dense_hca_attn(
-        _p(q), _p(entries), fmt, _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
+        _p(q), _p(entries), fmt, entries.shape[0], _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
         _p(q_pos), m, _p(sink), q_seq.numel(), B, H, D, W, softmax_scale, rope_theta, eps,
         max_n, _p(out), _p(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(),

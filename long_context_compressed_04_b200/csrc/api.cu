@@ -159,7 +159,7 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     return cuda_status(e, "top-k launch");
 }
 
-static csa_status_t attn_validate(const void* q, const void* entries, int32_t fmt,
+static csa_status_t attn_validate(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,
                                   const int64_t* seq_len, const int64_t* ent_off, const void* kv, const int64_t* kv_off,
                                   const int64_t* kv_pos0, const int32_t* q_seq,
                                   const int32_t* q_pos, const float* sink, int32_t B,
@@ -175,12 +175,13 @@ static csa_status_t attn_validate(const void* q, const void* entries, int32_t fm
     SUPPORT(fmt == CSA_KV_BF16 || D == 576, "fp8 entry format needs D = 576");
     SUPPORT(H == 16 || H == 64 || H == 128, "query heads %d not supported (16, 64, 128)", H);
     REQUIRE(W >= 0 && W <= 128, "window %d outside 0..128", W);
+    REQUIRE(ent_rows >= 0 && ent_rows < (1ll << 31), "ent_rows out of range");
     REQUIRE(B >= 1 && m >= 1, "B and m must be >= 1");
     REQUIRE(scale > 0.f && theta > 1.f && eps >= 0.f, "bad softmax_scale / rope_theta / eps");
     return ok();
 }
 
-csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt,
+csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,
                              const int64_t* seq_len, const int64_t* ent_off, const void* kv, const int64_t* kv_off,
                              const int64_t* kv_pos0, const int32_t* q_seq,
                              const int32_t* q_pos, const int32_t* idx, int32_t k, int32_t m,
@@ -189,26 +190,28 @@ csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt,
                              void* out, int32_t* dev_status, void* stream) {
     REQUIRE(Q >= 0, "Q must be >= 0");
     if (Q == 0) return ok();
-    csa_status_t v = attn_validate(q, entries, fmt, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
+    csa_status_t v = attn_validate(q, entries, fmt, ent_rows, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
                                    sink, B, H, D, W, m, softmax_scale, rope_theta, eps, out);
     if (v != CSA_OK) return v;
     REQUIRE(idx != nullptr, "idx must not be null");
     SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
     csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, ent_off, (const uint16_t*)kv,
-                    kv_off, kv_pos0, q_seq, q_pos, seq_len, idx, sink, (uint16_t*)out, dev_status,
+                    kv_off, kv_pos0, q_seq, q_pos, seq_len, idx, ent_rows, sink, (uint16_t*)out, dev_status,
                     k, m, B, H, W, fmt, softmax_scale, eps, log2((double)rope_theta)};
+    if (csa::attn_tc_supported(H, D, fmt))
+        return cuda_status(csa::launch_attn_tc(a, Q, 0, nullptr, (cudaStream_t)stream),
+                           "attention launch");
     return cuda_status(csa::launch_attn_simt(a, Q, D, (cudaStream_t)stream), "attention launch");
 }
 
 size_t dense_hca_workspace_size(int32_t Q, int32_t H, int32_t D, int32_t max_n) {
-    (void)Q;
-    (void)H;
-    (void)D;
-    (void)max_n;
-    return 256;
+    if (Q <= 0 || max_n < 0) return 256;
+    size_t need = 0;
+    if (csa::attn_tc_supported(H, D, CSA_KV_BF16)) need = csa::attn_tc_workspace_bytes(Q, max_n);
+    return round_up(need, 256) + 256;
 }
 
-csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
+csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,
                             const int64_t* seq_len, const int64_t* ent_off, const void* kv, const int64_t* kv_off,
                             const int64_t* kv_pos0, const int32_t* q_seq, const int32_t* q_pos,
                             int32_t m, const float* sink, int32_t Q, int32_t B, int32_t H,
@@ -217,7 +220,7 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
                             size_t workspace_bytes, int32_t* dev_status, void* stream) {
     REQUIRE(Q >= 0, "Q must be >= 0");
     if (Q == 0) return ok();
-    csa_status_t v = attn_validate(q, entries, fmt, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
+    csa_status_t v = attn_validate(q, entries, fmt, ent_rows, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
                                    sink, B, H, D, W, m, softmax_scale, rope_theta, eps, out);
     if (v != CSA_OK) return v;
     REQUIRE(max_n >= 0, "max_n must be >= 0");
@@ -225,8 +228,11 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt,
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
         return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", need);
     csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, ent_off, (const uint16_t*)kv,
-                    kv_off, kv_pos0, q_seq, q_pos, seq_len, nullptr, sink, (uint16_t*)out, dev_status,
+                    kv_off, kv_pos0, q_seq, q_pos, seq_len, nullptr, ent_rows, sink, (uint16_t*)out, dev_status,
                     0, m, B, H, W, fmt, softmax_scale, eps, log2((double)rope_theta)};
+    if (csa::attn_tc_supported(H, D, fmt))
+        return cuda_status(csa::launch_attn_tc(a, Q, max_n, workspace, (cudaStream_t)stream),
+                           "attention launch");
     return cuda_status(csa::launch_attn_simt(a, Q, D, (cudaStream_t)stream), "attention launch");
 }
 

@@ -34,7 +34,7 @@ __device__ __forceinline__ bool load_key(const AttnArgs& a, int b, int t, int n_
         const int e = a.idx ? a.idx[(int64_t)blockIdx.y * a.k + vk] : vk;
         if (e < 0) {
             valid = false;
-        } else if (e >= n_vis) {
+        } else if (e >= n_vis || a.ent_off[b] + e >= a.ent_rows) {
             valid = false;
             if (lane == 0 && blockIdx.x == 0) flag(a.st, CSA_DEV_OOB);
         } else {

@@ -1,0 +1,834 @@
+// Steps a5/a6 on the 5th-generation tensor cores: shared-KV MQA over compressed entries
+// plus the sliding window, with the attention sink and partial / inverse RoPE
+// ("DeepSeek-V4 深度分析报告" 2.1 CSA / HCA and "其他注意力技术细节").  Shape: 64 query
+// heads, head dim 128, bf16 entries.
+//
+// The keys of a query form a list of 128-key tiles: tile 0 is the window (its raw rows
+// RMSNormed and RoPEd here, one row per thread), tiles 1.. are the selected entries
+// (sparse, gathered by index) or all visible entries (dense, contiguous).  A work item is
+// (query, chunk of tiles).  Sparse attention uses one chunk per query and finishes in
+// this kernel.  Dense attention splits every query into fixed 8-tile chunks whose fp32
+// partial states (running max, sum, unnormalised output) a second kernel combines in
+// chunk order.  The split depends only on the query's own length, never on the batch, so
+// both paths are batch-invariant.
+//
+// Roles per CTA (8 warps, persistent over items):
+//   warp 0      producer: dense tiles by two 2D TMA loads (64 channels x 128 rows each,
+//               128-byte swizzle), sparse tiles by zero-filling 16-byte cp.async gathers to
+//               the same swizzled layout; a per-tile validity mask; 3-stage ring.
+//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
+//               S = Q K^T as two M=64 x N=64 halves (keys 0-63 -> TMEM lanes 0-15 of each
+//               quarter, keys 64-127 -> lanes 16-31) and O_tile = P V as two M=64 x N=64
+//               halves (channels 0-63 / 64-127), V being the key tile read MN-major.
+//   warps 4-7   per item: q heads RoPEd at t into shared memory and the window tile; per
+//               tile: S from TMEM (thread = one head x 64 keys), online softmax in the
+//               log2 domain with the sink as the initial state, P as bf16 into shared
+//               memory, then O += corr * O_tile kept in registers (thread = one head x 64
+//               channels); finally normalise, inverse RoPE, store (or write the partial).
+// All waits are bounded (timeout -> CSA_DEV_TIMEOUT, drain, free TMEM, return).
+#include <cstring>
+#include <mutex>
+
+#include "launchers.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+namespace {
+
+constexpr int kH = 64;
+constexpr int kD = 128;
+constexpr int kTK = 128;                     // keys per tile
+constexpr int kStages = 3;
+constexpr int kBlk = kTK * 128;              // one 64-channel slice of a key tile (16 KB)
+constexpr int kTileBytes = 2 * kBlk;         // 32 KB
+constexpr int kQBlk = kH * 128;              // one 64-channel slice of Q (8 KB)
+constexpr int kPBlk = kH * 128;              // one 64-key slice of P (8 KB)
+constexpr int kThreads = 256;
+constexpr int kDenseChunkTiles = 8;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct AttnTcArgs {
+    const uint16_t* q;
+    const uint8_t* entries;
+    const int64_t* ent_off;
+    const uint16_t* kv;
+    const int64_t* kv_off;
+    const int64_t* kv_pos0;
+    const int32_t* q_seq;
+    const int32_t* q_pos;
+    const int64_t* seq_len;
+    const int32_t* idx;   // nullptr: dense
+    const float* sink;
+    uint16_t* out;
+    float* part;          // dense partials [items][kH][kD + 2]
+    int32_t* st;
+    int64_t ent_rows;
+    int k, m, B, W, Q, chunk_tiles, chunks_per_q, total_items, max_n;
+    float scale_log2;
+    float eps;
+    double log2_theta;
+};
+
+struct AItem {
+    int q, b, t, c;
+    int n_vis;      // visible entries
+    int n_ent;      // entries in the key list (k for sparse, n_vis for dense)
+    int w0, n_win;
+    int tile0, ntiles;
+    bool single;    // sparse: the whole query in this item, finish here (dense never: its
+                    // chunk partials always go through the ordered combine, whatever the batch)
+    int64_t row0;
+};
+
+__device__ __forceinline__ bool get_item(const AttnTcArgs& a, int it, AItem& x, bool report) {
+    x.q = it / a.chunks_per_q;
+    x.c = it - x.q * a.chunks_per_q;
+    x.b = a.q_seq[x.q];
+    x.t = a.q_pos[x.q];
+    if (x.b < 0 || x.b >= a.B || x.t < 0 || (int64_t)x.t >= a.seq_len[x.b]) {
+        if (report && x.c == 0) flag(a.st, CSA_DEV_OOB);
+        return false;
+    }
+    x.n_vis = (x.t + 1) / a.m;
+    x.row0 = a.ent_off[x.b];
+    if (a.idx) {
+        x.n_ent = a.k;
+    } else {
+        int n = x.n_vis;
+        if (n > a.max_n) {
+            if (report && x.c == 0) flag(a.st, CSA_DEV_CAPACITY);
+            n = a.max_n;
+        }
+        const int64_t avail = a.ent_rows - x.row0;
+        if ((int64_t)n > avail) {
+            if (report && x.c == 0) flag(a.st, CSA_DEV_OOB);
+            n = avail > 0 ? (int)avail : 0;
+        }
+        x.n_ent = n;
+    }
+    x.w0 = x.t - a.W + 1 > 0 ? x.t - a.W + 1 : 0;
+    x.n_win = a.W > 0 ? x.t - x.w0 + 1 : 0;
+    const int total = 1 + (x.n_ent + kTK - 1) / kTK;
+    x.tile0 = x.c * a.chunk_tiles;
+    x.ntiles = min(a.chunk_tiles, total - x.tile0);
+    x.single = a.idx != nullptr;
+    return x.ntiles > 0;
+}
+
+// Byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-swizzled [rows x 128 B] block.
+__device__ __forceinline__ uint32_t swz(int r, int ch) {
+    return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
+                     sm100::smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// MN-major 128-byte-swizzled operand descriptor (rows of 128 B along MN, 8-row groups
+// 1024 B apart along K; LBO = distance between 64-element MN slices).
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(const void* tile, uint32_t lbo_bytes) {
+    const uint64_t addr = sm100::smem_addr(tile);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= 1ull << 46;
+    d |= 2ull << 61;
+    return d;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_e, const AttnTcArgs a) {
+    using namespace sm100;
+    constexpr uint32_t kIdescS = instr_desc(1, 1, 64, 64);
+    constexpr uint32_t kIdescPV = instr_desc(1, 1, 64, 64, 1);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint8_t* sK = smem;                              // [kStages][2][128 x 128 B]
+    uint8_t* sW = sK + kStages * kTileBytes;         // window tile [2][128 x 128 B]
+    uint8_t* sQ = sW + kTileBytes;                   // [2][64 x 128 B]
+    uint8_t* sP = sQ + 2 * kQBlk;                    // [2 buffers][2][64 x 128 B]
+    uint32_t* smask = reinterpret_cast<uint32_t*>(sP + 4 * kPBlk);   // [kStages + 1][4]
+    // per item RoPE tables, pair j of the last 64 dims: frequency, cos/sin at t, and
+    // cos/sin at the window's first position
+    float* rf = reinterpret_cast<float*>(smask + 4 * (kStages + 1));  // [32]
+    float* rqc = rf + 32;
+    float* rqs = rqc + 32;
+    float* rwc = rqs + 32;
+    float* rws = rwc + 32;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(rws + 32);
+    uint64_t* full = bars;                 // [kStages]  33 arrivals (+tx)
+    uint64_t* empty = full + kStages;      // [kStages]  MMA commit
+    uint64_t* prep_full = empty + kStages; // Q + window ready: 4 arrivals
+    uint64_t* prep_empty = prep_full + 1;  // item's MMAs done: MMA commit
+    uint64_t* s_full = prep_empty + 1;     // [2]
+    uint64_t* s_empty = s_full + 2;        // [2] 4 arrivals
+    uint64_t* p_full = s_empty + 2;        // [2] 4 arrivals
+    uint64_t* p_empty = p_full + 2;        // [2]
+    uint64_t* pv_full = p_empty + 2;       // [2]
+    uint64_t* pv_empty = pv_full + 2;      // [2] 4 arrivals
+    uint64_t* drain = pv_empty + 2;
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; s++) {
+            mbar_init(&full[s], 33);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(prep_full, 4);
+        mbar_init(prep_empty, 1);
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_empty[i], 4);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&p_empty[i], 1);
+            mbar_init(&pv_full[i], 1);
+            mbar_init(&pv_empty[i], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+        if (!a.idx) prefetch_tmap(&tmap_e);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base_smem, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_smem;
+    const uint32_t tmem_S = tmem_base;          // [2] x 64 columns
+    const uint32_t tmem_PV = tmem_base + 128;   // [2] x 64 columns
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        int stage = 0;
+        uint32_t ph = 0;
+        int issued[kStages] = {};
+        bool ok = true;
+        for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
+            AItem x;
+            if (!get_item(a, it, x, false)) continue;
+            for (int jj = 0; jj < x.ntiles; jj++) {
+                const int j = x.tile0 + jj;
+                if (j == 0) continue;  // the window tile is built by the softmax warps
+                if (!mbar_wait_warp(&empty[stage], ph ^ 1, abort_flag, a.st)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* dst = sK + stage * kTileBytes;
+                const int e0 = (j - 1) * kTK;
+                if (!a.idx) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[stage], kTileBytes);
+                        tma_load_2d(dst, &tmap_e, &full[stage], 0, (int32_t)(x.row0 + e0));
+                        tma_load_2d(dst + kBlk, &tmap_e, &full[stage], 64, (int32_t)(x.row0 + e0));
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < 4; rr++) {
+                        const unsigned v = __ballot_sync(0xffffffffu, e0 + lane + 32 * rr < x.n_ent);
+                        if (lane == 0) smask[stage * 4 + rr] = v;
+                    }
+                    __syncwarp();
+                    if (lane != 0) mbar_arrive(&full[stage]);
+                } else {
+                    const uint32_t dbase = smem_addr(dst);
+#pragma unroll
+                    for (int rr = 0; rr < 4; rr++) {
+                        const int r = lane + 32 * rr;
+                        const int v = e0 + r;
+                        bool valid = false;
+                        const uint8_t* src = a.entries;
+                        if (v < x.n_ent) {
+                            const int e = a.idx[(int64_t)x.q * a.k + v];
+                            if (e >= 0) {
+                                if (e < x.n_vis && x.row0 + e < a.ent_rows) {
+                                    valid = true;
+                                    src = a.entries + (x.row0 + e) * (int64_t)(kD * 2);
+                                } else {
+                                    flag(a.st, CSA_DEV_OOB);
+                                }
+                            }
+                        }
+                        const uint32_t nb = valid ? 16u : 0u;
+#pragma unroll
+                        for (int ch = 0; ch < 16; ch++)
+                            cp_async16(dbase + (ch >> 3) * kBlk + swz(r, ch & 7), src + ch * 16, nb);
+                        const unsigned vm = __ballot_sync(0xffffffffu, valid);
+                        if (lane == 0) smask[stage * 4 + rr] = vm;
+                    }
+                    cp_async_arrive_noinc(&full[stage]);
+                    __syncwarp();
+                }
+                if (lane == 0) mbar_arrive(&full[stage]);
+                issued[stage]++;
+                if (++stage == kStages) {
+                    stage = 0;
+                    ph ^= 1;
+                }
+            }
+        }
+        for (int s = 0; s < kStages; s++)
+            if (issued[s]) mbar_drain(&full[s], (issued[s] - 1) & 1, a.st);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            int stage = 0;
+            uint32_t ph = 0;
+            int nt = 0, nitem = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
+                AItem x;
+                if (!get_item(a, it, x, false)) continue;
+                if (!mbar_wait(prep_full, nitem & 1, abort_flag, a.st)) break;
+                fence_async_smem();
+                tc_fence_after();
+                const uint8_t* prev_k = nullptr;
+                int prev_stage = -1, prev_sb = 0;
+                for (int jj = 0; jj < x.ntiles && ok; jj++) {
+                    const int j = x.tile0 + jj;
+                    const uint8_t* kb;
+                    int my_stage = -1;
+                    if (j == 0) {
+                        kb = sW;
+                    } else {
+                        if (!mbar_wait(&full[stage], ph, abort_flag, a.st)) {
+                            ok = false;
+                            break;
+                        }
+                        // gathered tiles were written by cp.async (generic proxy)
+                        fence_async_smem();
+                        kb = sK + stage * kTileBytes;
+                        my_stage = stage;
+                        if (++stage == kStages) {
+                            stage = 0;
+                            ph ^= 1;
+                        }
+                    }
+                    const int sb = nt & 1;
+                    if (!mbar_wait(&s_empty[sb], ((nt >> 1) & 1) ^ 1, abort_flag, a.st)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int half = 0; half < 2; half++) {
+                        const uint32_t d = tmem_S + sb * 64 + ((uint32_t)(half * 16) << 16);
+#pragma unroll
+                        for (int kk = 0; kk < 8; kk++) {
+                            const int blk = kk >> 2;
+                            const uint32_t off = (uint32_t)((kk & 3) * 32) >> 4;
+                            const uint64_t ad = smem_desc_k_sw128(sQ + blk * kQBlk) + off;
+                            const uint64_t bd =
+                                smem_desc_k_sw128(kb + blk * kBlk + half * 64 * 128) + off;
+                            mma_f16(d, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&s_full[sb]);
+                    if (jj > 0) {
+                        // O_tile for the previous tile
+                        const int psb = prev_sb;
+                        if (!mbar_wait(&p_full[psb], ((nt - 1) >> 1) & 1, abort_flag, a.st) ||
+                            !mbar_wait(&pv_empty[psb], (((nt - 1) >> 1) & 1) ^ 1, abort_flag, a.st)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int half = 0; half < 2; half++) {
+                            const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
+#pragma unroll
+                            for (int kk = 0; kk < 8; kk++) {
+                                const uint64_t ad =
+                                    smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
+                                    ((uint32_t)((kk & 3) * 32) >> 4);
+                                const uint64_t bd =
+                                    smem_desc_mn_sw128(prev_k + half * kBlk + kk * 2048, kBlk);
+                                mma_f16(d, ad, bd, kIdescPV, kk > 0 ? 1u : 0u);
+                            }
+                        }
+                        mma_commit(&pv_full[psb]);
+                        mma_commit(&p_empty[psb]);
+                        if (prev_stage >= 0) mma_commit(&empty[prev_stage]);
+                    }
+                    prev_k = kb;
+                    prev_stage = my_stage;
+                    prev_sb = sb;
+                    nt++;
+                }
+                if (!ok) break;
+                {
+                    const int psb = prev_sb;
+                    if (!mbar_wait(&p_full[psb], ((nt - 1) >> 1) & 1, abort_flag, a.st) ||
+                        !mbar_wait(&pv_empty[psb], (((nt - 1) >> 1) & 1) ^ 1, abort_flag, a.st)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int half = 0; half < 2; half++) {
+                        const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
+#pragma unroll
+                        for (int kk = 0; kk < 8; kk++) {
+                            const uint64_t ad =
+                                smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
+                                ((uint32_t)((kk & 3) * 32) >> 4);
+                            const uint64_t bd =
+                                smem_desc_mn_sw128(prev_k + half * kBlk + kk * 2048, kBlk);
+                            mma_f16(d, ad, bd, kIdescPV, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(&pv_full[psb]);
+                    mma_commit(&p_empty[psb]);
+                    if (prev_stage >= 0) mma_commit(&empty[prev_stage]);
+                }
+                mma_commit(prep_empty);
+                nitem++;
+            }
+            mma_commit(drain);
+            mbar_drain(drain, 0, a.st);
+        }
+    } else if (warp >= 4) {
+        // ---------------- softmax / epilogue (warps 4..7) ----------------
+        const int quarter = warp & 3;
+        const int i = threadIdx.x - 128;        // 0..127
+        const int h = quarter * 16 + (lane & 15);
+        const int kh = lane >> 4;               // key half of S / channel half of O
+        int nt = 0, nitem = 0;
+        int kst = 0;   // ring position of the next entry tile (mirrors the producer)
+        bool ok = true;
+        for (int it = blockIdx.x; it < a.total_items; it += gridDim.x) {
+            AItem x;
+            if (!get_item(a, it, x, i == 0)) continue;
+            // ---- item prologue: q heads and (chunk 0) the window tile ----
+            // A failed wait in a warp only skips the rest of that item; here, once per item,
+            // all 128 threads meet and leave together if any of them failed.
+            const bool ready = ok && mbar_wait(prep_empty, (nitem & 1) ^ 1, abort_flag, a.st);
+            if (!named_barrier_and(1, 128, ready)) break;
+            if (i < 32) {
+                // angles in fp64, reduced, then sincosf (see rope_cos_sin)
+                float cs, sn;
+                rope_cos_sin((double)x.t, i, a.log2_theta, cs, sn);
+                rqc[i] = cs;
+                rqs[i] = sn;
+                rope_cos_sin((double)x.w0, i, a.log2_theta, cs, sn);
+                rwc[i] = cs;
+                rws[i] = sn;
+                rf[i] = (float)exp2(-(double)(2 * i) * (1.0 / 64.0) * a.log2_theta);
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            {
+                const int hq = i >> 1, hf = i & 1;
+                const uint16_t* src = a.q + ((int64_t)x.q * kH + hq) * kD + hf * 64;
+                float v[64];
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    const uint4 u = *reinterpret_cast<const uint4*>(src + 8 * c);
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int z = 0; z < 4; z++) {
+                        const float2 f = bf16x2_to_f32(w4[z]);
+                        v[8 * c + 2 * z] = f.x;
+                        v[8 * c + 2 * z + 1] = f.y;
+                    }
+                }
+                if (hf == 1) {
+#pragma unroll
+                    for (int pj = 0; pj < 32; pj++) {
+                        const float cs = rqc[pj], sn = rqs[pj];
+                        const float x0 = v[2 * pj], y0 = v[2 * pj + 1];
+                        v[2 * pj] = x0 * cs - y0 * sn;
+                        v[2 * pj + 1] = x0 * sn + y0 * cs;
+                    }
+                }
+                uint8_t* dst = sQ + hf * kQBlk;
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    uint4 u;
+                    u.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
+                    u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+                    u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+                    u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+                    *reinterpret_cast<uint4*>(dst + swz(hq, c)) = u;
+                }
+            }
+            if (x.tile0 == 0) {
+                // window row r = i: RMSNorm, RoPE at its position, bf16, swizzled store
+                const int r = i;
+                const int64_t p = (int64_t)x.w0 + r;
+                bool valid = r < x.n_win;
+                if (valid && p < a.kv_pos0[x.b]) {
+                    valid = false;
+                    flag(a.st, CSA_DEV_OOB);
+                }
+                float v[128];
+                if (valid) {
+                    const uint16_t* src = a.kv + (a.kv_off[x.b] + p - a.kv_pos0[x.b]) * kD;
+                    float ss = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; c++) {
+                        const uint4 u = *reinterpret_cast<const uint4*>(src + 8 * c);
+                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                        for (int z = 0; z < 4; z++) {
+                            const float2 f = bf16x2_to_f32(w4[z]);
+                            v[8 * c + 2 * z] = f.x;
+                            v[8 * c + 2 * z + 1] = f.y;
+                            ss += f.x * f.x + f.y * f.y;
+                        }
+                    }
+                    const float rn = rsqrtf(ss / (float)kD + a.eps);
+#pragma unroll
+                    for (int c = 0; c < 128; c++) v[c] *= rn;
+                    // angle (w0 + r) f_j = w0 f_j + r f_j: the first term from the fp64 table,
+                    // the second (< 128 rad) by sincosf; combined by the addition formula.
+                    // The per-row rotations go to a scratch row in the idle P buffers.
+                    float2* rot = reinterpret_cast<float2*>(sP) + r * 32;
+#pragma unroll 1
+                    for (int pj = 0; pj < 32; pj++) {
+                        float sb, cb;
+                        sincosf((float)r * rf[pj], &sb, &cb);
+                        rot[pj] = make_float2(rwc[pj] * cb - rws[pj] * sb, rws[pj] * cb + rwc[pj] * sb);
+                    }
+#pragma unroll
+                    for (int pj = 0; pj < 32; pj++) {
+                        const float2 cs = rot[pj];
+                        const float x0 = v[64 + 2 * pj], y0 = v[64 + 2 * pj + 1];
+                        v[64 + 2 * pj] = x0 * cs.x - y0 * cs.y;
+                        v[64 + 2 * pj + 1] = x0 * cs.y + y0 * cs.x;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 128; c++) v[c] = 0.f;
+                }
+#pragma unroll
+                for (int c = 0; c < 16; c++) {
+                    uint4 u;
+                    u.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
+                    u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+                    u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+                    u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+                    *reinterpret_cast<uint4*>(sW + (c >> 3) * kBlk + swz(r, c & 7)) = u;
+                }
+                const unsigned vm = __ballot_sync(0xffffffffu, valid);
+                if (lane == 0) smask[kStages * 4 + quarter] = vm;
+            }
+            fence_async_smem();
+            // all four warps' stores (including the window mask) before anyone reads them
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(prep_full);
+
+            // ---- running state of head h ----
+            const float sk = a.sink[h] * kLog2e;
+            float mrun = x.single ? sk : -INFINITY;
+            float lrun = (x.single && sk != -INFINITY) ? 1.f : 0.f;
+            float o[64];
+#pragma unroll
+            for (int c = 0; c < 64; c++) o[c] = 0.f;
+            float corr_prev = 1.f;
+            int prev_sb = 0;
+            for (int jj = 0; jj < x.ntiles && ok; jj++) {
+                const int j = x.tile0 + jj;
+                const int sb = nt & 1;
+                if (!mbar_wait_warp(&s_full[sb], (nt >> 1) & 1, abort_flag, a.st)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t sv[64];
+                tmem_ld64(tmem_S + sb * 64 + ((uint32_t)(quarter * 32) << 16), sv);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[sb]);
+                // validity of my 64 keys (the MMA has consumed the tile, so its mask is stable
+                // until the producer refills the stage after this tile's P.V)
+                const uint32_t* mk = smask + (j == 0 ? kStages : kst) * 4;
+                if (j != 0 && ++kst == kStages) kst = 0;
+                const uint32_t mw0 = mk[2 * kh], mw1 = mk[2 * kh + 1];
+                float tmax = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 64; c++) {
+                    const bool on = ((c < 32 ? mw0 >> c : mw1 >> (c - 32)) & 1u) != 0;
+                    const float xv = on ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
+                    sv[c] = __float_as_uint(xv);
+                    tmax = fmaxf(tmax, xv);
+                }
+                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+                const float mnew = fmaxf(mrun, tmax);
+                float corr = 1.f, rs = 0.f;
+                uint32_t pk[32];
+                if (mnew == -INFINITY) {
+#pragma unroll
+                    for (int c = 0; c < 32; c++) pk[c] = 0u;
+                } else {
+                    corr = exp2f(mrun - mnew);
+#pragma unroll
+                    for (int c = 0; c < 32; c++) {
+                        const float p0 = exp2f(__uint_as_float(sv[2 * c]) - mnew);
+                        const float p1 = exp2f(__uint_as_float(sv[2 * c + 1]) - mnew);
+                        rs += p0 + p1;
+                        pk[c] = pack_bf16x2(p0, p1);
+                    }
+                }
+                rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+                lrun = lrun * corr + rs;
+                mrun = mnew;
+                // P (bf16) into shared memory: head h, keys kh*64 .. kh*64+63
+                if (!mbar_wait_warp(&p_empty[sb], ((nt >> 1) & 1) ^ 1, abort_flag, a.st)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* prow = sP + sb * 2 * kPBlk + kh * kPBlk;
+#pragma unroll
+                for (int c = 0; c < 8; c++)
+                    *reinterpret_cast<uint4*>(prow + swz(h, c)) =
+                        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[sb]);
+                if (jj > 0) {
+                    if (!mbar_wait_warp(&pv_full[prev_sb], ((nt - 1) >> 1) & 1, abort_flag, a.st)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint32_t pv[64];
+                    tmem_ld64(tmem_PV + prev_sb * 64 + ((uint32_t)(quarter * 32) << 16), pv);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&pv_empty[prev_sb]);
+#pragma unroll
+                    for (int c = 0; c < 64; c++) o[c] = fmaf(o[c], corr_prev, __uint_as_float(pv[c]));
+                }
+                corr_prev = corr;
+                prev_sb = sb;
+                nt++;
+            }
+            if (ok) ok = mbar_wait_warp(&pv_full[prev_sb], ((nt - 1) >> 1) & 1, abort_flag, a.st);
+            if (ok) {
+                tc_fence_after();
+                uint32_t pv[64];
+                tmem_ld64(tmem_PV + prev_sb * 64 + ((uint32_t)(quarter * 32) << 16), pv);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pv_empty[prev_sb]);
+#pragma unroll
+                for (int c = 0; c < 64; c++) o[c] = fmaf(o[c], corr_prev, __uint_as_float(pv[c]));
+            }
+            if (!ok) {
+                // skip the rest of this item; the next item's barrier settles the exit
+            } else if (x.single) {
+                const float inv = lrun > 0.f ? 1.f / lrun : 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; c++) o[c] *= inv;
+                if (kh == 1) {
+#pragma unroll
+                    for (int pj = 0; pj < 32; pj++) {
+                        const float cs = rqc[pj], sn = -rqs[pj];   // rotation by -t
+                        const float x0 = o[2 * pj], y0 = o[2 * pj + 1];
+                        o[2 * pj] = x0 * cs - y0 * sn;
+                        o[2 * pj + 1] = x0 * sn + y0 * cs;
+                    }
+                }
+                uint16_t* dst = a.out + ((int64_t)x.q * kH + h) * kD + kh * 64;
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    uint4 u;
+                    u.x = pack_bf16x2(o[8 * c], o[8 * c + 1]);
+                    u.y = pack_bf16x2(o[8 * c + 2], o[8 * c + 3]);
+                    u.z = pack_bf16x2(o[8 * c + 4], o[8 * c + 5]);
+                    u.w = pack_bf16x2(o[8 * c + 6], o[8 * c + 7]);
+                    *reinterpret_cast<uint4*>(dst + 8 * c) = u;
+                }
+            } else {
+                float* pr = a.part + ((int64_t)it * kH + h) * (kD + 2);
+                if (kh == 0) {
+                    pr[0] = mrun;
+                    pr[1] = lrun;
+                }
+#pragma unroll
+                for (int c = 0; c < 64; c += 2)
+                    *reinterpret_cast<float2*>(pr + 2 + kh * 64 + c) = make_float2(o[c], o[c + 1]);
+            }
+            nitem++;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 256);
+    }
+}
+
+// Dense path: combine the chunk partials of one (query, head) in chunk order, add the
+// sink, normalise, inverse RoPE, store bf16.  Thread = channel.
+__global__ void __launch_bounds__(kD) attn_combine_kernel(const AttnTcArgs a) {
+    const int q = blockIdx.y, h = blockIdx.x, d = threadIdx.x;
+    const int b = a.q_seq[q], t = a.q_pos[q];
+    if (b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]) return;
+    int n = (t + 1) / a.m;
+    if (n > a.max_n) n = a.max_n;
+    const int64_t avail = a.ent_rows - a.ent_off[b];
+    if ((int64_t)n > avail) n = avail > 0 ? (int)avail : 0;
+    const int total = 1 + (n + kTK - 1) / kTK;
+    const int nch = (total + a.chunk_tiles - 1) / a.chunk_tiles;
+    const float sk = a.sink[h] * kLog2e;
+    const float* base = a.part + ((int64_t)q * a.chunks_per_q * kH + h) * (kD + 2);
+    const int64_t cstride = (int64_t)kH * (kD + 2);
+    float M = sk;
+    for (int c = 0; c < nch; c++) M = fmaxf(M, base[c * cstride]);
+    float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
+    float o = 0.f;
+    for (int c = 0; c < nch; c++) {
+        const float* pc = base + c * cstride;
+        const float mc = pc[0];
+        const float w = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        L = fmaf(w, pc[1], L);
+        o = fmaf(w, pc[2 + d], o);
+    }
+    o = L > 0.f ? o / L : 0.f;
+    const float other = __shfl_xor_sync(0xffffffffu, o, 1);
+    if (d >= kD - kRopeDims) {
+        float cs, sn;
+        rope_cos_sin(-(double)t, (d - (kD - kRopeDims)) >> 1, a.log2_theta, cs, sn);
+        o = (d & 1) ? (other * sn + o * cs) : (o * cs - other * sn);
+    }
+    a.out[((int64_t)q * kH + h) * kD + d] = (uint16_t)f32_to_bf16_bits(o);
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+    });
+    return fn;
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + kTileBytes + 2 * kQBlk + 4 * kPBlk +
+                              4 * (kStages + 1) * 4 + 5 * 32 * 4 + (2 * kStages + 15) * 8 + 16;
+
+int dense_chunks_per_q(int max_n) {
+    const int tiles = 1 + (max_n + kTK - 1) / kTK;
+    return (tiles + kDenseChunkTiles - 1) / kDenseChunkTiles;
+}
+
+}  // namespace
+
+bool attn_tc_supported(int H, int D, int fmt) { return H == kH && D == kD && fmt == CSA_KV_BF16; }
+
+size_t attn_tc_workspace_bytes(int Q, int max_n) {
+    return (size_t)Q * dense_chunks_per_q(max_n) * kH * (kD + 2) * sizeof(float);
+}
+
+cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace,
+                           cudaStream_t stream) {
+    if (Q == 0) return cudaSuccess;
+    AttnTcArgs a;
+    a.q = aa.q;
+    a.entries = aa.entries;
+    a.ent_off = aa.ent_off;
+    a.kv = aa.kv;
+    a.kv_off = aa.kv_off;
+    a.kv_pos0 = aa.kv_pos0;
+    a.q_seq = aa.q_seq;
+    a.q_pos = aa.q_pos;
+    a.seq_len = aa.seq_len;
+    a.idx = aa.idx;
+    a.sink = aa.sink;
+    a.out = aa.out;
+    a.part = reinterpret_cast<float*>(workspace);
+    a.st = aa.st;
+    a.ent_rows = aa.ent_rows;
+    a.k = aa.k;
+    a.m = aa.m;
+    a.B = aa.B;
+    a.W = aa.W;
+    a.Q = Q;
+    a.max_n = max_n;
+    a.scale_log2 = aa.scale * kLog2e;
+    a.eps = aa.eps;
+    a.log2_theta = aa.log2_theta;
+    if (aa.idx) {
+        a.chunk_tiles = 1 + (aa.k + kTK - 1) / kTK;
+        a.chunks_per_q = 1;
+    } else {
+        a.chunk_tiles = kDenseChunkTiles;
+        a.chunks_per_q = dense_chunks_per_q(max_n);
+    }
+    a.total_items = Q * a.chunks_per_q;
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof(map));
+    if (!aa.idx && aa.ent_rows > 0) {
+        EncodeFn enc = encode_fn();
+        if (!enc) return cudaErrorInvalidValue;
+        const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)aa.ent_rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+        const cuuint32_t box[2] = {64, (cuuint32_t)kTK};
+        const cuuint32_t estr[2] = {1, 1};
+        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint8_t*>(aa.entries), dims,
+                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = min(a.total_items, sm_count());
+    {
+        LaunchScope scope(kKAttnTc, stream);
+        attn_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map, a);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess || aa.idx) return e;
+    LaunchScope scope(kKAttnCombine, stream);
+    attn_combine_kernel<<<dim3(kH, Q), kD, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const bool live = e < x.n_vis;
                 const float kscale = live ? __ldg(a.ks + x.row0 + e) : 0.f;
                 const int ab = nacc & 1;
-                if (!mbar_wait(&accfull[ab], (nacc >> 1) & 1, abort_flag, a.st)) {
+                if (!mbar_wait_warp(&accfull[ab], (nacc >> 1) & 1, abort_flag, a.st)) {
                     ok = false;
                     break;
                 }

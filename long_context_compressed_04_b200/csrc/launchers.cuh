@@ -6,7 +6,16 @@
 namespace csa {
 
 // Kernel kinds for launch accounting (names in prof.cu).
-enum KernelKind { kKCompress = 0, kKIndexerSimt, kKTopk, kKAttnSimt, kKIndexerTc, kKernelKinds };
+enum KernelKind {
+    kKCompress = 0,
+    kKIndexerSimt,
+    kKTopk,
+    kKAttnSimt,
+    kKIndexerTc,
+    kKAttnTc,
+    kKAttnCombine,
+    kKernelKinds
+};
 
 // Counts one kernel launch; with timing enabled, brackets it with CUDA events on `stream`.
 class LaunchScope {
@@ -33,6 +42,7 @@ struct AttnArgs {
     const int32_t* q_pos;
     const int64_t* seq_len;
     const int32_t* idx;  // nullptr = dense over all visible entries
+    int64_t ent_rows;
     const float* sink;
     uint16_t* out;
     int32_t* st;
@@ -64,6 +74,10 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream);
 cudaError_t launch_attn_simt(const AttnArgs& a, int Q, int D, cudaStream_t stream);
+bool attn_tc_supported(int H, int D, int fmt);
+size_t attn_tc_workspace_bytes(int Q, int max_n);
+cudaError_t launch_attn_tc(const AttnArgs& a, int Q, int max_n, void* workspace,
+                           cudaStream_t stream);
 
 // Sets the thread-local message csa_last_error() returns (printf-style).
 void set_error_message(const char* fmt, ...);

@@ -80,6 +80,28 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int32
     return true;
 }
 
+// Bounded wait whose result is the same for every lane of the calling warp (all lanes
+// must call it): a warp never splits between a collective and an abort path.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag, int32_t* dev_status) {
+    const bool ok = mbar_wait(bar, parity, abort_flag, dev_status);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// AND of `v` over the `nthreads` threads meeting at named barrier `id` (all must arrive).
+__device__ __forceinline__ bool named_barrier_and(int id, int nthreads, bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.and.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -6,14 +6,24 @@
 // not depend on how the work is partitioned -- the result is batch-invariant by
 // construction.
 //
-// One CTA (1024 threads) per query: a 4-pass radix select (8 bits per pass) over
-// order-preserving 32-bit keys finds the k-th largest key T and how many of the keys equal
-// to T are needed; a final pass in ascending entry order takes every key > T and the first
-// needed keys == T, writing them with a block-wide prefix sum -- which emits the indices
-// already in ascending order.
+// One CTA (1024 threads) per query.  Scores map to order-preserving 32-bit keys.  Three
+// radix passes (11, 11 and 10 bits) find the k-th largest key T and how many keys equal
+// to T are needed: each pass histograms the keys that match the prefix found so far with
+// warp-aggregated shared-memory atomics (lanes hitting the same bin add once), then a
+// block-wide scan over the 2048 bins, from the top, picks the bin holding the k-th key.
+// A last pass in ascending entry order takes every key > T and the first needed keys
+// == T; one block-wide scan per 4096-entry chunk gives each thread its output slots, so
+// the indices come out already sorted.  Score rows are read with 16-byte loads.
 #include "launchers.cuh"
 
 namespace csa {
+
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+constexpr int kBins = 2048;
+constexpr int kChunk = 4 * kThreads;
 
 __device__ __forceinline__ uint32_t score_key(float s) {
     uint32_t u = __float_as_uint(s);
@@ -21,24 +31,24 @@ __device__ __forceinline__ uint32_t score_key(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix sum over the CTA; `total` receives the CTA sum.  tmp holds >= 33 ints.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int& total) {
+// Exclusive prefix sum over the CTA of `v`; `total` gets the CTA sum.  tmp: >= 33 ints.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* tmp,
+                                                         uint32_t& total) {
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int nw = blockDim.x >> 5;
-    int x = v;
+    uint32_t x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
     if (lane == 31) tmp[wid] = x;
     __syncthreads();
     if (wid == 0) {
-        const int wv = lane < nw ? tmp[lane] : 0;
-        int inc = wv;
+        const uint32_t wv = lane < kWarps ? tmp[lane] : 0u;
+        uint32_t inc = wv;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
             if (lane >= o) inc += y;
         }
         __syncwarp();
@@ -46,22 +56,35 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* tmp, int& total)
         if (lane == 31) tmp[32] = inc;
     }
     __syncthreads();
-    const int res = x - v + tmp[wid];
+    const uint32_t res = x - v + tmp[wid];
     total = tmp[32];
     __syncthreads();
     return res;
 }
 
-__global__ void __launch_bounds__(1024) topk_radix_kernel(
+// Keys of entries i .. i+3 (0 past n).  `vec`: the row is 16-byte aligned.
+__device__ __forceinline__ void load4(const float* s, int i, int n, bool vec, uint32_t* key) {
+    if (vec && i + 3 < n) {
+        const float4 v = *reinterpret_cast<const float4*>(s + i);
+        key[0] = score_key(v.x);
+        key[1] = score_key(v.y);
+        key[2] = score_key(v.z);
+        key[3] = score_key(v.w);
+    } else {
+#pragma unroll
+        for (int u = 0; u < 4; u++) key[u] = (i + u < n) ? score_key(s[i + u]) : 0u;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_seq,
     const int32_t* __restrict__ q_pos, const int64_t* __restrict__ seq_len, int B, int m,
     int max_n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ dev_status) {
-    __shared__ uint32_t hist[256];
-    __shared__ int scan_tmp[2][33];
-    __shared__ uint32_t sh_prefix;
-    __shared__ int sh_krem;
+    __shared__ uint32_t hist[kBins];
+    __shared__ uint32_t scan_tmp[33];
+    __shared__ uint32_t sh_bin, sh_krem;
     const int qq = blockIdx.x;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int b = q_seq[qq];
     const int t = q_pos[qq];
     // invalid queries (flagged by the scoring kernel) select nothing
@@ -71,62 +94,95 @@ __global__ void __launch_bounds__(1024) topk_radix_kernel(
     const float* s = scores + (int64_t)qq * ld;
     int32_t* out = idx_out + (int64_t)qq * k;
     if (n <= k) {
-        for (int j = tid; j < k; j += blockDim.x) out[j] = j < n ? j : -1;
+        for (int j = tid; j < k; j += kThreads) out[j] = j < n ? j : -1;
         return;
     }
-    uint32_t prefix = 0u, mask = 0u;
-    int krem = k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int x = tid; x < 256; x += blockDim.x) hist[x] = 0u;
+    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
+
+    uint32_t prefix = 0u, mask = 0u, krem = (uint32_t)k;
+    for (int pass = 0; pass < 3; pass++) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const uint32_t bmask = pass == 2 ? 1023u : 2047u;
+        for (int x = tid; x < kBins; x += kThreads) hist[x] = 0u;
         __syncthreads();
-        for (int i = tid; i < n; i += blockDim.x) {
-            const uint32_t key = score_key(s[i]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
-        }
-        __syncthreads();
-        if (tid == 0) {
-            int cum = 0;
-            for (int bin = 255; bin >= 0; bin--) {
-                const int h = (int)hist[bin];
-                if (cum + h >= krem) {
-                    sh_prefix = prefix | ((uint32_t)bin << shift);
-                    sh_krem = krem - cum;
-                    break;
-                }
-                cum += h;
+        for (int c0 = 0; c0 < n; c0 += kChunk) {   // uniform trip count: whole warps
+            const int i0 = c0 + 4 * tid;
+            uint32_t key[4];
+            load4(s, i0, n, vec, key);
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const bool hit = (i0 + u < n) && ((key[u] & mask) == prefix);
+                const uint32_t bin = hit ? ((key[u] >> shift) & bmask) : 0xFFFFFFFFu;
+                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+                if (hit && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
             }
         }
         __syncthreads();
-        prefix = sh_prefix;
+        // bins from the top: thread t owns bins 2047 - 2t and 2046 - 2t
+        const int bhi = kBins - 1 - 2 * tid, blo = bhi - 1;
+        const uint32_t chi = hist[bhi], clo = hist[blo];
+        uint32_t tot;
+        const uint32_t above = block_exclusive_scan(chi + clo, scan_tmp, tot);
+        if (above < krem && krem <= above + chi) {
+            sh_bin = (uint32_t)bhi;
+            sh_krem = krem - above;
+        } else if (above + chi < krem && krem <= above + chi + clo) {
+            sh_bin = (uint32_t)blo;
+            sh_krem = krem - above - chi;
+        }
+        __syncthreads();
+        prefix |= sh_bin << shift;
+        mask |= bmask << shift;
         krem = sh_krem;
-        mask |= 255u << shift;
         __syncthreads();
     }
-    const uint32_t T = prefix;  // the k-th largest key; krem keys equal to T are needed
-    int written = 0, ties_seen = 0;
-    for (int i0 = 0; i0 < n; i0 += blockDim.x) {
-        const int i = i0 + tid;
-        const uint32_t key = i < n ? score_key(s[i]) : 0u;
-        const int gt = (i < n) && key > T;
-        const int eq = (i < n) && key == T;
-        int eq_total, sel_total;
-        const int eq_rank = block_exclusive_scan(eq, scan_tmp[0], eq_total);
-        const int sel = gt || (eq && ties_seen + eq_rank < krem);
-        const int pos = block_exclusive_scan(sel, scan_tmp[1], sel_total);
-        if (sel && written + pos < k) out[written + pos] = i;
-        written += sel_total;
-        ties_seen += eq_total;
+    const uint32_t T = prefix;   // the k-th largest key; krem keys equal to T are taken
+    // ordered collection: 4096 entries per round, 4 consecutive per thread
+    uint32_t written = 0, ties_before = 0;
+    for (int c0 = 0; c0 < n; c0 += kChunk) {
+        const int i0 = c0 + 4 * tid;
+        uint32_t key[4];
+        load4(s, i0, n, vec, key);
+        uint32_t ngt = 0, neq = 0;
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const bool in = i0 + u < n;
+            ngt += (in && key[u] > T) ? 1u : 0u;
+            neq += (in && key[u] == T) ? 1u : 0u;
+        }
+        uint32_t tot;
+        const uint32_t packed = block_exclusive_scan(ngt | (neq << 16), scan_tmp, tot);
+        uint32_t eq_rank = ties_before + (packed >> 16);   // tie rank of my first tie
+        uint32_t pos = written + (packed & 0xFFFFu) + (min(eq_rank, krem) - min(ties_before, krem));
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const bool in = i0 + u < n;
+            bool take = in && key[u] > T;
+            if (in && key[u] == T) {
+                take = eq_rank < krem;
+                eq_rank++;
+            }
+            if (take) {
+                if (pos < (uint32_t)k) out[pos] = i0 + u;
+                pos++;
+            }
+        }
+        const uint32_t ties_after = ties_before + (tot >> 16);
+        written += (tot & 0xFFFFu) + (min(ties_after, krem) - min(ties_before, krem));
+        ties_before = ties_after;
     }
-    if (tid == 0 && written != k) flag(dev_status, CSA_DEV_NAN);  // only NaN keys can do this
+    if (tid == 0 && written != (uint32_t)k) flag(dev_status, CSA_DEV_NAN);
 }
+
+}  // namespace
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream) {
     if (Q == 0) return cudaSuccess;
     LaunchScope scope(kKTopk, stream);
-    topk_radix_kernel<<<Q, 1024, 0, stream>>>(scores, ld, q_seq, q_pos, seq_len, B, m, max_n, k,
-                                              idx_out, st);
+    topk_radix_kernel<<<Q, kThreads, 0, stream>>>(scores, ld, q_seq, q_pos, seq_len, B, m, max_n,
+                                                  k, idx_out, st);
     return cudaGetLastError();
 }
 

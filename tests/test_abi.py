@@ -65,15 +65,15 @@ def test_null_and_unsupported_arguments_fail_on_host():
                           10000.0, 1e-6, fake, None, None)
     assert st == 1 and b"aligned" in lib.csa_last_error()
     # fp8 format needs D = 576
-    st = lib.sparse_mqa_attn(fake, fake, 1, fake, fake, fake, fake, fake, fake, fake, fake, 8, 4, fake,
+    st = lib.sparse_mqa_attn(fake, fake, 1, 10, fake, fake, fake, fake, fake, fake, fake, fake, 8, 4, fake,
                              1, 1, 16, 128, 128, 0.08, 10000.0, 1e-6, fake, None, None)
     assert st == 2
     # window above 128
-    st = lib.sparse_mqa_attn(fake, fake, 0, fake, fake, fake, fake, fake, fake, fake, fake, 8, 4, fake,
+    st = lib.sparse_mqa_attn(fake, fake, 0, 10, fake, fake, fake, fake, fake, fake, fake, fake, 8, 4, fake,
                              1, 1, 16, 128, 129, 0.08, 10000.0, 1e-6, fake, None, None)
     assert st == 1 and b"window" in lib.csa_last_error()
     # unsupported heads
-    st = lib.dense_hca_attn(fake, fake, 0, fake, fake, fake, fake, fake, fake, fake, 128, fake, 1, 1, 48,
+    st = lib.dense_hca_attn(fake, fake, 0, 10, fake, fake, fake, fake, fake, fake, fake, 128, fake, 1, 1, 48,
                             128, 128, 0.08, 10000.0, 1e-6, 10, fake, fake, 1 << 20, None, None)
     assert st == 2
 

@@ -51,7 +51,7 @@ def test_sparse_attention(H, D, fmt, k, T):
     _orc.assert_out_close(buf.out, ref)
 
 
-@pytest.mark.parametrize("T", [[128 * 40 + 77, 128 * 7], [300]])
+@pytest.mark.parametrize("T", [[128 * 40 + 77, 128 * 7], [300], [128 * 2500 + 77, 130]])
 def test_dense_hca_attention(T):
     wl = synth.make_workload("t", B=len(T), T=T, D=128, H=64, m=128, span=128, seed=32,
                              device=DEV)
@@ -62,9 +62,10 @@ def test_dense_hca_attention(T):
     _orc.assert_out_close(buf.out, _orc.attention(wl.to("cpu"), rows, None))
 
 
-def test_short_window_and_no_window():
-    for W, T in [(128, [37]), (0, [400]), (5, [400])]:
-        wl = synth.make_workload("t", B=len(T), T=T, D=128, H=16, m=4, span=8, W=W, H_I=4,
+@pytest.mark.parametrize("H", [16, 64])
+def test_short_window_and_no_window(H):
+    for W, T in [(128, [37]), (0, [400]), (5, [400]), (128, [3])]:
+        wl = synth.make_workload("t", B=len(T), T=T, D=128, H=H, m=4, span=8, W=W, H_I=4,
                                  d_I=64, k=32, seed=33, device=DEV)
         buf, rows = _with_oracle_entries(wl)
         idx = _random_idx(wl, 2)
@@ -74,8 +75,9 @@ def test_short_window_and_no_window():
         _orc.assert_out_close(buf.out, _orc.attention(wl.to("cpu"), rows, idx))
 
 
-def test_sink_limits():
-    wl = synth.make_workload("t", B=1, T=[2000], D=128, H=16, m=4, span=8, H_I=4, d_I=64, k=64,
+@pytest.mark.parametrize("H", [16, 64])
+def test_sink_limits(H):
+    wl = synth.make_workload("t", B=1, T=[2000], D=128, H=H, m=4, span=8, H_I=4, d_I=64, k=64,
                              seed=34, device=DEV)
     buf, rows = _with_oracle_entries(wl)
     idx = _random_idx(wl, 3)
@@ -88,8 +90,9 @@ def test_sink_limits():
     assert buf.out.abs().max().item() < 1e-20   # sink = 60 >> logits: output ~ e^-50
 
 
-def test_out_of_range_index_is_flagged_and_skipped():
-    wl = synth.make_workload("t", B=1, T=[2000], D=128, H=16, m=4, span=8, H_I=4, d_I=64, k=64,
+@pytest.mark.parametrize("H", [16, 64])
+def test_out_of_range_index_is_flagged_and_skipped(H):
+    wl = synth.make_workload("t", B=1, T=[2000], D=128, H=H, m=4, span=8, H_I=4, d_I=64, k=64,
                              seed=35, device=DEV)
     buf, rows = _with_oracle_entries(wl)
     idx = _random_idx(wl, 4, pad=1)
