@@ -240,7 +240,10 @@ csa_status_t lightning_indexer_topk_noalloc(const uint8_t* qI, const float* qI_s
  *     recorded on its own stream (adds two event records per launch); 0 turns it off.
  *   csa_profile_collect: waits for the recorded events, writes one record per kernel
  *     kind timed since the last collect (launch count and total device milliseconds) to
- *     out[0 .. max_entries), returns how many it wrote, and resets the totals.
+ *     out[0 .. max_entries), returns how many it wrote, and resets the totals.  With
+ *     keep_pending != 0 the event pairs stay registered: launches captured into a CUDA
+ *     graph record the same events on every replay, so a collect after each replay reads
+ *     that replay's kernel times.
  * Thread-safe.  Uses the CUDA device that was current at each launch.
  */
 typedef struct {
@@ -250,7 +253,7 @@ typedef struct {
 } csa_kernel_time_t;
 long long csa_launch_count(void);
 void csa_profile_enable(int on);
-int csa_profile_collect(csa_kernel_time_t* out, int max_entries);
+int csa_profile_collect(csa_kernel_time_t* out, int max_entries, int keep_pending);
 
 #ifdef __cplusplus
 }

@@ -65,7 +65,7 @@ _SIGS = {
                                                       _I64, _P, _P]),
     "csa_launch_count": (ctypes.c_longlong, []),
     "csa_profile_enable": (None, [ctypes.c_int]),
-    "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int]),
+    "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -105,10 +105,11 @@ def csa_profile_enable(on: bool = True):
     _lib.csa_profile_enable(1 if on else 0)
 
 
-def csa_profile_collect() -> dict:
-    """{kernel name: (timed launches, total device ms)} since the last collect."""
+def csa_profile_collect(keep_pending: bool = False) -> dict:
+    """{kernel name: (timed launches, total device ms)} since the last collect.  With
+    keep_pending, the recorded event pairs stay registered (for CUDA-graph replays)."""
     arr = (_KernelTime * 32)()
-    n = _lib.csa_profile_collect(ctypes.cast(arr, ctypes.c_void_p), 32)
+    n = _lib.csa_profile_collect(ctypes.cast(arr, ctypes.c_void_p), 32, 1 if keep_pending else 0)
     return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}
 
 

@@ -114,6 +114,8 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
     float* corr_s = l_s + kHG;              // [kHG]
     int* kval = reinterpret_cast<int*>(corr_s + kHG);  // [kTK]
 
+    pdl_wait();
+    pdl_trigger();
     const int qq = blockIdx.y;
     const int h0 = blockIdx.x * kHG;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -242,11 +244,11 @@ cudaError_t launch_attn_simt(const AttnArgs& a, int Q, int D, cudaStream_t strea
     if (D == 128) {
         const size_t sm = attn_smem_bytes<128>();
         cudaFuncSetAttribute(attn_simt_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        attn_simt_kernel<128><<<grid, 256, sm, stream>>>(a);
+        return launch_pdl(attn_simt_kernel<128>, grid, dim3(256), sm, stream, a);
     } else {
         const size_t sm = attn_smem_bytes<576>();
         cudaFuncSetAttribute(attn_simt_kernel<576>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-        attn_simt_kernel<576><<<grid, 256, sm, stream>>>(a);
+        return launch_pdl(attn_simt_kernel<576>, grid, dim3(256), sm, stream, a);
     }
     return cudaGetLastError();
 }

@@ -46,6 +46,7 @@ constexpr int kQBlk = kH * 128;              // one 64-channel slice of Q (8 KB)
 constexpr int kPBlk = kH * 128;              // one 64-key slice of P (8 KB)
 constexpr int kThreads = 256;
 constexpr int kDenseChunkTiles = 8;
+constexpr int kMaxK = 2048;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnTcArgs {
@@ -170,7 +171,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* rqs = rqc + 32;
     float* rwc = rqs + 32;
     float* rws = rwc + 32;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(rws + 32);
+    int32_t* sidx = reinterpret_cast<int32_t*>(rws + 32);   // [kMaxK] the item's index row
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sidx + kMaxK);
     uint64_t* full = bars;                 // [kStages]  33 arrivals (+tx)
     uint64_t* empty = full + kStages;      // [kStages]  MMA commit
     uint64_t* prep_full = empty + kStages; // Q + window ready: 4 arrivals
@@ -219,6 +221,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ---------------- producer ----------------
+        // index sets (top-k) and entries (compression) come from earlier kernels; the
+        // prologue of the other roles (q heads, window rows) only reads inputs
+        pdl_wait();
+        if (lane == 0) pdl_trigger();
         int stage = 0;
         uint32_t ph = 0;
         int issued[kStages] = {};
@@ -226,6 +232,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
             AItem x;
             if (!get_item(a, it, x, false)) continue;
+            if (a.idx) {
+                // the query's whole index row, once per item (one load round trip, not one
+                // per tile); only this warp reads it
+                const int32_t* src = a.idx + (int64_t)x.q * a.k;
+                for (int v = lane; v < a.k; v += 32) sidx[v] = src[v];
+                __syncwarp();
+            }
             for (int jj = 0; jj < x.ntiles; jj++) {
                 const int j = x.tile0 + jj;
                 if (j == 0) continue;  // the window tile is built by the softmax warps
@@ -257,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         bool valid = false;
                         const uint8_t* src = a.entries;
                         if (v < x.n_ent) {
-                            const int e = a.idx[(int64_t)x.q * a.k + v];
+                            const int e = sidx[v];
                             if (e >= 0) {
                                 if (e < x.n_vis && x.row0 + e < a.ent_rows) {
                                     valid = true;
@@ -687,6 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // sink, normalise, inverse RoPE, store bf16.  Thread = channel.
 __global__ void __launch_bounds__(kD) attn_combine_kernel(const AttnTcArgs a) {
     const int q = blockIdx.y, h = blockIdx.x, d = threadIdx.x;
+    pdl_wait();   // chunk partials come from the attention kernel
+    pdl_trigger();
     const int b = a.q_seq[q], t = a.q_pos[q];
     if (b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]) return;
     int n = (t + 1) / a.m;
@@ -750,7 +765,8 @@ int sm_count() {
 }
 
 constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + kTileBytes + 2 * kQBlk + 4 * kPBlk +
-                              4 * (kStages + 1) * 4 + 5 * 32 * 4 + (2 * kStages + 15) * 8 + 16;
+                              4 * (kStages + 1) * 4 + 5 * 32 * 4 + kMaxK * 4 +
+                              (2 * kStages + 15) * 8 + 16;
 
 int dense_chunks_per_q(int max_n) {
     const int tiles = 1 + (max_n + kTK - 1) / kTK;
@@ -822,13 +838,11 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
     const int grid = min(a.total_items, sm_count());
     {
         LaunchScope scope(kKAttnTc, stream);
-        attn_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(map, a);
+        e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, map, a);
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess || aa.idx) return e;
     LaunchScope scope(kKAttnCombine, stream);
-    attn_combine_kernel<<<dim3(kH, Q), kD, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(attn_combine_kernel, dim3(kH, Q), dim3(kD), 0, stream, a);
 }
 
 }  // namespace csa

@@ -57,6 +57,18 @@ __device__ __forceinline__ void rope_cos_sin(double pos, int j, double log2_thet
     sincosf((float)r, &s, &c);
 }
 
+// Programmatic dependent launch.  Every libcsa kernel is launched so that it may start
+// while the previous kernel on the stream finishes.  pdl_wait() blocks the calling thread
+// until the previous grid has completed and its writes are visible; it must precede any
+// read of data an earlier kernel produces and any write that an earlier kernel may still
+// read.  pdl_trigger() lets the next kernel start launching; kernels issue it only after
+// their own wait, so at most two kernels ever overlap.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -15,8 +15,34 @@
 
 namespace csa {
 
+// Tokens of one entry are split over TG token groups (along the token axis) that walk
+// chunks of 8 tokens; a thread loads a chunk's 8 tokens x 4 channels at once (and the next
+// chunk's before reducing the current one), keeps an online softmax state per channel, and
+// the token groups merge their states in a fixed order through shared memory.
+constexpr int kChunkTok = 8;
+constexpr int kMaxMergeSlots = 480;   // (TG - 1) * channel lanes
+
+struct Chunk {
+    uint2 z[kChunkTok], v[kChunkTok];
+};
+
+__device__ __forceinline__ void load_chunk(const uint16_t* __restrict__ kv,
+                                           const uint16_t* __restrict__ gate, int64_t row_first,
+                                           int64_t first_pos, int D, int c0, Chunk& ch) {
+    // row_first holds position max(first_pos, 0); positions before the sequence start
+    // (entry 0 of CSA) re-read that row and are masked out of the softmax by the caller
+    const int64_t p_first = first_pos > 0 ? first_pos : 0;
+#pragma unroll
+    for (int jj = 0; jj < kChunkTok; jj++) {
+        const int64_t p = first_pos + jj;
+        const int64_t row = row_first + (p >= 0 ? p - p_first : 0);
+        ch.z[jj] = *reinterpret_cast<const uint2*>(gate + row * D + c0);
+        ch.v[jj] = *reinterpret_cast<const uint2*>(kv + row * D + c0);
+    }
+}
+
 template <int SPAN>
-__global__ void __launch_bounds__(160) compress_kernel(
+__global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
     const uint16_t* __restrict__ kv, const uint16_t* __restrict__ gate,
     const float* __restrict__ bias, const int64_t* __restrict__ seq_len,
     const int64_t* __restrict__ kv_off,
@@ -25,6 +51,10 @@ __global__ void __launch_bounds__(160) compress_kernel(
     int D, int fmt, double log2_theta, float eps, uint8_t* __restrict__ entries,
     int32_t* __restrict__ dev_status) {
     __shared__ float red[8];
+    __shared__ float4 st_m[SPAN == 8 ? 1 : kMaxMergeSlots], st_d[SPAN == 8 ? 1 : kMaxMergeSlots],
+        st_a[SPAN == 8 ? 1 : kMaxMergeSlots];
+    pdl_wait();   // entries may still be read by the previous step's attention
+    pdl_trigger();
     const int64_t it = blockIdx.x;
     const int b = item_seq[it];
     const int64_t i = item_ent[it];
@@ -40,55 +70,113 @@ __global__ void __launch_bounds__(160) compress_kernel(
         if (threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
         return;
     }
+    const int cw = 32 * ((D / 4 + 31) / 32);     // channel lanes per token group
+    const int TG = blockDim.x / cw;               // token groups
+    const int nch = SPAN / kChunkTok / TG;        // chunks per token group
     const int tid = threadIdx.x;
-    const int c0 = tid * 4;
+    const int cl = tid % cw, tg = tid / cw;
+    const int c0 = cl * 4;
     const bool active = c0 < D;
 
-    float e[4] = {0.f, 0.f, 0.f, 0.f};
-    if (active) {
-        float mx[4], den[4], acc[4];
+    float mx[4], den[4], acc[4];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            mx[u] = -INFINITY;
-            den[u] = 0.f;
-            acc[u] = 0.f;
-        }
-        const int j0 = first < 0 ? (int)(-first) : 0;
-#pragma unroll 4
-        for (int j = j0; j < SPAN; j++) {
-            const int64_t row = row0 + (first + j) - pos0;
-            const uint2 zz = *reinterpret_cast<const uint2*>(gate + row * D + c0);
-            const uint2 vv = *reinterpret_cast<const uint2*>(kv + row * D + c0);
-            const float4 bb = *reinterpret_cast<const float4*>(bias + (int64_t)j * D + c0);
-            const float2 z01 = bf16x2_to_f32(zz.x), z23 = bf16x2_to_f32(zz.y);
-            const float2 v01 = bf16x2_to_f32(vv.x), v23 = bf16x2_to_f32(vv.y);
-            const float l[4] = {z01.x + bb.x, z01.y + bb.y, z23.x + bb.z, z23.y + bb.w};
-            const float v[4] = {v01.x, v01.y, v23.x, v23.y};
+    for (int u = 0; u < 4; u++) {
+        mx[u] = -INFINITY;
+        den[u] = 0.f;
+        acc[u] = 0.f;
+    }
+    if (active) {
+        const int j_begin = tg * nch * kChunkTok;
+        Chunk cur, nxt;
+        // row of the first token of a chunk starting at pooled index j (clamped at entry 0)
+        auto chunk_row = [&](int j) { return row0 + (first + j >= 0 ? first + j : 0) - pos0; };
+        load_chunk(kv, gate, chunk_row(j_begin), first + j_begin, D, c0, cur);
+        for (int c = 0; c < nch; c++) {
+            const int j0 = j_begin + c * kChunkTok;
+            if (c + 1 < nch) load_chunk(kv, gate, chunk_row(j0 + kChunkTok), first + j0 + kChunkTok, D, c0, nxt);
+            float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int jj = 0; jj < kChunkTok; jj++) {
+                if (first + j0 + jj < 0) continue;
+                const float4 bb = *reinterpret_cast<const float4*>(bias + (int64_t)(j0 + jj) * D + c0);
+                const float2 z01 = bf16x2_to_f32(cur.z[jj].x), z23 = bf16x2_to_f32(cur.z[jj].y);
+                cm[0] = fmaxf(cm[0], z01.x + bb.x);
+                cm[1] = fmaxf(cm[1], z01.y + bb.y);
+                cm[2] = fmaxf(cm[2], z23.x + bb.z);
+                cm[3] = fmaxf(cm[3], z23.y + bb.w);
+            }
 #pragma unroll
             for (int u = 0; u < 4; u++) {
-                if (l[u] > mx[u]) {
-                    const float sc = expf(mx[u] - l[u]);
-                    den[u] = den[u] * sc + 1.f;
-                    acc[u] = acc[u] * sc + v[u];
-                    mx[u] = l[u];
-                } else {
+                const float M = fmaxf(mx[u], cm[u]);
+                if (M != -INFINITY && mx[u] != -INFINITY) {
+                    const float sc = expf(mx[u] - M);
+                    den[u] *= sc;
+                    acc[u] *= sc;
+                }
+                mx[u] = M;
+            }
+#pragma unroll
+            for (int jj = 0; jj < kChunkTok; jj++) {
+                if (first + j0 + jj < 0) continue;
+                const float4 bb = *reinterpret_cast<const float4*>(bias + (int64_t)(j0 + jj) * D + c0);
+                const float2 z01 = bf16x2_to_f32(cur.z[jj].x), z23 = bf16x2_to_f32(cur.z[jj].y);
+                const float2 v01 = bf16x2_to_f32(cur.v[jj].x), v23 = bf16x2_to_f32(cur.v[jj].y);
+                const float l[4] = {z01.x + bb.x, z01.y + bb.y, z23.x + bb.z, z23.y + bb.w};
+                const float v[4] = {v01.x, v01.y, v23.x, v23.y};
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
                     const float p = expf(l[u] - mx[u]);
                     den[u] += p;
                     acc[u] = fmaf(p, v[u], acc[u]);
                 }
             }
+            if (c + 1 < nch) cur = nxt;
         }
+    }
+    if (TG > 1) {
+        if (tg > 0) {
+            const int slot = (tg - 1) * cw + cl;
+            st_m[slot] = make_float4(mx[0], mx[1], mx[2], mx[3]);
+            st_d[slot] = make_float4(den[0], den[1], den[2], den[3]);
+            st_a[slot] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        }
+        __syncthreads();
+        if (tg > 0) return;
+        // merge the token groups' states in order 0, 1, .., TG-1
+        for (int g = 1; g < TG; g++) {
+            const float4 gm = st_m[(g - 1) * cw + cl], gd = st_d[(g - 1) * cw + cl],
+                         ga = st_a[(g - 1) * cw + cl];
+            const float om[4] = {gm.x, gm.y, gm.z, gm.w}, od[4] = {gd.x, gd.y, gd.z, gd.w},
+                        oa[4] = {ga.x, ga.y, ga.z, ga.w};
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const float M = fmaxf(mx[u], om[u]);
+                if (M == -INFINITY) continue;
+                const float s0 = mx[u] == -INFINITY ? 0.f : expf(mx[u] - M);
+                const float s1 = om[u] == -INFINITY ? 0.f : expf(om[u] - M);
+                den[u] = den[u] * s0 + od[u] * s1;
+                acc[u] = acc[u] * s0 + oa[u] * s1;
+                mx[u] = M;
+            }
+        }
+    }
+    float e[4] = {0.f, 0.f, 0.f, 0.f};
+    if (active) {
 #pragma unroll
         for (int u = 0; u < 4; u++) e[u] = acc[u] / den[u];
     }
 
-    // RMSNorm over all D channels (unit weight).
+    // RMSNorm over all D channels (unit weight); threads of token group 0 only from here.
     float ss = e[0] * e[0] + e[1] * e[1] + e[2] * e[2] + e[3] * e[3];
     ss = warp_sum(ss);
     if ((tid & 31) == 0) red[tid >> 5] = ss;
-    __syncthreads();
+    if (blockDim.x > cw) {
+        asm volatile("bar.sync 1, %0;" ::"r"(cw) : "memory");
+    } else {
+        __syncthreads();
+    }
     float tot = 0.f;
-    for (int w = 0; w < (int)(blockDim.x >> 5); w++) tot += red[w];
+    for (int w = 0; w < cw / 32; w++) tot += red[w];
     const float r = rsqrtf(tot / (float)D + eps);
 #pragma unroll
     for (int u = 0; u < 4; u++) e[u] *= r;
@@ -141,18 +229,20 @@ cudaError_t launch_compress(int span, const void* kv, const void* gate, const fl
                             int fmt, float theta, float eps, void* entries, int32_t* st,
                             cudaStream_t stream) {
     if (n_items == 0) return cudaSuccess;
-    const int threads = 32 * ((D / 4 + 31) / 32);
+    const int cw = 32 * ((D / 4 + 31) / 32);        // channel lanes: 32 (D=128) or 160 (576)
     const double log2_theta = log2((double)theta);
     const dim3 grid((unsigned)n_items);
     LaunchScope scope(kKCompress, stream);
     if (span == 8) {
-        compress_kernel<8><<<grid, threads, 0, stream>>>(
-            (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
-            item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
+        return launch_pdl(compress_kernel<8>, grid, dim3(cw), 0, stream, (const uint16_t*)kv,
+                          (const uint16_t*)gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
+                          item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
     } else {
-        compress_kernel<128><<<grid, threads, 0, stream>>>(
-            (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
-            item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
+        const int tg = cw == 32 ? 16 : 4;             // token groups: 16 x 8 or 4 x 32 tokens
+        return launch_pdl(compress_kernel<128>, grid, dim3(tg * cw), 0, stream,
+                          (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off,
+                          kv_pos0, ent_off, item_seq, item_ent, B, m, D, fmt, log2_theta, eps,
+                          (uint8_t*)entries, st);
     }
     return cudaGetLastError();
 }

@@ -20,6 +20,8 @@ __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
     const int32_t* __restrict__ q_pos, int B, int HI, int m, int max_n,
     float* __restrict__ scores, int64_t ld, int32_t* __restrict__ dev_status) {
     extern __shared__ float smem[];
+    pdl_wait();
+    pdl_trigger();
     float* qf = smem;              // [HI][DI]
     float* wsh = smem + HI * DI;   // [HI]
     const int qq = blockIdx.y;
@@ -82,13 +84,15 @@ cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float*
     const size_t smem = sizeof(float) * (size_t)(HI * dI + HI);
     LaunchScope scope(kKIndexerSimt, stream);
     if (dI == 64) {
-        indexer_score_simt_kernel<64><<<grid, 128, smem, stream>>>(
-            qI, qs, w, kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n, scores, ld, st);
+        return launch_pdl(indexer_score_simt_kernel<64>, grid, dim3(128), smem, stream, qI, qs, w,
+                          kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n,
+                          scores, ld, st);
     } else {
         cudaFuncSetAttribute(indexer_score_simt_kernel<128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        indexer_score_simt_kernel<128><<<grid, 128, smem, stream>>>(
-            qI, qs, w, kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n, scores, ld, st);
+        return launch_pdl(indexer_score_simt_kernel<128>, grid, dim3(128), smem, stream, qI, qs,
+                          w, kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n,
+                          scores, ld, st);
     }
     return cudaGetLastError();
 }

@@ -35,6 +35,7 @@ constexpr int kDI = 128;                 // indexer dim (MMA K total, bytes per 
 constexpr int kTileBytes = kTileRows * kDI;
 constexpr int kChunkTiles = 8;           // tiles per work item
 constexpr int kThreads = 192;
+constexpr int kMaxItems = 512;            // work items per CTA resolved up front
 
 struct IdxArgs {
     const float* qs;
@@ -88,6 +89,16 @@ __device__ __forceinline__ bool get_item(const IdxArgs& a, int it, Item& x, bool
     return x.ntiles > 0;
 }
 
+// Item ii of this CTA: from the table built at kernel start, or decoded directly past it.
+__device__ __forceinline__ bool fetch_item(const IdxArgs& a, const Item* items, int ii, Item& x,
+                                           bool report) {
+    if (ii < kMaxItems) {
+        x = items[ii];
+        return x.ntiles > 0;
+    }
+    return get_item(a, blockIdx.x + ii * gridDim.x, x, report);
+}
+
 template <int HI>
 __global__ void __launch_bounds__(kThreads, 2)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -110,7 +121,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t* drain = accempty + 2;                      // [1]
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
+    Item* items = reinterpret_cast<Item*>(tmem_base_smem + 4);   // [kMaxItems]
+    // this CTA's work items: it = blockIdx.x + i * gridDim.x
+    const int n_my = blockIdx.x < a.total_items
+                         ? (a.total_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    // resolve their metadata (dependent loads) in parallel, once; later items on the fly
+    for (int i = threadIdx.x; i < min(n_my, kMaxItems); i += kThreads) {
+        Item x;
+        if (!get_item(a, blockIdx.x + i * gridDim.x, x, true)) x.ntiles = 0;
+        items[i] = x;
+    }
 
+    // The indexer reads only its inputs (keys and query heads), never an earlier kernel's
+    // output, and its score writes are safe once it has started (the previous step's top-k
+    // finished before the kernel before this one passed its own wait): let the next kernel
+    // launch right away; the wait at the end keeps completion ordered for later kernels.
+    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; s++) {
@@ -147,9 +173,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             int issued[kStages] = {};
             int bissued[2] = {0, 0};
             bool ok = true;
-            for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
+            for (int ii = 0; ii < n_my && ok; ii++) {
                 Item x;
-                if (!get_item(a, it, x, false)) continue;
+                if (!fetch_item(a, items, ii, x, false)) continue;
                 const int bb = nitem & 1;
                 if (!mbar_wait(&bempty[bb], ((nitem >> 1) & 1) ^ 1, abort_flag, a.st)) break;
                 mbar_arrive_expect_tx(&bfull[bb], kQBytes);
@@ -184,9 +210,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint32_t sphase = 0;
             int nitem = 0, nacc = 0;
             bool ok = true;
-            for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
+            for (int ii = 0; ii < n_my && ok; ii++) {
                 Item x;
-                if (!get_item(a, it, x, false)) continue;
+                if (!fetch_item(a, items, ii, x, false)) continue;
                 const int bb = nitem & 1;
                 if (!mbar_wait(&bfull[bb], (nitem >> 1) & 1, abort_flag, a.st)) break;
                 tc_fence_after();
@@ -225,18 +251,27 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int row_in_tile = quarter * 32 + lane;
         int nacc = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
+        for (int ii = 0; ii < n_my && ok; ii++) {
             Item x;
-            if (!get_item(a, it, x, threadIdx.x == 64)) continue;
+            if (!fetch_item(a, items, ii, x, threadIdx.x == 64)) continue;
             float ws[HI];
 #pragma unroll
             for (int h = 0; h < HI; h++)
                 ws[h] = __ldg(a.w + (int64_t)x.q * HI + h) * __ldg(a.qs + (int64_t)x.q * HI + h);
             float* srow = a.scores + (int64_t)x.q * a.ld;
-            for (int tt = 0; tt < x.ntiles; tt++) {
+            // all key scales of the item at once: one load latency per item, not per tile
+            float kscales[kChunkTiles];
+#pragma unroll
+            for (int tt = 0; tt < kChunkTiles; tt++) {
+                const int e = (x.tile0 + tt) * kTileRows + row_in_tile;
+                kscales[tt] = (tt < x.ntiles && e < x.n_vis) ? __ldg(a.ks + x.row0 + e) : 0.f;
+            }
+#pragma unroll
+            for (int tt = 0; tt < kChunkTiles; tt++) {
+                if (tt >= x.ntiles) break;
                 const int e = (x.tile0 + tt) * kTileRows + row_in_tile;
                 const bool live = e < x.n_vis;
-                const float kscale = live ? __ldg(a.ks + x.row0 + e) : 0.f;
+                const float kscale = kscales[tt];
                 const int ab = nacc & 1;
                 if (!mbar_wait_warp(&accfull[ab], (nacc >> 1) & 1, abort_flag, a.st)) {
                     ok = false;
@@ -269,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     }
 
+    pdl_wait();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -279,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 template <int HI>
 size_t smem_bytes() {
-    return 1024 + kStages * kTileBytes + 2 * HI * kDI + (2 * kStages + 9) * 8 + 16;
+    return 1024 + kStages * kTileBytes + 2 * HI * kDI + (2 * kStages + 9) * 8 + 16 +
+           kMaxItems * sizeof(Item);
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -339,8 +376,7 @@ cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const IdxArgs& args,
     if (e != cudaSuccess) return e;
     const int grid = min(args.total_items, 2 * num_sms());
     LaunchScope scope(kKIndexerTc, stream);
-    indexer_tc_kernel<HI><<<grid, kThreads, sm, stream>>>(mk, mq, args);
-    return cudaGetLastError();
+    return launch_pdl(indexer_tc_kernel<HI>, dim3(grid), dim3(kThreads), sm, stream, mk, mq, args);
 }
 
 }  // namespace

@@ -26,6 +26,16 @@ std::vector<cudaEvent_t> g_pool;
 long long g_count[kKernelKinds];
 double g_ms[kKernelKinds];
 
+// Inside a stream capture an event record only orders work within the graph unless it is
+// recorded as an external node, which timestamps on every replay.
+void record(cudaEvent_t ev, cudaStream_t stream) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+        cudaEventRecordWithFlags(ev, stream, cudaEventRecordExternal);
+    else
+        cudaEventRecord(ev, stream);
+}
+
 cudaEvent_t take_event() {
     if (!g_pool.empty()) {
         cudaEvent_t e = g_pool.back();
@@ -51,13 +61,13 @@ LaunchScope::LaunchScope(int kind, cudaStream_t stream) : kind_(kind), stream_(s
         std::lock_guard<std::mutex> lk(g_mu);
         start_ = take_event();
         stop_ = take_event();
-        if (start_ && stop_) cudaEventRecord(start_, stream_);
+        if (start_ && stop_) record(start_, stream_);
     }
 }
 
 LaunchScope::~LaunchScope() {
     if (start_ && stop_) {
-        cudaEventRecord(stop_, stream_);
+        record(stop_, stream_);
         std::lock_guard<std::mutex> lk(g_mu);
         g_pending.push_back({kind_, start_, stop_});
     }
@@ -71,7 +81,7 @@ long long csa_launch_count(void) { return csa::g_launches.load(); }
 
 void csa_profile_enable(int on) { csa::g_timing.store(on ? 1 : 0); }
 
-int csa_profile_collect(csa_kernel_time_t* out, int max_entries) {
+int csa_profile_collect(csa_kernel_time_t* out, int max_entries, int keep_pending) {
     std::lock_guard<std::mutex> lk(csa::g_mu);
     for (const auto& p : csa::g_pending) {
         float ms = 0.f;
@@ -80,10 +90,12 @@ int csa_profile_collect(csa_kernel_time_t* out, int max_entries) {
             csa::g_count[p.kernel] += 1;
             csa::g_ms[p.kernel] += ms;
         }
-        csa::g_pool.push_back(p.start);
-        csa::g_pool.push_back(p.stop);
+        if (!keep_pending) {
+            csa::g_pool.push_back(p.start);
+            csa::g_pool.push_back(p.stop);
+        }
     }
-    csa::g_pending.clear();
+    if (!keep_pending) csa::g_pending.clear();
     int n = 0;
     for (int k = 0; k < csa::kKernelKinds && n < max_entries; k++) {
         if (csa::g_count[k] == 0) continue;

@@ -6,14 +6,19 @@
 // not depend on how the work is partitioned -- the result is batch-invariant by
 // construction.
 //
-// One CTA (1024 threads) per query.  Scores map to order-preserving 32-bit keys.  Three
-// radix passes (11, 11 and 10 bits) find the k-th largest key T and how many keys equal
-// to T are needed: each pass histograms the keys that match the prefix found so far with
-// warp-aggregated shared-memory atomics (lanes hitting the same bin add once), then a
-// block-wide scan over the 2048 bins, from the top, picks the bin holding the k-th key.
-// A last pass in ascending entry order takes every key > T and the first needed keys
-// == T; one block-wide scan per 4096-entry chunk gives each thread its output slots, so
-// the indices come out already sorted.  Score rows are read with 16-byte loads.
+// One CTA (1024 threads) per query, scores mapped to order-preserving 32-bit keys.  The
+// goal is the k-th largest key T and the number of keys equal to T to take.
+//  1. Rows of up to 50K scores are staged in shared memory with 16-byte loads; the OR and
+//     AND of all keys give the bits every key shares, so the radix starts at the highest
+//     bit that varies (scores of one query share sign and most exponent bits, and a fixed
+//     first digit would put nearly all of them in one bin).
+//  2. An 11-bit histogram of that digit (shared-memory atomics) and a block-wide scan over
+//     the bins, from the top, give the bin holding the k-th key.
+//  3. Keys in that bin are compacted to a short candidate list (if it fits), and the
+//     remaining bits are resolved on the list; otherwise further full passes run.
+//  4. A last pass in ascending entry order takes every key > T and the first needed keys
+//     == T; one block-wide scan per 4096-entry chunk gives each thread its output slots,
+//     so the indices come out already sorted.
 #include "launchers.cuh"
 
 namespace csa {
@@ -24,6 +29,7 @@ constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kChunk = 4 * kThreads;
+constexpr int kMaxCand = 4096;
 
 __device__ __forceinline__ uint32_t score_key(float s) {
     uint32_t u = __float_as_uint(s);
@@ -76,19 +82,48 @@ __device__ __forceinline__ void load4(const float* s, int i, int n, bool vec, ui
     }
 }
 
+struct Shared {
+    uint32_t hist[kBins];
+    uint32_t scan_tmp[33];
+    uint32_t bin, krem, key_or, key_and, ncand;
+    uint32_t cand[kMaxCand];
+};
+
+// After hist[] holds the counts of the current digit: picks the bin holding the krem-th
+// largest key (bins scanned from the top) and the rank left inside it.
+__device__ __forceinline__ void pick_bin(Shared& sh, uint32_t& krem) {
+    const int tid = threadIdx.x;
+    const int bhi = kBins - 1 - 2 * tid, blo = bhi - 1;
+    const uint32_t chi = sh.hist[bhi], clo = sh.hist[blo];
+    uint32_t tot;
+    const uint32_t above = block_exclusive_scan(chi + clo, sh.scan_tmp, tot);
+    if (above < krem && krem <= above + chi) {
+        sh.bin = (uint32_t)bhi;
+        sh.krem = krem - above;
+    } else if (above + chi < krem && krem <= above + chi + clo) {
+        sh.bin = (uint32_t)blo;
+        sh.krem = krem - above - chi;
+    }
+    __syncthreads();
+    krem = sh.krem;
+}
+
+// STAGED: the query's score row is first copied to shared memory (16-byte loads, eight in
+// flight per thread) and every pass reads it from there.
+template <bool STAGED>
 __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_seq,
     const int32_t* __restrict__ q_pos, const int64_t* __restrict__ seq_len, int B, int m,
     int max_n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ dev_status) {
-    __shared__ uint32_t hist[kBins];
-    __shared__ uint32_t scan_tmp[33];
-    __shared__ uint32_t sh_bin, sh_krem;
+    __shared__ Shared sh;
     const int qq = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31;
     const int b = q_seq[qq];
     const int t = q_pos[qq];
     // invalid queries (flagged by the scoring kernel) select nothing
     const bool valid = b >= 0 && b < B && t >= 0 && (int64_t)t < seq_len[b];
+    pdl_wait();   // scores come from the indexer
+    pdl_trigger();
     int n = valid ? (t + 1) / m : 0;
     if (n > max_n) n = max_n;  // capacity already flagged by the scoring kernel
     const float* s = scores + (int64_t)qq * ld;
@@ -97,44 +132,121 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         for (int j = tid; j < k; j += kThreads) out[j] = j < n ? j : -1;
         return;
     }
-    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
-
-    uint32_t prefix = 0u, mask = 0u, krem = (uint32_t)k;
-    for (int pass = 0; pass < 3; pass++) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const uint32_t bmask = pass == 2 ? 1023u : 2047u;
-        for (int x = tid; x < kBins; x += kThreads) hist[x] = 0u;
-        __syncthreads();
-        for (int c0 = 0; c0 < n; c0 += kChunk) {   // uniform trip count: whole warps
-            const int i0 = c0 + 4 * tid;
+    bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
+    if (tid == 0) {
+        sh.key_or = 0u;
+        sh.key_and = 0xFFFFFFFFu;
+        sh.ncand = 0u;
+    }
+    __syncthreads();
+    uint32_t kor = 0u, kand = 0xFFFFFFFFu;
+    if constexpr (STAGED) {
+        extern __shared__ float4 srow4[];
+        float* srow = reinterpret_cast<float*>(srow4);
+        constexpr int kBatch = 8;
+        for (int i0 = 4 * tid; i0 < n; i0 += 4 * kThreads * kBatch) {
+            float4 v[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; u++) {
+                const int i = i0 + u * 4 * kThreads;
+                if (vec && i + 3 < n) {
+                    v[u] = *reinterpret_cast<const float4*>(s + i);
+                } else {
+                    v[u].x = i < n ? s[i] : 0.f;
+                    v[u].y = i + 1 < n ? s[i + 1] : 0.f;
+                    v[u].z = i + 2 < n ? s[i + 2] : 0.f;
+                    v[u].w = i + 3 < n ? s[i + 3] : 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; u++) {
+                const int i = i0 + u * 4 * kThreads;
+                if (i < n) *reinterpret_cast<float4*>(srow + i) = v[u];
+                const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int z = 0; z < 4; z++) {
+                    if (i + z < n) {
+                        const uint32_t key = score_key(e[z]);
+                        kor |= key;
+                        kand &= key;
+                    }
+                }
+            }
+        }
+        s = srow;
+        vec = true;
+    } else {
+        for (int c0 = 0; c0 < n; c0 += kChunk) {
             uint32_t key[4];
-            load4(s, i0, n, vec, key);
+            load4(s, c0 + 4 * tid, n, vec, key);
 #pragma unroll
             for (int u = 0; u < 4; u++) {
-                const bool hit = (i0 + u < n) && ((key[u] & mask) == prefix);
-                const uint32_t bin = hit ? ((key[u] >> shift) & bmask) : 0xFFFFFFFFu;
-                const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-                if (hit && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+                if (c0 + 4 * tid + u < n) {
+                    kor |= key[u];
+                    kand &= key[u];
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+        kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+    }
+    if (lane == 0) {
+        atomicOr(&sh.key_or, kor);
+        atomicAnd(&sh.key_and, kand);
+    }
+    __syncthreads();
+    const uint32_t diff = sh.key_or ^ sh.key_and;   // bits that vary across the row
+    uint32_t prefix = sh.key_and & ~diff;           // = the bits all keys share
+    uint32_t mask = ~diff;
+    uint32_t krem = (uint32_t)k;
+    // digits from the highest varying bit down, 11 bits at a time
+    int top = diff ? 31 - __clz(diff) : -1;
+    bool compacted = false;
+    while (top >= 0) {
+        const int width = top >= 10 ? 11 : top + 1;
+        const int shift = top + 1 - width;
+        const uint32_t bmask = (1u << width) - 1u;
+        for (int x = tid; x < kBins; x += kThreads) sh.hist[x] = 0u;
+        __syncthreads();
+        if (!compacted) {
+            for (int c0 = 0; c0 < n; c0 += kChunk) {
+                uint32_t key[4];
+                load4(s, c0 + 4 * tid, n, vec, key);
+#pragma unroll
+                for (int u = 0; u < 4; u++)
+                    if (c0 + 4 * tid + u < n && (key[u] & mask) == prefix)
+                        atomicAdd(&sh.hist[(key[u] >> shift) & bmask], 1u);
+            }
+        } else {
+            for (uint32_t c = tid; c < sh.ncand; c += kThreads) {
+                const uint32_t key = sh.cand[c];
+                if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & bmask], 1u);
             }
         }
         __syncthreads();
-        // bins from the top: thread t owns bins 2047 - 2t and 2046 - 2t
-        const int bhi = kBins - 1 - 2 * tid, blo = bhi - 1;
-        const uint32_t chi = hist[bhi], clo = hist[blo];
-        uint32_t tot;
-        const uint32_t above = block_exclusive_scan(chi + clo, scan_tmp, tot);
-        if (above < krem && krem <= above + chi) {
-            sh_bin = (uint32_t)bhi;
-            sh_krem = krem - above;
-        } else if (above + chi < krem && krem <= above + chi + clo) {
-            sh_bin = (uint32_t)blo;
-            sh_krem = krem - above - chi;
-        }
-        __syncthreads();
-        prefix |= sh_bin << shift;
+        pick_bin(sh, krem);
+        const uint32_t bin = sh.bin;
+        const uint32_t in_bin = sh.hist[bin];
+        prefix |= bin << shift;
         mask |= bmask << shift;
-        krem = sh_krem;
+        top = shift - 1;
         __syncthreads();
+        if (!compacted && top >= 0 && in_bin <= (uint32_t)kMaxCand) {
+            // keys in the chosen bin become the candidate list for the remaining bits
+            for (int c0 = 0; c0 < n; c0 += kChunk) {
+                uint32_t key[4];
+                load4(s, c0 + 4 * tid, n, vec, key);
+#pragma unroll
+                for (int u = 0; u < 4; u++)
+                    if (c0 + 4 * tid + u < n && (key[u] & mask) == prefix)
+                        sh.cand[atomicAdd(&sh.ncand, 1u)] = key[u];
+            }
+            compacted = true;
+            __syncthreads();
+        }
     }
     const uint32_t T = prefix;   // the k-th largest key; krem keys equal to T are taken
     // ordered collection: 4096 entries per round, 4 consecutive per thread
@@ -151,7 +263,7 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
             neq += (in && key[u] == T) ? 1u : 0u;
         }
         uint32_t tot;
-        const uint32_t packed = block_exclusive_scan(ngt | (neq << 16), scan_tmp, tot);
+        const uint32_t packed = block_exclusive_scan(ngt | (neq << 16), sh.scan_tmp, tot);
         uint32_t eq_rank = ties_before + (packed >> 16);   // tie rank of my first tie
         uint32_t pos = written + (packed & 0xFFFFu) + (min(eq_rank, krem) - min(ties_before, krem));
 #pragma unroll
@@ -180,9 +292,22 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream) {
     if (Q == 0) return cudaSuccess;
-    LaunchScope scope(kKTopk, stream);
-    topk_radix_kernel<<<Q, kThreads, 0, stream>>>(scores, ld, q_seq, q_pos, seq_len, B, m, max_n,
-                                                  k, idx_out, st);
+    // rows of up to ~44K scores are staged in shared memory (with the ~25 KB of histogram
+    // and candidate space this stays under the 227 KB per-CTA limit)
+    const size_t row_bytes = (size_t)((max_n + 3) / 4) * 16;
+    cudaError_t e;
+    if (row_bytes <= (size_t)176 * 1024) {
+        e = cudaFuncSetAttribute(topk_radix_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)row_bytes);
+        if (e != cudaSuccess) return e;
+        LaunchScope scope(kKTopk, stream);
+        return launch_pdl(topk_radix_kernel<true>, dim3(Q), dim3(kThreads), row_bytes, stream,
+                          scores, ld, q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st);
+    } else {
+        LaunchScope scope(kKTopk, stream);
+        return launch_pdl(topk_radix_kernel<false>, dim3(Q), dim3(kThreads), 0, stream, scores, ld,
+                          q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st);
+    }
     return cudaGetLastError();
 }
 
