@@ -14,7 +14,8 @@
 //
 // Roles per CTA (8 warps, persistent over items):
 //   warp 0      producer: dense tiles by two 2D TMA loads (64 channels x 128 rows each,
-//               128-byte swizzle), sparse tiles by zero-filling 16-byte cp.async gathers to
+//               128-byte swizzle), sparse tiles by TMA tile::gather4 loads of the selected
+//               rows (4 rows x 64 channels each; an invalid index is row -1, zero-filled) into
 //               the same swizzled layout; a per-tile validity mask; 3-stage ring.
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
 //               S = Q K^T as two M=64 x N=64 halves (keys 0-63 -> TMEM lanes 0-15 of each
@@ -122,18 +123,6 @@ __device__ __forceinline__ uint32_t swz(int r, int ch) {
     return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-                 "r"(src_bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(
-                     sm100::smem_addr(bar))
-                 : "memory");
-}
-
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -152,7 +141,8 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(const void* tile, uint32_
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_e, const AttnTcArgs a) {
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_e,
+                   const __grid_constant__ CUtensorMap tmap_g, const AttnTcArgs a) {
     using namespace sm100;
     constexpr uint32_t kIdescS = instr_desc(1, 1, 64, 64);
     constexpr uint32_t kIdescPV = instr_desc(1, 1, 64, 64, 1);
@@ -172,7 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* rwc = rqs + 32;
     float* rws = rwc + 32;
     int32_t* sidx = reinterpret_cast<int32_t*>(rws + 32);   // [kMaxK] the item's index row
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sidx + kMaxK);
+    int32_t* srows = sidx + kMaxK;                          // [kStages][128] gather rows
+    uint64_t* bars = reinterpret_cast<uint64_t*>(srows + kStages * kTK);
     uint64_t* full = bars;                 // [kStages]  33 arrivals (+tx)
     uint64_t* empty = full + kStages;      // [kStages]  MMA commit
     uint64_t* prep_full = empty + kStages; // Q + window ready: 4 arrivals
@@ -206,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(drain, 1);
         *abort_flag = 0;
         mbar_fence_init();
-        if (!a.idx) prefetch_tmap(&tmap_e);
+        prefetch_tmap(a.idx ? &tmap_g : &tmap_e);
     }
     if (warp == 1) {
         tmem_alloc(tmem_base_smem, 256);
@@ -233,10 +224,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             AItem x;
             if (!get_item(a, it, x, false)) continue;
             if (a.idx) {
-                // the query's whole index row, once per item (one load round trip, not one
-                // per tile); only this warp reads it
+                // the query's whole index row, once per item: batches of 8 x 16-byte loads
+                // per lane in flight (one round trip for k <= 1024); only this warp reads it
                 const int32_t* src = a.idx + (int64_t)x.q * a.k;
-                for (int v = lane; v < a.k; v += 32) sidx[v] = src[v];
+                if ((a.k & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+                    const int n4 = a.k >> 2;
+                    for (int base = 0; base < n4; base += 32 * 8) {
+                        int4 v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; u++) {
+                            const int j4 = base + lane + 32 * u;
+                            if (j4 < n4) v[u] = *reinterpret_cast<const int4*>(src + 4 * j4);
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; u++) {
+                            const int j4 = base + lane + 32 * u;
+                            if (j4 < n4) *reinterpret_cast<int4*>(sidx + 4 * j4) = v[u];
+                        }
+                    }
+                } else {
+                    for (int base = 0; base < a.k; base += 32 * 8) {
+                        int v[8];
+#pragma unroll
+                        for (int u = 0; u < 8; u++) {
+                            const int j = base + lane + 32 * u;
+                            v[u] = j < a.k ? src[j] : -1;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; u++) {
+                            const int j = base + lane + 32 * u;
+                            if (j < a.k) sidx[j] = v[u];
+                        }
+                    }
+                }
                 __syncwarp();
             }
             for (int jj = 0; jj < x.ntiles; jj++) {
@@ -262,33 +282,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __syncwarp();
                     if (lane != 0) mbar_arrive(&full[stage]);
                 } else {
-                    const uint32_t dbase = smem_addr(dst);
+                    // rows of the selected entries: lanes resolve 4 each (invalid -> row -1,
+                    // which the TMA zero-fills), lane 0 issues 4-row gathers per 64 channels
+                    int32_t* rows = srows + stage * kTK;
 #pragma unroll
                     for (int rr = 0; rr < 4; rr++) {
                         const int r = lane + 32 * rr;
                         const int v = e0 + r;
-                        bool valid = false;
-                        const uint8_t* src = a.entries;
+                        int32_t row = -1;
                         if (v < x.n_ent) {
                             const int e = sidx[v];
                             if (e >= 0) {
                                 if (e < x.n_vis && x.row0 + e < a.ent_rows) {
-                                    valid = true;
-                                    src = a.entries + (x.row0 + e) * (int64_t)(kD * 2);
+                                    row = (int32_t)(x.row0 + e);
                                 } else {
                                     flag(a.st, CSA_DEV_OOB);
                                 }
                             }
                         }
-                        const uint32_t nb = valid ? 16u : 0u;
-#pragma unroll
-                        for (int ch = 0; ch < 16; ch++)
-                            cp_async16(dbase + (ch >> 3) * kBlk + swz(r, ch & 7), src + ch * 16, nb);
-                        const unsigned vm = __ballot_sync(0xffffffffu, valid);
+                        rows[r] = row;
+                        const unsigned vm = __ballot_sync(0xffffffffu, row >= 0);
                         if (lane == 0) smask[stage * 4 + rr] = vm;
                     }
-                    cp_async_arrive_noinc(&full[stage]);
                     __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&full[stage], kTileBytes);
+#pragma unroll 4
+                        for (int g = 0; g < kTK / 4; g++) {
+                            const int32_t r0 = rows[4 * g], r1 = rows[4 * g + 1],
+                                          r2 = rows[4 * g + 2], r3 = rows[4 * g + 3];
+                            tma_gather4(dst + 4 * g * 128, &tmap_g, &full[stage], 0, r0, r1, r2, r3);
+                            tma_gather4(dst + kBlk + 4 * g * 128, &tmap_g, &full[stage], 64, r0, r1,
+                                        r2, r3);
+                        }
+                    } else {
+                        mbar_arrive(&full[stage]);
+                    }
                 }
                 if (lane == 0) mbar_arrive(&full[stage]);
                 issued[stage]++;
@@ -326,8 +355,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ok = false;
                             break;
                         }
-                        // gathered tiles were written by cp.async (generic proxy)
-                        fence_async_smem();
                         kb = sK + stage * kTileBytes;
                         my_stage = stage;
                         if (++stage == kStages) {
@@ -765,7 +792,7 @@ int sm_count() {
 }
 
 constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + kTileBytes + 2 * kQBlk + 4 * kPBlk +
-                              4 * (kStages + 1) * 4 + 5 * 32 * 4 + kMaxK * 4 +
+                              4 * (kStages + 1) * 4 + 5 * 32 * 4 + kMaxK * 4 + kStages * kTK * 4 +
                               (2 * kStages + 15) * 8 + 16;
 
 int dense_chunks_per_q(int max_n) {
@@ -817,17 +844,20 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
         a.chunks_per_q = dense_chunks_per_q(max_n);
     }
     a.total_items = Q * a.chunks_per_q;
-    CUtensorMap map;
-    std::memset(&map, 0, sizeof(map));
-    if (!aa.idx && aa.ent_rows > 0) {
+    // dense: 128-row boxes of contiguous entries; sparse: one-row boxes for 4-row gathers
+    CUtensorMap map_e, map_g;
+    std::memset(&map_e, 0, sizeof(map_e));
+    std::memset(&map_g, 0, sizeof(map_g));
+    if (aa.ent_rows > 0) {
         EncodeFn enc = encode_fn();
         if (!enc) return cudaErrorInvalidValue;
         const cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)aa.ent_rows};
         const cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-        const cuuint32_t box[2] = {64, (cuuint32_t)kTK};
+        const cuuint32_t box[2] = {64, aa.idx ? 1u : (cuuint32_t)kTK};
         const cuuint32_t estr[2] = {1, 1};
-        if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint8_t*>(aa.entries), dims,
-                strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+        if (enc(aa.idx ? &map_g : &map_e, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                const_cast<uint8_t*>(aa.entries), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
@@ -838,7 +868,8 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
     const int grid = min(a.total_items, sm_count());
     {
         LaunchScope scope(kKAttnTc, stream);
-        e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, map, a);
+        e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, map_e,
+                       map_g, a);
     }
     if (e != cudaSuccess || aa.idx) return e;
     LaunchScope scope(kKAttnCombine, stream);

@@ -6,18 +6,26 @@
 //
 // Decode is HBM-bound (each 132-byte key row is read once and feeds 64 x 128 MACs, about
 // 124 FLOP/byte), but that intensity still needs the tensor pipe to keep up with HBM.
-// Persistent CTAs walk a static list of work items (query, chunk of 8 tiles of 128
-// entries); tiles are aligned to the query's sequence, so every entry is always computed
-// in the same tile row by the same instructions whatever the batch.  Roles per CTA
-// (6 warps):
-//   warp 0 lane 0  TMA producer: per item the query's heads (H_I x 128 e4m3, B operand),
-//                  per tile 128 key rows (128 x 128 e4m3, A operand), 128-byte swizzle,
-//                  into a 4-stage ring;
-//   warp 1         TMEM allocation; lane 0 issues tcgen05.mma kind::f8f6f4
-//                  (M=128 entries, N=H_I heads, 4 x K=32) into one of two TMEM
-//                  accumulators and commits to the stage's and accumulator's barriers;
-//   warps 2-5      epilogue: tcgen05.ld of one entry row (all heads) per thread, the
-//                  fixed-order fmaf chain, the key scale, a coalesced score store.
+// Work is counted in tiles of 128 entries, aligned to each query's sequence; query q owns
+// the tiles [q * T, q * T + T) of a virtual tile space (T = tiles of the longest query).
+// One persistent CTA per SM takes an equal contiguous range of that space and walks it as
+// items: the pieces of the range cut at query boundaries and every 8 tiles.  Every entry
+// is always computed in the same tile row by the same instructions whatever the batch.
+// Roles per CTA (11 warps):
+//   warp 0 lane 0  TMA producer: per query the heads (H_I x 128 e4m3, B operand, reused
+//                  across consecutive items of the query); per stage a group of up to four
+//                  tiles of 128 key rows (A operand), 128-byte swizzle, 3 x 64 KB ring; it
+//                  decodes its items itself and starts before the others' item table;
+//   warp 1         TMEM allocation; lane 0 issues tcgen05.mma kind::f8f6f4 (M=128 entries,
+//                  N=H_I heads, 4 x K=32 per tile) into one of two sets of four TMEM
+//                  accumulators, the K steps of the group's tiles interleaved;
+//   warp 2         item prefetch: w_h * qs_h of the item's query and the key scales of
+//                  its tiles into a shared-memory ring, ahead of the epilogue;
+//   warps 3-10     epilogue in two groups of four taking alternate tiles of a group:
+//                  tcgen05.ld of one entry row (all heads) per thread, the fixed-order fmaf
+//                  chain, the key scale, a coalesced score store.
+// Barriers are per group of tiles, not per tile: under load every mbarrier operation costs
+// the single issuing thread on the order of a hundred cycles.
 // Every wait is bounded; a timeout aborts the CTA, drains its own copies and MMAs,
 // frees TMEM and reports CSA_DEV_TIMEOUT.
 #include <mutex>
@@ -29,13 +37,19 @@ namespace csa {
 
 namespace {
 
-constexpr int kStages = 4;
+constexpr int kGroupTiles = 4;           // tiles per pipeline stage (one barrier each way)
+constexpr int kStages = 3;               // 3 x 64 KB of key tiles in flight per SM
+constexpr int kAccSets = 2;              // TMEM accumulator sets of kGroupTiles accumulators
+constexpr int kAux = 3;                  // prefetched items
 constexpr int kTileRows = 128;           // entries per tile (MMA M)
 constexpr int kDI = 128;                 // indexer dim (MMA K total, bytes per key row)
 constexpr int kTileBytes = kTileRows * kDI;
-constexpr int kChunkTiles = 8;           // tiles per work item
-constexpr int kThreads = 192;
-constexpr int kMaxItems = 512;            // work items per CTA resolved up front
+constexpr int kGroupBytes = kGroupTiles * kTileBytes;
+constexpr int kChunkTiles = 8;           // tiles per item at most
+constexpr int kFirstEpiWarp = 3;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
+constexpr int kMaxItems = 64;            // work items per CTA resolved up front
 
 struct IdxArgs {
     const float* qs;
@@ -49,7 +63,9 @@ struct IdxArgs {
     int64_t ld;
     int64_t ent_rows;
     int32_t* st;
-    int Q, B, m, max_n, chunks_per_q, total_items;
+    int Q, B, m, max_n;
+    int qtiles;              // virtual tiles per query: ceil(max_n / 128)
+    int chunks_per_q;        // ceil(qtiles / 8)
 };
 
 struct Item {
@@ -60,77 +76,110 @@ struct Item {
     int64_t row0;
 };
 
-// Decodes work item `it`; false when it has no tiles.  Every role calls this with the same
-// arguments and so walks the same item sequence.
-__device__ __forceinline__ bool get_item(const IdxArgs& a, int it, Item& x, bool report) {
-    x.q = it / a.chunks_per_q;
-    const int c = it - x.q * a.chunks_per_q;
+// Virtual tile range [v0, v1) of CTA `cta` of `grid`; equal shares of Q * qtiles.
+__device__ __forceinline__ void cta_range(const IdxArgs& a, int cta, int grid, int64_t& v0,
+                                          int64_t& v1) {
+    const int64_t V = (int64_t)a.Q * a.qtiles;
+    v0 = V * cta / grid;
+    v1 = V * (cta + 1) / grid;
+}
+
+__device__ __forceinline__ int64_t chunk_of(const IdxArgs& a, int64_t v) {
+    const int64_t q = v / a.qtiles;
+    return q * a.chunks_per_q + (v - q * a.qtiles) / kChunkTiles;
+}
+
+// Decodes item `ii` of the range [v0, v1) (the piece of the range inside its ii-th chunk);
+// false when it has no tiles.  Every role calls this with the same arguments and so walks
+// the same item sequence.
+__device__ __forceinline__ bool get_item(const IdxArgs& a, int64_t v0, int64_t v1, int ii,
+                                         Item& x, bool report) {
+    const int64_t g = chunk_of(a, v0) + ii;
+    x.q = (int)(g / a.chunks_per_q);
+    const int cq = (int)(g - (int64_t)x.q * a.chunks_per_q);
+    const int64_t cbeg = (int64_t)x.q * a.qtiles + (int64_t)cq * kChunkTiles;
+    const int64_t cend = min(cbeg + kChunkTiles, (int64_t)(x.q + 1) * a.qtiles);
+    const int lo = (int)(max(v0, cbeg) - cbeg);
+    const int hi = (int)(min(v1, cend) - cbeg);
+    report = report && cq == 0 && lo == 0;   // one piece per query reports its errors
     const int b = a.q_seq[x.q];
     const int t = a.q_pos[x.q];
     if (b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]) {
-        if (report && c == 0) flag(a.st, CSA_DEV_OOB);
+        if (report) flag(a.st, CSA_DEV_OOB);
         return false;
     }
     int n = (t + 1) / a.m;
     if (n > a.max_n) {
-        if (report && c == 0) flag(a.st, CSA_DEV_CAPACITY);
+        if (report) flag(a.st, CSA_DEV_CAPACITY);
         n = a.max_n;
     }
     x.row0 = a.ent_off[b];
     const int64_t avail = a.ent_rows - x.row0;
     if ((int64_t)n > avail) {
-        if (report && c == 0) flag(a.st, CSA_DEV_OOB);
+        if (report) flag(a.st, CSA_DEV_OOB);
         n = avail > 0 ? (int)avail : 0;
     }
     x.n_vis = n;
-    x.tile0 = c * kChunkTiles;
+    x.tile0 = cq * kChunkTiles + lo;
     const int tiles = (n + kTileRows - 1) / kTileRows;
-    x.ntiles = min(kChunkTiles, tiles - x.tile0);
+    x.ntiles = min(cq * kChunkTiles + hi, tiles) - x.tile0;
     return x.ntiles > 0;
 }
 
 // Item ii of this CTA: from the table built at kernel start, or decoded directly past it.
-__device__ __forceinline__ bool fetch_item(const IdxArgs& a, const Item* items, int ii, Item& x,
-                                           bool report) {
+__device__ __forceinline__ bool fetch_item(const IdxArgs& a, const Item* items, int64_t v0,
+                                           int64_t v1, int ii, Item& x, bool report) {
     if (ii < kMaxItems) {
         x = items[ii];
         return x.ntiles > 0;
     }
-    return get_item(a, blockIdx.x + ii * gridDim.x, x, report);
+    return get_item(a, v0, v1, ii, x, report);
+}
+
+// TMEM columns: kAccSets x kGroupTiles accumulators of HI fp32 columns, rounded to a power
+// of two >= 32.
+template <int HI>
+__host__ __device__ constexpr uint32_t tmem_cols() {
+    constexpr int c = kAccSets * kGroupTiles * HI;
+    return c <= 32 ? 32u : c <= 64 ? 64u : c <= 128 ? 128u : c <= 256 ? 256u : 512u;
+}
+
+// Floats of one prefetch slot: w*qs for the heads, then the key scales of up to 8 tiles.
+template <int HI>
+__host__ __device__ constexpr int aux_floats() {
+    return HI + kChunkTiles * kTileRows;
 }
 
 template <int HI>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_q, const IdxArgs a) {
     using namespace sm100;
     constexpr int kQBytes = HI * kDI;
+    constexpr int kAuxFloats = aux_floats<HI>();
     constexpr uint32_t kIdesc = instr_desc(0, 0, kTileRows, HI);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* sA = smem;                                  // [kStages][128 x 128]
-    uint8_t* sB = sA + kStages * kTileBytes;             // [2][HI x 128]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + 2 * kQBytes);
+    uint8_t* sA = smem;                                  // [kStages][kGroupTiles][128 x 128]
+    uint8_t* sB = sA + kStages * kGroupBytes;            // [2][HI x 128]
+    float* aux = reinterpret_cast<float*>(sB + 2 * kQBytes);   // [kAux][kAuxFloats]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(aux + kAux * kAuxFloats);
     uint64_t* full = bars;                               // [kStages]
     uint64_t* empty = full + kStages;                    // [kStages]
     uint64_t* bfull = empty + kStages;                   // [2]
     uint64_t* bempty = bfull + 2;                        // [2]
-    uint64_t* accfull = bempty + 2;                      // [2]
-    uint64_t* accempty = accfull + 2;                    // [2]
-    uint64_t* drain = accempty + 2;                      // [1]
+    uint64_t* accfull = bempty + 2;                      // [kAccSets]
+    uint64_t* accempty = accfull + kAccSets;             // [kAccSets]
+    uint64_t* auxfull = accempty + kAccSets;             // [kAux]
+    uint64_t* auxempty = auxfull + kAux;                 // [kAux]
+    uint64_t* drain = auxempty + kAux;                   // [1]
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
     Item* items = reinterpret_cast<Item*>(tmem_base_smem + 4);   // [kMaxItems]
-    // this CTA's work items: it = blockIdx.x + i * gridDim.x
-    const int n_my = blockIdx.x < a.total_items
-                         ? (a.total_items - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
-    // resolve their metadata (dependent loads) in parallel, once; later items on the fly
-    for (int i = threadIdx.x; i < min(n_my, kMaxItems); i += kThreads) {
-        Item x;
-        if (!get_item(a, blockIdx.x + i * gridDim.x, x, true)) x.ntiles = 0;
-        items[i] = x;
-    }
+    int64_t v0, v1;
+    cta_range(a, blockIdx.x, gridDim.x, v0, v1);
+    const int n_my = v1 > v0 ? (int)(chunk_of(a, v1 - 1) - chunk_of(a, v0) + 1) : 0;
 
     // The indexer reads only its inputs (keys and query heads), never an earlier kernel's
     // output, and its score writes are safe once it has started (the previous step's top-k
@@ -146,8 +195,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = 0; i < 2; i++) {
             mbar_init(&bfull[i], 1);
             mbar_init(&bempty[i], 1);
+        }
+        for (int i = 0; i < kAccSets; i++) {
             mbar_init(&accfull[i], 1);
-            mbar_init(&accempty[i], 4);
+            mbar_init(&accempty[i], kEpiWarps);
+        }
+        for (int i = 0; i < kAux; i++) {
+            mbar_init(&auxfull[i], 32);               // every lane of the prefetch warp
+            mbar_init(&auxempty[i], kEpiWarps);
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -156,41 +211,53 @@ __global__ void __launch_bounds__(kThreads, 2)
         prefetch_tmap(&tmap_q);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_base_smem, 2 * HI < 32 ? 32 : 2 * HI);
+        tmem_alloc(tmem_base_smem, tmem_cols<HI>());
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
+    if (warp > 0) {
+        // every role but the producer resolves the items' metadata (dependent loads) in
+        // parallel, once; items past the table are decoded on the fly
+        for (int i = threadIdx.x - 32; i < min(n_my, kMaxItems); i += kThreads - 32) {
+            Item x;
+            if (!get_item(a, v0, v1, i, x, true)) x.ntiles = 0;
+            items[i] = x;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kThreads - 32) : "memory");
+    }
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
             int stage = 0;
             uint32_t ephase = 0;
-            int nitem = 0;
-            int issued[kStages] = {};
-            int bissued[2] = {0, 0};
+            int nq = 0, cur_q = -1, ng = 0;   // queries and groups issued
             bool ok = true;
             for (int ii = 0; ii < n_my && ok; ii++) {
                 Item x;
-                if (!fetch_item(a, items, ii, x, false)) continue;
-                const int bb = nitem & 1;
-                if (!mbar_wait(&bempty[bb], ((nitem >> 1) & 1) ^ 1, abort_flag, a.st)) break;
-                mbar_arrive_expect_tx(&bfull[bb], kQBytes);
-                tma_load_2d(sB + bb * kQBytes, &tmap_q, &bfull[bb], 0, x.q * HI);
-                bissued[bb]++;
-                nitem++;
-                for (int tt = 0; tt < x.ntiles; tt++) {
+                if (!get_item(a, v0, v1, ii, x, false)) continue;
+                if (x.q != cur_q) {
+                    const int bb = nq & 1;
+                    if (!mbar_wait(&bempty[bb], ((nq >> 1) & 1) ^ 1, abort_flag, a.st)) break;
+                    mbar_arrive_expect_tx(&bfull[bb], kQBytes);
+                    tma_load_2d(sB + bb * kQBytes, &tmap_q, &bfull[bb], 0, x.q * HI);
+                    nq++;
+                    cur_q = x.q;
+                }
+                for (int g0 = 0; g0 < x.ntiles; g0 += kGroupTiles) {
+                    const int gt = min(kGroupTiles, x.ntiles - g0);
                     if (!mbar_wait(&empty[stage], ephase ^ 1, abort_flag, a.st)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], kTileBytes);
-                    tma_load_2d(sA + stage * kTileBytes, &tmap_k, &full[stage], 0,
-                                (int32_t)(x.row0 + (int64_t)(x.tile0 + tt) * kTileRows));
-                    issued[stage]++;
+                    mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
+                    for (int j = 0; j < gt; j++)
+                        tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k, &full[stage], 0,
+                                    (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows));
+                    ng++;
                     if (++stage == kStages) {
                         stage = 0;
                         ephase ^= 1;
@@ -198,109 +265,165 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
             // drain: every copy this thread issued must have landed before smem is released
-            for (int s = 0; s < kStages; s++)
-                if (issued[s]) mbar_drain(&full[s], (issued[s] - 1) & 1, a.st);
-            for (int i = 0; i < 2; i++)
-                if (bissued[i]) mbar_drain(&bfull[i], (bissued[i] - 1) & 1, a.st);
+            for (int s = 0; s < kStages; s++) {
+                const int cnt = ng / kStages + (s < ng % kStages ? 1 : 0);
+                if (cnt) mbar_drain(&full[s], (cnt - 1) & 1, a.st);
+            }
+            for (int i = 0; i < 2; i++) {
+                const int cnt = (nq - i + 1) / 2;
+                if (cnt) mbar_drain(&bfull[i], (cnt - 1) & 1, a.st);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
+            // One stage = one group of up to four tiles of one item.  The K steps of the
+            // group's tiles are interleaved across their accumulators: a small-N MMA chained
+            // on one accumulator waits for the previous one, so independent chains keep the
+            // tensor pipe busy.
             int stage = 0;
             uint32_t sphase = 0;
-            int nitem = 0, nacc = 0;
+            int nq = 0, cur_q = -1, ng = 0;
+            uint64_t bdesc = 0;
             bool ok = true;
             for (int ii = 0; ii < n_my && ok; ii++) {
                 Item x;
-                if (!fetch_item(a, items, ii, x, false)) continue;
-                const int bb = nitem & 1;
-                if (!mbar_wait(&bfull[bb], (nitem >> 1) & 1, abort_flag, a.st)) break;
-                tc_fence_after();
-                const uint64_t bdesc = smem_desc_k_sw128(sB + bb * kQBytes);
-                for (int tt = 0; tt < x.ntiles; tt++) {
-                    const int ab = nacc & 1;
-                    if (!mbar_wait(&accempty[ab], ((nacc >> 1) & 1) ^ 1, abort_flag, a.st) ||
+                if (!fetch_item(a, items, v0, v1, ii, x, false)) continue;
+                if (x.q != cur_q) {
+                    // the previous query's heads are free once the MMAs issued so far finish
+                    if (nq > 0) mma_commit(&bempty[(nq - 1) & 1]);
+                    const int bb = nq & 1;
+                    if (!mbar_wait(&bfull[bb], (nq >> 1) & 1, abort_flag, a.st)) break;
+                    tc_fence_after();
+                    bdesc = smem_desc_k_sw128(sB + bb * kQBytes);
+                    nq++;
+                    cur_q = x.q;
+                }
+                for (int g0 = 0; g0 < x.ntiles; g0 += kGroupTiles) {
+                    const int gt = min(kGroupTiles, x.ntiles - g0);
+                    const int set = ng & (kAccSets - 1);
+                    if (!mbar_wait(&accempty[set], ((ng / kAccSets) & 1) ^ 1, abort_flag, a.st) ||
                         !mbar_wait(&full[stage], sphase, abort_flag, a.st)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t adesc = smem_desc_k_sw128(sA + stage * kTileBytes);
-                    const uint32_t d = tmem_base + (uint32_t)(ab * HI);
+                    const uint64_t adesc = smem_desc_k_sw128(sA + stage * kGroupBytes);
+                    const uint32_t d0 = tmem_base + (uint32_t)(set * kGroupTiles * HI);
 #pragma unroll
-                    for (int kk = 0; kk < kDI / 32; kk++)   // K = 32 e4m3 = 32 bytes per MMA
-                        mma_f8f6f4(d, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kDI / 32; kk++) {   // K = 32 e4m3 = 32 bytes per MMA
+#pragma unroll
+                        for (int j = 0; j < kGroupTiles; j++)
+                            if (j < gt)
+                                mma_f8f6f4(d0 + (uint32_t)(j * HI),
+                                           adesc + (uint64_t)((j * kTileBytes) >> 4) + 2 * kk,
+                                           bdesc + 2 * kk, kIdesc, kk > 0 ? 1u : 0u);
+                    }
                     mma_commit(&empty[stage]);
-                    mma_commit(&accfull[ab]);
-                    nacc++;
+                    mma_commit(&accfull[set]);
+                    ng++;
                     if (++stage == kStages) {
                         stage = 0;
                         sphase ^= 1;
                     }
                 }
-                if (ok) mma_commit(&bempty[bb]);
-                nitem++;
             }
             // drain: all issued MMAs complete before TMEM is released
             mma_commit(drain);
             mbar_drain(drain, 0, a.st);
         }
+    } else if (warp == 2) {
+        // ---------------- item prefetch ----------------
+        int nit = 0;
+        for (int ii = 0; ii < n_my; ii++) {
+            Item x;
+            if (!fetch_item(a, items, v0, v1, ii, x, lane == 0)) continue;
+            const int slot = nit % kAux;
+            if (!mbar_wait_warp(&auxempty[slot], ((nit / kAux) & 1) ^ 1, abort_flag, a.st)) break;
+            float* ws_s = aux + slot * kAuxFloats;
+            float* ks_s = ws_s + HI;
+#pragma unroll
+            for (int h = lane; h < HI; h += 32)
+                ws_s[h] = __ldg(a.w + (int64_t)x.q * HI + h) * __ldg(a.qs + (int64_t)x.q * HI + h);
+            // all of the item's key scales in flight at once (one memory latency per item)
+            const int64_t e0 = (int64_t)x.tile0 * kTileRows;
+            const int nrows = x.ntiles * kTileRows;
+            float v[kChunkTiles * kTileRows / 32];
+#pragma unroll
+            for (int k = 0; k < kChunkTiles * kTileRows / 32; k++) {
+                const int j = lane + 32 * k;
+                v[k] = (j < nrows && e0 + j < x.n_vis) ? __ldg(a.ks + x.row0 + e0 + j) : 0.f;
+            }
+#pragma unroll
+            for (int k = 0; k < kChunkTiles * kTileRows / 32; k++)
+                if (lane + 32 * k < nrows) ks_s[lane + 32 * k] = v[k];
+            mbar_arrive(&auxfull[slot]);
+            nit++;
+        }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
-        const int quarter = warp & 3;               // TMEM lanes this warp may access
+        // ---------------- epilogue (warps 3..10) ----------------
+        const int grp = (warp - kFirstEpiWarp) / 4;   // takes the group's tiles j % 2 == grp
+        const int quarter = warp & 3;                 // TMEM lanes this warp may access
         const int row_in_tile = quarter * 32 + lane;
-        int nacc = 0;
+        int ng = 0, nit = 0;
         bool ok = true;
         for (int ii = 0; ii < n_my && ok; ii++) {
             Item x;
-            if (!fetch_item(a, items, ii, x, threadIdx.x == 64)) continue;
+            if (!fetch_item(a, items, v0, v1, ii, x, false)) continue;
+            const int slot = nit % kAux;
+            if (!mbar_wait_warp(&auxfull[slot], (nit / kAux) & 1, abort_flag, a.st)) break;
+            const float* ws_s = aux + slot * kAuxFloats;
+            const float* ks_s = ws_s + HI;
             float ws[HI];
 #pragma unroll
-            for (int h = 0; h < HI; h++)
-                ws[h] = __ldg(a.w + (int64_t)x.q * HI + h) * __ldg(a.qs + (int64_t)x.q * HI + h);
-            float* srow = a.scores + (int64_t)x.q * a.ld;
-            // all key scales of the item at once: one load latency per item, not per tile
-            float kscales[kChunkTiles];
-#pragma unroll
-            for (int tt = 0; tt < kChunkTiles; tt++) {
-                const int e = (x.tile0 + tt) * kTileRows + row_in_tile;
-                kscales[tt] = (tt < x.ntiles && e < x.n_vis) ? __ldg(a.ks + x.row0 + e) : 0.f;
+            for (int h = 0; h < HI; h += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(ws_s + h);
+                ws[h] = v4.x;
+                ws[h + 1] = v4.y;
+                ws[h + 2] = v4.z;
+                ws[h + 3] = v4.w;
             }
-#pragma unroll
-            for (int tt = 0; tt < kChunkTiles; tt++) {
-                if (tt >= x.ntiles) break;
-                const int e = (x.tile0 + tt) * kTileRows + row_in_tile;
-                const bool live = e < x.n_vis;
-                const float kscale = kscales[tt];
-                const int ab = nacc & 1;
-                if (!mbar_wait_warp(&accfull[ab], (nacc >> 1) & 1, abort_flag, a.st)) {
+            float* srow = a.scores + (int64_t)x.q * a.ld;
+            for (int g0 = 0; g0 < x.ntiles; g0 += kGroupTiles) {
+                const int gt = min(kGroupTiles, x.ntiles - g0);
+                const int set = ng & (kAccSets - 1);
+                if (!mbar_wait_warp(&accfull[set], (ng / kAccSets) & 1, abort_flag, a.st)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                uint32_t d[HI];
-                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(ab * HI);
-                if constexpr (HI == 64) {
-                    tmem_ld64(taddr, d);
-                } else if constexpr (HI == 32) {
-                    tmem_ld32(taddr, d);
-                } else {
-                    tmem_ld16(taddr, d);
+                for (int j = grp; j < gt; j += 2) {
+                    const int tt = g0 + j;
+                    const int e = (x.tile0 + tt) * kTileRows + row_in_tile;
+                    uint32_t d[HI];
+                    const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                           (uint32_t)((set * kGroupTiles + j) * HI);
+                    if constexpr (HI == 64) {
+                        tmem_ld64(taddr, d);
+                    } else if constexpr (HI == 32) {
+                        tmem_ld32(taddr, d);
+                    } else {
+                        tmem_ld16(taddr, d);
+                    }
+                    tmem_ld_wait();
+                    if (e < x.n_vis) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int h = 0; h < HI; h++)
+                            acc = fmaf(ws[h], fmaxf(__uint_as_float(d[h]), 0.f), acc);
+                        const float sc = acc * ks_s[tt * kTileRows + row_in_tile];
+                        if (sc != sc) flag(a.st, CSA_DEV_NAN);
+                        srow[e] = sc;
+                    }
                 }
-                tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[ab]);
-                nacc++;
-                if (live) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int h = 0; h < HI; h++) acc = fmaf(ws[h], fmaxf(__uint_as_float(d[h]), 0.f), acc);
-                    const float s = acc * kscale;
-                    if (s != s) flag(a.st, CSA_DEV_NAN);
-                    srow[e] = s;
-                }
+                if (lane == 0) mbar_arrive(&accempty[set]);
+                ng++;
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&auxempty[slot]);
+            nit++;
         }
     }
 
@@ -309,14 +432,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, 2 * HI < 32 ? 32 : 2 * HI);
+        tmem_dealloc(tmem_base, tmem_cols<HI>());
     }
 }
 
 template <int HI>
 size_t smem_bytes() {
-    return 1024 + kStages * kTileBytes + 2 * HI * kDI + (2 * kStages + 9) * 8 + 16 +
-           kMaxItems * sizeof(Item);
+    return 1024 + kStages * kGroupBytes + 2 * HI * kDI + kAux * aux_floats<HI>() * sizeof(float) +
+           (2 * kStages + 4 + 2 * kAccSets + 2 * kAux + 1) * 8 + 16 + kMaxItems * sizeof(Item);
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -374,7 +497,8 @@ cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const IdxArgs& args,
     cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<HI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    const int grid = min(args.total_items, 2 * num_sms());
+    const int64_t tiles = (int64_t)args.Q * args.qtiles;
+    const int grid = (int)(tiles < (int64_t)num_sms() ? tiles : (int64_t)num_sms());
     LaunchScope scope(kKIndexerTc, stream);
     return launch_pdl(indexer_tc_kernel<HI>, dim3(grid), dim3(kThreads), sm, stream, mk, mq, args);
 }
@@ -408,8 +532,8 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
     args.B = B;
     args.m = m;
     args.max_n = max_n;
-    args.chunks_per_q = (max_n + kChunkTiles * kTileRows - 1) / (kChunkTiles * kTileRows);
-    args.total_items = Q * args.chunks_per_q;
+    args.qtiles = (max_n + kTileRows - 1) / kTileRows;
+    args.chunks_per_q = (args.qtiles + kChunkTiles - 1) / kChunkTiles;
     switch (HI) {
         case 64: return launch_hi<64>(qI, kI, args, stream);
         case 32: return launch_hi<32>(qI, kI, args, stream);

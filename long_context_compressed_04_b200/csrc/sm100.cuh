@@ -37,7 +37,8 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// True when the phase of the given parity has completed.
+// True when the phase of the given parity has completed; a thread whose phase is not complete
+// may be suspended for a short, system-dependent time first.
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -50,6 +51,38 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking: true when the phase of the given parity has completed (never suspends).
+__device__ __forceinline__ bool mbar_ready(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// As mbar_test, but a thread whose phase is not complete is suspended in hardware until it
+// completes or about `hint_ns` nanoseconds pass, instead of returning at once: waiting
+// roles then take no issue slots from the ones doing work.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Suspend limit of one try_wait inside the bounded waits (the abort flag and the clock are
+// checked between them).
+constexpr uint32_t kSleepHintNs = 20000;
+
 // Bounded wait.  Returns false when the CTA has been aborted by another role or this wait
 // ran out of time (then it aborts the CTA and flags CSA_DEV_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -57,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_test(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_test(bar, parity)) return true;
+        if (mbar_test_sleep(bar, parity, kSleepHintNs)) return true;
         if (*abort_flag) return false;
         if (clock64() - t0 > kWaitLimitCycles) {
             *abort_flag = 1;
@@ -71,7 +104,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // copies and MMAs before it releases shared memory and tensor memory.
 __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, int32_t* dev_status) {
     const long long t0 = clock64();
-    while (!mbar_test(bar, parity)) {
+    while (!mbar_test_sleep(bar, parity, kSleepHintNs)) {
         if (clock64() - t0 > kWaitLimitCycles) {
             flag(dev_status, CSA_DEV_TIMEOUT);
             return false;
@@ -114,6 +147,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
         "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+// TMA gather of 4 rows (row coordinates r0..r3, each may be out of range -> zero fill) of a
+// 2D tensor map whose box is one row high; the rows land consecutively at dst.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t r0, int32_t r1, int32_t r2,
+                                            int32_t r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(r0), "r"(r1),
+        "r"(r2), "r"(r3)
         : "memory");
 }
 
