@@ -6,11 +6,15 @@
 // The keys of a query form a list of 128-key tiles: tile 0 is the window (its raw rows
 // RMSNormed and RoPEd here, one row per thread), tiles 1.. are the selected entries
 // (sparse, gathered by index) or all visible entries (dense, contiguous).  A work item is
-// (query, chunk of tiles).  Sparse attention uses one chunk per query and finishes in
-// this kernel.  Dense attention splits every query into fixed 8-tile chunks whose fp32
-// partial states (running max, sum, unnormalised output) a second kernel combines in
-// chunk order.  The split depends only on the query's own length, never on the batch, so
-// both paths are batch-invariant.
+// (query, chunk of tiles); a chunk ends as an fp32 partial softmax state (running max, sum,
+// unnormalised output) per head.  Sparse attention runs one thread-block cluster per query:
+// rank 0 takes the window tile, ranks 1.. split the selected-entry tiles; each rank then
+// stores its partial state of every head straight into the shared memory of the rank that
+// finishes that head (posted distributed-shared-memory stores), and each rank combines its
+// slice of the heads locally (ranks in order, the sink first).  Dense attention splits every
+// query into fixed 8-tile chunks whose partial states a second kernel combines in chunk
+// order.  Both splits depend only on k or on the query's own length, never on the batch,
+// so both paths are batch-invariant.
 //
 // Roles per CTA (8 warps, persistent over items):
 //   warp 0      producer: dense tiles by two 2D TMA loads (64 channels x 128 rows each,
@@ -23,9 +27,9 @@
 //               halves (channels 0-63 / 64-127), V being the key tile read MN-major.
 //   warps 4-7   per item: q heads RoPEd at t into shared memory and the window tile; per
 //               tile: S from TMEM (thread = one head x 64 keys), online softmax in the
-//               log2 domain with the sink as the initial state, P as bf16 into shared
-//               memory, then O += corr * O_tile kept in registers (thread = one head x 64
-//               channels); finally normalise, inverse RoPE, store (or write the partial).
+//               log2 domain, P as bf16 into shared memory, then O += corr * O_tile kept in
+//               registers (thread = one head x 64 channels); finally the partial state,
+//               combined across the cluster (sparse) or written for the combine kernel.
 // All waits are bounded (timeout -> CSA_DEV_TIMEOUT, drain, free TMEM, return).
 #include <cstring>
 #include <mutex>
@@ -48,6 +52,16 @@ constexpr int kPBlk = kH * 128;              // one 64-key slice of P (8 KB)
 constexpr int kThreads = 256;
 constexpr int kDenseChunkTiles = 8;
 constexpr int kMaxK = 2048;
+constexpr int kMaxCluster = 8;
+// sparse receive buffer: C ranks x ceil(kH / C) heads x (kD + 2) floats, largest over C
+constexpr int recv_floats(int C) {
+    return C > kMaxCluster ? 0
+                           : (C * ((kH + C - 1) / C) * (kD + 2) > recv_floats(C + 1)
+                                  ? C * ((kH + C - 1) / C) * (kD + 2)
+                                  : recv_floats(C + 1));
+}
+constexpr int kRecvFloats = recv_floats(2);
+constexpr int kWtabFloats = ((kH + 1) / 2) * (kMaxCluster + 1);
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnTcArgs {
@@ -67,6 +81,7 @@ struct AttnTcArgs {
     int32_t* st;
     int64_t ent_rows;
     int k, m, B, W, Q, chunk_tiles, chunks_per_q, total_items, max_n;
+    int cluster;          // sparse: CTAs per query (one cluster); dense: 1
     float scale_log2;
     float eps;
     double log2_theta;
@@ -78,8 +93,6 @@ struct AItem {
     int n_ent;      // entries in the key list (k for sparse, n_vis for dense)
     int w0, n_win;
     int tile0, ntiles;
-    bool single;    // sparse: the whole query in this item, finish here (dense never: its
-                    // chunk partials always go through the ordered combine, whatever the batch)
     int64_t row0;
 };
 
@@ -111,10 +124,23 @@ __device__ __forceinline__ bool get_item(const AttnTcArgs& a, int it, AItem& x, 
     }
     x.w0 = x.t - a.W + 1 > 0 ? x.t - a.W + 1 : 0;
     x.n_win = a.W > 0 ? x.t - x.w0 + 1 : 0;
-    const int total = 1 + (x.n_ent + kTK - 1) / kTK;
+    const int n_et = (x.n_ent + kTK - 1) / kTK;   // entry tiles
+    if (a.idx) {
+        // sparse: rank 0 of the query's cluster takes the window tile, ranks 1..C-1 split
+        // the entry tiles contiguously (the host picks C - 1 <= n_et: every rank has one)
+        const int C = a.cluster;
+        if (x.c == 0) {
+            x.tile0 = 0;
+            x.ntiles = 1;
+        } else {
+            const int lo = 1 + (x.c - 1) * n_et / (C - 1), hi = 1 + x.c * n_et / (C - 1);
+            x.tile0 = lo;
+            x.ntiles = hi - lo;
+        }
+        return x.ntiles > 0;
+    }
     x.tile0 = x.c * a.chunk_tiles;
-    x.ntiles = min(a.chunk_tiles, total - x.tile0);
-    x.single = a.idx != nullptr;
+    x.ntiles = min(a.chunk_tiles, 1 + n_et - x.tile0);
     return x.ntiles > 0;
 }
 
@@ -163,7 +189,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* rws = rwc + 32;
     int32_t* sidx = reinterpret_cast<int32_t*>(rws + 32);   // [kMaxK] the item's index row
     int32_t* srows = sidx + kMaxK;                          // [kStages][128] gather rows
-    uint64_t* bars = reinterpret_cast<uint64_t*>(srows + kStages * kTK);
+    // sparse: receive buffer of the partial states of this rank's heads from every rank,
+    // [cluster][nh][kD] O then [cluster][2][nh] m, l (nh = heads per rank); then the
+    // per-head combine weights [nh][cluster + 1]
+    float* recv = reinterpret_cast<float*>(srows + kStages * kTK);
+    float* wtab = recv + kRecvFloats;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(wtab + kWtabFloats);
     uint64_t* full = bars;                 // [kStages]  33 arrivals (+tx)
     uint64_t* empty = full + kStages;      // [kStages]  MMA commit
     uint64_t* prep_full = empty + kStages; // Q + window ready: 4 arrivals
@@ -174,7 +205,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* p_empty = p_full + 2;        // [2]
     uint64_t* pv_full = p_empty + 2;       // [2]
     uint64_t* pv_empty = pv_full + 2;      // [2] 4 arrivals
-    uint64_t* drain = pv_empty + 2;
+    uint64_t* cpart_full = pv_empty + 2;  // every rank's partials are in: 4 x cluster
+    uint64_t* cpart_free = cpart_full + 1; // every rank has combined the previous query (its
+                                           // receive buffer is free again): 4 x cluster
+    uint64_t* drain = cpart_free + 1;
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
@@ -194,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&pv_full[i], 1);
             mbar_init(&pv_empty[i], 4);
         }
+        mbar_init(cpart_full, 4 * a.cluster);
+        mbar_init(cpart_free, 4 * a.cluster);
         mbar_init(drain, 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -205,6 +241,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc_fence_before();
     __syncthreads();
+    // the cluster's barriers are initialised before any rank arrives on another's
+    if (a.cluster > 1) cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
     const uint32_t tmem_S = tmem_base;          // [2] x 64 columns
@@ -223,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
             AItem x;
             if (!get_item(a, it, x, false)) continue;
-            if (a.idx) {
+            if (a.idx && x.tile0 + x.ntiles > 1) {
                 // the query's whole index row, once per item: batches of 8 x 16-byte loads
                 // per lane in flight (one round trip for k <= 1024); only this warp reads it
                 const int32_t* src = a.idx + (int64_t)x.q * a.k;
@@ -368,11 +406,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
+                    // the two key halves are independent accumulators: interleave their chains
 #pragma unroll
-                    for (int half = 0; half < 2; half++) {
-                        const uint32_t d = tmem_S + sb * 64 + ((uint32_t)(half * 16) << 16);
+                    for (int kk = 0; kk < 8; kk++) {
 #pragma unroll
-                        for (int kk = 0; kk < 8; kk++) {
+                        for (int half = 0; half < 2; half++) {
+                            const uint32_t d = tmem_S + sb * 64 + ((uint32_t)(half * 16) << 16);
                             const int blk = kk >> 2;
                             const uint32_t off = (uint32_t)((kk & 3) * 32) >> 4;
                             const uint64_t ad = smem_desc_k_sw128(sQ + blk * kQBlk) + off;
@@ -392,10 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         tc_fence_after();
 #pragma unroll
-                        for (int half = 0; half < 2; half++) {
-                            const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
+                        for (int kk = 0; kk < 8; kk++) {
 #pragma unroll
-                            for (int kk = 0; kk < 8; kk++) {
+                            for (int half = 0; half < 2; half++) {
+                                const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
                                 const uint64_t ad =
                                     smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
                                     ((uint32_t)((kk & 3) * 32) >> 4);
@@ -423,10 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc_fence_after();
 #pragma unroll
-                    for (int half = 0; half < 2; half++) {
-                        const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
+                    for (int kk = 0; kk < 8; kk++) {
 #pragma unroll
-                        for (int kk = 0; kk < 8; kk++) {
+                        for (int half = 0; half < 2; half++) {
+                            const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
                             const uint64_t ad =
                                 smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
                                 ((uint32_t)((kk & 3) * 32) >> 4);
@@ -577,9 +616,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(prep_full);
 
             // ---- running state of head h ----
-            const float sk = a.sink[h] * kLog2e;
-            float mrun = x.single ? sk : -INFINITY;
-            float lrun = (x.single && sk != -INFINITY) ? 1.f : 0.f;
+            // sparse: the sink of head h0 + i of this rank's slice, for the combine
+            float sk_mine = -INFINITY;
+            if (a.idx) {
+                const int h0 = x.c * kH / a.cluster, h1 = (x.c + 1) * kH / a.cluster;
+                if (i < h1 - h0) sk_mine = a.sink[h0 + i] * kLog2e;
+            }
+            // the chunk's own keys only: the sink enters when the partial states are combined
+            float mrun = -INFINITY;
+            float lrun = 0.f;
             float o[64];
 #pragma unroll
             for (int c = 0; c < 64; c++) o[c] = 0.f;
@@ -676,32 +721,94 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 64; c++) o[c] = fmaf(o[c], corr_prev, __uint_as_float(pv[c]));
             }
-            if (!ok) {
-                // skip the rest of this item; the next item's barrier settles the exit
-            } else if (x.single) {
-                const float inv = lrun > 0.f ? 1.f / lrun : 0.f;
+            if (a.idx) {
+                // ---- sparse: exchange partial states across the cluster ----
+                const int C = a.cluster;
+                const int nh = (kH + C - 1) / C;
+                float* recv_ml = recv + C * nh * kD;
+                // every rank's receive buffer is free of the previous query's partials
+                if (ok) ok = mbar_wait_cluster_warp(cpart_free, (nitem & 1) ^ 1, abort_flag, a.st);
+                if (ok) {
+                    // head h is finished by rank `own` (heads [own*kH/C, (own+1)*kH/C))
+                    int own = 0;
+                    while (own + 1 < C && (own + 1) * kH / C <= h) own++;
+                    const int lh = h - own * kH / C;
+                    const uint32_t dst = mapa(recv + ((x.c * nh + lh) * kD + kh * 64), (uint32_t)own);
 #pragma unroll
-                for (int c = 0; c < 64; c++) o[c] *= inv;
-                if (kh == 1) {
-#pragma unroll
-                    for (int pj = 0; pj < 32; pj++) {
-                        const float cs = rqc[pj], sn = -rqs[pj];   // rotation by -t
-                        const float x0 = o[2 * pj], y0 = o[2 * pj + 1];
-                        o[2 * pj] = x0 * cs - y0 * sn;
-                        o[2 * pj + 1] = x0 * sn + y0 * cs;
+                    for (int c = 0; c < 64; c += 4)
+                        st_cluster_f4(dst + 4 * c, make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]));
+                    if (kh == 0) {
+                        st_cluster_f32(mapa(recv_ml + (2 * x.c) * nh + lh, (uint32_t)own), mrun);
+                        st_cluster_f32(mapa(recv_ml + (2 * x.c + 1) * nh + lh, (uint32_t)own), lrun);
                     }
+                    fence_cluster();
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int r = 0; r < C; r++) mbar_arrive_cluster(mapa(cpart_full, (uint32_t)r));
+                    ok = mbar_wait_cluster_warp(cpart_full, nitem & 1, abort_flag, a.st);
                 }
-                uint16_t* dst = a.out + ((int64_t)x.q * kH + h) * kD + kh * 64;
-#pragma unroll
-                for (int c = 0; c < 8; c++) {
-                    uint4 u;
-                    u.x = pack_bf16x2(o[8 * c], o[8 * c + 1]);
-                    u.y = pack_bf16x2(o[8 * c + 2], o[8 * c + 3]);
-                    u.z = pack_bf16x2(o[8 * c + 4], o[8 * c + 5]);
-                    u.w = pack_bf16x2(o[8 * c + 6], o[8 * c + 7]);
-                    *reinterpret_cast<uint4*>(dst + 8 * c) = u;
+                if (named_barrier_and(1, 128, ok)) {
+                    // this rank's heads; first the combine weights, one thread per head:
+                    // M = max(sink, m_r), w_r = 2^(m_r - M), L = 2^(sink - M) + sum_r w_r l_r
+                    const int h0 = x.c * kH / C, h1 = (x.c + 1) * kH / C;
+                    if (i < h1 - h0) {
+                        const float sk = sk_mine;
+                        float M = sk;
+                        for (int r = 0; r < C; r++) M = fmaxf(M, recv_ml[(2 * r) * nh + i]);
+                        float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
+                        for (int r = 0; r < C; r++) {
+                            const float mr = recv_ml[(2 * r) * nh + i];
+                            const float w = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
+                            L = fmaf(w, recv_ml[(2 * r + 1) * nh + i], L);
+                            wtab[i * (kMaxCluster + 1) + r] = w;
+                        }
+                        wtab[i * (kMaxCluster + 1) + kMaxCluster] = L;
+                    }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    // then (head, 4 channels) per work unit: sum_r w_r O_r / L, inverse RoPE
+                    // (the pairs sit inside the 4 channels), 4 bf16 stored at once
+                    const int units = (h1 - h0) * (kD / 4);
+#pragma unroll 2
+                    for (int w = i; w < units; w += 128) {
+                        const int lh = w / (kD / 4), c4 = (w % (kD / 4)) * 4;
+                        const float* wt = wtab + lh * (kMaxCluster + 1);
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int r = 0; r < C; r++) {
+                            const float wr = wt[r];
+                            const float4 v = *reinterpret_cast<const float4*>(recv + (r * nh + lh) * kD + c4);
+                            acc.x = fmaf(wr, v.x, acc.x);
+                            acc.y = fmaf(wr, v.y, acc.y);
+                            acc.z = fmaf(wr, v.z, acc.z);
+                            acc.w = fmaf(wr, v.w, acc.w);
+                        }
+                        const float L = wt[kMaxCluster];
+                        if (L > 0.f) {
+                            acc.x /= L;
+                            acc.y /= L;
+                            acc.z /= L;
+                            acc.w /= L;
+                        } else {
+                            acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                        if (c4 >= kD - kRopeDims) {
+                            // rotation by -t: (x, y) -> (x cos + y sin, y cos - x sin)
+                            const int pj = (c4 - (kD - kRopeDims)) >> 1;
+                            const float c0 = rqc[pj], s0 = rqs[pj], c1 = rqc[pj + 1], s1 = rqs[pj + 1];
+                            acc = make_float4(acc.x * c0 + acc.y * s0, acc.y * c0 - acc.x * s0,
+                                              acc.z * c1 + acc.w * s1, acc.w * c1 - acc.z * s1);
+                        }
+                        *reinterpret_cast<uint2*>(a.out + ((int64_t)x.q * kH + h0 + lh) * kD + c4) =
+                            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+                    }
+                    // my receive buffer may take the next query's partials
+                    fence_cluster();
+                    __syncwarp();
+                    if (lane == 0)
+                        for (int r = 0; r < C; r++) mbar_arrive_cluster(mapa(cpart_free, (uint32_t)r));
+                } else {
+                    ok = false;
                 }
-            } else {
+            } else if (ok) {
                 float* pr = a.part + ((int64_t)it * kH + h) * (kD + 2);
                 if (kh == 0) {
                     pr[0] = mrun;
@@ -721,6 +828,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, 256);
     }
+    // no rank leaves while another may still read its shared memory or arrive on it
+    if (a.cluster > 1) cluster_sync_all();
 }
 
 // Dense path: combine the chunk partials of one (query, head) in chunk order, add the
@@ -793,7 +902,42 @@ int sm_count() {
 
 constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + kTileBytes + 2 * kQBlk + 4 * kPBlk +
                               4 * (kStages + 1) * 4 + 5 * 32 * 4 + kMaxK * 4 + kStages * kTK * 4 +
-                              (2 * kStages + 15) * 8 + 16;
+                              (kRecvFloats + kWtabFloats) * 4 + (2 * kStages + 17) * 8 + 16;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+
+// CTAs per query for sparse attention: rank 0 takes the window tile, the others about two
+// selected-entry tiles each.  A function of k alone, so the result is batch-invariant.
+int sparse_cluster(int k) {
+    const int n_et = (k + kTK - 1) / kTK;
+    return min(kMaxCluster, 1 + (n_et + 1) / 2);
+}
+
+// Clusters of `C` CTAs that can be resident at once (0 when unknown).
+int max_active_clusters(int C) {
+    static int cache[kMaxCluster + 1] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[C] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(C * 64);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = sm_count() / C;
+        }
+        cache[C] = n;
+    }
+    return cache[C];
+}
 
 int dense_chunks_per_q(int max_n) {
     const int tiles = 1 + (max_n + kTK - 1) / kTK;
@@ -837,9 +981,11 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
     a.eps = aa.eps;
     a.log2_theta = aa.log2_theta;
     if (aa.idx) {
-        a.chunk_tiles = 1 + (aa.k + kTK - 1) / kTK;
-        a.chunks_per_q = 1;
+        a.cluster = sparse_cluster(aa.k);
+        a.chunk_tiles = 0;   // ranks take their tiles by rank
+        a.chunks_per_q = a.cluster;
     } else {
+        a.cluster = 1;
         a.chunk_tiles = kDenseChunkTiles;
         a.chunks_per_q = dense_chunks_per_q(max_n);
     }
@@ -865,11 +1011,18 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    const int grid = min(a.total_items, sm_count());
     {
         LaunchScope scope(kKAttnTc, stream);
-        e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, map_e,
-                       map_g, a);
+        if (aa.idx) {
+            // one cluster per query at a time; clusters walk the queries persistently
+            const int nclusters = max(1, min(Q, max_active_clusters(a.cluster)));
+            e = launch_pdl_cluster(attn_tc_kernel, dim3(nclusters * a.cluster), dim3(kThreads),
+                                   kSmemBytes, stream, a.cluster, map_e, map_g, a);
+        } else {
+            const int grid = min(a.total_items, sm_count());
+            e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, map_e,
+                           map_g, a);
+        }
     }
     if (e != cudaSuccess || aa.idx) return e;
     LaunchScope scope(kKAttnCombine, stream);
