@@ -8,17 +8,19 @@
 //
 // One CTA (1024 threads) per query, scores mapped to order-preserving 32-bit keys.  The
 // goal is the k-th largest key T and the number of keys equal to T to take.
-//  1. Rows of up to 50K scores are staged in shared memory with 16-byte loads; the OR and
-//     AND of all keys give the bits every key shares, so the radix starts at the highest
-//     bit that varies (scores of one query share sign and most exponent bits, and a fixed
-//     first digit would put nearly all of them in one bin).
+//  1. Rows of up to 44K scores are staged in shared memory as keys (16-byte loads); the OR
+//     and AND of all keys give the bits every key shares, so the radix starts at the
+//     highest bit that varies (scores of one query share sign and most exponent bits, and a
+//     fixed first digit would put nearly all of them in one bin).
 //  2. An 11-bit histogram of that digit (shared-memory atomics) and a block-wide scan over
 //     the bins, from the top, give the bin holding the k-th key.
-//  3. Keys in that bin are compacted to a short candidate list (if it fits), and the
-//     remaining bits are resolved on the list; otherwise further full passes run.
-//  4. A last pass in ascending entry order takes every key > T and the first needed keys
-//     == T; one block-wide scan per 4096-entry chunk gives each thread its output slots,
-//     so the indices come out already sorted.
+//  3. Keys in that bin are compacted to a short candidate list (if it fits; one shared
+//     atomic per warp and key slot), and the remaining bits are resolved on the list;
+//     otherwise further full passes run.
+//  4. Each warp owns a contiguous run of the row.  A counting pass (ballots) gives every
+//     warp its keys > T and == T, one scan over the 32 warps its output offset and tie
+//     rank, and a writing pass in ascending entry order takes every key > T and the first
+//     needed keys == T, so the indices come out already sorted.
 #include "launchers.cuh"
 
 namespace csa {
@@ -86,8 +88,15 @@ struct Shared {
     uint32_t hist[kBins];
     uint32_t scan_tmp[33];
     uint32_t bin, krem, key_or, key_and, ncand;
+    uint32_t wgt[kWarps], weq[kWarps];   // per warp: keys > T, == T; then exclusive prefixes
     uint32_t cand[kMaxCand];
 };
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
 
 // After hist[] holds the counts of the current digit: picks the bin holding the krem-th
 // largest key (bins scanned from the top) and the rank left inside it.
@@ -108,7 +117,7 @@ __device__ __forceinline__ void pick_bin(Shared& sh, uint32_t& krem) {
     krem = sh.krem;
 }
 
-// STAGED: the query's score row is first copied to shared memory (16-byte loads, eight in
+// STAGED: the query's row is first copied to shared memory as keys (16-byte loads, eight in
 // flight per thread) and every pass reads it from there.
 template <bool STAGED>
 __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
@@ -140,9 +149,29 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     }
     __syncthreads();
     uint32_t kor = 0u, kand = 0xFFFFFFFFu;
+    extern __shared__ uint4 skey4[];
+    const uint32_t* skey = reinterpret_cast<const uint32_t*>(skey4);
+    // keys of entries i .. i+3 (0 past n) and of entry i
+    auto get4 = [&](int i, uint32_t* key) {
+        if constexpr (STAGED) {
+            // only the staged part of the row is read (past n the buffer may end)
+            const uint4 v = i < n ? skey4[i >> 2] : make_uint4(0u, 0u, 0u, 0u);
+            key[0] = i < n ? v.x : 0u;
+            key[1] = i + 1 < n ? v.y : 0u;
+            key[2] = i + 2 < n ? v.z : 0u;
+            key[3] = i + 3 < n ? v.w : 0u;
+        } else {
+            load4(s, i, n, vec, key);
+        }
+    };
+    auto get1 = [&](int i) -> uint32_t {
+        if constexpr (STAGED) {
+            return skey[i];
+        } else {
+            return score_key(s[i]);
+        }
+    };
     if constexpr (STAGED) {
-        extern __shared__ float4 srow4[];
-        float* srow = reinterpret_cast<float*>(srow4);
         constexpr int kBatch = 8;
         for (int i0 = 4 * tid; i0 < n; i0 += 4 * kThreads * kBatch) {
             float4 v[kBatch];
@@ -161,20 +190,19 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
 #pragma unroll
             for (int u = 0; u < kBatch; u++) {
                 const int i = i0 + u * 4 * kThreads;
-                if (i < n) *reinterpret_cast<float4*>(srow + i) = v[u];
                 const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                uint32_t kk[4];
 #pragma unroll
                 for (int z = 0; z < 4; z++) {
+                    kk[z] = score_key(e[z]);
                     if (i + z < n) {
-                        const uint32_t key = score_key(e[z]);
-                        kor |= key;
-                        kand &= key;
+                        kor |= kk[z];
+                        kand &= kk[z];
                     }
                 }
+                if (i < n) skey4[i >> 2] = make_uint4(kk[0], kk[1], kk[2], kk[3]);
             }
         }
-        s = srow;
-        vec = true;
     } else {
         for (int c0 = 0; c0 < n; c0 += kChunk) {
             uint32_t key[4];
@@ -214,7 +242,7 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         if (!compacted) {
             for (int c0 = 0; c0 < n; c0 += kChunk) {
                 uint32_t key[4];
-                load4(s, c0 + 4 * tid, n, vec, key);
+                get4(c0 + 4 * tid, key);
 #pragma unroll
                 for (int u = 0; u < 4; u++)
                     if (c0 + 4 * tid + u < n && (key[u] & mask) == prefix)
@@ -235,55 +263,83 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         top = shift - 1;
         __syncthreads();
         if (!compacted && top >= 0 && in_bin <= (uint32_t)kMaxCand) {
-            // keys in the chosen bin become the candidate list for the remaining bits
+            // keys in the chosen bin become the candidate list for the remaining bits (one
+            // shared atomic per warp and key slot)
             for (int c0 = 0; c0 < n; c0 += kChunk) {
                 uint32_t key[4];
-                load4(s, c0 + 4 * tid, n, vec, key);
+                get4(c0 + 4 * tid, key);
 #pragma unroll
-                for (int u = 0; u < 4; u++)
-                    if (c0 + 4 * tid + u < n && (key[u] & mask) == prefix)
-                        sh.cand[atomicAdd(&sh.ncand, 1u)] = key[u];
+                for (int u = 0; u < 4; u++) {
+                    const bool p = c0 + 4 * tid + u < n && (key[u] & mask) == prefix;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, p);
+                    uint32_t slot = 0;
+                    if (lane == 0 && bal) slot = atomicAdd(&sh.ncand, (uint32_t)__popc(bal));
+                    slot = __shfl_sync(0xffffffffu, slot, 0);
+                    if (p) sh.cand[slot + __popc(bal & lanemask_lt())] = key[u];
+                }
             }
             compacted = true;
             __syncthreads();
         }
     }
     const uint32_t T = prefix;   // the k-th largest key; krem keys equal to T are taken
-    // ordered collection: 4096 entries per round, 4 consecutive per thread
-    uint32_t written = 0, ties_before = 0;
-    for (int c0 = 0; c0 < n; c0 += kChunk) {
-        const int i0 = c0 + 4 * tid;
-        uint32_t key[4];
-        load4(s, i0, n, vec, key);
-        uint32_t ngt = 0, neq = 0;
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const bool in = i0 + u < n;
-            ngt += (in && key[u] > T) ? 1u : 0u;
-            neq += (in && key[u] == T) ? 1u : 0u;
+    // warp w owns rounds [w * rpw, (w + 1) * rpw) of 32 consecutive entries
+    const int wid = tid >> 5;
+    const int rounds = (n + 31) >> 5;
+    const int rpw = (rounds + kWarps - 1) / kWarps;
+    const int r0 = min(wid * rpw, rounds), r1 = min(r0 + rpw, rounds);
+    {
+        uint32_t gtc = 0, eqc = 0;
+        for (int r = r0; r < r1; r++) {
+            const int i = (r << 5) + lane;
+            const bool in = i < n;
+            const uint32_t key = in ? get1(i) : 0u;
+            gtc += __popc(__ballot_sync(0xffffffffu, in && key > T));
+            eqc += __popc(__ballot_sync(0xffffffffu, in && key == T));
         }
-        uint32_t tot;
-        const uint32_t packed = block_exclusive_scan(ngt | (neq << 16), sh.scan_tmp, tot);
-        uint32_t eq_rank = ties_before + (packed >> 16);   // tie rank of my first tie
-        uint32_t pos = written + (packed & 0xFFFFu) + (min(eq_rank, krem) - min(ties_before, krem));
-#pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const bool in = i0 + u < n;
-            bool take = in && key[u] > T;
-            if (in && key[u] == T) {
-                take = eq_rank < krem;
-                eq_rank++;
-            }
-            if (take) {
-                if (pos < (uint32_t)k) out[pos] = i0 + u;
-                pos++;
-            }
+        if (lane == 0) {
+            sh.wgt[wid] = gtc;
+            sh.weq[wid] = eqc;
         }
-        const uint32_t ties_after = ties_before + (tot >> 16);
-        written += (tot & 0xFFFFu) + (min(ties_after, krem) - min(ties_before, krem));
-        ties_before = ties_after;
     }
-    if (tid == 0 && written != (uint32_t)k) flag(dev_status, CSA_DEV_NAN);
+    __syncthreads();
+    if (wid == 0) {
+        const uint32_t g = sh.wgt[lane], e = sh.weq[lane];
+        uint32_t gi = g, ei = e;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t yg = __shfl_up_sync(0xffffffffu, gi, o);
+            const uint32_t ye = __shfl_up_sync(0xffffffffu, ei, o);
+            if (lane >= o) {
+                gi += yg;
+                ei += ye;
+            }
+        }
+        __syncwarp();
+        sh.wgt[lane] = gi - g;
+        sh.weq[lane] = ei - e;
+    }
+    __syncthreads();
+    // in entry order: every key > T, and the ties whose rank among all ties is < krem
+    uint32_t ties = sh.weq[wid];
+    uint32_t pos = sh.wgt[wid] + min(ties, krem);
+    const uint32_t lt = lanemask_lt();
+    for (int r = r0; r < r1; r++) {
+        const int i = (r << 5) + lane;
+        const bool in = i < n;
+        const uint32_t key = in ? get1(i) : 0u;
+        const uint32_t eq = __ballot_sync(0xffffffffu, in && key == T);
+        const bool take = (in && key > T) || (in && key == T && ties + __popc(eq & lt) < krem);
+        const uint32_t tk = __ballot_sync(0xffffffffu, take);
+        if (take) {
+            const uint32_t p = pos + __popc(tk & lt);
+            if (p < (uint32_t)k) out[p] = i;
+        }
+        pos += __popc(tk);
+        ties += __popc(eq);
+    }
+    // every warp ends at the row's total; NaN scores (no total order) break it
+    if (wid == kWarps - 1 && lane == 0 && pos != (uint32_t)k) flag(dev_status, CSA_DEV_NAN);
 }
 
 }  // namespace
@@ -292,8 +348,8 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream) {
     if (Q == 0) return cudaSuccess;
-    // rows of up to ~44K scores are staged in shared memory (with the ~25 KB of histogram
-    // and candidate space this stays under the 227 KB per-CTA limit)
+    // rows of up to ~44K scores are staged in shared memory as keys (with the ~25 KB of
+    // histogram and candidate space this stays under the 227 KB per-CTA limit)
     const size_t row_bytes = (size_t)((max_n + 3) / 4) * 16;
     cudaError_t e;
     if (row_bytes <= (size_t)176 * 1024) {
