@@ -17,10 +17,10 @@
 //  3. Keys in that bin are compacted to a short candidate list (if it fits; one shared
 //     atomic per warp and key slot), and the remaining bits are resolved on the list;
 //     otherwise further full passes run.
-//  4. Each warp owns a contiguous run of the row.  A counting pass (ballots) gives every
-//     warp its keys > T and == T, one scan over the 32 warps its output offset and tie
-//     rank, and a writing pass in ascending entry order takes every key > T and the first
-//     needed keys == T, so the indices come out already sorted.
+//  4. A marking pass stores, per 32 consecutive entries, the ballot words of keys > T and
+//     keys == T.  One block-wide scan over the words gives each its output offset and tie
+//     rank; every key > T and the first needed keys == T are written from the words' bits
+//     in ascending entry order, so the indices come out already sorted.
 #include "launchers.cuh"
 
 namespace csa {
@@ -87,10 +87,42 @@ __device__ __forceinline__ void load4(const float* s, int i, int n, bool vec, ui
 struct Shared {
     uint32_t hist[kBins];
     uint32_t scan_tmp[33];
+    unsigned long long scan64[33];
     uint32_t bin, krem, key_or, key_and, ncand;
-    uint32_t wgt[kWarps], weq[kWarps];   // per warp: keys > T, == T; then exclusive prefixes
     uint32_t cand[kMaxCand];
 };
+
+// Exclusive prefix sum over the CTA of a 64-bit `v`; `total` gets the CTA sum.
+__device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long v,
+                                                                     unsigned long long* tmp,
+                                                                     unsigned long long& total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    unsigned long long x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) tmp[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        const unsigned long long wv = lane < kWarps ? tmp[lane] : 0ull;
+        unsigned long long inc = wv;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        __syncwarp();
+        tmp[lane] = inc - wv;
+        if (lane == 31) tmp[32] = inc;
+    }
+    __syncthreads();
+    const unsigned long long res = x - v + tmp[wid];
+    total = tmp[32];
+    __syncthreads();
+    return res;
+}
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
@@ -149,7 +181,12 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     }
     __syncthreads();
     uint32_t kor = 0u, kand = 0xFFFFFFFFu;
-    extern __shared__ uint4 skey4[];
+    // dynamic shared memory: the selection words (2 per 32 entries), then the staged keys
+    extern __shared__ uint4 dyn4[];
+    const int nwords = (n + 31) >> 5;
+    uint32_t* selw = reinterpret_cast<uint32_t*>(dyn4);
+    uint32_t* tiew = selw + ((max_n + 31) >> 5);
+    uint4* skey4 = dyn4 + ((2 * ((max_n + 31) >> 5) + 3) >> 2);
     const uint32_t* skey = reinterpret_cast<const uint32_t*>(skey4);
     // keys of entries i .. i+3 (0 past n) and of entry i
     auto get4 = [&](int i, uint32_t* key) {
@@ -283,63 +320,53 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         }
     }
     const uint32_t T = prefix;   // the k-th largest key; krem keys equal to T are taken
-    // warp w owns rounds [w * rpw, (w + 1) * rpw) of 32 consecutive entries
+    // marking: word r holds the entries 32 r .. 32 r + 31 (bit = lane)
     const int wid = tid >> 5;
-    const int rounds = (n + 31) >> 5;
-    const int rpw = (rounds + kWarps - 1) / kWarps;
-    const int r0 = min(wid * rpw, rounds), r1 = min(r0 + rpw, rounds);
-    {
-        uint32_t gtc = 0, eqc = 0;
-        for (int r = r0; r < r1; r++) {
-            const int i = (r << 5) + lane;
-            const bool in = i < n;
-            const uint32_t key = in ? get1(i) : 0u;
-            gtc += __popc(__ballot_sync(0xffffffffu, in && key > T));
-            eqc += __popc(__ballot_sync(0xffffffffu, in && key == T));
-        }
-        if (lane == 0) {
-            sh.wgt[wid] = gtc;
-            sh.weq[wid] = eqc;
-        }
-    }
-    __syncthreads();
-    if (wid == 0) {
-        const uint32_t g = sh.wgt[lane], e = sh.weq[lane];
-        uint32_t gi = g, ei = e;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t yg = __shfl_up_sync(0xffffffffu, gi, o);
-            const uint32_t ye = __shfl_up_sync(0xffffffffu, ei, o);
-            if (lane >= o) {
-                gi += yg;
-                ei += ye;
-            }
-        }
-        __syncwarp();
-        sh.wgt[lane] = gi - g;
-        sh.weq[lane] = ei - e;
-    }
-    __syncthreads();
-    // in entry order: every key > T, and the ties whose rank among all ties is < krem
-    uint32_t ties = sh.weq[wid];
-    uint32_t pos = sh.wgt[wid] + min(ties, krem);
-    const uint32_t lt = lanemask_lt();
-    for (int r = r0; r < r1; r++) {
+    for (int r = wid; r < nwords; r += kWarps) {
         const int i = (r << 5) + lane;
         const bool in = i < n;
         const uint32_t key = in ? get1(i) : 0u;
+        const uint32_t gt = __ballot_sync(0xffffffffu, in && key > T);
         const uint32_t eq = __ballot_sync(0xffffffffu, in && key == T);
-        const bool take = (in && key > T) || (in && key == T && ties + __popc(eq & lt) < krem);
-        const uint32_t tk = __ballot_sync(0xffffffffu, take);
-        if (take) {
-            const uint32_t p = pos + __popc(tk & lt);
-            if (p < (uint32_t)k) out[p] = i;
+        if (lane == 0) {
+            selw[r] = gt;
+            tiew[r] = eq;
         }
-        pos += __popc(tk);
-        ties += __popc(eq);
     }
-    // every warp ends at the row's total; NaN scores (no total order) break it
-    if (wid == kWarps - 1 && lane == 0 && pos != (uint32_t)k) flag(dev_status, CSA_DEV_NAN);
+    __syncthreads();
+    // each thread a run of words: counts, one 64-bit scan (ties high, keys > T low), write
+    const int wpt = (nwords + kThreads - 1) / kThreads;
+    const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
+    uint32_t cg = 0, ce = 0;
+    for (int w = w0; w < w1; w++) {
+        cg += __popc(selw[w]);
+        ce += __popc(tiew[w]);
+    }
+    unsigned long long tot;
+    const unsigned long long pre =
+        block_exclusive_scan64(((unsigned long long)ce << 32) | cg, sh.scan64, tot);
+    uint32_t ties = (uint32_t)(pre >> 32);
+    uint32_t pos = (uint32_t)pre + min(ties, krem);
+    for (int w = w0; w < w1; w++) {
+        uint32_t take = selw[w];
+        uint32_t tw = tiew[w];
+        // the lowest-index ties while the budget lasts
+        while (tw && ties < krem) {
+            take |= tw & (0u - tw);
+            tw &= tw - 1;
+            ties++;
+        }
+        ties += __popc(tw);
+        while (take) {
+            const int bit = __ffs(take) - 1;
+            if (pos < (uint32_t)k) out[pos] = (w << 5) + bit;
+            pos++;
+            take &= take - 1;
+        }
+    }
+    // the row's total; NaN scores (no total order) break it
+    if (tid == 0 && (uint32_t)tot + min((uint32_t)(tot >> 32), krem) != (uint32_t)k)
+        flag(dev_status, CSA_DEV_NAN);
 }
 
 }  // namespace
@@ -351,20 +378,16 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
     // rows of up to ~44K scores are staged in shared memory as keys (with the ~25 KB of
     // histogram and candidate space this stays under the 227 KB per-CTA limit)
     const size_t row_bytes = (size_t)((max_n + 3) / 4) * 16;
-    cudaError_t e;
-    if (row_bytes <= (size_t)176 * 1024) {
-        e = cudaFuncSetAttribute(topk_radix_kernel<true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)row_bytes);
-        if (e != cudaSuccess) return e;
-        LaunchScope scope(kKTopk, stream);
-        return launch_pdl(topk_radix_kernel<true>, dim3(Q), dim3(kThreads), row_bytes, stream,
-                          scores, ld, q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st);
-    } else {
-        LaunchScope scope(kKTopk, stream);
-        return launch_pdl(topk_radix_kernel<false>, dim3(Q), dim3(kThreads), 0, stream, scores, ld,
-                          q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st);
-    }
-    return cudaGetLastError();
+    const size_t word_bytes = (size_t)((2 * ((max_n + 31) / 32) + 3) / 4) * 16;
+    const bool staged = word_bytes + row_bytes <= (size_t)176 * 1024;
+    const size_t smem = word_bytes + (staged ? row_bytes : 0);
+    auto kernel = staged ? topk_radix_kernel<true> : topk_radix_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    LaunchScope scope(kKTopk, stream);
+    return launch_pdl(kernel, dim3(Q), dim3(kThreads), smem, stream, scores, ld, q_seq, q_pos,
+                      seq_len, B, m, max_n, k, idx_out, st);
 }
 
 }  // namespace csa
