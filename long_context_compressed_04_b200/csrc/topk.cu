@@ -21,7 +21,16 @@
 //     keys == T.  One block-wide scan over the words gives each its output offset and tie
 //     rank; every key > T and the first needed keys == T are written from the words' bits
 //     in ascending entry order, so the indices come out already sorted.
+//
+// Rows too long for one CTA's shared memory (1M-token contexts: 262144 entries) run one
+// thread-block cluster of up to 8 CTAs per query instead; rank r owns a contiguous slice of
+// the row.  Each digit's histogram is summed across the cluster through distributed shared
+// memory, so every rank picks the same bin.  As soon as the chosen bin holds at most 4096
+// keys of the row, one exchange gives every rank all ranks' candidates and their counts of
+// keys above the bin; the remaining bits are then resolved on every rank alone, and the
+// lower ranks' counts give each rank its output offset and tie budget.
 #include "launchers.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -128,6 +137,27 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
+}
+
+// Over the counts `h` of the current digit: picks the bin holding the krem-th largest key
+// (bins scanned from the top) and the rank left inside it; 1024 threads, 2 bins each.
+__device__ __forceinline__ void pick_bin_in(const uint32_t* h, uint32_t* scan_tmp,
+                                            uint32_t* bin_out, uint32_t* krem_out,
+                                            uint32_t& krem) {
+    const int tid = threadIdx.x;
+    const int bhi = kBins - 1 - 2 * tid, blo = bhi - 1;
+    const uint32_t chi = h[bhi], clo = h[blo];
+    uint32_t tot;
+    const uint32_t above = block_exclusive_scan(chi + clo, scan_tmp, tot);
+    if (above < krem && krem <= above + chi) {
+        *bin_out = (uint32_t)bhi;
+        *krem_out = krem - above;
+    } else if (above + chi < krem && krem <= above + chi + clo) {
+        *bin_out = (uint32_t)blo;
+        *krem_out = krem - above - chi;
+    }
+    __syncthreads();
+    krem = *krem_out;
 }
 
 // After hist[] holds the counts of the current digit: picks the bin holding the krem-th
@@ -369,6 +399,352 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         flag(dev_status, CSA_DEV_NAN);
 }
 
+// ---- long rows: one cluster per query ------------------------------------------------
+constexpr int kMaxCluster = 8;
+constexpr int kClusterSlice = 32768;    // entries per rank the cluster size aims at
+
+struct __align__(16) ClShared {
+    uint32_t hist[2][kBins];   // this rank's digit histogram, double-buffered across digits
+    uint32_t hsum[kBins];      // the cluster's summed histogram
+    uint32_t cand[kMaxCand];   // this rank's candidates, read by the others
+    uint32_t acand[kMaxCand];  // every rank's candidates, in rank order
+    uint32_t scan_tmp[33];
+    unsigned long long scan64[33];
+    uint32_t bin, krem, ncand, above, key_or, key_and, ngt, neq, g_or, g_and, out_base, take_eq;
+    uint32_t r_ncand[kMaxCluster], r_above[kMaxCluster], r_off[kMaxCluster + 1];
+    uint32_t r_gt[kMaxCluster], r_eq[kMaxCluster];
+};
+
+template <bool STAGED>
+__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(
+    const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_seq,
+    const int32_t* __restrict__ q_pos, const int64_t* __restrict__ seq_len, int B, int m,
+    int max_n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ dev_status) {
+    using namespace sm100;
+    extern __shared__ uint4 dyn4[];
+    ClShared& sh = *reinterpret_cast<ClShared*>(dyn4);
+    const int R = (int)cluster_nctarank();
+    const int rank = (int)cluster_ctarank();
+    const int qq = blockIdx.x / R;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int b = q_seq[qq];
+    const int t = q_pos[qq];
+    const bool valid = b >= 0 && b < B && t >= 0 && (int64_t)t < seq_len[b];
+    pdl_wait();   // scores come from the indexer
+    pdl_trigger();
+    int n = valid ? (t + 1) / m : 0;
+    if (n > max_n) n = max_n;
+    int32_t* out = idx_out + (int64_t)qq * k;
+    if (n <= k) {
+        // the same branch on every rank of the cluster: no cluster barrier is reached
+        if (rank == 0)
+            for (int j = tid; j < k; j += kThreads) out[j] = j < n ? j : -1;
+        return;
+    }
+    // my slice; inner boundaries on multiples of 32 entries (whole words, 16-byte loads)
+    const int lo = rank == 0 ? 0 : (int)(((int64_t)n * rank / R) & ~31LL);
+    const int hi = rank == R - 1 ? n : (int)(((int64_t)n * (rank + 1) / R) & ~31LL);
+    const int ns = hi - lo;
+    const float* s = scores + (int64_t)qq * ld + lo;
+    const bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
+    // after the shared state: the selection words of my slice, then its staged keys
+    const int slice_max = (max_n + R - 1) / R + 32;
+    const int wmax = (slice_max + 31) >> 5;
+    uint32_t* selw = reinterpret_cast<uint32_t*>(&sh + 1);
+    uint32_t* tiew = selw + wmax;
+    uint4* skey4 = reinterpret_cast<uint4*>(selw) + ((2 * wmax + 3) >> 2);
+    const uint32_t* skey = reinterpret_cast<const uint32_t*>(skey4);
+    if (tid == 0) {
+        sh.key_or = 0u;
+        sh.key_and = 0xFFFFFFFFu;
+        sh.ncand = 0u;
+        sh.above = 0u;
+        sh.ngt = 0u;
+        sh.neq = 0u;
+    }
+    __syncthreads();
+    auto get4 = [&](int i, uint32_t* key) {
+        if constexpr (STAGED) {
+            const uint4 v = i < ns ? skey4[i >> 2] : make_uint4(0u, 0u, 0u, 0u);
+            key[0] = i < ns ? v.x : 0u;
+            key[1] = i + 1 < ns ? v.y : 0u;
+            key[2] = i + 2 < ns ? v.z : 0u;
+            key[3] = i + 3 < ns ? v.w : 0u;
+        } else {
+            load4(s, i, ns, vec, key);
+        }
+    };
+    auto get1 = [&](int i) -> uint32_t {
+        if constexpr (STAGED) {
+            return skey[i];
+        } else {
+            return score_key(s[i]);
+        }
+    };
+    uint32_t kor = 0u, kand = 0xFFFFFFFFu;
+    for (int c0 = 0; c0 < ns; c0 += kChunk) {
+        const int i = c0 + 4 * tid;
+        uint32_t key[4];
+        load4(s, i, ns, vec, key);
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            if (i + u < ns) {
+                kor |= key[u];
+                kand &= key[u];
+            }
+        }
+        if constexpr (STAGED) {
+            if (i < ns) skey4[i >> 2] = make_uint4(key[0], key[1], key[2], key[3]);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+        kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+    }
+    if (lane == 0) {
+        atomicOr(&sh.key_or, kor);
+        atomicAnd(&sh.key_and, kand);
+    }
+    __syncthreads();
+    cluster_sync_all();   // every rank's OR / AND
+    if (wid == 0) {
+        uint32_t o = 0u, a = 0xFFFFFFFFu;
+        if (lane < R) {
+            o = ld_cluster_u32(mapa(&sh.key_or, (uint32_t)lane));
+            a = ld_cluster_u32(mapa(&sh.key_and, (uint32_t)lane));
+        }
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) {
+            o |= __shfl_xor_sync(0xffffffffu, o, x);
+            a &= __shfl_xor_sync(0xffffffffu, a, x);
+        }
+        if (lane == 0) {
+            sh.g_or = o;
+            sh.g_and = a;
+        }
+    }
+    __syncthreads();
+    const uint32_t diff = sh.g_or ^ sh.g_and;
+    uint32_t prefix = sh.g_and & ~diff;
+    uint32_t mask = ~diff;
+    uint32_t krem = (uint32_t)k;
+    int top = diff ? 31 - __clz(diff) : -1;
+    int digit = 0;
+    bool exchange = false;
+    // cluster-wide digits on the full slices, until the chosen bin is small
+    while (top >= 0) {
+        const int width = top >= 10 ? 11 : top + 1;
+        const int shift = top + 1 - width;
+        const uint32_t bmask = (1u << width) - 1u;
+        uint32_t* hist = sh.hist[digit & 1];
+        for (int x = tid; x < kBins; x += kThreads) hist[x] = 0u;
+        __syncthreads();
+        for (int c0 = 0; c0 < ns; c0 += kChunk) {
+            uint32_t key[4];
+            get4(c0 + 4 * tid, key);
+#pragma unroll
+            for (int u = 0; u < 4; u++)
+                if (c0 + 4 * tid + u < ns && (key[u] & mask) == prefix)
+                    atomicAdd(&hist[(key[u] >> shift) & bmask], 1u);
+        }
+        __syncthreads();
+        // every rank's histogram of this digit is complete (and every rank is done reading
+        // the previous digit's, which this buffer's next use overwrites)
+        cluster_sync_all();
+        if (tid < kBins / 4) {
+            uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+            for (int rr = 0; rr < R; rr++) {
+                const uint4 v = ld_cluster_u4(mapa(hist + 4 * tid, (uint32_t)rr));
+                acc.x += v.x;
+                acc.y += v.y;
+                acc.z += v.z;
+                acc.w += v.w;
+            }
+            *reinterpret_cast<uint4*>(sh.hsum + 4 * tid) = acc;
+        }
+        __syncthreads();
+        pick_bin_in(sh.hsum, sh.scan_tmp, &sh.bin, &sh.krem, krem);
+        const uint32_t in_bin = sh.hsum[sh.bin];   // over the whole row: the same on every rank
+        prefix |= sh.bin << shift;
+        mask |= bmask << shift;
+        top = shift - 1;
+        digit++;
+        __syncthreads();
+        if (top >= 0 && in_bin <= (uint32_t)kMaxCand) {
+            exchange = true;
+            break;
+        }
+    }
+    if (exchange) {
+        // my keys in the chosen region become candidates; keys above it are counted
+        uint32_t above = 0;
+        for (int c0 = 0; c0 < ns; c0 += kChunk) {
+            uint32_t key[4];
+            get4(c0 + 4 * tid, key);
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const bool in = c0 + 4 * tid + u < ns;
+                const uint32_t mk = key[u] & mask;
+                const bool p = in && mk == prefix;
+                above += (in && mk > prefix) ? 1u : 0u;
+                const uint32_t bal = __ballot_sync(0xffffffffu, p);
+                uint32_t slot = 0;
+                if (lane == 0 && bal) slot = atomicAdd(&sh.ncand, (uint32_t)__popc(bal));
+                slot = __shfl_sync(0xffffffffu, slot, 0);
+                if (p) sh.cand[slot + __popc(bal & lanemask_lt())] = key[u];
+            }
+        }
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) above += __shfl_xor_sync(0xffffffffu, above, x);
+        if (lane == 0) atomicAdd(&sh.above, above);
+        __syncthreads();
+        cluster_sync_all();   // every rank's candidates and counts
+        if (wid == 0) {
+            uint32_t nc = 0, ab = 0;
+            if (lane < R) {
+                nc = ld_cluster_u32(mapa(&sh.ncand, (uint32_t)lane));
+                ab = ld_cluster_u32(mapa(&sh.above, (uint32_t)lane));
+            }
+            uint32_t inc = nc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += y;
+            }
+            if (lane < R) {
+                sh.r_ncand[lane] = nc;
+                sh.r_above[lane] = ab;
+                sh.r_off[lane] = inc - nc;
+                sh.r_gt[lane] = 0u;
+                sh.r_eq[lane] = 0u;
+            }
+            if (lane == R - 1) sh.r_off[R] = inc;
+        }
+        __syncthreads();
+        const uint32_t nall = sh.r_off[R];   // the chosen bin's count over the row
+        for (int rr = 0; rr < R; rr++) {
+            const uint32_t nc = sh.r_ncand[rr], off = sh.r_off[rr];
+            for (uint32_t c = tid; c < nc; c += kThreads)
+                sh.acand[off + c] = ld_cluster_u32(mapa(sh.cand + c, (uint32_t)rr));
+        }
+        __syncthreads();
+        // the remaining bits on the full candidate list, on this rank alone
+        while (top >= 0) {
+            const int width = top >= 10 ? 11 : top + 1;
+            const int shift = top + 1 - width;
+            const uint32_t bmask = (1u << width) - 1u;
+            for (int x = tid; x < kBins; x += kThreads) sh.hsum[x] = 0u;
+            __syncthreads();
+            for (uint32_t c = tid; c < nall; c += kThreads) {
+                const uint32_t key = sh.acand[c];
+                if ((key & mask) == prefix) atomicAdd(&sh.hsum[(key >> shift) & bmask], 1u);
+            }
+            __syncthreads();
+            pick_bin_in(sh.hsum, sh.scan_tmp, &sh.bin, &sh.krem, krem);
+            prefix |= sh.bin << shift;
+            mask |= bmask << shift;
+            top = shift - 1;
+            __syncthreads();
+        }
+        // every rank's keys > T and == T among the candidates (runs are in rank order)
+        for (uint32_t c = tid; c < nall; c += kThreads) {
+            const uint32_t key = sh.acand[c];
+            int rr = 0;
+            while (rr + 1 < R && sh.r_off[rr + 1] <= c) rr++;
+            if (key > prefix) atomicAdd(&sh.r_gt[rr], 1u);
+            if (key == prefix) atomicAdd(&sh.r_eq[rr], 1u);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            uint32_t g = 0, e = 0;
+            for (int rr = 0; rr < rank; rr++) {
+                g += sh.r_above[rr] + sh.r_gt[rr];
+                e += sh.r_eq[rr];
+            }
+            sh.out_base = g + min(e, krem);
+            sh.take_eq = min(sh.r_eq[rank], krem - min(e, krem));
+        }
+        __syncthreads();
+    }
+    const uint32_t T = prefix;   // the k-th largest key of the row
+    // marking: word r holds my entries 32 r .. 32 r + 31 (bit = lane)
+    const int nwords = (ns + 31) >> 5;
+    for (int r = wid; r < nwords; r += kWarps) {
+        const int i = (r << 5) + lane;
+        const bool in = i < ns;
+        const uint32_t key = in ? get1(i) : 0u;
+        const uint32_t gt = __ballot_sync(0xffffffffu, in && key > T);
+        const uint32_t eq = __ballot_sync(0xffffffffu, in && key == T);
+        if (lane == 0) {
+            selw[r] = gt;
+            tiew[r] = eq;
+        }
+    }
+    __syncthreads();
+    const int wpt = (nwords + kThreads - 1) / kThreads;
+    const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
+    uint32_t cg = 0, ce = 0;
+    for (int w = w0; w < w1; w++) {
+        cg += __popc(selw[w]);
+        ce += __popc(tiew[w]);
+    }
+    unsigned long long tot;
+    const unsigned long long pre =
+        block_exclusive_scan64(((unsigned long long)ce << 32) | cg, sh.scan64, tot);
+    if (!exchange) {
+        // every bit was resolved cluster-wide: exchange the counts at T
+        if (tid == 0) {
+            sh.ngt = (uint32_t)tot;
+            sh.neq = (uint32_t)(tot >> 32);
+        }
+        __syncthreads();
+        cluster_sync_all();   // every rank's counts
+        if (wid == 0) {
+            uint32_t g = 0u, e = 0u;
+            if (lane < rank) {
+                g = ld_cluster_u32(mapa(&sh.ngt, (uint32_t)lane));
+                e = ld_cluster_u32(mapa(&sh.neq, (uint32_t)lane));
+            }
+#pragma unroll
+            for (int x = 16; x > 0; x >>= 1) {
+                g += __shfl_xor_sync(0xffffffffu, g, x);
+                e += __shfl_xor_sync(0xffffffffu, e, x);
+            }
+            if (lane == 0) {
+                sh.out_base = g + min(e, krem);
+                sh.take_eq = min(sh.neq, krem - min(e, krem));
+            }
+        }
+        __syncthreads();
+    }
+    const uint32_t budget = sh.take_eq;
+    uint32_t ties = (uint32_t)(pre >> 32);
+    uint32_t pos = sh.out_base + (uint32_t)pre + min(ties, budget);
+    for (int w = w0; w < w1; w++) {
+        uint32_t take = selw[w];
+        uint32_t tw = tiew[w];
+        while (tw && ties < budget) {
+            take |= tw & (0u - tw);
+            tw &= tw - 1;
+            ties++;
+        }
+        ties += __popc(tw);
+        while (take) {
+            const int bit = __ffs(take) - 1;
+            if (pos < (uint32_t)k) out[pos] = lo + (w << 5) + bit;
+            pos++;
+            take &= take - 1;
+        }
+    }
+    // the last rank ends at the row's total; NaN scores (no total order) break it
+    if (tid == 0 && rank == R - 1 &&
+        sh.out_base + (uint32_t)tot + min((uint32_t)(tot >> 32), budget) != (uint32_t)k)
+        flag(dev_status, CSA_DEV_NAN);
+    // no rank leaves while another may still read its shared memory
+    cluster_sync_all();
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
@@ -379,15 +755,33 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
     // histogram and candidate space this stays under the 227 KB per-CTA limit)
     const size_t row_bytes = (size_t)((max_n + 3) / 4) * 16;
     const size_t word_bytes = (size_t)((2 * ((max_n + 31) / 32) + 3) / 4) * 16;
-    const bool staged = word_bytes + row_bytes <= (size_t)176 * 1024;
-    const size_t smem = word_bytes + (staged ? row_bytes : 0);
-    auto kernel = staged ? topk_radix_kernel<true> : topk_radix_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    cudaError_t e;
+    if (word_bytes + row_bytes <= (size_t)176 * 1024) {
+        const size_t smem = word_bytes + row_bytes;
+        e = cudaFuncSetAttribute(topk_radix_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        LaunchScope scope(kKTopk, stream);
+        return launch_pdl(topk_radix_kernel<true>, dim3(Q), dim3(kThreads), smem, stream, scores,
+                          ld, q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st);
+    }
+    // long rows: a cluster of R CTAs per query, about kClusterSlice entries each (the
+    // selected set is unique under the total order, so the split does not change it)
+    int R = (max_n + kClusterSlice - 1) / kClusterSlice;
+    R = R < 2 ? 2 : (R > kMaxCluster ? kMaxCluster : R);
+    const int slice_max = (max_n + R - 1) / R + 32;
+    const int wmax = (slice_max + 31) / 32;
+    const size_t cl_words = (size_t)((2 * wmax + 3) / 4) * 16;
+    const size_t cl_row = (size_t)((slice_max + 3) / 4) * 16;
+    static_assert(sizeof(ClShared) % 16 == 0, "the words follow the shared state");
+    const bool staged = sizeof(ClShared) + cl_words + cl_row <= (size_t)220 * 1024;
+    const size_t smem = sizeof(ClShared) + cl_words + (staged ? cl_row : 0);
+    auto kernel = staged ? topk_cluster_kernel<true> : topk_cluster_kernel<false>;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchScope scope(kKTopk, stream);
-    return launch_pdl(kernel, dim3(Q), dim3(kThreads), smem, stream, scores, ld, q_seq, q_pos,
-                      seq_len, B, m, max_n, k, idx_out, st);
+    return launch_pdl_cluster(kernel, dim3(Q * R), dim3(kThreads), smem, stream, R, scores, ld,
+                              q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st);
 }
 
 }  // namespace csa

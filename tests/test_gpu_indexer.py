@@ -69,6 +69,26 @@ def test_ties_break_toward_lower_index():
     _exact(wl)
 
 
+def test_long_rows_cluster_of_seven_bit_exact():
+    # 210K and 70K visible entries: rows past one CTA's shared memory take the per-query
+    # cluster path, here 7 ranks (a cluster size that is not a power of two)
+    wl = synth.make_workload("t", B=2, T=[840003, 280001], D=128, H=16, m=4, span=8, H_I=16,
+                             d_I=128, k=1024, keep_raw=64, seed=28, device=DEV)
+    _exact(wl)
+
+
+def test_long_rows_massive_ties_bit_exact():
+    # only 3 distinct key rows over 150K entries: no bin ever gets small, so every bit is
+    # resolved across the cluster and the ties split between ranks by entry order
+    wl = synth.make_workload("t", B=1, T=[600001], D=128, H=16, m=4, span=8, H_I=16,
+                             d_I=128, k=1024, keep_raw=64, seed=29, device=DEV)
+    g = torch.Generator(device=DEV).manual_seed(1)
+    rows = wl.kI[torch.randint(0, 3, (wl.kI.shape[0],), device=DEV, generator=g)]
+    wl.kI.copy_(rows)
+    wl.w.fill_(1.0)
+    _exact(wl)
+
+
 def _abs_bound(wl, q):
     """fp32 rounding bound of one query's scores: the dot products accumulate 128 e4m3
     products in fp32 (error <= 2^-17 of the sum of |products| each, doubled for margin)
