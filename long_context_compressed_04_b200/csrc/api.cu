@@ -201,6 +201,8 @@ csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt, in
     if (csa::attn_tc_supported(H, D, fmt))
         return cuda_status(csa::launch_attn_tc(a, Q, 0, nullptr, (cudaStream_t)stream),
                            "attention launch");
+    if (csa::attn576_tc_supported(H, D, fmt))
+        return cuda_status(csa::launch_attn576_tc(a, Q, (cudaStream_t)stream), "attention launch");
     return cuda_status(csa::launch_attn_simt(a, Q, D, (cudaStream_t)stream), "attention launch");
 }
 

@@ -54,6 +54,7 @@ enum KernelKind {
     kKIndexerTc,
     kKAttnTc,
     kKAttnCombine,
+    kKAttn576Tc,
     kKernelKinds
 };
 
@@ -115,6 +116,8 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream);
 cudaError_t launch_attn_simt(const AttnArgs& a, int Q, int D, cudaStream_t stream);
 bool attn_tc_supported(int H, int D, int fmt);
+bool attn576_tc_supported(int H, int D, int fmt);
+cudaError_t launch_attn576_tc(const AttnArgs& a, int Q, cudaStream_t stream);
 size_t attn_tc_workspace_bytes(int Q, int max_n);
 cudaError_t launch_attn_tc(const AttnArgs& a, int Q, int max_n, void* workspace,
                            cudaStream_t stream);

@@ -360,6 +360,21 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t* r) {
     tmem_ld32(taddr + 32, r + 32);
 }
 
+// Stores 32 lanes x 16 consecutive 32-bit columns (thread i: row lane base + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor for a K-major tile stored with the 128-byte swizzle
 // (rows of 128 bytes, 8-row groups 1024 bytes apart; tile base 1024-byte aligned).
 // Advancing along K inside the 128-byte row adds (bytes >> 4) to the start address.

@@ -36,6 +36,7 @@ def _random_idx(wl, seed, pad=0):
     (16, 128, 0, 64, [4096]),                      # CSA decode 4K shape
     (64, 128, 0, 512, [7001, 3000, 2100]),         # CSA decode, ragged, k = 512
     (128, 576, 1, 256, [3000, 1500]),              # 576-dim fp8 + bf16 RoPE entries
+    (128, 576, 1, 1024, [9000, 3333, 200]),        # 1M-config shape: k = 1024, short rows padded
     (64, 576, 0, 128, [1203]),                     # 576-dim bf16 entries
 ])
 def test_sparse_attention(H, D, fmt, k, T):
@@ -62,11 +63,11 @@ def test_dense_hca_attention(T):
     _orc.assert_out_close(buf.out, _orc.attention(wl.to("cpu"), rows, None))
 
 
-@pytest.mark.parametrize("H", [16, 64])
-def test_short_window_and_no_window(H):
-    for W, T in [(128, [37]), (0, [400]), (5, [400]), (128, [3])]:
-        wl = synth.make_workload("t", B=len(T), T=T, D=128, H=H, m=4, span=8, W=W, H_I=4,
-                                 d_I=64, k=32, seed=33, device=DEV)
+@pytest.mark.parametrize("H,D,fmt", [(16, 128, 0), (64, 128, 0), (128, 576, 1)])
+def test_short_window_and_no_window(H, D, fmt):
+    for W, T in [(128, [37]), (0, [400]), (5, [400]), (128, [3]), (70, [900])]:
+        wl = synth.make_workload("t", B=len(T), T=T, D=D, H=H, m=4, span=8, W=W, H_I=4,
+                                 d_I=64, k=32, fmt=fmt, seed=33, device=DEV)
         buf, rows = _with_oracle_entries(wl)
         idx = _random_idx(wl, 2)
         buf.idx.copy_(torch.from_numpy(idx))
@@ -75,10 +76,10 @@ def test_short_window_and_no_window(H):
         _orc.assert_out_close(buf.out, _orc.attention(wl.to("cpu"), rows, idx))
 
 
-@pytest.mark.parametrize("H", [16, 64])
-def test_sink_limits(H):
-    wl = synth.make_workload("t", B=1, T=[2000], D=128, H=H, m=4, span=8, H_I=4, d_I=64, k=64,
-                             seed=34, device=DEV)
+@pytest.mark.parametrize("H,D,fmt", [(16, 128, 0), (64, 128, 0), (128, 576, 1)])
+def test_sink_limits(H, D, fmt):
+    wl = synth.make_workload("t", B=1, T=[2000], D=D, H=H, m=4, span=8, H_I=4, d_I=64, k=64,
+                             fmt=fmt, seed=34, device=DEV)
     buf, rows = _with_oracle_entries(wl)
     idx = _random_idx(wl, 3)
     buf.idx.copy_(torch.from_numpy(idx))
@@ -90,10 +91,10 @@ def test_sink_limits(H):
     assert buf.out.abs().max().item() < 1e-20   # sink = 60 >> logits: output ~ e^-50
 
 
-@pytest.mark.parametrize("H", [16, 64])
-def test_out_of_range_index_is_flagged_and_skipped(H):
-    wl = synth.make_workload("t", B=1, T=[2000], D=128, H=H, m=4, span=8, H_I=4, d_I=64, k=64,
-                             seed=35, device=DEV)
+@pytest.mark.parametrize("H,D,fmt", [(16, 128, 0), (64, 128, 0), (128, 576, 1)])
+def test_out_of_range_index_is_flagged_and_skipped(H, D, fmt):
+    wl = synth.make_workload("t", B=1, T=[2000], D=D, H=H, m=4, span=8, H_I=4, d_I=64, k=64,
+                             fmt=fmt, seed=35, device=DEV)
     buf, rows = _with_oracle_entries(wl)
     idx = _random_idx(wl, 4, pad=1)
     bad = idx.copy()
@@ -123,3 +124,37 @@ def test_batch_invariance_bitwise():
     vals = list(outs.values())
     for v in vals[1:]:
         assert torch.equal(v.view(torch.int16), vals[0].view(torch.int16))
+
+
+def test_batch_invariance_bitwise_576_fp8_sweep():
+    # the 1M configuration's sweep on the attention stage: the same queries inside batches of
+    # 1, 7, 32 and 64 with random neighbour sequences; entries stored directly (656-byte rows)
+    g = torch.Generator().manual_seed(5)
+    lens = [int(x) for x in torch.randint(4096, 200000, (64,), generator=g)]
+    base = synth.make_workload("t", B=64, T=lens, D=576, H=128, m=4, span=8, fmt=1, H_I=4,
+                               d_I=64, k=1024, keep_raw=128, seed=37, device=DEV)
+    parts = synth.split(base)
+    targets = [0, 1]
+    gd = torch.Generator(device=DEV).manual_seed(9)
+    ents = synth.random_entries(base.ent_rows, 1, 576, gd, DEV)
+    idx_all = torch.from_numpy(_random_idx(base, 11))
+    outs = {}
+    for batch in ([0], [1], [0, 1] + list(range(2, 7)), list(range(32)), list(range(63, -1, -1))):
+        wl = synth.merge([parts[i] for i in batch])
+        buf = pipeline.alloc(wl, DEV)
+        for slot, i in enumerate(batch):
+            e0, n = int(base.ent_off[i]), int(base.n_ent[i])
+            f0 = int(wl.ent_off[slot])
+            buf.entries[f0:f0 + n].copy_(ents[e0:e0 + n])
+            buf.idx[slot].copy_(idx_all[i])
+        pipeline.attend(wl, buf)
+        torch.cuda.synchronize()
+        assert int(buf.dev_status.item()) == 0
+        for tgt in targets:
+            if tgt in batch:
+                outs.setdefault(tgt, []).append(buf.out[batch.index(tgt)].clone())
+    for tgt in targets:
+        ref = outs[tgt][0]
+        assert len(outs[tgt]) >= 3
+        for v in outs[tgt][1:]:
+            assert torch.equal(v.view(torch.int16), ref.view(torch.int16))
