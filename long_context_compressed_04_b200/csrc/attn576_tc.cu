@@ -9,8 +9,8 @@
 //   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once; per
 //              tile, 2 threads per key row dequantize the gathered FP8 row (or normalise the
 //              raw window row) into bf16, 128-byte swizzled, 9 blocks of 64 channels; the
-//              next entry tile's bytes are loaded into registers while the previous tile
-//              is still in use.
+//              next entry tile's rows are copied (cp.async) into a raw staging buffer while
+//              the previous tile is still in use.
 //   warp 4     TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
 //              S = Q K^T (M = 64 heads, N = 64 keys, 36 K steps of 16 channels) into one of
 //              two S buffers, then O += P V straight into the TMEM accumulator: channels
@@ -99,51 +99,63 @@ __device__ __forceinline__ void put8(uint8_t* tile, int r, int d0, uint4 v) {
     *reinterpret_cast<uint4*>(tile + (d0 >> 6) * kBlk + swz(r, (d0 & 63) >> 3)) = v;
 }
 
+// Two e4m3 codes (low 16 bits; the lower byte first) to two floats, exactly, by the packed
+// hardware conversion to f16.
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t two) {
+    uint32_t h;
+    asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+        : "=r"(h)
+        : "r"(two));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
 // 16 e4m3 codes times `sc`, as 16 bf16 (two 16-byte chunks).
 __device__ __forceinline__ void dequant16(uint4 c, float sc, uint4& lo, uint4& hi) {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
     uint32_t o[8];
 #pragma unroll
     for (int z = 0; z < 4; z++) {
-        const uint32_t x = w[z];
-        o[2 * z] = pack_bf16x2(e4m3_to_f32(x & 0xFFu) * sc, e4m3_to_f32((x >> 8) & 0xFFu) * sc);
-        o[2 * z + 1] = pack_bf16x2(e4m3_to_f32((x >> 16) & 0xFFu) * sc, e4m3_to_f32(x >> 24) * sc);
+        const float2 a = e4m3x2_to_f32x2(w[z] & 0xFFFFu);
+        const float2 b = e4m3x2_to_f32x2(w[z] >> 16);
+        o[2 * z] = pack_bf16x2(a.x * sc, a.y * sc);
+        o[2 * z + 1] = pack_bf16x2(b.x * sc, b.y * sc);
     }
     lo = make_uint4(o[0], o[1], o[2], o[3]);
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// One loader thread's half of a selected entry row: fp8 channels [256 hf, 256 hf + 256),
-// the row's four scales, RoPE channels [32 hf, 32 hf + 32).
-struct EntryHalf {
-    uint4 f[16];
-    uint4 sc;
-    uint4 rope[4];
-    bool valid;
-};
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_addr(dst)),
+                 "l"(src)
+                 : "memory");
+}
 
-// Loads entry v of the query's index row, staged in shared memory (flags an out-of-range
-// index once per row).
-__device__ __forceinline__ void fetch_entry(const A576Args& a, const int32_t* sidx, int v,
-                                            int n_vis, int64_t row0, int hf, EntryHalf& x) {
+// Starts copying one loader thread's half of entry v of the query's index row (staged in
+// shared memory) into its raw row slot: fp8 channels [256 hf, 256 hf + 256), RoPE channels
+// [32 hf, 32 hf + 32), and (hf = 0) the four scales.  False for an invalid index (an
+// out-of-range one is flagged once per row).
+__device__ __forceinline__ bool fetch_entry(const A576Args& a, const int32_t* sidx, int v,
+                                            int n_vis, int64_t row0, int hf, uint8_t* raw) {
     const int e = v < a.k ? sidx[v] : -1;
-    x.valid = false;
+    bool valid = false;
     if (e >= 0) {
         if (e < n_vis && row0 + e < a.ent_rows) {
-            x.valid = true;
+            valid = true;
         } else if (hf == 0) {
             flag(a.st, CSA_DEV_OOB);
         }
     }
-    if (x.valid) {
+    if (valid) {
         const uint8_t* er = a.entries + (row0 + e) * (int64_t)kRowBytes;
 #pragma unroll
-        for (int u = 0; u < 16; u++) x.f[u] = *reinterpret_cast<const uint4*>(er + 256 * hf + 16 * u);
-        x.sc = *reinterpret_cast<const uint4*>(er + 512);
+        for (int u = 0; u < 16; u++) cp_async16(raw + 256 * hf + 16 * u, er + 256 * hf + 16 * u);
 #pragma unroll
         for (int u = 0; u < 4; u++)
-            x.rope[u] = *reinterpret_cast<const uint4*>(er + 528 + 64 * hf + 16 * u);
+            cp_async16(raw + 528 + 64 * hf + 16 * u, er + 528 + 64 * hf + 16 * u);
+        if (hf == 0) cp_async16(raw + 512, er + 512);
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    return valid;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args a) {
@@ -164,7 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     float* rwc = rf + 32;                                 // [32] cos / sin of pair j at w0
     float* rws = rwc + 32;
     int32_t* sidx = reinterpret_cast<int32_t*>(rws + 32); // [kMaxK] the query's index row
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sidx + kMaxK);
+    uint8_t* sRaw = reinterpret_cast<uint8_t*>(sidx + kMaxK);   // [64][656] next entry rows
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + kTK * kRowBytes);
     uint64_t* qfull = bars;          // 4 loader warps
     uint64_t* kfull = bars + 1;      // 4 loader warps
     uint64_t* kfree = bars + 2;      // MMA commit after the tile's P V
@@ -245,29 +258,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         if (valid) {
             // q head row r at t: channels [288 hf, 288 hf + 288), RoPE on 512..575
             const uint16_t* qrow = a.q + ((int64_t)qi * a.H + kHC * g + r) * kD;
-#pragma unroll 4
-            for (int c = 0; c < 36; c++) {
-                const int d0 = 288 * hf + 8 * c;
-                uint4 u = *reinterpret_cast<const uint4*>(qrow + d0);
-                if (d0 >= kD - kRopeDims) {
-                    uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                    for (int z = 0; z < 4; z++) {
-                        const int pj = (d0 - (kD - kRopeDims)) / 2 + z;
-                        const float2 f = bf16x2_to_f32(w[z]);
-                        w[z] = pack_bf16x2(f.x * rqc[pj] - f.y * rqs[pj], f.x * rqs[pj] + f.y * rqc[pj]);
+            for (int half = 0; half < 2; half++) {
+                uint4 u[18];   // 18 loads in flight
+#pragma unroll
+                for (int c = 0; c < 18; c++)
+                    u[c] = *reinterpret_cast<const uint4*>(qrow + 288 * hf + 144 * half + 8 * c);
+#pragma unroll
+                for (int c = 0; c < 18; c++) {
+                    const int d0 = 288 * hf + 144 * half + 8 * c;
+                    if (d0 >= kD - kRopeDims) {
+                        uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+#pragma unroll
+                        for (int z = 0; z < 4; z++) {
+                            const int pj = (d0 - (kD - kRopeDims)) / 2 + z;
+                            const float2 f = bf16x2_to_f32(w[z]);
+                            w[z] = pack_bf16x2(f.x * rqc[pj] - f.y * rqs[pj], f.x * rqs[pj] + f.y * rqc[pj]);
+                        }
+                        u[c] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    u = make_uint4(w[0], w[1], w[2], w[3]);
+                    put8(sQ, r, d0, u[c]);
                 }
-                put8(sQ, r, d0, u);
             }
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(qfull);
         }
-        EntryHalf ex;
-        ex.valid = false;
-        if (n_wt == 0 && ntiles > 0) fetch_entry(a, sidx, r, n_vis, row0, hf, ex);
+        uint8_t* myraw = sRaw + r * kRowBytes;
+        bool ex_valid = false;
+        if (n_wt == 0 && ntiles > 0) ex_valid = fetch_entry(a, sidx, r, n_vis, row0, hf, myraw);
         for (int j = 0; j < ntiles && ok; j++) {
             // the key buffer is free once the previous tile's P V has completed
             if (j > 0 && !mbar_wait_warp(kfree, (j - 1) & 1, abort_flag, a.st)) {
@@ -287,28 +306,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 }
                 const uint16_t* src =
                     vrow ? a.kv + (a.kv_off[b] + p - a.kv_pos0[b]) * (int64_t)kD : nullptr;
+                // pass 1: the raw row into the tile (18 loads in flight) and its sum of squares
                 float ss = 0.f;
-                if (vrow) {
-#pragma unroll 4
-                    for (int c = 0; c < 36; c++) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(src + 288 * hf + 8 * c);
-                        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int half = 0; half < 2; half++) {
+                    uint4 u[18];
+#pragma unroll
+                    for (int c = 0; c < 18; c++)
+                        u[c] = vrow ? *reinterpret_cast<const uint4*>(src + 288 * hf + 144 * half + 8 * c)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int c = 0; c < 18; c++) {
+                        const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
 #pragma unroll
                         for (int z = 0; z < 4; z++) {
                             const float2 f = bf16x2_to_f32(w[z]);
                             ss += f.x * f.x + f.y * f.y;
                         }
+                        put8(sK, r, 288 * hf + 144 * half + 8 * c, u[c]);
                     }
                 }
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
                 const float rn = rsqrtf(ss / (float)kD + a.eps);
-#pragma unroll 2
-                for (int c = 0; c < 36; c++) {
-                    const int d0 = 288 * hf + 8 * c;
-                    uint32_t w[4] = {0u, 0u, 0u, 0u};
-                    if (vrow) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(src + d0);
+                // pass 2, in place in shared memory: normalise, RoPE at the row's position
+                if (vrow) {
+#pragma unroll 4
+                    for (int c = 0; c < 36; c++) {
+                        const int d0 = 288 * hf + 8 * c;
+                        uint4* cell = reinterpret_cast<uint4*>(sK + (d0 >> 6) * kBlk + swz(r, (d0 & 63) >> 3));
+                        const uint4 u = *cell;
                         const uint32_t wi[4] = {u.x, u.y, u.z, u.w};
+                        uint32_t w[4];
 #pragma unroll
                         for (int z = 0; z < 4; z++) {
                             float2 f = bf16x2_to_f32(wi[z]);
@@ -326,24 +354,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                             }
                             w[z] = pack_bf16x2(f.x, f.y);
                         }
+                        *cell = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    put8(sK, r, d0, make_uint4(w[0], w[1], w[2], w[3]));
                 }
             } else {
-                vrow = ex.valid;
-                const float sc0 = __uint_as_float(hf ? ex.sc.z : ex.sc.x);
-                const float sc1 = __uint_as_float(hf ? ex.sc.w : ex.sc.y);
-#pragma unroll
+                vrow = ex_valid;
+                // this thread's copies, then its partner's (the scales) are visible
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+                __syncwarp();
+                const float* scl = reinterpret_cast<const float*>(myraw + 512);
+                const float sc0 = vrow ? scl[2 * hf] : 0.f, sc1 = vrow ? scl[2 * hf + 1] : 0.f;
+#pragma unroll 4
                 for (int u = 0; u < 16; u++) {
                     uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-                    if (vrow) dequant16(ex.f[u], u < 8 ? sc0 : sc1, lo, hi);
+                    if (vrow)
+                        dequant16(*reinterpret_cast<const uint4*>(myraw + 256 * hf + 16 * u),
+                                  u < 8 ? sc0 : sc1, lo, hi);
                     const int d0 = 256 * hf + 16 * u;
                     put8(sK, r, d0, lo);
                     put8(sK, r, d0 + 8, hi);
                 }
 #pragma unroll
                 for (int u = 0; u < 4; u++)
-                    put8(sK, r, 512 + 32 * hf + 8 * u, vrow ? ex.rope[u] : make_uint4(0u, 0u, 0u, 0u));
+                    put8(sK, r, 512 + 32 * hf + 8 * u,
+                         vrow ? *reinterpret_cast<const uint4*>(myraw + 528 + 64 * hf + 16 * u)
+                              : make_uint4(0u, 0u, 0u, 0u));
+                // the raw slot is read: the partner may overwrite its half with the next row
+                __syncwarp();
             }
             // valid keys of the tile: this warp's 16 rows (even lanes carry them)
             const uint32_t bal = __ballot_sync(0xffffffffu, vrow && hf == 0);
@@ -356,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             if (lane == 0) mbar_arrive(kfull);
             // the next entry tile's bytes in flight while this one is used
             if (j + 1 >= n_wt && j + 1 < ntiles)
-                fetch_entry(a, sidx, (j + 1 - n_wt) * kTK + r, n_vis, row0, hf, ex);
+                ex_valid = fetch_entry(a, sidx, (j + 1 - n_wt) * kTK + r, n_vis, row0, hf, myraw);
         }
     } else if (warp == 4) {
         if (lane == 0 && ntiles > 0) {
@@ -556,8 +593,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     }
 }
 
-constexpr size_t kSmemBytes =
-    1024 + kQBytes + kKBytes + 2 * kPBytes + 8 * 2 + 5 * 32 * 4 + kMaxK * 4 + 13 * 8 + 16;
+constexpr size_t kSmemBytes = 1024 + kQBytes + kKBytes + 2 * kPBytes + 8 * 2 + 5 * 32 * 4 +
+                              kMaxK * 4 + kTK * kRowBytes + 13 * 8 + 16;
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 }  // namespace
 
