@@ -8,6 +8,8 @@ sets must match bit for bit; with N(0,1) FP8 inputs (the benchmark's) the scores
 within their fp32 rounding bound of the oracle's and the selections may differ only among
 keys within that bound of the k-th score.  Attention outputs are compared within the
 bf16 / fp8-storage tolerance, on the GPU's own index sets (stage-isolated)."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -46,9 +48,18 @@ def _score_bound(part, s_o):
     return (2.0 ** -16 * mag).numpy() + 2.0 ** -18 * 64 * np.abs(s_o[:n])
 
 
+def _only_queries(wl, qs):
+    """The same sequences with only the listed queries (for the oracle)."""
+    sel = torch.tensor(qs, dtype=torch.int64, device=wl.q.device)
+    f = dict(q_seq=wl.q_seq[sel], q_pos=wl.q_pos[sel], q=wl.q[sel])
+    if wl.H_I:
+        f.update(qI=wl.qI[sel], qs=wl.qs[sel], w=wl.w[sel])
+    return dataclasses.replace(wl, **f)
+
+
 def _check_csa_query(wl, buf, sc, q, exact):
     b = int(wl.q_seq[q])
-    part = synth.split(wl)[b].to("cpu")
+    part = _only_queries(synth.split(wl)[b], [int((wl.q_seq[:q] == b).sum())]).to("cpu")
     rows, _ = _orc.compress(part)
     idx_o, s_o = _orc.indexer(part)
     idx_g = buf.idx[q].cpu().numpy()
@@ -90,3 +101,12 @@ def test_csa_decode_1m_b8_fp8_entries_sampled():
     wl = synth.csa_decode_1m_fp8(device=DEV, indexer="fp8")
     buf, sc = _run_full(wl)
     _check_csa_query(wl, buf, sc, wl.Q - 1, exact=False)
+
+
+def test_csa_prefill_8k_on_64k_sampled():
+    # causal prefill chunk: 8192 new queries after 65536 prior tokens, top-1024; the oracle
+    # recomputes a few queries across the chunk (early, middle, last)
+    wl = synth.csa_prefill_64k(device=DEV)
+    buf, sc = _run_full(wl)
+    for q in (0, 4097, wl.Q - 1):
+        _check_csa_query(wl, buf, sc, q, exact=True)
