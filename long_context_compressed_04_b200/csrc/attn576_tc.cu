@@ -4,24 +4,26 @@
 // window, with the attention sink and partial / inverse RoPE ("DeepSeek-V4 深度分析报告"
 // 2.1 CSA and "其他注意力技术细节").
 //
-// One CTA per (query, group of 64 heads).  The keys of the query are tiles of 64: the
-// window's raw rows first (RMSNormed and RoPEd here), then the selected entries.
+// One CTA per (query, group of 64 heads).  The keys of the query are tiles of 32: the
+// window's raw rows first (RMSNormed and RoPEd here), then the selected entries; two key
+// buffers let one tile be built while the previous one is in the tensor cores.
 //   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once; per
-//              tile, 2 threads per key row dequantize the gathered FP8 row (or normalise the
+//              tile, 4 threads per key row dequantize the gathered FP8 row (or normalise the
 //              raw window row) into bf16, 128-byte swizzled, 9 blocks of 64 channels; the
 //              next entry tile's rows are copied (cp.async) into a raw staging buffer while
-//              the previous tile is still in use.
+//              the previous one is converted.
 //   warp 4     TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
-//              S = Q K^T (M = 64 heads, N = 64 keys, 36 K steps of 16 channels) into one of
-//              two S buffers, then O += P V straight into the TMEM accumulator: channels
-//              0-255 in TMEM lanes 0-15 of each quarter, 256-511 in lanes 16-31, 512-575 in
-//              lanes 0-15 again (N = 256 + 256 + 64), V being the key tile read MN-major.
+//              S = Q K^T (M = 64 heads, N = 32 keys, 36 K steps of 16 channels) into one of
+//              two S buffers, one tile ahead of O += P V, which goes straight into the TMEM
+//              accumulator: channels 0-255 in TMEM lanes 0-15 of each quarter, 256-511 in
+//              lanes 16-31, 512-575 in lanes 0-15 again (N = 256 + 256 + 64), V being the
+//              key tile read MN-major.
 //   warps 5-8  online softmax in the log2 domain, one head row per lane: P as bf16 into
 //              shared memory; the running maximum is a reference that moves only when a
 //              tile's maximum exceeds it by 2^8, and then the head's O row in TMEM is
 //              rescaled; finally the sink, the normalisation, inverse RoPE and the store.
-// A 64 x 576 fp32 accumulator takes 320 TMEM columns, and the query's Q tile (72 KB) and
-// one key tile (72 KB) fill most of shared memory: hence 64 heads per CTA, 64-key tiles.
+// A 64 x 576 fp32 accumulator takes 320 TMEM columns, and the query's Q tile (72 KB) fills
+// a third of shared memory: hence 64 heads per CTA and two key buffers of 32 rows.
 // All waits are bounded (timeout -> CSA_DEV_TIMEOUT, drain, free TMEM, return).  A query's
 // arithmetic never depends on the batch.
 #include <mutex>
@@ -36,20 +38,33 @@ namespace {
 constexpr int kHC = 64;                  // heads per CTA (MMA M)
 constexpr int kD = 576;
 constexpr int kNB = kD / 64;             // 9 blocks of 64 channels (128 bytes of bf16)
-constexpr int kTK = 64;                  // keys per tile (MMA N of S)
-constexpr int kBlk = 64 * 128;           // one 64-row x 128-byte swizzled block
-constexpr int kQBytes = kNB * kBlk;      // 72 KB
-constexpr int kKBytes = kNB * kBlk;      // 72 KB
-constexpr int kPBytes = kBlk;            // 8 KB
+constexpr int kTK = 32;                  // keys per tile (MMA N of S)
+constexpr int kQBlk = 64 * 128;          // one 64-row x 128-byte swizzled block of Q
+constexpr int kKBlk = kTK * 128;         // one 32-row x 128-byte swizzled block of K
+constexpr int kQBytes = kNB * kQBlk;     // 72 KB
+constexpr int kKBytes = kNB * kKBlk;     // 36 KB per key buffer
+constexpr int kPBytes = 64 * 128;        // 8 KB (rows of 128 B, the first 64 B used)
 constexpr int kRowBytes = 656;
 constexpr int kThreads = 288;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.f;          // the reference maximum moves by more than 2^8 only
 constexpr uint32_t kColO = 0;            // O channels 0-255 (lanes 0-15) / 256-511 (lanes 16-31)
 constexpr uint32_t kColOr = 256;         // O channels 512-575 (lanes 0-15)
-constexpr uint32_t kColS = 320;          // S buffers at 320 and 384 (lanes 0-15)
+constexpr uint32_t kColS = 320;          // S buffers at 320 and 352 (lanes 0-15)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxK = 2048;
+// shared-memory layout (byte offsets from the 1024-aligned base)
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kNB * 64 * 128;            // after Q (72 KB)
+constexpr int kOffP = kOffK + 2 * kNB * 32 * 128;        // after two key buffers
+constexpr int kOffRaw = kOffP + 2 * 64 * 128;            // after two P buffers
+constexpr int kOffMask = kOffRaw + 32 * 656;
+constexpr int kOffRope = kOffMask + 16;
+constexpr int kOffIdx = kOffRope + 5 * 32 * 4;
+constexpr int kOffBars = kOffIdx + kMaxK * 4;
+constexpr int kOffEnd = kOffBars + 16 * 8 + 16;
+static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles on 1024 B");
+static_assert(kOffRaw % 16 == 0 && kOffIdx % 16 == 0 && kOffBars % 8 == 0, "alignment");
 
 struct A576Args {
     const uint16_t* q;
@@ -94,9 +109,9 @@ __device__ __forceinline__ uint64_t desc_mn(const void* tile, uint32_t lbo_bytes
 }
 
 // 8 channels (16 bytes of bf16) of row `r`, channel `d0` (a multiple of 8), into a
-// [9 blocks][64 rows x 128 B] swizzled tile.
-__device__ __forceinline__ void put8(uint8_t* tile, int r, int d0, uint4 v) {
-    *reinterpret_cast<uint4*>(tile + (d0 >> 6) * kBlk + swz(r, (d0 & 63) >> 3)) = v;
+// [9 blocks][rows x 128 B] swizzled tile with blocks `blk` bytes apart.
+__device__ __forceinline__ uint4* cell8(uint8_t* tile, int blk, int r, int d0) {
+    return reinterpret_cast<uint4*>(tile + (d0 >> 6) * blk + swz(r, (d0 & 63) >> 3));
 }
 
 // Two e4m3 codes (low 16 bits; the lower byte first) to two floats, exactly, by the packed
@@ -130,29 +145,29 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
                  : "memory");
 }
 
-// Starts copying one loader thread's half of entry v of the query's index row (staged in
-// shared memory) into its raw row slot: fp8 channels [256 hf, 256 hf + 256), RoPE channels
-// [32 hf, 32 hf + 32), and (hf = 0) the four scales.  False for an invalid index (an
+// Starts copying one loader thread's quarter of entry v of the query's index row (staged in
+// shared memory) into its raw row slot: fp8 channels [128 qt, 128 qt + 128), RoPE channels
+// [16 qt, 16 qt + 16), and (qt = 0) the four scales.  False for an invalid index (an
 // out-of-range one is flagged once per row).
 __device__ __forceinline__ bool fetch_entry(const A576Args& a, const int32_t* sidx, int v,
-                                            int n_vis, int64_t row0, int hf, uint8_t* raw) {
+                                            int n_vis, int64_t row0, int qt, uint8_t* raw) {
     const int e = v < a.k ? sidx[v] : -1;
     bool valid = false;
     if (e >= 0) {
         if (e < n_vis && row0 + e < a.ent_rows) {
             valid = true;
-        } else if (hf == 0) {
+        } else if (qt == 0) {
             flag(a.st, CSA_DEV_OOB);
         }
     }
     if (valid) {
         const uint8_t* er = a.entries + (row0 + e) * (int64_t)kRowBytes;
 #pragma unroll
-        for (int u = 0; u < 16; u++) cp_async16(raw + 256 * hf + 16 * u, er + 256 * hf + 16 * u);
+        for (int u = 0; u < 8; u++) cp_async16(raw + 128 * qt + 16 * u, er + 128 * qt + 16 * u);
 #pragma unroll
-        for (int u = 0; u < 4; u++)
-            cp_async16(raw + 528 + 64 * hf + 16 * u, er + 528 + 64 * hf + 16 * u);
-        if (hf == 0) cp_async16(raw + 512, er + 512);
+        for (int u = 0; u < 2; u++)
+            cp_async16(raw + 528 + 32 * qt + 16 * u, er + 528 + 32 * qt + 16 * u);
+        if (qt == 0) cp_async16(raw + 512, er + 512);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
     return valid;
@@ -160,34 +175,37 @@ __device__ __forceinline__ bool fetch_entry(const A576Args& a, const int32_t* si
 
 __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args a) {
     using namespace sm100;
-    constexpr uint32_t kIdescS = instr_desc(1, 1, 64, 64);
+    constexpr uint32_t kIdescS = instr_desc(1, 1, 64, kTK);
     constexpr uint32_t kIdescPV = instr_desc(1, 1, 64, 256, 1);
     constexpr uint32_t kIdescPVr = instr_desc(1, 1, 64, 64, 1);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* sQ = smem;                                   // [9][64 x 128 B]
-    uint8_t* sK = sQ + kQBytes;                           // [9][64 x 128 B]
-    uint8_t* sP = sK + kKBytes;                           // [2][64 x 128 B]
-    uint16_t* smask = reinterpret_cast<uint16_t*>(sP + 2 * kPBytes);   // [2][4] valid keys
-    float* rqc = reinterpret_cast<float*>(smask + 8);     // [32] cos / sin of pair j at t
+    uint8_t* sQ = smem + kOffQ;                           // [9][64 x 128 B]
+    uint8_t* sK = smem + kOffK;                           // [2][9][32 x 128 B]
+    uint8_t* sP = smem + kOffP;                           // [2][64 x 128 B]
+    uint8_t* sRaw = smem + kOffRaw;                       // [32][656] next entry rows (16 B
+                                                          // aligned: cp.async destinations)
+    uint8_t* smask = smem + kOffMask;                     // [2][4] valid keys, 8 per warp
+    float* rqc = reinterpret_cast<float*>(smem + kOffRope);   // [32] cos / sin of pair j at t
     float* rqs = rqc + 32;
     float* rf = rqs + 32;                                 // [32] frequency of pair j
     float* rwc = rf + 32;                                 // [32] cos / sin of pair j at w0
     float* rws = rwc + 32;
-    int32_t* sidx = reinterpret_cast<int32_t*>(rws + 32); // [kMaxK] the query's index row
-    uint8_t* sRaw = reinterpret_cast<uint8_t*>(sidx + kMaxK);   // [64][656] next entry rows
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sRaw + kTK * kRowBytes);
+    int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);   // [kMaxK] the index row
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
     uint64_t* qfull = bars;          // 4 loader warps
-    uint64_t* kfull = bars + 1;      // 4 loader warps
-    uint64_t* kfree = bars + 2;      // MMA commit after the tile's P V
-    uint64_t* sfull = bars + 3;      // [2] MMA commit
-    uint64_t* sfree = bars + 5;      // [2] 4 softmax warps
-    uint64_t* pfull = bars + 7;      // [2] 4 softmax warps
-    uint64_t* pfree = bars + 9;      // [2] MMA commit
-    uint64_t* pvdone = bars + 11;    // MMA commit after every P V
-    uint64_t* drain = bars + 12;
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 13);
+    uint64_t* kfull = bars + 1;      // [2] 4 loader warps
+    uint64_t* kfree = bars + 3;      // [2] MMA commit after the tile's P V
+    uint64_t* sfull = bars + 5;      // [2] MMA commit
+    uint64_t* sfree = bars + 7;      // [2] 4 softmax warps
+    uint64_t* pfull = bars + 9;      // [2] 4 softmax warps
+    uint64_t* pfree = bars + 11;     // [2] MMA commit
+    uint64_t* pvdone = bars + 13;    // MMA commit after every P V (a rescale waits for the
+                                     // previous tile's: never more than one phase behind)
+    uint64_t* odone = bars + 14;     // MMA commit after the last P V (one phase)
+    uint64_t* drain = bars + 15;
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 16);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -199,15 +217,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     const bool valid = b >= 0 && b < a.B && t >= 0 && (int64_t)t < a.seq_len[b];
     if (threadIdx.x == 0) {
         mbar_init(qfull, 4);
-        mbar_init(kfull, 4);
-        mbar_init(kfree, 1);
         for (int i = 0; i < 2; i++) {
+            mbar_init(&kfull[i], 4);
+            mbar_init(&kfree[i], 1);
             mbar_init(&sfull[i], 1);
             mbar_init(&sfree[i], 4);
             mbar_init(&pfull[i], 4);
             mbar_init(&pfree[i], 1);
         }
         mbar_init(pvdone, 1);
+        mbar_init(odone, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -277,43 +296,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                         }
                         u[c] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    put8(sQ, r, d0, u[c]);
+                    *cell8(sQ, kQBlk, r, d0) = u[c];
                 }
             }
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(qfull);
         }
-        uint8_t* myraw = sRaw + r * kRowBytes;
+        // tiles: 4 threads per key row, quarter qt
+        const int kr = tid >> 2, qt = tid & 3;
+        uint8_t* myraw = sRaw + kr * kRowBytes;
         bool ex_valid = false;
-        if (n_wt == 0 && ntiles > 0) ex_valid = fetch_entry(a, sidx, r, n_vis, row0, hf, myraw);
+        if (n_wt == 0 && ntiles > 0) ex_valid = fetch_entry(a, sidx, kr, n_vis, row0, qt, myraw);
         for (int j = 0; j < ntiles && ok; j++) {
-            // the key buffer is free once the previous tile's P V has completed
-            if (j > 0 && !mbar_wait_warp(kfree, (j - 1) & 1, abort_flag, a.st)) {
+            const int kb = j & 1;
+            uint8_t* tile = sK + kb * kKBytes;
+            // this key buffer is free once the P V of the tile two back has completed
+            if (!mbar_wait_warp(&kfree[kb], ((j >> 1) & 1) ^ 1, abort_flag, a.st)) {
                 ok = false;
                 break;
             }
             bool vrow;
             if (j < n_wt) {
-                // window row: RMSNorm over all 576 channels (the two halves meet by shuffle),
-                // RoPE at its own position on 512..575
-                const int wr = j * kTK + r;
+                // window row: RMSNorm over all 576 channels (the four quarters meet by
+                // shuffle), RoPE at its own position on 512..575
+                const int wr = j * kTK + kr;
                 const int64_t p = (int64_t)w0 + wr;
                 vrow = wr < n_win;
                 if (vrow && p < a.kv_pos0[b]) {
                     vrow = false;
-                    if (hf == 0) flag(a.st, CSA_DEV_OOB);
+                    if (qt == 0) flag(a.st, CSA_DEV_OOB);
                 }
                 const uint16_t* src =
                     vrow ? a.kv + (a.kv_off[b] + p - a.kv_pos0[b]) * (int64_t)kD : nullptr;
-                // pass 1: the raw row into the tile (18 loads in flight) and its sum of squares
+                // pass 1: my quarter of the raw row into the tile (18 loads in flight) and its
+                // sum of squares
                 float ss = 0.f;
-#pragma unroll
-                for (int half = 0; half < 2; half++) {
+                {
                     uint4 u[18];
 #pragma unroll
                     for (int c = 0; c < 18; c++)
-                        u[c] = vrow ? *reinterpret_cast<const uint4*>(src + 288 * hf + 144 * half + 8 * c)
+                        u[c] = vrow ? *reinterpret_cast<const uint4*>(src + 144 * qt + 8 * c)
                                     : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
                     for (int c = 0; c < 18; c++) {
@@ -323,18 +346,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                             const float2 f = bf16x2_to_f32(w[z]);
                             ss += f.x * f.x + f.y * f.y;
                         }
-                        put8(sK, r, 288 * hf + 144 * half + 8 * c, u[c]);
+                        *cell8(tile, kKBlk, kr, 144 * qt + 8 * c) = u[c];
                     }
                 }
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                ss += __shfl_xor_sync(0xffffffffu, ss, 2);
                 const float rn = rsqrtf(ss / (float)kD + a.eps);
                 // pass 2, in place in shared memory: normalise, RoPE at the row's position
                 if (vrow) {
-#pragma unroll 4
-                    for (int c = 0; c < 36; c++) {
-                        const int d0 = 288 * hf + 8 * c;
-                        uint4* cell = reinterpret_cast<uint4*>(sK + (d0 >> 6) * kBlk + swz(r, (d0 & 63) >> 3));
-                        const uint4 u = *cell;
+#pragma unroll 3
+                    for (int c = 0; c < 18; c++) {
+                        const int d0 = 144 * qt + 8 * c;
+                        uint4* cl = cell8(tile, kKBlk, kr, d0);
+                        const uint4 u = *cl;
                         const uint32_t wi[4] = {u.x, u.y, u.z, u.w};
                         uint32_t w[4];
 #pragma unroll
@@ -354,89 +378,98 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                             }
                             w[z] = pack_bf16x2(f.x, f.y);
                         }
-                        *cell = make_uint4(w[0], w[1], w[2], w[3]);
+                        *cl = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
             } else {
                 vrow = ex_valid;
-                // this thread's copies, then its partner's (the scales) are visible
+                // this thread's copies, then its row partners' (the scales) are visible
                 asm volatile("cp.async.wait_group 0;" ::: "memory");
                 __syncwarp();
-                const float* scl = reinterpret_cast<const float*>(myraw + 512);
-                const float sc0 = vrow ? scl[2 * hf] : 0.f, sc1 = vrow ? scl[2 * hf + 1] : 0.f;
+                const float sc = vrow ? reinterpret_cast<const float*>(myraw + 512)[qt] : 0.f;
 #pragma unroll 4
-                for (int u = 0; u < 16; u++) {
+                for (int u = 0; u < 8; u++) {
                     uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-                    if (vrow)
-                        dequant16(*reinterpret_cast<const uint4*>(myraw + 256 * hf + 16 * u),
-                                  u < 8 ? sc0 : sc1, lo, hi);
-                    const int d0 = 256 * hf + 16 * u;
-                    put8(sK, r, d0, lo);
-                    put8(sK, r, d0 + 8, hi);
+                    if (vrow) dequant16(*reinterpret_cast<const uint4*>(myraw + 128 * qt + 16 * u), sc, lo, hi);
+                    const int d0 = 128 * qt + 16 * u;
+                    *cell8(tile, kKBlk, kr, d0) = lo;
+                    *cell8(tile, kKBlk, kr, d0 + 8) = hi;
                 }
 #pragma unroll
-                for (int u = 0; u < 4; u++)
-                    put8(sK, r, 512 + 32 * hf + 8 * u,
-                         vrow ? *reinterpret_cast<const uint4*>(myraw + 528 + 64 * hf + 16 * u)
-                              : make_uint4(0u, 0u, 0u, 0u));
-                // the raw slot is read: the partner may overwrite its half with the next row
+                for (int u = 0; u < 2; u++)
+                    *cell8(tile, kKBlk, kr, 512 + 16 * qt + 8 * u) =
+                        vrow ? *reinterpret_cast<const uint4*>(myraw + 528 + 32 * qt + 16 * u)
+                             : make_uint4(0u, 0u, 0u, 0u);
+                // the raw slot is read: the row partners may overwrite it with the next row
                 __syncwarp();
             }
-            // valid keys of the tile: this warp's 16 rows (even lanes carry them)
-            const uint32_t bal = __ballot_sync(0xffffffffu, vrow && hf == 0);
-            uint32_t m16 = 0;
+            // valid keys of the tile: this warp's 8 rows (lanes 0, 4, ..., 28 carry them)
+            const uint32_t bal = __ballot_sync(0xffffffffu, vrow && qt == 0);
+            uint32_t m8 = 0;
 #pragma unroll
-            for (int i = 0; i < 16; i++) m16 |= ((bal >> (2 * i)) & 1u) << i;
-            if (lane == 0) smask[(j & 1) * 4 + warp] = (uint16_t)m16;
+            for (int i = 0; i < 8; i++) m8 |= ((bal >> (4 * i)) & 1u) << i;
+            if (lane == 0) smask[kb * 4 + warp] = (uint8_t)m8;
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(kfull);
-            // the next entry tile's bytes in flight while this one is used
+            if (lane == 0) mbar_arrive(&kfull[kb]);
+            // the next entry tile's rows in flight while this one is used
             if (j + 1 >= n_wt && j + 1 < ntiles)
-                ex_valid = fetch_entry(a, sidx, (j + 1 - n_wt) * kTK + r, n_vis, row0, hf, myraw);
+                ex_valid = fetch_entry(a, sidx, (j + 1 - n_wt) * kTK + kr, n_vis, row0, qt, myraw);
         }
     } else if (warp == 4) {
         if (lane == 0 && ntiles > 0) {
             // ---------------- MMA issuer ----------------
+            // S of a tile is issued before the P V of the previous one, so the softmax of
+            // one tile overlaps the tensor work of its neighbours
             bool ok = mbar_wait(qfull, 0, abort_flag, a.st);
             tc_fence_after();
-            for (int j = 0; j < ntiles && ok; j++) {
-                const int sb = j & 1;
-                if (!mbar_wait(kfull, j & 1, abort_flag, a.st) ||
-                    !mbar_wait(&sfree[sb], ((j >> 1) & 1) ^ 1, abort_flag, a.st)) {
-                    ok = false;
-                    break;
-                }
+            auto issue_s = [&](int j) -> bool {
+                const int kb = j & 1;
+                if (!mbar_wait(&kfull[kb], (j >> 1) & 1, abort_flag, a.st) ||
+                    !mbar_wait(&sfree[kb], ((j >> 1) & 1) ^ 1, abort_flag, a.st))
+                    return false;
                 tc_fence_after();
-                const uint32_t ds = tmem + kColS + (uint32_t)(sb * 64);
+                const uint32_t ds = tmem + kColS + (uint32_t)(kb * kTK);
+                const uint8_t* tile = sK + kb * kKBytes;
 #pragma unroll 1
-                for (int kb = 0; kb < kNB; kb++) {
-                    const uint64_t ad = smem_desc_k_sw128(sQ + kb * kBlk);
-                    const uint64_t bd = smem_desc_k_sw128(sK + kb * kBlk);
+                for (int cb = 0; cb < kNB; cb++) {
+                    const uint64_t ad = smem_desc_k_sw128(sQ + cb * kQBlk);
+                    const uint64_t bd = smem_desc_k_sw128(tile + cb * kKBlk);
 #pragma unroll
                     for (int kk = 0; kk < 4; kk++)   // K = 16 bf16 = 32 bytes per MMA
-                        mma_f16(ds, ad + 2 * kk, bd + 2 * kk, kIdescS, (kb | kk) ? 1u : 0u);
+                        mma_f16(ds, ad + 2 * kk, bd + 2 * kk, kIdescS, (cb | kk) ? 1u : 0u);
                 }
-                mma_commit(&sfull[sb]);
-                if (!mbar_wait(&pfull[sb], (j >> 1) & 1, abort_flag, a.st)) {
+                mma_commit(&sfull[kb]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; j < ntiles && ok; j++) {
+                if (j + 1 < ntiles && !issue_s(j + 1)) {
+                    ok = false;
+                    break;
+                }
+                const int kb = j & 1;
+                if (!mbar_wait(&pfull[kb], (j >> 1) & 1, abort_flag, a.st)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t pa = smem_desc_k_sw128(sP + sb * kPBytes);
+                const uint64_t pa = smem_desc_k_sw128(sP + kb * kPBytes);
+                const uint8_t* tile = sK + kb * kKBytes;
 #pragma unroll
-                for (int kk = 0; kk < 4; kk++) {   // 16 keys per MMA
+                for (int kk = 0; kk < kTK / 16; kk++) {   // 16 keys per MMA
                     const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-                    mma_f16(tmem + kColO, pa + 2 * kk, desc_mn(sK + kk * 2048, kBlk), kIdescPV, acc);
+                    mma_f16(tmem + kColO, pa + 2 * kk, desc_mn(tile + kk * 2048, kKBlk), kIdescPV, acc);
                     mma_f16(tmem + kColO + (16u << 16), pa + 2 * kk,
-                            desc_mn(sK + 4 * kBlk + kk * 2048, kBlk), kIdescPV, acc);
-                    mma_f16(tmem + kColOr, pa + 2 * kk, desc_mn(sK + 8 * kBlk + kk * 2048, kBlk),
+                            desc_mn(tile + 4 * kKBlk + kk * 2048, kKBlk), kIdescPV, acc);
+                    mma_f16(tmem + kColOr, pa + 2 * kk, desc_mn(tile + 8 * kKBlk + kk * 2048, kKBlk),
                             kIdescPVr, acc);
                 }
-                mma_commit(kfree);
-                mma_commit(&pfree[sb]);
+                mma_commit(&kfree[kb]);
+                mma_commit(&pfree[kb]);
                 mma_commit(pvdone);
             }
+            if (ok) mma_commit(odone);
             // drain: all issued MMAs complete before TMEM is released
             mma_commit(drain);
             mbar_drain(drain, 0, a.st);
@@ -456,19 +489,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 break;
             }
             tc_fence_after();
-            uint32_t sv[64];
-            tmem_ld64(tmem + kColS + (uint32_t)(sb * 64) + lane_base, sv);
+            uint32_t sv[kTK];
+            tmem_ld32(tmem + kColS + (uint32_t)(sb * kTK) + lane_base, sv);
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sfree[sb]);
-            const uint16_t* mk = smask + sb * 4;
-            const uint32_t mlo = (uint32_t)mk[0] | ((uint32_t)mk[1] << 16);
-            const uint32_t mhi = (uint32_t)mk[2] | ((uint32_t)mk[3] << 16);
+            const uint8_t* mk = smask + sb * 4;
+            const uint32_t mbits = (uint32_t)mk[0] | ((uint32_t)mk[1] << 8) |
+                                   ((uint32_t)mk[2] << 16) | ((uint32_t)mk[3] << 24);
             float tmax = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 64; c++) {
-                const bool on = mine && (((c < 32 ? mlo >> c : mhi >> (c - 32)) & 1u) != 0);
+            for (int c = 0; c < kTK; c++) {
+                const bool on = mine && ((mbits >> c) & 1u) != 0;
                 const float xv = on ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
                 sv[c] = __float_as_uint(xv);
                 tmax = fmaxf(tmax, xv);
@@ -507,9 +540,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 mref = mnew;
             }
             float rs = 0.f;
-            uint32_t pk[32];
+            uint32_t pk[kTK / 2];
 #pragma unroll
-            for (int c = 0; c < 32; c++) {
+            for (int c = 0; c < kTK / 2; c++) {
                 const float x0 = __uint_as_float(sv[2 * c]), x1 = __uint_as_float(sv[2 * c + 1]);
                 const float p0 = x0 == -INFINITY ? 0.f : exp2f(x0 - mref);
                 const float p1 = x1 == -INFINITY ? 0.f : exp2f(x1 - mref);
@@ -524,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             if (mine) {
                 uint8_t* prow = sP + sb * kPBytes;
 #pragma unroll
-                for (int c = 0; c < 8; c++)
+                for (int c = 0; c < kTK / 8; c++)
                     *reinterpret_cast<uint4*>(prow + swz(hl, c)) =
                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
             }
@@ -532,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             __syncwarp();
             if (lane == 0) mbar_arrive(&pfull[sb]);
         }
-        if (ok && ntiles > 0) ok = mbar_wait_warp(pvdone, (ntiles - 1) & 1, abort_flag, a.st);
+        if (ok && ntiles > 0) ok = mbar_wait_warp(odone, 0, abort_flag, a.st);
         if (ok && ntiles > 0) {
             tc_fence_after();
             // o = O 2^(mref - M) / (2^(sink - M) + l 2^(mref - M)),  M = max(mref, sink)
@@ -593,8 +626,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     }
 }
 
-constexpr size_t kSmemBytes = 1024 + kQBytes + kKBytes + 2 * kPBytes + 8 * 2 + 5 * 32 * 4 +
-                              kMaxK * 4 + kTK * kRowBytes + 13 * 8 + 16;
+static_assert(kOffK == kQBytes && kOffP == kOffK + 2 * kKBytes &&
+                  kOffRaw == kOffP + 2 * kPBytes && kOffMask == kOffRaw + kTK * kRowBytes,
+              "layout");
+constexpr size_t kSmemBytes = 1024 + kOffEnd;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 }  // namespace
