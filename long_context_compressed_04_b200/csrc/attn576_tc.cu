@@ -4,9 +4,13 @@
 // window, with the attention sink and partial / inverse RoPE ("DeepSeek-V4 深度分析报告"
 // 2.1 CSA and "其他注意力技术细节").
 //
-// One CTA per (query, group of 64 heads).  The keys of the query are tiles of 32: the
-// window's raw rows first (RMSNormed and RoPEd here), then the selected entries; two key
-// buffers let one tile be built while the previous one is in the tensor cores.
+// One cluster of 4 CTAs per (query, group of 64 heads).  The keys of the query are tiles
+// of 32 -- the window's raw rows first (RMSNormed and RoPEd here), then the selected entries
+// -- dealt to the ranks in turn (tile j to rank j mod 4).  Each rank ends with an fp32
+// partial state per head (running maximum, sum, unnormalised O) and stores it straight
+// into the shared memory of the rank that finishes that head (16 heads each, posted
+// st.shared::cluster); each rank combines its heads in rank order, the sink first.  Two
+// key buffers let one tile be built while the previous one is in the tensor cores.
 //   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once; per
 //              tile, 4 threads per key row dequantize the gathered FP8 row (or normalise the
 //              raw window row) into bf16, 128-byte swizzled, 9 blocks of 64 channels; the
@@ -21,7 +25,8 @@
 //   warps 5-8  online softmax in the log2 domain, one head row per lane: P as bf16 into
 //              shared memory; the running maximum is a reference that moves only when a
 //              tile's maximum exceeds it by 2^8, and then the head's O row in TMEM is
-//              rescaled; finally the sink, the normalisation, inverse RoPE and the store.
+//              rescaled; finally the partial states across the cluster, and for this
+//              rank's heads the combine, the sink, inverse RoPE and the store.
 // A 64 x 576 fp32 accumulator takes 320 TMEM columns, and the query's Q tile (72 KB) fills
 // a third of shared memory: hence 64 heads per CTA and two key buffers of 32 rows.
 // All waits are bounded (timeout -> CSA_DEV_TIMEOUT, drain, free TMEM, return).  A query's
@@ -53,6 +58,8 @@ constexpr uint32_t kColOr = 256;         // O channels 512-575 (lanes 0-15)
 constexpr uint32_t kColS = 320;          // S buffers at 320 and 352 (lanes 0-15)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxK = 2048;
+constexpr int kCl = 4;                   // CTAs per (query, head group)
+constexpr int kHO = kHC / kCl;           // heads finished by each rank
 // shared-memory layout (byte offsets from the 1024-aligned base)
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kNB * 64 * 128;            // after Q (72 KB)
@@ -62,7 +69,11 @@ constexpr int kOffMask = kOffRaw + 32 * 656;
 constexpr int kOffRope = kOffMask + 16;
 constexpr int kOffIdx = kOffRope + 5 * 32 * 4;
 constexpr int kOffBars = kOffIdx + kMaxK * 4;
-constexpr int kOffEnd = kOffBars + 16 * 8 + 16;
+constexpr int kOffEnd = kOffBars + 18 * 8 + 16;
+// the partial states of this rank's heads from every rank, [kCl][kHO][576] O then
+// [kCl][2][kHO] m, l, over Q, the key, P and staging buffers once this rank's MMAs are done
+constexpr int kRecvO = kCl * kHO * 576;
+static_assert((kRecvO + kCl * 2 * kHO) * 4 <= kOffMask, "receive buffer");
 static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles on 1024 B");
 static_assert(kOffRaw % 16 == 0 && kOffIdx % 16 == 0 && kOffBars % 8 == 0, "alignment");
 
@@ -205,12 +216,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                                      // previous tile's: never more than one phase behind)
     uint64_t* odone = bars + 14;     // MMA commit after the last P V (one phase)
     uint64_t* drain = bars + 15;
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 16);
+    uint64_t* recv_ready = bars + 16;   // every rank's MMAs are done: 4 x cluster
+    uint64_t* cpart_full = bars + 17;   // every rank's partials are in: 4 x cluster
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 18);
+    float* recv = reinterpret_cast<float*>(smem + kOffQ);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = a.H / kHC;
-    const int qi = blockIdx.x / G, g = blockIdx.x - qi * G;
+    const int rank = (int)cluster_ctarank();
+    const int item = blockIdx.x / kCl;
+    const int qi = item / G, g = item - qi * G;
     // the query (the same decision in every thread)
     const int b = a.q_seq[qi];
     const int t = a.q_pos[qi];
@@ -228,9 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         mbar_init(pvdone, 1);
         mbar_init(odone, 1);
         mbar_init(drain, 1);
+        mbar_init(recv_ready, 4 * kCl);
+        mbar_init(cpart_full, 4 * kCl);
         *abort_flag = 0;
         mbar_fence_init();
-        if (!valid && g == 0) flag(a.st, CSA_DEV_OOB);
+        if (!valid && g == 0 && rank == 0) flag(a.st, CSA_DEV_OOB);
     }
     if (threadIdx.x < 32 && valid) {
         // per query: cos / sin of every RoPE pair at t and at the window's first position
@@ -258,6 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     }
     tc_fence_before();
     __syncthreads();
+    // the cluster's barriers are initialised before any rank arrives on another's
+    cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_smem;
 
@@ -268,6 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     const int n_wt = (a.W + kTK - 1) / kTK;          // window tiles (masked past n_win)
     const int n_et = (a.k + kTK - 1) / kTK;          // selected-entry tiles
     const int ntiles = valid ? n_wt + n_et : 0;
+    // this rank's tiles: global tile rank + kCl j for local j < nloc
+    const int nloc = ntiles > rank ? (ntiles - rank + kCl - 1) / kCl : 0;
 
     if (warp < 4) {
         // ---------------- loaders ----------------
@@ -307,8 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         const int kr = tid >> 2, qt = tid & 3;
         uint8_t* myraw = sRaw + kr * kRowBytes;
         bool ex_valid = false;
-        if (n_wt == 0 && ntiles > 0) ex_valid = fetch_entry(a, sidx, kr, n_vis, row0, qt, myraw);
-        for (int j = 0; j < ntiles && ok; j++) {
+        if (nloc > 0 && rank >= n_wt)
+            ex_valid = fetch_entry(a, sidx, (rank - n_wt) * kTK + kr, n_vis, row0, qt, myraw);
+        for (int j = 0; j < nloc && ok; j++) {
+            const int jg = rank + kCl * j;   // global tile
             const int kb = j & 1;
             uint8_t* tile = sK + kb * kKBytes;
             // this key buffer is free once the P V of the tile two back has completed
@@ -317,10 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 break;
             }
             bool vrow;
-            if (j < n_wt) {
+            if (jg < n_wt) {
                 // window row: RMSNorm over all 576 channels (the four quarters meet by
                 // shuffle), RoPE at its own position on 512..575
-                const int wr = j * kTK + kr;
+                const int wr = jg * kTK + kr;
                 const int64_t p = (int64_t)w0 + wr;
                 vrow = wr < n_win;
                 if (vrow && p < a.kv_pos0[b]) {
@@ -413,11 +437,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             __syncwarp();
             if (lane == 0) mbar_arrive(&kfull[kb]);
             // the next entry tile's rows in flight while this one is used
-            if (j + 1 >= n_wt && j + 1 < ntiles)
-                ex_valid = fetch_entry(a, sidx, (j + 1 - n_wt) * kTK + kr, n_vis, row0, qt, myraw);
+            if (j + 1 < nloc && jg + kCl >= n_wt)
+                ex_valid = fetch_entry(a, sidx, (jg + kCl - n_wt) * kTK + kr, n_vis, row0, qt, myraw);
         }
     } else if (warp == 4) {
-        if (lane == 0 && ntiles > 0) {
+        if (lane == 0 && nloc > 0) {
             // ---------------- MMA issuer ----------------
             // S of a tile is issued before the P V of the previous one, so the softmax of
             // one tile overlaps the tensor work of its neighbours
@@ -443,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 return true;
             };
             if (ok) ok = issue_s(0);
-            for (int j = 0; j < ntiles && ok; j++) {
-                if (j + 1 < ntiles && !issue_s(j + 1)) {
+            for (int j = 0; j < nloc && ok; j++) {
+                if (j + 1 < nloc && !issue_s(j + 1)) {
                     ok = false;
                     break;
                 }
@@ -482,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         float mref = -INFINITY, lrun = 0.f;
         bool ok = true;
-        for (int j = 0; j < ntiles && ok; j++) {
+        for (int j = 0; j < nloc && ok; j++) {
             const int sb = j & 1;
             if (!mbar_wait_warp(&sfull[sb], (j >> 1) & 1, abort_flag, a.st)) {
                 ok = false;
@@ -565,56 +589,99 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             __syncwarp();
             if (lane == 0) mbar_arrive(&pfull[sb]);
         }
-        if (ok && ntiles > 0) ok = mbar_wait_warp(odone, 0, abort_flag, a.st);
-        if (ok && ntiles > 0) {
-            tc_fence_after();
-            // o = O 2^(mref - M) / (2^(sink - M) + l 2^(mref - M)),  M = max(mref, sink)
-            const int h = kHC * g + hl;
-            const float sk = a.sink[h] * kLog2e;
-            const float M = fmaxf(mref, sk);
-            float inv = 0.f;
-            if (M != -INFINITY) {
-                const float so = mref == -INFINITY ? 0.f : exp2f(mref - M);
-                const float L = lrun * so + (sk == -INFINITY ? 0.f : exp2f(sk - M));
-                inv = L > 0.f ? so / L : 0.f;
+        if (ok && nloc > 0) ok = mbar_wait_warp(odone, 0, abort_flag, a.st);
+        if (ntiles > 0) {
+            // ---- partial states across the cluster ----
+            // my MMAs are done: my Q / key / P / staging buffers may take the partials
+            if (ok) {
+                tc_fence_after();
+                __syncwarp();
+                if (lane == 0)
+                    for (int rr = 0; rr < kCl; rr++) mbar_arrive_cluster(mapa(recv_ready, (uint32_t)rr));
+                ok = mbar_wait_cluster_warp(recv_ready, 0, abort_flag, a.st);
             }
-            inv = __shfl_sync(0xffffffffu, inv, lane & 15);
-            uint16_t* orow = a.out + ((int64_t)qi * a.H + h) * kD;
-            // channels 0-255 (lanes 0-15) and 256-511 (lanes 16-31)
+            if (ok) {
+                // head hl goes to rank hl / kHO (this warp's 16 heads: rank `quarter`)
+                const int own = hl / kHO, lh = hl - own * kHO;
+                float* recv_ml = recv + kRecvO;
+                const uint32_t dst = mapa(recv + (rank * kHO + lh) * 576 + (mine ? 0 : 256), (uint32_t)own);
 #pragma unroll 1
-            for (int cc = 0; cc < 16; cc++) {
-                uint32_t ov[16];
-                tmem_ld16(tmem + kColO + 16u * cc + lane_base, ov);
-                tmem_ld_wait();
-                uint32_t w[8];
+                for (int cc = 0; cc < 20; cc++) {
+                    // 16 columns at a time: 0-255 (both lane halves), then 256-319 (lanes 0-15)
+                    const uint32_t col = cc < 16 ? kColO + 16u * cc : kColOr + 16u * (cc - 16);
+                    uint32_t ov[16];
+                    if (nloc > 0) {
+                        tmem_ld16(tmem + col + lane_base, ov);
+                        tmem_ld_wait();
+                    } else {
 #pragma unroll
-                for (int z = 0; z < 8; z++)
-                    w[z] = pack_bf16x2(__uint_as_float(ov[2 * z]) * inv, __uint_as_float(ov[2 * z + 1]) * inv);
-                uint4* dst = reinterpret_cast<uint4*>(orow + (mine ? 0 : 256) + 16 * cc);
-                dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            }
-            // channels 512-575 (lanes 0-15): inverse RoPE (rotation by -t)
-#pragma unroll 1
-            for (int cc = 0; cc < 4; cc++) {
-                uint32_t ov[16];
-                tmem_ld16(tmem + kColOr + 16u * cc + lane_base, ov);
-                tmem_ld_wait();
-                if (mine) {
-                    uint32_t w[8];
-#pragma unroll
-                    for (int z = 0; z < 8; z++) {
-                        const int pj = 8 * cc + z;
-                        const float x = __uint_as_float(ov[2 * z]) * inv;
-                        const float y = __uint_as_float(ov[2 * z + 1]) * inv;
-                        w[z] = pack_bf16x2(x * rqc[pj] + y * rqs[pj], y * rqc[pj] - x * rqs[pj]);
+                        for (int z = 0; z < 16; z++) ov[z] = 0u;
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(orow + 512 + 16 * cc);
-                    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-                    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                    if (cc < 16 || mine) {
+                        // lanes 0-15: channels 0-255 then 512-575; lanes 16-31: 256-511
+                        const uint32_t off = (cc < 16 ? 16u * cc : 512u + 16u * (cc - 16)) * 4u;
+#pragma unroll
+                        for (int z = 0; z < 16; z += 4)
+                            st_cluster_f4(dst + off + 4u * z,
+                                          make_float4(__uint_as_float(ov[z]), __uint_as_float(ov[z + 1]),
+                                                      __uint_as_float(ov[z + 2]), __uint_as_float(ov[z + 3])));
+                    }
+                }
+                if (mine) {
+                    st_cluster_f32(mapa(recv_ml + (2 * rank) * kHO + lh, (uint32_t)own), mref);
+                    st_cluster_f32(mapa(recv_ml + (2 * rank + 1) * kHO + lh, (uint32_t)own), lrun);
+                }
+                tc_fence_before();
+                fence_cluster();
+                __syncwarp();
+                if (lane == 0)
+                    for (int rr = 0; rr < kCl; rr++) mbar_arrive_cluster(mapa(cpart_full, (uint32_t)rr));
+                ok = mbar_wait_cluster_warp(cpart_full, 0, abort_flag, a.st);
+            }
+            if (named_barrier_and(2, 128, ok)) {
+                // this rank's heads: (head, 4 channels) per work unit, ranks in order, sink first
+                const float* recv_ml = recv + kRecvO;
+                const int i = threadIdx.x - 160;
+#pragma unroll 1
+                for (int w = i; w < kHO * (576 / 4); w += 128) {
+                    const int lh = w / (576 / 4), c4 = (w - lh * (576 / 4)) * 4;
+                    const int h = kHC * g + rank * kHO + lh;
+                    const float sk = a.sink[h] * kLog2e;
+                    float M = sk;
+#pragma unroll
+                    for (int rr = 0; rr < kCl; rr++) M = fmaxf(M, recv_ml[(2 * rr) * kHO + lh]);
+                    float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int rr = 0; rr < kCl; rr++) {
+                        const float mr = recv_ml[(2 * rr) * kHO + lh];
+                        const float wgt = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
+                        L = fmaf(wgt, recv_ml[(2 * rr + 1) * kHO + lh], L);
+                        const float4 v = *reinterpret_cast<const float4*>(recv + (rr * kHO + lh) * 576 + c4);
+                        acc.x = fmaf(wgt, v.x, acc.x);
+                        acc.y = fmaf(wgt, v.y, acc.y);
+                        acc.z = fmaf(wgt, v.z, acc.z);
+                        acc.w = fmaf(wgt, v.w, acc.w);
+                    }
+                    if (L > 0.f) {
+                        acc.x /= L;
+                        acc.y /= L;
+                        acc.z /= L;
+                        acc.w /= L;
+                    } else {
+                        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    if (c4 >= kD - kRopeDims) {
+                        // rotation by -t: (x, y) -> (x cos + y sin, y cos - x sin)
+                        const int pj = (c4 - (kD - kRopeDims)) >> 1;
+                        const float c0 = rqc[pj], s0 = rqs[pj], c1 = rqc[pj + 1], s1 = rqs[pj + 1];
+                        acc = make_float4(acc.x * c0 + acc.y * s0, acc.y * c0 - acc.x * s0,
+                                          acc.z * c1 + acc.w * s1, acc.w * c1 - acc.z * s1);
+                    }
+                    *reinterpret_cast<uint2*>(a.out + ((int64_t)qi * a.H + h) * kD + c4) =
+                        make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
                 }
             }
-            tc_fence_before();
         }
     }
 
@@ -624,6 +691,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    // no rank leaves while another may still store into its shared memory
+    cluster_sync_all();
 }
 
 static_assert(kOffK == kQBytes && kOffP == kOffK + 2 * kKBytes &&
@@ -668,8 +737,8 @@ cudaError_t launch_attn576_tc(const AttnArgs& aa, int Q, cudaStream_t stream) {
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     LaunchScope scope(kKAttn576Tc, stream);
-    return launch_pdl(attn576_tc_kernel, dim3(Q * (aa.H / kHC)), dim3(kThreads), kSmemBytes,
-                      stream, a);
+    return launch_pdl_cluster(attn576_tc_kernel, dim3(Q * (aa.H / kHC) * kCl), dim3(kThreads),
+                              kSmemBytes, stream, kCl, a);
 }
 
 }  // namespace csa
