@@ -62,20 +62,22 @@ constexpr int kCl = 4;                   // CTAs per (query, head group)
 constexpr int kHO = kHC / kCl;           // heads finished by each rank
 // shared-memory layout (byte offsets from the 1024-aligned base)
 constexpr int kOffQ = 0;
+constexpr int kKBuf = 3;                 // key buffers
 constexpr int kOffK = kOffQ + kNB * 64 * 128;            // after Q (72 KB)
-constexpr int kOffP = kOffK + 2 * kNB * 32 * 128;        // after two key buffers
-constexpr int kOffRaw = kOffP + 2 * 64 * 128;            // after two P buffers
-constexpr int kOffMask = kOffRaw + 32 * 656;
+constexpr int kOffP = kOffK + kKBuf * kNB * 32 * 128;    // after the key buffers
+constexpr int kOffMask = kOffP + 2 * 64 * 128;           // after two P buffers
 constexpr int kOffRope = kOffMask + 16;
 constexpr int kOffIdx = kOffRope + 5 * 32 * 4;
-constexpr int kOffBars = kOffIdx + kMaxK * 4;
-constexpr int kOffEnd = kOffBars + 18 * 8 + 16;
+constexpr int kOffRot = kOffIdx + kMaxK * 4;              // [32 rows][32 pairs] cos, sin
+constexpr int kOffWt = kOffRot + 32 * 32 * 8;              // [16 heads][kCl + 1] weights, L
+constexpr int kOffBars = kOffWt + 16 * 8 * 4;
+constexpr int kOffEnd = kOffBars + 22 * 8 + 16;
 // the partial states of this rank's heads from every rank, [kCl][kHO][576] O then
 // [kCl][2][kHO] m, l, over Q, the key, P and staging buffers once this rank's MMAs are done
 constexpr int kRecvO = kCl * kHO * 576;
 static_assert((kRecvO + kCl * 2 * kHO) * 4 <= kOffMask, "receive buffer");
 static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles on 1024 B");
-static_assert(kOffRaw % 16 == 0 && kOffIdx % 16 == 0 && kOffBars % 8 == 0, "alignment");
+static_assert(kOffIdx % 16 == 0 && kOffBars % 8 == 0, "alignment");
 
 struct A576Args {
     const uint16_t* q;
@@ -150,38 +152,37 @@ __device__ __forceinline__ void dequant16(uint4 c, float sc, uint4& lo, uint4& h
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sm100::smem_addr(dst)),
-                 "l"(src)
-                 : "memory");
-}
+// One loader thread's quarter of a selected entry row: fp8 channels [128 qt, 128 qt + 128)
+// with their scale, RoPE channels [16 qt, 16 qt + 16).
+struct EntryQuarter {
+    uint4 f[8];
+    uint4 rope[2];
+    float sc;
+    bool valid;
+};
 
-// Starts copying one loader thread's quarter of entry v of the query's index row (staged in
-// shared memory) into its raw row slot: fp8 channels [128 qt, 128 qt + 128), RoPE channels
-// [16 qt, 16 qt + 16), and (qt = 0) the four scales.  False for an invalid index (an
-// out-of-range one is flagged once per row).
-__device__ __forceinline__ bool fetch_entry(const A576Args& a, const int32_t* sidx, int v,
-                                            int n_vis, int64_t row0, int qt, uint8_t* raw) {
+// Loads entry v of the query's index row (staged in shared memory) into registers (flags an
+// out-of-range index once per row).
+__device__ __forceinline__ void fetch_entry(const A576Args& a, const int32_t* sidx, int v,
+                                            int n_vis, int64_t row0, int qt, EntryQuarter& x) {
     const int e = v < a.k ? sidx[v] : -1;
-    bool valid = false;
+    x.valid = false;
     if (e >= 0) {
         if (e < n_vis && row0 + e < a.ent_rows) {
-            valid = true;
+            x.valid = true;
         } else if (qt == 0) {
             flag(a.st, CSA_DEV_OOB);
         }
     }
-    if (valid) {
+    if (x.valid) {
         const uint8_t* er = a.entries + (row0 + e) * (int64_t)kRowBytes;
 #pragma unroll
-        for (int u = 0; u < 8; u++) cp_async16(raw + 128 * qt + 16 * u, er + 128 * qt + 16 * u);
+        for (int u = 0; u < 8; u++) x.f[u] = *reinterpret_cast<const uint4*>(er + 128 * qt + 16 * u);
 #pragma unroll
         for (int u = 0; u < 2; u++)
-            cp_async16(raw + 528 + 32 * qt + 16 * u, er + 528 + 32 * qt + 16 * u);
-        if (qt == 0) cp_async16(raw + 512, er + 512);
+            x.rope[u] = *reinterpret_cast<const uint4*>(er + 528 + 32 * qt + 16 * u);
+        x.sc = *reinterpret_cast<const float*>(er + 512 + 4 * qt);
     }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    return valid;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args a) {
@@ -193,32 +194,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
     uint8_t* sQ = smem + kOffQ;                           // [9][64 x 128 B]
-    uint8_t* sK = smem + kOffK;                           // [2][9][32 x 128 B]
+    uint8_t* sK = smem + kOffK;                           // [3][9][32 x 128 B]
     uint8_t* sP = smem + kOffP;                           // [2][64 x 128 B]
-    uint8_t* sRaw = smem + kOffRaw;                       // [32][656] next entry rows (16 B
-                                                          // aligned: cp.async destinations)
-    uint8_t* smask = smem + kOffMask;                     // [2][4] valid keys, 8 per warp
+    uint8_t* smask = smem + kOffMask;                     // [3][4] valid keys, 8 per warp
     float* rqc = reinterpret_cast<float*>(smem + kOffRope);   // [32] cos / sin of pair j at t
     float* rqs = rqc + 32;
     float* rf = rqs + 32;                                 // [32] frequency of pair j
     float* rwc = rf + 32;                                 // [32] cos / sin of pair j at w0
     float* rws = rwc + 32;
     int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);   // [kMaxK] the index row
+    float2* srot = reinterpret_cast<float2*>(smem + kOffRot);    // window RoPE rotations
+    float* swt = reinterpret_cast<float*>(smem + kOffWt);        // combine weights
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
     uint64_t* qfull = bars;          // 4 loader warps
-    uint64_t* kfull = bars + 1;      // [2] 4 loader warps
-    uint64_t* kfree = bars + 3;      // [2] MMA commit after the tile's P V
-    uint64_t* sfull = bars + 5;      // [2] MMA commit
-    uint64_t* sfree = bars + 7;      // [2] 4 softmax warps
-    uint64_t* pfull = bars + 9;      // [2] 4 softmax warps
-    uint64_t* pfree = bars + 11;     // [2] MMA commit
-    uint64_t* pvdone = bars + 13;    // MMA commit after every P V (a rescale waits for the
+    uint64_t* kfull = bars + 1;      // [3] 4 loader warps
+    uint64_t* kfree = bars + 4;      // [3] MMA commit after the tile's P V
+    uint64_t* sfull = bars + 7;      // [2] MMA commit
+    uint64_t* sfree = bars + 9;      // [2] 4 softmax warps
+    uint64_t* pfull = bars + 11;     // [2] 4 softmax warps
+    uint64_t* pfree = bars + 13;     // [2] MMA commit
+    uint64_t* pvdone = bars + 15;    // MMA commit after every P V (a rescale waits for the
                                      // previous tile's: never more than one phase behind)
-    uint64_t* odone = bars + 14;     // MMA commit after the last P V (one phase)
-    uint64_t* drain = bars + 15;
-    uint64_t* recv_ready = bars + 16;   // every rank's MMAs are done: 4 x cluster
-    uint64_t* cpart_full = bars + 17;   // every rank's partials are in: 4 x cluster
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 18);
+    uint64_t* odone = bars + 16;     // MMA commit after the last P V (one phase)
+    uint64_t* drain = bars + 17;
+    uint64_t* recv_ready = bars + 18;   // every rank's MMAs are done: 4 x cluster
+    uint64_t* cpart_full = bars + 19;   // every rank's partials are in: 4 x cluster
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 20);
     float* recv = reinterpret_cast<float*>(smem + kOffQ);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
@@ -233,9 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     const bool valid = b >= 0 && b < a.B && t >= 0 && (int64_t)t < a.seq_len[b];
     if (threadIdx.x == 0) {
         mbar_init(qfull, 4);
-        for (int i = 0; i < 2; i++) {
+        for (int i = 0; i < kKBuf; i++) {
             mbar_init(&kfull[i], 4);
             mbar_init(&kfree[i], 1);
+        }
+        for (int i = 0; i < 2; i++) {
             mbar_init(&sfull[i], 1);
             mbar_init(&sfree[i], 4);
             mbar_init(&pfull[i], 4);
@@ -327,16 +330,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         }
         // tiles: 4 threads per key row, quarter qt
         const int kr = tid >> 2, qt = tid & 3;
-        uint8_t* myraw = sRaw + kr * kRowBytes;
-        bool ex_valid = false;
-        if (nloc > 0 && rank >= n_wt)
-            ex_valid = fetch_entry(a, sidx, (rank - n_wt) * kTK + kr, n_vis, row0, qt, myraw);
+        EntryQuarter ex;
+        ex.valid = false;
+        if (nloc > 0 && rank >= n_wt) fetch_entry(a, sidx, (rank - n_wt) * kTK + kr, n_vis, row0, qt, ex);
         for (int j = 0; j < nloc && ok; j++) {
             const int jg = rank + kCl * j;   // global tile
-            const int kb = j & 1;
+            const int kb = j % kKBuf;
             uint8_t* tile = sK + kb * kKBytes;
-            // this key buffer is free once the P V of the tile two back has completed
-            if (!mbar_wait_warp(&kfree[kb], ((j >> 1) & 1) ^ 1, abort_flag, a.st)) {
+            // this key buffer is free once the P V of the tile kKBuf back has completed
+            if (!mbar_wait_warp(&kfree[kb], ((j / kKBuf) & 1) ^ 1, abort_flag, a.st)) {
                 ok = false;
                 break;
             }
@@ -376,6 +378,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
                 ss += __shfl_xor_sync(0xffffffffu, ss, 2);
                 const float rn = rsqrtf(ss / (float)kD + a.eps);
+                // rotations of the tile's 32 rows x 32 pairs, 8 per loader thread:
+                // angle (w0 + wr) f_j = w0 f_j (fp64 table) + wr f_j (< 128 rad, sincosf),
+                // combined by the addition formula
+#pragma unroll 1
+                for (int e = tid; e < kTK * 32; e += 128) {
+                    const int er = e >> 5, pj = e & 31;
+                    float sb_, cb_;
+                    sincosf((float)(jg * kTK + er) * rf[pj], &sb_, &cb_);
+                    srot[e] = make_float2(rwc[pj] * cb_ - rws[pj] * sb_, rws[pj] * cb_ + rwc[pj] * sb_);
+                }
+                asm volatile("bar.sync 3, 128;" ::: "memory");
                 // pass 2, in place in shared memory: normalise, RoPE at the row's position
                 if (vrow) {
 #pragma unroll 3
@@ -391,41 +404,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                             f.x *= rn;
                             f.y *= rn;
                             if (d0 >= kD - kRopeDims) {
-                                // angle (w0 + wr) f_j = w0 f_j (fp64 table) + wr f_j (< 128 rad,
-                                // sincosf), combined by the addition formula
-                                const int pj = (d0 - (kD - kRopeDims)) / 2 + z;
-                                float sb_, cb_;
-                                sincosf((float)wr * rf[pj], &sb_, &cb_);
-                                const float cs = rwc[pj] * cb_ - rws[pj] * sb_;
-                                const float sn = rws[pj] * cb_ + rwc[pj] * sb_;
-                                f = make_float2(f.x * cs - f.y * sn, f.x * sn + f.y * cs);
+                                const float2 cs = srot[kr * 32 + (d0 - (kD - kRopeDims)) / 2 + z];
+                                f = make_float2(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
                             }
                             w[z] = pack_bf16x2(f.x, f.y);
                         }
                         *cl = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 }
+                // every loader is done with this tile's rotations before the next tile's
+                asm volatile("bar.sync 3, 128;" ::: "memory");
             } else {
-                vrow = ex_valid;
-                // this thread's copies, then its row partners' (the scales) are visible
-                asm volatile("cp.async.wait_group 0;" ::: "memory");
-                __syncwarp();
-                const float sc = vrow ? reinterpret_cast<const float*>(myraw + 512)[qt] : 0.f;
-#pragma unroll 4
+                vrow = ex.valid;
+#pragma unroll
                 for (int u = 0; u < 8; u++) {
                     uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-                    if (vrow) dequant16(*reinterpret_cast<const uint4*>(myraw + 128 * qt + 16 * u), sc, lo, hi);
+                    if (vrow) dequant16(ex.f[u], ex.sc, lo, hi);
                     const int d0 = 128 * qt + 16 * u;
                     *cell8(tile, kKBlk, kr, d0) = lo;
                     *cell8(tile, kKBlk, kr, d0 + 8) = hi;
                 }
 #pragma unroll
                 for (int u = 0; u < 2; u++)
-                    *cell8(tile, kKBlk, kr, 512 + 16 * qt + 8 * u) =
-                        vrow ? *reinterpret_cast<const uint4*>(myraw + 528 + 32 * qt + 16 * u)
-                             : make_uint4(0u, 0u, 0u, 0u);
-                // the raw slot is read: the row partners may overwrite it with the next row
-                __syncwarp();
+                    *cell8(tile, kKBlk, kr, 512 + 16 * qt + 8 * u) = vrow ? ex.rope[u] : make_uint4(0u, 0u, 0u, 0u);
             }
             // valid keys of the tile: this warp's 8 rows (lanes 0, 4, ..., 28 carry them)
             const uint32_t bal = __ballot_sync(0xffffffffu, vrow && qt == 0);
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             if (lane == 0) mbar_arrive(&kfull[kb]);
             // the next entry tile's rows in flight while this one is used
             if (j + 1 < nloc && jg + kCl >= n_wt)
-                ex_valid = fetch_entry(a, sidx, (jg + kCl - n_wt) * kTK + kr, n_vis, row0, qt, myraw);
+                fetch_entry(a, sidx, (jg + kCl - n_wt) * kTK + kr, n_vis, row0, qt, ex);
         }
     } else if (warp == 4) {
         if (lane == 0 && nloc > 0) {
@@ -448,12 +449,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             bool ok = mbar_wait(qfull, 0, abort_flag, a.st);
             tc_fence_after();
             auto issue_s = [&](int j) -> bool {
-                const int kb = j & 1;
-                if (!mbar_wait(&kfull[kb], (j >> 1) & 1, abort_flag, a.st) ||
-                    !mbar_wait(&sfree[kb], ((j >> 1) & 1) ^ 1, abort_flag, a.st))
+                const int kb = j % kKBuf, sb = j & 1;
+                if (!mbar_wait(&kfull[kb], (j / kKBuf) & 1, abort_flag, a.st) ||
+                    !mbar_wait(&sfree[sb], ((j >> 1) & 1) ^ 1, abort_flag, a.st))
                     return false;
                 tc_fence_after();
-                const uint32_t ds = tmem + kColS + (uint32_t)(kb * kTK);
+                const uint32_t ds = tmem + kColS + (uint32_t)(sb * kTK);
                 const uint8_t* tile = sK + kb * kKBytes;
 #pragma unroll 1
                 for (int cb = 0; cb < kNB; cb++) {
@@ -463,7 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                     for (int kk = 0; kk < 4; kk++)   // K = 16 bf16 = 32 bytes per MMA
                         mma_f16(ds, ad + 2 * kk, bd + 2 * kk, kIdescS, (cb | kk) ? 1u : 0u);
                 }
-                mma_commit(&sfull[kb]);
+                mma_commit(&sfull[sb]);
                 return true;
             };
             if (ok) ok = issue_s(0);
@@ -472,13 +473,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                     ok = false;
                     break;
                 }
-                const int kb = j & 1;
-                if (!mbar_wait(&pfull[kb], (j >> 1) & 1, abort_flag, a.st)) {
+                const int kb = j % kKBuf, sb = j & 1;
+                if (!mbar_wait(&pfull[sb], (j >> 1) & 1, abort_flag, a.st)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t pa = smem_desc_k_sw128(sP + kb * kPBytes);
+                const uint64_t pa = smem_desc_k_sw128(sP + sb * kPBytes);
                 const uint8_t* tile = sK + kb * kKBytes;
 #pragma unroll
                 for (int kk = 0; kk < kTK / 16; kk++) {   // 16 keys per MMA
@@ -490,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                             kIdescPVr, acc);
                 }
                 mma_commit(&kfree[kb]);
-                mma_commit(&pfree[kb]);
+                mma_commit(&pfree[sb]);
                 mma_commit(pvdone);
             }
             if (ok) mma_commit(odone);
@@ -519,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sfree[sb]);
-            const uint8_t* mk = smask + sb * 4;
+            const uint8_t* mk = smask + (j % kKBuf) * 4;
             const uint32_t mbits = (uint32_t)mk[0] | ((uint32_t)mk[1] << 8) |
                                    ((uint32_t)mk[2] << 16) | ((uint32_t)mk[3] << 24);
             float tmax = -INFINITY;
@@ -606,22 +607,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 float* recv_ml = recv + kRecvO;
                 const uint32_t dst = mapa(recv + (rank * kHO + lh) * 576 + (mine ? 0 : 256), (uint32_t)own);
 #pragma unroll 1
-                for (int cc = 0; cc < 20; cc++) {
-                    // 16 columns at a time: 0-255 (both lane halves), then 256-319 (lanes 0-15)
-                    const uint32_t col = cc < 16 ? kColO + 16u * cc : kColOr + 16u * (cc - 16);
-                    uint32_t ov[16];
+                for (int cc = 0; cc < 5; cc++) {
+                    // 64 columns at a time: 0-255 (both lane halves), then 256-319 (lanes 0-15)
+                    const uint32_t col = cc < 4 ? kColO + 64u * cc : kColOr;
+                    uint32_t ov[64];
                     if (nloc > 0) {
-                        tmem_ld16(tmem + col + lane_base, ov);
+                        tmem_ld64(tmem + col + lane_base, ov);
                         tmem_ld_wait();
                     } else {
 #pragma unroll
-                        for (int z = 0; z < 16; z++) ov[z] = 0u;
+                        for (int z = 0; z < 64; z++) ov[z] = 0u;
                     }
-                    if (cc < 16 || mine) {
+                    if (cc < 4 || mine) {
                         // lanes 0-15: channels 0-255 then 512-575; lanes 16-31: 256-511
-                        const uint32_t off = (cc < 16 ? 16u * cc : 512u + 16u * (cc - 16)) * 4u;
+                        const uint32_t off = (cc < 4 ? 64u * cc : 512u) * 4u;
 #pragma unroll
-                        for (int z = 0; z < 16; z += 4)
+                        for (int z = 0; z < 64; z += 4)
                             st_cluster_f4(dst + off + 4u * z,
                                           make_float4(__uint_as_float(ov[z]), __uint_as_float(ov[z + 1]),
                                                       __uint_as_float(ov[z + 2]), __uint_as_float(ov[z + 3])));
@@ -639,24 +640,36 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 ok = mbar_wait_cluster_warp(cpart_full, 0, abort_flag, a.st);
             }
             if (named_barrier_and(2, 128, ok)) {
-                // this rank's heads: (head, 4 channels) per work unit, ranks in order, sink first
+                // this rank's heads; first the combine weights, one thread per head:
+                // M = max(sink, m_r), w_r = 2^(m_r - M), L = 2^(sink - M) + sum_r w_r l_r
                 const float* recv_ml = recv + kRecvO;
                 const int i = threadIdx.x - 160;
-#pragma unroll 1
+                if (i < kHO) {
+                    const float sk = a.sink[kHC * g + rank * kHO + i] * kLog2e;
+                    float M = sk;
+#pragma unroll
+                    for (int rr = 0; rr < kCl; rr++) M = fmaxf(M, recv_ml[(2 * rr) * kHO + i]);
+                    float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
+#pragma unroll
+                    for (int rr = 0; rr < kCl; rr++) {
+                        const float mr = recv_ml[(2 * rr) * kHO + i];
+                        const float wgt = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
+                        L = fmaf(wgt, recv_ml[(2 * rr + 1) * kHO + i], L);
+                        swt[i * 8 + rr] = wgt;
+                    }
+                    swt[i * 8 + kCl] = L;
+                }
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+                // then (head, 4 channels) per work unit: sum_r w_r O_r / L
+#pragma unroll 2
                 for (int w = i; w < kHO * (576 / 4); w += 128) {
                     const int lh = w / (576 / 4), c4 = (w - lh * (576 / 4)) * 4;
                     const int h = kHC * g + rank * kHO + lh;
-                    const float sk = a.sink[h] * kLog2e;
-                    float M = sk;
-#pragma unroll
-                    for (int rr = 0; rr < kCl; rr++) M = fmaxf(M, recv_ml[(2 * rr) * kHO + lh]);
-                    float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
+                    const float L = swt[lh * 8 + kCl];
                     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                     for (int rr = 0; rr < kCl; rr++) {
-                        const float mr = recv_ml[(2 * rr) * kHO + lh];
-                        const float wgt = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
-                        L = fmaf(wgt, recv_ml[(2 * rr + 1) * kHO + lh], L);
+                        const float wgt = swt[lh * 8 + rr];
                         const float4 v = *reinterpret_cast<const float4*>(recv + (rr * kHO + lh) * 576 + c4);
                         acc.x = fmaf(wgt, v.x, acc.x);
                         acc.y = fmaf(wgt, v.y, acc.y);
@@ -695,8 +708,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     cluster_sync_all();
 }
 
-static_assert(kOffK == kQBytes && kOffP == kOffK + 2 * kKBytes &&
-                  kOffRaw == kOffP + 2 * kPBytes && kOffMask == kOffRaw + kTK * kRowBytes,
+static_assert(kOffK == kQBytes && kOffP == kOffK + kKBuf * kKBytes &&
+                  kOffMask == kOffP + 2 * kPBytes,
               "layout");
 constexpr size_t kSmemBytes = 1024 + kOffEnd;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
