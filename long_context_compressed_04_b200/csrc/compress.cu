@@ -18,9 +18,12 @@ namespace csa {
 // Tokens of one entry are split over TG token groups (along the token axis) that walk
 // chunks of 8 tokens; a thread loads a chunk's 8 tokens x 4 channels at once (and the next
 // chunk's before reducing the current one), keeps an online softmax state per channel, and
-// the token groups merge their states in a fixed order through shared memory.
+// the token groups merge their states pairwise in a fixed tree through shared memory.  All
+// inputs (item lists, offsets, raw tokens, the positional bias) are read before the wait on
+// the previous kernel: no earlier libcsa kernel writes them, so in a PDL pipeline their
+// latency overlaps it; only the entry store needs the wait.
 constexpr int kChunkTok = 8;
-constexpr int kMaxMergeSlots = 480;   // (TG - 1) * channel lanes
+constexpr int kMaxMergeSlots = 640;   // TG * channel lanes
 
 struct Chunk {
     uint2 z[kChunkTok], v[kChunkTok];
@@ -41,8 +44,12 @@ __device__ __forceinline__ void load_chunk(const uint16_t* __restrict__ kv,
     }
 }
 
-template <int SPAN>
-__global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
+// NCH: chunks per token group (1 for CSA's 8 tokens, and for HCA's 128 tokens over 16
+// token groups; 4 for HCA over 4 token groups).  With one chunk the bias rows of the chunk
+// sit in registers next to its tokens; with several the next chunk's tokens do, and the
+// bias is read where it is used.
+template <int SPAN, int NCH>
+__global__ void __launch_bounds__(SPAN == 8 ? 160 : (NCH == 1 ? 512 : 640)) compress_kernel(
     const uint16_t* __restrict__ kv, const uint16_t* __restrict__ gate,
     const float* __restrict__ bias, const int64_t* __restrict__ seq_len,
     const int64_t* __restrict__ kv_off,
@@ -53,30 +60,23 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
     __shared__ float red[8];
     __shared__ float4 st_m[SPAN == 8 ? 1 : kMaxMergeSlots], st_d[SPAN == 8 ? 1 : kMaxMergeSlots],
         st_a[SPAN == 8 ? 1 : kMaxMergeSlots];
-    pdl_wait();   // entries may still be read by the previous step's attention
-    pdl_trigger();
     const int64_t it = blockIdx.x;
     const int b = item_seq[it];
     const int64_t i = item_ent[it];
-    if (b < 0 || b >= B || i < 0) {
-        if (threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
-        return;
-    }
+    bool ok = !(b < 0 || b >= B || i < 0);
     const int64_t first = (i + 1) * (int64_t)m - SPAN;
-    const int64_t pos0 = kv_pos0[b];
-    const int64_t row0 = kv_off[b];
+    const int64_t pos0 = ok ? kv_pos0[b] : 0;
+    const int64_t row0 = ok ? kv_off[b] : 0;
+    const int64_t erow = ok ? ent_off[b] + i : 0;
     // every pooled token must be stored: positions max(first, 0) .. (i+1)m-1
-    if ((first > 0 ? first : 0) < pos0 || (i + 1) * (int64_t)m > seq_len[b]) {
-        if (threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
-        return;
-    }
+    if (ok && ((first > 0 ? first : 0) < pos0 || (i + 1) * (int64_t)m > seq_len[b])) ok = false;
     const int cw = 32 * ((D / 4 + 31) / 32);     // channel lanes per token group
     const int TG = blockDim.x / cw;               // token groups
-    const int nch = SPAN / kChunkTok / TG;        // chunks per token group
+    constexpr int nch = NCH;                      // chunks per token group
     const int tid = threadIdx.x;
     const int cl = tid % cw, tg = tid / cw;
     const int c0 = cl * 4;
-    const bool active = c0 < D;
+    const bool active = ok && c0 < D;
 
     float mx[4], den[4], acc[4];
 #pragma unroll
@@ -85,12 +85,31 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
         den[u] = 0.f;
         acc[u] = 0.f;
     }
+    const int j_begin = tg * nch * kChunkTok;
+    Chunk cur, nxt;
+    float4 bcur[NCH == 1 ? kChunkTok : 1] = {};   // the chunk's positional bias rows (one chunk)
+    auto bias_row = [&](int j) -> float4 {
+        if constexpr (NCH == 1) return bcur[j - j_begin];
+        else return *reinterpret_cast<const float4*>(bias + (int64_t)j * D + c0);
+    };
+    // row of the first token of a chunk starting at pooled index j (clamped at entry 0)
+    auto chunk_row = [&](int j) { return row0 + (first + j >= 0 ? first + j : 0) - pos0; };
     if (active) {
-        const int j_begin = tg * nch * kChunkTok;
-        Chunk cur, nxt;
-        // row of the first token of a chunk starting at pooled index j (clamped at entry 0)
-        auto chunk_row = [&](int j) { return row0 + (first + j >= 0 ? first + j : 0) - pos0; };
         load_chunk(kv, gate, chunk_row(j_begin), first + j_begin, D, c0, cur);
+        if constexpr (NCH == 1) {
+#pragma unroll
+            for (int jj = 0; jj < kChunkTok; jj++)
+                bcur[jj] = *reinterpret_cast<const float4*>(bias + (int64_t)(j_begin + jj) * D + c0);
+        }
+    }
+    pdl_wait();   // entries may still be read by the previous step's attention
+    pdl_trigger();
+    if (!ok) {
+        if (threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
+        return;
+    }
+    if (active) {
+#pragma unroll 1
         for (int c = 0; c < nch; c++) {
             const int j0 = j_begin + c * kChunkTok;
             if (c + 1 < nch) load_chunk(kv, gate, chunk_row(j0 + kChunkTok), first + j0 + kChunkTok, D, c0, nxt);
@@ -98,7 +117,7 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
 #pragma unroll
             for (int jj = 0; jj < kChunkTok; jj++) {
                 if (first + j0 + jj < 0) continue;
-                const float4 bb = *reinterpret_cast<const float4*>(bias + (int64_t)(j0 + jj) * D + c0);
+                const float4 bb = bias_row(j0 + jj);
                 const float2 z01 = bf16x2_to_f32(cur.z[jj].x), z23 = bf16x2_to_f32(cur.z[jj].y);
                 cm[0] = fmaxf(cm[0], z01.x + bb.x);
                 cm[1] = fmaxf(cm[1], z01.y + bb.y);
@@ -118,7 +137,7 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
 #pragma unroll
             for (int jj = 0; jj < kChunkTok; jj++) {
                 if (first + j0 + jj < 0) continue;
-                const float4 bb = *reinterpret_cast<const float4*>(bias + (int64_t)(j0 + jj) * D + c0);
+                const float4 bb = bias_row(j0 + jj);
                 const float2 z01 = bf16x2_to_f32(cur.z[jj].x), z23 = bf16x2_to_f32(cur.z[jj].y);
                 const float2 v01 = bf16x2_to_f32(cur.v[jj].x), v23 = bf16x2_to_f32(cur.v[jj].y);
                 const float l[4] = {z01.x + bb.x, z01.y + bb.y, z23.x + bb.z, z23.y + bb.w};
@@ -134,31 +153,34 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
         }
     }
     if (TG > 1) {
-        if (tg > 0) {
-            const int slot = (tg - 1) * cw + cl;
-            st_m[slot] = make_float4(mx[0], mx[1], mx[2], mx[3]);
-            st_d[slot] = make_float4(den[0], den[1], den[2], den[3]);
-            st_a[slot] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        }
-        __syncthreads();
-        if (tg > 0) return;
-        // merge the token groups' states in order 0, 1, .., TG-1
-        for (int g = 1; g < TG; g++) {
-            const float4 gm = st_m[(g - 1) * cw + cl], gd = st_d[(g - 1) * cw + cl],
-                         ga = st_a[(g - 1) * cw + cl];
-            const float om[4] = {gm.x, gm.y, gm.z, gm.w}, od[4] = {gd.x, gd.y, gd.z, gd.w},
-                        oa[4] = {ga.x, ga.y, ga.z, ga.w};
+        // merge the token groups' states pairwise: (0,1) (2,3) .., then (0,2) .., a fixed
+        // tree; a group's state goes to its own slot, its partner reads it
+        for (int stride = 1; stride < TG; stride <<= 1) {
+            if (tg % (2 * stride) == stride) {
+                const int slot = tg * cw + cl;
+                st_m[slot] = make_float4(mx[0], mx[1], mx[2], mx[3]);
+                st_d[slot] = make_float4(den[0], den[1], den[2], den[3]);
+                st_a[slot] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            }
+            __syncthreads();
+            if (tg % (2 * stride) == 0 && tg + stride < TG) {
+                const int slot = (tg + stride) * cw + cl;
+                const float4 gm = st_m[slot], gd = st_d[slot], ga = st_a[slot];
+                const float om[4] = {gm.x, gm.y, gm.z, gm.w}, od[4] = {gd.x, gd.y, gd.z, gd.w},
+                            oa[4] = {ga.x, ga.y, ga.z, ga.w};
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const float M = fmaxf(mx[u], om[u]);
-                if (M == -INFINITY) continue;
-                const float s0 = mx[u] == -INFINITY ? 0.f : expf(mx[u] - M);
-                const float s1 = om[u] == -INFINITY ? 0.f : expf(om[u] - M);
-                den[u] = den[u] * s0 + od[u] * s1;
-                acc[u] = acc[u] * s0 + oa[u] * s1;
-                mx[u] = M;
+                for (int u = 0; u < 4; u++) {
+                    const float M = fmaxf(mx[u], om[u]);
+                    if (M == -INFINITY) continue;
+                    const float s0 = mx[u] == -INFINITY ? 0.f : expf(mx[u] - M);
+                    const float s1 = om[u] == -INFINITY ? 0.f : expf(om[u] - M);
+                    den[u] = den[u] * s0 + od[u] * s1;
+                    acc[u] = acc[u] * s0 + oa[u] * s1;
+                    mx[u] = M;
+                }
             }
         }
+        if (tg > 0) return;
     }
     float e[4] = {0.f, 0.f, 0.f, 0.f};
     if (active) {
@@ -196,7 +218,6 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : 640) compress_kernel(
     }
 
     // Store.
-    const int64_t erow = ent_off[b] + i;
     if (fmt == CSA_KV_BF16) {
         if (active) {
             uint8_t* dst = entries + erow * (int64_t)(2 * D) + 2 * c0;
@@ -234,12 +255,17 @@ cudaError_t launch_compress(int span, const void* kv, const void* gate, const fl
     const dim3 grid((unsigned)n_items);
     LaunchScope scope(kKCompress, stream);
     if (span == 8) {
-        return launch_pdl(compress_kernel<8>, grid, dim3(cw), 0, stream, (const uint16_t*)kv,
+        return launch_pdl(compress_kernel<8, 1>, grid, dim3(cw), 0, stream, (const uint16_t*)kv,
                           (const uint16_t*)gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
                           item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
     } else {
-        const int tg = cw == 32 ? 16 : 4;             // token groups: 16 x 8 or 4 x 32 tokens
-        return launch_pdl(compress_kernel<128>, grid, dim3(tg * cw), 0, stream,
+        // token groups: 16 x 8 tokens (D=128) or 4 x 32 tokens (D=576)
+        if (cw == 32)
+            return launch_pdl(compress_kernel<128, 1>, grid, dim3(16 * cw), 0, stream,
+                              (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off,
+                              kv_pos0, ent_off, item_seq, item_ent, B, m, D, fmt, log2_theta, eps,
+                              (uint8_t*)entries, st);
+        return launch_pdl(compress_kernel<128, 4>, grid, dim3(4 * cw), 0, stream,
                           (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off,
                           kv_pos0, ent_off, item_seq, item_ent, B, m, D, fmt, log2_theta, eps,
                           (uint8_t*)entries, st);
