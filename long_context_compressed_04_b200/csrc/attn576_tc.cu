@@ -523,14 +523,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             const uint8_t* mk = smask + (j % kKBuf) * 4;
             const uint32_t mbits = (uint32_t)mk[0] | ((uint32_t)mk[1] << 8) |
                                    ((uint32_t)mk[2] << 16) | ((uint32_t)mk[3] << 24);
-            float tmax = -INFINITY;
+            // raw scores (masked keys -inf); the scale is positive, so the maximum of the
+            // scaled scores is the scaled maximum
+            const uint32_t mon = mine ? mbits : 0u;
+            float rmax = -INFINITY;
+            if (mon == 0xffffffffu) {
 #pragma unroll
-            for (int c = 0; c < kTK; c++) {
-                const bool on = mine && ((mbits >> c) & 1u) != 0;
-                const float xv = on ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
-                sv[c] = __float_as_uint(xv);
-                tmax = fmaxf(tmax, xv);
+                for (int c = 0; c < kTK; c++) rmax = fmaxf(rmax, __uint_as_float(sv[c]));
+            } else {
+#pragma unroll
+                for (int c = 0; c < kTK; c++) {
+                    const float xv = ((mon >> c) & 1u) ? __uint_as_float(sv[c]) : -INFINITY;
+                    sv[c] = __float_as_uint(xv);
+                    rmax = fmaxf(rmax, xv);
+                }
             }
+            const float tmax = rmax * a.scale_log2;
             // move the reference maximum only on a jump of more than 2^8
             const bool need = mine && tmax > mref + kRescale;
             if (__any_sync(0xffffffffu, need)) {
@@ -564,15 +572,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 lrun *= corr;
                 mref = mnew;
             }
+            // P = 2^(s * scale - mref): one FMA and one ex2 per key (a masked key is -inf,
+            // giving 0); with no valid key yet (mref = -inf) every P of the tile is 0
             float rs = 0.f;
             uint32_t pk[kTK / 2];
+            if (mref == -INFINITY) {
 #pragma unroll
-            for (int c = 0; c < kTK / 2; c++) {
-                const float x0 = __uint_as_float(sv[2 * c]), x1 = __uint_as_float(sv[2 * c + 1]);
-                const float p0 = x0 == -INFINITY ? 0.f : exp2f(x0 - mref);
-                const float p1 = x1 == -INFINITY ? 0.f : exp2f(x1 - mref);
-                rs += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+                for (int c = 0; c < kTK / 2; c++) pk[c] = 0u;
+            } else {
+                const float nm = -mref;
+#pragma unroll
+                for (int c = 0; c < kTK / 2; c++) {
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), a.scale_log2, nm));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), a.scale_log2, nm));
+                    rs += p0 + p1;
+                    pk[c] = pack_bf16x2(p0, p1);
+                }
             }
             lrun += rs;
             if (!mbar_wait_warp(&pfree[sb], ((j >> 1) & 1) ^ 1, abort_flag, a.st)) {

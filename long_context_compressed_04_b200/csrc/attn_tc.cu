@@ -16,20 +16,23 @@
 // order.  Both splits depend only on k or on the query's own length, never on the batch,
 // so both paths are batch-invariant.
 //
-// Roles per CTA (8 warps, persistent over items):
+// Roles per CTA (10 warps, persistent over items):
 //   warp 0      producer: dense tiles by two 2D TMA loads (64 channels x 128 rows each,
 //               128-byte swizzle), sparse tiles by TMA tile::gather4 loads of the selected
 //               rows (4 rows x 64 channels each; an invalid index is row -1, zero-filled) into
 //               the same swizzled layout; a per-tile validity mask; 3-stage ring.
 //   warp 1      TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
 //               S = Q K^T as two M=64 x N=64 halves (keys 0-63 -> TMEM lanes 0-15 of each
-//               quarter, keys 64-127 -> lanes 16-31) and O_tile = P V as two M=64 x N=64
-//               halves (channels 0-63 / 64-127), V being the key tile read MN-major.
-//   warps 4-7   per item: q heads RoPEd at t into shared memory and the window tile; per
-//               tile: S from TMEM (thread = one head x 64 keys), online softmax in the
-//               log2 domain, P as bf16 into shared memory, then O += corr * O_tile kept in
-//               registers (thread = one head x 64 channels); finally the partial state,
-//               combined across the cluster (sparse) or written for the combine kernel.
+//               quarter, keys 64-127 -> lanes 16-31), and P V accumulated in TMEM as two
+//               outputs O_0 / O_1 (the key column-halves below), each two M=64 x N=64 halves
+//               (channels 0-63 / 64-127), V being the key tile read MN-major.
+//   warps 2-9   two warps per TMEM lane quarter.  Per item: q heads RoPEd at t and the
+//               window tile into shared memory (all 256 threads).  Per tile: 32 keys of one
+//               head per thread from TMEM, softmax in the log2 domain against a reference
+//               maximum that moves only on a jump of more than 2^8 (then O_ch is rescaled in
+//               TMEM), P as bf16 into shared memory.  Per item: O_0 and O_1 merged, then the
+//               partial state combined across the cluster (sparse) or written for the
+//               combine kernel.
 // All waits are bounded (timeout -> CSA_DEV_TIMEOUT, drain, free TMEM, return).
 #include <cstring>
 #include <mutex>
@@ -49,7 +52,9 @@ constexpr int kBlk = kTK * 128;              // one 64-channel slice of a key ti
 constexpr int kTileBytes = 2 * kBlk;         // 32 KB
 constexpr int kQBlk = kH * 128;              // one 64-channel slice of Q (8 KB)
 constexpr int kPBlk = kH * 128;              // one 64-key slice of P (8 KB)
-constexpr int kThreads = 256;
+constexpr int kThreads = 320;
+constexpr float kRescale = 8.f;              // a tile moves the reference maximum only when
+                                             // it exceeds it by more than 2^8
 constexpr int kDenseChunkTiles = 8;
 constexpr int kMaxK = 2048;
 constexpr int kMaxCluster = 8;
@@ -194,18 +199,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // per-head combine weights [nh][cluster + 1]
     float* recv = reinterpret_cast<float*>(srows + kStages * kTK);
     float* wtab = recv + kRecvFloats;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(wtab + kWtabFloats);
+    float* xml = wtab + kWtabFloats;       // [128][2] column-half 1's m, l per (head, half)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(xml + 256);
     uint64_t* full = bars;                 // [kStages]  33 arrivals (+tx)
     uint64_t* empty = full + kStages;      // [kStages]  MMA commit
-    uint64_t* prep_full = empty + kStages; // Q + window ready: 4 arrivals
+    uint64_t* prep_full = empty + kStages; // Q + window ready: 8 arrivals
     uint64_t* prep_empty = prep_full + 1;  // item's MMAs done: MMA commit
     uint64_t* s_full = prep_empty + 1;     // [2]
-    uint64_t* s_empty = s_full + 2;        // [2] 4 arrivals
-    uint64_t* p_full = s_empty + 2;        // [2] 4 arrivals
+    uint64_t* s_empty = s_full + 2;        // [2] 8 arrivals
+    uint64_t* p_full = s_empty + 2;        // [2] 8 arrivals
     uint64_t* p_empty = p_full + 2;        // [2]
-    uint64_t* pv_full = p_empty + 2;       // [2]
-    uint64_t* pv_empty = pv_full + 2;      // [2] 4 arrivals
-    uint64_t* cpart_full = pv_empty + 2;  // every rank's partials are in: 4 x cluster
+    uint64_t* pvdone = p_empty + 2;        // MMA commit after every tile's P V (a rescale
+                                           // waits for the previous one)
+    uint64_t* odone = pvdone + 1;          // MMA commit after an item's last P V
+    uint64_t* cpart_full = odone + 3;     // every rank's partials are in: 4 x cluster
     uint64_t* cpart_free = cpart_full + 1; // every rank has combined the previous query (its
                                            // receive buffer is free again): 4 x cluster
     uint64_t* drain = cpart_free + 1;
@@ -218,16 +225,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&full[s], 33);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(prep_full, 4);
+        mbar_init(prep_full, 8);
         mbar_init(prep_empty, 1);
         for (int i = 0; i < 2; i++) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 4);
-            mbar_init(&p_full[i], 4);
+            mbar_init(&s_empty[i], 8);
+            mbar_init(&p_full[i], 8);
             mbar_init(&p_empty[i], 1);
-            mbar_init(&pv_full[i], 1);
-            mbar_init(&pv_empty[i], 4);
         }
+        mbar_init(pvdone, 1);
+        mbar_init(odone, 1);
         mbar_init(cpart_full, 4 * a.cluster);
         mbar_init(cpart_free, 4 * a.cluster);
         mbar_init(drain, 1);
@@ -246,21 +253,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
     const uint32_t tmem_S = tmem_base;          // [2] x 64 columns
-    const uint32_t tmem_PV = tmem_base + 128;   // [2] x 64 columns
+    const uint32_t tmem_O = tmem_base + 128;    // O_0, O_1: 64 columns each
 
     if (warp == 0) {
         // ---------------- producer ----------------
         // index sets (top-k) and entries (compression) come from earlier kernels; the
         // prologue of the other roles (q heads, window rows) only reads inputs
-        pdl_wait();
-        if (lane == 0) pdl_trigger();
         int stage = 0;
         uint32_t ph = 0;
         int issued[kStages] = {};
         bool ok = true;
+        bool waited = false;
         for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
             AItem x;
-            if (!get_item(a, it, x, false)) continue;
+            const bool have = get_item(a, it, x, false);
+            if (have && !a.idx) {
+                // dense: the item's entry tiles are contiguous rows; all of them are
+                // prefetched into L2 at once (before the wait on the previous kernel for the
+                // first item: a prefetch returns no data, and L2 holds the coherent copy of
+                // the entries the previous kernel writes), so the tile loads below meet L2
+                for (int jj = lane; jj < x.ntiles; jj += 32) {
+                    const int j = x.tile0 + jj;
+                    const int e0 = (j - 1) * kTK;
+                    const int rows = j == 0 ? 0 : min(kTK, x.n_ent - e0);
+                    if (rows > 0)
+                        prefetch_l2_bulk(a.entries + (x.row0 + e0) * (int64_t)(kD * 2),
+                                         (uint32_t)(rows * kD * 2));
+                }
+            }
+            if (!waited) {
+                pdl_wait();
+                if (lane == 0) pdl_trigger();
+                waited = true;
+            }
+            if (!have) continue;
             if (a.idx && x.tile0 + x.ntiles > 1) {
                 // the query's whole index row, once per item: batches of 8 x 16-byte loads
                 // per lane in flight (one round trip for k <= 1024); only this warp reads it
@@ -365,11 +391,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        if (!waited) {
+            pdl_wait();
+            if (lane == 0) pdl_trigger();
+        }
         for (int s = 0; s < kStages; s++)
             if (issued[s]) mbar_drain(&full[s], (issued[s] - 1) & 1, a.st);
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
+            // S of a tile is issued before the P V of the previous one.  P V accumulates into
+            // the item's two running outputs in TMEM, one per key column-half: O_0 takes keys
+            // 0-31 and 64-95 of every tile (K-steps 0, 1, 4, 5), O_1 keys 32-63 and 96-127.
             int stage = 0;
             uint32_t ph = 0;
             int nt = 0, nitem = 0;
@@ -382,6 +415,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint8_t* prev_k = nullptr;
                 int prev_stage = -1, prev_sb = 0;
+                auto issue_pv = [&](bool first) -> bool {
+                    const int psb = prev_sb;
+                    if (!mbar_wait(&p_full[psb], ((nt - 1) >> 1) & 1, abort_flag, a.st)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ch = 0; ch < 2; ch++) {
+#pragma unroll
+                        for (int t = 0; t < 4; t++) {
+                            const int kk = (t >> 1) * 4 + ch * 2 + (t & 1);
+                            const uint64_t ad =
+                                smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
+                                ((uint32_t)((kk & 3) * 32) >> 4);
+#pragma unroll
+                            for (int half = 0; half < 2; half++) {
+                                const uint32_t d = tmem_O + ch * 64 + ((uint32_t)(half * 16) << 16);
+                                const uint64_t bd =
+                                    smem_desc_mn_sw128(prev_k + half * kBlk + kk * 2048, kBlk);
+                                mma_f16(d, ad, bd, kIdescPV, (first && t == 0) ? 0u : 1u);
+                            }
+                        }
+                    }
+                    mma_commit(&p_empty[psb]);
+                    if (prev_stage >= 0) mma_commit(&empty[prev_stage]);
+                    mma_commit(pvdone);
+                    return true;
+                };
                 for (int jj = 0; jj < x.ntiles && ok; jj++) {
                     const int j = x.tile0 + jj;
                     const uint8_t* kb;
@@ -421,31 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     mma_commit(&s_full[sb]);
-                    if (jj > 0) {
-                        // O_tile for the previous tile
-                        const int psb = prev_sb;
-                        if (!mbar_wait(&p_full[psb], ((nt - 1) >> 1) & 1, abort_flag, a.st) ||
-                            !mbar_wait(&pv_empty[psb], (((nt - 1) >> 1) & 1) ^ 1, abort_flag, a.st)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < 8; kk++) {
-#pragma unroll
-                            for (int half = 0; half < 2; half++) {
-                                const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
-                                const uint64_t ad =
-                                    smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
-                                    ((uint32_t)((kk & 3) * 32) >> 4);
-                                const uint64_t bd =
-                                    smem_desc_mn_sw128(prev_k + half * kBlk + kk * 2048, kBlk);
-                                mma_f16(d, ad, bd, kIdescPV, kk > 0 ? 1u : 0u);
-                            }
-                        }
-                        mma_commit(&pv_full[psb]);
-                        mma_commit(&p_empty[psb]);
-                        if (prev_stage >= 0) mma_commit(&empty[prev_stage]);
+                    if (jj > 0 && !issue_pv(jj == 1)) {
+                        ok = false;
+                        break;
                     }
                     prev_k = kb;
                     prev_stage = my_stage;
@@ -453,43 +490,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                     nt++;
                 }
                 if (!ok) break;
-                {
-                    const int psb = prev_sb;
-                    if (!mbar_wait(&p_full[psb], ((nt - 1) >> 1) & 1, abort_flag, a.st) ||
-                        !mbar_wait(&pv_empty[psb], (((nt - 1) >> 1) & 1) ^ 1, abort_flag, a.st)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; kk++) {
-#pragma unroll
-                        for (int half = 0; half < 2; half++) {
-                            const uint32_t d = tmem_PV + psb * 64 + ((uint32_t)(half * 16) << 16);
-                            const uint64_t ad =
-                                smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
-                                ((uint32_t)((kk & 3) * 32) >> 4);
-                            const uint64_t bd =
-                                smem_desc_mn_sw128(prev_k + half * kBlk + kk * 2048, kBlk);
-                            mma_f16(d, ad, bd, kIdescPV, kk > 0 ? 1u : 0u);
-                        }
-                    }
-                    mma_commit(&pv_full[psb]);
-                    mma_commit(&p_empty[psb]);
-                    if (prev_stage >= 0) mma_commit(&empty[prev_stage]);
-                }
+                if (!issue_pv(x.ntiles == 1)) break;
+                mma_commit(odone);
                 mma_commit(prep_empty);
                 nitem++;
             }
             mma_commit(drain);
             mbar_drain(drain, 0, a.st);
         }
-    } else if (warp >= 4) {
-        // ---------------- softmax / epilogue (warps 4..7) ----------------
+    } else if (warp >= 2) {
+        // ---------------- softmax / epilogue (warps 2..9) ----------------
+        // Two warps share each TMEM lane quarter (the quarter is fixed by the warp's rank
+        // modulo 4): warp column-half `ch` reads S columns ch*32 .. ch*32+31 of its lanes, so a
+        // thread holds 32 keys of one head (lanes 0-15: keys ch*32 + c, lanes 16-31: keys
+        // 64 + ch*32 + c).  Each (head, column-half) keeps its own running maximum, sum and
+        // output O_ch; the two are merged once per item.
         const int quarter = warp & 3;
-        const int i = threadIdx.x - 128;        // 0..127
+        const int ch = (warp - 2) >> 2;
+        const int i = threadIdx.x - 64;         // 0..255
         const int h = quarter * 16 + (lane & 15);
         const int kh = lane >> 4;               // key half of S / channel half of O
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         int nt = 0, nitem = 0;
         int kst = 0;   // ring position of the next entry tile (mirrors the producer)
         bool ok = true;
@@ -498,9 +519,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!get_item(a, it, x, i == 0)) continue;
             // ---- item prologue: q heads and (chunk 0) the window tile ----
             // A failed wait in a warp only skips the rest of that item; here, once per item,
-            // all 128 threads meet and leave together if any of them failed.
+            // all 256 threads meet and leave together if any of them failed.
             const bool ready = ok && mbar_wait(prep_empty, (nitem & 1) ^ 1, abort_flag, a.st);
-            if (!named_barrier_and(1, 128, ready)) break;
+            if (!named_barrier_and(1, 256, ready)) break;
             if (i < 32) {
                 // angles in fp64, reduced, then sincosf (see rope_cos_sin)
                 float cs, sn;
@@ -511,16 +532,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 rwc[i] = cs;
                 rws[i] = sn;
                 rf[i] = (float)exp2(-(double)(2 * i) * (1.0 / 64.0) * a.log2_theta);
+            } else if (i < 36 && x.tile0 == 0) {
+                // window validity words: rows r with r < n_win and w0 + r >= kv_pos0
+                const int wd = i - 32;
+                const int64_t lo64 = a.kv_pos0[x.b] - (int64_t)x.w0;
+                const int lo = lo64 > 0 ? (lo64 > kTK ? kTK : (int)lo64) : 0;
+                const int a0 = max(lo - 32 * wd, 0), a1 = min(x.n_win - 32 * wd, 32);
+                uint32_t wbits = 0;
+                if (a1 > a0) wbits = (a1 - a0 == 32 ? 0xffffffffu : ((1u << (a1 - a0)) - 1u)) << a0;
+                smask[kStages * 4 + wd] = wbits;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             {
-                const int hq = i >> 1, hf = i & 1;
-                const uint16_t* src = a.q + ((int64_t)x.q * kH + hq) * kD + hf * 64;
-                float v[64];
+                // q head hq, channels u*32 .. u*32+31 (RoPE on the last 64: u = 2, 3)
+                const int hq = i >> 2, u = i & 3;
+                const uint16_t* src = a.q + ((int64_t)x.q * kH + hq) * kD + u * 32;
+                float v[32];
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
-                    const uint4 u = *reinterpret_cast<const uint4*>(src + 8 * c);
-                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+                for (int c = 0; c < 4; c++) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(src + 8 * c);
+                    const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int z = 0; z < 4; z++) {
                         const float2 f = bf16x2_to_f32(w4[z]);
@@ -528,43 +559,46 @@ __global__ void __launch_bounds__(kThreads, 1)
                         v[8 * c + 2 * z + 1] = f.y;
                     }
                 }
-                if (hf == 1) {
+                if (u >= 2) {
 #pragma unroll
-                    for (int pj = 0; pj < 32; pj++) {
+                    for (int k = 0; k < 16; k++) {
+                        const int pj = (u - 2) * 16 + k;
                         const float cs = rqc[pj], sn = rqs[pj];
-                        const float x0 = v[2 * pj], y0 = v[2 * pj + 1];
-                        v[2 * pj] = x0 * cs - y0 * sn;
-                        v[2 * pj + 1] = x0 * sn + y0 * cs;
+                        const float x0 = v[2 * k], y0 = v[2 * k + 1];
+                        v[2 * k] = x0 * cs - y0 * sn;
+                        v[2 * k + 1] = x0 * sn + y0 * cs;
                     }
                 }
-                uint8_t* dst = sQ + hf * kQBlk;
+                uint8_t* dst = sQ + (u >> 1) * kQBlk;
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
-                    uint4 u;
-                    u.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
-                    u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
-                    u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
-                    u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
-                    *reinterpret_cast<uint4*>(dst + swz(hq, c)) = u;
+                for (int c = 0; c < 4; c++) {
+                    uint4 w;
+                    w.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
+                    w.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+                    w.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+                    w.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+                    *reinterpret_cast<uint4*>(dst + swz(hq, (u & 1) * 4 + c)) = w;
                 }
             }
             if (x.tile0 == 0) {
-                // window row r = i: RMSNorm, RoPE at its position, bf16, swizzled store
-                const int r = i;
+                // window row r = i / 2; thread u = i % 2 takes channels u*32 .. u*32+31 and
+                // 64 + u*32 .. 64 + u*32+31 (16 RoPE pairs each): RMSNorm over the row (the
+                // pair's sums of squares added), RoPE at the row's position, bf16, swizzled
+                const int r = i >> 1, u = i & 1;
                 const int64_t p = (int64_t)x.w0 + r;
                 bool valid = r < x.n_win;
                 if (valid && p < a.kv_pos0[x.b]) {
                     valid = false;
                     flag(a.st, CSA_DEV_OOB);
                 }
-                float v[128];
+                float v[64];
+                float ss = 0.f;
                 if (valid) {
-                    const uint16_t* src = a.kv + (a.kv_off[x.b] + p - a.kv_pos0[x.b]) * kD;
-                    float ss = 0.f;
+                    const uint16_t* src = a.kv + (a.kv_off[x.b] + p - a.kv_pos0[x.b]) * kD + u * 32;
 #pragma unroll
-                    for (int c = 0; c < 16; c++) {
-                        const uint4 u = *reinterpret_cast<const uint4*>(src + 8 * c);
-                        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+                    for (int c = 0; c < 8; c++) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(src + (c >> 2) * 64 + 8 * (c & 3));
+                        const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                         for (int z = 0; z < 4; z++) {
                             const float2 f = bf16x2_to_f32(w4[z]);
@@ -573,63 +607,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                             ss += f.x * f.x + f.y * f.y;
                         }
                     }
-                    const float rn = rsqrtf(ss / (float)kD + a.eps);
-#pragma unroll
-                    for (int c = 0; c < 128; c++) v[c] *= rn;
-                    // angle (w0 + r) f_j = w0 f_j + r f_j: the first term from the fp64 table,
-                    // the second (< 128 rad) by sincosf; combined by the addition formula.
-                    // The per-row rotations go to a scratch row in the idle P buffers.
-                    float2* rot = reinterpret_cast<float2*>(sP) + r * 32;
-#pragma unroll 1
-                    for (int pj = 0; pj < 32; pj++) {
-                        float sb, cb;
-                        sincosf((float)r * rf[pj], &sb, &cb);
-                        rot[pj] = make_float2(rwc[pj] * cb - rws[pj] * sb, rws[pj] * cb + rwc[pj] * sb);
-                    }
-#pragma unroll
-                    for (int pj = 0; pj < 32; pj++) {
-                        const float2 cs = rot[pj];
-                        const float x0 = v[64 + 2 * pj], y0 = v[64 + 2 * pj + 1];
-                        v[64 + 2 * pj] = x0 * cs.x - y0 * cs.y;
-                        v[64 + 2 * pj + 1] = x0 * cs.y + y0 * cs.x;
-                    }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 128; c++) v[c] = 0.f;
+                    for (int c = 0; c < 64; c++) v[c] = 0.f;
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                if (valid) {
+                    const float rn = rsqrtf(ss / (float)kD + a.eps);
+#pragma unroll
+                    for (int c = 0; c < 64; c++) v[c] *= rn;
+                    // angle (w0 + r) f_j = w0 f_j + r f_j: the first term from the fp64 table,
+                    // the second (< 128 rad) by sincosf; combined by the addition formula
+#pragma unroll
+                    for (int k = 0; k < 16; k++) {
+                        const int pj = u * 16 + k;
+                        float sb, cb;
+                        sincosf((float)r * rf[pj], &sb, &cb);
+                        const float cs = rwc[pj] * cb - rws[pj] * sb, sn = rws[pj] * cb + rwc[pj] * sb;
+                        const float x0 = v[32 + 2 * k], y0 = v[32 + 2 * k + 1];
+                        v[32 + 2 * k] = x0 * cs - y0 * sn;
+                        v[32 + 2 * k + 1] = x0 * sn + y0 * cs;
+                    }
                 }
 #pragma unroll
-                for (int c = 0; c < 16; c++) {
-                    uint4 u;
-                    u.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
-                    u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
-                    u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
-                    u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
-                    *reinterpret_cast<uint4*>(sW + (c >> 3) * kBlk + swz(r, c & 7)) = u;
+                for (int c = 0; c < 8; c++) {
+                    uint4 w;
+                    w.x = pack_bf16x2(v[8 * c], v[8 * c + 1]);
+                    w.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+                    w.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+                    w.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+                    *reinterpret_cast<uint4*>(sW + (c >> 2) * kBlk + swz(r, u * 4 + (c & 3))) = w;
                 }
-                const unsigned vm = __ballot_sync(0xffffffffu, valid);
-                if (lane == 0) smask[kStages * 4 + quarter] = vm;
             }
             fence_async_smem();
-            // all four warps' stores (including the window mask) before anyone reads them
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            // all warps' stores (including the window mask) before anyone reads them
+            asm volatile("bar.sync 1, 256;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(prep_full);
 
-            // ---- running state of head h ----
             // sparse: the sink of head h0 + i of this rank's slice, for the combine
             float sk_mine = -INFINITY;
             if (a.idx) {
                 const int h0 = x.c * kH / a.cluster, h1 = (x.c + 1) * kH / a.cluster;
                 if (i < h1 - h0) sk_mine = a.sink[h0 + i] * kLog2e;
             }
-            // the chunk's own keys only: the sink enters when the partial states are combined
-            float mrun = -INFINITY;
+            // ---- running state of (head h, column-half ch) ----
+            // the chunk's own keys only: the sink enters when the partial states are combined.
+            // mref is the reference maximum of P = 2^(s - mref); it moves only when a tile's
+            // maximum exceeds it by more than 2^kRescale, and then O_ch is rescaled in TMEM.
+            float mref = -INFINITY;
             float lrun = 0.f;
-            float o[64];
-#pragma unroll
-            for (int c = 0; c < 64; c++) o[c] = 0.f;
-            float corr_prev = 1.f;
-            int prev_sb = 0;
             for (int jj = 0; jj < x.ntiles && ok; jj++) {
                 const int j = x.tile0 + jj;
                 const int sb = nt & 1;
@@ -638,116 +665,164 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                uint32_t sv[64];
-                tmem_ld64(tmem_S + sb * 64 + ((uint32_t)(quarter * 32) << 16), sv);
+                uint32_t sv[32];
+                tmem_ld32(tmem_S + sb * 64 + ch * 32 + lane_base, sv);
                 tmem_ld_wait();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[sb]);
-                // validity of my 64 keys (the MMA has consumed the tile, so its mask is stable
+                // validity of my 32 keys (the MMA has consumed the tile, so its mask is stable
                 // until the producer refills the stage after this tile's P.V)
                 const uint32_t* mk = smask + (j == 0 ? kStages : kst) * 4;
                 if (j != 0 && ++kst == kStages) kst = 0;
-                const uint32_t mw0 = mk[2 * kh], mw1 = mk[2 * kh + 1];
-                float tmax = -INFINITY;
+                const uint32_t mw = mk[2 * kh + ch];
+                // raw scores (masked keys -inf); the scale is positive, so the maximum of the
+                // scaled scores is the scaled maximum
+                float rmax = -INFINITY;
+                if (mw == 0xffffffffu) {
 #pragma unroll
-                for (int c = 0; c < 64; c++) {
-                    const bool on = ((c < 32 ? mw0 >> c : mw1 >> (c - 32)) & 1u) != 0;
-                    const float xv = on ? __uint_as_float(sv[c]) * a.scale_log2 : -INFINITY;
-                    sv[c] = __float_as_uint(xv);
-                    tmax = fmaxf(tmax, xv);
-                }
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
-                const float mnew = fmaxf(mrun, tmax);
-                float corr = 1.f, rs = 0.f;
-                uint32_t pk[32];
-                if (mnew == -INFINITY) {
-#pragma unroll
-                    for (int c = 0; c < 32; c++) pk[c] = 0u;
+                    for (int c = 0; c < 32; c++) rmax = fmaxf(rmax, __uint_as_float(sv[c]));
                 } else {
-                    corr = exp2f(mrun - mnew);
 #pragma unroll
                     for (int c = 0; c < 32; c++) {
-                        const float p0 = exp2f(__uint_as_float(sv[2 * c]) - mnew);
-                        const float p1 = exp2f(__uint_as_float(sv[2 * c + 1]) - mnew);
+                        const float xv = ((mw >> c) & 1u) ? __uint_as_float(sv[c]) : -INFINITY;
+                        sv[c] = __float_as_uint(xv);
+                        rmax = fmaxf(rmax, xv);
+                    }
+                }
+                float tmax = rmax * a.scale_log2;
+                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+                const bool need = tmax > mref + kRescale;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float mnew = need ? tmax : mref;
+                    const float corr = !need ? 1.f : (mref == -INFINITY ? 0.f : exp2f(mref - mnew));
+                    if (jj > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
+                        // O_ch must hold every earlier P V of the item before it is rescaled
+                        if (!mbar_wait_warp(pvdone, (nt - 1) & 1, abort_flag, a.st)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int cc = 0; cc < 4; cc++) {
+                            uint32_t ov[16];
+                            const uint32_t col = tmem_O + ch * 64 + 16 * cc + lane_base;
+                            tmem_ld16(col, ov);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int z = 0; z < 16; z++)
+                                ov[z] = __float_as_uint(__uint_as_float(ov[z]) * corr);
+                            tmem_st16(col, ov);
+                        }
+                        tmem_st_wait();
+                        tc_fence_before();
+                    }
+                    lrun *= corr;
+                    mref = mnew;
+                }
+                // P = 2^(s * scale - mref): one FMA and one ex2 per key (a masked key is -inf,
+                // giving 0); with no valid key yet (mref = -inf) every P of the tile is 0
+                float rs = 0.f;
+                uint32_t pk[16];
+                if (mref == -INFINITY) {
+#pragma unroll
+                    for (int c = 0; c < 16; c++) pk[c] = 0u;
+                } else {
+                    const float nm = -mref;
+#pragma unroll
+                    for (int c = 0; c < 16; c++) {
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), a.scale_log2, nm));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), a.scale_log2, nm));
                         rs += p0 + p1;
                         pk[c] = pack_bf16x2(p0, p1);
                     }
                 }
                 rs += __shfl_xor_sync(0xffffffffu, rs, 16);
-                lrun = lrun * corr + rs;
-                mrun = mnew;
-                // P (bf16) into shared memory: head h, keys kh*64 .. kh*64+63
+                lrun += rs;
+                // P (bf16) into shared memory: head h, keys kh*64 + ch*32 .. +31
                 if (!mbar_wait_warp(&p_empty[sb], ((nt >> 1) & 1) ^ 1, abort_flag, a.st)) {
                     ok = false;
                     break;
                 }
                 uint8_t* prow = sP + sb * 2 * kPBlk + kh * kPBlk;
 #pragma unroll
-                for (int c = 0; c < 8; c++)
-                    *reinterpret_cast<uint4*>(prow + swz(h, c)) =
+                for (int c = 0; c < 4; c++)
+                    *reinterpret_cast<uint4*>(prow + swz(h, ch * 4 + c)) =
                         make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[sb]);
-                if (jj > 0) {
-                    if (!mbar_wait_warp(&pv_full[prev_sb], ((nt - 1) >> 1) & 1, abort_flag, a.st)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    uint32_t pv[64];
-                    tmem_ld64(tmem_PV + prev_sb * 64 + ((uint32_t)(quarter * 32) << 16), pv);
-                    tmem_ld_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&pv_empty[prev_sb]);
-#pragma unroll
-                    for (int c = 0; c < 64; c++) o[c] = fmaf(o[c], corr_prev, __uint_as_float(pv[c]));
-                }
-                corr_prev = corr;
-                prev_sb = sb;
                 nt++;
             }
-            if (ok) ok = mbar_wait_warp(&pv_full[prev_sb], ((nt - 1) >> 1) & 1, abort_flag, a.st);
-            if (ok) {
-                tc_fence_after();
-                uint32_t pv[64];
-                tmem_ld64(tmem_PV + prev_sb * 64 + ((uint32_t)(quarter * 32) << 16), pv);
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&pv_empty[prev_sb]);
+            // ---- the item's output: O_ch from TMEM, the two column-halves merged ----
+            if (ok) ok = mbar_wait_warp(odone, nitem & 1, abort_flag, a.st);
+            float o[64];
+            {
+                uint32_t ov[64];
 #pragma unroll
-                for (int c = 0; c < 64; c++) o[c] = fmaf(o[c], corr_prev, __uint_as_float(pv[c]));
+                for (int c = 0; c < 64; c++) ov[c] = 0u;
+                if (ok) {
+                    tc_fence_after();
+                    tmem_ld64(tmem_O + ch * 64 + lane_base, ov);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                }
+#pragma unroll
+                for (int c = 0; c < 64; c++) o[c] = __uint_as_float(ov[c]);
+            }
+            // column-half 1 hands its state to column-half 0 through the idle window buffer
+            // (every MMA of the item is complete), thread slot = quarter * 32 + lane
+            float* xo = reinterpret_cast<float*>(sW);
+            const int slot = quarter * 32 + lane;
+            if (ok && ch == 1) {
+#pragma unroll
+                for (int c = 0; c < 64; c++) xo[c * 128 + slot] = o[c];
+                xml[2 * slot] = mref;
+                xml[2 * slot + 1] = lrun;
+            }
+            if (!named_barrier_and(1, 256, ok)) {
+                ok = false;
+                break;
+            }
+            float mrun = mref;
+            if (ch == 0) {
+                const float m1 = xml[2 * slot], l1 = xml[2 * slot + 1];
+                mrun = fmaxf(mref, m1);
+                const float w0 = mref == -INFINITY ? 0.f : exp2f(mref - mrun);
+                const float w1 = m1 == -INFINITY ? 0.f : exp2f(m1 - mrun);
+                lrun = lrun * w0 + l1 * w1;
+#pragma unroll
+                for (int c = 0; c < 64; c++) o[c] = o[c] * w0 + xo[c * 128 + slot] * w1;
             }
             if (a.idx) {
                 // ---- sparse: exchange partial states across the cluster ----
                 const int C = a.cluster;
                 const int nh = (kH + C - 1) / C;
                 float* recv_ml = recv + C * nh * kD;
-                // every rank's receive buffer is free of the previous query's partials
-                if (ok) ok = mbar_wait_cluster_warp(cpart_free, (nitem & 1) ^ 1, abort_flag, a.st);
-                if (ok) {
-                    // head h is finished by rank `own` (heads [own*kH/C, (own+1)*kH/C))
-                    int own = 0;
-                    while (own + 1 < C && (own + 1) * kH / C <= h) own++;
-                    const int lh = h - own * kH / C;
-                    const uint32_t dst = mapa(recv + ((x.c * nh + lh) * kD + kh * 64), (uint32_t)own);
+                if (ch == 0) {
+                    // every rank's receive buffer is free of the previous query's partials
+                    ok = mbar_wait_cluster_warp(cpart_free, (nitem & 1) ^ 1, abort_flag, a.st);
+                    if (ok) {
+                        // head h is finished by rank `own` (heads [own*kH/C, (own+1)*kH/C))
+                        int own = 0;
+                        while (own + 1 < C && (own + 1) * kH / C <= h) own++;
+                        const int lh = h - own * kH / C;
+                        const uint32_t dst = mapa(recv + ((x.c * nh + lh) * kD + kh * 64), (uint32_t)own);
 #pragma unroll
-                    for (int c = 0; c < 64; c += 4)
-                        st_cluster_f4(dst + 4 * c, make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]));
-                    if (kh == 0) {
-                        st_cluster_f32(mapa(recv_ml + (2 * x.c) * nh + lh, (uint32_t)own), mrun);
-                        st_cluster_f32(mapa(recv_ml + (2 * x.c + 1) * nh + lh, (uint32_t)own), lrun);
+                        for (int c = 0; c < 64; c += 4)
+                            st_cluster_f4(dst + 4 * c, make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]));
+                        if (kh == 0) {
+                            st_cluster_f32(mapa(recv_ml + (2 * x.c) * nh + lh, (uint32_t)own), mrun);
+                            st_cluster_f32(mapa(recv_ml + (2 * x.c + 1) * nh + lh, (uint32_t)own), lrun);
+                        }
+                        fence_cluster();
+                        __syncwarp();
+                        if (lane == 0)
+                            for (int r = 0; r < C; r++) mbar_arrive_cluster(mapa(cpart_full, (uint32_t)r));
+                        ok = mbar_wait_cluster_warp(cpart_full, nitem & 1, abort_flag, a.st);
                     }
-                    fence_cluster();
-                    __syncwarp();
-                    if (lane == 0)
-                        for (int r = 0; r < C; r++) mbar_arrive_cluster(mapa(cpart_full, (uint32_t)r));
-                    ok = mbar_wait_cluster_warp(cpart_full, nitem & 1, abort_flag, a.st);
                 }
-                if (named_barrier_and(1, 128, ok)) {
+                if (named_barrier_and(1, 256, ok)) {
                     // this rank's heads; first the combine weights, one thread per head:
                     // M = max(sink, m_r), w_r = 2^(m_r - M), L = 2^(sink - M) + sum_r w_r l_r
                     const int h0 = x.c * kH / C, h1 = (x.c + 1) * kH / C;
@@ -764,12 +839,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         wtab[i * (kMaxCluster + 1) + kMaxCluster] = L;
                     }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    asm volatile("bar.sync 1, 256;" ::: "memory");
                     // then (head, 4 channels) per work unit: sum_r w_r O_r / L, inverse RoPE
                     // (the pairs sit inside the 4 channels), 4 bf16 stored at once
                     const int units = (h1 - h0) * (kD / 4);
 #pragma unroll 2
-                    for (int w = i; w < units; w += 128) {
+                    for (int w = i; w < units; w += 256) {
                         const int lh = w / (kD / 4), c4 = (w % (kD / 4)) * 4;
                         const float* wt = wtab + lh * (kMaxCluster + 1);
                         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -800,20 +875,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         *reinterpret_cast<uint2*>(a.out + ((int64_t)x.q * kH + h0 + lh) * kD + c4) =
                             make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
                     }
-                    // my receive buffer may take the next query's partials
-                    fence_cluster();
-                    __syncwarp();
-                    if (lane == 0)
-                        for (int r = 0; r < C; r++) mbar_arrive_cluster(mapa(cpart_free, (uint32_t)r));
+                    // every thread's reads of the receive buffer are done; then it may take
+                    // the next query's partials
+                    asm volatile("bar.sync 1, 256;" ::: "memory");
+                    if (ch == 0) {
+                        fence_cluster();
+                        __syncwarp();
+                        if (lane == 0)
+                            for (int r = 0; r < C; r++) mbar_arrive_cluster(mapa(cpart_free, (uint32_t)r));
+                    }
                 } else {
                     ok = false;
                 }
-            } else if (ok) {
+            } else if (ok && ch == 0) {
                 float* pr = a.part + ((int64_t)it * kH + h) * (kD + 2);
                 if (kh == 0) {
                     pr[0] = mrun;
                     pr[1] = lrun;
                 }
+                // rows are kD + 2 floats: 8-byte aligned
 #pragma unroll
                 for (int c = 0; c < 64; c += 2)
                     *reinterpret_cast<float2*>(pr + 2 + kh * 64 + c) = make_float2(o[c], o[c + 1]);
@@ -836,23 +916,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 // sink, normalise, inverse RoPE, store bf16.  Thread = channel.
 __global__ void __launch_bounds__(kD) attn_combine_kernel(const AttnTcArgs a) {
     const int q = blockIdx.y, h = blockIdx.x, d = threadIdx.x;
+    // query metadata and the sink are inputs: read before the wait on the attention kernel
+    const int b = a.q_seq[q], t = a.q_pos[q];
+    const bool valid = !(b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]);
+    int nch = 0;
+    if (valid) {
+        int n = (t + 1) / a.m;
+        if (n > a.max_n) n = a.max_n;
+        const int64_t avail = a.ent_rows - a.ent_off[b];
+        if ((int64_t)n > avail) n = avail > 0 ? (int)avail : 0;
+        const int total = 1 + (n + kTK - 1) / kTK;
+        nch = (total + a.chunk_tiles - 1) / a.chunk_tiles;
+    }
+    const float sk = a.sink[h] * kLog2e;
+    float cs = 1.f, sn = 0.f;   // inverse RoPE of the last 64 channels
+    if (valid && d >= kD - kRopeDims)
+        rope_cos_sin(-(double)t, (d - (kD - kRopeDims)) >> 1, a.log2_theta, cs, sn);
     pdl_wait();   // chunk partials come from the attention kernel
     pdl_trigger();
-    const int b = a.q_seq[q], t = a.q_pos[q];
-    if (b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]) return;
-    int n = (t + 1) / a.m;
-    if (n > a.max_n) n = a.max_n;
-    const int64_t avail = a.ent_rows - a.ent_off[b];
-    if ((int64_t)n > avail) n = avail > 0 ? (int)avail : 0;
-    const int total = 1 + (n + kTK - 1) / kTK;
-    const int nch = (total + a.chunk_tiles - 1) / a.chunk_tiles;
-    const float sk = a.sink[h] * kLog2e;
+    if (!valid) return;
     const float* base = a.part + ((int64_t)q * a.chunks_per_q * kH + h) * (kD + 2);
     const int64_t cstride = (int64_t)kH * (kD + 2);
     float M = sk;
+#pragma unroll 8
     for (int c = 0; c < nch; c++) M = fmaxf(M, base[c * cstride]);
     float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
     float o = 0.f;
+#pragma unroll 8
     for (int c = 0; c < nch; c++) {
         const float* pc = base + c * cstride;
         const float mc = pc[0];
@@ -862,11 +952,7 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(const AttnTcArgs a) {
     }
     o = L > 0.f ? o / L : 0.f;
     const float other = __shfl_xor_sync(0xffffffffu, o, 1);
-    if (d >= kD - kRopeDims) {
-        float cs, sn;
-        rope_cos_sin(-(double)t, (d - (kD - kRopeDims)) >> 1, a.log2_theta, cs, sn);
-        o = (d & 1) ? (other * sn + o * cs) : (o * cs - other * sn);
-    }
+    if (d >= kD - kRopeDims) o = (d & 1) ? (other * sn + o * cs) : (o * cs - other * sn);
     a.out[((int64_t)q * kH + h) * kD + d] = (uint16_t)f32_to_bf16_bits(o);
 }
 
@@ -902,8 +988,9 @@ int sm_count() {
 
 constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + kTileBytes + 2 * kQBlk + 4 * kPBlk +
                               4 * (kStages + 1) * 4 + 5 * 32 * 4 + kMaxK * 4 + kStages * kTK * 4 +
-                              (kRecvFloats + kWtabFloats) * 4 + (2 * kStages + 17) * 8 + 16;
+                              (kRecvFloats + kWtabFloats + 256) * 4 + (2 * kStages + 17) * 8 + 16;
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+static_assert((kRecvFloats + kWtabFloats + 256) % 2 == 0, "mbarriers 8-byte aligned");
 
 // CTAs per query for sparse attention: rank 0 takes the window tile, the others about two
 // selected-entry tiles each.  A function of k alone, so the result is batch-invariant.

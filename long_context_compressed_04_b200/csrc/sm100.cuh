@@ -251,6 +251,19 @@ __device__ __forceinline__ bool named_barrier_and(int id, int nthreads, bool v) 
     return r != 0;
 }
 
+// 2^x by the PTX approximate base-2 exponential (flush-to-zero; 2^-inf = +0), for softmax
+// weights that are rounded to bf16 afterwards.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// L2 prefetch of `bytes` contiguous bytes (16-byte aligned address, multiple of 16 bytes).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
