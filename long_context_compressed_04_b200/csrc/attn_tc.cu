@@ -16,16 +16,17 @@
 // order.  Both splits depend only on k or on the query's own length, never on the batch,
 // so both paths are batch-invariant.
 //
-// Roles per CTA (10 warps, persistent over items):
+// Roles per CTA (11 warps, persistent over items):
 //   warp 0      producer: dense tiles by two 2D TMA loads (64 channels x 128 rows each,
 //               128-byte swizzle), sparse tiles by TMA tile::gather4 loads of the selected
 //               rows (4 rows x 64 channels each; an invalid index is row -1, zero-filled) into
 //               the same swizzled layout; a per-tile validity mask; 3-stage ring.
-//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
-//               S = Q K^T as two M=64 x N=64 halves (keys 0-63 -> TMEM lanes 0-15 of each
-//               quarter, keys 64-127 -> lanes 16-31), and P V accumulated in TMEM as two
-//               outputs O_0 / O_1 (the key column-halves below), each two M=64 x N=64 halves
-//               (channels 0-63 / 64-127), V being the key tile read MN-major.
+//   warp 1      TMEM allocation; lane 0 issues tcgen05.mma kind::f16 S = Q K^T as two
+//               M=64 x N=64 halves (keys 0-63 -> TMEM lanes 0-15 of each quarter, keys
+//               64-127 -> lanes 16-31).
+//   warp 10     lane 0 issues P V, accumulated in TMEM as two outputs O_0 / O_1 (the key
+//               column-halves below), each two M=64 x N=64 halves (channels 0-63 / 64-127),
+//               V being the key tile read MN-major.
 //   warps 2-9   two warps per TMEM lane quarter.  Per item: q heads RoPEd at t and the
 //               window tile into shared memory (all 256 threads).  Per tile: 32 keys of one
 //               head per thread from TMEM, softmax in the log2 domain against a reference
@@ -52,7 +53,8 @@ constexpr int kBlk = kTK * 128;              // one 64-channel slice of a key ti
 constexpr int kTileBytes = 2 * kBlk;         // 32 KB
 constexpr int kQBlk = kH * 128;              // one 64-channel slice of Q (8 KB)
 constexpr int kPBlk = kH * 128;              // one 64-key slice of P (8 KB)
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
+constexpr int kPvWarp = 10;                  // the P V issuer
 constexpr float kRescale = 8.f;              // a tile moves the reference maximum only when
                                              // it exceeds it by more than 2^8
 constexpr int kDenseChunkTiles = 8;
@@ -237,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(odone, 1);
         mbar_init(cpart_full, 4 * a.cluster);
         mbar_init(cpart_free, 4 * a.cluster);
-        mbar_init(drain, 1);
+        mbar_init(drain, 2);   // both MMA issuers
         *abort_flag = 0;
         mbar_fence_init();
         prefetch_tmap(a.idx ? &tmap_g : &tmap_e);
@@ -397,12 +399,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < kStages; s++)
             if (issued[s]) mbar_drain(&full[s], (issued[s] - 1) & 1, a.st);
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == kPvWarp) {
         if (lane == 0) {
-            // ---------------- MMA issuer ----------------
-            // S of a tile is issued before the P V of the previous one.  P V accumulates into
-            // the item's two running outputs in TMEM, one per key column-half: O_0 takes keys
-            // 0-31 and 64-95 of every tile (K-steps 0, 1, 4, 5), O_1 keys 32-63 and 96-127.
+            // ---------------- MMA issuers ----------------
+            // One tcgen05.mma costs its issuing thread tens of cycles however small it is, so
+            // the small MMAs here are issued by two threads: warp 1 issues S = Q K^T of every
+            // tile (as soon as its keys and an S buffer are there), warp kPvWarp issues P V.
+            // P V accumulates into the item's two running outputs in TMEM, one per key
+            // column-half: O_0 takes keys 0-31 and 64-95 of every tile (K-steps 0, 1, 4, 5),
+            // O_1 keys 32-63 and 96-127.  P of a tile being ready implies its S was consumed,
+            // so the P V issuer follows the key ring without waiting on the loads, and its
+            // commits alone release key stages, P buffers and the item.
+            const bool s_role = warp == 1;
             int stage = 0;
             uint32_t ph = 0;
             int nt = 0, nitem = 0;
@@ -410,37 +418,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
                 AItem x;
                 if (!get_item(a, it, x, false)) continue;
-                if (!mbar_wait(prep_full, nitem & 1, abort_flag, a.st)) break;
-                fence_async_smem();
-                tc_fence_after();
-                const uint8_t* prev_k = nullptr;
-                int prev_stage = -1, prev_sb = 0;
-                auto issue_pv = [&](bool first) -> bool {
-                    const int psb = prev_sb;
-                    if (!mbar_wait(&p_full[psb], ((nt - 1) >> 1) & 1, abort_flag, a.st)) return false;
+                if (s_role) {
+                    if (!mbar_wait(prep_full, nitem & 1, abort_flag, a.st)) break;
+                    fence_async_smem();
                     tc_fence_after();
-#pragma unroll
-                    for (int ch = 0; ch < 2; ch++) {
-#pragma unroll
-                        for (int t = 0; t < 4; t++) {
-                            const int kk = (t >> 1) * 4 + ch * 2 + (t & 1);
-                            const uint64_t ad =
-                                smem_desc_k_sw128(sP + psb * 2 * kPBlk + (kk >> 2) * kPBlk) +
-                                ((uint32_t)((kk & 3) * 32) >> 4);
-#pragma unroll
-                            for (int half = 0; half < 2; half++) {
-                                const uint32_t d = tmem_O + ch * 64 + ((uint32_t)(half * 16) << 16);
-                                const uint64_t bd =
-                                    smem_desc_mn_sw128(prev_k + half * kBlk + kk * 2048, kBlk);
-                                mma_f16(d, ad, bd, kIdescPV, (first && t == 0) ? 0u : 1u);
-                            }
-                        }
-                    }
-                    mma_commit(&p_empty[psb]);
-                    if (prev_stage >= 0) mma_commit(&empty[prev_stage]);
-                    mma_commit(pvdone);
-                    return true;
-                };
+                }
                 for (int jj = 0; jj < x.ntiles && ok; jj++) {
                     const int j = x.tile0 + jj;
                     const uint8_t* kb;
@@ -448,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (j == 0) {
                         kb = sW;
                     } else {
-                        if (!mbar_wait(&full[stage], ph, abort_flag, a.st)) {
+                        if (s_role && !mbar_wait(&full[stage], ph, abort_flag, a.st)) {
                             ok = false;
                             break;
                         }
@@ -460,45 +442,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     const int sb = nt & 1;
-                    if (!mbar_wait(&s_empty[sb], ((nt >> 1) & 1) ^ 1, abort_flag, a.st)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    // the two key halves are independent accumulators: interleave their chains
-#pragma unroll
-                    for (int kk = 0; kk < 8; kk++) {
-#pragma unroll
-                        for (int half = 0; half < 2; half++) {
-                            const uint32_t d = tmem_S + sb * 64 + ((uint32_t)(half * 16) << 16);
-                            const int blk = kk >> 2;
-                            const uint32_t off = (uint32_t)((kk & 3) * 32) >> 4;
-                            const uint64_t ad = smem_desc_k_sw128(sQ + blk * kQBlk) + off;
-                            const uint64_t bd =
-                                smem_desc_k_sw128(kb + blk * kBlk + half * 64 * 128) + off;
-                            mma_f16(d, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+                    if (s_role) {
+                        if (!mbar_wait(&s_empty[sb], ((nt >> 1) & 1) ^ 1, abort_flag, a.st)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        // the two key halves are independent accumulators: interleave their chains
+#pragma unroll
+                        for (int kk = 0; kk < 8; kk++) {
+#pragma unroll
+                            for (int half = 0; half < 2; half++) {
+                                const uint32_t d = tmem_S + sb * 64 + ((uint32_t)(half * 16) << 16);
+                                const int blk = kk >> 2;
+                                const uint32_t off = (uint32_t)((kk & 3) * 32) >> 4;
+                                const uint64_t ad = smem_desc_k_sw128(sQ + blk * kQBlk) + off;
+                                const uint64_t bd =
+                                    smem_desc_k_sw128(kb + blk * kBlk + half * 64 * 128) + off;
+                                mma_f16(d, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+                            }
+                        }
+                        mma_commit(&s_full[sb]);
+                    } else {
+                        if (!mbar_wait(&p_full[sb], (nt >> 1) & 1, abort_flag, a.st)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int ch = 0; ch < 2; ch++) {
+#pragma unroll
+                            for (int t = 0; t < 4; t++) {
+                                const int kk = (t >> 1) * 4 + ch * 2 + (t & 1);
+                                const uint64_t ad =
+                                    smem_desc_k_sw128(sP + sb * 2 * kPBlk + (kk >> 2) * kPBlk) +
+                                    ((uint32_t)((kk & 3) * 32) >> 4);
+#pragma unroll
+                                for (int half = 0; half < 2; half++) {
+                                    const uint32_t d = tmem_O + ch * 64 + ((uint32_t)(half * 16) << 16);
+                                    const uint64_t bd =
+                                        smem_desc_mn_sw128(kb + half * kBlk + kk * 2048, kBlk);
+                                    mma_f16(d, ad, bd, kIdescPV, (jj == 0 && t == 0) ? 0u : 1u);
+                                }
+                            }
+                        }
+                        mma_commit(&p_empty[sb]);
+                        if (my_stage >= 0) mma_commit(&empty[my_stage]);
+                        mma_commit(pvdone);
                     }
-                    mma_commit(&s_full[sb]);
-                    if (jj > 0 && !issue_pv(jj == 1)) {
-                        ok = false;
-                        break;
-                    }
-                    prev_k = kb;
-                    prev_stage = my_stage;
-                    prev_sb = sb;
                     nt++;
                 }
                 if (!ok) break;
-                if (!issue_pv(x.ntiles == 1)) break;
-                mma_commit(odone);
-                mma_commit(prep_empty);
+                if (!s_role) {
+                    mma_commit(odone);
+                    mma_commit(prep_empty);
+                }
                 nitem++;
             }
             mma_commit(drain);
             mbar_drain(drain, 0, a.st);
         }
-    } else if (warp >= 2) {
+    } else if (warp >= 2 && warp < 10) {
         // ---------------- softmax / epilogue (warps 2..9) ----------------
         // Two warps share each TMEM lane quarter (the quarter is fixed by the warp's rank
         // modulo 4): warp column-half `ch` reads S columns ch*32 .. ch*32+31 of its lanes, so a
@@ -697,8 +701,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float mnew = need ? tmax : mref;
                     const float corr = !need ? 1.f : (mref == -INFINITY ? 0.f : exp2f(mref - mnew));
                     if (jj > 0 && __any_sync(0xffffffffu, corr != 1.f)) {
-                        // O_ch must hold every earlier P V of the item before it is rescaled
-                        if (!mbar_wait_warp(pvdone, (nt - 1) & 1, abort_flag, a.st)) {
+                        // O_ch must hold every earlier P V of the item before it is rescaled.
+                        // P V of tile nt - 2 is complete once this tile's P buffer is free;
+                        // then pvdone has completed nt - 1 or nt phases, and its parity wait
+                        // for phase nt - 1 cannot alias an older one
+                        if (!mbar_wait_warp(&p_empty[sb], ((nt >> 1) & 1) ^ 1, abort_flag, a.st) ||
+                            !mbar_wait_warp(pvdone, (nt - 1) & 1, abort_flag, a.st)) {
                             ok = false;
                             break;
                         }

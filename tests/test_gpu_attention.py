@@ -158,3 +158,74 @@ def test_batch_invariance_bitwise_576_fp8_sweep():
         assert len(outs[tgt]) >= 3
         for v in outs[tgt][1:]:
             assert torch.equal(v.view(torch.int16), ref.view(torch.int16))
+
+
+def _scale_rows_pow2(rows, fmt, D, p):
+    """Entry e multiplied by 2^p[e] (exact: bf16 values, fp8 block scales and the bf16 RoPE
+    part all scale by a power of two without rounding)."""
+    out = rows.copy()
+    f = np.exp2(p.astype(np.float64)).astype(np.float32)[:, None]
+    def bf16_scale(u16):
+        x = (u16.astype(np.uint32) << 16).view(np.float32) * f
+        return (x.view(np.uint32) >> 16).astype(np.uint16)
+    if fmt == 0:
+        out.view(np.uint16)[:] = bf16_scale(out.view(np.uint16))
+    else:
+        out[:, 512:528].view(np.float32)[:] = out[:, 512:528].view(np.float32) * f
+        out[:, 528:656].view(np.uint16)[:] = bf16_scale(out[:, 528:656].view(np.uint16))
+    return out
+
+
+@pytest.mark.parametrize("mode,H,D,fmt", [("sparse", 64, 128, 0), ("dense", 64, 128, 0),
+                                          ("sparse", 128, 576, 1)])
+def test_rising_scores_move_the_reference_maximum(mode, H, D, fmt):
+    # Entry e is scaled by 2^min(e // 128, 3): in entry order the scores of later key tiles
+    # exceed the running reference maximum by far more than 2^8 in the exponent, so the
+    # kernels must rescale their partial outputs; in reverse order the maximum comes first
+    # and later tiles never move it.  Attention is invariant under the order of its keys,
+    # and both runs see the same rounded q and keys (so the same logits), so the outputs
+    # may differ only by the rounding of P and of the bf16 output: a few ulps of the output's
+    # largest binade (2^-6 of its magnitude).  (The
+    # oracle keeps q unrounded, which at these logit magnitudes leaves near-tied heads
+    # ill-conditioned; the unscaled cases above pin both orders' arithmetic to it.)
+    if mode == "dense":
+        wl = synth.make_workload("t", B=1, T=[128 * 2500 + 77], D=D, H=H, m=128, span=128,
+                                 seed=36, device=DEV)
+    else:
+        wl = synth.make_workload("t", B=2, T=[20000, 9000], D=D, H=H, m=4, span=8, H_I=4,
+                                 d_I=64, k=512, fmt=fmt, seed=36, device=DEV)
+    rows, _ = _orc.compress(wl.to("cpu"))
+    ent_off = _orc.i64(wl.ent_off)
+    bounds = [(int(ent_off[b]), int(ent_off[b + 1]) if b + 1 < wl.B else rows.shape[0])
+              for b in range(wl.B)]
+    p = np.zeros(rows.shape[0], np.int64)
+    for lo, hi in bounds:
+        p[lo:hi] = np.minimum(np.arange(hi - lo) // 128, 3)
+    rows = _scale_rows_pow2(rows, fmt, D, p)
+    outs = []
+    for order in ("rising", "falling"):
+        buf = pipeline.alloc(wl, DEV)
+        if mode == "dense":
+            r = rows.copy()
+            if order == "falling":
+                for lo, hi in bounds:
+                    r[lo:hi] = rows[lo:hi][::-1]
+            buf.entries.copy_(torch.from_numpy(r))
+        else:
+            buf.entries.copy_(torch.from_numpy(rows))
+            idx = _random_idx(wl, 5, pad=3)
+            if order == "falling":
+                for q in range(wl.Q):
+                    v = idx[q][idx[q] >= 0][::-1]
+                    idx[q, :len(v)] = v
+            buf.idx.copy_(torch.from_numpy(idx))
+        pipeline.attend(wl, buf)
+        torch.cuda.synchronize()
+        assert int(buf.dev_status.item()) == 0
+        outs.append(buf.out.float().cpu().numpy())
+    a, b = outs
+    assert np.all(np.isfinite(a)) and np.all(np.isfinite(b))
+    mag = np.abs(b).max()
+    assert mag > 4.0                     # the scaled entries dominate the output
+    assert np.abs(a - b).max() <= mag * 2.0 ** -6
+    assert np.linalg.norm(a - b) <= 5e-3 * np.linalg.norm(b)
