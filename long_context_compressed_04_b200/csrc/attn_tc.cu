@@ -12,8 +12,8 @@
 // stores its partial state of every head straight into the shared memory of the rank that
 // finishes that head (posted distributed-shared-memory stores), and each rank combines its
 // slice of the heads locally (ranks in order, the sink first).  Dense attention splits every
-// query into fixed 8-tile chunks whose partial states a second kernel combines in chunk
-// order.  Both splits depend only on k or on the query's own length, never on the batch,
+// query into the window tile and fixed 8-tile chunks of entries, whose partial states a
+// second kernel combines in chunk order.  Both splits depend only on k or on the query's own length, never on the batch,
 // so both paths are batch-invariant.
 //
 // Roles per CTA (11 warps, persistent over items):
@@ -54,6 +54,7 @@ constexpr int kTileBytes = 2 * kBlk;         // 32 KB
 constexpr int kQBlk = kH * 128;              // one 64-channel slice of Q (8 KB)
 constexpr int kPBlk = kH * 128;              // one 64-key slice of P (8 KB)
 constexpr int kThreads = 352;
+static_assert(kTK / 4 == 32, "one 4-row gather group per producer lane");
 constexpr int kPvWarp = 10;                  // the P V issuer
 constexpr float kRescale = 8.f;              // a tile moves the reference maximum only when
                                              // it exceeds it by more than 2^8
@@ -146,8 +147,15 @@ __device__ __forceinline__ bool get_item(const AttnTcArgs& a, int it, AItem& x, 
         }
         return x.ntiles > 0;
     }
-    x.tile0 = x.c * a.chunk_tiles;
-    x.ntiles = min(a.chunk_tiles, 1 + n_et - x.tile0);
+    // dense: chunk 0 is the window tile alone (its rows are built in-kernel, which takes as
+    // long as several entry tiles), chunks 1.. take chunk_tiles entry tiles each
+    if (x.c == 0) {
+        x.tile0 = 0;
+        x.ntiles = 1;
+    } else {
+        x.tile0 = 1 + (x.c - 1) * a.chunk_tiles;
+        x.ntiles = min(a.chunk_tiles, 1 + n_et - x.tile0);
+    }
     return x.ntiles > 0;
 }
 
@@ -370,20 +378,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const unsigned vm = __ballot_sync(0xffffffffu, row >= 0);
                         if (lane == 0) smask[stage * 4 + rr] = vm;
                     }
+                    // the tile's byte count is expected before any gather is issued; then every
+                    // lane issues the two gathers (both channel halves) of its own 4-row group,
+                    // since one thread issuing all 64 would serialise on the issue cost
+                    if (lane == 0) mbar_arrive_expect_tx(&full[stage], kTileBytes);
                     __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(&full[stage], kTileBytes);
-#pragma unroll 4
-                        for (int g = 0; g < kTK / 4; g++) {
-                            const int32_t r0 = rows[4 * g], r1 = rows[4 * g + 1],
-                                          r2 = rows[4 * g + 2], r3 = rows[4 * g + 3];
-                            tma_gather4(dst + 4 * g * 128, &tmap_g, &full[stage], 0, r0, r1, r2, r3);
-                            tma_gather4(dst + kBlk + 4 * g * 128, &tmap_g, &full[stage], 64, r0, r1,
-                                        r2, r3);
-                        }
-                    } else {
-                        mbar_arrive(&full[stage]);
+                    {
+                        const int g = lane;   // kTK / 4 = 32 row groups
+                        const int32_t r0 = rows[4 * g], r1 = rows[4 * g + 1], r2 = rows[4 * g + 2],
+                                      r3 = rows[4 * g + 3];
+                        tma_gather4(dst + 4 * g * 128, &tmap_g, &full[stage], 0, r0, r1, r2, r3);
+                        tma_gather4(dst + kBlk + 4 * g * 128, &tmap_g, &full[stage], 64, r0, r1, r2, r3);
                     }
+                    if (lane != 0) mbar_arrive(&full[stage]);
                 }
                 if (lane == 0) mbar_arrive(&full[stage]);
                 issued[stage]++;
@@ -933,8 +940,7 @@ __global__ void __launch_bounds__(kD) attn_combine_kernel(const AttnTcArgs a) {
         if (n > a.max_n) n = a.max_n;
         const int64_t avail = a.ent_rows - a.ent_off[b];
         if ((int64_t)n > avail) n = avail > 0 ? (int)avail : 0;
-        const int total = 1 + (n + kTK - 1) / kTK;
-        nch = (total + a.chunk_tiles - 1) / a.chunk_tiles;
+        nch = 1 + ((n + kTK - 1) / kTK + a.chunk_tiles - 1) / a.chunk_tiles;
     }
     const float sk = a.sink[h] * kLog2e;
     float cs = 1.f, sn = 0.f;   // inverse RoPE of the last 64 channels
@@ -1034,9 +1040,9 @@ int max_active_clusters(int C) {
     return cache[C];
 }
 
+// the window chunk, then the entry tiles in chunks of kDenseChunkTiles
 int dense_chunks_per_q(int max_n) {
-    const int tiles = 1 + (max_n + kTK - 1) / kTK;
-    return (tiles + kDenseChunkTiles - 1) / kDenseChunkTiles;
+    return 1 + ((max_n + kTK - 1) / kTK + kDenseChunkTiles - 1) / kDenseChunkTiles;
 }
 
 }  // namespace
