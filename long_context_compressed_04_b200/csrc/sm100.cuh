@@ -279,6 +279,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// Bulk copy of `bytes` contiguous bytes global -> shared (16-byte aligned addresses, a
+// multiple of 16 bytes), completing on `bar` with its byte count.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // TMA gather of 4 rows (row coordinates r0..r3, each may be out of range -> zero fill) of a
 // 2D tensor map whose box is one row high; the rows land consecutively at dst.
 __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,

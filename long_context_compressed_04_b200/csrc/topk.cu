@@ -98,8 +98,12 @@ struct Shared {
     uint32_t scan_tmp[33];
     unsigned long long scan64[33];
     uint32_t bin, krem, key_or, key_and, ncand;
+    uint32_t s_or, s_and, c_or, c_and;   // OR / AND of the sample and of the candidates
+    uint64_t stage_bar;                   // bulk copies of the row into shared memory
+    int abort;
     uint32_t cand[kMaxCand];
 };
+
 
 // Exclusive prefix sum over the CTA of a 64-bit `v`; `total` gets the CTA sum.
 __device__ __forceinline__ unsigned long long block_exclusive_scan64(unsigned long long v,
@@ -179,6 +183,37 @@ __device__ __forceinline__ void pick_bin(Shared& sh, uint32_t& krem) {
     krem = sh.krem;
 }
 
+// The kth largest (1-based, kth <= cnt) of the cnt keys list[0 .. cnt) in shared memory,
+// whose OR and AND are kor / kand: 11-bit radix digits from the highest bit that varies;
+// `krem` gets the number of keys equal to it that the kth largest include.  All threads
+// call it; it ends with the CTA synchronised.
+__device__ __forceinline__ uint32_t select_kth_list(Shared& sh, const uint32_t* list,
+                                                    uint32_t cnt, uint32_t kth, uint32_t kor,
+                                                    uint32_t kand, uint32_t& krem) {
+    const uint32_t vary = kor ^ kand;
+    uint32_t prefix = kand & ~vary, mask = ~vary;
+    krem = kth;
+    int top = vary ? 31 - __clz(vary) : -1;
+    while (top >= 0) {
+        const int width = top >= 10 ? 11 : top + 1;
+        const int shift = top + 1 - width;
+        const uint32_t bmask = (1u << width) - 1u;
+        for (int x = threadIdx.x; x < kBins; x += kThreads) sh.hist[x] = 0u;
+        __syncthreads();
+        for (uint32_t c = threadIdx.x; c < cnt; c += kThreads) {
+            const uint32_t key = list[c];
+            if ((key & mask) == prefix) atomicAdd(&sh.hist[(key >> shift) & bmask], 1u);
+        }
+        __syncthreads();
+        pick_bin(sh, krem);
+        prefix |= sh.bin << shift;
+        mask |= bmask << shift;
+        top = shift - 1;
+        __syncthreads();
+    }
+    return prefix;
+}
+
 // STAGED: the query's row is first copied to shared memory as keys (16-byte loads, eight in
 // flight per thread) and every pass reads it from there.
 template <bool STAGED>
@@ -186,6 +221,7 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_seq,
     const int32_t* __restrict__ q_pos, const int64_t* __restrict__ seq_len, int B, int m,
     int max_n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ dev_status) {
+    using namespace sm100;
     __shared__ Shared sh;
     const int qq = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31;
@@ -208,6 +244,8 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         sh.key_or = 0u;
         sh.key_and = 0xFFFFFFFFu;
         sh.ncand = 0u;
+        sh.s_or = sh.c_or = 0u;
+        sh.s_and = sh.c_and = 0xFFFFFFFFu;
     }
     __syncthreads();
     uint32_t kor = 0u, kand = 0xFFFFFFFFu;
@@ -239,6 +277,55 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         }
     };
     if constexpr (STAGED) {
+      if (vec) {
+        // the whole row in flight at once: bulk copies (8 KB each, one per lane of warp 0)
+        // straight into shared memory, then one pass turns the scores into keys in place
+        const int n4 = n >> 2;
+        const uint32_t bytes = (uint32_t)n4 * 16u;
+        if (tid == 0) {
+            mbar_init(&sh.stage_bar, 1);
+            mbar_fence_init();
+            sh.abort = 0;
+        }
+        __syncthreads();
+        if (tid < 32) {
+            if (lane == 0) mbar_arrive_expect_tx(&sh.stage_bar, bytes);
+            __syncwarp();
+            constexpr uint32_t kPiece = 8192;
+            for (uint32_t off = (uint32_t)lane * kPiece; off < bytes; off += 32 * kPiece)
+                bulk_load(reinterpret_cast<uint8_t*>(skey4) + off,
+                          reinterpret_cast<const uint8_t*>(s) + off, min(kPiece, bytes - off),
+                          &sh.stage_bar);
+        }
+        if (!named_barrier_and(1, kThreads, mbar_wait(&sh.stage_bar, 0, &sh.abort, dev_status))) {
+            // timed out (flagged): let the copies drain before the CTA leaves
+            mbar_drain(&sh.stage_bar, 0, dev_status);
+            return;
+        }
+        for (int j = tid; j < ((n + 3) >> 2); j += kThreads) {
+            float e[4];
+            if (j < n4) {
+                const uint4 v = skey4[j];
+                e[0] = __uint_as_float(v.x);
+                e[1] = __uint_as_float(v.y);
+                e[2] = __uint_as_float(v.z);
+                e[3] = __uint_as_float(v.w);
+            } else {
+#pragma unroll
+                for (int z = 0; z < 4; z++) e[z] = 4 * j + z < n ? s[4 * j + z] : 0.f;
+            }
+            uint32_t kk[4];
+#pragma unroll
+            for (int z = 0; z < 4; z++) {
+                kk[z] = score_key(e[z]);
+                if (4 * j + z < n) {
+                    kor |= kk[z];
+                    kand &= kk[z];
+                }
+            }
+            skey4[j] = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+        }
+      } else {
         constexpr int kBatch = 8;
         for (int i0 = 4 * tid; i0 < n; i0 += 4 * kThreads * kBatch) {
             float4 v[kBatch];
@@ -270,6 +357,7 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
                 if (i < n) skey4[i >> 2] = make_uint4(kk[0], kk[1], kk[2], kk[3]);
             }
         }
+      }
     } else {
         for (int c0 = 0; c0 < n; c0 += kChunk) {
             uint32_t key[4];
@@ -294,6 +382,125 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     }
     __syncthreads();
     const uint32_t diff = sh.key_or ^ sh.key_and;   // bits that vary across the row
+    const int wid = tid >> 5;
+    if constexpr (STAGED) {
+        // Rows much longer than k: a bound B from a fixed strided sample of the row, chosen so
+        // that about 2k keys of the row are >= B.  One pass marks the keys >= B in words of 32
+        // entries; if they number between k and kMaxCand they hold the k largest, which are
+        // then selected among them alone and written from the words.  The sample only decides
+        // how fast the unique result is found: otherwise the general passes below run.
+        const long long r_ll = (2LL * k * kThreads + n - 1) / n + 8;
+        if (diff != 0u && r_ll <= kThreads / 2) {
+            // B: the lower edge of the bin (of one 11-bit digit from the sample's highest
+            // varying bit) that holds the sample's r-th largest key; at least r keys are >= B
+            const uint32_t sv = skey[(int)(((long long)tid * n) / kThreads)];
+            {
+                uint32_t so = sv, sa = sv;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    so |= __shfl_xor_sync(0xffffffffu, so, o);
+                    sa &= __shfl_xor_sync(0xffffffffu, sa, o);
+                }
+                if (lane == 0) {
+                    atomicOr(&sh.s_or, so);
+                    atomicAnd(&sh.s_and, sa);
+                }
+            }
+            for (int x = tid; x < kBins; x += kThreads) sh.hist[x] = 0u;
+            __syncthreads();
+            const uint32_t svary = sh.s_or ^ sh.s_and;
+            uint32_t B = sh.s_and;   // all sample keys equal
+            if (svary) {
+                const int stop = 31 - __clz(svary);
+                const int width = stop >= 10 ? 11 : stop + 1;
+                const int shift = stop + 1 - width;
+                atomicAdd(&sh.hist[(sv >> shift) & ((1u << width) - 1u)], 1u);
+                __syncthreads();
+                uint32_t rk = (uint32_t)r_ll;
+                pick_bin(sh, rk);
+                const uint32_t hi = stop >= 31 ? 0u : (sh.s_and >> (stop + 1)) << (stop + 1);
+                B = hi | (sh.bin << shift);
+            }
+            for (int r = wid; r < nwords; r += kWarps) {
+                const int i = (r << 5) + lane;
+                const bool in = i < n;
+                const uint32_t key = in ? skey[i] : 0u;
+                const uint32_t ge = __ballot_sync(0xffffffffu, in && key >= B);
+                if (lane == 0) selw[r] = ge;
+            }
+            __syncthreads();
+            const int wpt = (nwords + kThreads - 1) / kThreads;
+            const int w0 = min(tid * wpt, nwords), w1 = min(w0 + wpt, nwords);
+            uint32_t cnt = 0;
+            for (int w = w0; w < w1; w++) cnt += __popc(selw[w]);
+            uint32_t total;
+            uint32_t off = block_exclusive_scan(cnt, sh.scan_tmp, total);
+            if (total >= (uint32_t)k && total <= (uint32_t)kMaxCand) {
+                // the candidates' keys, in entry order, and their OR / AND
+                uint32_t co = 0u, ca = 0xFFFFFFFFu;
+                for (int w = w0; w < w1; w++) {
+                    uint32_t bits = selw[w];
+                    while (bits) {
+                        const int bit = __ffs(bits) - 1;
+                        const uint32_t key = skey[(w << 5) + bit];
+                        sh.cand[off++] = key;
+                        co |= key;
+                        ca &= key;
+                        bits &= bits - 1;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    co |= __shfl_xor_sync(0xffffffffu, co, o);
+                    ca &= __shfl_xor_sync(0xffffffffu, ca, o);
+                }
+                if (lane == 0) {
+                    atomicOr(&sh.c_or, co);
+                    atomicAnd(&sh.c_and, ca);
+                }
+                __syncthreads();
+                uint32_t kr;
+                const uint32_t T =
+                    select_kth_list(sh, sh.cand, total, (uint32_t)k, sh.c_or, sh.c_and, kr);
+                // keys > T and the first kr keys == T, in entry order: per thread its words'
+                // counts, one 64-bit scan (ties high, keys > T low), then the writes
+                uint32_t cg = 0, ce = 0;
+                for (int w = w0; w < w1; w++) {
+                    uint32_t bits = selw[w];
+                    while (bits) {
+                        const uint32_t key = skey[(w << 5) + __ffs(bits) - 1];
+                        cg += key > T;
+                        ce += key == T;
+                        bits &= bits - 1;
+                    }
+                }
+                unsigned long long tot;
+                const unsigned long long pre =
+                    block_exclusive_scan64(((unsigned long long)ce << 32) | cg, sh.scan64, tot);
+                uint32_t ties = (uint32_t)(pre >> 32);
+                uint32_t pos = (uint32_t)pre + min(ties, kr);
+                for (int w = w0; w < w1; w++) {
+                    uint32_t bits = selw[w];
+                    while (bits) {
+                        const int bit = __ffs(bits) - 1;
+                        const uint32_t key = skey[(w << 5) + bit];
+                        bool take = key > T;
+                        if (key == T) take = ties++ < kr;
+                        if (take) {
+                            if (pos < (uint32_t)k) out[pos] = (w << 5) + bit;
+                            pos++;
+                        }
+                        bits &= bits - 1;
+                    }
+                }
+                // the row's total; NaN scores (no total order) break it
+                if (tid == 0 && (uint32_t)tot + min((uint32_t)(tot >> 32), kr) != (uint32_t)k)
+                    flag(dev_status, CSA_DEV_NAN);
+                return;
+            }
+            __syncthreads();   // the general passes reuse the shared state
+        }
+    }
     uint32_t prefix = sh.key_and & ~diff;           // = the bits all keys share
     uint32_t mask = ~diff;
     uint32_t krem = (uint32_t)k;
@@ -351,7 +558,6 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     }
     const uint32_t T = prefix;   // the k-th largest key; krem keys equal to T are taken
     // marking: word r holds the entries 32 r .. 32 r + 31 (bit = lane)
-    const int wid = tid >> 5;
     for (int r = wid; r < nwords; r += kWarps) {
         const int i = (r << 5) + lane;
         const bool in = i < n;

@@ -89,6 +89,47 @@ def test_long_rows_massive_ties_bit_exact():
     _exact(wl)
 
 
+def _scores_from_scales(wl, ks):
+    """Every key row and every query head the same positive vector, all weights 1: each
+    entry's score is its key scale times one positive constant per query, so the scales
+    set the ranking exactly."""
+    row = wl.kI[0].clone()
+    row[row == 0] = 0x38   # e4m3 1.0 wherever the row is 0, so q.k = |k|^2 > 0
+    wl.kI[:] = row
+    wl.qI[:] = row
+    wl.w.fill_(1.0)
+    wl.qs.fill_(1.0)
+    wl.ks.copy_(torch.as_tensor(ks, dtype=torch.float32, device=DEV))
+
+
+def test_sampled_bound_too_high_falls_back():
+    # 40000 entries, top-512: the strided sample the selection starts from holds the 1024
+    # largest scores of the row (distinct), so fewer than k keys reach the bound taken
+    # from it and the general radix passes must run; the result stays the unique top-k
+    wl = synth.make_workload("t", B=1, T=[160000], D=128, H=16, m=4, span=8, H_I=16,
+                             d_I=128, k=512, seed=24, device=DEV)
+    n = 40000
+    ks = np.random.default_rng(7).uniform(1.0, 2.0, wl.kI.shape[0]).astype(np.float32)
+    sample = (np.arange(1024, dtype=np.int64) * n) // 1024
+    ks[sample] = 100.0 + np.arange(1024, dtype=np.float32)
+    _scores_from_scales(wl, ks)
+    idx = _exact(wl)
+    # the top 512 are the upper half of the sample positions
+    assert np.array_equal(idx[0], np.sort(sample[512:]))
+
+
+def test_sampled_bound_too_many_candidates_falls_back():
+    # all but one score equal: every key reaches the bound, far more than the candidate list
+    # holds, so the general passes run; ties go to the lowest entries
+    wl = synth.make_workload("t", B=1, T=[160000], D=128, H=16, m=4, span=8, H_I=16,
+                             d_I=128, k=512, seed=25, device=DEV)
+    ks = np.full(wl.kI.shape[0], 1.5, np.float32)
+    ks[777] = 0.5
+    _scores_from_scales(wl, ks)
+    idx = _exact(wl)
+    assert np.array_equal(idx[0], np.arange(512))
+
+
 def _abs_bound(wl, q):
     """fp32 rounding bound of one query's scores: the dot products accumulate 128 e4m3
     products in fp32 (error <= 2^-17 of the sum of |products| each, doubled for margin)
