@@ -37,6 +37,10 @@ WORKLOADS = {
     "hca_decode_1m_b16": dict(kind="hca", B=16, T=1 << 20, jitter=0, D=128, H=64, fmt=0),
     "csa_decode_1m_b8_fp8": dict(kind="csa", B=8, T=1 << 20, jitter=0, D=576, H=128, H_I=64,
                                  d_I=128, k=1024, fmt=1),
+    # a causal prefill chunk: 8192 new query tokens after 65536 prior tokens; the step
+    # compresses the 2048 entries that pool new tokens, then scores, selects and attends
+    "csa_prefill_8k_on_64k": dict(kind="csa_prefill", B=1, T=65536 + 8192, jitter=0, D=128,
+                                  H=64, H_I=64, d_I=128, k=1024, fmt=0, n_new=8192),
 }
 
 
@@ -72,9 +76,23 @@ def _peaks():
     return 6650.0, "fallback"
 
 
+def _tensor_peak_fp8():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return round(2.0 * float(d["bf16_tflops_sustained"]), 1), \
+            "measured bf16_tflops_sustained x 2 (nominal fp8 / bf16 ratio)"
+    return round(2.0 * 1400.0, 1), "fallback sustained bf16 1400 TFLOP/s x 2 (nominal fp8 / bf16 ratio)"
+
+
 def make_workload(name: str, rank: int, device):
     from long_context_compressed_04_b200 import synth
     c = WORKLOADS[name]
+    if c["kind"] == "csa_prefill":
+        return synth.make_workload(name, B=c["B"], T=c["T"], D=c["D"], H=c["H"], m=4, span=8,
+                                   W=128, fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
+                                   indexer="fp8", queries="prefill", n_new=c["n_new"],
+                                   seed=rank, device=device)
     T = synth.jittered_lengths(c["B"], c["T"], c["jitter"], 1000 + rank) if c["jitter"] else c["T"]
     if c["kind"] == "csa":
         return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
@@ -82,6 +100,37 @@ def make_workload(name: str, rank: int, device):
                                    indexer="fp8", seed=rank, device=device)
     return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=128, span=128, W=128,
                                fmt=c["fmt"], seed=rank, device=device)
+
+
+def new_tokens(wl, name):
+    """Tokens that are new in one step: the last one of every sequence (decode), or the
+    last n_new of every sequence (prefill)."""
+    return WORKLOADS[name].get("n_new", 1)
+
+
+def step_items(wl, name, device):
+    """(item_seq, item_ent): the entries one step compresses, i.e. those that pool a new
+    token (entry i pools positions up to (i+1)m - 1)."""
+    from long_context_compressed_04_b200 import pipeline
+    nn = new_tokens(wl, name)
+    if nn == 1:
+        return pipeline.newest_entry_items(wl, device)
+    seqs, ents = [], []
+    for b in range(wl.B):
+        T_b = int(wl.T[b]) if wl.T.dim() else int(wl.T)
+        first = T_b - nn
+        i0 = max(0, -(-(first + 1) // wl.m) - 1)
+        n_b = int(wl.n_ent[b])
+        ents.append(torch.arange(i0, n_b, dtype=torch.int32))
+        seqs.append(torch.full((n_b - i0,), b, dtype=torch.int32))
+    return torch.cat(seqs).to(device), torch.cat(ents).to(device)
+
+
+def indexer_flops(wl):
+    """Multiply-adds x 2 of the indexer's dot products: every visible (query, entry) pair,
+    every indexer head."""
+    n_vis = ((wl.q_pos.cpu().to(torch.int64) + 1) // wl.m)
+    return int(n_vis.sum()) * wl.H_I * wl.d_I * 2
 
 
 def algorithmic_bytes(wl):
@@ -179,7 +228,8 @@ def gpu_index_for_smi(dev: int) -> str:
     return str(dev)
 
 
-CPU_SAMPLE_SEQS = {"csa_decode_128k_b32": 32, "hca_decode_1m_b16": 16, "csa_decode_1m_b8_fp8": 2}
+CPU_SAMPLE_SEQS = {"csa_decode_128k_b32": 32, "hca_decode_1m_b16": 16, "csa_decode_1m_b8_fp8": 2,
+                   "csa_prefill_8k_on_64k": 64}   # prefill: sampled queries of the chunk
 
 
 def cpu_baseline(name: str, n_seq: int | None = None):
@@ -194,6 +244,25 @@ def cpu_baseline(name: str, n_seq: int | None = None):
     from long_context_compressed_04_b200 import synth
 
     c = WORKLOADS[name]
+    if c["kind"] == "csa_prefill":
+        # the chunk's entry compression plus n_seq of its queries, spread over the chunk
+        import dataclasses
+        wl = make_workload(name, 0, "cpu")
+        sel = torch.linspace(0, wl.Q - 1, n_seq).round().long()
+        ws = dataclasses.replace(wl, q_seq=wl.q_seq[sel], q_pos=wl.q_pos[sel], q=wl.q[sel],
+                                 qI=wl.qI[sel], qs=wl.qs[sel], w=wl.w[sel])
+        rows, _ = _orc.compress(wl)                      # the cache (untimed set-up)
+        iseq, ient = step_items(wl, name, "cpu")
+        t0 = time.perf_counter()
+        _orc.compress(wl, iseq.numpy(), ient.numpy(), entries=rows)
+        idx = _orc.indexer(ws, want_scores=False)
+        _orc.attention(ws, rows, idx)
+        dt = time.perf_counter() - t0
+        return {"value": n_seq / dt, "unit": UNIT, "cores": min(oracle.num_threads(), n_seq),
+                "kind": "oracle",
+                "sample": f"{n_seq} of the {wl.Q} prefill queries of {name} with the chunk's "
+                          f"{int(iseq.numel())} new entries compressed (indexer over every "
+                          f"visible entry, top-k, attention), {dt:.2f} s"}
     T = synth.jittered_lengths(n_seq, c["T"], c["jitter"], 99) if c["jitter"] else [c["T"]] * n_seq
     if c["kind"] == "csa":
         wl = synth.make_workload(name, B=n_seq, T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
@@ -276,7 +345,7 @@ def main():
     buf = pipeline.alloc(wl, dev)
     all_seq, all_ent = pipeline.all_entry_items(wl, dev)
     pipeline.compress(wl, buf, all_seq, all_ent)          # build the compressed cache
-    new_seq, new_ent = pipeline.newest_entry_items(wl, dev)
+    new_seq, new_ent = step_items(wl, args.workload, dev)
     torch.cuda.synchronize()
     del all_seq, all_ent
 
@@ -373,11 +442,14 @@ def main():
     h_in = {k2: v for k2, v in h_in.items() if v is not None}
     pinned = {k2: torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v.cpu())
               for k2, v in h_in.items()}
-    last_rows = (wl.kv_off + (wl.T.to(dev) - 1 - wl.kv_pos0)).long()
-    pin_kv = torch.empty((wl.B, wl.D), dtype=wl.kv.dtype, pin_memory=True).copy_(wl.kv[last_rows].cpu())
-    pin_gate = torch.empty((wl.B, wl.D), dtype=wl.gate.dtype, pin_memory=True).copy_(wl.gate[last_rows].cpu())
-    dev_kv = torch.empty((wl.B, wl.D), dtype=wl.kv.dtype, device=dev)
-    dev_gate = torch.empty((wl.B, wl.D), dtype=wl.gate.dtype, device=dev)
+    nn = new_tokens(wl, args.workload)
+    last_rows = torch.cat([(wl.kv_off[b] + (wl.T.to(dev)[b] - nn - wl.kv_pos0[b]))
+                           + torch.arange(nn, device=dev) for b in range(wl.B)]).long()
+    nr = last_rows.numel()
+    pin_kv = torch.empty((nr, wl.D), dtype=wl.kv.dtype, pin_memory=True).copy_(wl.kv[last_rows].cpu())
+    pin_gate = torch.empty((nr, wl.D), dtype=wl.gate.dtype, pin_memory=True).copy_(wl.gate[last_rows].cpu())
+    dev_kv = torch.empty((nr, wl.D), dtype=wl.kv.dtype, device=dev)
+    dev_gate = torch.empty((nr, wl.D), dtype=wl.gate.dtype, device=dev)
     out_host = torch.empty(buf.out.shape, dtype=buf.out.dtype, pin_memory=True)
     h2d = sum(v.numel() * v.element_size() for v in pinned.values()) + 2 * pin_kv.numel() * 2
     d2h = out_host.numel() * out_host.element_size()
@@ -431,7 +503,19 @@ def main():
     dom_name = next((n for n in (["indexer_score_tc", "indexer_score_simt"] if wl.H_I else [])
                      + ["attn_tc", "attn_simt"] if n in per_kernel), None)
     roof = None
-    if dom_name:
+    if WORKLOADS[args.workload]["kind"] == "csa_prefill" and "indexer_score_tc" in per_kernel:
+        # prefill: the indexer's FP8 dot products bound it (tensor pipe); the peak is the
+        # measured sustained bf16 GEMM rate times the nominal fp8 / bf16 ratio of 2
+        n_l, tot_ms = per_kernel["indexer_score_tc"]
+        avg_s = tot_ms / n_l / 1e3
+        fl = indexer_flops(wl)
+        tpk, tkind = _tensor_peak_fp8()
+        ach = fl / avg_s / 1e12
+        roof = {"bound": "tensor", "kernel": "indexer_score_tc", "achieved": round(ach, 1),
+                "peak": tpk, "unit": "TFLOP/s", "frac": round(ach / tpk, 4), "traffic": None,
+                "peak_source": tkind, "algorithmic_flops_per_launch": fl,
+                "avg_launch_us": round(avg_s * 1e6, 2)}
+    elif dom_name:
         n_l, tot_ms = per_kernel[dom_name]
         avg_s = tot_ms / n_l / 1e3
         alg = alg_of[dom_name]

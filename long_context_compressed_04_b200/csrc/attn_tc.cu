@@ -134,10 +134,14 @@ __device__ __forceinline__ bool get_item(const AttnTcArgs& a, int it, AItem& x, 
     x.n_win = a.W > 0 ? x.t - x.w0 + 1 : 0;
     const int n_et = (x.n_ent + kTK - 1) / kTK;   // entry tiles
     if (a.idx) {
-        // sparse: rank 0 of the query's cluster takes the window tile, ranks 1..C-1 split
-        // the entry tiles contiguously (the host picks C - 1 <= n_et: every rank has one)
+        // sparse: a cluster of one CTA takes every tile; in a larger cluster rank 0 takes
+        // the window tile and ranks 1..C-1 split the entry tiles contiguously (the host
+        // picks C - 1 <= n_et: every rank has one)
         const int C = a.cluster;
-        if (x.c == 0) {
+        if (C == 1) {
+            x.tile0 = 0;
+            x.ntiles = 1 + n_et;
+        } else if (x.c == 0) {
             x.tile0 = 0;
             x.ntiles = 1;
         } else {
@@ -1006,10 +1010,14 @@ constexpr size_t kSmemBytes = 1024 + kStages * kTileBytes + kTileBytes + 2 * kQB
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 static_assert((kRecvFloats + kWtabFloats + 256) % 2 == 0, "mbarriers 8-byte aligned");
 
-// CTAs per query for sparse attention: rank 0 takes the window tile, the others about two
-// selected-entry tiles each.  A function of k alone, so the result is batch-invariant.
+// CTAs per query for sparse attention, a function of k alone (so the result is
+// batch-invariant).  Up to 4 selected-entry tiles (k <= 512, decode): a cluster whose rank
+// 0 takes the window tile and the others about two entry tiles each, for latency.  More
+// (k >= 1024, as in prefill chunks of thousands of queries): one CTA per query over every
+// tile, persistent over queries, which saves each query's cross-CTA exchange.
 int sparse_cluster(int k) {
     const int n_et = (k + kTK - 1) / kTK;
+    if (n_et >= 8) return 1;
     return min(kMaxCluster, 1 + (n_et + 1) / 2);
 }
 
