@@ -9,26 +9,27 @@
 // -- dealt to the ranks in turn (tile j to rank j mod 4).  Each rank ends with an fp32
 // partial state per head (running maximum, sum, unnormalised O) and stores it straight
 // into the shared memory of the rank that finishes that head (16 heads each, posted
-// st.shared::cluster); each rank combines its heads in rank order, the sink first.  Two
-// key buffers let one tile be built while the previous one is in the tensor cores.
+// st.shared::cluster); each rank combines its heads in rank order, the sink first.  Three
+// key buffers let tiles be built while earlier ones are in the tensor cores.
 //   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once; per
 //              tile, 4 threads per key row dequantize the gathered FP8 row (or normalise the
-//              raw window row) into bf16, 128-byte swizzled, 9 blocks of 64 channels; the
-//              next entry tile's rows are copied (cp.async) into a raw staging buffer while
-//              the previous one is converted.
+//              raw window row in place) into bf16, 128-byte swizzled, 9 blocks of 64
+//              channels; each thread's quarter of the next entry row is loaded into
+//              registers while the current tile is converted.
 //   warp 4     TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
 //              S = Q K^T (M = 64 heads, N = 32 keys, 36 K steps of 16 channels) into one of
 //              two S buffers, one tile ahead of O += P V, which goes straight into the TMEM
 //              accumulator: channels 0-255 in TMEM lanes 0-15 of each quarter, 256-511 in
 //              lanes 16-31, 512-575 in lanes 0-15 again (N = 256 + 256 + 64), V being the
 //              key tile read MN-major.
-//   warps 5-8  online softmax in the log2 domain, one head row per lane: P as bf16 into
-//              shared memory; the running maximum is a reference that moves only when a
-//              tile's maximum exceeds it by 2^8, and then the head's O row in TMEM is
-//              rescaled; finally the partial states across the cluster, and for this
-//              rank's heads the combine, the sink, inverse RoPE and the store.
-// A 64 x 576 fp32 accumulator takes 320 TMEM columns, and the query's Q tile (72 KB) fills
-// a third of shared memory: hence 64 heads per CTA and two key buffers of 32 rows.
+//   warps 5-8  online softmax in the log2 domain, one head row per lane, weights by
+//              ex2.approx of one FMA per key: P as bf16 into shared memory; the running
+//              maximum is a reference that moves only when a tile's maximum exceeds it by
+//              2^8, and then the head's O row in TMEM is rescaled; finally the partial
+//              states across the cluster, and for this rank's heads the combine, the sink,
+//              inverse RoPE and the store.
+// A 64 x 576 fp32 accumulator takes 320 TMEM columns, and the query's Q tile (72 KB) takes a
+// third of shared memory: hence 64 heads per CTA and three key buffers of 32 rows.
 // All waits are bounded (timeout -> CSA_DEV_TIMEOUT, drain, free TMEM, return).  A query's
 // arithmetic never depends on the batch.
 #include <mutex>

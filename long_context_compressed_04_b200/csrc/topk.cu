@@ -8,10 +8,14 @@
 //
 // One CTA (1024 threads) per query, scores mapped to order-preserving 32-bit keys.  The
 // goal is the k-th largest key T and the number of keys equal to T to take.
-//  1. Rows of up to 44K scores are staged in shared memory as keys (16-byte loads); the OR
-//     and AND of all keys give the bits every key shares, so the radix starts at the
-//     highest bit that varies (scores of one query share sign and most exponent bits, and a
-//     fixed first digit would put nearly all of them in one bin).
+//  0. Rows of up to 44K scores are staged in shared memory as keys (bulk copies); the OR
+//     and AND of all keys give the bits every key shares.  Rows much longer than k first
+//     try a bound B from a fixed strided sample of 1024 keys (the lower edge of the digit
+//     bin holding the sample's ~(2k * 1024 / n)-th largest): one marking pass finds the
+//     keys >= B; if they number between k and 4096 they hold the k largest, T is selected
+//     among them alone and the output is written from the marks (as in 4).  Otherwise:
+//  1. The radix starts at the highest bit that varies (scores of one query share sign and
+//     most exponent bits, and a fixed first digit would put nearly all of them in one bin).
 //  2. An 11-bit histogram of that digit (shared-memory atomics) and a block-wide scan over
 //     the bins, from the top, give the bin holding the k-th key.
 //  3. Keys in that bin are compacted to a short candidate list (if it fits; one shared
