@@ -85,6 +85,31 @@ def _tensor_peak_fp8():
     return round(2.0 * 1400.0, 1), "fallback sustained bf16 1400 TFLOP/s x 2 (nominal fp8 / bf16 ratio)"
 
 
+def rank_lengths(name: str, rank: int):
+    """Context lengths of the sequences rank `rank` owns: every rank draws its own jittered
+    lengths (and its own inputs, seeded by the rank), so the ranks' sequences are disjoint
+    units of the same shape (weak scaling, no data-path collective)."""
+    from long_context_compressed_04_b200 import synth
+    c = WORKLOADS[name]
+    if c["jitter"]:
+        return synth.jittered_lengths(c["B"], c["T"], c["jitter"], 1000 + rank)
+    return [c["T"]] * c["B"]
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest `x` over the ranks (x itself on one process): a run's time is that of its
+    slowest rank."""
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    if dist:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, steps: int, ms: float) -> float:
+    """Units per second of the whole job: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world * steps / (ms / 1e3)
+
+
 def make_workload(name: str, rank: int, device):
     from long_context_compressed_04_b200 import synth
     c = WORKLOADS[name]
@@ -93,7 +118,7 @@ def make_workload(name: str, rank: int, device):
                                    W=128, fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
                                    indexer="fp8", queries="prefill", n_new=c["n_new"],
                                    seed=rank, device=device)
-    T = synth.jittered_lengths(c["B"], c["T"], c["jitter"], 1000 + rank) if c["jitter"] else c["T"]
+    T = rank_lengths(name, rank) if c["jitter"] else c["T"]
     if c["kind"] == "csa":
         return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
                                    fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
@@ -406,11 +431,7 @@ def main():
             ev[i][1].record()
         barrier()
     launches = L.csa_launch_count() - launches0 + kernels_per_step * K
-    ms = sum(a.elapsed_time(b) for a, b in ev)
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if dist:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dist, dev)
     assert int(buf.dev_status.item()) == 0, "device status flagged during the run"
 
     # second pass: the same step captured into a CUDA graph with a CUDA event pair around
@@ -485,16 +506,11 @@ def main():
             e2e_step()
         ee[i][1].record()
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in ee)
-    te = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-    if dist:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), dist, dev)
 
     peak, peak_kind = _peaks()
     total_bytes, key_bytes = algorithmic_bytes(wl)
-    Qtot = wl.Q * world
-    value = Qtot * K / (ms_max / 1e3)
+    value = whole_job_rate(wl.Q, world, K, ms_max)
     step_s = ms_max / K / 1e3
     # the dominant kernel is the one that moves the method's dominant bytes: the indexer
     # (every visible key, each step) for CSA decode, the attention (every entry) for HCA
@@ -539,7 +555,7 @@ def main():
         "kernels": {k2: {"launches": v[0], "avg_us": round(v[1] / v[0] * 1e3, 2),
                          "share": round(v[1] / sum(x[1] for x in per_kernel.values()), 4)}
                     for k2, v in per_kernel.items()},
-        "e2e": {"value": Qtot * E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(wl.Q, world, E, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "launch": "cuda graph replay" if graph is not None else "eager",
