@@ -61,15 +61,16 @@ constexpr float kRescale = 8.f;              // a tile moves the reference maxim
 constexpr int kDenseChunkTiles = 8;
 constexpr int kMaxK = 2048;
 constexpr int kMaxCluster = 8;
-// sparse receive buffer: C ranks x ceil(kH / C) heads x (kD + 2) floats, largest over C
+// sparse receive buffer: C ranks x ceil(kH / C) heads x (kD + 2) floats, largest over C >= 1
 constexpr int recv_floats(int C) {
     return C > kMaxCluster ? 0
                            : (C * ((kH + C - 1) / C) * (kD + 2) > recv_floats(C + 1)
                                   ? C * ((kH + C - 1) / C) * (kD + 2)
                                   : recv_floats(C + 1));
 }
-constexpr int kRecvFloats = recv_floats(2);
-constexpr int kWtabFloats = ((kH + 1) / 2) * (kMaxCluster + 1);
+constexpr int kRecvFloats = recv_floats(1);
+// combine weights [heads a rank finishes][kMaxCluster + 1]: all kH heads for a cluster of one
+constexpr int kWtabFloats = kH * (kMaxCluster + 1);
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnTcArgs {
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int32_t* srows = sidx + kMaxK;                          // [kStages][128] gather rows
     // sparse: receive buffer of the partial states of this rank's heads from every rank,
     // [cluster][nh][kD] O then [cluster][2][nh] m, l (nh = heads per rank); then the
-    // per-head combine weights [nh][cluster + 1]
+    // per-head combine weights [nh][kMaxCluster + 1], nh <= kH
     float* recv = reinterpret_cast<float*>(srows + kStages * kTK);
     float* wtab = recv + kRecvFloats;
     float* xml = wtab + kWtabFloats;       // [128][2] column-half 1's m, l per (head, half)
