@@ -71,6 +71,13 @@ constexpr int recv_floats(int C) {
 constexpr int kRecvFloats = recv_floats(1);
 // combine weights [heads a rank finishes][kMaxCluster + 1]: all kH heads for a cluster of one
 constexpr int kWtabFloats = kH * (kMaxCluster + 1);
+// a rank of a C-CTA cluster finishes at most ceil(kH / C) heads, each with kMaxCluster + 1
+// weights: the table must hold that for every cluster size the launcher may pick
+constexpr bool wtab_fits(int C) {
+    return C > kMaxCluster ||
+           ((kH + C - 1) / C * (kMaxCluster + 1) <= kWtabFloats && wtab_fits(C + 1));
+}
+static_assert(wtab_fits(1), "combine-weight table too small for some cluster size");
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttnTcArgs {
@@ -527,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = quarter * 16 + (lane & 15);
         const int kh = lane >> 4;               // key half of S / channel half of O
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        bool waited_prev = false;
         int nt = 0, nitem = 0;
         int kst = 0;   // ring position of the next entry tile (mirrors the producer)
         bool ok = true;
@@ -776,6 +784,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // ---- the item's output: O_ch from TMEM, the two column-halves merged ----
             if (ok) ok = mbar_wait_warp(odone, nitem & 1, abort_flag, a.st);
+            // the stores below (out, or the chunk partials of the workspace) may overwrite
+            // what the previous kernel still reads (an earlier call's combine on the same
+            // workspace); a window-only item reaches them without passing the producer's
+            // wait, so every thread here waits for the previous grid once
+            if (!waited_prev) {
+                pdl_wait();
+                waited_prev = true;
+            }
             float o[64];
             {
                 uint32_t ov[64];

@@ -181,10 +181,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     cta_range(a, blockIdx.x, gridDim.x, v0, v1);
     const int n_my = v1 > v0 ? (int)(chunk_of(a, v1 - 1) - chunk_of(a, v0) + 1) : 0;
 
-    // The indexer reads only its inputs (keys and query heads), never an earlier kernel's
-    // output, and its score writes are safe once it has started (the previous step's top-k
-    // finished before the kernel before this one passed its own wait): let the next kernel
-    // launch right away; the wait at the end keeps completion ordered for later kernels.
+    // The indexer reads only its inputs (keys, query heads, weights and scales), never an
+    // earlier libcsa kernel's output, so its loads and MMAs may overlap the kernel before
+    // it.  Its score stores may not: an earlier top-k can still be reading the same score
+    // rows (two calls in a row on one workspace), so every epilogue thread waits for the
+    // previous grid before its first store.  The next kernel (the top-k, which waits for
+    // this grid before reading) may launch right away; the wait at the end keeps
+    // completion ordered for the kernels after it.
     pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -367,6 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row_in_tile = quarter * 32 + lane;
         int ng = 0, nit = 0;
         bool ok = true;
+        bool waited = false;   // for the previous grid, before this thread's first store
         for (int ii = 0; ii < n_my && ok; ii++) {
             Item x;
             if (!fetch_item(a, items, v0, v1, ii, x, false)) continue;
@@ -392,6 +396,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
+                if (!waited) {
+                    pdl_wait();
+                    waited = true;
+                }
                 for (int j = grp; j < gt; j += 2) {
                     const int tt = g0 + j;
                     const int e = (x.tile0 + tt) * kTileRows + row_in_tile;

@@ -35,6 +35,8 @@ def _random_idx(wl, seed, pad=0):
 @pytest.mark.parametrize("H,D,fmt,k,T", [
     (16, 128, 0, 64, [4096]),                      # CSA decode 4K shape
     (64, 128, 0, 512, [7001, 3000, 2100]),         # CSA decode, ragged, k = 512
+    (64, 128, 0, 1024, [9001, 4000, 300]),         # k = 1024: one CTA per query combines
+    (64, 128, 0, 2048, [20003, 9000]),             # all 64 heads (the prefill kernel shape)
     (128, 576, 1, 256, [3000, 1500]),              # 576-dim fp8 + bf16 RoPE entries
     (128, 576, 1, 1024, [9000, 3333, 200]),        # 1M-config shape: k = 1024, short rows padded
     (64, 576, 0, 128, [1203]),                     # 576-dim bf16 entries
