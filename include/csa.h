@@ -137,7 +137,8 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
  *   idx_out int32 [Q, k]
  *   scores_out: nullable fp32 [Q, ld_scores] receiving s_i for i < n_vis (ld_scores >= max_n)
  *   workspace: device buffer of at least csa_indexer_workspace_size(Q, max_n, k) bytes,
- *   256-byte aligned; contents on entry are ignored.
+ *   256-byte aligned; contents on entry are ignored.  It holds only the score rows, so it
+ *   may be NULL (with workspace_bytes 0) when scores_out is given.
  * kI and qI must be 16-byte aligned.  Errors as above; CSA_DEV_NAN, CSA_DEV_CAPACITY.
  */
 size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k);
@@ -213,14 +214,16 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int
  *   CSA_NOALLOC_SCRATCH_BYTES bytes; it allocates nothing.
  *   - A call needing more than that (csa_indexer_workspace_size(Q, max_n, k) > the size)
  *     returns CSA_ERR_WORKSPACE with a message and launches nothing.  16 MiB covers, e.g.,
- *     32 queries of up to 131040 visible entries.
+ *     32 queries of up to 131040 visible entries.  With scores_out given, the scores are
+ *     written there, the array is not used and there is no such limit.
  *   - Every GPU that loads the library holds the array until the process exits.
  *   - All calls on a device share the array, which keeps the last call's contents;
  *     nothing in it has to start at zero.  Calls whose kernels overlap on the GPU (e.g.
  *     on two unordered streams) race on it: order them on one stream.
- *   - The first call on each device resolves the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it: make that first
- *     call before any stream capture.
+ *   - Each call made outside stream capture resolves the array's device address on the
+ *     current device (cudaGetSymbolAddress) and caches it; a call made while `stream` is
+ *     being captured uses the cached address.  So make one call on each device before any
+ *     stream capture, and again after a cudaDeviceReset (which invalidates the address).
  */
 #define CSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 csa_status_t lightning_indexer_topk_noalloc(const uint8_t* qI, const float* qI_scale,
@@ -254,6 +257,23 @@ typedef struct {
 long long csa_launch_count(void);
 void csa_profile_enable(int on);
 int csa_profile_collect(csa_kernel_time_t* out, int max_entries, int keep_pending);
+
+/*
+ * csa_debug_set_wait_limit -- test hook for the device-side failure path (no counterpart
+ * on the pages).
+ *   Every wait of the tensor-core kernels on an mbarrier is bounded: past the limit it
+ *   flags CSA_DEV_TIMEOUT in dev_status and the CTA winds down (it waits for its own
+ *   copies and MMAs in flight, frees its tensor memory and returns).  This call sets that
+ *   limit, in SM clock cycles, for every kernel of the library; cycles <= 0 restores the
+ *   default of 4e9 cycles (about 2 s).  The drains of a CTA's own copies and MMAs always
+ *   keep the default.  A limit of a few hundred cycles makes waits give up at once, so a
+ *   test can check that the timeout path reports CSA_DEV_TIMEOUT and that later calls are
+ *   exact again.  Lower it only around kernels launched without thread-block clusters.
+ *   Unlike the other calls, this one copies to device memory synchronously: call it with
+ *   no libcsa kernel in flight and never during stream capture.
+ * Errors: CSA_ERR_CUDA.
+ */
+csa_status_t csa_debug_set_wait_limit(long long cycles);
 
 #ifdef __cplusplus
 }

@@ -66,6 +66,7 @@ _SIGS = {
     "csa_launch_count": (ctypes.c_longlong, []),
     "csa_profile_enable": (None, [ctypes.c_int]),
     "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
+    "csa_debug_set_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -111,6 +112,12 @@ def csa_profile_collect(keep_pending: bool = False) -> dict:
     arr = (_KernelTime * 32)()
     n = _lib.csa_profile_collect(ctypes.cast(arr, ctypes.c_void_p), 32, 1 if keep_pending else 0)
     return {arr[i].name.decode(): (arr[i].launches, arr[i].total_ms) for i in range(n)}
+
+
+def csa_debug_set_wait_limit(cycles: int = 0):
+    """Test hook: limit (SM clocks) of the kernels' bounded waits; 0 restores the default.
+    Synchronous; call it with no libcsa kernel in flight and outside stream capture."""
+    _check(_lib.csa_debug_set_wait_limit(int(cycles)))
 
 
 def csa_version() -> int:

@@ -76,11 +76,41 @@ void set_error_message(const char* fmt, ...) {
     vsnprintf(g_err, sizeof(g_err), fmt, ap);
     va_end(ap);
 }
+
+namespace {
+// Setters of the per-file wait limits, filled while the library loads (static
+// initialisation of the kernel files), read by csa_debug_set_wait_limit.
+constexpr int kMaxWaitLimitSetters = 16;
+struct WaitLimitSetters {
+    cudaError_t (*fn[kMaxWaitLimitSetters])(long long);
+    int n;
+};
+WaitLimitSetters& wait_limit_setters() {
+    static WaitLimitSetters s = {};
+    return s;
+}
+}  // namespace
+
+void register_wait_limit_setter(cudaError_t (*set)(long long cycles)) {
+    WaitLimitSetters& s = wait_limit_setters();
+    if (s.n < kMaxWaitLimitSetters) s.fn[s.n++] = set;
+}
 }  // namespace csa
 
 extern "C" {
 
 int csa_version(void) { return 100; }
+
+csa_status_t csa_debug_set_wait_limit(long long cycles) {
+    const long long c = cycles > 0 ? cycles : 4000000000LL;
+    csa::WaitLimitSetters& s = csa::wait_limit_setters();
+    if (s.n == 0) return fail(CSA_ERR_CUDA, "csa_debug_set_wait_limit: no kernel file registered");
+    for (int i = 0; i < s.n; i++) {
+        const cudaError_t e = s.fn[i](c);
+        if (e != cudaSuccess) return cuda_status(e, "csa_debug_set_wait_limit");
+    }
+    return ok();
+}
 
 const char* csa_last_error(void) { return g_err; }
 
@@ -139,8 +169,9 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     SUPPORT(d_I == 64 || d_I == 128, "indexer dim %d not supported (64 or 128)", d_I);
     SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
     REQUIRE(scores_out == nullptr || ld_scores >= max_n, "ld_scores must be >= max_n");
+    // the workspace holds only the score rows: with scores_out it is not used
     const size_t need = csa_indexer_workspace_size(Q, max_n, k);
-    if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+    if (!scores_out && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
         return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", need);
     float* scores = scores_out ? scores_out : (float*)workspace;
     const int64_t ld = scores_out ? ld_scores : (int64_t)round_up((size_t)max_n, 32);

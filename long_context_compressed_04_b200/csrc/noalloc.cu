@@ -18,9 +18,11 @@
 //  - all calls on a device share the one array and it keeps what the last call wrote;
 //    nothing in it needs to start at zero (each score is written before it is read), but
 //    calls whose kernels overlap on the GPU (different streams, no ordering) race on it;
-//  - the first call on a device looks up the array's device address with
-//    cudaGetSymbolAddress while that device is current, and caches it; make that first
-//    call before any stream capture.
+//  - with scores_out given, the scores go there and the array is not used (no size limit);
+//  - each call that is not being captured into a CUDA graph looks up the array's device
+//    address with cudaGetSymbolAddress on the current device and caches it; a call made
+//    during stream capture uses the cached address, so make one call on each device before
+//    capturing (and again after a cudaDeviceReset, which invalidates the cached address).
 #include <mutex>
 
 #include "launchers.cuh"
@@ -41,12 +43,14 @@ extern "C" csa_status_t lightning_indexer_topk_noalloc(
     const int32_t* q_pos, int32_t Q, int32_t B, int32_t H_I, int32_t d_I, int32_t m, int32_t k,
     int32_t max_n, int32_t* idx_out, float* scores_out, int64_t ld_scores, int32_t* dev_status,
     void* stream) {
-    if (Q == 0) return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
-                                              q_seq, q_pos, Q, B, H_I, d_I, m, k, max_n, idx_out,
-                                              scores_out, ld_scores, nullptr, 0, dev_status,
-                                              stream);
+    // the scores go to the caller's buffer (no scratch needed), or there is nothing to do,
+    // or the arguments are invalid: lightning_indexer_topk handles and reports these
     const size_t need = csa_indexer_workspace_size(Q, max_n, k);
-    if (need == 0 || need > (size_t)CSA_NOALLOC_SCRATCH_BYTES) {
+    if (Q <= 0 || scores_out != nullptr || need == 0)
+        return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
+                                      q_seq, q_pos, Q, B, H_I, d_I, m, k, max_n, idx_out,
+                                      scores_out, ld_scores, nullptr, 0, dev_status, stream);
+    if (need > (size_t)CSA_NOALLOC_SCRATCH_BYTES) {
         csa::set_error_message("lightning_indexer_topk_noalloc: Q=%d, max_n=%d needs %zu bytes of "
                               "scratch, more than the built-in %zu",
                               Q, max_n, need, (size_t)CSA_NOALLOC_SCRATCH_BYTES);
@@ -59,10 +63,15 @@ extern "C" csa_status_t lightning_indexer_topk_noalloc(
                               cudaGetErrorString(e));
         return CSA_ERR_CUDA;
     }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing((cudaStream_t)stream, &cap) != cudaSuccess) {
+        csa::set_error_message("lightning_indexer_topk_noalloc: invalid stream");
+        return CSA_ERR_INVALID_ARG;
+    }
     void* scratch = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_mu);
-        if (!g_scratch_ptr[dev]) {
+        if (cap == cudaStreamCaptureStatusNone || !g_scratch_ptr[dev]) {
             void* p = nullptr;
             e = cudaGetSymbolAddress(&p, g_indexer_scratch);
             if (e != cudaSuccess || p == nullptr) {

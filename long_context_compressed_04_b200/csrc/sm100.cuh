@@ -14,6 +14,18 @@ namespace sm100 {
 // reports CSA_DEV_TIMEOUT, so a broken pipeline ends the kernel instead of hanging it.
 constexpr long long kWaitLimitCycles = 4000000000LL;
 
+// The limit the bounded waits below use, in SM clocks.  Every kernel file that includes
+// this header holds its own copy (internal linkage); csa_debug_set_wait_limit sets all of
+// them.  The drains of a CTA's own copies and MMAs keep kWaitLimitCycles whatever this is,
+// so a lowered limit never lets a CTA leave with asynchronous work still in flight.
+namespace {
+__device__ long long g_wait_limit_cycles = kWaitLimitCycles;
+}
+
+__device__ __forceinline__ long long wait_limit_cycles() {
+    return *reinterpret_cast<volatile long long*>(&g_wait_limit_cycles);
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -37,20 +49,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
-// True when the phase of the given parity has completed; a thread whose phase is not complete
-// may be suspended for a short, system-dependent time first.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Non-blocking: true when the phase of the given parity has completed (never suspends).
 __device__ __forceinline__ bool mbar_ready(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
@@ -64,9 +62,9 @@ __device__ __forceinline__ bool mbar_ready(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// As mbar_test, but a thread whose phase is not complete is suspended in hardware until it
-// completes or about `hint_ns` nanoseconds pass, instead of returning at once: waiting
-// roles then take no issue slots from the ones doing work.
+// True when the phase of the given parity has completed; a thread whose phase is not complete
+// is first suspended in hardware until it completes or about `hint_ns` nanoseconds pass:
+// waiting roles then take no issue slots from the ones doing work.
 __device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
     uint32_t ok;
     asm volatile(
@@ -83,16 +81,24 @@ __device__ __forceinline__ bool mbar_test_sleep(uint64_t* bar, uint32_t parity, 
 // checked between them).
 constexpr uint32_t kSleepHintNs = 20000;
 
+// Limits below this many clocks make the waits poll (test_wait, never suspending) instead
+// of suspending in try_wait: a suspended thread may sleep until the phase completes, so a
+// short limit would otherwise never be reached.
+constexpr long long kPollBelowCycles = 1000000;
+
 // Bounded wait.  Returns false when the CTA has been aborted by another role or this wait
 // ran out of time (then it aborts the CTA and flags CSA_DEV_TIMEOUT).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int32_t* dev_status) {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_ready(bar, parity)) return true;
+    const long long limit = wait_limit_cycles();
+    const bool poll = limit < kPollBelowCycles;
     const long long t0 = clock64();
     for (;;) {
-        if (mbar_test_sleep(bar, parity, kSleepHintNs)) return true;
+        if (poll ? mbar_ready(bar, parity) : mbar_test_sleep(bar, parity, kSleepHintNs))
+            return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             flag(dev_status, CSA_DEV_TIMEOUT);
             return false;
@@ -196,7 +202,7 @@ __device__ __forceinline__ bool mbar_wait_cluster_warp(uint64_t* bar, uint32_t p
                 ok = false;
                 break;
             }
-            if (clock64() - t0 > kWaitLimitCycles) {
+            if (clock64() - t0 > wait_limit_cycles()) {
                 *abort_flag = 1;
                 flag(dev_status, CSA_DEV_TIMEOUT);
                 ok = false;
@@ -421,4 +427,15 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t a_fmt, uint32_t b_fmt
 }
 
 }  // namespace sm100
+
+// Host side of the wait limit: each kernel file registers a setter of its own copy of
+// g_wait_limit_cycles when the library loads (csa_debug_set_wait_limit calls them all).
+void register_wait_limit_setter(cudaError_t (*set)(long long cycles));
+namespace {
+cudaError_t set_wait_limit_of_this_file(long long cycles) {
+    return cudaMemcpyToSymbol(sm100::g_wait_limit_cycles, &cycles, sizeof(cycles));
+}
+const bool g_wait_limit_setter_registered =
+    (register_wait_limit_setter(&set_wait_limit_of_this_file), true);
+}  // namespace
 }  // namespace csa
