@@ -2,11 +2,15 @@
 
 One step = one pass of the whole hot path over one batch: compress each sequence's newest
 entry, lightning indexer + top-k (CSA), sparse (CSA) or dense (HCA) attention.  The
-default workload is CSA decode with 32 sequences of 131072 +- 1024 tokens, 64 query heads
-of dim 128, a 64 x 128 FP8 indexer and top-512.  Inputs are synthetic and seeded; the
-compressed cache is built with the library itself before timing.
+default workload is CSA decode at 1,048,576 tokens: 8 sequences, 128 query heads over
+576-dim entries (512 FP8 channels with 1x128 scales + 64 bf16 RoPE channels), a 64 x 128
+FP8 indexer and top-1024.  The same run also measures CSA decode with 32 sequences of
+131072 +- 1024 tokens (64 heads of dim 128, top-512) and HCA decode with 16 sequences of
+1,048,576 tokens, reported under "also".  Inputs are synthetic and seeded; the compressed
+cache is built with the library itself before timing.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--no-also]
+                  [--impl reference]
 
 Prints one JSON line (rank 0).  Under torchrun each rank runs its own batch (sequences
 shard across GPUs with no data-path collective; weak scaling); the timed region is
@@ -253,7 +257,7 @@ def gpu_index_for_smi(dev: int) -> str:
     return str(dev)
 
 
-CPU_SAMPLE_SEQS = {"csa_decode_128k_b32": 32, "hca_decode_1m_b16": 16, "csa_decode_1m_b8_fp8": 2,
+CPU_SAMPLE_SEQS = {"csa_decode_128k_b32": 32, "hca_decode_1m_b16": 16, "csa_decode_1m_b8_fp8": 8,
                    "csa_prefill_8k_on_64k": 64}   # prefill: sampled queries of the chunk
 
 
@@ -337,45 +341,65 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="csa_decode_128k_b32", choices=sorted(WORKLOADS))
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
-    if args.impl == "reference":
-        return run_reference(args)
+DEFAULT_WORKLOAD = "csa_decode_1m_b8_fp8"
+# measured in the same run as the default workload and reported under "also"
+ALSO_WORKLOADS = ("csa_decode_128k_b32", "hca_decode_1m_b16")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
 
+def fp8_gemm_peak(dev, n: int = 8192, seconds: float = 4.0):
+    """Dense e4m3 GEMM rate of this GPU (torch._scaled_mm, n x n x n, fp32 scales, bf16
+    out): best of 10 single launches (burst) and the mean over `seconds` of back-to-back
+    launches (sustained), in TFLOP/s."""
+    a = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn)
+    b = torch.randn((n, n), device=dev).to(torch.float8_e4m3fn).t()
+    one = torch.ones((), device=dev)
+    mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)  # noqa: E731
+    for _ in range(3):
+        mm()
+    torch.cuda.synchronize()
+    flop = 2.0 * n ** 3
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1) / 1e3)
+    reps = 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_end = time.time() + seconds
+    e0.record()
+    while time.time() < t_end:
+        for _ in range(20):
+            mm()
+        reps += 20
+        torch.cuda.synchronize()
+    e1.record()
+    torch.cuda.synchronize()
+    sustained = flop * reps / (e0.elapsed_time(e1) / 1e3) / 1e12
+    return {"burst": round(flop / best / 1e12, 1), "sustained": round(sustained, 1),
+            "how": f"torch._scaled_mm e4m3 {n}^3, bf16 out: best of 10 (burst), "
+                   f"{seconds:.0f} s back to back (sustained)"}
+
+
+def measure(name: str, args, dist, dev, rank: int, world: int, full: bool):
+    """Times K steps of workload `name` (graph replay, L2 flushed before each), then the
+    per-kernel device times in a second replayed graph; with `full`, also the end-to-end
+    rate through host buffers.  Returns the fields of the JSON line."""
     import long_context_compressed_04_b200 as L
     from long_context_compressed_04_b200 import pipeline
 
-    wl = make_workload(args.workload, rank, dev)
+    wl = make_workload(name, rank, dev)
     buf = pipeline.alloc(wl, dev)
     all_seq, all_ent = pipeline.all_entry_items(wl, dev)
     pipeline.compress(wl, buf, all_seq, all_ent)          # build the compressed cache
-    new_seq, new_ent = step_items(wl, args.workload, dev)
+    new_seq, new_ent = step_items(wl, name, dev)
     torch.cuda.synchronize()
     del all_seq, all_ent
 
-    def step_eager():
-        pipeline.step(wl, buf, new_seq, new_ent)
+    def step_eager(b=buf, w=wl):
+        pipeline.step(w, b, new_seq, new_ent)
 
     # the step's launches are captured once into a CUDA graph and replayed, so the timed
     # region measures device work rather than Python/ctypes launch overhead
@@ -422,7 +446,7 @@ def main():
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(K)]
     launches0 = L.csa_launch_count()
-    with ClockSampler(gpu_index_for_smi(local)) as clk:
+    with ClockSampler(gpu_index_for_smi(dev.index)) as clk:
         barrier()
         for i in range(K):
             flush_l2()
@@ -432,7 +456,7 @@ def main():
         barrier()
     launches = L.csa_launch_count() - launches0 + kernels_per_step * K
     ms_max = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dist, dev)
-    assert int(buf.dev_status.item()) == 0, "device status flagged during the run"
+    assert int(buf.dev_status.item()) == 0, f"device status flagged during the {name} run"
 
     # second pass: the same step captured into a CUDA graph with a CUDA event pair around
     # every libcsa kernel (recorded on the launching stream); each replay re-records them,
@@ -449,64 +473,16 @@ def main():
         flush_l2()
         pgraph.replay()
         torch.cuda.synchronize()
-        for name, (n_l, tot_ms) in L.csa_profile_collect(keep_pending=True).items():
-            c, t_ = per_kernel.get(name, (0, 0.0))
-            per_kernel[name] = (c + n_l, t_ + tot_ms)
+        for kname, (n_l, tot_ms) in L.csa_profile_collect(keep_pending=True).items():
+            c, t_ = per_kernel.get(kname, (0, 0.0))
+            per_kernel[kname] = (c + n_l, t_ + tot_ms)
     del pgraph
     L.csa_profile_collect()
 
-    # e2e: host buffers.  Each step copies its inputs from pinned host memory (the query
-    # heads, the indexer's query heads, scales and weights, and the new token's raw KV and
-    # gate rows), runs the step, and copies the output back; all of it is captured into one
-    # CUDA graph, so every replay performs the copies.
-    h_in = {"q": wl.q, "qI": wl.qI, "qs": wl.qs, "w": wl.w}
-    h_in = {k2: v for k2, v in h_in.items() if v is not None}
-    pinned = {k2: torch.empty(v.shape, dtype=v.dtype, pin_memory=True).copy_(v.cpu())
-              for k2, v in h_in.items()}
-    nn = new_tokens(wl, args.workload)
-    last_rows = torch.cat([(wl.kv_off[b] + (wl.T.to(dev)[b] - nn - wl.kv_pos0[b]))
-                           + torch.arange(nn, device=dev) for b in range(wl.B)]).long()
-    nr = last_rows.numel()
-    pin_kv = torch.empty((nr, wl.D), dtype=wl.kv.dtype, pin_memory=True).copy_(wl.kv[last_rows].cpu())
-    pin_gate = torch.empty((nr, wl.D), dtype=wl.gate.dtype, pin_memory=True).copy_(wl.gate[last_rows].cpu())
-    dev_kv = torch.empty((nr, wl.D), dtype=wl.kv.dtype, device=dev)
-    dev_gate = torch.empty((nr, wl.D), dtype=wl.gate.dtype, device=dev)
-    out_host = torch.empty(buf.out.shape, dtype=buf.out.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in pinned.values()) + 2 * pin_kv.numel() * 2
-    d2h = out_host.numel() * out_host.element_size()
-
-    def e2e_step():
-        for k2, v in pinned.items():
-            h_in[k2].copy_(v, non_blocking=True)
-        dev_kv.copy_(pin_kv, non_blocking=True)
-        dev_gate.copy_(pin_gate, non_blocking=True)
-        wl.kv.index_copy_(0, last_rows, dev_kv)
-        wl.gate.index_copy_(0, last_rows, dev_gate)
-        step_eager()
-        out_host.copy_(buf.out, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize()
-    egraph = None
-    if not args.no_graph:
-        egraph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(egraph):
-            e2e_step()
-        torch.cuda.synchronize()
-    E = max(K // 2, 10)
-    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(E)]
-    barrier()
-    for i in range(E):
-        flush_l2()
-        ee[i][0].record()
-        if egraph is not None:
-            egraph.replay()
-        else:
-            e2e_step()
-        ee[i][1].record()
-    barrier()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), dist, dev)
+    e2e = None
+    if full:
+        e2e = measure_e2e(name, wl, buf, new_seq, new_ent, args, dist, dev, world, flush_l2,
+                          barrier)
 
     peak, peak_kind = _peaks()
     total_bytes, key_bytes = algorithmic_bytes(wl)
@@ -519,17 +495,19 @@ def main():
     dom_name = next((n for n in (["indexer_score_tc", "indexer_score_simt"] if wl.H_I else [])
                      + ["attn_tc", "attn_simt"] if n in per_kernel), None)
     roof = None
-    if WORKLOADS[args.workload]["kind"] == "csa_prefill" and "indexer_score_tc" in per_kernel:
-        # prefill: the indexer's FP8 dot products bound it (tensor pipe); the peak is the
-        # measured sustained bf16 GEMM rate times the nominal fp8 / bf16 ratio of 2
+    if WORKLOADS[name]["kind"] == "csa_prefill" and "indexer_score_tc" in per_kernel:
+        # prefill: the indexer's FP8 dot products bound it (tensor pipe); the peak is this
+        # GPU's e4m3 GEMM rate, measured here (sustained: the indexer runs for milliseconds)
         n_l, tot_ms = per_kernel["indexer_score_tc"]
         avg_s = tot_ms / n_l / 1e3
         fl = indexer_flops(wl)
-        tpk, tkind = _tensor_peak_fp8()
+        fp8 = fp8_gemm_peak(dev)
         ach = fl / avg_s / 1e12
         roof = {"bound": "tensor", "kernel": "indexer_score_tc", "achieved": round(ach, 1),
-                "peak": tpk, "unit": "TFLOP/s", "frac": round(ach / tpk, 4), "traffic": None,
-                "peak_source": tkind, "algorithmic_flops_per_launch": fl,
+                "peak": fp8["sustained"], "unit": "TFLOP/s",
+                "frac": round(ach / fp8["sustained"], 4), "traffic": None,
+                "peak_source": "measured in this run (sustained); " + fp8["how"],
+                "fp8_gemm_burst": fp8["burst"], "algorithmic_flops_per_launch": fl,
                 "avg_launch_us": round(avg_s * 1e6, 2)}
     elif dom_name:
         n_l, tot_ms = per_kernel[dom_name]
@@ -538,15 +516,13 @@ def main():
         ach = alg / avg_s / 1e9
         roof = {"bound": "hbm", "kernel": dom_name, "achieved": round(ach, 1), "peak": peak,
                 "unit": "GB/s", "frac": round(ach / peak, 4),
-                "traffic": measured_traffic(args.workload, dom_name),
+                "traffic": measured_traffic(name, dom_name),
                 "peak_source": f"{peak_kind} hbm_gbs (copy)",
                 "algorithmic_bytes_per_launch": alg, "avg_launch_us": round(avg_s * 1e6, 2)}
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": args.workload, **WORKLOADS[args.workload],
-                   "queries_per_gpu": wl.Q, "l2": "flushed before every timed step (256 MB write, then 256 MB read)",
+    out = {
+        "value": value, "ms_per_step": ms_max / K,
+        "config": {"workload": name, **WORKLOADS[name], "queries_per_gpu": wl.Q,
+                   "l2": "flushed before every timed step (256 MB write, then 256 MB read)",
                    "indexer_inputs": "fp8 e4m3 N(0,1), 1x128 scales"},
         "roofline": roof,
         "step_roofline": {"algorithmic_bytes": total_bytes,
@@ -555,12 +531,168 @@ def main():
         "kernels": {k2: {"launches": v[0], "avg_us": round(v[1] / v[0] * 1e3, 2),
                          "share": round(v[1] / sum(x[1] for x in per_kernel.values()), 4)}
                     for k2, v in per_kernel.items()},
-        "e2e": {"value": whole_job_rate(wl.Q, world, E, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "launch": "cuda graph replay" if graph is not None else "eager",
         "clocks": clk.summary(),
     }
+    if e2e is not None:
+        out["e2e"] = e2e
+    del graph, buf, wl
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_e2e(name, wl, buf, new_seq, new_ent, args, dist, dev, world, flush_l2, barrier):
+    """The same metric through the public API with host buffers.  Every step copies its
+    inputs from pinned host memory (the query heads, the indexer's query heads, scales and
+    weights, and the new tokens' raw KV and gate rows) and copies its output back.  The
+    copies are double-buffered on a second stream: step i+1's inputs go up and step i-1's
+    output comes down while step i computes.  A run of E steps is captured into one CUDA
+    graph (the two streams forked and joined inside it) and replayed; the rate is E steps
+    over the replay's device time."""
+    from long_context_compressed_04_b200 import pipeline
+    import dataclasses
+
+    nn = new_tokens(wl, name)
+    last_rows = torch.cat([(wl.kv_off[b] + (wl.T.to(dev)[b] - nn - wl.kv_pos0[b]))
+                           + torch.arange(nn, device=dev) for b in range(wl.B)]).long()
+    nr = last_rows.numel()
+    fields = [f for f in ("q", "qI", "qs", "w") if getattr(wl, f) is not None]
+    pinned = {f: torch.empty(getattr(wl, f).shape, dtype=getattr(wl, f).dtype,
+                             pin_memory=True).copy_(getattr(wl, f).cpu()) for f in fields}
+    pin_kv = torch.empty((nr, wl.D), dtype=wl.kv.dtype, pin_memory=True).copy_(wl.kv[last_rows].cpu())
+    pin_gate = torch.empty((nr, wl.D), dtype=wl.gate.dtype, pin_memory=True).copy_(wl.gate[last_rows].cpu())
+    # two sets of device inputs and outputs; the compressed cache and raw KV are shared
+    sets = []
+    for j in range(2):
+        dev_in = {f: torch.empty_like(getattr(wl, f)) for f in fields}
+        w_j = dataclasses.replace(wl, **dev_in)
+        b_j = dataclasses.replace(buf, out=torch.empty_like(buf.out),
+                                  idx=None if buf.idx is None else torch.empty_like(buf.idx),
+                                  workspace=torch.empty_like(buf.workspace))
+        sets.append(dict(wl=w_j, buf=b_j, kv=torch.empty((nr, wl.D), dtype=wl.kv.dtype, device=dev),
+                         gate=torch.empty((nr, wl.D), dtype=wl.gate.dtype, device=dev),
+                         up=torch.cuda.Event(), done=torch.cuda.Event(),
+                         down=torch.cuda.Event(),
+                         host_out=torch.empty(buf.out.shape, dtype=buf.out.dtype,
+                                              pin_memory=True)))
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values()) + 2 * pin_kv.numel() * 2
+    d2h = sets[0]["host_out"].numel() * sets[0]["host_out"].element_size()
+    copy = torch.cuda.Stream()
+
+    def upload(st):
+        for f in fields:
+            getattr(st["wl"], f).copy_(pinned[f], non_blocking=True)
+        st["kv"].copy_(pin_kv, non_blocking=True)
+        st["gate"].copy_(pin_gate, non_blocking=True)
+        st["up"].record(copy)
+
+    def run(E):
+        comp = torch.cuda.current_stream()   # the capture stream while a graph is captured
+        # fork: the copy stream joins the capture
+        copy.wait_stream(comp)
+        with torch.cuda.stream(copy):
+            upload(sets[0])
+        for i in range(E):
+            st, nxt = sets[i % 2], sets[(i + 1) % 2]
+            if i + 1 < E:
+                with torch.cuda.stream(copy):
+                    if i >= 1:
+                        copy.wait_event(nxt["down"])    # step i-1's output is read back
+                    upload(nxt)
+            comp.wait_event(st["up"])
+            wl.kv.index_copy_(0, last_rows, st["kv"])
+            wl.gate.index_copy_(0, last_rows, st["gate"])
+            pipeline.step(st["wl"], st["buf"], new_seq, new_ent)
+            st["done"].record(comp)
+            with torch.cuda.stream(copy):
+                copy.wait_event(st["done"])
+                st["host_out"].copy_(st["buf"].out, non_blocking=True)
+                st["down"].record(copy)
+        comp.wait_stream(copy)                          # join
+
+    E = 16
+    run(E)
+    torch.cuda.synchronize()
+    egraph = None
+    if not args.no_graph:
+        egraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(egraph):
+            run(E)
+        torch.cuda.synchronize()
+    R = max(args.steps // E, 4)
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(R)]
+    barrier()
+    for i in range(R):
+        flush_l2()
+        ee[i][0].record()
+        if egraph is not None:
+            egraph.replay()
+        else:
+            run(E)
+        ee[i][1].record()
+    barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), dist, dev)
+    for st in sets:
+        assert int(st["buf"].dev_status.item()) == 0
+    return {"value": whole_job_rate(wl.Q, world, R * E, e2e_ms), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": e2e_ms / (R * E),
+            "how": f"pinned h2d of each step's inputs and d2h of its output on a second stream, "
+                   f"double-buffered; {E} pipelined steps per captured graph, {R} replays"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-also", action="store_true",
+                    help="measure only --workload (not the other decode workloads)")
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    head = measure(args.workload, args, dist, dev, rank, world, full=True)
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+    }
+    line.update({k: v for k, v in head.items() if k not in ("value", "ms_per_step")})
+    if args.workload == DEFAULT_WORKLOAD and not args.no_also:
+        # every rank measures the same workloads in the same order
+        line["also"] = {}
+        for name in ALSO_WORKLOADS:
+            r = measure(name, args, dist, dev, rank, world, full=False)
+            line["also"][name] = {
+                "value": r["value"], "unit": UNIT, "ms_per_step": r["ms_per_step"],
+                "step_frac": r["step_roofline"]["frac"],
+                "dominant_kernel": None if r["roofline"] is None else r["roofline"]["kernel"],
+                "dominant_frac": None if r["roofline"] is None else r["roofline"]["frac"],
+                "kernels": r["kernels"], "gpu_launches": r["gpu_launches"],
+                "clocks": r["clocks"]}
+            line["gpu_launches"] += r["gpu_launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload)
     if dist:
