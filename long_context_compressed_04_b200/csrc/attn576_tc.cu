@@ -6,28 +6,35 @@
 //
 // One cluster of 4 CTAs per (query, group of 64 heads).  The keys of the query are tiles
 // of 32 -- the window's raw rows first (RMSNormed and RoPEd here), then the selected entries
-// -- dealt to the ranks in turn (tile j to rank j mod 4).  Each rank ends with an fp32
-// partial state per head (running maximum, sum, unnormalised O) and stores it straight
-// into the shared memory of the rank that finishes that head (16 heads each, posted
-// st.shared::cluster); each rank combines its heads in rank order, the sink first.  Three
-// key buffers let tiles be built while earlier ones are in the tensor cores.
-//   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once; per
-//              tile, 4 threads per key row dequantize the gathered FP8 row (or normalise the
-//              raw window row in place) into bf16, 128-byte swizzled, 9 blocks of 64
-//              channels; each thread's quarter of the next entry row is loaded into
-//              registers while the current tile is converted.
-//   warp 4     TMEM allocation; lane 0 issues tcgen05.mma kind::f16:
-//              S = Q K^T (M = 64 heads, N = 32 keys, 36 K steps of 16 channels) into one of
-//              two S buffers, one tile ahead of O += P V, which goes straight into the TMEM
-//              accumulator: channels 0-255 in TMEM lanes 0-15 of each quarter, 256-511 in
-//              lanes 16-31, 512-575 in lanes 0-15 again (N = 256 + 256 + 64), V being the
-//              key tile read MN-major.
+// -- dealt to the ranks in turn (tile j to rank j mod 4, so every rank's first tile is a
+// window tile).  The query tile and the window tile depend only on the call's inputs, so
+// they are built, scored and accumulated before the kernel waits for the one before it
+// (the top-k): only the index row and the entries wait.  Each rank ends with an fp32
+// partial state per head (running maximum, sum, unnormalised O) in its own shared memory;
+// the rank that finishes a head pulls the four partial states of it (ld.shared::cluster)
+// and combines them in rank order, the sink first.  Three key buffers let tiles be built
+// while earlier ones are in the tensor cores.
+//   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once (as
+//              fp16, scaled by 2^-s if needed, see below); the window tile; then, after the
+//              wait, the index row and a bulk L2 prefetch of every entry row this rank
+//              gathers; per tile, 4 threads per key row convert their quarter of the FP8 row
+//              (e4m3 -> fp16 exactly, times the block scale) into a 128-byte-swizzled tile
+//              of 9 blocks of 64 channels; the rows of tile j + 2 are loaded into registers
+//              while tile j is converted (two register sets).
+//   warp 4     TMEM allocation; lane 0 issues O += P V (tcgen05.mma kind::f16, fp16
+//              operands) straight into the TMEM accumulator: channels 0-255 in TMEM lanes
+//              0-15 of each quarter, 256-511 in lanes 16-31, 512-575 in lanes 0-15 again
+//              (N = 256 + 256 + 64), V being the key tile read MN-major.
+//   warps 9-10 lane 0 issues S = Q K^T of the even (warp 9) or odd (warp 10) tiles
+//              (M = 64 heads, N = 32 keys, 36 K steps of 16 channels) into its own S
+//              buffer, as 4 partial accumulators (see s_col): one MMA costs its issuing
+//              thread tens of cycles whatever its shape, so S has two issuers.
 //   warps 5-8  online softmax in the log2 domain, one head row per lane, weights by
-//              ex2.approx of one FMA per key: P as bf16 into shared memory; the running
+//              ex2.approx of one FMA per key: P as fp16 into shared memory; the running
 //              maximum is a reference that moves only when a tile's maximum exceeds it by
-//              2^8, and then the head's O row in TMEM is rescaled; finally the partial
-//              states across the cluster, and for this rank's heads the combine, the sink,
-//              inverse RoPE and the store.
+//              2^8, and then the head's O row in TMEM is rescaled; then the partial state
+//              into shared memory.
+//   warps 0-3, 5-8  the combine of this rank's 16 heads: inverse RoPE, bf16 store.
 // A 64 x 576 fp32 accumulator takes 320 TMEM columns, and the query's Q tile (72 KB) takes a
 // third of shared memory: hence 64 heads per CTA and three key buffers of 32 rows.
 // All waits are bounded (timeout -> CSA_DEV_TIMEOUT, drain, free TMEM, return).  A query's
@@ -43,7 +50,7 @@ namespace {
 
 constexpr int kHC = 64;                  // heads per CTA (MMA M)
 constexpr int kD = 576;
-constexpr int kNB = kD / 64;             // 9 blocks of 64 channels (128 bytes of bf16)
+constexpr int kNB = kD / 64;             // 9 blocks of 64 channels (128 bytes of fp16)
 constexpr int kTK = 32;                  // keys per tile (MMA N of S)
 constexpr int kQBlk = 64 * 128;          // one 64-row x 128-byte swizzled block of Q
 constexpr int kKBlk = kTK * 128;         // one 32-row x 128-byte swizzled block of K
@@ -51,32 +58,40 @@ constexpr int kQBytes = kNB * kQBlk;     // 72 KB
 constexpr int kKBytes = kNB * kKBlk;     // 36 KB per key buffer
 constexpr int kPBytes = 64 * 128;        // 8 KB (rows of 128 B, the first 64 B used)
 constexpr int kRowBytes = 656;
-constexpr int kThreads = 288;
+constexpr int kFirstSWarp = 9;           // warps 9 and 10 issue S (see the MMA issuers)
+constexpr int kThreads = 32 * (kFirstSWarp + 2);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescale = 8.f;          // the reference maximum moves by more than 2^8 only
 constexpr uint32_t kColO = 0;            // O channels 0-255 (lanes 0-15) / 256-511 (lanes 16-31)
 constexpr uint32_t kColOr = 256;         // O channels 512-575 (lanes 0-15)
-constexpr uint32_t kColS = 320;          // S buffers at 320 and 352 (lanes 0-15)
+constexpr uint32_t kColS = 320;          // S: [2 buffers][4 partials] x 32 columns, see s_col
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxK = 2048;
 constexpr int kCl = 4;                   // CTAs per (query, head group)
 constexpr int kHO = kHC / kCl;           // heads finished by each rank
+constexpr int kWtStride = kCl + 1;       // combine weights of a head: kCl ranks, then L
+static_assert(kCl >= 4, "the window (at most 4 tiles of 32 rows) is one tile per rank");
 // shared-memory layout (byte offsets from the 1024-aligned base)
 constexpr int kOffQ = 0;
-constexpr int kKBuf = 3;                 // key buffers
+constexpr int kKBuf = 3;                 // key buffers (fp16)
 constexpr int kOffK = kOffQ + kNB * 64 * 128;            // after Q (72 KB)
 constexpr int kOffP = kOffK + kKBuf * kNB * 32 * 128;    // after the key buffers
 constexpr int kOffMask = kOffP + 2 * 64 * 128;           // after two P buffers
-constexpr int kOffRope = kOffMask + 16;
-constexpr int kOffIdx = kOffRope + 5 * 32 * 4;
+constexpr int kOffRope = kOffMask + 16;   // [kKBuf][4] key masks
+constexpr int kOffQMax = kOffRope + 5 * 32 * 4;       // [4] per-warp max |q|, then the q scale
+constexpr int kOffIdx = kOffQMax + 32;
 constexpr int kOffRot = kOffIdx + kMaxK * 4;              // [32 rows][32 pairs] cos, sin
 constexpr int kOffWt = kOffRot + 32 * 32 * 8;              // [16 heads][kCl + 1] weights, L
 constexpr int kOffBars = kOffWt + 16 * 8 * 4;
-constexpr int kOffEnd = kOffBars + 22 * 8 + 16;
-// the partial states of this rank's heads from every rank, [kCl][kHO][576] O then
-// [kCl][2][kHO] m, l, over Q, the key, P and staging buffers once this rank's MMAs are done
-constexpr int kRecvO = kCl * kHO * 576;
-static_assert((kRecvO + kCl * 2 * kHO) * 4 <= kOffMask, "receive buffer");
+static_assert(kHO * kWtStride <= 16 * 8, "combine-weight table");
+constexpr int kOffEnd = kOffBars + 21 * 8 + 16;
+// this rank's partial state, written over Q / K / P once its MMAs are done and read by the
+// rank that finishes each head: O as [64 heads][kPS] fp32 (rows padded from 576 to 580
+// floats, so that the lanes writing 16 head rows at once hit distinct banks), then the
+// running maximum m [64] and sum l [64]
+constexpr int kPS = 580;
+constexpr int kPartML = kHC * kPS;
+static_assert((kPartML + 2 * kHC) * 4 <= kOffMask, "partial state over Q / K / P");
 static_assert(kOffK % 1024 == 0 && kOffP % 1024 == 0, "swizzled tiles on 1024 B");
 static_assert(kOffIdx % 16 == 0 && kOffBars % 8 == 0, "alignment");
 
@@ -100,6 +115,16 @@ struct A576Args {
     double log2_theta;
 };
 
+// S of a key tile is accumulated in 4 independent partials, partial p taking the K steps
+// 4 cb + p (cb = the 64-channel block): a chain of MMAs into one accumulator waits for each
+// step's result, four chains keep the tensor pipe busy.  Partial p of S buffer sb sits at
+// columns kColS + 32 (2 sb + p / 2), in TMEM lanes 0-15 (p even) or 16-31 (p odd) of each
+// lane quarter (an M = 64 accumulator uses 16 lanes per quarter).
+__host__ __device__ constexpr uint32_t s_col(int sb, int p) {
+    return kColS + 32u * (uint32_t)(2 * sb + (p >> 1)) + ((uint32_t)(p & 1) << 20);
+}
+static_assert(s_col(1, 3) - (16u << 16) + 32 <= kTmemCols, "S partials fit the allocation");
+
 // Byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-swizzled [rows x 128 B] block.
 __device__ __forceinline__ uint32_t swz(int r, int ch) {
     return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4));
@@ -122,39 +147,54 @@ __device__ __forceinline__ uint64_t desc_mn(const void* tile, uint32_t lbo_bytes
     return d;
 }
 
-// 8 channels (16 bytes of bf16) of row `r`, channel `d0` (a multiple of 8), into a
+// 8 channels (16 bytes of fp16) of row `r`, channel `d0` (a multiple of 8), into a
 // [9 blocks][rows x 128 B] swizzled tile with blocks `blk` bytes apart.
 __device__ __forceinline__ uint4* cell8(uint8_t* tile, int blk, int r, int d0) {
     return reinterpret_cast<uint4*>(tile + (d0 >> 6) * blk + swz(r, (d0 & 63) >> 3));
 }
 
-// Two e4m3 codes (low 16 bits; the lower byte first) to two floats, exactly, by the packed
-// hardware conversion to f16.
-__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t two) {
+// The MMAs of this kernel take fp16 operands (Q, K = V and P; fp32 accumulation).  An e4m3
+// code is exact in fp16, so an entry channel is one conversion and one multiply by its
+// block's scale (rounded to fp16); entries and window rows are RMS-normalised (|x| <= sqrt(D)),
+// and fp16 keeps 3 more mantissa bits than bf16.  The query is scaled by an exact power of
+// two when its magnitude would leave the fp16 range (see the query load).
+
+// Two floats to packed fp16 (round to nearest even; the first in the low half).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Two e4m3 codes (low 16 bits; the lower byte first) to packed fp16, exactly.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
     uint32_t h;
     asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
         : "=r"(h)
         : "r"(two));
-    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+    return h;
 }
 
-// 16 e4m3 codes times `sc`, as 16 bf16 (two 16-byte chunks).
-__device__ __forceinline__ void dequant16(uint4 c, float sc, uint4& lo, uint4& hi) {
+__device__ __forceinline__ uint32_t hmul2(uint32_t x, uint32_t y) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(y));
+    return r;
+}
+
+// 16 e4m3 codes times the scale `sc2` (fp16, in both halves), as 16 fp16 (two 16-byte chunks).
+__device__ __forceinline__ void dequant16(uint4 c, uint32_t sc2, uint4& lo, uint4& hi) {
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
     uint32_t o[8];
 #pragma unroll
     for (int z = 0; z < 4; z++) {
-        const float2 a = e4m3x2_to_f32x2(w[z] & 0xFFFFu);
-        const float2 b = e4m3x2_to_f32x2(w[z] >> 16);
-        o[2 * z] = pack_bf16x2(a.x * sc, a.y * sc);
-        o[2 * z + 1] = pack_bf16x2(b.x * sc, b.y * sc);
+        o[2 * z] = hmul2(e4m3x2_to_f16x2(w[z] & 0xFFFFu), sc2);
+        o[2 * z + 1] = hmul2(e4m3x2_to_f16x2(w[z] >> 16), sc2);
     }
     lo = make_uint4(o[0], o[1], o[2], o[3]);
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// One loader thread's quarter of a selected entry row: fp8 channels [128 qt, 128 qt + 128)
-// with their scale, RoPE channels [16 qt, 16 qt + 16).
+// One loader thread's quarter of a selected entry row, in registers: fp8 channels
+// [128 qt, 128 qt + 128) with their scale, RoPE channels [16 qt, 16 qt + 16).
 struct EntryQuarter {
     uint4 f[8];
     uint4 rope[2];
@@ -162,8 +202,8 @@ struct EntryQuarter {
     bool valid;
 };
 
-// Loads entry v of the query's index row (staged in shared memory) into registers (flags an
-// out-of-range index once per row).
+// Issues the loads of entry v of the query's index row (staged in shared memory) into
+// registers (flags an out-of-range index once per row).
 __device__ __forceinline__ void fetch_entry(const A576Args& a, const int32_t* sidx, int v,
                                             int n_vis, int64_t row0, int qt, EntryQuarter& x) {
     const int e = v < a.k ? sidx[v] : -1;
@@ -188,9 +228,9 @@ __device__ __forceinline__ void fetch_entry(const A576Args& a, const int32_t* si
 
 __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args a) {
     using namespace sm100;
-    constexpr uint32_t kIdescS = instr_desc(1, 1, 64, kTK);
-    constexpr uint32_t kIdescPV = instr_desc(1, 1, 64, 256, 1);
-    constexpr uint32_t kIdescPVr = instr_desc(1, 1, 64, 64, 1);
+    constexpr uint32_t kIdescS = instr_desc(0, 0, 64, kTK);         // fp16 x fp16 -> fp32
+    constexpr uint32_t kIdescPV = instr_desc(0, 0, 64, 256, 1);
+    constexpr uint32_t kIdescPVr = instr_desc(0, 0, 64, 64, 1);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
@@ -204,6 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     float* rwc = rf + 32;                                 // [32] cos / sin of pair j at w0
     float* rws = rwc + 32;
     int32_t* sidx = reinterpret_cast<int32_t*>(smem + kOffIdx);   // [kMaxK] the index row
+    uint32_t* qmax = reinterpret_cast<uint32_t*>(smem + kOffQMax);   // [4] largest |q| bits
+    float* qscale = reinterpret_cast<float*>(smem + kOffQMax + 16);   // 2^s of the q scaling
     float2* srot = reinterpret_cast<float2*>(smem + kOffRot);    // window RoPE rotations
     float* swt = reinterpret_cast<float*>(smem + kOffWt);        // combine weights
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBars);
@@ -218,10 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                                      // previous tile's: never more than one phase behind)
     uint64_t* odone = bars + 16;     // MMA commit after the last P V (one phase)
     uint64_t* drain = bars + 17;
-    uint64_t* recv_ready = bars + 18;   // every rank's MMAs are done: 4 x cluster
-    uint64_t* cpart_full = bars + 19;   // every rank's partials are in: 4 x cluster
+    uint64_t* cpart_full = bars + 19;   // every rank's partial state is written: 4 x cluster
     uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 20);
-    float* recv = reinterpret_cast<float*>(smem + kOffQ);
+    float* part = reinterpret_cast<float*>(smem + kOffQ);          // [64][kPS] O, m[64], l[64]
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -247,8 +288,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         }
         mbar_init(pvdone, 1);
         mbar_init(odone, 1);
-        mbar_init(drain, 1);
-        mbar_init(recv_ready, 4 * kCl);
+        mbar_init(drain, 3);   // the three MMA issuers
+
         mbar_init(cpart_full, 4 * kCl);
         *abort_flag = 0;
         mbar_fence_init();
@@ -271,13 +312,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         tmem_alloc(tmem_base_smem, kTmemCols);
         tmem_relinquish();
     }
-    // the index sets come from the top-k and the entries from compression
-    pdl_wait();
-    if (threadIdx.x == 0) pdl_trigger();
-    if (valid) {
-        // the query's index row, once (only the loaders read it)
-        for (int v = threadIdx.x; v < a.k; v += kThreads) sidx[v] = a.idx[(int64_t)qi * a.k + v];
-    }
+    // Nothing up to the loaders' wait below reads what an earlier libcsa kernel writes: the
+    // query's heads, the window's raw rows and the sink are inputs.  So the query tile and
+    // the window tile (S, softmax and P V included) overlap the kernel before this one (the
+    // top-k); only the index row and the entries it selects wait for it.
     tc_fence_before();
     __syncthreads();
     // the cluster's barriers are initialised before any rank arrives on another's
@@ -301,28 +339,56 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         const int r = tid >> 1, hf = tid & 1;        // key (or head) row, half of it
         bool ok = true;
         if (valid) {
-            // q head row r at t: channels [288 hf, 288 hf + 288), RoPE on 512..575
-            const uint16_t* qrow = a.q + ((int64_t)qi * a.H + kHC * g + r) * kD;
+            // q head row r at t: channels [288 hf, 288 hf + 288), RoPE on 512..575.  Pass 1:
+            // the largest |q| of the CTA's 64 heads; if it could leave the fp16 range after
+            // the rotation (which grows a pair's component by at most sqrt 2), every q value
+            // is scaled by 2^-s (exact) with s the least such that max |q| 2^-s < 2^15, and
+            // the softmax scale is multiplied by 2^s.  Pass 2: rotate, scale, store as fp16.
+            const uint16_t* qrow = a.q + ((int64_t)qi * a.H + kHC * g + r) * kD + 288 * hf;
+            uint32_t mx = 0;   // largest |q| as bf16 bits (the order of non-negative values)
+#pragma unroll
+            for (int half = 0; half < 2; half++) {
+                uint4 u[18];
+#pragma unroll
+                for (int c = 0; c < 18; c++) u[c] = *reinterpret_cast<const uint4*>(qrow + 144 * half + 8 * c);
+#pragma unroll
+                for (int c = 0; c < 18; c++) {
+                    const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+#pragma unroll
+                    for (int z = 0; z < 4; z++)
+                        mx = max(mx, max(w[z] & 0x7FFFu, (w[z] >> 16) & 0x7FFFu));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) qmax[warp] = mx;
+            asm volatile("bar.sync 3, 128;" ::: "memory");
+            mx = max(max(qmax[0], qmax[1]), max(qmax[2], qmax[3]));
+            int e2 = 0;
+            frexpf(bf16_bits_to_f32(mx), &e2);   // max |q| < 2^e2
+            const int sh = e2 > 15 ? e2 - 15 : 0;
+            const float qs = ldexpf(1.f, -sh);
+            if (tid == 0) *qscale = ldexpf(1.f, sh);
 #pragma unroll
             for (int half = 0; half < 2; half++) {
                 uint4 u[18];   // 18 loads in flight
 #pragma unroll
                 for (int c = 0; c < 18; c++)
-                    u[c] = *reinterpret_cast<const uint4*>(qrow + 288 * hf + 144 * half + 8 * c);
+                    u[c] = *reinterpret_cast<const uint4*>(qrow + 144 * half + 8 * c);
 #pragma unroll
                 for (int c = 0; c < 18; c++) {
                     const int d0 = 288 * hf + 144 * half + 8 * c;
-                    if (d0 >= kD - kRopeDims) {
-                        uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+                    uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
 #pragma unroll
-                        for (int z = 0; z < 4; z++) {
+                    for (int z = 0; z < 4; z++) {
+                        float2 f = bf16x2_to_f32(w[z]);
+                        if (d0 >= kD - kRopeDims) {
                             const int pj = (d0 - (kD - kRopeDims)) / 2 + z;
-                            const float2 f = bf16x2_to_f32(w[z]);
-                            w[z] = pack_bf16x2(f.x * rqc[pj] - f.y * rqs[pj], f.x * rqs[pj] + f.y * rqc[pj]);
+                            f = make_float2(f.x * rqc[pj] - f.y * rqs[pj], f.x * rqs[pj] + f.y * rqc[pj]);
                         }
-                        u[c] = make_uint4(w[0], w[1], w[2], w[3]);
+                        w[z] = pack_f16x2(f.x * qs, f.y * qs);
                     }
-                    *cell8(sQ, kQBlk, r, d0) = u[c];
+                    *cell8(sQ, kQBlk, r, d0) = make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }
             fence_async_smem();
@@ -331,105 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         }
         // tiles: 4 threads per key row, quarter qt
         const int kr = tid >> 2, qt = tid & 3;
-        EntryQuarter ex;
-        ex.valid = false;
-        if (nloc > 0 && rank >= n_wt) fetch_entry(a, sidx, (rank - n_wt) * kTK + kr, n_vis, row0, qt, ex);
-        for (int j = 0; j < nloc && ok; j++) {
-            const int jg = rank + kCl * j;   // global tile
-            const int kb = j % kKBuf;
-            uint8_t* tile = sK + kb * kKBytes;
-            // this key buffer is free once the P V of the tile kKBuf back has completed
-            if (!mbar_wait_warp(&kfree[kb], ((j / kKBuf) & 1) ^ 1, abort_flag, a.st)) {
-                ok = false;
-                break;
-            }
-            bool vrow;
-            if (jg < n_wt) {
-                // window row: RMSNorm over all 576 channels (the four quarters meet by
-                // shuffle), RoPE at its own position on 512..575
-                const int wr = jg * kTK + kr;
-                const int64_t p = (int64_t)w0 + wr;
-                vrow = wr < n_win;
-                if (vrow && p < a.kv_pos0[b]) {
-                    vrow = false;
-                    if (qt == 0) flag(a.st, CSA_DEV_OOB);
-                }
-                const uint16_t* src =
-                    vrow ? a.kv + (a.kv_off[b] + p - a.kv_pos0[b]) * (int64_t)kD : nullptr;
-                // pass 1: my quarter of the raw row into the tile (18 loads in flight) and its
-                // sum of squares
-                float ss = 0.f;
-                {
-                    uint4 u[18];
-#pragma unroll
-                    for (int c = 0; c < 18; c++)
-                        u[c] = vrow ? *reinterpret_cast<const uint4*>(src + 144 * qt + 8 * c)
-                                    : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                    for (int c = 0; c < 18; c++) {
-                        const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
-#pragma unroll
-                        for (int z = 0; z < 4; z++) {
-                            const float2 f = bf16x2_to_f32(w[z]);
-                            ss += f.x * f.x + f.y * f.y;
-                        }
-                        *cell8(tile, kKBlk, kr, 144 * qt + 8 * c) = u[c];
-                    }
-                }
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                ss += __shfl_xor_sync(0xffffffffu, ss, 2);
-                const float rn = rsqrtf(ss / (float)kD + a.eps);
-                // rotations of the tile's 32 rows x 32 pairs, 8 per loader thread:
-                // angle (w0 + wr) f_j = w0 f_j (fp64 table) + wr f_j (< 128 rad, sincosf),
-                // combined by the addition formula
-#pragma unroll 1
-                for (int e = tid; e < kTK * 32; e += 128) {
-                    const int er = e >> 5, pj = e & 31;
-                    float sb_, cb_;
-                    sincosf((float)(jg * kTK + er) * rf[pj], &sb_, &cb_);
-                    srot[e] = make_float2(rwc[pj] * cb_ - rws[pj] * sb_, rws[pj] * cb_ + rwc[pj] * sb_);
-                }
-                asm volatile("bar.sync 3, 128;" ::: "memory");
-                // pass 2, in place in shared memory: normalise, RoPE at the row's position
-                if (vrow) {
-#pragma unroll 3
-                    for (int c = 0; c < 18; c++) {
-                        const int d0 = 144 * qt + 8 * c;
-                        uint4* cl = cell8(tile, kKBlk, kr, d0);
-                        const uint4 u = *cl;
-                        const uint32_t wi[4] = {u.x, u.y, u.z, u.w};
-                        uint32_t w[4];
-#pragma unroll
-                        for (int z = 0; z < 4; z++) {
-                            float2 f = bf16x2_to_f32(wi[z]);
-                            f.x *= rn;
-                            f.y *= rn;
-                            if (d0 >= kD - kRopeDims) {
-                                const float2 cs = srot[kr * 32 + (d0 - (kD - kRopeDims)) / 2 + z];
-                                f = make_float2(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
-                            }
-                            w[z] = pack_bf16x2(f.x, f.y);
-                        }
-                        *cl = make_uint4(w[0], w[1], w[2], w[3]);
-                    }
-                }
-                // every loader is done with this tile's rotations before the next tile's
-                asm volatile("bar.sync 3, 128;" ::: "memory");
-            } else {
-                vrow = ex.valid;
-#pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-                    if (vrow) dequant16(ex.f[u], ex.sc, lo, hi);
-                    const int d0 = 128 * qt + 16 * u;
-                    *cell8(tile, kKBlk, kr, d0) = lo;
-                    *cell8(tile, kKBlk, kr, d0 + 8) = hi;
-                }
-#pragma unroll
-                for (int u = 0; u < 2; u++)
-                    *cell8(tile, kKBlk, kr, 512 + 16 * qt + 8 * u) = vrow ? ex.rope[u] : make_uint4(0u, 0u, 0u, 0u);
-            }
-            // valid keys of the tile: this warp's 8 rows (lanes 0, 4, ..., 28 carry them)
+        // the valid keys of a tile: this warp's 8 rows (lanes 0, 4, ..., 28 carry them); then
+        // the tile is handed to the MMA issuer
+        auto publish = [&](int kb, bool vrow) {
             const uint32_t bal = __ballot_sync(0xffffffffu, vrow && qt == 0);
             uint32_t m8 = 0;
 #pragma unroll
@@ -438,65 +408,232 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             fence_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&kfull[kb]);
-            // the next entry tile's rows in flight while this one is used
-            if (j + 1 < nloc && jg + kCl >= n_wt)
-                fetch_entry(a, sidx, (jg + kCl - n_wt) * kTK + kr, n_vis, row0, qt, ex);
-        }
-    } else if (warp == 4) {
-        if (lane == 0 && nloc > 0) {
-            // ---------------- MMA issuer ----------------
-            // S of a tile is issued before the P V of the previous one, so the softmax of
-            // one tile overlaps the tensor work of its neighbours
-            bool ok = mbar_wait(qfull, 0, abort_flag, a.st);
-            tc_fence_after();
-            auto issue_s = [&](int j) -> bool {
-                const int kb = j % kKBuf, sb = j & 1;
-                if (!mbar_wait(&kfull[kb], (j / kKBuf) & 1, abort_flag, a.st) ||
-                    !mbar_wait(&sfree[sb], ((j >> 1) & 1) ^ 1, abort_flag, a.st))
-                    return false;
-                tc_fence_after();
-                const uint32_t ds = tmem + kColS + (uint32_t)(sb * kTK);
-                const uint8_t* tile = sK + kb * kKBytes;
-#pragma unroll 1
-                for (int cb = 0; cb < kNB; cb++) {
-                    const uint64_t ad = smem_desc_k_sw128(sQ + cb * kQBlk);
-                    const uint64_t bd = smem_desc_k_sw128(tile + cb * kKBlk);
-#pragma unroll
-                    for (int kk = 0; kk < 4; kk++)   // K = 16 bf16 = 32 bytes per MMA
-                        mma_f16(ds, ad + 2 * kk, bd + 2 * kk, kIdescS, (cb | kk) ? 1u : 0u);
-                }
-                mma_commit(&sfull[sb]);
-                return true;
-            };
-            if (ok) ok = issue_s(0);
-            for (int j = 0; j < nloc && ok; j++) {
-                if (j + 1 < nloc && !issue_s(j + 1)) {
-                    ok = false;
-                    break;
-                }
-                const int kb = j % kKBuf, sb = j & 1;
-                if (!mbar_wait(&pfull[sb], (j >> 1) & 1, abort_flag, a.st)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint64_t pa = smem_desc_k_sw128(sP + sb * kPBytes);
-                const uint8_t* tile = sK + kb * kKBytes;
-#pragma unroll
-                for (int kk = 0; kk < kTK / 16; kk++) {   // 16 keys per MMA
-                    const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-                    mma_f16(tmem + kColO, pa + 2 * kk, desc_mn(tile + kk * 2048, kKBlk), kIdescPV, acc);
-                    mma_f16(tmem + kColO + (16u << 16), pa + 2 * kk,
-                            desc_mn(tile + 4 * kKBlk + kk * 2048, kKBlk), kIdescPV, acc);
-                    mma_f16(tmem + kColOr, pa + 2 * kk, desc_mn(tile + 8 * kKBlk + kk * 2048, kKBlk),
-                            kIdescPVr, acc);
-                }
-                mma_commit(&kfree[kb]);
-                mma_commit(&pfree[sb]);
-                mma_commit(pvdone);
+        };
+        // ---- the window tile (global tile `rank`, this rank's first) into key buffer 0 ----
+        // (a fresh buffer: no wait).  RMSNorm over all 576 channels (the four quarters of a
+        // row meet by shuffle), RoPE at the row's own position on 512..575.
+        const bool has_win = nloc > 0 && rank < n_wt;
+        if (has_win) {
+            uint8_t* tile = sK;
+            const int wr = rank * kTK + kr;
+            const int64_t p = (int64_t)w0 + wr;
+            bool vrow = wr < n_win;
+            if (vrow && p < a.kv_pos0[b]) {
+                vrow = false;
+                if (qt == 0) flag(a.st, CSA_DEV_OOB);
             }
-            if (ok) mma_commit(odone);
-            // drain: all issued MMAs complete before TMEM is released
+            const uint16_t* src =
+                vrow ? a.kv + (a.kv_off[b] + p - a.kv_pos0[b]) * (int64_t)kD : nullptr;
+            // pass 1: my quarter of the raw row into the tile (18 loads in flight) and its
+            // sum of squares
+            float ss = 0.f;
+            {
+                uint4 u[18];
+#pragma unroll
+                for (int c = 0; c < 18; c++)
+                    u[c] = vrow ? *reinterpret_cast<const uint4*>(src + 144 * qt + 8 * c)
+                                : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int c = 0; c < 18; c++) {
+                    const uint32_t w[4] = {u[c].x, u[c].y, u[c].z, u[c].w};
+#pragma unroll
+                    for (int z = 0; z < 4; z++) {
+                        const float2 f = bf16x2_to_f32(w[z]);
+                        ss += f.x * f.x + f.y * f.y;
+                    }
+                    *cell8(tile, kKBlk, kr, 144 * qt + 8 * c) = u[c];
+                }
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            const float rn = rsqrtf(ss / (float)kD + a.eps);
+            // rotations of the tile's 32 rows x 32 pairs, 8 per loader thread:
+            // angle (w0 + wr) f_j = w0 f_j (fp64 table) + wr f_j (< 128 rad, sincosf),
+            // combined by the addition formula
+#pragma unroll 1
+            for (int e = tid; e < kTK * 32; e += 128) {
+                const int er = e >> 5, pj = e & 31;
+                float sb_, cb_;
+                sincosf((float)(rank * kTK + er) * rf[pj], &sb_, &cb_);
+                srot[e] = make_float2(rwc[pj] * cb_ - rws[pj] * sb_, rws[pj] * cb_ + rwc[pj] * sb_);
+            }
+            asm volatile("bar.sync 3, 128;" ::: "memory");
+            // pass 2, in place in shared memory: normalise, RoPE at the row's position
+            if (vrow) {
+#pragma unroll 3
+                for (int c = 0; c < 18; c++) {
+                    const int d0 = 144 * qt + 8 * c;
+                    uint4* cl = cell8(tile, kKBlk, kr, d0);
+                    const uint4 u = *cl;
+                    const uint32_t wi[4] = {u.x, u.y, u.z, u.w};
+                    uint32_t w[4];
+#pragma unroll
+                    for (int z = 0; z < 4; z++) {
+                        float2 f = bf16x2_to_f32(wi[z]);
+                        f.x *= rn;
+                        f.y *= rn;
+                        if (d0 >= kD - kRopeDims) {
+                            const float2 cs = srot[kr * 32 + (d0 - (kD - kRopeDims)) / 2 + z];
+                            f = make_float2(f.x * cs.x - f.y * cs.y, f.x * cs.y + f.y * cs.x);
+                        }
+                        w[z] = pack_f16x2(f.x, f.y);
+                    }
+                    *cl = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            publish(0, vrow);
+        }
+        // ---- the index row: the first read of another kernel's output ----
+        // Every loader thread waits for the previous grid (the top-k writes the index row,
+        // compression the entries), then the row is staged in shared memory and every entry
+        // row this rank will gather is prefetched into L2 at once (one bulk prefetch per
+        // 656-byte row), so the gathers below meet L2 rather than HBM.
+        pdl_wait();
+        if (tid == 0) pdl_trigger();
+        if (valid) {
+            // all of the row's loads in flight at once (16-byte loads when aligned)
+            const int32_t* src = a.idx + (int64_t)qi * a.k;
+            if ((a.k & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+                const int n4 = a.k >> 2;   // <= kMaxK / 4 = 4 per thread
+                int4 v[kMaxK / 4 / 128];
+#pragma unroll
+                for (int u = 0; u < kMaxK / 4 / 128; u++)
+                    if (tid + 128 * u < n4) v[u] = reinterpret_cast<const int4*>(src)[tid + 128 * u];
+#pragma unroll
+                for (int u = 0; u < kMaxK / 4 / 128; u++)
+                    if (tid + 128 * u < n4) reinterpret_cast<int4*>(sidx)[tid + 128 * u] = v[u];
+            } else {
+                int v[kMaxK / 128];
+#pragma unroll
+                for (int u = 0; u < kMaxK / 128; u++)
+                    v[u] = tid + 128 * u < a.k ? src[tid + 128 * u] : -1;
+#pragma unroll
+                for (int u = 0; u < kMaxK / 128; u++)
+                    if (tid + 128 * u < a.k) sidx[tid + 128 * u] = v[u];
+            }
+        }
+        asm volatile("bar.sync 3, 128;" ::: "memory");
+        if (valid) {
+            for (int u = tid; u < nloc * kTK; u += 128) {
+                const int jg = rank + kCl * (u / kTK);
+                const int v = (jg - n_wt) * kTK + u % kTK;
+                if (jg < n_wt || v >= a.k) continue;
+                const int e = sidx[v];
+                if (e >= 0 && e < n_vis && row0 + e < a.ent_rows)
+                    prefetch_l2_bulk(a.entries + (row0 + e) * (int64_t)kRowBytes, kRowBytes);
+            }
+        }
+        // ---- the selected entries ----
+        // Each thread converts its quarter of a key row from registers (e4m3 x scale ->
+        // fp16, the bf16 RoPE channels to fp16) into the key buffer.  Two register sets: the
+        // loads of tile j + 2 are issued as soon as tile j is converted, so every gather
+        // has two tiles' time to arrive (the rows are also being prefetched into L2).
+        const int j0 = has_win ? 1 : 0;
+        EntryQuarter exa, exb;
+        exa.valid = exb.valid = false;
+        auto entry_of = [&](int j) { return (rank + kCl * j - n_wt) * kTK + kr; };
+        if (j0 < nloc) fetch_entry(a, sidx, entry_of(j0), n_vis, row0, qt, exa);
+        if (j0 + 1 < nloc) fetch_entry(a, sidx, entry_of(j0 + 1), n_vis, row0, qt, exb);
+        // converts tile j from `ex`, then issues tile j + 2's loads into it
+        auto tile_step = [&](int j, EntryQuarter& ex) -> bool {
+            const int kb = j % kKBuf;
+            uint8_t* tile = sK + kb * kKBytes;
+            // this key buffer is free once the P V of the tile kKBuf back has completed
+            if (j >= kKBuf && !mbar_wait_warp(&kfree[kb], ((j / kKBuf) & 1) ^ 1, abort_flag, a.st))
+                return false;
+            const bool vrow = ex.valid;
+            const uint32_t sc2 = vrow ? pack_f16x2(ex.sc, ex.sc) : 0u;
+#pragma unroll
+            for (int u = 0; u < 8; u++) {
+                uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+                if (vrow) dequant16(ex.f[u], sc2, lo, hi);
+                const int d0 = 128 * qt + 16 * u;
+                *cell8(tile, kKBlk, kr, d0) = lo;
+                *cell8(tile, kKBlk, kr, d0 + 8) = hi;
+            }
+            // the RoPE channels are stored as bf16: to fp16 (exact within the fp16 range)
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                uint4 h = make_uint4(0u, 0u, 0u, 0u);
+                if (vrow) {
+                    const uint32_t w[4] = {ex.rope[u].x, ex.rope[u].y, ex.rope[u].z, ex.rope[u].w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int z = 0; z < 4; z++) {
+                        const float2 f = bf16x2_to_f32(w[z]);
+                        o[z] = pack_f16x2(f.x, f.y);
+                    }
+                    h = make_uint4(o[0], o[1], o[2], o[3]);
+                }
+                *cell8(tile, kKBlk, kr, 512 + 16 * qt + 8 * u) = h;
+            }
+            publish(kb, vrow);
+            if (j + 2 < nloc) fetch_entry(a, sidx, entry_of(j + 2), n_vis, row0, qt, ex);
+            return true;
+        };
+        for (int j = j0; j < nloc && ok; j += 2) {
+            ok = tile_step(j, exa);
+            if (ok && j + 1 < nloc) ok = tile_step(j + 1, exb);
+        }
+    } else if (warp == 4 || warp >= kFirstSWarp) {
+        if (lane == 0 && nloc > 0) {
+            // ---------------- MMA issuers ----------------
+            // One tcgen05.mma costs its issuing thread tens of cycles whatever its shape, and
+            // S takes 36 per tile: the S of even tiles is issued by warp kFirstSWarp, of odd
+            // tiles by warp kFirstSWarp + 1 (each owns one S buffer), and P V by warp 4.
+            // K buffer kb is released by P V's commit: the tile's S was complete before its P
+            // (hence its P V) existed.
+            bool ok = true;
+            if (warp >= kFirstSWarp) {
+                const int e = warp - kFirstSWarp;   // S buffer and tile parity
+                ok = mbar_wait(qfull, 0, abort_flag, a.st);
+                tc_fence_after();
+                for (int j = e; j < nloc && ok; j += 2) {
+                    const int kb = j % kKBuf;
+                    if (!mbar_wait(&kfull[kb], (j / kKBuf) & 1, abort_flag, a.st) ||
+                        !mbar_wait(&sfree[e], ((j >> 1) & 1) ^ 1, abort_flag, a.st)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint8_t* tile = sK + kb * kKBytes;
+#pragma unroll 1
+                    for (int cb = 0; cb < kNB; cb++) {
+                        const uint64_t ad = smem_desc_k_sw128(sQ + cb * kQBlk);
+                        const uint64_t bd = smem_desc_k_sw128(tile + cb * kKBlk);
+#pragma unroll
+                        for (int kk = 0; kk < 4; kk++)   // K = 16 fp16 = 32 bytes, partial kk
+                            mma_f16(tmem + s_col(e, kk), ad + 2 * kk, bd + 2 * kk, kIdescS,
+                                    cb ? 1u : 0u);
+                    }
+                    mma_commit(&sfull[e]);
+                }
+            } else {
+                for (int j = 0; j < nloc && ok; j++) {
+                    const int kb = j % kKBuf, sb = j & 1;
+                    if (!mbar_wait(&pfull[sb], (j >> 1) & 1, abort_flag, a.st)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t pa = smem_desc_k_sw128(sP + sb * kPBytes);
+                    const uint8_t* tile = sK + kb * kKBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kTK / 16; kk++) {   // 16 keys per MMA
+                        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+                        mma_f16(tmem + kColO, pa + 2 * kk, desc_mn(tile + kk * 2048, kKBlk), kIdescPV, acc);
+                        mma_f16(tmem + kColO + (16u << 16), pa + 2 * kk,
+                                desc_mn(tile + 4 * kKBlk + kk * 2048, kKBlk), kIdescPV, acc);
+                        mma_f16(tmem + kColOr, pa + 2 * kk, desc_mn(tile + 8 * kKBlk + kk * 2048, kKBlk),
+                                kIdescPVr, acc);
+                    }
+                    mma_commit(&kfree[kb]);
+                    mma_commit(&pfree[sb]);
+                    mma_commit(pvdone);
+                }
+                if (ok) mma_commit(odone);
+            }
+            // drain: every issuer's MMAs complete before TMEM is released
             mma_commit(drain);
             mbar_drain(drain, 0, a.st);
         }
@@ -507,6 +644,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         const bool mine = lane < 16;                 // S rows live in lanes 0-15
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         float mref = -INFINITY, lrun = 0.f;
+        // S carries the query's 2^-s scaling: the softmax scale takes 2^s (exact)
+        float sl2 = a.scale_log2;
+        if (nloc > 0) {
+            if (mbar_wait_warp(qfull, 0, abort_flag, a.st)) sl2 *= *qscale;
+        }
         bool ok = true;
         for (int j = 0; j < nloc && ok; j++) {
             const int sb = j & 1;
@@ -515,9 +657,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 break;
             }
             tc_fence_after();
+            // S = (p0 + p2) + (p1 + p3): lanes 0-15 read partials 0 and 2 of head hl, lanes
+            // 16-31 partials 1 and 3 of the same head; one exchange across the half-warps
+            // gives every lane the same sums (a fixed order, whatever the batch)
             uint32_t sv[kTK];
-            tmem_ld32(tmem + kColS + (uint32_t)(sb * kTK) + lane_base, sv);
-            tmem_ld_wait();
+            {
+                uint32_t s0[kTK], s1[kTK];
+                tmem_ld32(tmem + s_col(sb, 0) + lane_base, s0);
+                tmem_ld32(tmem + s_col(sb, 2) + lane_base, s1);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < kTK; c++) {
+                    const float v = __uint_as_float(s0[c]) + __uint_as_float(s1[c]);
+                    sv[c] = __float_as_uint(v + __shfl_xor_sync(0xffffffffu, v, 16));
+                }
+            }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sfree[sb]);
@@ -539,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                     rmax = fmaxf(rmax, xv);
                 }
             }
-            const float tmax = rmax * a.scale_log2;
+            const float tmax = rmax * sl2;
             // move the reference maximum only on a jump of more than 2^8
             const bool need = mine && tmax > mref + kRescale;
             if (__any_sync(0xffffffffu, need)) {
@@ -584,10 +738,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 const float nm = -mref;
 #pragma unroll
                 for (int c = 0; c < kTK / 2; c++) {
-                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), a.scale_log2, nm));
-                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), a.scale_log2, nm));
+                    const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * c]), sl2, nm));
+                    const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, nm));
                     rs += p0 + p1;
-                    pk[c] = pack_bf16x2(p0, p1);
+                    pk[c] = pack_f16x2(p0, p1);
                 }
             }
             lrun += rs;
@@ -607,109 +761,108 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             if (lane == 0) mbar_arrive(&pfull[sb]);
         }
         if (ok && nloc > 0) ok = mbar_wait_warp(odone, 0, abort_flag, a.st);
-        if (ntiles > 0) {
-            // ---- partial states across the cluster ----
-            // my MMAs are done: my Q / key / P / staging buffers may take the partials
-            if (ok) {
-                tc_fence_after();
-                __syncwarp();
-                if (lane == 0)
-                    for (int rr = 0; rr < kCl; rr++) mbar_arrive_cluster(mapa(recv_ready, (uint32_t)rr));
-                ok = mbar_wait_cluster_warp(recv_ready, 0, abort_flag, a.st);
-            }
-            if (ok) {
-                // head hl goes to rank hl / kHO (this warp's 16 heads: rank `quarter`)
-                const int own = hl / kHO, lh = hl - own * kHO;
-                float* recv_ml = recv + kRecvO;
-                const uint32_t dst = mapa(recv + (rank * kHO + lh) * 576 + (mine ? 0 : 256), (uint32_t)own);
+        if (ntiles > 0 && ok) {
+            // ---- this rank's partial state into its own shared memory ----
+            // Every MMA of this rank is complete, so Q / K / P may take it.  Lanes 0-15 hold
+            // head hl's channels 0-255 (then 512-575), lanes 16-31 its channels 256-511.
+            tc_fence_after();
+            float* prow = part + hl * kPS;
+            const int half = lane >> 4;
 #pragma unroll 1
-                for (int cc = 0; cc < 5; cc++) {
-                    // 64 columns at a time: 0-255 (both lane halves), then 256-319 (lanes 0-15)
-                    const uint32_t col = cc < 4 ? kColO + 64u * cc : kColOr;
-                    uint32_t ov[64];
-                    if (nloc > 0) {
-                        tmem_ld64(tmem + col + lane_base, ov);
-                        tmem_ld_wait();
-                    } else {
+            for (int cc = 0; cc < 5; cc++) {
+                const uint32_t col = cc < 4 ? kColO + 64u * cc : kColOr;
+                uint32_t ov[64];
+                if (nloc > 0) {
+                    tmem_ld64(tmem + col + lane_base, ov);
+                    tmem_ld_wait();
+                } else {
 #pragma unroll
-                        for (int z = 0; z < 64; z++) ov[z] = 0u;
-                    }
-                    if (cc < 4 || mine) {
-                        // lanes 0-15: channels 0-255 then 512-575; lanes 16-31: 256-511
-                        const uint32_t off = (cc < 4 ? 64u * cc : 512u) * 4u;
+                    for (int z = 0; z < 64; z++) ov[z] = 0u;
+                }
+                if (cc < 4 || mine) {
+                    float* dst = prow + (cc < 4 ? 256 * half + 64 * cc : 512);
 #pragma unroll
-                        for (int z = 0; z < 64; z += 4)
-                            st_cluster_f4(dst + off + 4u * z,
-                                          make_float4(__uint_as_float(ov[z]), __uint_as_float(ov[z + 1]),
-                                                      __uint_as_float(ov[z + 2]), __uint_as_float(ov[z + 3])));
-                    }
+                    for (int z = 0; z < 64; z += 4)
+                        *reinterpret_cast<float4*>(dst + z) =
+                            make_float4(__uint_as_float(ov[z]), __uint_as_float(ov[z + 1]),
+                                        __uint_as_float(ov[z + 2]), __uint_as_float(ov[z + 3]));
                 }
-                if (mine) {
-                    st_cluster_f32(mapa(recv_ml + (2 * rank) * kHO + lh, (uint32_t)own), mref);
-                    st_cluster_f32(mapa(recv_ml + (2 * rank + 1) * kHO + lh, (uint32_t)own), lrun);
-                }
-                tc_fence_before();
-                fence_cluster();
-                __syncwarp();
-                if (lane == 0)
-                    for (int rr = 0; rr < kCl; rr++) mbar_arrive_cluster(mapa(cpart_full, (uint32_t)rr));
-                ok = mbar_wait_cluster_warp(cpart_full, 0, abort_flag, a.st);
             }
-            if (named_barrier_and(2, 128, ok)) {
-                // this rank's heads; first the combine weights, one thread per head:
-                // M = max(sink, m_r), w_r = 2^(m_r - M), L = 2^(sink - M) + sum_r w_r l_r
-                const float* recv_ml = recv + kRecvO;
-                const int i = threadIdx.x - 160;
-                if (i < kHO) {
-                    const float sk = a.sink[kHC * g + rank * kHO + i] * kLog2e;
-                    float M = sk;
+            if (mine) {
+                part[kPartML + hl] = mref;
+                part[kPartML + kHC + hl] = lrun;
+            }
+            tc_fence_before();
+            // released to every rank of the cluster
+            fence_cluster();
+            __syncwarp();
+            if (lane == 0)
+                for (int rr = 0; rr < kCl; rr++) mbar_arrive_cluster(mapa(cpart_full, (uint32_t)rr));
+        }
+    }
+
+    // ---- combine: this rank's kHO heads, by the loader and softmax warps (256 threads) ----
+    // Each pulls the kCl partial states of its heads from the ranks' shared memory
+    // (ld.shared::cluster, 16 consecutive bytes per lane) and sums them in rank order.
+    if ((warp < 4 || (warp > 4 && warp < kFirstSWarp)) && ntiles > 0) {
+        const int ci = warp < 4 ? threadIdx.x : threadIdx.x - 32;   // 0 .. 255
+        const bool okc = mbar_wait_cluster_warp(cpart_full, 0, abort_flag, a.st);
+        if (named_barrier_and(2, 256, okc)) {
+            // the combine weights, one thread per head, the sink first:
+            // M = max(sink, m_r), w_r = 2^(m_r - M), L = 2^(sink - M) + sum_r w_r l_r
+            if (ci < kHO) {
+                const int h = rank * kHO + ci;
+                const float sk = a.sink[kHC * g + h] * kLog2e;
+                float mr[kCl], lr[kCl];
 #pragma unroll
-                    for (int rr = 0; rr < kCl; rr++) M = fmaxf(M, recv_ml[(2 * rr) * kHO + i]);
-                    float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
-#pragma unroll
-                    for (int rr = 0; rr < kCl; rr++) {
-                        const float mr = recv_ml[(2 * rr) * kHO + i];
-                        const float wgt = (mr == -INFINITY) ? 0.f : exp2f(mr - M);
-                        L = fmaf(wgt, recv_ml[(2 * rr + 1) * kHO + i], L);
-                        swt[i * 8 + rr] = wgt;
-                    }
-                    swt[i * 8 + kCl] = L;
+                for (int rr = 0; rr < kCl; rr++) {
+                    mr[rr] = ld_cluster_f32(mapa(part + kPartML + h, (uint32_t)rr));
+                    lr[rr] = ld_cluster_f32(mapa(part + kPartML + kHC + h, (uint32_t)rr));
                 }
-                asm volatile("bar.sync 2, 128;" ::: "memory");
-                // then (head, 4 channels) per work unit: sum_r w_r O_r / L
-#pragma unroll 2
-                for (int w = i; w < kHO * (576 / 4); w += 128) {
-                    const int lh = w / (576 / 4), c4 = (w - lh * (576 / 4)) * 4;
-                    const int h = kHC * g + rank * kHO + lh;
-                    const float L = swt[lh * 8 + kCl];
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                float M = sk;
 #pragma unroll
-                    for (int rr = 0; rr < kCl; rr++) {
-                        const float wgt = swt[lh * 8 + rr];
-                        const float4 v = *reinterpret_cast<const float4*>(recv + (rr * kHO + lh) * 576 + c4);
-                        acc.x = fmaf(wgt, v.x, acc.x);
-                        acc.y = fmaf(wgt, v.y, acc.y);
-                        acc.z = fmaf(wgt, v.z, acc.z);
-                        acc.w = fmaf(wgt, v.w, acc.w);
-                    }
-                    if (L > 0.f) {
-                        acc.x /= L;
-                        acc.y /= L;
-                        acc.z /= L;
-                        acc.w /= L;
-                    } else {
-                        acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-                    if (c4 >= kD - kRopeDims) {
-                        // rotation by -t: (x, y) -> (x cos + y sin, y cos - x sin)
-                        const int pj = (c4 - (kD - kRopeDims)) >> 1;
-                        const float c0 = rqc[pj], s0 = rqs[pj], c1 = rqc[pj + 1], s1 = rqs[pj + 1];
-                        acc = make_float4(acc.x * c0 + acc.y * s0, acc.y * c0 - acc.x * s0,
-                                          acc.z * c1 + acc.w * s1, acc.w * c1 - acc.z * s1);
-                    }
-                    *reinterpret_cast<uint2*>(a.out + ((int64_t)qi * a.H + h) * kD + c4) =
-                        make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+                for (int rr = 0; rr < kCl; rr++) M = fmaxf(M, mr[rr]);
+                float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
+#pragma unroll
+                for (int rr = 0; rr < kCl; rr++) {
+                    const float wgt = (mr[rr] == -INFINITY) ? 0.f : exp2f(mr[rr] - M);
+                    L = fmaf(wgt, lr[rr], L);
+                    swt[ci * kWtStride + rr] = wgt;
                 }
+                swt[ci * kWtStride + kCl] = L > 0.f ? 1.f / L : 0.f;
+            }
+            asm volatile("bar.sync 2, 256;" ::: "memory");
+            // the output may still be read by the kernel before this one: wait for it
+            // (long finished by now whenever this rank gathered entries)
+            pdl_wait();
+            // (head, 4 channels) per work unit: sum_r w_r O_r / L, inverse RoPE, 4 bf16
+#pragma unroll 3
+            for (int w = ci; w < kHO * (576 / 4); w += 256) {
+                const int lh = w / (576 / 4), c4 = (w - lh * (576 / 4)) * 4;
+                const int h = rank * kHO + lh;
+                float4 v[kCl];
+#pragma unroll
+                for (int rr = 0; rr < kCl; rr++) v[rr] = ld_cluster_f4(mapa(part + h * kPS + c4, (uint32_t)rr));
+                const float invL = swt[lh * kWtStride + kCl];
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int rr = 0; rr < kCl; rr++) {
+                    const float wgt = swt[lh * kWtStride + rr];
+                    acc.x = fmaf(wgt, v[rr].x, acc.x);
+                    acc.y = fmaf(wgt, v[rr].y, acc.y);
+                    acc.z = fmaf(wgt, v[rr].z, acc.z);
+                    acc.w = fmaf(wgt, v[rr].w, acc.w);
+                }
+                acc = make_float4(acc.x * invL, acc.y * invL, acc.z * invL, acc.w * invL);
+                if (c4 >= kD - kRopeDims) {
+                    // rotation by -t: (x, y) -> (x cos + y sin, y cos - x sin)
+                    const int pj = (c4 - (kD - kRopeDims)) >> 1;
+                    const float c0 = rqc[pj], s0 = rqs[pj], c1 = rqc[pj + 1], s1 = rqs[pj + 1];
+                    acc = make_float4(acc.x * c0 + acc.y * s0, acc.y * c0 - acc.x * s0,
+                                      acc.z * c1 + acc.w * s1, acc.w * c1 - acc.z * s1);
+                }
+                *reinterpret_cast<uint2*>(a.out + ((int64_t)qi * a.H + kHC * g + h) * kD + c4) =
+                    make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
             }
         }
     }
