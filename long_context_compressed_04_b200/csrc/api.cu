@@ -43,6 +43,23 @@ bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Workspace of lightning_indexer_topk: first the group maxima (the largest score key of
+// every 32 consecutive entries of every query, which the top-k selects from), then the
+// score rows (round_up(max_n, 32) floats per query), which scores_out replaces.
+struct IndexerWorkspace {
+    int64_t ld, ld_g;
+    size_t gmax_bytes, off_scores, total;
+};
+IndexerWorkspace indexer_workspace(int32_t Q, int32_t max_n) {
+    IndexerWorkspace w;
+    w.ld = (int64_t)round_up((size_t)max_n, 32);
+    w.ld_g = w.ld / 32;
+    w.gmax_bytes = round_up((size_t)Q * w.ld_g * 4, 256);
+    w.off_scores = w.gmax_bytes;
+    w.total = w.off_scores + round_up((size_t)Q * w.ld * sizeof(float), 256) + 256;
+    return w;
+}
+
 csa_status_t compress_common(int m, int span, const void* kv, const void* gate,
                              const float* bias, const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
                              const int64_t* ent_off, const int32_t* item_seq,
@@ -143,8 +160,7 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
 
 size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k) {
     if (Q <= 0 || max_n < 0 || k <= 0) return 0;
-    (void)k;
-    return round_up((size_t)Q * round_up((size_t)max_n, 32) * sizeof(float), 256) + 256;
+    return indexer_workspace(Q, max_n).total;
 }
 
 csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, const float* w,
@@ -169,24 +185,30 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     SUPPORT(d_I == 64 || d_I == 128, "indexer dim %d not supported (64 or 128)", d_I);
     SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
     REQUIRE(scores_out == nullptr || ld_scores >= max_n, "ld_scores must be >= max_n");
-    // the workspace holds only the score rows: with scores_out it is not used
-    const size_t need = csa_indexer_workspace_size(Q, max_n, k);
-    if (!scores_out && (!workspace || workspace_bytes < need || !aligned(workspace, 256)))
-        return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", need);
-    float* scores = scores_out ? scores_out : (float*)workspace;
-    const int64_t ld = scores_out ? ld_scores : (int64_t)round_up((size_t)max_n, 32);
+    // With scores_out the score rows go there and the workspace needs only its group-maxima
+    // region (a smaller or missing workspace then leaves the top-k to the full rows).
+    const IndexerWorkspace L = indexer_workspace(Q, max_n);
+    if (!scores_out && (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)))
+        return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", L.total);
+    float* scores = scores_out ? scores_out : (float*)((uint8_t*)workspace + L.off_scores);
+    const int64_t ld = scores_out ? ld_scores : L.ld;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (csa::indexer_tc_supported(H_I, d_I))
+    uint32_t* gmax = nullptr;
+    if (csa::indexer_tc_supported(H_I, d_I)) {
+        if (workspace && workspace_bytes >= L.gmax_bytes && aligned(workspace, 256))
+            gmax = (uint32_t*)workspace;
         e = csa::launch_indexer_tc(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
-                                   q_seq, q_pos, Q, B, H_I, m, max_n, scores, ld, dev_status, s);
-    else
+                                   q_seq, q_pos, Q, B, H_I, m, max_n, scores, ld, dev_status, s,
+                                   gmax, L.ld_g);
+    } else {
         e = csa::launch_indexer_simt(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
                                      q_seq, q_pos, Q, B, H_I, d_I, m, max_n, scores, ld,
                                      dev_status, s);
+    }
     if (e != cudaSuccess) return cuda_status(e, "indexer launch");
     e = csa::launch_topk(scores, ld, q_seq, q_pos, seq_len, Q, B, m, max_n, k, idx_out, dev_status,
-                         s);
+                         s, gmax, L.ld_g);
     return cuda_status(e, "top-k launch");
 }
 

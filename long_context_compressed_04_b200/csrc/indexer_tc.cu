@@ -66,6 +66,10 @@ struct IdxArgs {
     int Q, B, m, max_n;
     int qtiles;              // virtual tiles per query: ceil(max_n / 128)
     int chunks_per_q;        // ceil(qtiles / 8)
+    // nullable: per query, the largest score key (order_key) of every group of 32
+    // consecutive entries, group g of query q at gmax[q * ld_g + g] (see the top-k)
+    uint32_t* gmax;
+    int64_t ld_g;
 };
 
 struct Item {
@@ -414,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_ld16(taddr, d);
                     }
                     tmem_ld_wait();
+                    uint32_t key = 0u;   // below every score's key
                     if (e < x.n_vis) {
                         float acc = 0.f;
 #pragma unroll
@@ -422,6 +427,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float sc = acc * ks_s[tt * kTileRows + row_in_tile];
                         if (sc != sc) flag(a.st, CSA_DEV_NAN);
                         srow[e] = sc;
+                        key = order_key(sc);
+                    }
+                    if (a.gmax) {
+                        // the warp's 32 rows are one group of 32 consecutive entries
+                        key = __reduce_max_sync(0xffffffffu, key);
+                        const int e0 = e - lane;
+                        if (lane == 0 && e0 < x.n_vis) a.gmax[(int64_t)x.q * a.ld_g + (e0 >> 5)] = key;
                     }
                 }
                 tc_fence_before();
@@ -522,7 +534,7 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
                               const int64_t* seq_len, const int64_t* ent_off,
                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
                               int m, int max_n, float* scores, int64_t ld, int32_t* st,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, uint32_t* gmax, int64_t ld_g) {
     if (Q == 0 || max_n == 0 || ent_rows == 0) return cudaSuccess;
     IdxArgs args;
     args.qs = qs;
@@ -540,6 +552,8 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
     args.B = B;
     args.m = m;
     args.max_n = max_n;
+    args.gmax = gmax;
+    args.ld_g = ld_g;
     args.qtiles = (max_n + kTileRows - 1) / kTileRows;
     args.chunks_per_q = (args.qtiles + kChunkTiles - 1) / kChunkTiles;
     switch (HI) {

@@ -110,10 +110,11 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
                               const int64_t* seq_len, const int64_t* ent_off,
                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
                               int m, int max_n, float* scores, int64_t ld, int32_t* st,
-                              cudaStream_t stream);
+                              cudaStream_t stream, uint32_t* gmax = nullptr, int64_t ld_g = 0);
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
-                        int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream);
+                        int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream,
+                        const uint32_t* gmax = nullptr, int64_t ld_g = 0);
 cudaError_t launch_attn_simt(const AttnArgs& a, int Q, int D, cudaStream_t stream);
 bool attn_tc_supported(int H, int D, int fmt);
 bool attn576_tc_supported(int H, int D, int fmt);

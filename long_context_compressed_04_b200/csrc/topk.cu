@@ -33,6 +33,8 @@
 // keys of the row, one exchange gives every rank all ranks' candidates and their counts of
 // keys above the bin; the remaining bits are then resolved on every rank alone, and the
 // lower ranks' counts give each rank its output offset and tie budget.
+#include <algorithm>
+
 #include "launchers.cuh"
 #include "sm100.cuh"
 
@@ -46,11 +48,7 @@ constexpr int kBins = 2048;
 constexpr int kChunk = 4 * kThreads;
 constexpr int kMaxCand = 4096;
 
-__device__ __forceinline__ uint32_t score_key(float s) {
-    uint32_t u = __float_as_uint(s);
-    if (u == 0x80000000u) u = 0u;  // -0 ties with +0
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
+__device__ __forceinline__ uint32_t score_key(float s) { return order_key(s); }
 
 // Exclusive prefix sum over the CTA of `v`; `total` gets the CTA sum.  tmp: >= 33 ints.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* tmp,
@@ -105,6 +103,7 @@ struct Shared {
     uint32_t s_or, s_and, c_or, c_and;   // OR / AND of the sample and of the candidates
     uint64_t stage_bar;                   // bulk copies of the row into shared memory
     int abort;
+    uint32_t cor[2], ngrp, nsel;          // the group path (see topk_by_groups)
     uint32_t cand[kMaxCand];
 };
 
@@ -218,13 +217,231 @@ __device__ __forceinline__ uint32_t select_kth_list(Shared& sh, const uint32_t* 
     return prefix;
 }
 
+// As select_kth_list, over shared-memory scratch given by pointers: hist >= kBins words,
+// scan_tmp >= 33 words, bin_out / krem_out one word each.  With max_digits > 0 it stops
+// after that many digits and returns the lower edge of the bin reached, a value <= the kth
+// largest (krem is then not meaningful).
+__device__ __forceinline__ uint32_t select_kth_raw(const uint32_t* list, uint32_t cnt, uint32_t kth,
+                                                   uint32_t kor, uint32_t kand, uint32_t& krem,
+                                                   uint32_t* hist, uint32_t* scan_tmp,
+                                                   uint32_t* bin_out, uint32_t* krem_out,
+                                                   int max_digits = 0) {
+    const uint32_t vary = kor ^ kand;
+    uint32_t prefix = kand & ~vary, mask = ~vary;
+    krem = kth;
+    int top = vary ? 31 - __clz(vary) : -1;
+    for (int digit = 0; top >= 0 && (max_digits == 0 || digit < max_digits); digit++) {
+        const int width = top >= 10 ? 11 : top + 1;
+        const int shift = top + 1 - width;
+        const uint32_t bmask = (1u << width) - 1u;
+        for (int x = threadIdx.x; x < kBins; x += kThreads) hist[x] = 0u;
+        __syncthreads();
+        for (uint32_t c = threadIdx.x; c < cnt; c += kThreads) {
+            const uint32_t key = list[c];
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & bmask], 1u);
+        }
+        __syncthreads();
+        pick_bin_in(hist, scan_tmp, bin_out, krem_out, krem);
+        prefix |= *bin_out << shift;
+        mask |= bmask << shift;
+        top = shift - 1;
+        __syncthreads();
+    }
+    return prefix;
+}
+
+// Shared memory of the group path (see topk_by_groups): two words per group of 32 entries
+// (the group keys and the list of groups reaching the bound, later the selection words),
+// then cap candidate keys and cap candidate entries.
+__host__ __device__ constexpr size_t group_smem_bytes(int max_n, int cap) {
+    return (size_t)((2 * ((max_n + 31) / 32) + 3) / 4) * 16 + (size_t)cap * 8;
+}
+
+// OR / AND of `v` over the CTA into or_and[0] / or_and[1] (initialised by the caller before
+// a barrier); ends with the CTA synchronised.
+__device__ __forceinline__ void block_or_and(uint32_t o, uint32_t a, uint32_t* or_and) {
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+        o |= __shfl_xor_sync(0xffffffffu, o, s);
+        a &= __shfl_xor_sync(0xffffffffu, a, s);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicOr(&or_and[0], o);
+        atomicAnd(&or_and[1], a);
+    }
+    __syncthreads();
+}
+
+// Top-k of a query from the group maxima the indexer wrote: qg[g] is the largest score key
+// of entries 32g .. 32g + 31.  B, the k-th largest of the G = ceil(n / 32) group keys (one
+// needs G >= k), bounds the k-th largest score from below, since the k groups at or above B
+// each hold an entry whose key is >= B.  So the top-k are among the entries >= B, and those
+// lie in the groups whose key is >= B (about k of them): only those groups' scores are
+// read.  The entries >= B are listed (at least k of them; the call returns false, with
+// nothing written, when more than cap), the k-th largest key T is selected among them, and
+// the selection -- every entry > T and the lowest-indexed ties -- is written in ascending
+// entry order from bit words of 32 entries.  The result is the unique top-k under the tie
+// order.  All 1024 threads call it; dyn holds group_smem_bytes(n, cap) bytes.
+__device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
+                               const uint32_t* __restrict__ qg, int n, int k, int cap,
+                               int32_t* __restrict__ out, uint8_t* dyn, Shared& sh) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int G = (n + 31) >> 5;
+    uint32_t* gk = reinterpret_cast<uint32_t*>(dyn);
+    uint32_t* glist = gk + G;
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dyn + ((2 * G + 3) / 4) * 16);
+    uint32_t* cent = ckey + cap;
+    // 1. the group keys
+    if (tid == 0) {
+        sh.cor[0] = 0u;
+        sh.cor[1] = 0xFFFFFFFFu;
+        sh.ngrp = 0u;
+        sh.nsel = 0u;
+    }
+    __syncthreads();
+    uint32_t kor = 0u, kand = 0xFFFFFFFFu;
+    for (int g = tid; g < G; g += kThreads) {
+        const uint32_t v = qg[g];
+        gk[g] = v;
+        kor |= v;
+        kand &= v;
+    }
+    block_or_and(kor, kand, sh.cor);
+    // 2. B: the lower edge of the bin of the k-th largest group key after two 11-bit
+    // digits from the highest varying bit (a lower bound of it, as exact as needed)
+    uint32_t krem;
+    const uint32_t B = select_kth_raw(gk, (uint32_t)G, (uint32_t)k, sh.cor[0], sh.cor[1], krem,
+                                      sh.hist, sh.scan_tmp, &sh.bin, &sh.krem, 2);
+    // 3. the groups reaching B (any order)
+    for (int g0 = 0; g0 < G; g0 += kThreads) {
+        const int g = g0 + tid;
+        const bool pass = g < G && gk[g] >= B;
+        const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+        uint32_t base = 0u;
+        if (lane == 0 && bal) base = atomicAdd(&sh.ngrp, (uint32_t)__popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (pass) glist[base + __popc(bal & lanemask_lt())] = (uint32_t)g;
+    }
+    __syncthreads();
+    const uint32_t ng = sh.ngrp;
+    // 4. their entries reaching B: 8 slots of 4 entries per group, up to 4 slots per thread
+    // with all of their loads in flight; each thread's passing entries are placed by one
+    // warp scan and one shared atomic per warp
+    const uint32_t nslots = ng * 8u;
+    for (uint32_t b0 = 0; b0 < nslots; b0 += 4u * kThreads) {
+        uint32_t key[4][4] = {};
+        int e0[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const uint32_t slot = b0 + (uint32_t)tid + (uint32_t)(u * kThreads);
+            e0[u] = slot < nslots ? (int)(glist[slot >> 3] * 32u + (slot & 7u) * 4u) : n;
+            if (e0[u] < n) load4(s, e0[u], n, vec, key[u]);
+        }
+        uint32_t pm = 0u;   // bit 4u + z: entry e0[u] + z reaches B
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+#pragma unroll
+            for (int z = 0; z < 4; z++)
+                if (e0[u] + z < n && key[u][z] >= B) pm |= 1u << (4 * u + z);
+        const uint32_t cnt = __popc(pm);
+        uint32_t inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        uint32_t base = 0u;
+        if (lane == 31 && inc) base = atomicAdd(&sh.nsel, inc);
+        base = __shfl_sync(0xffffffffu, base, 31);
+        uint32_t pos = base + inc - cnt;
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+#pragma unroll
+            for (int z = 0; z < 4; z++)
+                if ((pm >> (4 * u + z)) & 1u) {
+                    if (pos < (uint32_t)cap) {
+                        ckey[pos] = key[u][z];
+                        cent[pos] = (uint32_t)(e0[u] + z);
+                    }
+                    pos++;
+                }
+    }
+    if (tid == 0) {
+        sh.cor[0] = 0u;
+        sh.cor[1] = 0xFFFFFFFFu;
+    }
+    __syncthreads();
+    const uint32_t c = sh.nsel;
+    // the same value in every thread; fewer than k only if some group maximum was not
+    // written (an entry row past the key store, flagged by the indexer)
+    if (c > (uint32_t)cap || c < (uint32_t)k) return false;
+    // 5. T among the c >= k candidates
+    kor = 0u;
+    kand = 0xFFFFFFFFu;
+    for (uint32_t i = tid; i < c; i += kThreads) {
+        kor |= ckey[i];
+        kand &= ckey[i];
+    }
+    block_or_and(kor, kand, sh.cor);
+    const uint32_t T = select_kth_raw(ckey, c, (uint32_t)k, sh.cor[0], sh.cor[1], krem,
+                                      sh.hist, sh.scan_tmp, &sh.bin, &sh.krem);
+    // 6. selection words over the row (over the group keys and list, no longer needed)
+    const int nw = G;
+    uint32_t* selw = gk;
+    uint32_t* tiew = gk + nw;
+    for (int w = tid; w < 2 * nw; w += kThreads) selw[w] = 0u;
+    __syncthreads();
+    for (uint32_t i = tid; i < c; i += kThreads) {
+        const uint32_t key = ckey[i], e = cent[i];
+        if (key > T) atomicOr(&selw[e >> 5], 1u << (e & 31));
+        else if (key == T) atomicOr(&tiew[e >> 5], 1u << (e & 31));
+    }
+    __syncthreads();
+    // each thread a contiguous run of words: its counts of selected and tied entries; the
+    // CTA's prefix gives its output position and the ties before it
+    const int per = (nw + kThreads - 1) / kThreads;
+    const int w0 = tid * per, w1 = min(nw, w0 + per);
+    uint32_t cs = 0u, ct = 0u;
+    for (int w = w0; w < w1; w++) {
+        cs += __popc(selw[w]);
+        ct += __popc(tiew[w]);
+    }
+    unsigned long long tot;
+    const unsigned long long pre =
+        block_exclusive_scan64(((unsigned long long)cs << 32) | ct, sh.scan64, tot);
+    uint32_t ties = (uint32_t)pre;
+    uint32_t pos = (uint32_t)(pre >> 32) + min(ties, krem);
+    for (int w = w0; w < w1; w++) {
+        const uint32_t sw = selw[w], tw = tiew[w];
+        uint32_t take_t = 0u;
+        if (ties < krem) {
+            uint32_t need = krem - ties, tt = tw;
+            while (need && tt) {
+                take_t |= tt & (0u - tt);
+                tt &= tt - 1u;
+                need--;
+            }
+        }
+        ties += __popc(tw);
+        uint32_t take = sw | take_t;
+        while (take) {
+            const int bit = __ffs(take) - 1;
+            if (pos < (uint32_t)k) out[pos] = (w << 5) + bit;
+            pos++;
+            take &= take - 1;
+        }
+    }
+    return true;
+}
+
 // STAGED: the query's row is first copied to shared memory as keys (16-byte loads, eight in
 // flight per thread) and every pass reads it from there.
 template <bool STAGED>
 __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
     const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ q_seq,
     const int32_t* __restrict__ q_pos, const int64_t* __restrict__ seq_len, int B, int m,
-    int max_n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ dev_status) {
+    int max_n, int k, int32_t* __restrict__ idx_out, int32_t* __restrict__ dev_status,
+    const uint32_t* __restrict__ gmax, int64_t ld_g, int cap) {
     using namespace sm100;
     __shared__ Shared sh;
     const int qq = blockIdx.x;
@@ -244,6 +461,14 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         return;
     }
     bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
+    if (gmax && ((n + 31) >> 5) >= k) {
+        // from the indexer's group maxima (see topk_by_groups); the full row below only if
+        // more than cap entries reach the bound
+        extern __shared__ uint4 dyn_g[];
+        if (topk_by_groups(s, vec, gmax + (int64_t)qq * ld_g, n, k, cap, out,
+                           reinterpret_cast<uint8_t*>(dyn_g), sh))
+            return;
+    }
     if (tid == 0) {
         sh.key_or = 0u;
         sh.key_and = 0xFFFFFFFFu;
@@ -959,21 +1184,38 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(
 
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
-                        int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream) {
+                        int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream,
+                        const uint32_t* gmax, int64_t ld_g) {
     if (Q == 0) return cudaSuccess;
     // rows of up to ~44K scores are staged in shared memory as keys (with the ~25 KB of
     // histogram and candidate space this stays under the 227 KB per-CTA limit)
     const size_t row_bytes = (size_t)((max_n + 3) / 4) * 16;
     const size_t word_bytes = (size_t)((2 * ((max_n + 31) / 32) + 3) / 4) * 16;
+    const bool staged = word_bytes + row_bytes <= (size_t)176 * 1024;
     cudaError_t e;
-    if (word_bytes + row_bytes <= (size_t)176 * 1024) {
+    // With the indexer's group maxima every row takes one CTA: the group path reads about
+    // k groups of the row; only a query whose bound admits more than cap entries falls back
+    // to its full row in the same CTA (staged in shared memory when it fits).
+    const int cap = 4 * k;
+    const size_t gbytes = group_smem_bytes(max_n, cap);
+    if (gmax && gbytes <= (size_t)176 * 1024) {
+        const size_t sm = std::max(staged ? word_bytes + row_bytes : word_bytes, gbytes);
+        auto kernel = staged ? topk_radix_kernel<true> : topk_radix_kernel<false>;
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        LaunchScope scope(kKTopk, stream);
+        return launch_pdl(kernel, dim3(Q), dim3(kThreads), sm, stream, scores, ld, q_seq, q_pos,
+                          seq_len, B, m, max_n, k, idx_out, st, gmax, ld_g, cap);
+    }
+    if (staged) {
         const size_t smem = word_bytes + row_bytes;
         e = cudaFuncSetAttribute(topk_radix_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         LaunchScope scope(kKTopk, stream);
         return launch_pdl(topk_radix_kernel<true>, dim3(Q), dim3(kThreads), smem, stream, scores,
-                          ld, q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st);
+                          ld, q_seq, q_pos, seq_len, B, m, max_n, k, idx_out, st,
+                          (const uint32_t*)nullptr, (int64_t)0, 0);
     }
     // long rows: a cluster of R CTAs per query, about kClusterSlice entries each (the
     // selected set is unique under the total order, so the split does not change it)
@@ -984,9 +1226,9 @@ cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
     const size_t cl_words = (size_t)((2 * wmax + 3) / 4) * 16;
     const size_t cl_row = (size_t)((slice_max + 3) / 4) * 16;
     static_assert(sizeof(ClShared) % 16 == 0, "the words follow the shared state");
-    const bool staged = sizeof(ClShared) + cl_words + cl_row <= (size_t)220 * 1024;
-    const size_t smem = sizeof(ClShared) + cl_words + (staged ? cl_row : 0);
-    auto kernel = staged ? topk_cluster_kernel<true> : topk_cluster_kernel<false>;
+    const bool cl_staged = sizeof(ClShared) + cl_words + cl_row <= (size_t)220 * 1024;
+    const size_t smem = sizeof(ClShared) + cl_words + (cl_staged ? cl_row : 0);
+    auto kernel = cl_staged ? topk_cluster_kernel<true> : topk_cluster_kernel<false>;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     LaunchScope scope(kKTopk, stream);

@@ -130,6 +130,29 @@ def test_sampled_bound_too_many_candidates_falls_back():
     assert np.array_equal(idx[0], np.arange(512))
 
 
+@pytest.mark.parametrize("hot", [2048, 8192])
+def test_group_bound_with_clustered_top_scores(hot):
+    # 60000 entries, top-1024: the `hot` first entries score highest, so the k largest group
+    # maxima come from few groups.  hot = 2048: about 3000 entries reach the bound (the
+    # group path); hot = 8192: more than its 4096-entry list, so the full row is used
+    wl = synth.make_workload("t", B=1, T=[240000], D=128, H=16, m=4, span=8, H_I=16,
+                             d_I=128, k=1024, seed=27, device=DEV)
+    ks = np.random.default_rng(8).uniform(1.0, 2.0, wl.kI.shape[0]).astype(np.float32)
+    ks[:hot] = 10.0 + np.random.default_rng(9).uniform(0.0, 1.0, hot).astype(np.float32)
+    _scores_from_scales(wl, ks)
+    idx = _exact(wl)
+    assert np.all(idx[0] < hot)
+
+
+def test_group_path_across_a_ragged_batch_bit_exact():
+    # long and short rows in one batch: rows of at least 32k entries select from the group
+    # maxima, the shorter ones from their full rows
+    wl = synth.make_workload("t", B=5, T=[400003, 8000, 250001, 160000, 1001], D=128, H=16,
+                             m=4, span=8, H_I=64, d_I=128, k=512, keep_raw=64, seed=30,
+                             device=DEV)
+    _exact(wl)
+
+
 def _abs_bound(wl, q):
     """fp32 rounding bound of one query's scores: the dot products accumulate 128 e4m3
     products in fp32 (error <= 2^-17 of the sum of |products| each, doubled for margin)
