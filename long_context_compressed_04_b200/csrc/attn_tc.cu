@@ -98,6 +98,9 @@ struct AttnTcArgs {
     int64_t ent_rows;
     int k, m, B, W, Q, chunk_tiles, chunks_per_q, total_items, max_n;
     int cluster;          // sparse: CTAs per query (one cluster); dense: 1
+    // dense only: 0 = the chunks of a query spread over CTAs, combined by
+    // attn_combine_kernel; 1 = one CTA takes all chunks of a query and combines them itself
+    int single;
     float scale_log2;
     float eps;
     double log2_theta;
@@ -169,6 +172,66 @@ __device__ __forceinline__ bool get_item(const AttnTcArgs& a, int it, AItem& x, 
         x.ntiles = min(a.chunk_tiles, 1 + n_et - x.tile0);
     }
     return x.ntiles > 0;
+}
+
+// The i-th item this CTA takes, or -1 past its last.  Spread (dense chunks and sparse
+// queries): items blockIdx.x, blockIdx.x + gridDim.x, ...  Single (dense): every chunk of
+// queries blockIdx.x, blockIdx.x + gridDim.x, ..., a query's chunks in order.
+__device__ __forceinline__ int item_id(const AttnTcArgs& a, int i) {
+    if (!a.single) {
+        const int it = (int)blockIdx.x + i * (int)gridDim.x;
+        return it < a.total_items ? it : -1;
+    }
+    const int q = (int)blockIdx.x + (i / a.chunks_per_q) * (int)gridDim.x;
+    return q < a.Q ? q * a.chunks_per_q + i % a.chunks_per_q : -1;
+}
+
+// Chunks of a dense query: the window chunk, then its entry tiles in chunks of
+// chunk_tiles (a function of the query's own visible entries).
+__device__ __forceinline__ int dense_chunks(const AttnTcArgs& a, int q, int& t) {
+    const int b = a.q_seq[q];
+    t = a.q_pos[q];
+    if (b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]) return 0;
+    int n = (t + 1) / a.m;
+    if (n > a.max_n) n = a.max_n;
+    const int64_t avail = a.ent_rows - a.ent_off[b];
+    if ((int64_t)n > avail) n = avail > 0 ? (int)avail : 0;
+    return 1 + ((n + kTK - 1) / kTK + a.chunk_tiles - 1) / a.chunk_tiles;
+}
+
+// The output of channels d, d + 1 (d even) of head h of dense query q at position t: the
+// nch chunk partials combined in chunk order with the sink first (M = max(sink, m_c),
+// w_c = 2^(m_c - M), L = 2^(sink - M) + sum_c w_c l_c, o = sum_c w_c O_c / L), then the
+// inverse RoPE on the last 64 channels.  Both dense variants combine with this function, so
+// a query's bits do not depend on which one ran.
+__device__ __forceinline__ float2 combine_pair(const AttnTcArgs& a, int q, int t, int nch,
+                                               int h, int d) {
+    const float* base = a.part + ((int64_t)q * a.chunks_per_q * kH + h) * (kD + 2);
+    const int64_t cstride = (int64_t)kH * (kD + 2);
+    const float sk = a.sink[h] * kLog2e;
+    float M = sk;
+    for (int c = 0; c < nch; c++) M = fmaxf(M, base[c * cstride]);
+    float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
+    float o0 = 0.f, o1 = 0.f;
+    for (int c = 0; c < nch; c++) {
+        const float* pc = base + c * cstride;
+        const float mc = pc[0];
+        const float w = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
+        L = fmaf(w, pc[1], L);
+        const float2 v = *reinterpret_cast<const float2*>(pc + 2 + d);
+        o0 = fmaf(w, v.x, o0);
+        o1 = fmaf(w, v.y, o1);
+    }
+    o0 = L > 0.f ? o0 / L : 0.f;
+    o1 = L > 0.f ? o1 / L : 0.f;
+    if (d >= kD - kRopeDims) {
+        float cs, sn;   // rotation by -t
+        rope_cos_sin(-(double)t, (d - (kD - kRopeDims)) >> 1, a.log2_theta, cs, sn);
+        const float x = o0, y = o1;
+        o0 = x * cs - y * sn;
+        o1 = x * sn + y * cs;
+    }
+    return make_float2(o0, o1);
 }
 
 // Byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-swizzled [rows x 128 B] block.
@@ -286,7 +349,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         int issued[kStages] = {};
         bool ok = true;
         bool waited = false;
-        for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
+        for (int ii = 0; ok; ii++) {
+            const int it = item_id(a, ii);
+            if (it < 0) break;
             AItem x;
             const bool have = get_item(a, it, x, false);
             if (have && !a.idx) {
@@ -434,7 +499,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ph = 0;
             int nt = 0, nitem = 0;
             bool ok = true;
-            for (int it = blockIdx.x; it < a.total_items && ok; it += gridDim.x) {
+            for (int ii = 0; ok; ii++) {
+                const int it = item_id(a, ii);
+                if (it < 0) break;
                 AItem x;
                 if (!get_item(a, it, x, false)) continue;
                 if (s_role) {
@@ -538,9 +605,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nt = 0, nitem = 0;
         int kst = 0;   // ring position of the next entry tile (mirrors the producer)
         bool ok = true;
-        for (int it = blockIdx.x; it < a.total_items; it += gridDim.x) {
+        // single dense variant: after the last chunk of each query, its combine (all 256
+        // threads, the query's partials written by this CTA before the barrier)
+        auto combine_here = [&](int it) {
+            if (!a.single || it % a.chunks_per_q != a.chunks_per_q - 1) return;
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            const int q = it / a.chunks_per_q;
+            int t;
+            const int nch = dense_chunks(a, q, t);
+            if (nch == 0) return;
+            if (!waited_prev) {
+                pdl_wait();
+                waited_prev = true;
+            }
+            for (int u = i; u < kH * (kD / 2); u += 256) {
+                const int hh = u / (kD / 2), d = 2 * (u % (kD / 2));
+                const float2 o = combine_pair(a, q, t, nch, hh, d);
+                *reinterpret_cast<uint32_t*>(a.out + ((int64_t)q * kH + hh) * kD + d) = pack_bf16x2(o.x, o.y);
+            }
+        };
+        for (int ii = 0;; ii++) {
+            const int it = item_id(a, ii);
+            if (it < 0) break;
             AItem x;
-            if (!get_item(a, it, x, i == 0)) continue;
+            if (!get_item(a, it, x, i == 0)) {
+                combine_here(it);
+                continue;
+            }
             // ---- item prologue: q heads and (chunk 0) the window tile ----
             // A failed wait in a warp only skips the rest of that item; here, once per item,
             // all 256 threads meet and leave together if any of them failed.
@@ -935,6 +1026,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<float2*>(pr + 2 + kh * 64 + c) = make_float2(o[c], o[c + 1]);
             }
             nitem++;
+            if (ok) combine_here(it);
         }
     }
 
@@ -948,47 +1040,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (a.cluster > 1) cluster_sync_all();
 }
 
-// Dense path: combine the chunk partials of one (query, head) in chunk order, add the
-// sink, normalise, inverse RoPE, store bf16.  Thread = channel.
-__global__ void __launch_bounds__(kD) attn_combine_kernel(const AttnTcArgs a) {
-    const int q = blockIdx.y, h = blockIdx.x, d = threadIdx.x;
-    // query metadata and the sink are inputs: read before the wait on the attention kernel
-    const int b = a.q_seq[q], t = a.q_pos[q];
-    const bool valid = !(b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]);
-    int nch = 0;
-    if (valid) {
-        int n = (t + 1) / a.m;
-        if (n > a.max_n) n = a.max_n;
-        const int64_t avail = a.ent_rows - a.ent_off[b];
-        if ((int64_t)n > avail) n = avail > 0 ? (int)avail : 0;
-        nch = 1 + ((n + kTK - 1) / kTK + a.chunk_tiles - 1) / a.chunk_tiles;
-    }
-    const float sk = a.sink[h] * kLog2e;
-    float cs = 1.f, sn = 0.f;   // inverse RoPE of the last 64 channels
-    if (valid && d >= kD - kRopeDims)
-        rope_cos_sin(-(double)t, (d - (kD - kRopeDims)) >> 1, a.log2_theta, cs, sn);
+// Dense path, spread variant: combine the chunk partials of one (query, head) (see
+// combine_pair).  Thread = pair of channels.
+__global__ void __launch_bounds__(kD / 2) attn_combine_kernel(const AttnTcArgs a) {
+    const int q = blockIdx.y, h = blockIdx.x, d = 2 * threadIdx.x;
+    // query metadata is an input: read before the wait on the attention kernel
+    int t;
+    const int nch = dense_chunks(a, q, t);
     pdl_wait();   // chunk partials come from the attention kernel
     pdl_trigger();
-    if (!valid) return;
-    const float* base = a.part + ((int64_t)q * a.chunks_per_q * kH + h) * (kD + 2);
-    const int64_t cstride = (int64_t)kH * (kD + 2);
-    float M = sk;
-#pragma unroll 8
-    for (int c = 0; c < nch; c++) M = fmaxf(M, base[c * cstride]);
-    float L = (M == -INFINITY || sk == -INFINITY) ? 0.f : exp2f(sk - M);
-    float o = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < nch; c++) {
-        const float* pc = base + c * cstride;
-        const float mc = pc[0];
-        const float w = (mc == -INFINITY) ? 0.f : exp2f(mc - M);
-        L = fmaf(w, pc[1], L);
-        o = fmaf(w, pc[2 + d], o);
-    }
-    o = L > 0.f ? o / L : 0.f;
-    const float other = __shfl_xor_sync(0xffffffffu, o, 1);
-    if (d >= kD - kRopeDims) o = (d & 1) ? (other * sn + o * cs) : (o * cs - other * sn);
-    a.out[((int64_t)q * kH + h) * kD + d] = (uint16_t)f32_to_bf16_bits(o);
+    if (nch == 0) return;
+    const float2 o = combine_pair(a, q, t, nch, h, d);
+    *reinterpret_cast<uint32_t*>(a.out + ((int64_t)q * kH + h) * kD + d) = pack_bf16x2(o.x, o.y);
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1115,6 +1178,11 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
         a.chunk_tiles = kDenseChunkTiles;
         a.chunks_per_q = dense_chunks_per_q(max_n);
     }
+    // dense: the query's chunks spread over CTAs (low latency while the chunks of the batch
+    // leave SMs idle otherwise), or one CTA per query from as many queries as SMs on (high
+    // throughput: no combine kernel, each query's partials stay with its CTA).  Both give the
+    // same bits, so the choice may follow the batch.
+    a.single = (!aa.idx && Q >= sm_count()) ? 1 : 0;
     a.total_items = Q * a.chunks_per_q;
     // dense: 128-row boxes of contiguous entries; sparse: one-row boxes for 4-row gathers
     CUtensorMap map_e, map_g;
@@ -1145,14 +1213,14 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
             e = launch_pdl_cluster(attn_tc_kernel, dim3(nclusters * a.cluster), dim3(kThreads),
                                    kSmemBytes, stream, a.cluster, map_e, map_g, a);
         } else {
-            const int grid = min(a.total_items, sm_count());
+            const int grid = min(a.single ? Q : a.total_items, sm_count());
             e = launch_pdl(attn_tc_kernel, dim3(grid), dim3(kThreads), kSmemBytes, stream, map_e,
                            map_g, a);
         }
     }
-    if (e != cudaSuccess || aa.idx) return e;
+    if (e != cudaSuccess || aa.idx || a.single) return e;
     LaunchScope scope(kKAttnCombine, stream);
-    return launch_pdl(attn_combine_kernel, dim3(kH, Q), dim3(kD), 0, stream, a);
+    return launch_pdl(attn_combine_kernel, dim3(kH, Q), dim3(kD / 2), 0, stream, a);
 }
 
 }  // namespace csa

@@ -8,6 +8,7 @@ import pytest
 import torch
 
 import _orc
+import long_context_compressed_04_b200 as L
 from long_context_compressed_04_b200 import CSA_DEV_OOB, pipeline, synth
 
 pytestmark = pytest.mark.gpu
@@ -231,3 +232,37 @@ def test_rising_scores_move_the_reference_maximum(mode, H, D, fmt):
     assert mag > 4.0                     # the scaled entries dominate the output
     assert np.abs(a - b).max() <= mag * 2.0 ** -6
     assert np.linalg.norm(a - b) <= 5e-3 * np.linalg.norm(b)
+
+
+def test_dense_dual_kernels_bitwise_equal():
+    # HCA dense attention runs in one of two variants chosen by the batch: small batches
+    # spread each query's chunks over CTAs and combine them in a second kernel; batches of
+    # at least as many queries as SMs give each query one CTA that combines its own chunks.
+    # The chunks and the combine arithmetic are the same, so a query's output must be
+    # bitwise the same in both; the variant is seen in the number of launches (2 vs 1).
+    g = torch.Generator().manual_seed(17)
+    lens = [int(x) for x in torch.randint(128 * 8, 128 * 1500, (160,), generator=g)]
+    base = synth.make_workload("t", B=160, T=lens, D=128, H=64, m=128, span=128,
+                               keep_raw=256, seed=38, device=DEV)
+    parts = synth.split(base)
+    gd = torch.Generator(device=DEV).manual_seed(19)
+    rows = [synth.random_entries(int(p.n_ent[0]), 0, 128, gd, DEV) for p in parts]
+
+    def run(order):
+        wl = synth.merge([parts[i] for i in order])
+        buf = pipeline.alloc(wl, DEV)
+        for slot, i in enumerate(order):
+            e0 = int(wl.ent_off[slot])
+            buf.entries[e0:e0 + rows[i].shape[0]].copy_(rows[i])
+        n0 = L.csa_launch_count()
+        pipeline.attend(wl, buf)
+        torch.cuda.synchronize()
+        assert int(buf.dev_status.item()) == 0
+        return buf.out, L.csa_launch_count() - n0
+
+    big, n_big = run(list(range(160)))
+    assert n_big == 1
+    for tgt in (0, 77, 159):
+        small, n_small = run([tgt])
+        assert n_small == 2
+        assert torch.equal(small[0].view(torch.int16), big[tgt].view(torch.int16))
