@@ -48,15 +48,16 @@ WORKLOADS = {
 }
 
 
-# DRAM traffic (read + write, bytes per launch) from the ncu capture summarised in
-# profiles/csa_decode_128k_b32_kernels_ncu.md, valid only while the kernel's sources are
-# byte-identical to the ones captured (sha256 of the files, first 16 hex digits).
+# DRAM traffic (read + write, bytes per launch) of the dominant kernel from the ncu capture
+# summarised in profiles/csa_decode_1m_b8_fp8_launch_list.md, valid only while the kernel's
+# sources are byte-identical to the ones captured (sha256 of the files, first 16 hex digits).
 MEASURED_TRAFFIC = {
-    ("csa_decode_128k_b32", "indexer_score_tc"): {
-        "bytes": 144_134_912,
+    ("csa_decode_1m_b8_fp8", "indexer_score_tc"): {
+        "bytes": 285_380_352,
         "files": ["long_context_compressed_04_b200/csrc/indexer_tc.cu",
-                  "long_context_compressed_04_b200/csrc/sm100.cuh"],
-        "sha": "03dc463c2890a225",
+                  "long_context_compressed_04_b200/csrc/sm100.cuh",
+                  "long_context_compressed_04_b200/csrc/common.cuh"],
+        "sha": "966246eaff27f9b4",
     },
 }
 
@@ -114,7 +115,7 @@ def whole_job_rate(units_per_rank: int, world: int, steps: int, ms: float) -> fl
     return units_per_rank * world * steps / (ms / 1e3)
 
 
-def make_workload(name: str, rank: int, device):
+def make_workload(name: str, rank: int, device, keep_raw=None):
     from long_context_compressed_04_b200 import synth
     c = WORKLOADS[name]
     if c["kind"] == "csa_prefill":
@@ -126,9 +127,9 @@ def make_workload(name: str, rank: int, device):
     if c["kind"] == "csa":
         return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
                                    fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
-                                   indexer="fp8", seed=rank, device=device)
+                                   indexer="fp8", keep_raw=keep_raw, seed=rank, device=device)
     return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=128, span=128, W=128,
-                               fmt=c["fmt"], seed=rank, device=device)
+                               fmt=c["fmt"], keep_raw=keep_raw, seed=rank, device=device)
 
 
 def new_tokens(wl, name):
@@ -390,13 +391,21 @@ def measure(name: str, args, dist, dev, rank: int, world: int, full: bool):
     import long_context_compressed_04_b200 as L
     from long_context_compressed_04_b200 import pipeline
 
-    wl = make_workload(name, rank, dev)
+    raw_tail = getattr(args, "raw_tail", False) and WORKLOADS[name]["kind"] != "csa_prefill"
+    wl = make_workload(name, rank, dev, keep_raw=256 if raw_tail else None)
     buf = pipeline.alloc(wl, dev)
-    all_seq, all_ent = pipeline.all_entry_items(wl, dev)
-    pipeline.compress(wl, buf, all_seq, all_ent)          # build the compressed cache
+    if raw_tail:
+        # the raw store keeps each sequence's last 256 tokens (the window and the newest
+        # block); the compressed cache before the step is drawn as stored-format rows
+        from long_context_compressed_04_b200 import synth
+        g = torch.Generator(device=dev).manual_seed(1000 + rank)
+        buf.entries.copy_(synth.random_entries(buf.entries.shape[0], wl.fmt, wl.D, g, dev))
+    else:
+        all_seq, all_ent = pipeline.all_entry_items(wl, dev)
+        pipeline.compress(wl, buf, all_seq, all_ent)      # build the compressed cache
+        del all_seq, all_ent
     new_seq, new_ent = step_items(wl, name, dev)
     torch.cuda.synchronize()
-    del all_seq, all_ent
 
     def step_eager(b=buf, w=wl):
         pipeline.step(w, b, new_seq, new_ent)
@@ -522,6 +531,8 @@ def measure(name: str, args, dist, dev, rank: int, world: int, full: bool):
     out = {
         "value": value, "ms_per_step": ms_max / K,
         "config": {"workload": name, **WORKLOADS[name], "queries_per_gpu": wl.Q,
+                   **({"cache": "stored rows drawn directly; raw store keeps the last 256 tokens"}
+                      if raw_tail else {}),
                    "l2": "flushed before every timed step (256 MB write, then 256 MB read)",
                    "indexer_inputs": "fp8 e4m3 N(0,1), 1x128 scales"},
         "roofline": roof,
@@ -655,6 +666,10 @@ def main():
     ap.add_argument("--no-also", action="store_true",
                     help="measure only --workload (not the other decode workloads)")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of a CUDA graph")
+    ap.add_argument("--raw-tail", action="store_true",
+                    help="keep only each sequence's last 256 raw tokens and draw the compressed "
+                         "cache as stored rows (the same step, a few GB on the device; for "
+                         "profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
