@@ -137,8 +137,11 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
  *   idx_out int32 [Q, k]
  *   scores_out: nullable fp32 [Q, ld_scores] receiving s_i for i < n_vis (ld_scores >= max_n)
  *   workspace: device buffer of at least csa_indexer_workspace_size(Q, max_n, k) bytes,
- *   256-byte aligned; contents on entry are ignored.  It holds only the score rows, so it
- *   may be NULL (with workspace_bytes 0) when scores_out is given.
+ *   256-byte aligned; contents on entry are ignored.  It holds the largest score of every
+ *   32 consecutive entries of every query (which the selection starts from), then the score
+ *   rows.  With scores_out given the score rows go there: the workspace may then be just
+ *   large enough for the first part (ceil(Q * ceil(max_n / 32) * 4 / 256) * 256 bytes), or
+ *   NULL (with workspace_bytes 0), in which case the selection reads the full score rows.
  * kI and qI must be 16-byte aligned.  Errors as above; CSA_DEV_NAN, CSA_DEV_CAPACITY.
  */
 size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k);
@@ -214,7 +217,7 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int
  *   CSA_NOALLOC_SCRATCH_BYTES bytes; it allocates nothing.
  *   - A call needing more than that (csa_indexer_workspace_size(Q, max_n, k) > the size)
  *     returns CSA_ERR_WORKSPACE with a message and launches nothing.  16 MiB covers, e.g.,
- *     32 queries of up to 131040 visible entries.  With scores_out given, the scores are
+ *     32 queries of up to 127072 visible entries.  With scores_out given, the scores are
  *     written there, the array is not used and there is no such limit.
  *   - Every GPU that loads the library holds the array until the process exits.
  *   - All calls on a device share the array, which keeps the last call's contents;
