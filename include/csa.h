@@ -156,6 +156,30 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
                                     int32_t* dev_status, void* stream);
 
 /*
+ * csa_topk_merge -- the top-k of a sequence from the top-k of its slices (context-parallel
+ * decode; the stuffyNLP post's context parallelism applied to the selection of
+ * "DeepSeek-V4 深度分析报告" 2.1 CSA).
+ *   A sequence's entries are split into contiguous slices (say one per GPU), and each
+ *   slice's top-k is selected with lightning_indexer_topk (with scores_out).  Since the
+ *   order within a slice is the order of the whole sequence, every entry of the sequence's
+ *   top-k is in its slice's top-k, and this call selects the sequence's top-k from the
+ *   slices' candidates, with the same order (larger score first, lower entry index first
+ *   among equal scores, -0 = +0) and the same output (ascending entry order, -1 padded)
+ *   as lightning_indexer_topk over the whole sequence.
+ * Arguments:
+ *   cand_scores fp32 [Q, n_cand], cand_idx int32 [Q, n_cand]: per query, the slices'
+ *     index sets translated to entry indices of the whole sequence (-1 = no candidate) and
+ *     the scores of those entries, slices in ascending entry order, each slice's set
+ *     ascending -- so the candidates are in ascending entry order.  1 <= n_cand <= 16384.
+ *   k in 1..2048; idx_out int32 [Q, k].
+ * Errors: CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA; a NaN score sets
+ * CSA_DEV_NAN.
+ */
+csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx, int32_t Q,
+                            int32_t n_cand, int32_t k, int32_t* idx_out, int32_t* dev_status,
+                            void* stream);
+
+/*
  * sparse_mqa_attn -- CSA shared-KV MQA over the selected entries and the window (a5).
  *   "DeepSeek-V4 深度分析报告" 2.1 CSA (top-k entries plus a 128-token sliding window);
  *   "其他注意力技术细节": Shared Key-Value MQA (an entry is both key and value, all heads

@@ -4,7 +4,7 @@ Argument marshalling only: every function here passes tensor pointers, sizes and
 current CUDA stream to the C ABI of ``libcsa.so`` (declared in ``include/csa.h``) and raises
 ``CSAError`` when it returns a non-zero status.  All computation happens in the CUDA
 kernels.  There is no CPU fallback: importing this package fails if ``libcsa.so`` has not
-been built (``python -m long_context_compressed_04_b200.build``).
+been built (``python long_context_compressed_04_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -35,7 +35,7 @@ class CSAError(RuntimeError):
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m long_context_compressed_04_b200.build` (needs nvcc)")
+                      "`python long_context_compressed_04_b200/build.py` (needs nvcc)")
 
 _lib = ctypes.CDLL(LIB_PATH)
 _P, _I32, _I64, _F32, _SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
@@ -67,6 +67,7 @@ _SIGS = {
     "csa_profile_enable": (None, [ctypes.c_int]),
     "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
     "csa_debug_set_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
+    "csa_topk_merge": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -181,6 +182,13 @@ def lightning_indexer_topk_noalloc(qI, qI_scale, w, kI, kI_scale, seq_len, ent_o
         _p(ent_off), _p(q_seq),
         _p(q_pos), q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out),
         ld_scores, _p(dev_status), _s(stream)))
+
+
+def csa_topk_merge(cand_scores, cand_idx, idx_out, *, dev_status=None, stream=None):
+    """Top-k of sequences from their slices' candidates (see include/csa.h)."""
+    Q, n_cand = cand_idx.shape
+    _check(_lib.csa_topk_merge(_p(cand_scores), _p(cand_idx), Q, n_cand, idx_out.shape[1],
+                               _p(idx_out), _p(dev_status), _s(stream)))
 
 
 def sparse_mqa_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos, idx, sink,

@@ -212,6 +212,20 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     return cuda_status(e, "top-k launch");
 }
 
+csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx, int32_t Q,
+                            int32_t n_cand, int32_t k, int32_t* idx_out, int32_t* dev_status,
+                            void* stream) {
+    REQUIRE(Q >= 0, "Q must be >= 0");
+    if (Q == 0) return ok();
+    REQUIRE(cand_scores && cand_idx && idx_out, "null pointer argument");
+    SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
+    SUPPORT(csa::topk_merge_supported(n_cand, k),
+            "n_cand = %d not supported (1..16384 candidates per query)", n_cand);
+    return cuda_status(csa::launch_topk_merge(cand_scores, cand_idx, Q, n_cand, k, idx_out,
+                                              dev_status, (cudaStream_t)stream),
+                       "top-k merge launch");
+}
+
 static csa_status_t attn_validate(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,
                                   const int64_t* seq_len, const int64_t* ent_off, const void* kv, const int64_t* kv_off,
                                   const int64_t* kv_pos0, const int32_t* q_seq,

@@ -55,6 +55,7 @@ enum KernelKind {
     kKAttnTc,
     kKAttnCombine,
     kKAttn576Tc,
+    kKTopkMerge,
     kKernelKinds
 };
 
@@ -122,6 +123,11 @@ cudaError_t launch_attn576_tc(const AttnArgs& a, int Q, cudaStream_t stream);
 size_t attn_tc_workspace_bytes(int Q, int max_n);
 cudaError_t launch_attn_tc(const AttnArgs& a, int Q, int max_n, void* workspace,
                            cudaStream_t stream);
+
+bool topk_merge_supported(int n_cand, int k);
+cudaError_t launch_topk_merge(const float* cand_scores, const int32_t* cand_idx, int Q,
+                              int n_cand, int k, int32_t* idx_out, int32_t* st,
+                              cudaStream_t stream);
 
 // Sets the thread-local message csa_last_error() returns (printf-style).
 void set_error_message(const char* fmt, ...);

@@ -51,7 +51,7 @@ cudaEvent_t take_event() {
 const char* kernel_name(int kind) {
     static const char* names[kKernelKinds] = {"compress", "indexer_score_simt", "topk_radix",
                                               "attn_simt", "indexer_score_tc", "attn_tc",
-                                              "attn_combine", "attn576_tc"};
+                                              "attn_combine", "attn576_tc", "topk_merge"};
     return (kind >= 0 && kind < kKernelKinds) ? names[kind] : "?";
 }
 
