@@ -655,6 +655,102 @@ def measure_e2e(name, wl, buf, new_seq, new_ent, args, dist, dev, world, flush_l
                    f"double-buffered; {E} pipelined steps per captured graph, {R} replays"}
 
 
+def measure_cp(world: int, args, dev):
+    """Context-parallel decode of the headline workload, its W ranks' slices on this one GPU
+    (long_context_compressed_04_b200.cp).  On W GPUs the slices' selections run at once, so
+    each part is timed on its own, from a CUDA graph, with L2 flushed before it: every
+    rank's selection (the slowest is the step's share), the merge, every rank's row pack and
+    the attention over the gathered rows.  The two exchanges run here as stand-ins (a copy
+    and a sum) outside the timed parts; their bytes per rank are reported, with the time
+    they take at the measured peer bandwidth (770 GB/s per direction), launch latency not
+    included.  The cache is drawn as stored rows (the raw store keeps the last 256 tokens)."""
+    from long_context_compressed_04_b200 import cp, pipeline, synth
+    name = DEFAULT_WORKLOAD
+    wl = make_workload(name, 0, dev, keep_raw=256)
+    g = torch.Generator(device=dev).manual_seed(1000)
+    rows = synth.random_entries(wl.ent_rows, wl.fmt, wl.D, g, dev)
+    ent_off = wl.ent_off.cpu()
+    ranks = []
+    for r in range(world):
+        kI, ks, ents, off, base = [], [], [], [], 0
+        for b in range(wl.B):
+            lo, hi = cp.slice_bounds(int(wl.n_ent[b]), world, r)
+            r0 = int(ent_off[b])
+            kI.append(wl.kI[r0 + lo:r0 + hi])
+            ks.append(wl.ks[r0 + lo:r0 + hi])
+            ents.append(rows[r0 + lo:r0 + hi])
+            off.append(base)
+            base += hi - lo
+        sl = cp.make_slice(wl, world, r, torch.tensor(off, dtype=torch.int64))
+        ranks.append((sl, torch.cat(kI).contiguous(), torch.cat(ks).contiguous(),
+                      torch.cat(ents).contiguous(), cp.alloc(wl, sl, world, dev)))
+    one = pipeline.alloc(wl, dev)
+    one.entries.copy_(rows)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def graph(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        return gr
+
+    reps = max(args.steps, 10)
+
+    def timed(gr):
+        ts = []
+        for _ in range(reps):
+            flush.zero_()          # still running when the graph is launched behind it
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            gr.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(ts)
+
+    sel_g = [graph(lambda sl=sl, kI=kI, ks=ks, buf=buf: cp.select_local(wl, sl, kI, ks, buf))
+             for sl, kI, ks, _e, buf in ranks]
+    sel_us = [timed(gr) for gr in sel_g]
+    cands = torch.stack([buf.cand for *_x, buf in ranks])
+    for *_x, buf in ranks:
+        cp.exchange_candidates(buf, all_gather=lambda out, inp: out.copy_(cands))
+    buf0 = ranks[0][4]
+    merge_us = timed(graph(lambda: cp.merge(wl, buf0)))
+    for *_x, buf in ranks[1:]:
+        buf.idx.copy_(buf0.idx)
+    pack_us = [timed(graph(lambda sl=sl, ents=ents, buf=buf: cp.pack(wl, sl, ents, buf)))
+               for sl, _k, _s, ents, buf in ranks]
+    total = torch.stack([buf.packed.view(torch.int32) for *_x, buf in ranks]).sum(
+        0, dtype=torch.int32)
+    cp.exchange_rows(buf0, all_reduce=lambda t: t.copy_(total))
+    attn_us = timed(graph(lambda: cp.attend(wl, buf0)))
+    one_sel_us = timed(graph(lambda: pipeline.indexer_topk(wl, one)))
+    one_attn_us = timed(graph(lambda: pipeline.attend(wl, one)))
+    torch.cuda.synchronize()
+    ok = (all(int(buf.dev_status.item()) == 0 for *_x, buf in ranks)
+          and int(one.dev_status.item()) == 0)
+    same = bool(torch.equal(one.idx, buf0.idx)) and bool(
+        torch.equal(one.out.view(torch.int16), buf0.out.view(torch.int16)))
+    cand_b, rows_b = cp.exchange_bytes(wl, world)
+    # all_gather: each rank receives (W - 1) buffers; ring all_reduce: 2 (W - 1) / W x size
+    xfer = (world - 1) * cand_b + 2 * (world - 1) / world * rows_b
+    xfer_us = xfer / 770e9 * 1e6
+    step_us = max(sel_us) + merge_us + max(pack_us) + attn_us
+    return {"mode": "context-parallel, the ranks' parts timed in turn on one GPU",
+            "workload": name, "world": world,
+            "slice_select_us": [round(x, 1) for x in sel_us], "merge_us": round(merge_us, 1),
+            "pack_us": [round(x, 1) for x in pack_us], "attention_us": round(attn_us, 1),
+            "rank_compute_us": round(step_us, 1),
+            "exchange_bytes_in_per_rank": int(xfer), "exchange_us_at_770GBps": round(xfer_us, 1),
+            "one_gpu_select_us": round(one_sel_us, 1), "one_gpu_attention_us": round(one_attn_us, 1),
+            "bitwise_equal_one_gpu": same, "dev_status_clean": ok,
+            "timing": f"median of {reps} graph replays, each behind a 256 MB L2 flush, "
+                      "CUDA events"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -670,10 +766,17 @@ def main():
                     help="keep only each sequence's last 256 raw tokens and draw the compressed "
                          "cache as stored rows (the same step, a few GB on the device; for "
                          "profiling)")
+    ap.add_argument("--cp", type=int, default=0,
+                    help="time context-parallel decode of the headline workload over this many "
+                         "slices, the ranks in turn on one GPU (a separate JSON line)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         return run_reference(args)
+    if args.cp:
+        torch.cuda.set_device(0)
+        print(json.dumps(measure_cp(args.cp, args, torch.device("cuda", 0))), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -156,28 +156,66 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
                                     int32_t* dev_status, void* stream);
 
 /*
- * csa_topk_merge -- the top-k of a sequence from the top-k of its slices (context-parallel
- * decode; the stuffyNLP post's context parallelism applied to the selection of
- * "DeepSeek-V4 深度分析报告" 2.1 CSA).
- *   A sequence's entries are split into contiguous slices (say one per GPU), and each
- *   slice's top-k is selected with lightning_indexer_topk (with scores_out).  Since the
- *   order within a slice is the order of the whole sequence, every entry of the sequence's
- *   top-k is in its slice's top-k, and this call selects the sequence's top-k from the
- *   slices' candidates, with the same order (larger score first, lower entry index first
- *   among equal scores, -0 = +0) and the same output (ascending entry order, -1 padded)
- *   as lightning_indexer_topk over the whole sequence.
- * Arguments:
- *   cand_scores fp32 [Q, n_cand], cand_idx int32 [Q, n_cand]: per query, the slices'
- *     index sets translated to entry indices of the whole sequence (-1 = no candidate) and
- *     the scores of those entries, slices in ascending entry order, each slice's set
- *     ascending -- so the candidates are in ascending entry order.  1 <= n_cand <= 16384.
+ * Context-parallel decode (the stuffyNLP post's context parallelism applied to the
+ * selection and attention of "DeepSeek-V4 深度分析报告" 2.1 CSA).  A sequence's entries
+ * are split into W contiguous slices (say one per GPU, slice r on rank r, slices in
+ * ascending entry order), and a rank holds the key and entry rows of its slice only.  One
+ * decode step: each rank selects its slice's top-k with lightning_indexer_topk (with
+ * scores_out), csa_cp_candidates turns that into candidates, the ranks' candidates are
+ * gathered (slice-major), csa_topk_merge selects the sequence's top-k from them,
+ * csa_cp_pack_rows writes the selected rows this rank holds, an integer sum over the
+ * ranks' packed buffers gathers every selected row, and sparse_mqa_attn runs over them.
+ * Since the order within a slice is the order of the whole sequence, every entry of the
+ * sequence's top-k is in its slice's top-k; the merge uses the order of the selection
+ * (larger score first, lower entry index first among equal scores, -0 = +0) and writes the
+ * same output (ascending entry order, -1 padded), so the index set is bit for bit the one
+ * lightning_indexer_topk selects over the whole sequence.
+ *
+ * csa_cp_candidates -- a slice's selection as candidates of the whole sequence.
+ *   idx int32 [Q, k]: lightning_indexer_topk's output over the slice (indices within the
+ *   slice, -1 padded); scores fp32 [Q, ld_scores]: its scores_out rows; q_seq int32 [Q];
+ *   slice_lo int64 [B]: the slice's first entry of each sequence.  Writes cand_idx int32
+ *   [Q, k] = idx + slice_lo[q_seq] (-1 kept) and cand_scores fp32 [Q, k] = the entry's
+ *   score (0 for -1).  An index >= ld_scores, a sum above INT32_MAX or a q_seq outside
+ *   0..B-1 sets CSA_DEV_OOB and gives -1.
+ *
+ * csa_topk_merge -- the sequence's top-k from the W slices' candidates.
+ *   cand_scores fp32, cand_idx int32: candidate j of slice r for query q at element
+ *     r * slice_stride + q * k_in + j (so [W, Q, k_in] with slice_stride = Q * k_in, the
+ *     layout a gather of every rank's [Q, k_in] gives), slices in ascending entry order,
+ *     each slice's set ascending (as csa_cp_candidates writes them) -- so the candidates
+ *     are in ascending entry order.  -1 = no candidate.  1 <= W * k_in <= 16384.
  *   k in 1..2048; idx_out int32 [Q, k].
- * Errors: CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA; a NaN score sets
- * CSA_DEV_NAN.
+ *   A NaN score sets CSA_DEV_NAN.
+ *
+ * csa_cp_pack_rows -- the selected rows this rank holds, at their output positions.
+ *   idx int32 [Q, k]: the merged selection (entry indices of the whole sequence); q_seq
+ *   int32 [Q]; slice_lo, slice_n int64 [B]: this rank's slice of each sequence (entries
+ *   slice_lo .. slice_lo + slice_n - 1); ent_off int64 [B]: where each sequence's slice
+ *   starts in `entries` (this rank's store, ent_rows rows of row_bytes bytes, as
+ *   csa_entry_row_bytes gives; row_bytes a multiple of 16).  Writes out uint8 [Q, k,
+ *   row_bytes]: row (q, j) is the entry row of idx[q, j] if this rank's slice holds it, else
+ *   zeros.  Every position has exactly one rank with its row, so the element-wise integer
+ *   sum of the W ranks' buffers (say NCCL all_reduce on an int32 view) is the gathered
+ *   [Q * k, row_bytes] store that sparse_mqa_attn reads with entry indices 0..k-1 of query
+ *   q at rows q * k ... (ent_off = q * k for one query per sequence).  local_idx
+ *   (nullable) int32 [Q, k] receives those indices: j where idx[q, j] >= 0, else -1.  A
+ *   row outside 0..ent_rows-1 sets CSA_DEV_OOB and is written as zeros.  entries and out
+ *   16-byte aligned.
+ * Errors (all three): CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_CUDA.
  */
-csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx, int32_t Q,
-                            int32_t n_cand, int32_t k, int32_t* idx_out, int32_t* dev_status,
-                            void* stream);
+csa_status_t csa_cp_candidates(const int32_t* idx, const float* scores, int64_t ld_scores,
+                               const int32_t* q_seq, const int64_t* slice_lo, int32_t Q,
+                               int32_t B, int32_t k, int32_t* cand_idx, float* cand_scores,
+                               int32_t* dev_status, void* stream);
+csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx,
+                            int64_t slice_stride, int32_t W, int32_t Q, int32_t k_in, int32_t k,
+                            int32_t* idx_out, int32_t* dev_status, void* stream);
+csa_status_t csa_cp_pack_rows(const int32_t* idx, const int32_t* q_seq, const int64_t* slice_lo,
+                              const int64_t* slice_n, const int64_t* ent_off,
+                              const uint8_t* entries, int64_t ent_rows, int32_t row_bytes,
+                              int32_t Q, int32_t B, int32_t k, uint8_t* out,
+                              int32_t* local_idx, int32_t* dev_status, void* stream);
 
 /*
  * sparse_mqa_attn -- CSA shared-KV MQA over the selected entries and the window (a5).

@@ -67,7 +67,11 @@ _SIGS = {
     "csa_profile_enable": (None, [ctypes.c_int]),
     "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
     "csa_debug_set_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
-    "csa_topk_merge": (ctypes.c_int, [_P, _P, _I32, _I32, _I32, _P, _P, _P]),
+    "csa_topk_merge": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
+    "csa_cp_candidates": (ctypes.c_int, [_P, _P, _I64, _P, _P, _I32, _I32, _I32, _P, _P, _P,
+                                         _P]),
+    "csa_cp_pack_rows": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32, _I32,
+                                        _P, _P, _P, _P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -185,10 +189,30 @@ def lightning_indexer_topk_noalloc(qI, qI_scale, w, kI, kI_scale, seq_len, ent_o
 
 
 def csa_topk_merge(cand_scores, cand_idx, idx_out, *, dev_status=None, stream=None):
-    """Top-k of sequences from their slices' candidates (see include/csa.h)."""
-    Q, n_cand = cand_idx.shape
-    _check(_lib.csa_topk_merge(_p(cand_scores), _p(cand_idx), Q, n_cand, idx_out.shape[1],
-                               _p(idx_out), _p(dev_status), _s(stream)))
+    """Top-k of sequences from their slices' candidates, [W, Q, k_in] (see include/csa.h)."""
+    W, Q, k_in = cand_idx.shape
+    assert cand_scores.shape == cand_idx.shape
+    assert cand_idx.stride() == cand_scores.stride() and cand_idx.stride()[1:] == (k_in, 1)
+    _check(_lib.csa_topk_merge(_p(cand_scores), _p(cand_idx), cand_idx.stride(0), W, Q, k_in,
+                               idx_out.shape[1], _p(idx_out), _p(dev_status), _s(stream)))
+
+
+def csa_cp_candidates(idx, scores, q_seq, slice_lo, cand_idx, cand_scores, *, B: int,
+                      dev_status=None, stream=None):
+    """A slice's selection as candidates of the whole sequence (see include/csa.h)."""
+    Q, k = idx.shape
+    _check(_lib.csa_cp_candidates(_p(idx), _p(scores), scores.stride(0), _p(q_seq),
+                                  _p(slice_lo), Q, B, k, _p(cand_idx), _p(cand_scores),
+                                  _p(dev_status), _s(stream)))
+
+
+def csa_cp_pack_rows(idx, q_seq, slice_lo, slice_n, ent_off, entries, out, local_idx=None, *,
+                     B: int, dev_status=None, stream=None):
+    """The selected rows this rank's slice holds, at their positions (see include/csa.h)."""
+    Q, k = idx.shape
+    _check(_lib.csa_cp_pack_rows(_p(idx), _p(q_seq), _p(slice_lo), _p(slice_n), _p(ent_off),
+                                 _p(entries), entries.shape[0], entries.shape[1], Q, B, k,
+                                 _p(out), _p(local_idx), _p(dev_status), _s(stream)))
 
 
 def sparse_mqa_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos, idx, sink,

@@ -212,18 +212,55 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     return cuda_status(e, "top-k launch");
 }
 
-csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx, int32_t Q,
-                            int32_t n_cand, int32_t k, int32_t* idx_out, int32_t* dev_status,
-                            void* stream) {
+csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx,
+                            int64_t slice_stride, int32_t W, int32_t Q, int32_t k_in, int32_t k,
+                            int32_t* idx_out, int32_t* dev_status, void* stream) {
     REQUIRE(Q >= 0, "Q must be >= 0");
     if (Q == 0) return ok();
     REQUIRE(cand_scores && cand_idx && idx_out, "null pointer argument");
+    REQUIRE(W >= 1 && k_in >= 1, "W and k_in must be >= 1");
+    REQUIRE(W == 1 || slice_stride >= (int64_t)Q * k_in,
+            "slice_stride %lld < Q * k_in", (long long)slice_stride);
     SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
-    SUPPORT(csa::topk_merge_supported(n_cand, k),
-            "n_cand = %d not supported (1..16384 candidates per query)", n_cand);
-    return cuda_status(csa::launch_topk_merge(cand_scores, cand_idx, Q, n_cand, k, idx_out,
-                                              dev_status, (cudaStream_t)stream),
+    SUPPORT((int64_t)W * k_in <= (1 << 30) && csa::topk_merge_supported(W * k_in, k),
+            "W * k_in = %lld not supported (1..16384 candidates per query)",
+            (long long)W * k_in);
+    return cuda_status(csa::launch_topk_merge(cand_scores, cand_idx, slice_stride, W, Q, k_in,
+                                              k, idx_out, dev_status, (cudaStream_t)stream),
                        "top-k merge launch");
+}
+
+csa_status_t csa_cp_candidates(const int32_t* idx, const float* scores, int64_t ld_scores,
+                               const int32_t* q_seq, const int64_t* slice_lo, int32_t Q,
+                               int32_t B, int32_t k, int32_t* cand_idx, float* cand_scores,
+                               int32_t* dev_status, void* stream) {
+    REQUIRE(Q >= 0 && k >= 1 && B >= 1, "need Q >= 0, k >= 1, B >= 1");
+    if (Q == 0) return ok();
+    REQUIRE(idx && scores && q_seq && slice_lo && cand_idx && cand_scores,
+            "null pointer argument");
+    REQUIRE(ld_scores >= 1, "ld_scores must be >= 1");
+    return cuda_status(csa::launch_cp_candidates(idx, scores, ld_scores, q_seq, slice_lo, Q, B,
+                                                 k, cand_idx, cand_scores, dev_status,
+                                                 (cudaStream_t)stream),
+                       "candidate launch");
+}
+
+csa_status_t csa_cp_pack_rows(const int32_t* idx, const int32_t* q_seq, const int64_t* slice_lo,
+                              const int64_t* slice_n, const int64_t* ent_off,
+                              const uint8_t* entries, int64_t ent_rows, int32_t row_bytes,
+                              int32_t Q, int32_t B, int32_t k, uint8_t* out,
+                              int32_t* local_idx, int32_t* dev_status, void* stream) {
+    REQUIRE(Q >= 0 && k >= 1 && B >= 1, "need Q >= 0, k >= 1, B >= 1");
+    if (Q == 0) return ok();
+    REQUIRE(idx && q_seq && slice_lo && slice_n && ent_off && entries && out,
+            "null pointer argument");
+    REQUIRE(row_bytes >= 16 && row_bytes % 16 == 0, "row_bytes must be a positive multiple of 16");
+    REQUIRE(aligned(entries, 16) && aligned(out, 16), "entries and out must be 16-byte aligned");
+    REQUIRE(ent_rows >= 0, "ent_rows must be >= 0");
+    return cuda_status(csa::launch_cp_pack_rows(idx, q_seq, slice_lo, slice_n, ent_off, entries,
+                                                ent_rows, row_bytes, Q, B, k, out, local_idx,
+                                                dev_status, (cudaStream_t)stream),
+                       "row pack launch");
 }
 
 static csa_status_t attn_validate(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,

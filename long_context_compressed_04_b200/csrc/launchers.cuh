@@ -56,6 +56,8 @@ enum KernelKind {
     kKAttnCombine,
     kKAttn576Tc,
     kKTopkMerge,
+    kKCpCandidates,
+    kKCpPackRows,
     kKernelKinds
 };
 
@@ -125,9 +127,18 @@ cudaError_t launch_attn_tc(const AttnArgs& a, int Q, int max_n, void* workspace,
                            cudaStream_t stream);
 
 bool topk_merge_supported(int n_cand, int k);
-cudaError_t launch_topk_merge(const float* cand_scores, const int32_t* cand_idx, int Q,
-                              int n_cand, int k, int32_t* idx_out, int32_t* st,
-                              cudaStream_t stream);
+cudaError_t launch_topk_merge(const float* cand_scores, const int32_t* cand_idx,
+                              int64_t slice_stride, int W, int Q, int k_in, int k,
+                              int32_t* idx_out, int32_t* st, cudaStream_t stream);
+cudaError_t launch_cp_candidates(const int32_t* idx, const float* scores, int64_t ld,
+                                 const int32_t* q_seq, const int64_t* lo, int Q, int B, int k,
+                                 int32_t* cand_idx, float* cand_scores, int32_t* st,
+                                 cudaStream_t stream);
+cudaError_t launch_cp_pack_rows(const int32_t* idx, const int32_t* q_seq, const int64_t* lo,
+                                const int64_t* n, const int64_t* ent_off,
+                                const uint8_t* entries, int64_t ent_rows, int row_bytes, int Q,
+                                int B, int k, uint8_t* out, int32_t* local_idx, int32_t* st,
+                                cudaStream_t stream);
 
 // Sets the thread-local message csa_last_error() returns (printf-style).
 void set_error_message(const char* fmt, ...);

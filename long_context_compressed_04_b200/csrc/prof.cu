@@ -51,7 +51,8 @@ cudaEvent_t take_event() {
 const char* kernel_name(int kind) {
     static const char* names[kKernelKinds] = {"compress", "indexer_score_simt", "topk_radix",
                                               "attn_simt", "indexer_score_tc", "attn_tc",
-                                              "attn_combine", "attn576_tc", "topk_merge"};
+                                              "attn_combine", "attn576_tc", "topk_merge",
+                                              "cp_candidates", "cp_pack_rows"};
     return (kind >= 0 && kind < kKernelKinds) ? names[kind] : "?";
 }
 

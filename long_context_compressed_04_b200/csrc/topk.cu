@@ -281,7 +281,7 @@ __device__ __forceinline__ void block_or_and(uint32_t o, uint32_t a, uint32_t* o
 // nothing written, when more than cap), the k-th largest key T is selected among them, and
 // the selection -- every entry > T and the lowest-indexed ties -- is written in ascending
 // entry order from bit words of 32 entries.  The result is the unique top-k under the tie
-// order.  All 1024 threads call it; dyn holds group_smem_bytes(n, cap) bytes.
+// order.  All 1024 threads call it (for G >= 2k); dyn holds group_smem_bytes(n, cap) bytes.
 __device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
                                const uint32_t* __restrict__ qg, int n, int k, int cap,
                                int32_t* __restrict__ out, uint8_t* dyn, Shared& sh) {
@@ -461,9 +461,11 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(
         return;
     }
     bool vec = (reinterpret_cast<uintptr_t>(s) & 15) == 0;
-    if (gmax && ((n + 31) >> 5) >= k) {
+    if (gmax && ((n + 31) >> 5) >= 2 * k) {
         // from the indexer's group maxima (see topk_by_groups); the full row below only if
-        // more than cap entries reach the bound
+        // more than cap entries reach the bound.  With fewer than 2k groups the bound is
+        // the maximum of nearly every group and admits most of the row, so the row's own
+        // selection is taken straight away.
         extern __shared__ uint4 dyn_g[];
         if (topk_by_groups(s, vec, gmax + (int64_t)qq * ld_g, n, k, cap, out,
                            reinterpret_cast<uint8_t*>(dyn_g), sh))

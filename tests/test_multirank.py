@@ -81,38 +81,42 @@ def _cp_worker(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
-        # two sequences of 1000 and 37 entries, one decode query each (all entries visible)
-        n_ent = torch.tensor([1000, 37])
-        wl = types.SimpleNamespace(n_ent=n_ent, q_seq=torch.tensor([0, 1], dtype=torch.int32),
+        # three sequences of 1000, 37 and 1 entries, one decode query each (all entries
+        # visible); rank 0's slice of the third is empty
+        n_ent = torch.tensor([1000, 37, 1])
+        Q, k = 3, 8
+        wl = types.SimpleNamespace(n_ent=n_ent, q_seq=torch.tensor([0, 1, 2], dtype=torch.int32),
                                    q_pos=(n_ent * 4 - 1).to(torch.int32), m=4)
         bounds = [cp.slice_bounds(int(x), world, rank) for x in n_ent]
-        off = torch.tensor([0, bounds[0][1] - bounds[0][0]], dtype=torch.int64)
-        sl = cp.make_slice(wl, world, rank, off)
-        # this rank's store: row i holds the global entry index of its slice's row i
-        rows = []
-        for b, (lo, hi) in enumerate(bounds):
-            for e in range(lo, hi):
-                rows.append([b, e % 256, e // 256, rank])
-        store = torch.tensor(rows, dtype=torch.uint8)
-        # candidates: the slice's entries divisible by 7, ascending, padded to k = 8 with -1
-        k = 8
-        cand = torch.full((2, k), -1, dtype=torch.int32)
+        sl = cp.make_slice(wl, world, rank, torch.zeros(3, dtype=torch.int64))
+        # this rank's candidates, as csa_cp_candidates lays them out: the slice's entries
+        # divisible by 7, ascending, -1 padded; their scores (bits in the second half)
+        cand = torch.full((2, Q, k), -1, dtype=torch.int32)
         for b, (lo, hi) in enumerate(bounds):
             sel = [e for e in range(lo, hi) if e % 7 == 0][:k]
-            cand[b, :len(sel)] = torch.tensor(sel, dtype=torch.int32)
-        parts = cp.exchange(cand)
-        merged_in_order = torch.cat(parts, dim=1)
-        # the top-k: the 3 lowest candidates of every sequence, ascending (a stand-in for
-        # the library's merge), -1 padded
-        idx = torch.full((2, k), -1, dtype=torch.int32)
-        for b in range(2):
-            v = merged_in_order[b][merged_in_order[b] >= 0]
-            idx[b, :3] = v[:3]
-        packed = cp.pack_rows(idx, sl, wl.q_seq, store, 4)
-        got = cp.unpack_rows(cp.exchange(packed), idx, [cp.make_slice(wl, world, r, off) for r in range(world)],
-                             wl.q_seq)
-        out.put((rank, merged_in_order.tolist(), idx.tolist(), got.tolist(),
-                 sl.q_pos.tolist(), sl.q_live.tolist()))
+            cand[0, b, :len(sel)] = torch.tensor(sel, dtype=torch.int32)
+            cand[1, b] = torch.full((k,), float(rank + 1)).view(torch.int32)
+        buf = types.SimpleNamespace(cand=cand, gathered=torch.zeros((world, 2, Q, k),
+                                                                    dtype=torch.int32))
+        cp.exchange_candidates(buf)
+        # the merged selection (a stand-in for csa_topk_merge): the 3 lowest candidates
+        idx = torch.full((Q, k), -1, dtype=torch.int32)
+        for b in range(Q):
+            v = buf.gathered[:, 0, b].flatten()
+            v = v[v >= 0]
+            idx[b, :min(3, v.numel())] = v[:3]
+        # the packed rows, as csa_cp_pack_rows lays them out: the row if this rank's slice
+        # holds the entry (here [b, e % 256, e // 256, rank + 1]), zeros otherwise
+        buf.packed = torch.zeros((Q, k, 4), dtype=torch.uint8)
+        for b, (lo, hi) in enumerate(bounds):
+            for j in range(k):
+                e = int(idx[b, j])
+                if e >= 0 and lo <= e < hi:
+                    buf.packed[b, j] = torch.tensor([b, e % 256, e // 256, rank + 1],
+                                                    dtype=torch.uint8)
+        cp.exchange_rows(buf)
+        out.put((rank, buf.gathered.tolist(), idx.tolist(), buf.packed.tolist(),
+                 sl.q_pos.tolist(), sl.seq_len.tolist(), sl.max_n))
     finally:
         dist.destroy_process_group()
 
@@ -128,22 +132,33 @@ def test_context_parallel_exchange_two_gloo_ranks():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (_, m0, idx0, got0, qp0, live0), (_, m1, idx1, got1, qp1, live1) = res
-    # both ranks gather the same candidates, slices in rank order: ascending per sequence
-    assert m0 == m1
-    for b in range(2):
-        v = [x for x in m0[b] if x >= 0]
+    (_, g0, idx0, got0, qp0, sq0, mx0), (_, g1, idx1, got1, qp1, sq1, mx1) = res
+    # both ranks gather the same candidates, slices in rank order: ascending per sequence,
+    # each rank's scores with it
+    assert g0 == g1
+    for b in range(3):
+        v = [x for r in range(2) for x in g0[r][0][b] if x >= 0]
         assert v == sorted(v) and len(set(v)) == len(v)
-    assert idx0 == idx1 == [[0, 7, 14, -1, -1, -1, -1, -1], [0, 7, 14, -1, -1, -1, -1, -1]]
-    # every selected row arrives from the rank whose slice holds it, at its position
-    for got in (got0, got1):
-        for b in range(2):
-            for j, e in enumerate(idx0[b]):
-                if e < 0:
-                    assert got[b][j] == [0, 0, 0, 0]
-                else:
-                    lo1 = [500, 18][b]
-                    assert got[b][j] == [b, e % 256, e // 256, 0 if e < lo1 else 1]
-    # slices as sequences of their own: rank 0 sees entries 0..499 and 0..17, rank 1 the rest
-    assert qp0 == [500 * 4 - 1, 18 * 4 - 1] and qp1 == [500 * 4 - 1, 19 * 4 - 1]
-    assert live0 == live1 == [True, True]
+        for r in range(2):
+            assert all(x == torch_float_bits(float(r + 1)) for x in g0[r][1][b])
+    assert idx0 == idx1 == [[0, 7, 14, -1, -1, -1, -1, -1], [0, 7, 14, -1, -1, -1, -1, -1],
+                            [0, -1, -1, -1, -1, -1, -1, -1]]
+    # the integer sum is the gather: every selected row from the rank whose slice holds it
+    assert got0 == got1
+    lo1 = [500, 18, 0]
+    for b in range(3):
+        for j, e in enumerate(idx0[b]):
+            if e < 0:
+                assert got0[b][j] == [0, 0, 0, 0]
+            else:
+                assert got0[b][j] == [b, e % 256, e // 256, 1 if e < lo1[b] else 2]
+    # slices as sequences of their own: rank 0 sees entries 0..499, 0..17 and none of the
+    # third; rank 1 the rest; m - 1 extra tokens make position 0 valid for an empty slice
+    assert qp0 == [500 * 4 - 1, 18 * 4 - 1, 0] and qp1 == [500 * 4 - 1, 19 * 4 - 1, 1 * 4 - 1]
+    assert sq0 == [500 * 4 + 3, 18 * 4 + 3, 3] and sq1 == [500 * 4 + 3, 19 * 4 + 3, 4 + 3]
+    assert mx0 == mx1 == 500
+
+
+def torch_float_bits(x: float) -> int:
+    import struct
+    return struct.unpack("<i", struct.pack("<f", x))[0]
