@@ -65,6 +65,13 @@ def lib() -> ctypes.CDLL:
             L.orc_compress.argtypes = [P, P, P, P, P, P, P, P, I64, I, I, I, I, D, D, P, P]
             L.orc_indexer_topk.restype = I
             L.orc_indexer_topk.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, P, P, I64]
+            L.orc_e2m1_value.restype = D
+            L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+            L.orc_e8m0_value.restype = D
+            L.orc_e8m0_value.argtypes = [ctypes.c_uint8]
+            L.orc_indexer_topk_mxfp4.restype = I
+            L.orc_indexer_topk_mxfp4.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, P,
+                                                 P, I64]
             L.orc_attention.restype = I
             L.orc_attention.argtypes = [P, P, I, P, P, P, P, P, P, P, I, I, P, I, I, I, I,
                                         D, D, D, P]
@@ -109,6 +116,19 @@ def e4m3_round(x) -> np.ndarray:
     out = np.empty(x.shape, np.uint8)
     lib().orc_e4m3_round_array(_p(x), x.size, _p(out))
     return out
+
+
+def e2m1_value(codes) -> np.ndarray:
+    """FP4 E2M1 values of the low 4 bits of each code."""
+    c = _c(codes, np.uint8)
+    table = np.array([lib().orc_e2m1_value(v) for v in range(16)])
+    return table[c & 0x0F]
+
+
+def e8m0_value(codes) -> np.ndarray:
+    c = _c(codes, np.uint8)
+    table = np.array([lib().orc_e8m0_value(v) for v in range(256)])
+    return table[c]
 
 
 # ---- building blocks -----------------------------------------------------------------
@@ -189,6 +209,33 @@ def indexer_topk(qI, qs, w, kI, ks, ent_off, q_seq, q_pos, *, H_I: int, d_I: int
                                 _p(scores), int(ld_scores or 0))
     if rc != 0:
         raise ValueError(f"orc_indexer_topk failed: {rc}")
+    return (idx, scores) if want_scores else idx
+
+
+def indexer_topk_mxfp4(qI, qI_sf, w, kI, kI_sf, ent_off, q_seq, q_pos, *, H_I: int, d_I: int,
+                       m: int, k: int, select_bf16: bool = False, want_scores: bool = False,
+                       ld_scores: int | None = None):
+    """MXFP4 indexer + top-k.  qI uint8 [Q, H_I, d_I/2] packed (element 2j in the low
+    nibble), qI_sf uint8 [Q, H_I, d_I/32] (E8M0), kI uint8 [rows, d_I/2], kI_sf uint8
+    [rows, d_I/32].  Returns idx int32 [Q, k] (and fp32 scores [Q, ld_scores], NaN where not
+    visible; the BF16-rounded values when select_bf16)."""
+    qI, qI_sf, kI, kI_sf = (_c(a, np.uint8) for a in (qI, qI_sf, kI, kI_sf))
+    w = _c(w, np.float32)
+    ent_off = _c(ent_off, np.int64)
+    q_seq, q_pos = _c(q_seq, np.int32), _c(q_pos, np.int32)
+    Q = q_seq.size
+    idx = np.empty((Q, k), np.int32)
+    scores = None
+    if want_scores:
+        if ld_scores is None:
+            ld_scores = int(((q_pos.astype(np.int64) + 1) // m).max()) if Q else 0
+        scores = np.full((Q, max(ld_scores, 1)), np.nan, np.float32)
+    rc = lib().orc_indexer_topk_mxfp4(_p(qI), _p(qI_sf), _p(w), _p(kI), _p(kI_sf), _p(ent_off),
+                                      _p(q_seq), _p(q_pos), Q, H_I, d_I, m, k,
+                                      1 if select_bf16 else 0, _p(idx), _p(scores),
+                                      int(ld_scores or 0))
+    if rc != 0:
+        raise ValueError(f"orc_indexer_topk_mxfp4 failed: {rc}")
     return (idx, scores) if want_scores else idx
 
 

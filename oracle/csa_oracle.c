@@ -335,6 +335,93 @@ int orc_indexer_topk(const uint8_t* qI, const float* qs, const float* w,
 }
 
 /* ------------------------------------------------------------------------------------ */
+/* Steps a3/a4 in FP4 ([P2] Figure 2 "Lightning Indexer FP4 Precision"; section 3.4: MXFP4
+ * on the QK path of CSA, indexer scores quantised FP32 -> BF16 for the top-k selector).  */
+
+/* FP4 E2M1: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0.  Exponent field 0 is
+ * subnormal: 0.5 * mantissa. */
+double orc_e2m1_value(uint8_t code) {
+    int sign = (code >> 3) & 1, e = (code >> 1) & 3, mant = code & 1;
+    double v = (e == 0) ? 0.5 * mant : ldexp(1.0 + 0.5 * mant, e - 1);
+    return sign ? -v : v;
+}
+
+/* E8M0: an unsigned biased exponent, 2^(e-127); all ones is NaN. */
+double orc_e8m0_value(uint8_t code) {
+    if (code == 0xFF) return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
+/* Element c of a packed MXFP4 vector. */
+static double mxfp4_elem(const uint8_t* packed, int c) {
+    uint8_t byte = packed[c >> 1];
+    return orc_e2m1_value((c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0x0F));
+}
+
+int orc_indexer_topk_mxfp4(const uint8_t* qI, const uint8_t* qI_sf, const float* w,
+                           const uint8_t* kI, const uint8_t* kI_sf, const int64_t* ent_off,
+                           const int32_t* q_seq, const int32_t* q_pos, int Q, int HI, int dI,
+                           int m, int k, int select_bf16, int32_t* idx_out, float* scores,
+                           int64_t ld_scores) {
+    int rc = 0;
+    const int nb = dI / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int qq = 0; qq < Q; qq++) {
+        int b = q_seq[qq];
+        int64_t t = q_pos[qq];
+        int n = (int)((t + 1) / m);
+        if (scores && n > ld_scores) {
+#pragma omp atomic write
+            rc = -3;
+            continue;
+        }
+        double* qv = (double*)malloc(sizeof(double) * HI * dI);
+        double* qsc = (double*)malloc(sizeof(double) * HI * nb);
+        double* kvv = (double*)malloc(sizeof(double) * dI);
+        double* ksc = (double*)malloc(sizeof(double) * nb);
+        float* s = (float*)malloc(sizeof(float) * (n > 0 ? n : 1));
+        for (int h = 0; h < HI; h++) {
+            const uint8_t* qp = qI + ((int64_t)qq * HI + h) * (dI / 2);
+            for (int c = 0; c < dI; c++) qv[h * dI + c] = mxfp4_elem(qp, c);
+            for (int bl = 0; bl < nb; bl++)
+                qsc[h * nb + bl] = orc_e8m0_value(qI_sf[((int64_t)qq * HI + h) * nb + bl]);
+        }
+        int bad = 0;
+        for (int i = 0; i < n; i++) {
+            int64_t row = ent_off[b] + i;
+            for (int c = 0; c < dI; c++) kvv[c] = mxfp4_elem(kI + row * (dI / 2), c);
+            for (int bl = 0; bl < nb; bl++) ksc[bl] = orc_e8m0_value(kI_sf[row * nb + bl]);
+            float acc = 0.0f;
+            for (int h = 0; h < HI; h++) {
+                double dot = 0.0;
+                for (int bl = 0; bl < nb; bl++) {
+                    double blk = 0.0; /* exact: products of E2M1 values have <= 4 bits */
+                    for (int c = 32 * bl; c < 32 * bl + 32; c++) blk += qv[h * dI + c] * kvv[c];
+                    dot += blk * qsc[h * nb + bl] * ksc[bl];
+                }
+                float d = (float)dot;
+                acc = fmaf(w[(int64_t)qq * HI + h], fmaxf(d, 0.0f), acc);
+            }
+            if (select_bf16) acc = (float)orc_bf16_value(orc_bf16_round((double)acc));
+            s[i] = acc;
+            if (isnan(s[i])) bad = 1;
+        }
+        if (bad) {
+#pragma omp atomic write
+            rc = -2;
+        }
+        select_topk(s, n, k, idx_out + (int64_t)qq * k);
+        if (scores) memcpy(scores + (int64_t)qq * ld_scores, s, sizeof(float) * n);
+        free(qv);
+        free(qsc);
+        free(kvv);
+        free(ksc);
+        free(s);
+    }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------------------ */
 /* Steps a5/a6: shared-KV MQA over compressed entries plus the sliding window, with an
  * attention sink and partial / inverse RoPE.
  * [P2] 2.1: CSA attends to the top-k entries, HCA densely to all entries; both add a

@@ -83,6 +83,32 @@ int orc_indexer_topk(const uint8_t* qI, const float* qs, const float* w,
                      const int32_t* q_seq, const int32_t* q_pos, int Q, int HI, int dI,
                      int m, int k, int32_t* idx_out, float* scores, int64_t ld_scores);
 
+/* ---- steps a3/a4 in FP4: MXFP4 lightning indexer, FP32 or BF16 selector scores ----
+ * [P2] Figure 2 ("Lightning Indexer FP4 Precision") and "其他注意力技术细节" (the indexer
+ * computes in FP4); section 3.4 (MXFP4 quantisation on the QK path of CSA; the indexer
+ * scores quantised from FP32 to BF16 for the top-k selector).
+ * MXFP4 is the OCP microscaling format: FP4 E2M1 elements (1 sign, 2 exponent bits with
+ * bias 1, 1 mantissa bit: +-{0, 0.5, 1, 1.5, 2, 3, 4, 6}) sharing one E8M0 scale per 32
+ * consecutive elements (value 2^(e-127); e = 255 is NaN).  Storage: two elements per byte,
+ * element 2j in the low nibble.
+ * qI [Q, HI, dI/2] packed, qI_sf [Q, HI, dI/32]; w fp32 [Q, HI]; kI [rows, dI/2] packed,
+ * kI_sf [rows, dI/32]; dI a multiple of 32.  The block scales carry the magnitudes, so
+ * there is no per-head or per-entry factor besides w.
+ * Score (fp32, fixed order): acc = +0; for h: acc = fmaf(w, max(dot_h, 0), acc); s = acc,
+ * where dot_h = sum over blocks of 2^(eq + ek - 254) * (exact block dot of the elements),
+ * summed in fp64 and rounded once to fp32.
+ * select_bf16 = 0: top-k of s as in orc_indexer_topk.  select_bf16 = 1: each score is
+ * rounded to BF16 (nearest, ties to even) first; the top-k is taken on the rounded values
+ * with the same order (ties: lower index first), and scores receives the rounded values.
+ * Returns as orc_indexer_topk. */
+double orc_e2m1_value(uint8_t code);        /* the low 4 bits of code */
+double orc_e8m0_value(uint8_t code);
+int orc_indexer_topk_mxfp4(const uint8_t* qI, const uint8_t* qI_sf, const float* w,
+                           const uint8_t* kI, const uint8_t* kI_sf, const int64_t* ent_off,
+                           const int32_t* q_seq, const int32_t* q_pos, int Q, int HI, int dI,
+                           int m, int k, int select_bf16, int32_t* idx_out, float* scores,
+                           int64_t ld_scores);
+
 /* ---- steps a5/a6: sparse (idx != NULL) or dense (idx == NULL) shared-KV MQA ----
  * q bf16 [Q, H, D]; entries in format fmt at rows ent_off[b] + i; kv raw bf16 window rows
  * addressed as in orc_compress.  n = floor((t+1)/m) entries are visible to a query at t.
