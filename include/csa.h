@@ -156,6 +156,45 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
                                     int32_t* dev_status, void* stream);
 
 /*
+ * lightning_indexer_topk_mxfp4 -- steps a3 + a4 with MXFP4 query heads and keys and,
+ * optionally, BF16-rounded selector scores ("DeepSeek-V4 深度分析报告" Figure 2, "Lightning
+ * Indexer FP4 Precision"; "其他注意力技术细节": the indexer computes in FP4; section 3.4:
+ * MXFP4 quantisation on the QK path of CSA, the indexer scores quantised from FP32 to BF16
+ * for the top-k selector).
+ *   MXFP4 is the OCP microscaling format: e2m1 elements (+-{0, 0.5, 1, 1.5, 2, 3, 4, 6}),
+ *   two per byte with element 2j in the low nibble, and one UE8M0 scale byte (2^(e-127),
+ *   0xFF = NaN) per 32 consecutive elements.
+ *   s_i = sum_h w_h * ReLU(q_h . k_i) over h ascending by fmaf in fp32, q_h . k_i the
+ *   block-scaled dot product accumulated in fp32 by the tensor cores (exact when the
+ *   blocks' partial sums are: the integer-valued inputs of the tests).  No per-head or
+ *   per-entry factor besides w: the block scales carry the magnitudes.
+ *   select_bf16 = 1: every score is rounded to BF16 (nearest, ties to even) and the top-k
+ *   is taken on the rounded values with the same order (larger first, lower index first
+ *   among equal values); the score rows then hold the rounded values (as fp32).  The
+ *   section 3.4 reading: this variant trades the FP32 selection's bit-exact index set for a
+ *   recall figure (the pages quote 99.7 % of the entries kept).  select_bf16 = 0 selects on
+ *   the FP32 scores exactly as lightning_indexer_topk does.
+ * Arguments: as lightning_indexer_topk, with
+ *   qI uint8 [Q, H_I, d_I / 2] packed e2m1; qI_sf uint8 [Q, H_I, d_I / 32] UE8M0;
+ *   w fp32 [Q, H_I]; kI uint8 [ent_rows, d_I / 2]; kI_sf uint8 [ent_rows, d_I / 32];
+ *   H_I in {16, 32, 64}, d_I = 128.  qI, kI 16-byte aligned; qI_sf, kI_sf 4-byte aligned.
+ *   The workspace is csa_indexer_workspace_size(Q, max_n, k) bytes, used as by
+ *   lightning_indexer_topk.
+ * Errors as lightning_indexer_topk.
+ */
+csa_status_t lightning_indexer_topk_mxfp4(const uint8_t* qI, const uint8_t* qI_sf,
+                                          const float* w, const uint8_t* kI,
+                                          const uint8_t* kI_sf, int64_t ent_rows,
+                                          const int64_t* seq_len, const int64_t* ent_off,
+                                          const int32_t* q_seq, const int32_t* q_pos, int32_t Q,
+                                          int32_t B, int32_t H_I, int32_t d_I, int32_t m,
+                                          int32_t k, int32_t max_n, int32_t select_bf16,
+                                          int32_t* idx_out, float* scores_out,
+                                          int64_t ld_scores, void* workspace,
+                                          size_t workspace_bytes, int32_t* dev_status,
+                                          void* stream);
+
+/*
  * Context-parallel decode (the stuffyNLP post's context parallelism applied to the
  * selection and attention of "DeepSeek-V4 深度分析报告" 2.1 CSA).  A sequence's entries
  * are split into W contiguous slices (say one per GPU, slice r on rank r, slices in

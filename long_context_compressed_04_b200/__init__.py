@@ -67,6 +67,9 @@ _SIGS = {
     "csa_profile_enable": (None, [ctypes.c_int]),
     "csa_profile_collect": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_int]),
     "csa_debug_set_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
+    "lightning_indexer_topk_mxfp4": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P,
+                                                    _I32, _I32, _I32, _I32, _I32, _I32, _I32,
+                                                    _I32, _P, _P, _I64, _P, _SZ, _P, _P]),
     "csa_topk_merge": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "csa_cp_candidates": (ctypes.c_int, [_P, _P, _I64, _P, _P, _I32, _I32, _I32, _P, _P, _P,
                                          _P]),
@@ -186,6 +189,20 @@ def lightning_indexer_topk_noalloc(qI, qI_scale, w, kI, kI_scale, seq_len, ent_o
         _p(ent_off), _p(q_seq),
         _p(q_pos), q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out),
         ld_scores, _p(dev_status), _s(stream)))
+
+
+def lightning_indexer_topk_mxfp4(qI, qI_sf, w, kI, kI_sf, seq_len, ent_off, q_seq, q_pos,
+                                 idx_out, workspace, *, B: int, H_I: int, d_I: int, m: int,
+                                 k: int, max_n: int, select_bf16: bool = False, scores_out=None,
+                                 ld_scores: int = 0, dev_status=None, stream=None):
+    """MXFP4 indexer + top-k (see include/csa.h).  qI / kI: packed e2m1 bytes; qI_sf /
+    kI_sf: UE8M0 bytes."""
+    _check(_lib.lightning_indexer_topk_mxfp4(
+        _p(qI), _p(qI_sf), _p(w), _p(kI), _p(kI_sf), kI.shape[0], _p(seq_len), _p(ent_off),
+        _p(q_seq), _p(q_pos), q_seq.numel(), B, H_I, d_I, m, k, max_n, 1 if select_bf16 else 0,
+        _p(idx_out), _p(scores_out), ld_scores, _p(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _p(dev_status), _s(stream)))
 
 
 def csa_topk_merge(cand_scores, cand_idx, idx_out, *, dev_status=None, stream=None):

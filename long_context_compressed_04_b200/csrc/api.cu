@@ -212,6 +212,52 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     return cuda_status(e, "top-k launch");
 }
 
+csa_status_t lightning_indexer_topk_mxfp4(const uint8_t* qI, const uint8_t* qI_sf,
+                                          const float* w, const uint8_t* kI,
+                                          const uint8_t* kI_sf, int64_t ent_rows,
+                                          const int64_t* seq_len, const int64_t* ent_off,
+                                          const int32_t* q_seq, const int32_t* q_pos, int32_t Q,
+                                          int32_t B, int32_t H_I, int32_t d_I, int32_t m,
+                                          int32_t k, int32_t max_n, int32_t select_bf16,
+                                          int32_t* idx_out, float* scores_out,
+                                          int64_t ld_scores, void* workspace,
+                                          size_t workspace_bytes, int32_t* dev_status,
+                                          void* stream) {
+    REQUIRE(Q >= 0, "Q must be >= 0");
+    if (Q == 0) return ok();
+    REQUIRE(qI && qI_sf && w && seq_len && ent_off && q_seq && q_pos && idx_out,
+            "null pointer argument");
+    REQUIRE(max_n >= 0, "max_n must be >= 0");
+    REQUIRE(ent_rows >= 0 && ent_rows < (1ll << 31), "ent_rows out of range");
+    REQUIRE(max_n == 0 || ent_rows == 0 || (kI && kI_sf), "null key pointer");
+    REQUIRE(aligned(qI, 16) && (kI == nullptr || aligned(kI, 16)), "qI and kI must be 16-byte aligned");
+    REQUIRE(aligned(qI_sf, 4) && (kI_sf == nullptr || aligned(kI_sf, 4)),
+            "qI_sf and kI_sf must be 4-byte aligned");
+    REQUIRE(B >= 1 && m >= 1, "B and m must be >= 1");
+    REQUIRE(select_bf16 == 0 || select_bf16 == 1, "select_bf16 must be 0 or 1");
+    SUPPORT(csa::indexer_fp4_supported(H_I, d_I),
+            "MXFP4 indexer shape H_I = %d, d_I = %d not supported (16, 32 or 64 heads; d_I = 128)",
+            H_I, d_I);
+    SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
+    REQUIRE(scores_out == nullptr || ld_scores >= max_n, "ld_scores must be >= max_n");
+    const IndexerWorkspace L = indexer_workspace(Q, max_n);
+    if (!scores_out && (!workspace || workspace_bytes < L.total || !aligned(workspace, 256)))
+        return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", L.total);
+    float* scores = scores_out ? scores_out : (float*)((uint8_t*)workspace + L.off_scores);
+    const int64_t ld = scores_out ? ld_scores : L.ld;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint32_t* gmax = nullptr;
+    if (workspace && workspace_bytes >= L.gmax_bytes && aligned(workspace, 256))
+        gmax = (uint32_t*)workspace;
+    cudaError_t e = csa::launch_indexer_fp4(qI, qI_sf, w, kI, kI_sf, ent_rows, seq_len, ent_off,
+                                            q_seq, q_pos, Q, B, H_I, m, max_n, select_bf16,
+                                            scores, ld, dev_status, s, gmax, L.ld_g);
+    if (e != cudaSuccess) return cuda_status(e, "MXFP4 indexer launch");
+    e = csa::launch_topk(scores, ld, q_seq, q_pos, seq_len, Q, B, m, max_n, k, idx_out, dev_status,
+                         s, gmax, L.ld_g);
+    return cuda_status(e, "top-k launch");
+}
+
 csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx,
                             int64_t slice_stride, int32_t W, int32_t Q, int32_t k_in, int32_t k,
                             int32_t* idx_out, int32_t* dev_status, void* stream) {

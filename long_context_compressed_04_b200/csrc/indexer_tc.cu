@@ -31,6 +31,7 @@
 #include <mutex>
 
 #include "launchers.cuh"
+#include "indexer_items.cuh"
 #include "sm100.cuh"
 
 namespace csa {
@@ -41,15 +42,12 @@ constexpr int kGroupTiles = 4;           // tiles per pipeline stage (one barrie
 constexpr int kStages = 3;               // 3 x 64 KB of key tiles in flight per SM
 constexpr int kAccSets = 2;              // TMEM accumulator sets of kGroupTiles accumulators
 constexpr int kAux = 3;                  // prefetched items
-constexpr int kTileRows = 128;           // entries per tile (MMA M)
 constexpr int kDI = 128;                 // indexer dim (MMA K total, bytes per key row)
 constexpr int kTileBytes = kTileRows * kDI;
 constexpr int kGroupBytes = kGroupTiles * kTileBytes;
-constexpr int kChunkTiles = 8;           // tiles per item at most
 constexpr int kFirstEpiWarp = 3;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
-constexpr int kMaxItems = 64;            // work items per CTA resolved up front
 
 struct IdxArgs {
     const float* qs;
@@ -71,74 +69,6 @@ struct IdxArgs {
     uint32_t* gmax;
     int64_t ld_g;
 };
-
-struct Item {
-    int q;
-    int n_vis;
-    int tile0;
-    int ntiles;
-    int64_t row0;
-};
-
-// Virtual tile range [v0, v1) of CTA `cta` of `grid`; equal shares of Q * qtiles.
-__device__ __forceinline__ void cta_range(const IdxArgs& a, int cta, int grid, int64_t& v0,
-                                          int64_t& v1) {
-    const int64_t V = (int64_t)a.Q * a.qtiles;
-    v0 = V * cta / grid;
-    v1 = V * (cta + 1) / grid;
-}
-
-__device__ __forceinline__ int64_t chunk_of(const IdxArgs& a, int64_t v) {
-    const int64_t q = v / a.qtiles;
-    return q * a.chunks_per_q + (v - q * a.qtiles) / kChunkTiles;
-}
-
-// Decodes item `ii` of the range [v0, v1) (the piece of the range inside its ii-th chunk);
-// false when it has no tiles.  Every role calls this with the same arguments and so walks
-// the same item sequence.
-__device__ __forceinline__ bool get_item(const IdxArgs& a, int64_t v0, int64_t v1, int ii,
-                                         Item& x, bool report) {
-    const int64_t g = chunk_of(a, v0) + ii;
-    x.q = (int)(g / a.chunks_per_q);
-    const int cq = (int)(g - (int64_t)x.q * a.chunks_per_q);
-    const int64_t cbeg = (int64_t)x.q * a.qtiles + (int64_t)cq * kChunkTiles;
-    const int64_t cend = min(cbeg + kChunkTiles, (int64_t)(x.q + 1) * a.qtiles);
-    const int lo = (int)(max(v0, cbeg) - cbeg);
-    const int hi = (int)(min(v1, cend) - cbeg);
-    report = report && cq == 0 && lo == 0;   // one piece per query reports its errors
-    const int b = a.q_seq[x.q];
-    const int t = a.q_pos[x.q];
-    if (b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]) {
-        if (report) flag(a.st, CSA_DEV_OOB);
-        return false;
-    }
-    int n = (t + 1) / a.m;
-    if (n > a.max_n) {
-        if (report) flag(a.st, CSA_DEV_CAPACITY);
-        n = a.max_n;
-    }
-    x.row0 = a.ent_off[b];
-    const int64_t avail = a.ent_rows - x.row0;
-    if ((int64_t)n > avail) {
-        if (report) flag(a.st, CSA_DEV_OOB);
-        n = avail > 0 ? (int)avail : 0;
-    }
-    x.n_vis = n;
-    x.tile0 = cq * kChunkTiles + lo;
-    const int tiles = (n + kTileRows - 1) / kTileRows;
-    x.ntiles = min(cq * kChunkTiles + hi, tiles) - x.tile0;
-    return x.ntiles > 0;
-}
-
-// Item ii of this CTA: from the table built at kernel start, or decoded directly past it.
-__device__ __forceinline__ bool fetch_item(const IdxArgs& a, const Item* items, int64_t v0,
-                                           int64_t v1, int ii, Item& x, bool report) {
-    if (ii < kMaxItems) {
-        x = items[ii];
-        return x.ntiles > 0;
-    }
-    return get_item(a, v0, v1, ii, x, report);
-}
 
 // TMEM columns: kAccSets x kGroupTiles accumulators of HI fp32 columns, rounded to a power
 // of two >= 32.

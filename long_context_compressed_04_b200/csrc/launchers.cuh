@@ -58,6 +58,7 @@ enum KernelKind {
     kKTopkMerge,
     kKCpCandidates,
     kKCpPackRows,
+    kKIndexerFp4,
     kKernelKinds
 };
 
@@ -114,6 +115,13 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
                               int m, int max_n, float* scores, int64_t ld, int32_t* st,
                               cudaStream_t stream, uint32_t* gmax = nullptr, int64_t ld_g = 0);
+bool indexer_fp4_supported(int HI, int dI);
+cudaError_t launch_indexer_fp4(const uint8_t* qI, const uint8_t* qI_sf, const float* w,
+                               const uint8_t* kI, const uint8_t* kI_sf, int64_t ent_rows,
+                               const int64_t* seq_len, const int64_t* ent_off,
+                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
+                               int m, int max_n, int bf16, float* scores, int64_t ld,
+                               int32_t* st, cudaStream_t stream, uint32_t* gmax, int64_t ld_g);
 cudaError_t launch_topk(const float* scores, int64_t ld, const int32_t* q_seq,
                         const int32_t* q_pos, const int64_t* seq_len, int Q, int B, int m,
                         int max_n, int k, int32_t* idx_out, int32_t* st, cudaStream_t stream,

@@ -52,7 +52,8 @@ const char* kernel_name(int kind) {
     static const char* names[kKernelKinds] = {"compress", "indexer_score_simt", "topk_radix",
                                               "attn_simt", "indexer_score_tc", "attn_tc",
                                               "attn_combine", "attn576_tc", "topk_merge",
-                                              "cp_candidates", "cp_pack_rows"};
+                                              "cp_candidates", "cp_pack_rows",
+                                              "indexer_score_fp4"};
     return (kind >= 0 && kind < kKernelKinds) ? names[kind] : "?";
 }
 

@@ -418,6 +418,68 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw128(const void* tile) {
     return d;
 }
 
+// K-major tile with the 64-byte swizzle (rows of 64 bytes, 8-row groups 512 bytes apart;
+// tile base 512-byte aligned).  Advancing along K inside the row adds (bytes >> 4).
+__device__ __forceinline__ uint64_t smem_desc_k_sw64(const void* tile) {
+    const uint64_t addr = smem_addr(tile);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;          // start address
+    d |= 1ull << 16;                       // leading-dim byte offset (unused with swizzle)
+    d |= (uint64_t)(512 >> 4) << 32;       // stride-dim byte offset: 8 rows x 64 B
+    d |= 1ull << 46;                       // descriptor version for sm_100
+    d |= 4ull << 61;                       // 64-byte swizzle
+    return d;
+}
+
+// 32 rows x 16 bytes stored contiguously (no swizzle: 8-row core matrices 128 bytes apart),
+// the source of a tcgen05.cp of shape 32x128b.
+__device__ __forceinline__ uint64_t smem_desc_rows16(const void* p) {
+    const uint64_t addr = smem_addr(p);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;
+    d |= (uint64_t)(128 >> 4) << 16;
+    d |= (uint64_t)(128 >> 4) << 32;
+    d |= 1ull << 46;
+    return d;
+}
+
+// Copies 32 rows x 128 bits of shared memory into TMEM columns [col, col + 4) of all four
+// 32-lane quarters (row r to lanes r, 32 + r, 64 + r, 96 + r).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy reads
+// (TMA, tcgen05.cp, tcgen05.mma).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// D[tmem] (+)= (A x SFA)[smem] x (B x SFB)[smem]^T, MXFP4: packed e2m1 A and B (K = 64 per
+// instruction), one UE8M0 scale per 32 elements from TMEM (sfa / sfb: column addresses;
+// the instruction descriptor selects the bytes).
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t sfa, uint32_t sfb,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], "
+        "p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
+// Instruction descriptor of kind::mxf4 with UE8M0 scales: e2m1 A and B, K-major, M x N,
+// dense K = 64; sf_a / sf_b: the byte of each 32-bit TMEM scale column this instruction's
+// first 32-element block reads (0 or 2: two blocks per instruction).
+__host__ __device__ constexpr uint32_t instr_desc_mxf4(int M, int N, uint32_t sf_a,
+                                                       uint32_t sf_b) {
+    return (sf_b << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(M >> 4) << 24) | (sf_a << 29);
+}
+
 // Instruction descriptor: fp32 accumulate, A/B K-major, shape M x N.
 // a_fmt / b_fmt: e4m3 = 0 (kind::f8f6f4); bf16 = 1 (kind::f16).
 __host__ __device__ constexpr uint32_t instr_desc(uint32_t a_fmt, uint32_t b_fmt, int M, int N,

@@ -12,7 +12,7 @@ import torch
 
 from . import (CSA_KV_BF16, csa_compress, csa_entry_row_bytes, csa_indexer_workspace_size,
                dense_hca_attn, dense_hca_workspace_size, hca_compress, lightning_indexer_topk,
-               sparse_mqa_attn)
+               lightning_indexer_topk_mxfp4, sparse_mqa_attn)
 from .synth import Workload
 
 
@@ -77,6 +77,18 @@ def indexer_topk(wl: Workload, buf: Buffers, scores_out=None, stream=None):
                            k=wl.k, max_n=buf.max_n, scores_out=scores_out,
                            ld_scores=0 if scores_out is None else scores_out.shape[1],
                            dev_status=buf.dev_status, stream=stream)
+
+
+def indexer_topk_mxfp4(wl: Workload, fp4, buf: Buffers, select_bf16: bool = False,
+                       scores_out=None, stream=None):
+    """The MXFP4 indexer + top-k into buf.idx; fp4 = (qI, qI_sf, kI, kI_sf)."""
+    qI, qsf, kI, ksf = fp4
+    lightning_indexer_topk_mxfp4(qI, qsf, wl.w, kI, ksf, wl.seq_len, wl.ent_off, wl.q_seq,
+                                 wl.q_pos, buf.idx, buf.workspace, B=wl.B, H_I=wl.H_I,
+                                 d_I=wl.d_I, m=wl.m, k=wl.k, max_n=buf.max_n,
+                                 select_bf16=select_bf16, scores_out=scores_out,
+                                 ld_scores=0 if scores_out is None else scores_out.shape[1],
+                                 dev_status=buf.dev_status, stream=stream)
 
 
 def attend(wl: Workload, buf: Buffers, stream=None):

@@ -9,7 +9,9 @@ Distributions follow the workloads the method is specified on: raw per-token KV 
 logits ~N(0,1) stored as bf16, positional bias ~N(0, 0.1) fp32, attention-sink logits
 ~N(0,1) per head, queries ~N(0,1) bf16, indexer heads in FP8 E4M3 -- either
 integer-valued in [-3, 3] with unit scales (exact-arithmetic runs) or N(0,1) quantised
-with one scale per 1x128 row -- and per-head indexer weights ~U(0,1).
+with one scale per 1x128 row -- and per-head indexer weights ~U(0,1).  MXFP4 indexer
+inputs (packed e2m1 + UE8M0 block scales) are drawn either as uniform codes with scales
+near 1 or as N(0,1) values quantised per 32-element block.
 
 Random numbers come from ``torch.Generator`` seeded per workload, on the device the
 tensors are made on; a given (workload, seed, device) always yields the same tensors.
@@ -240,6 +242,57 @@ def csa_decode_1m_fp8(device="cpu", seed=0, indexer="int", B=8, keep_raw=None) -
     return make_workload("csa_decode_1m_b8_fp8", B=B, T=1 << 20, D=576, H=128, m=4, span=8,
                          W=128, fmt=1, H_I=64, d_I=128, k=1024, indexer=indexer,
                          keep_raw=keep_raw, seed=seed, device=device)
+
+
+# ---- MXFP4 indexer inputs -----------------------------------------------------------
+# Packed e2m1 codes (element 2j in the low nibble) and one UE8M0 scale byte per 32
+# elements, the layout lightning_indexer_topk_mxfp4 reads.
+
+# e2m1 magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6 (codes 0..7); the midpoints between them
+_E2M1_MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
+
+
+def _pack_nibbles(codes: torch.Tensor) -> torch.Tensor:
+    c = codes.to(torch.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).contiguous()
+
+
+def mxfp4_integer(rows, cols, g, device, exp_lo=126, exp_hi=128):
+    """Uniformly drawn e2m1 codes and block exponents in [exp_lo, exp_hi] (scales 2^-1 ..
+    2^1 by default): every block dot product and their sums are exact in fp32.
+    Returns (packed uint8 [rows, cols / 2], scales uint8 [rows, cols / 32])."""
+    codes = torch.randint(0, 16, (rows, cols), generator=g, device=device)
+    sf = torch.randint(exp_lo, exp_hi + 1, (rows, cols // 32), generator=g, device=device)
+    return _pack_nibbles(codes), sf.to(torch.uint8).contiguous()
+
+
+def mxfp4_from_normal(rows, cols, g, device):
+    """N(0,1) values quantised to MXFP4 the usual way: per block of 32 the scale exponent is
+    floor(log2(amax)) - 2 (the largest e2m1 exponent), each value divided by the scale goes
+    to the nearest e2m1 magnitude (saturating at 6; exact midpoints, of probability zero,
+    go up).  Returns (packed uint8 [rows, cols / 2], scales uint8 [rows, cols / 32])."""
+    x = torch.randn((rows, cols // 32, 32), generator=g, device=device)
+    amax = x.abs().amax(dim=2).clamp_min(2.0 ** -100)
+    e = torch.floor(torch.log2(amax)) - 2
+    y = x / torch.exp2(e)[:, :, None]
+    mids = torch.tensor(_E2M1_MIDPOINTS, device=device)
+    mag = torch.bucketize(y.abs().contiguous(), mids, right=True)
+    codes = mag | ((y < 0).to(mag.dtype) << 3)
+    sf = (e + 127).clamp(0, 254).to(torch.uint8)
+    return _pack_nibbles(codes.reshape(rows, cols)), sf.contiguous()
+
+
+def mxfp4_indexer(wl: Workload, kind: str = "int", seed: int = 0):
+    """MXFP4 query heads and keys for `wl`'s indexer shapes ("int": mxfp4_integer, "normal":
+    mxfp4_from_normal).  Returns (qI [Q, H_I, d_I / 2], qI_sf [Q, H_I, d_I / 32],
+    kI [ent_rows, d_I / 2], kI_sf [ent_rows, d_I / 32]); the head weights stay wl.w."""
+    dev = wl.q.device
+    g = _gen(seed * 7919 + 4, dev)
+    make = mxfp4_integer if kind == "int" else mxfp4_from_normal
+    kI, ksf = make(max(wl.ent_rows, 1), wl.d_I, g, dev)
+    qI, qsf = make(wl.Q * wl.H_I, wl.d_I, g, dev)
+    return (qI.reshape(wl.Q, wl.H_I, wl.d_I // 2), qsf.reshape(wl.Q, wl.H_I, wl.d_I // 32),
+            kI, ksf)
 
 
 # ---- re-batching (for batch-invariance runs) -----------------------------------------

@@ -9,6 +9,7 @@ import torch
 from . import attention as _attention
 from . import compress as _compress
 from . import indexer_topk as _indexer_topk
+from . import indexer_topk_mxfp4 as _indexer_topk_mxfp4
 
 
 def u16(t: torch.Tensor) -> np.ndarray:
@@ -49,6 +50,18 @@ def indexer(wl, want_scores=True):
     return _indexer_topk(u8(wl.qI), f32(wl.qs), f32(wl.w), u8(wl.kI), f32(wl.ks),
                                i64(wl.ent_off), i32(wl.q_seq), i32(wl.q_pos), H_I=wl.H_I,
                                d_I=wl.d_I, m=wl.m, k=wl.k, want_scores=want_scores,
+                               ld_scores=max(max_n, 1))
+
+
+def indexer_mxfp4(wl, fp4, select_bf16=False, want_scores=True):
+    """The MXFP4 indexer on `wl`'s queries; fp4 = (qI, qI_sf, kI, kI_sf) as the synthetic
+    generator lays them out."""
+    qI, qsf, kI, ksf = fp4
+    max_n = int(((i64(wl.q_pos) + 1) // wl.m).max())
+    return _indexer_topk_mxfp4(u8(qI), u8(qsf), f32(wl.w), u8(kI), u8(ksf),
+                               i64(wl.ent_off), i32(wl.q_seq), i32(wl.q_pos),
+                               H_I=wl.H_I, d_I=wl.d_I, m=wl.m, k=wl.k,
+                               select_bf16=select_bf16, want_scores=want_scores,
                                ld_scores=max(max_n, 1))
 
 

@@ -6,7 +6,8 @@ import numpy as np
 import torch
 
 import oracle
-from oracle.workload import attention, compress, f32, i32, i64, indexer, u8, u16  # noqa: F401
+from oracle.workload import (attention, compress, f32, i32, i64, indexer, indexer_mxfp4,  # noqa: F401
+                             u8, u16)
 
 # Output tolerance for bf16 / fp8 storage with fp32 accumulation: max abs and relative L2.
 ATOL = 2e-2
