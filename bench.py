@@ -41,6 +41,11 @@ WORKLOADS = {
     "hca_decode_1m_b16": dict(kind="hca", B=16, T=1 << 20, jitter=0, D=128, H=64, fmt=0),
     "csa_decode_1m_b8_fp8": dict(kind="csa", B=8, T=1 << 20, jitter=0, D=576, H=128, H_I=64,
                                  d_I=128, k=1024, fmt=1),
+    # the 1M decode step with the pages' FP4 indexer: MXFP4 query heads and keys (N(0,1)
+    # quantised per 32-element block) and the top-k taken on BF16-rounded scores
+    "csa_decode_1m_b8_mxfp4": dict(kind="csa", B=8, T=1 << 20, jitter=0, D=576, H=128,
+                                   H_I=64, d_I=128, k=1024, fmt=1, indexer_fmt="mxfp4",
+                                   select_bf16=True),
     # a causal prefill chunk: 8192 new query tokens after 65536 prior tokens; the step
     # compresses the 2048 entries that pool new tokens, then scores, selects and attends
     "csa_prefill_8k_on_64k": dict(kind="csa_prefill", B=1, T=65536 + 8192, jitter=0, D=128,
@@ -125,9 +130,16 @@ def make_workload(name: str, rank: int, device, keep_raw=None):
                                    seed=rank, device=device)
     T = rank_lengths(name, rank) if c["jitter"] else c["T"]
     if c["kind"] == "csa":
-        return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
-                                   fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
-                                   indexer="fp8", keep_raw=keep_raw, seed=rank, device=device)
+        fp4 = c.get("indexer_fmt") == "mxfp4"
+        wl = synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
+                                 fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
+                                 indexer="int" if fp4 else "fp8", keep_raw=keep_raw, seed=rank,
+                                 device=device)
+        if fp4:
+            wl.qI4, wl.qsf4, wl.kI4, wl.ksf4 = synth.mxfp4_indexer(wl, "normal", seed=rank)
+            wl.select_bf16 = bool(c.get("select_bf16", False))
+            wl.kI = wl.ks = wl.qI = wl.qs = None
+        return wl
     return synth.make_workload(name, B=c["B"], T=T, D=c["D"], H=c["H"], m=128, span=128, W=128,
                                fmt=c["fmt"], keep_raw=keep_raw, seed=rank, device=device)
 
@@ -173,7 +185,13 @@ def algorithmic_bytes(wl):
     win = torch.clamp(wl.q_pos.cpu().to(torch.int64) + 1, max=wl.W)
     qo = wl.Q * wl.H * wl.D * 2 * 2
     comp = wl.B * (wl.span * wl.D * 2 * 2 + rb)
-    if wl.H_I:
+    if wl.H_I and wl.kI4 is not None:
+        # MXFP4: d_I / 2 element bytes + d_I / 32 scale bytes per key; the same per head
+        # plus its fp32 weight
+        row4 = wl.d_I // 2 + wl.d_I // 32
+        keys = int(n_vis.sum()) * row4 + wl.Q * wl.H_I * (row4 + 4)
+        sel = int(torch.clamp(n_vis, max=wl.k).sum()) * rb + wl.Q * wl.k * 4
+    elif wl.H_I:
         keys = int(n_vis.sum()) * (wl.d_I + 4) + wl.Q * wl.H_I * (wl.d_I + 8)
         sel = int(torch.clamp(n_vis, max=wl.k).sum()) * rb + wl.Q * wl.k * 4
     else:
@@ -259,6 +277,7 @@ def gpu_index_for_smi(dev: int) -> str:
 
 
 CPU_SAMPLE_SEQS = {"csa_decode_128k_b32": 32, "hca_decode_1m_b16": 16, "csa_decode_1m_b8_fp8": 8,
+                   "csa_decode_1m_b8_mxfp4": 8,
                    "csa_prefill_8k_on_64k": 64}   # prefill: sampled queries of the chunk
 
 
@@ -294,10 +313,13 @@ def cpu_baseline(name: str, n_seq: int | None = None):
                           f"{int(iseq.numel())} new entries compressed (indexer over every "
                           f"visible entry, top-k, attention), {dt:.2f} s"}
     T = synth.jittered_lengths(n_seq, c["T"], c["jitter"], 99) if c["jitter"] else [c["T"]] * n_seq
+    fp4 = None
     if c["kind"] == "csa":
         wl = synth.make_workload(name, B=n_seq, T=T, D=c["D"], H=c["H"], m=4, span=8, W=128,
                                  fmt=c["fmt"], H_I=c["H_I"], d_I=c["d_I"], k=c["k"],
                                  indexer="fp8", keep_raw=256, seed=7)
+        if c.get("indexer_fmt") == "mxfp4":
+            fp4 = synth.mxfp4_indexer(wl, "normal", seed=7)
     else:
         wl = synth.make_workload(name, B=n_seq, T=T, D=c["D"], H=c["H"], m=128, span=128, W=128,
                                  fmt=c["fmt"], keep_raw=256, seed=7)
@@ -312,7 +334,11 @@ def cpu_baseline(name: str, n_seq: int | None = None):
     oracle.compress(_orc.u16(wl.kv), _orc.u16(wl.gate), _orc.f32(wl.bias), _orc.i64(wl.kv_off),
                     _orc.i64(wl.kv_pos0), _orc.i64(wl.ent_off), item_seq, item_ent, m=wl.m,
                     span=wl.span, D=wl.D, fmt=wl.fmt, entries=rows)
-    idx = _orc.indexer(wl, want_scores=False) if wl.H_I else None
+    if fp4 is not None:
+        idx = _orc.indexer_mxfp4(wl, fp4, select_bf16=bool(c.get("select_bf16")),
+                                 want_scores=False)
+    else:
+        idx = _orc.indexer(wl, want_scores=False) if wl.H_I else None
     _orc.attention(wl, rows, idx)
     dt = time.perf_counter() - t0
     return {"value": wl.Q / dt, "unit": UNIT, "cores": min(oracle.num_threads(), wl.Q),
@@ -344,7 +370,7 @@ def run_reference(args):
 
 DEFAULT_WORKLOAD = "csa_decode_1m_b8_fp8"
 # measured in the same run as the default workload and reported under "also"
-ALSO_WORKLOADS = ("csa_decode_128k_b32", "hca_decode_1m_b16")
+ALSO_WORKLOADS = ("csa_decode_128k_b32", "hca_decode_1m_b16", "csa_decode_1m_b8_mxfp4")
 
 
 def fp8_gemm_peak(dev, n: int = 8192, seconds: float = 4.0):
@@ -500,8 +526,10 @@ def measure(name: str, args, dist, dev, rank: int, world: int, full: bool):
     # the dominant kernel is the one that moves the method's dominant bytes: the indexer
     # (every visible key, each step) for CSA decode, the attention (every entry) for HCA
     alg_of = {"indexer_score_tc": key_bytes, "indexer_score_simt": key_bytes,
+              "indexer_score_fp4": key_bytes,
               "attn_tc": total_bytes - key_bytes, "attn_simt": total_bytes - key_bytes}
-    dom_name = next((n for n in (["indexer_score_tc", "indexer_score_simt"] if wl.H_I else [])
+    dom_name = next((n for n in (["indexer_score_tc", "indexer_score_fp4", "indexer_score_simt"]
+                                 if wl.H_I else [])
                      + ["attn_tc", "attn_simt"] if n in per_kernel), None)
     roof = None
     if WORKLOADS[name]["kind"] == "csa_prefill" and "indexer_score_tc" in per_kernel:
@@ -534,7 +562,10 @@ def measure(name: str, args, dist, dev, rank: int, world: int, full: bool):
                    **({"cache": "stored rows drawn directly; raw store keeps the last 256 tokens"}
                       if raw_tail else {}),
                    "l2": "flushed before every timed step (256 MB write, then 256 MB read)",
-                   "indexer_inputs": "fp8 e4m3 N(0,1), 1x128 scales"},
+                   "indexer_inputs": ("mxfp4 (e2m1, one UE8M0 scale per 32) from N(0,1)"
+                                      + ("; top-k on BF16-rounded scores" if wl.select_bf16
+                                         else "")) if wl.kI4 is not None
+                   else "fp8 e4m3 N(0,1), 1x128 scales"},
         "roofline": roof,
         "step_roofline": {"algorithmic_bytes": total_bytes,
                           "achieved_gbs": round(total_bytes / step_s / 1e9, 1),
@@ -569,7 +600,7 @@ def measure_e2e(name, wl, buf, new_seq, new_ent, args, dist, dev, world, flush_l
     last_rows = torch.cat([(wl.kv_off[b] + (wl.T.to(dev)[b] - nn - wl.kv_pos0[b]))
                            + torch.arange(nn, device=dev) for b in range(wl.B)]).long()
     nr = last_rows.numel()
-    fields = [f for f in ("q", "qI", "qs", "w") if getattr(wl, f) is not None]
+    fields = [f for f in ("q", "qI", "qs", "qI4", "qsf4", "w") if getattr(wl, f) is not None]
     pinned = {f: torch.empty(getattr(wl, f).shape, dtype=getattr(wl, f).dtype,
                              pin_memory=True).copy_(getattr(wl, f).cpu()) for f in fields}
     pin_kv = torch.empty((nr, wl.D), dtype=wl.kv.dtype, pin_memory=True).copy_(wl.kv[last_rows].cpu())

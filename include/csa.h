@@ -71,6 +71,29 @@ typedef enum {
 #define CSA_KV_BF16 0
 #define CSA_KV_FP8_576 1
 
+/*
+ * Cache layout ("DeepSeek-V4 深度分析报告" 3.5, KV cache management: a fixed-size state
+ * cache holds the sliding-window KV and the not yet compressed tail; the classical cache
+ * holds the compressed CSA / HCA entries in blocks of lcm(m, m') = 128 tokens).  Passed by
+ * pointer to the calls below; NULL keeps the contiguous layout described above.
+ *   block_table  nullable int32 [B, bt_stride]: the classical cache in blocks of 128 tokens,
+ *                i.e. 32 CSA entries (m = 4 only).  Entry i of sequence b is row
+ *                block_table[b * bt_stride + i / 32] * 32 + i % 32 of the entry (and
+ *                indexer-key) store; ent_off is then unused (may be NULL).  A block index
+ *                < 0, or whose rows lie past ent_rows, sets CSA_DEV_OOB and its entries are
+ *                skipped.  Dense HCA attention takes no block table (CSA_ERR_UNSUPPORTED).
+ *   kv_ring      0: the raw store is linear as above.  > 0: the state cache is a ring of
+ *                kv_ring rows per sequence; raw token p of sequence b is row
+ *                kv_off[b] + p mod kv_ring, and positions seq_len[b] - kv_ring ..
+ *                seq_len[b] - 1 are held (kv_pos0 is unused and may be NULL).  The ring
+ *                must hold the window and the tokens an entry pools, else CSA_DEV_OOB.
+ */
+typedef struct {
+    const int32_t* block_table;
+    int64_t bt_stride;
+    int64_t kv_ring;
+} csa_cache_layout_t;
+
 int csa_version(void);
 const char* csa_last_error(void);
 /* Bytes per stored entry row for (fmt, D), or -1 if unsupported. */
@@ -89,7 +112,10 @@ int32_t csa_entry_row_bytes(int32_t fmt, int32_t D);
  *   kv, gate   bf16 [rows, D] raw KV and gate logits (row addressing as above)
  *   pos_bias   fp32 [8, D], row j pairs with the j-th pooled position
  *   item_seq, item_ent  int32 [n_items]: compute entry item_ent[n] of sequence item_seq[n]
- *   entries    output rows, format fmt; only the listed rows are written
+ *   entries    output rows, format fmt; only the listed rows are written (with a block
+ *              table in the layout, entry i's row comes from it; the caller provides rows
+ *              for every block it names)
+ *   layout     nullable cache layout (block table, state-cache ring)
  *   B          number of sequences (item_seq must be < B; the entry's last pooled
  *              position (i+1)*4-1 must be < seq_len[b], else CSA_DEV_OOB and no write)
  *   D          128 (fmt CSA_KV_BF16) or 576 (either format)
@@ -102,7 +128,8 @@ csa_status_t csa_compress(const void* kv, const void* gate, const float* pos_bia
                           const int64_t* ent_off,
                           const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
                           int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
-                          void* entries, int32_t* dev_status, void* stream);
+                          void* entries, const csa_cache_layout_t* layout, int32_t* dev_status,
+                          void* stream);
 
 /*
  * hca_compress -- HCA 128:1 compression (step a2).
@@ -116,7 +143,8 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
                           const int64_t* ent_off,
                           const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
                           int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
-                          void* entries, int32_t* dev_status, void* stream);
+                          void* entries, const csa_cache_layout_t* layout, int32_t* dev_status,
+                          void* stream);
 
 /*
  * lightning_indexer_topk -- lightning-indexer scores and top-k selection (steps a3, a4).
@@ -142,6 +170,8 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
  *   rows.  With scores_out given the score rows go there: the workspace may then be just
  *   large enough for the first part (ceil(Q * ceil(max_n / 32) * 4 / 256) * 256 bytes), or
  *   NULL (with workspace_bytes 0), in which case the selection reads the full score rows.
+ *   layout: nullable cache layout; with a block table the key rows (and kI_scale) follow
+ *   it, block by block.
  * kI and qI must be 16-byte aligned.  Errors as above; CSA_DEV_NAN, CSA_DEV_CAPACITY.
  */
 size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k);
@@ -153,7 +183,8 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
                                     int32_t d_I, int32_t m, int32_t k, int32_t max_n,
                                     int32_t* idx_out, float* scores_out, int64_t ld_scores,
                                     void* workspace, size_t workspace_bytes,
-                                    int32_t* dev_status, void* stream);
+                                    const csa_cache_layout_t* layout, int32_t* dev_status,
+                                    void* stream);
 
 /*
  * lightning_indexer_topk_mxfp4 -- steps a3 + a4 with MXFP4 query heads and keys and,
@@ -191,8 +222,33 @@ csa_status_t lightning_indexer_topk_mxfp4(const uint8_t* qI, const uint8_t* qI_s
                                           int32_t k, int32_t max_n, int32_t select_bf16,
                                           int32_t* idx_out, float* scores_out,
                                           int64_t ld_scores, void* workspace,
-                                          size_t workspace_bytes, int32_t* dev_status,
-                                          void* stream);
+                                          size_t workspace_bytes,
+                                          const csa_cache_layout_t* layout,
+                                          int32_t* dev_status, void* stream);
+
+/*
+ * csa_cache_append -- one decode token per sequence into the hybrid cache
+ * ("DeepSeek-V4 深度分析报告" 3.5: the state cache holds the window's KV and the tokens not
+ * yet compressed; the classical cache holds the entries in blocks of 128 tokens).
+ *   For every sequence b, with p = seq_len[b] on entry: the token's raw KV and gate rows
+ *   (kv_new, gate_new bf16 [B, D]) are written to its state-cache row (kv_off[b] + p mod
+ *   kv_ring with a ring in the layout, else kv_off[b] + p - kv_pos0[b]; the row must be
+ *   < kv_rows); if p + 1 is a multiple of m, the entry (p + 1) / m - 1 it completes gets its
+ *   indexer key row kI_new[b] (e4m3 [B, d_I]) and scale kI_scale_new[b] written to the key
+ *   store (kI [ent_rows, d_I], kI_scale [ent_rows]) at the entry's row (block table or
+ *   ent_off; kI_new may be NULL to skip); then seq_len[b] = p + 1.  The entry itself is
+ *   then compressed by csa_compress (with the same layout), after this call.
+ *   A row outside kv_rows / ent_rows sets CSA_DEV_OOB and leaves seq_len[b] unchanged.
+ *   The kernels after this call on the stream start only when it has completed.
+ * Errors: CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED (D), CSA_ERR_CUDA.
+ */
+csa_status_t csa_cache_append(const void* kv_new, const void* gate_new, const uint8_t* kI_new,
+                              const float* kI_scale_new, int32_t d_I, int64_t* seq_len,
+                              const int64_t* kv_off, const int64_t* kv_pos0, int64_t kv_rows,
+                              const int64_t* ent_off, int64_t ent_rows, int32_t B, int32_t D,
+                              int32_t m, void* kv, void* gate, uint8_t* kI, float* kI_scale,
+                              const csa_cache_layout_t* layout, int32_t* dev_status,
+                              void* stream);
 
 /*
  * Context-parallel decode (the stuffyNLP post's context parallelism applied to the
@@ -273,6 +329,8 @@ csa_status_t csa_cp_pack_rows(const int32_t* idx, const int32_t* q_seq, const in
  *   idx int32 [Q, k] (entries < n_vis(t) for ratio m, or -1 = skip); sink fp32 [H]
  *   H in {16, 64, 128}; D 128 (bf16) or 576 (either format); 0 <= W <= 128
  *   out bf16 [Q, H, D]
+ *   layout: nullable cache layout (the selected entries' rows through a block table; the
+ *   window's raw rows through a state-cache ring)
  * Pointers q/kv/entries/out must be 16-byte aligned.  Out-of-range indices set CSA_DEV_OOB
  * and are skipped.
  */
@@ -283,7 +341,8 @@ csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt, in
                              const int32_t* q_pos, const int32_t* idx, int32_t k, int32_t m,
                              const float* sink, int32_t Q, int32_t B, int32_t H, int32_t D,
                              int32_t W, float softmax_scale, float rope_theta, float eps,
-                             void* out, int32_t* dev_status, void* stream);
+                             void* out, const csa_cache_layout_t* layout, int32_t* dev_status,
+                             void* stream);
 
 /*
  * dense_hca_attn -- HCA dense MQA over every visible entry plus the window (a6).
@@ -297,6 +356,8 @@ csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt, in
  *   on the query's own n_vis and the shape, so results do not depend on the batch).
  */
 size_t dense_hca_workspace_size(int32_t Q, int32_t H, int32_t D, int32_t max_n);
+/* layout: nullable; its kv_ring applies to the window, a block table is refused (the dense
+ * pass reads each sequence's entries as one contiguous array). */
 csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int64_t ent_rows,
                             const int64_t* seq_len, const int64_t* ent_off, const void* kv,
                             const int64_t* kv_off,
@@ -304,7 +365,8 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int
                             int32_t m, const float* sink, int32_t Q, int32_t B, int32_t H,
                             int32_t D, int32_t W, float softmax_scale, float rope_theta,
                             float eps, int32_t max_n, void* out, void* workspace,
-                            size_t workspace_bytes, int32_t* dev_status, void* stream);
+                            size_t workspace_bytes, const csa_cache_layout_t* layout,
+                            int32_t* dev_status, void* stream);
 
 /*
  * lightning_indexer_topk_noalloc -- the same scores and selection as

@@ -45,20 +45,20 @@ _SIGS = {
     "csa_last_error": (ctypes.c_char_p, []),
     "csa_entry_row_bytes": (_I32, [_I32, _I32]),
     "csa_compress": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32,
-                                    _F32, _F32, _P, _P, _P]),
+                                    _F32, _F32, _P, _P, _P, _P]),
     "hca_compress": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32, _I32, _I32,
-                                    _F32, _F32, _P, _P, _P]),
+                                    _F32, _F32, _P, _P, _P, _P]),
     "csa_indexer_workspace_size": (_SZ, [_I32, _I32, _I32]),
     "lightning_indexer_topk": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32,
                                               _I32, _I32, _I32, _I32, _P, _P, _I64, _P, _SZ, _P,
-                                              _P]),
+                                              _P, _P]),
     "sparse_mqa_attn": (ctypes.c_int, [_P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32, _P,
                                        _I32, _I32, _I32, _I32, _I32, _F32, _F32, _F32, _P, _P,
-                                       _P]),
+                                       _P, _P]),
     "dense_hca_workspace_size": (_SZ, [_I32, _I32, _I32, _I32]),
     "dense_hca_attn": (ctypes.c_int, [_P, _P, _I32, _I64, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32,
                                       _I32, _I32, _I32, _F32, _F32, _F32, _I32, _P, _P, _SZ, _P,
-                                      _P]),
+                                      _P, _P]),
     "lightning_indexer_topk_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P,
                                                       _I32,
                                                       _I32, _I32, _I32, _I32, _I32, _I32, _P, _P,
@@ -69,7 +69,9 @@ _SIGS = {
     "csa_debug_set_wait_limit": (ctypes.c_int, [ctypes.c_longlong]),
     "lightning_indexer_topk_mxfp4": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _P, _P, _P, _P,
                                                     _I32, _I32, _I32, _I32, _I32, _I32, _I32,
-                                                    _I32, _P, _P, _I64, _P, _SZ, _P, _P]),
+                                                    _I32, _P, _P, _I64, _P, _SZ, _P, _P, _P]),
+    "csa_cache_append": (ctypes.c_int, [_P, _P, _P, _P, _I32, _P, _P, _P, _I64, _P, _I64, _I32,
+                                        _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
     "csa_topk_merge": (ctypes.c_int, [_P, _P, _I64, _I32, _I32, _I32, _I32, _P, _P, _P]),
     "csa_cp_candidates": (ctypes.c_int, [_P, _P, _I64, _P, _P, _I32, _I32, _I32, _P, _P, _P,
                                          _P]),
@@ -82,6 +84,29 @@ for _name, (_res, _args) in _SIGS.items():
     _fn.argtypes = _args
 
 EXPORTED = tuple(_SIGS)
+
+
+class CacheLayout(ctypes.Structure):
+    """csa_cache_layout_t (see include/csa.h): the classical cache's block table and the
+    state cache's ring size."""
+    _fields_ = [("block_table", ctypes.c_void_p), ("bt_stride", ctypes.c_int64),
+                ("kv_ring", ctypes.c_int64)]
+
+
+def cache_layout(block_table=None, kv_ring: int = 0):
+    """A cache layout for the calls' ``layout`` argument, or None for the contiguous one.
+    block_table: int32 [B, bt_stride] device tensor (blocks of 32 CSA entries); kv_ring:
+    rows of each sequence's state-cache ring (0 = linear raw store)."""
+    if block_table is None and not kv_ring:
+        return None
+    lay = CacheLayout(None if block_table is None else block_table.data_ptr(),
+                      0 if block_table is None else block_table.stride(0), int(kv_ring))
+    lay._block_table = block_table      # keeps the tensor alive with the struct
+    return lay
+
+
+def _lay(layout):
+    return None if layout is None else ctypes.byref(layout)
 
 
 def _p(t):
@@ -147,31 +172,34 @@ def dense_hca_workspace_size(Q: int, H: int, D: int, max_n: int) -> int:
 def csa_compress(kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq, item_ent,
                  entries, *,
                  B: int, D: int, fmt: int = CSA_KV_BF16, rope_theta: float = 10000.0,
-                 eps: float = 1e-6, dev_status=None, stream=None):
+                 eps: float = 1e-6, layout=None, dev_status=None, stream=None):
     _check(_lib.csa_compress(_p(kv), _p(gate), _p(pos_bias), _p(seq_len), _p(kv_off), _p(kv_pos0),
                              _p(ent_off), _p(item_seq), _p(item_ent), item_seq.numel(), B, D, fmt,
-                             rope_theta, eps, _p(entries), _p(dev_status), _s(stream)))
+                             rope_theta, eps, _p(entries), _lay(layout), _p(dev_status),
+                             _s(stream)))
 
 
 def hca_compress(kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq, item_ent,
                  entries, *,
                  B: int, D: int, fmt: int = CSA_KV_BF16, rope_theta: float = 10000.0,
-                 eps: float = 1e-6, dev_status=None, stream=None):
+                 eps: float = 1e-6, layout=None, dev_status=None, stream=None):
     _check(_lib.hca_compress(_p(kv), _p(gate), _p(pos_bias), _p(seq_len), _p(kv_off), _p(kv_pos0),
                              _p(ent_off), _p(item_seq), _p(item_ent), item_seq.numel(), B, D, fmt,
-                             rope_theta, eps, _p(entries), _p(dev_status), _s(stream)))
+                             rope_theta, eps, _p(entries), _lay(layout), _p(dev_status),
+                             _s(stream)))
 
 
 def lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, seq_len, ent_off, q_seq, q_pos, idx_out,
                            workspace, *, B: int, H_I: int, d_I: int, m: int, k: int, max_n: int,
-                           scores_out=None, ld_scores: int = 0, dev_status=None, stream=None):
+                           scores_out=None, ld_scores: int = 0, layout=None, dev_status=None,
+                           stream=None):
     _check(_lib.lightning_indexer_topk(
         _p(qI), _p(qI_scale), _p(w), _p(kI), _p(kI_scale), kI_scale.numel(), _p(seq_len),
         _p(ent_off), _p(q_seq),
         _p(q_pos),
         q_seq.numel(), B, H_I, d_I, m, k, max_n, _p(idx_out), _p(scores_out), ld_scores,
         _p(workspace), 0 if workspace is None else workspace.numel() * workspace.element_size(),
-        _p(dev_status), _s(stream)))
+        _lay(layout), _p(dev_status), _s(stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -194,7 +222,8 @@ def lightning_indexer_topk_noalloc(qI, qI_scale, w, kI, kI_scale, seq_len, ent_o
 def lightning_indexer_topk_mxfp4(qI, qI_sf, w, kI, kI_sf, seq_len, ent_off, q_seq, q_pos,
                                  idx_out, workspace, *, B: int, H_I: int, d_I: int, m: int,
                                  k: int, max_n: int, select_bf16: bool = False, scores_out=None,
-                                 ld_scores: int = 0, dev_status=None, stream=None):
+                                 ld_scores: int = 0, layout=None, dev_status=None,
+                                 stream=None):
     """MXFP4 indexer + top-k (see include/csa.h).  qI / kI: packed e2m1 bytes; qI_sf /
     kI_sf: UE8M0 bytes."""
     _check(_lib.lightning_indexer_topk_mxfp4(
@@ -202,7 +231,19 @@ def lightning_indexer_topk_mxfp4(qI, qI_sf, w, kI, kI_sf, seq_len, ent_off, q_se
         _p(q_seq), _p(q_pos), q_seq.numel(), B, H_I, d_I, m, k, max_n, 1 if select_bf16 else 0,
         _p(idx_out), _p(scores_out), ld_scores, _p(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(),
-        _p(dev_status), _s(stream)))
+        _lay(layout), _p(dev_status), _s(stream)))
+
+
+def csa_cache_append(kv_new, gate_new, seq_len, kv_off, kv_pos0, kv, gate, *, B: int, D: int,
+                     m: int, kI_new=None, kI_scale_new=None, ent_off=None, kI=None,
+                     kI_scale=None, layout=None, dev_status=None, stream=None):
+    """One decode token per sequence into the state cache (and, for the entries it
+    completes, their indexer keys into the key store); see include/csa.h."""
+    _check(_lib.csa_cache_append(
+        _p(kv_new), _p(gate_new), _p(kI_new), _p(kI_scale_new),
+        0 if kI is None else kI.shape[1], _p(seq_len), _p(kv_off), _p(kv_pos0), kv.shape[0],
+        _p(ent_off), 0 if kI is None else kI.shape[0], B, D, m, _p(kv), _p(gate), _p(kI),
+        _p(kI_scale), _lay(layout), _p(dev_status), _s(stream)))
 
 
 def csa_topk_merge(cand_scores, cand_idx, idx_out, *, dev_status=None, stream=None):
@@ -236,20 +277,20 @@ def sparse_mqa_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_
                     out, *,
                     fmt: int, B: int, H: int, D: int, W: int, m: int, k: int,
                     softmax_scale: float, rope_theta: float = 10000.0, eps: float = 1e-6,
-                    dev_status=None, stream=None):
+                    layout=None, dev_status=None, stream=None):
     _check(_lib.sparse_mqa_attn(
         _p(q), _p(entries), fmt, entries.shape[0], _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
         _p(q_pos), _p(idx), k, m, _p(sink), q_seq.numel(), B, H, D, W, softmax_scale,
-        rope_theta, eps, _p(out), _p(dev_status), _s(stream)))
+        rope_theta, eps, _p(out), _lay(layout), _p(dev_status), _s(stream)))
 
 
 def dense_hca_attn(q, entries, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos, sink, out,
                    workspace, *, fmt: int, B: int, H: int, D: int, W: int, m: int, max_n: int,
                    softmax_scale: float, rope_theta: float = 10000.0, eps: float = 1e-6,
-                   dev_status=None, stream=None):
+                   layout=None, dev_status=None, stream=None):
     _check(_lib.dense_hca_attn(
         _p(q), _p(entries), fmt, entries.shape[0], _p(seq_len), _p(ent_off), _p(kv), _p(kv_off), _p(kv_pos0), _p(q_seq),
         _p(q_pos), m, _p(sink), q_seq.numel(), B, H, D, W, softmax_scale, rope_theta, eps,
         max_n, _p(out), _p(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(),
-        _p(dev_status), _s(stream)))
+        _lay(layout), _p(dev_status), _s(stream)))

@@ -60,17 +60,46 @@ IndexerWorkspace indexer_workspace(int32_t Q, int32_t max_n) {
     return w;
 }
 
+// Entry and raw-row maps of a call.  A block table needs m = 4 (blocks of 128 tokens = 32
+// CSA entries); without one, entries are contiguous from ent_off.  A ring makes kv_pos0
+// unused.
+csa_status_t make_rows(const csa_cache_layout_t* L, int m, const int64_t* ent_off,
+                       const int64_t* kv_off, const int64_t* kv_pos0, bool need_raw,
+                       csa::EntryRows* er, csa::RawRows* raw, bool need_ent = true) {
+    const int32_t* bt = L ? L->block_table : nullptr;
+    const int64_t ring = L ? L->kv_ring : 0;
+    REQUIRE(!bt || (m == 4 && L->bt_stride >= 1),
+            "a block table needs m = 4 (blocks of 32 entries) and bt_stride >= 1");
+    REQUIRE(!need_ent || bt || ent_off, "ent_off must not be null without a block table");
+    REQUIRE(ring >= 0, "kv_ring must be >= 0");
+    if (need_raw) {
+        REQUIRE(kv_off && (ring > 0 || kv_pos0), "kv_off (and kv_pos0 without a ring) must not be null");
+    }
+    er->ent_off = ent_off;
+    er->bt = bt;
+    er->bt_stride = bt ? L->bt_stride : 0;
+    er->pe_shift = 5;
+    raw->kv_off = kv_off;
+    raw->kv_pos0 = kv_pos0;
+    raw->ring = ring;
+    return ok();
+}
+
 csa_status_t compress_common(int m, int span, const void* kv, const void* gate,
                              const float* bias, const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
                              const int64_t* ent_off, const int32_t* item_seq,
                              const int32_t* item_ent, int64_t n_items, int32_t B, int32_t D,
                              int32_t fmt, float theta, float eps, void* entries,
-                             int32_t* dev_status, void* stream) {
+                             const csa_cache_layout_t* layout, int32_t* dev_status,
+                             void* stream) {
     REQUIRE(n_items >= 0 && n_items < (1ll << 31), "n_items out of range: %lld", (long long)n_items);
     if (n_items == 0) return ok();
-    REQUIRE(kv && gate && bias && seq_len && kv_off && kv_pos0 && ent_off && item_seq && item_ent &&
-                entries,
+    REQUIRE(kv && gate && bias && seq_len && item_seq && item_ent && entries,
             "null pointer argument");
+    csa::EntryRows er;
+    csa::RawRows raw;
+    csa_status_t lv = make_rows(layout, m, ent_off, kv_off, kv_pos0, true, &er, &raw);
+    if (lv != CSA_OK) return lv;
     REQUIRE(aligned(kv, 16) && aligned(gate, 16) && aligned(entries, 16) && aligned(bias, 16),
             "kv, gate, pos_bias and entries must be 16-byte aligned");
     REQUIRE(B >= 1, "B must be >= 1");
@@ -78,7 +107,7 @@ csa_status_t compress_common(int m, int span, const void* kv, const void* gate,
     SUPPORT(D == 128 || D == 576, "head dim %d not supported (128 or 576)", D);
     SUPPORT(fmt == CSA_KV_BF16 || D == 576, "fp8 entry format needs D = 576");
     REQUIRE(theta > 1.f && eps >= 0.f, "rope_theta must be > 1 and eps >= 0");
-    cudaError_t e = csa::launch_compress(span, kv, gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
+    cudaError_t e = csa::launch_compress(span, kv, gate, bias, seq_len, raw, er, item_seq,
                                          item_ent, n_items, B, m, D, fmt, theta, eps, entries,
                                          dev_status, (cudaStream_t)stream);
     return cuda_status(e, "compress launch");
@@ -142,9 +171,10 @@ csa_status_t csa_compress(const void* kv, const void* gate, const float* pos_bia
                           const int64_t* ent_off,
                           const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
                           int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
-                          void* entries, int32_t* dev_status, void* stream) {
+                          void* entries, const csa_cache_layout_t* layout, int32_t* dev_status,
+                          void* stream) {
     return compress_common(4, 8, kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq, item_ent,
-                           n_items, B, D, fmt, rope_theta, eps, entries, dev_status, stream);
+                           n_items, B, D, fmt, rope_theta, eps, entries, layout, dev_status, stream);
 }
 
 csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bias,
@@ -152,10 +182,11 @@ csa_status_t hca_compress(const void* kv, const void* gate, const float* pos_bia
                           const int64_t* ent_off,
                           const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
                           int32_t B, int32_t D, int32_t fmt, float rope_theta, float eps,
-                          void* entries, int32_t* dev_status, void* stream) {
+                          void* entries, const csa_cache_layout_t* layout, int32_t* dev_status,
+                          void* stream) {
     return compress_common(128, 128, kv, gate, pos_bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
-                           item_ent, n_items, B, D, fmt, rope_theta, eps, entries, dev_status,
-                           stream);
+                           item_ent, n_items, B, D, fmt, rope_theta, eps, entries, layout,
+                           dev_status, stream);
 }
 
 size_t csa_indexer_workspace_size(int32_t Q, int32_t max_n, int32_t k) {
@@ -171,11 +202,16 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
                                     int32_t d_I, int32_t m, int32_t k, int32_t max_n,
                                     int32_t* idx_out, float* scores_out, int64_t ld_scores,
                                     void* workspace, size_t workspace_bytes,
-                                    int32_t* dev_status, void* stream) {
+                                    const csa_cache_layout_t* layout, int32_t* dev_status,
+                                    void* stream) {
     REQUIRE(Q >= 0, "Q must be >= 0");
     if (Q == 0) return ok();
-    REQUIRE(qI && qI_scale && w && seq_len && ent_off && q_seq && q_pos && idx_out,
+    REQUIRE(qI && qI_scale && w && seq_len && q_seq && q_pos && idx_out,
             "null pointer argument");
+    csa::EntryRows er;
+    csa::RawRows raw;
+    csa_status_t lv = make_rows(layout, m, ent_off, nullptr, nullptr, false, &er, &raw);
+    if (lv != CSA_OK) return lv;
     REQUIRE(max_n >= 0, "max_n must be >= 0");
     REQUIRE(ent_rows >= 0 && ent_rows < (1ll << 31), "ent_rows out of range");
     REQUIRE(max_n == 0 || ent_rows == 0 || (kI && kI_scale), "null key pointer");
@@ -198,11 +234,11 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     if (csa::indexer_tc_supported(H_I, d_I)) {
         if (workspace && workspace_bytes >= L.gmax_bytes && aligned(workspace, 256))
             gmax = (uint32_t*)workspace;
-        e = csa::launch_indexer_tc(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
+        e = csa::launch_indexer_tc(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, er,
                                    q_seq, q_pos, Q, B, H_I, m, max_n, scores, ld, dev_status, s,
                                    gmax, L.ld_g);
     } else {
-        e = csa::launch_indexer_simt(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
+        e = csa::launch_indexer_simt(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, er,
                                      q_seq, q_pos, Q, B, H_I, d_I, m, max_n, scores, ld,
                                      dev_status, s);
     }
@@ -221,12 +257,17 @@ csa_status_t lightning_indexer_topk_mxfp4(const uint8_t* qI, const uint8_t* qI_s
                                           int32_t k, int32_t max_n, int32_t select_bf16,
                                           int32_t* idx_out, float* scores_out,
                                           int64_t ld_scores, void* workspace,
-                                          size_t workspace_bytes, int32_t* dev_status,
-                                          void* stream) {
+                                          size_t workspace_bytes,
+                                          const csa_cache_layout_t* layout,
+                                          int32_t* dev_status, void* stream) {
     REQUIRE(Q >= 0, "Q must be >= 0");
     if (Q == 0) return ok();
-    REQUIRE(qI && qI_sf && w && seq_len && ent_off && q_seq && q_pos && idx_out,
+    REQUIRE(qI && qI_sf && w && seq_len && q_seq && q_pos && idx_out,
             "null pointer argument");
+    csa::EntryRows er;
+    csa::RawRows raw;
+    csa_status_t lv = make_rows(layout, m, ent_off, nullptr, nullptr, false, &er, &raw);
+    if (lv != CSA_OK) return lv;
     REQUIRE(max_n >= 0, "max_n must be >= 0");
     REQUIRE(ent_rows >= 0 && ent_rows < (1ll << 31), "ent_rows out of range");
     REQUIRE(max_n == 0 || ent_rows == 0 || (kI && kI_sf), "null key pointer");
@@ -249,13 +290,45 @@ csa_status_t lightning_indexer_topk_mxfp4(const uint8_t* qI, const uint8_t* qI_s
     uint32_t* gmax = nullptr;
     if (workspace && workspace_bytes >= L.gmax_bytes && aligned(workspace, 256))
         gmax = (uint32_t*)workspace;
-    cudaError_t e = csa::launch_indexer_fp4(qI, qI_sf, w, kI, kI_sf, ent_rows, seq_len, ent_off,
+    cudaError_t e = csa::launch_indexer_fp4(qI, qI_sf, w, kI, kI_sf, ent_rows, seq_len, er,
                                             q_seq, q_pos, Q, B, H_I, m, max_n, select_bf16,
                                             scores, ld, dev_status, s, gmax, L.ld_g);
     if (e != cudaSuccess) return cuda_status(e, "MXFP4 indexer launch");
     e = csa::launch_topk(scores, ld, q_seq, q_pos, seq_len, Q, B, m, max_n, k, idx_out, dev_status,
                          s, gmax, L.ld_g);
     return cuda_status(e, "top-k launch");
+}
+
+csa_status_t csa_cache_append(const void* kv_new, const void* gate_new, const uint8_t* kI_new,
+                              const float* kI_scale_new, int32_t d_I, int64_t* seq_len,
+                              const int64_t* kv_off, const int64_t* kv_pos0, int64_t kv_rows,
+                              const int64_t* ent_off, int64_t ent_rows, int32_t B, int32_t D,
+                              int32_t m, void* kv, void* gate, uint8_t* kI, float* kI_scale,
+                              const csa_cache_layout_t* layout, int32_t* dev_status,
+                              void* stream) {
+    REQUIRE(B >= 0, "B must be >= 0");
+    if (B == 0) return ok();
+    REQUIRE(kv_new && gate_new && seq_len && kv && gate, "null pointer argument");
+    REQUIRE(aligned(kv_new, 16) && aligned(gate_new, 16) && aligned(kv, 16) && aligned(gate, 16),
+            "kv_new, gate_new, kv and gate must be 16-byte aligned");
+    SUPPORT(D == 128 || D == 576, "head dim %d not supported (128 or 576)", D);
+    REQUIRE(m >= 1 && kv_rows >= 0 && ent_rows >= 0, "bad m / kv_rows / ent_rows");
+    if (kI_new) {
+        REQUIRE(kI_scale_new && kI && kI_scale, "null indexer-key pointer");
+        REQUIRE(d_I == 64 || d_I == 128, "d_I must be 64 or 128");
+        REQUIRE(aligned(kI_new, 16) && aligned(kI, 16), "kI_new and kI must be 16-byte aligned");
+    }
+    csa::EntryRows er;
+    csa::RawRows raw;
+    csa_status_t v = make_rows(layout, m, ent_off, kv_off, kv_pos0, true, &er, &raw,
+                               kI_new != nullptr);
+    if (v != CSA_OK) return v;
+    return cuda_status(csa::launch_cache_append((const uint16_t*)kv_new, (const uint16_t*)gate_new,
+                                                kI_new, kI_scale_new, seq_len, raw, er, B, D, d_I,
+                                                m, kv_rows, ent_rows, (uint16_t*)kv,
+                                                (uint16_t*)gate, kI, kI_scale, dev_status,
+                                                (cudaStream_t)stream),
+                       "cache append launch");
 }
 
 csa_status_t csa_topk_merge(const float* cand_scores, const int32_t* cand_idx,
@@ -315,8 +388,7 @@ static csa_status_t attn_validate(const void* q, const void* entries, int32_t fm
                                   const int32_t* q_pos, const float* sink, int32_t B,
                                   int32_t H, int32_t D, int32_t W, int32_t m, float scale,
                                   float theta, float eps, void* out) {
-    REQUIRE(q && entries && seq_len && ent_off && kv && kv_off && kv_pos0 && q_seq && q_pos && sink &&
-                out,
+    REQUIRE(q && entries && seq_len && kv && q_seq && q_pos && sink && out,
             "null pointer argument");
     REQUIRE(aligned(q, 16) && aligned(entries, 16) && aligned(kv, 16) && aligned(out, 16),
             "q, entries, kv and out must be 16-byte aligned");
@@ -337,7 +409,8 @@ csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt, in
                              const int32_t* q_pos, const int32_t* idx, int32_t k, int32_t m,
                              const float* sink, int32_t Q, int32_t B, int32_t H, int32_t D,
                              int32_t W, float softmax_scale, float rope_theta, float eps,
-                             void* out, int32_t* dev_status, void* stream) {
+                             void* out, const csa_cache_layout_t* layout, int32_t* dev_status,
+                             void* stream) {
     REQUIRE(Q >= 0, "Q must be >= 0");
     if (Q == 0) return ok();
     csa_status_t v = attn_validate(q, entries, fmt, ent_rows, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
@@ -345,8 +418,12 @@ csa_status_t sparse_mqa_attn(const void* q, const void* entries, int32_t fmt, in
     if (v != CSA_OK) return v;
     REQUIRE(idx != nullptr, "idx must not be null");
     SUPPORT(k >= 1 && k <= 2048, "k = %d not supported (1..2048)", k);
-    csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, ent_off, (const uint16_t*)kv,
-                    kv_off, kv_pos0, q_seq, q_pos, seq_len, idx, ent_rows, sink, (uint16_t*)out, dev_status,
+    csa::EntryRows er;
+    csa::RawRows raw;
+    v = make_rows(layout, m, ent_off, kv_off, kv_pos0, true, &er, &raw);
+    if (v != CSA_OK) return v;
+    csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, er, (const uint16_t*)kv,
+                    raw, q_seq, q_pos, seq_len, idx, ent_rows, sink, (uint16_t*)out, dev_status,
                     k, m, B, H, W, fmt, softmax_scale, eps, log2((double)rope_theta)};
     if (csa::attn_tc_supported(H, D, fmt))
         return cuda_status(csa::launch_attn_tc(a, Q, 0, nullptr, (cudaStream_t)stream),
@@ -369,7 +446,8 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int
                             int32_t m, const float* sink, int32_t Q, int32_t B, int32_t H,
                             int32_t D, int32_t W, float softmax_scale, float rope_theta,
                             float eps, int32_t max_n, void* out, void* workspace,
-                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
+                            size_t workspace_bytes, const csa_cache_layout_t* layout,
+                            int32_t* dev_status, void* stream) {
     REQUIRE(Q >= 0, "Q must be >= 0");
     if (Q == 0) return ok();
     csa_status_t v = attn_validate(q, entries, fmt, ent_rows, seq_len, ent_off, kv, kv_off, kv_pos0, q_seq, q_pos,
@@ -379,8 +457,14 @@ csa_status_t dense_hca_attn(const void* q, const void* entries, int32_t fmt, int
     const size_t need = dense_hca_workspace_size(Q, H, D, max_n);
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
         return fail(CSA_ERR_WORKSPACE, "workspace must be >= %zu bytes, 256-byte aligned", need);
-    csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, ent_off, (const uint16_t*)kv,
-                    kv_off, kv_pos0, q_seq, q_pos, seq_len, nullptr, ent_rows, sink, (uint16_t*)out, dev_status,
+    SUPPORT(!layout || !layout->block_table,
+            "dense attention reads contiguous entries: no block table");
+    csa::EntryRows er;
+    csa::RawRows raw;
+    v = make_rows(layout, m, ent_off, kv_off, kv_pos0, true, &er, &raw);
+    if (v != CSA_OK) return v;
+    csa::AttnArgs a{(const uint16_t*)q, (const uint8_t*)entries, er, (const uint16_t*)kv,
+                    raw, q_seq, q_pos, seq_len, nullptr, ent_rows, sink, (uint16_t*)out, dev_status,
                     0, m, B, H, W, fmt, softmax_scale, eps, log2((double)rope_theta)};
     if (csa::attn_tc_supported(H, D, fmt))
         return cuda_status(csa::launch_attn_tc(a, Q, max_n, workspace, (cudaStream_t)stream),

@@ -34,21 +34,23 @@ __device__ __forceinline__ bool load_key(const AttnArgs& a, int b, int t, int n_
         const int e = a.idx ? a.idx[(int64_t)blockIdx.y * a.k + vk] : vk;
         if (e < 0) {
             valid = false;
-        } else if (e >= n_vis || a.ent_off[b] + e >= a.ent_rows) {
-            valid = false;
-            if (lane == 0 && blockIdx.x == 0) flag(a.st, CSA_DEV_OOB);
         } else {
-            const int rb = a.fmt == CSA_KV_BF16 ? 2 * D : 656;
-            erow = a.entries + (a.ent_off[b] + e) * (int64_t)rb;
+            const int64_t re = e < n_vis ? a.er.row(b, e) : -1;
+            if (re < 0 || re >= a.ent_rows) {
+                valid = false;
+                if (lane == 0 && blockIdx.x == 0) flag(a.st, CSA_DEV_OOB);
+            } else {
+                const int rb = a.fmt == CSA_KV_BF16 ? 2 * D : 656;
+                erow = a.entries + re * (int64_t)rb;
+            }
         }
     } else {
         wpos = (int64_t)w0 + (vk - n_sel);
-        const int64_t p0 = a.kv_pos0[b];
-        if (wpos < p0) {
+        if (wpos < a.raw.first(b, a.seq_len[b])) {
             valid = false;
             if (lane == 0 && blockIdx.x == 0) flag(a.st, CSA_DEV_OOB);
         } else {
-            wrow = a.kv + (a.kv_off[b] + wpos - p0) * (int64_t)D;
+            wrow = a.kv + a.raw.row(b, wpos) * (int64_t)D;
         }
     }
     float2 v[NP];

@@ -98,10 +98,9 @@ static_assert(kOffIdx % 16 == 0 && kOffBars % 8 == 0, "alignment");
 struct A576Args {
     const uint16_t* q;
     const uint8_t* entries;
-    const int64_t* ent_off;
+    EntryRows er;
     const uint16_t* kv;
-    const int64_t* kv_off;
-    const int64_t* kv_pos0;
+    RawRows raw;
     const int32_t* q_seq;
     const int32_t* q_pos;
     const int64_t* seq_len;
@@ -205,18 +204,21 @@ struct EntryQuarter {
 // Issues the loads of entry v of the query's index row (staged in shared memory) into
 // registers (flags an out-of-range index once per row).
 __device__ __forceinline__ void fetch_entry(const A576Args& a, const int32_t* sidx, int v,
-                                            int n_vis, int64_t row0, int qt, EntryQuarter& x) {
+                                            int n_vis, int b, int64_t row0, int qt,
+                                            EntryQuarter& x) {
     const int e = v < a.k ? sidx[v] : -1;
     x.valid = false;
+    int64_t re = 0;
     if (e >= 0) {
-        if (e < n_vis && row0 + e < a.ent_rows) {
+        re = a.er.bt ? (e < n_vis ? a.er.row(b, e) : -1) : row0 + e;
+        if (e < n_vis && re >= 0 && re < a.ent_rows) {
             x.valid = true;
         } else if (qt == 0) {
             flag(a.st, CSA_DEV_OOB);
         }
     }
     if (x.valid) {
-        const uint8_t* er = a.entries + (row0 + e) * (int64_t)kRowBytes;
+        const uint8_t* er = a.entries + re * (int64_t)kRowBytes;
 #pragma unroll
         for (int u = 0; u < 8; u++) x.f[u] = *reinterpret_cast<const uint4*>(er + 128 * qt + 16 * u);
 #pragma unroll
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
     const uint32_t tmem = *tmem_base_smem;
 
     const int n_vis = valid ? (t + 1) / a.m : 0;
-    const int64_t row0 = valid ? a.ent_off[b] : 0;
+    const int64_t row0 = valid && !a.er.bt ? a.er.ent_off[b] : 0;
     const int w0 = t - a.W + 1 > 0 ? t - a.W + 1 : 0;
     const int n_win = a.W > 0 ? t - w0 + 1 : 0;
     const int n_wt = (a.W + kTK - 1) / kTK;          // window tiles (masked past n_win)
@@ -418,12 +420,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             const int wr = rank * kTK + kr;
             const int64_t p = (int64_t)w0 + wr;
             bool vrow = wr < n_win;
-            if (vrow && p < a.kv_pos0[b]) {
+            if (vrow && p < a.raw.first(b, a.seq_len[b])) {
                 vrow = false;
                 if (qt == 0) flag(a.st, CSA_DEV_OOB);
             }
             const uint16_t* src =
-                vrow ? a.kv + (a.kv_off[b] + p - a.kv_pos0[b]) * (int64_t)kD : nullptr;
+                vrow ? a.kv + a.raw.row(b, p) * (int64_t)kD : nullptr;
             // pass 1: my quarter of the raw row into the tile (18 loads in flight) and its
             // sum of squares
             float ss = 0.f;
@@ -519,8 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 const int v = (jg - n_wt) * kTK + u % kTK;
                 if (jg < n_wt || v >= a.k) continue;
                 const int e = sidx[v];
-                if (e >= 0 && e < n_vis && row0 + e < a.ent_rows)
-                    prefetch_l2_bulk(a.entries + (row0 + e) * (int64_t)kRowBytes, kRowBytes);
+                if (e >= 0 && e < n_vis) {
+                    const int64_t re = a.er.bt ? a.er.row(b, e) : row0 + e;
+                    if (re >= 0 && re < a.ent_rows)
+                        prefetch_l2_bulk(a.entries + re * (int64_t)kRowBytes, kRowBytes);
+                }
             }
         }
         // ---- the selected entries ----
@@ -532,8 +537,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         EntryQuarter exa, exb;
         exa.valid = exb.valid = false;
         auto entry_of = [&](int j) { return (rank + kCl * j - n_wt) * kTK + kr; };
-        if (j0 < nloc) fetch_entry(a, sidx, entry_of(j0), n_vis, row0, qt, exa);
-        if (j0 + 1 < nloc) fetch_entry(a, sidx, entry_of(j0 + 1), n_vis, row0, qt, exb);
+        if (j0 < nloc) fetch_entry(a, sidx, entry_of(j0), n_vis, b, row0, qt, exa);
+        if (j0 + 1 < nloc) fetch_entry(a, sidx, entry_of(j0 + 1), n_vis, b, row0, qt, exb);
         // converts tile j from `ex`, then issues tile j + 2's loads into it
         auto tile_step = [&](int j, EntryQuarter& ex) -> bool {
             const int kb = j % kKBuf;
@@ -568,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 *cell8(tile, kKBlk, kr, 512 + 16 * qt + 8 * u) = h;
             }
             publish(kb, vrow);
-            if (j + 2 < nloc) fetch_entry(a, sidx, entry_of(j + 2), n_vis, row0, qt, ex);
+            if (j + 2 < nloc) fetch_entry(a, sidx, entry_of(j + 2), n_vis, b, row0, qt, ex);
             return true;
         };
         for (int j = j0; j < nloc && ok; j += 2) {
@@ -894,10 +899,9 @@ cudaError_t launch_attn576_tc(const AttnArgs& aa, int Q, cudaStream_t stream) {
     A576Args a;
     a.q = aa.q;
     a.entries = aa.entries;
-    a.ent_off = aa.ent_off;
+    a.er = aa.er;
     a.kv = aa.kv;
-    a.kv_off = aa.kv_off;
-    a.kv_pos0 = aa.kv_pos0;
+    a.raw = aa.raw;
     a.q_seq = aa.q_seq;
     a.q_pos = aa.q_pos;
     a.seq_len = aa.seq_len;

@@ -83,10 +83,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct AttnTcArgs {
     const uint16_t* q;
     const uint8_t* entries;
-    const int64_t* ent_off;
+    EntryRows er;
     const uint16_t* kv;
-    const int64_t* kv_off;
-    const int64_t* kv_pos0;
+    RawRows raw;
     const int32_t* q_seq;
     const int32_t* q_pos;
     const int64_t* seq_len;
@@ -125,7 +124,7 @@ __device__ __forceinline__ bool get_item(const AttnTcArgs& a, int it, AItem& x, 
         return false;
     }
     x.n_vis = (x.t + 1) / a.m;
-    x.row0 = a.ent_off[x.b];
+    x.row0 = a.er.bt ? 0 : a.er.ent_off[x.b];   // dense reads contiguous rows only
     if (a.idx) {
         x.n_ent = a.k;
     } else {
@@ -194,7 +193,7 @@ __device__ __forceinline__ int dense_chunks(const AttnTcArgs& a, int q, int& t) 
     if (b < 0 || b >= a.B || t < 0 || (int64_t)t >= a.seq_len[b]) return 0;
     int n = (t + 1) / a.m;
     if (n > a.max_n) n = a.max_n;
-    const int64_t avail = a.ent_rows - a.ent_off[b];
+    const int64_t avail = a.ent_rows - a.er.ent_off[b];
     if ((int64_t)n > avail) n = avail > 0 ? (int)avail : 0;
     return 1 + ((n + kTK - 1) / kTK + a.chunk_tiles - 1) / a.chunk_tiles;
 }
@@ -444,8 +443,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (v < x.n_ent) {
                             const int e = sidx[v];
                             if (e >= 0) {
-                                if (e < x.n_vis && x.row0 + e < a.ent_rows) {
-                                    row = (int32_t)(x.row0 + e);
+                                const int64_t re = a.er.bt ? a.er.row(x.b, e) : x.row0 + e;
+                                if (e < x.n_vis && re >= 0 && re < a.ent_rows) {
+                                    row = (int32_t)re;
                                 } else {
                                     flag(a.st, CSA_DEV_OOB);
                                 }
@@ -650,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (i < 36 && x.tile0 == 0) {
                 // window validity words: rows r with r < n_win and w0 + r >= kv_pos0
                 const int wd = i - 32;
-                const int64_t lo64 = a.kv_pos0[x.b] - (int64_t)x.w0;
+                const int64_t lo64 = a.raw.first(x.b, a.seq_len[x.b]) - (int64_t)x.w0;
                 const int lo = lo64 > 0 ? (lo64 > kTK ? kTK : (int)lo64) : 0;
                 const int a0 = max(lo - 32 * wd, 0), a1 = min(x.n_win - 32 * wd, 32);
                 uint32_t wbits = 0;
@@ -702,14 +702,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int r = i >> 1, u = i & 1;
                 const int64_t p = (int64_t)x.w0 + r;
                 bool valid = r < x.n_win;
-                if (valid && p < a.kv_pos0[x.b]) {
+                if (valid && p < a.raw.first(x.b, a.seq_len[x.b])) {
                     valid = false;
                     flag(a.st, CSA_DEV_OOB);
                 }
                 float v[64];
                 float ss = 0.f;
                 if (valid) {
-                    const uint16_t* src = a.kv + (a.kv_off[x.b] + p - a.kv_pos0[x.b]) * kD + u * 32;
+                    const uint16_t* src = a.kv + a.raw.row(x.b, p) * kD + u * 32;
 #pragma unroll
                     for (int c = 0; c < 8; c++) {
                         const uint4 w = *reinterpret_cast<const uint4*>(src + (c >> 2) * 64 + 8 * (c & 3));
@@ -1147,10 +1147,9 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
     AttnTcArgs a;
     a.q = aa.q;
     a.entries = aa.entries;
-    a.ent_off = aa.ent_off;
+    a.er = aa.er;
     a.kv = aa.kv;
-    a.kv_off = aa.kv_off;
-    a.kv_pos0 = aa.kv_pos0;
+    a.raw = aa.raw;
     a.q_seq = aa.q_seq;
     a.q_pos = aa.q_pos;
     a.seq_len = aa.seq_len;

@@ -69,6 +69,40 @@ __device__ __forceinline__ void pdl_trigger() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Where the classical cache holds entry i of sequence b ("DeepSeek-V4 深度分析报告" 3.5: the
+// compressed entries are managed in blocks of lcm(m, m') = 128 tokens).  Without a block
+// table: row ent_off[b] + i of a contiguous per-sequence array.  With one: entry i lies in
+// the sequence's block i / E (E = 128 / m entries per block, E = 2^pe_shift), at row
+// bt[b * bt_stride + i / E] * E + i % E.
+struct EntryRows {
+    const int64_t* ent_off;
+    const int32_t* bt;       // nullable
+    int64_t bt_stride;
+    int pe_shift;
+    __device__ __forceinline__ int64_t row(int b, int64_t i) const {
+        if (!bt) return ent_off[b] + i;
+        const int64_t blk = bt[(int64_t)b * bt_stride + (i >> pe_shift)];
+        return (blk << pe_shift) + (i & ((1ll << pe_shift) - 1));
+    }
+};
+
+// Where the state cache holds raw token p of sequence b.  Linear (ring = 0): row
+// kv_off[b] + p - kv_pos0[b], positions kv_pos0[b] .. seq_len[b] - 1 stored.  Ring
+// (ring > 0): a fixed-size ring of `ring` rows per sequence, row kv_off[b] + p mod ring,
+// positions max(seq_len[b] - ring, 0) .. seq_len[b] - 1 stored.
+struct RawRows {
+    const int64_t* kv_off;
+    const int64_t* kv_pos0;  // unused with a ring
+    int64_t ring;
+    __device__ __forceinline__ int64_t first(int b, int64_t seq_len_b) const {
+        if (ring) return seq_len_b > ring ? seq_len_b - ring : 0;
+        return kv_pos0[b];
+    }
+    __device__ __forceinline__ int64_t row(int b, int64_t p) const {
+        return ring ? kv_off[b] + p % ring : kv_off[b] + p - kv_pos0[b];
+    }
+};
+
 // Order-preserving 32-bit key of a score: larger score, larger key; -0 and +0 equal.
 __device__ __forceinline__ uint32_t order_key(float s) {
     uint32_t u = __float_as_uint(s);

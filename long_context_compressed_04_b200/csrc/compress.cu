@@ -30,15 +30,14 @@ struct Chunk {
 };
 
 __device__ __forceinline__ void load_chunk(const uint16_t* __restrict__ kv,
-                                           const uint16_t* __restrict__ gate, int64_t row_first,
-                                           int64_t first_pos, int D, int c0, Chunk& ch) {
-    // row_first holds position max(first_pos, 0); positions before the sequence start
-    // (entry 0 of CSA) re-read that row and are masked out of the softmax by the caller
-    const int64_t p_first = first_pos > 0 ? first_pos : 0;
+                                           const uint16_t* __restrict__ gate, const RawRows& raw,
+                                           int b, int64_t first_pos, int D, int c0, Chunk& ch) {
+    // positions before the sequence start (entry 0 of CSA) re-read position 0's row and
+    // are masked out of the softmax by the caller
 #pragma unroll
     for (int jj = 0; jj < kChunkTok; jj++) {
         const int64_t p = first_pos + jj;
-        const int64_t row = row_first + (p >= 0 ? p - p_first : 0);
+        const int64_t row = raw.row(b, p >= 0 ? p : 0);
         ch.z[jj] = *reinterpret_cast<const uint2*>(gate + row * D + c0);
         ch.v[jj] = *reinterpret_cast<const uint2*>(kv + row * D + c0);
     }
@@ -51,10 +50,8 @@ __device__ __forceinline__ void load_chunk(const uint16_t* __restrict__ kv,
 template <int SPAN, int NCH>
 __global__ void __launch_bounds__(SPAN == 8 ? 160 : (NCH == 1 ? 512 : 640)) compress_kernel(
     const uint16_t* __restrict__ kv, const uint16_t* __restrict__ gate,
-    const float* __restrict__ bias, const int64_t* __restrict__ seq_len,
-    const int64_t* __restrict__ kv_off,
-    const int64_t* __restrict__ kv_pos0, const int64_t* __restrict__ ent_off,
-    const int32_t* __restrict__ item_seq, const int32_t* __restrict__ item_ent, int B, int m,
+    const float* __restrict__ bias, const int64_t* __restrict__ seq_len, const RawRows raw,
+    const EntryRows er, const int32_t* __restrict__ item_seq, const int32_t* __restrict__ item_ent, int B, int m,
     int D, int fmt, double log2_theta, float eps, uint8_t* __restrict__ entries,
     int32_t* __restrict__ dev_status) {
     __shared__ float red[8];
@@ -65,9 +62,8 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : (NCH == 1 ? 512 : 640)) comp
     const int64_t i = item_ent[it];
     bool ok = !(b < 0 || b >= B || i < 0);
     const int64_t first = (i + 1) * (int64_t)m - SPAN;
-    const int64_t pos0 = ok ? kv_pos0[b] : 0;
-    const int64_t row0 = ok ? kv_off[b] : 0;
-    const int64_t erow = ok ? ent_off[b] + i : 0;
+    const int64_t pos0 = ok ? raw.first(b, seq_len[b]) : 0;
+    const int64_t erow = ok ? er.row(b, i) : 0;
     // every pooled token must be stored: positions max(first, 0) .. (i+1)m-1
     if (ok && ((first > 0 ? first : 0) < pos0 || (i + 1) * (int64_t)m > seq_len[b])) ok = false;
     const int cw = 32 * ((D / 4 + 31) / 32);     // channel lanes per token group
@@ -92,10 +88,8 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : (NCH == 1 ? 512 : 640)) comp
         if constexpr (NCH == 1) return bcur[j - j_begin];
         else return *reinterpret_cast<const float4*>(bias + (int64_t)j * D + c0);
     };
-    // row of the first token of a chunk starting at pooled index j (clamped at entry 0)
-    auto chunk_row = [&](int j) { return row0 + (first + j >= 0 ? first + j : 0) - pos0; };
     if (active) {
-        load_chunk(kv, gate, chunk_row(j_begin), first + j_begin, D, c0, cur);
+        load_chunk(kv, gate, raw, b, first + j_begin, D, c0, cur);
         if constexpr (NCH == 1) {
 #pragma unroll
             for (int jj = 0; jj < kChunkTok; jj++)
@@ -112,7 +106,7 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : (NCH == 1 ? 512 : 640)) comp
 #pragma unroll 1
         for (int c = 0; c < nch; c++) {
             const int j0 = j_begin + c * kChunkTok;
-            if (c + 1 < nch) load_chunk(kv, gate, chunk_row(j0 + kChunkTok), first + j0 + kChunkTok, D, c0, nxt);
+            if (c + 1 < nch) load_chunk(kv, gate, raw, b, first + j0 + kChunkTok, D, c0, nxt);
             float cm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int jj = 0; jj < kChunkTok; jj++) {
@@ -244,11 +238,10 @@ __global__ void __launch_bounds__(SPAN == 8 ? 160 : (NCH == 1 ? 512 : 640)) comp
 }
 
 cudaError_t launch_compress(int span, const void* kv, const void* gate, const float* bias,
-                            const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
-                            const int64_t* ent_off, const int32_t* item_seq,
-                            const int32_t* item_ent, int64_t n_items, int B, int m, int D,
-                            int fmt, float theta, float eps, void* entries, int32_t* st,
-                            cudaStream_t stream) {
+                            const int64_t* seq_len, const RawRows& raw, const EntryRows& er,
+                            const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
+                            int B, int m, int D, int fmt, float theta, float eps, void* entries,
+                            int32_t* st, cudaStream_t stream) {
     if (n_items == 0) return cudaSuccess;
     const int cw = 32 * ((D / 4 + 31) / 32);        // channel lanes: 32 (D=128) or 160 (576)
     const double log2_theta = log2((double)theta);
@@ -256,19 +249,19 @@ cudaError_t launch_compress(int span, const void* kv, const void* gate, const fl
     LaunchScope scope(kKCompress, stream);
     if (span == 8) {
         return launch_pdl(compress_kernel<8, 1>, grid, dim3(cw), 0, stream, (const uint16_t*)kv,
-                          (const uint16_t*)gate, bias, seq_len, kv_off, kv_pos0, ent_off, item_seq,
-                          item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
+                          (const uint16_t*)gate, bias, seq_len, raw, er, item_seq, item_ent, B,
+                          m, D, fmt, log2_theta, eps, (uint8_t*)entries, st);
     } else {
         // token groups: 16 x 8 tokens (D=128) or 4 x 32 tokens (D=576)
         if (cw == 32)
             return launch_pdl(compress_kernel<128, 1>, grid, dim3(16 * cw), 0, stream,
-                              (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off,
-                              kv_pos0, ent_off, item_seq, item_ent, B, m, D, fmt, log2_theta, eps,
+                              (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, raw, er,
+                              item_seq, item_ent, B, m, D, fmt, log2_theta, eps,
                               (uint8_t*)entries, st);
         return launch_pdl(compress_kernel<128, 4>, grid, dim3(4 * cw), 0, stream,
-                          (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, kv_off,
-                          kv_pos0, ent_off, item_seq, item_ent, B, m, D, fmt, log2_theta, eps,
-                          (uint8_t*)entries, st);
+                          (const uint16_t*)kv, (const uint16_t*)gate, bias, seq_len, raw, er,
+                          item_seq, item_ent, B, m, D, fmt, log2_theta, eps, (uint8_t*)entries,
+                          st);
     }
     return cudaGetLastError();
 }

@@ -9,8 +9,8 @@
 // (nearest, ties to even) before it is stored and selected.
 //
 // A key row is 64 bytes of elements + 4 scale bytes, half the FP8 row: decode stays
-// HBM-bound.  The kernel has the FP8 indexer's structure (same work items, persistent CTAs,
-// 11 warps); what differs:
+// HBM-bound.  The kernel has the FP8 indexer's structure (same work items, persistent CTAs);
+// what differs:
 //   warp 0 lane 0  TMA producer: per query the heads (H_I x 64 bytes, B operand); per stage
 //                  a group of up to three 128-row key tiles (64-byte rows, 64-byte swizzle),
 //                  8 x 24 KB in flight;
@@ -18,11 +18,14 @@
 //                  32x128b broadcast to the four lane quarters) and issues
 //                  tcgen05.mma kind::mxf4.block_scale (M = 128 entries, N = H_I heads,
 //                  2 x K = 64 per tile) into one of two sets of three accumulators;
-//   warp 2         scale-factor staging: the keys' and heads' UE8M0 bytes rearranged into
-//                  the tensor cores' scale layout (row r = r0 + 32 r1: bytes at 16 r0 +
-//                  4 r1 + block) in a shared-memory ring, and the head weights per item;
-//   warps 3-10     epilogue: tcgen05.ld of one entry row per thread, the fmaf chain, the
-//                  optional BF16 rounding, the score store and the group maxima.
+//   warp 2         scale-factor staging: the keys' UE8M0 bytes copied by 4-byte cp.async
+//                  straight into the tensor cores' scale layout (row r = r0 + 32 r1: bytes
+//                  at 16 r0 + 4 r1 + block), three groups ahead; the heads' scales and the
+//                  head weights per query / item;
+//   warps 3-14     epilogue in three groups of four, group j taking tile j of every stage
+//                  group: tcgen05.ld of one entry row per thread (in halves of 32 heads),
+//                  the fmaf chain, the optional BF16 rounding, the score store and the
+//                  group maxima.
 // Every wait is bounded; a timeout aborts the CTA, drains its own copies and MMAs, frees
 // TMEM and reports CSA_DEV_TIMEOUT.
 #include "indexer_items.cuh"
@@ -43,7 +46,8 @@ constexpr int kTileBytes = kTileRows * kRowBytes;
 constexpr int kGroupBytes = kGroupTiles * kTileBytes;
 constexpr int kSfBytes = 512;            // scale factors of 128 rows x 4 blocks
 constexpr int kFirstEpiWarp = 3;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiGroups = kGroupTiles;  // epilogue warp groups: one per tile of a group
+constexpr int kEpiWarps = 4 * kEpiGroups;
 constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
 
 struct Fp4Args {
@@ -51,7 +55,7 @@ struct Fp4Args {
     const float* w;          // [Q, HI]
     const uint8_t* ksf;      // [ent_rows, 4]
     const int64_t* seq_len;
-    const int64_t* ent_off;
+    EntryRows er;
     const int32_t* q_seq;
     const int32_t* q_pos;
     float* scores;
@@ -92,6 +96,54 @@ __device__ __forceinline__ void stage_scales(uint8_t* dst, const uint8_t* src, i
         v[r1] = r < nrows ? __ldg(reinterpret_cast<const uint32_t*>(src) + r) : 0u;
     }
     *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(v[0], v[1], v[2], v[3]);
+}
+
+// Walks the CTA's groups of tiles in order (items with tiles, kGroupTiles per group).
+struct GroupCursor {
+    int ii;
+    Item x;
+    int g0;
+    bool valid;
+    template <class A>
+    __device__ __forceinline__ void seek(const A& a, const Item* items, int64_t v0, int64_t v1,
+                                         int n_my) {
+        for (; ii < n_my; ii++)
+            if (fetch_item(a, items, v0, v1, ii, x, false)) {
+                valid = true;
+                return;
+            }
+        valid = false;
+    }
+    template <class A>
+    __device__ __forceinline__ void start(const A& a, const Item* items, int64_t v0, int64_t v1,
+                                          int n_my) {
+        ii = 0;
+        g0 = 0;
+        seek(a, items, v0, v1, n_my);
+    }
+    template <class A>
+    __device__ __forceinline__ void next(const A& a, const Item* items, int64_t v0, int64_t v1,
+                                         int n_my) {
+        g0 += kGroupTiles;
+        if (g0 < x.ntiles) return;
+        g0 = 0;
+        ii++;
+        seek(a, items, v0, v1, n_my);
+    }
+};
+
+// 4-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 template <int HI>
@@ -200,11 +252,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
-                    for (int j = 0; j < gt; j++)
-                        tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k,
-                                    &full[stage], 0,
-                                    (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows));
+                    if (!a.er.bt) {
+                        mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
+                        for (int j = 0; j < gt; j++)
+                            tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k,
+                                        &full[stage], 0,
+                                        (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows));
+                    } else {
+                        int32_t rows[kGroupTiles][kTilePages];
+                        int nb = 0;
+                        for (int j = 0; j < gt; j++) nb += tile_pages(a, x, x.tile0 + g0 + j, rows[j]);
+                        mbar_arrive_expect_tx(&full[stage], (uint32_t)nb * (kPageRows * kRowBytes));
+                        for (int j = 0; j < gt; j++)
+#pragma unroll
+                            for (int p = 0; p < kTilePages; p++)
+                                if (rows[j][p] >= 0)
+                                    tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes +
+                                                    p * (kPageRows * kRowBytes),
+                                                &tmap_k, &full[stage], 0, rows[j][p]);
+                    }
                     ng++;
                     if (++stage == kStages) {
                         stage = 0;
@@ -293,53 +359,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 2) {
         // ---------------- scale staging and head weights ----------------
-        int stage = 0;
-        uint32_t ephase = 0;
-        int nq = 0, cur_q = -1, nit = 0;
+        // The keys' scale bytes go straight to their places in the tensor cores' layout by
+        // 4-byte asynchronous copies, kLookAhead groups ahead of the group whose scales are
+        // being released to the MMA thread, so that no global-load latency is serialised
+        // per group.  The heads' scales and weights are loaded when the released group is
+        // the first of its query / item.
+        constexpr int kLookAhead = 3;
+        GroupCursor iss, rel;
+        iss.start(a, items, v0, v1, n_my);
+        rel.start(a, items, v0, v1, n_my);
+        int istage = 0, rstage = 0;
+        uint32_t iphase = 0;
+        int issued = 0, released = 0;
+        int nq = 0, cur_q = -1, nit = 0, cur_ii = -1;
         bool ok = true;
-        for (int ii = 0; ii < n_my && ok; ii++) {
-            Item x;
-            if (!fetch_item(a, items, v0, v1, ii, x, lane == 0)) continue;
-            if (x.q != cur_q) {
-                const int bb = nq & 1;
-                if (!mbar_wait_warp(&sfbempty[bb], ((nq >> 1) & 1) ^ 1, abort_flag, a.st)) break;
-                stage_scales(sSfb + bb * kSfBytes, a.qsf + (int64_t)x.q * HI * 4, HI, lane);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sfbfull[bb]);
-                nq++;
-                cur_q = x.q;
-            }
-            const int slot = nit % kAux;
-            if (!mbar_wait_warp(&auxempty[slot], ((nit / kAux) & 1) ^ 1, abort_flag, a.st)) break;
-#pragma unroll
-            for (int h = lane; h < HI; h += 32) aux[slot * HI + h] = __ldg(a.w + (int64_t)x.q * HI + h);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&auxfull[slot]);
-            nit++;
-            for (int g0 = 0; g0 < x.ntiles; g0 += kGroupTiles) {
-                const int gt = min(kGroupTiles, x.ntiles - g0);
-                if (!mbar_wait_warp(&empty[stage], ephase ^ 1, abort_flag, a.st)) {
+        while (rel.valid && ok) {
+            while (iss.valid && issued - released < kLookAhead) {
+                if (!mbar_wait_warp(&empty[istage], iphase ^ 1, abort_flag, a.st)) {
                     ok = false;
                     break;
                 }
+                const int gt = min(kGroupTiles, iss.x.ntiles - iss.g0);
                 for (int j = 0; j < gt; j++) {
-                    const int64_t r0 = x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows;
-                    const int64_t left = a.ent_rows - r0;
-                    stage_scales(sSfa + (stage * kGroupTiles + j) * kSfBytes, a.ksf + r0 * 4,
-                                 left < kTileRows ? (int)(left > 0 ? left : 0) : kTileRows, lane);
+                    const int64_t e0 = (int64_t)(iss.x.tile0 + iss.g0 + j) * kTileRows;
+                    const uint32_t dst = smem_addr(sSfa + (istage * kGroupTiles + j) * kSfBytes) + 16 * lane;
+#pragma unroll
+                    for (int r1 = 0; r1 < 4; r1++) {
+                        const int64_t e = e0 + lane + 32 * r1;
+                        int64_t row = iss.x.row0 + e;
+                        if (a.er.bt) row = e < iss.x.n_vis ? a.er.row(iss.x.b, e) : -1;
+                        const bool in = row >= 0 && row < a.ent_rows;
+                        cp_async4(dst + 4 * r1, a.ksf + (in ? row : 0) * 4, in ? 4u : 0u);
+                    }
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sfafull[stage]);
-                if (++stage == kStages) {
-                    stage = 0;
-                    ephase ^= 1;
+                cp_async_commit();
+                issued++;
+                if (++istage == kStages) {
+                    istage = 0;
+                    iphase ^= 1;
                 }
+                iss.next(a, items, v0, v1, n_my);
             }
+            if (!ok) break;
+            if (rel.ii != cur_ii) {
+                // the released group is the first of its item
+                cur_ii = rel.ii;
+                if (rel.x.q != cur_q) {
+                    const int bb = nq & 1;
+                    if (!mbar_wait_warp(&sfbempty[bb], ((nq >> 1) & 1) ^ 1, abort_flag, a.st)) break;
+                    stage_scales(sSfb + bb * kSfBytes, a.qsf + (int64_t)rel.x.q * HI * 4, HI, lane);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sfbfull[bb]);
+                    nq++;
+                    cur_q = rel.x.q;
+                }
+                const int slot = nit % kAux;
+                if (!mbar_wait_warp(&auxempty[slot], ((nit / kAux) & 1) ^ 1, abort_flag, a.st)) break;
+#pragma unroll
+                for (int h = lane; h < HI; h += 32)
+                    aux[slot * HI + h] = __ldg(a.w + (int64_t)rel.x.q * HI + h);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&auxfull[slot]);
+                nit++;
+            }
+            // the released group's copies are done once at most (issued - released - 1)
+            // later groups are pending
+            const int pending = issued - released - 1;
+            if (pending >= 2) {
+                cp_async_wait<2>();
+            } else if (pending == 1) {
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfafull[rstage]);
+            released++;
+            if (++rstage == kStages) rstage = 0;
+            rel.next(a, items, v0, v1, n_my);
         }
+        // no copy of this warp may still be writing shared memory when the CTA ends
+        cp_async_wait<0>();
     } else {
-        // ---------------- epilogue (warps 3..10) ----------------
+        // ---------------- epilogue (warps 3..14) ----------------
         const int grp = (warp - kFirstEpiWarp) / 4;
         const int quarter = warp & 3;
         const int row_in_tile = quarter * 32 + lane;
@@ -376,29 +480,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pdl_wait();
                     waited = true;
                 }
-                // the two epilogue groups take alternate tiles of the running tile count
-                // (three tiles per group: 2 + 1, then 1 + 2)
-                for (int j = 0; j < gt; j++) {
-                    if (((ng * kGroupTiles + j) & 1) != grp) continue;
+                // epilogue group grp takes tile grp of the group; the accumulator row is
+                // read in halves of at most 32 heads (fewer live registers), the heads still
+                // accumulated in ascending order
+                const int j = grp;
+                if (j < gt) {
                     const int tt = g0 + j;
                     const int e = (x.tile0 + tt) * kTileRows + row_in_tile;
-                    uint32_t d[HI];
                     const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
                                            (uint32_t)((set * kGroupTiles + j) * HI);
-                    if constexpr (HI == 64) {
-                        tmem_ld64(taddr, d);
-                    } else if constexpr (HI == 32) {
-                        tmem_ld32(taddr, d);
-                    } else {
-                        tmem_ld16(taddr, d);
+                    constexpr int kHalf = HI < 32 ? HI : 32;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int h0 = 0; h0 < HI; h0 += kHalf) {
+                        uint32_t d[kHalf];
+                        if constexpr (kHalf == 32) {
+                            tmem_ld32(taddr + (uint32_t)h0, d);
+                        } else {
+                            tmem_ld16(taddr + (uint32_t)h0, d);
+                        }
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h = 0; h < kHalf; h++)
+                            acc = fmaf(ws[h0 + h], fmaxf(__uint_as_float(d[h]), 0.f), acc);
                     }
-                    tmem_ld_wait();
                     uint32_t key = 0u;
                     if (e < x.n_vis) {
-                        float acc = 0.f;
-#pragma unroll
-                        for (int h = 0; h < HI; h++)
-                            acc = fmaf(ws[h], fmaxf(__uint_as_float(d[h]), 0.f), acc);
                         if (a.bf16) acc = __bfloat162float(__float2bfloat16_rn(acc));
                         if (acc != acc) flag(a.st, CSA_DEV_NAN);
                         srow[e] = acc;
@@ -483,7 +590,7 @@ template <int HI>
 cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const Fp4Args& args,
                       cudaStream_t stream) {
     CUtensorMap mk, mq;
-    if (!make_rows64_map(&mk, kI, (uint64_t)args.ent_rows, kTileRows) ||
+    if (!make_rows64_map(&mk, kI, (uint64_t)args.ent_rows, args.er.bt ? kPageRows : kTileRows) ||
         !make_rows64_map(&mq, qI, (uint64_t)args.Q * HI, HI))
         return cudaErrorInvalidValue;
     const size_t sm = smem_bytes<HI>();
@@ -505,7 +612,7 @@ bool indexer_fp4_supported(int HI, int dI) {
 
 cudaError_t launch_indexer_fp4(const uint8_t* qI, const uint8_t* qI_sf, const float* w,
                                const uint8_t* kI, const uint8_t* kI_sf, int64_t ent_rows,
-                               const int64_t* seq_len, const int64_t* ent_off,
+                               const int64_t* seq_len, const EntryRows& er,
                                const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
                                int m, int max_n, int bf16, float* scores, int64_t ld,
                                int32_t* st, cudaStream_t stream, uint32_t* gmax, int64_t ld_g) {
@@ -515,7 +622,7 @@ cudaError_t launch_indexer_fp4(const uint8_t* qI, const uint8_t* qI_sf, const fl
     args.w = w;
     args.ksf = kI_sf;
     args.seq_len = seq_len;
-    args.ent_off = ent_off;
+    args.er = er;
     args.q_seq = q_seq;
     args.q_pos = q_pos;
     args.scores = scores;

@@ -3,8 +3,9 @@
 // virtual tile space (T = tiles of the longest query); one persistent CTA per SM takes an
 // equal contiguous range of that space and walks it as items, the pieces of the range cut
 // at query boundaries and every 8 tiles.  The argument structs of both kernels carry the
-// fields read here (seq_len, ent_off, q_seq, q_pos, ent_rows, st, Q, B, m, max_n, qtiles,
-// chunks_per_q).
+// fields read here (seq_len, er, q_seq, q_pos, ent_rows, st, Q, B, m, max_n, qtiles,
+// chunks_per_q).  With a block table (er.bt) the key rows of a tile come block by block
+// (kPageRows entries each) and are checked there; row0 is then unused.
 #pragma once
 
 #include "common.cuh"
@@ -15,9 +16,12 @@ namespace {
 constexpr int kTileRows = 128;           // entries per tile (MMA M)
 constexpr int kChunkTiles = 8;           // tiles per item at most
 constexpr int kMaxItems = 64;            // work items per CTA resolved up front
+constexpr int kPageRows = 32;            // entries per classical-cache block (128 tokens, m = 4)
+constexpr int kTilePages = kTileRows / kPageRows;
 
 struct Item {
     int q;
+    int b;
     int n_vis;
     int tile0;
     int ntiles;
@@ -64,11 +68,16 @@ __device__ __forceinline__ bool get_item(const A& a, int64_t v0, int64_t v1, int
         if (report) flag(a.st, CSA_DEV_CAPACITY);
         n = a.max_n;
     }
-    x.row0 = a.ent_off[b];
-    const int64_t avail = a.ent_rows - x.row0;
-    if ((int64_t)n > avail) {
-        if (report) flag(a.st, CSA_DEV_OOB);
-        n = avail > 0 ? (int)avail : 0;
+    x.b = b;
+    if (a.er.bt) {
+        x.row0 = 0;
+    } else {
+        x.row0 = a.er.ent_off[b];
+        const int64_t avail = a.ent_rows - x.row0;
+        if ((int64_t)n > avail) {
+            if (report) flag(a.st, CSA_DEV_OOB);
+            n = avail > 0 ? (int)avail : 0;
+        }
     }
     x.n_vis = n;
     x.tile0 = cq * kChunkTiles + lo;
@@ -86,6 +95,30 @@ __device__ __forceinline__ bool fetch_item(const A& a, const Item* items, int64_
         return x.ntiles > 0;
     }
     return get_item(a, v0, v1, ii, x, report);
+}
+
+// Rows of the kTilePages blocks of virtual tile `tile` of item x (-1: not loaded, because it
+// holds no visible entry or, flagged, its block lies outside the key store); returns the
+// number of blocks to load.
+template <class A>
+__device__ __forceinline__ int tile_pages(const A& a, const Item& x, int tile,
+                                          int32_t (&rows)[kTilePages]) {
+    int n = 0;
+#pragma unroll
+    for (int p = 0; p < kTilePages; p++) {
+        const int e = tile * kTileRows + p * kPageRows;
+        rows[p] = -1;
+        if (e >= x.n_vis) continue;
+        const int64_t blk = a.er.bt[(int64_t)x.b * a.er.bt_stride + e / kPageRows];
+        const int64_t r = blk * kPageRows;
+        if (blk < 0 || r + kPageRows > a.ent_rows) {
+            flag(a.st, CSA_DEV_OOB);
+            continue;
+        }
+        rows[p] = (int32_t)r;
+        n++;
+    }
+    return n;
 }
 
 }  // namespace

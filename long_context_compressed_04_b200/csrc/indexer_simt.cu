@@ -16,7 +16,7 @@ template <int DI>
 __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
     const uint8_t* __restrict__ qI, const float* __restrict__ qs, const float* __restrict__ w,
     const uint8_t* __restrict__ kI, const float* __restrict__ ks, int64_t ent_rows,
-    const int64_t* __restrict__ seq_len, const int64_t* __restrict__ ent_off, const int32_t* __restrict__ q_seq,
+    const int64_t* __restrict__ seq_len, const EntryRows er, const int32_t* __restrict__ q_seq,
     const int32_t* __restrict__ q_pos, int B, int HI, int m, int max_n,
     float* __restrict__ scores, int64_t ld, int32_t* __restrict__ dev_status) {
     extern __shared__ float smem[];
@@ -36,10 +36,12 @@ __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
         if (blockIdx.x == 0 && threadIdx.x == 0) flag(dev_status, CSA_DEV_CAPACITY);
         n = max_n;
     }
-    const int64_t avail = ent_rows - ent_off[b];
-    if ((int64_t)n > avail) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
-        n = avail > 0 ? (int)avail : 0;
+    if (!er.bt) {
+        const int64_t avail = ent_rows - er.ent_off[b];
+        if ((int64_t)n > avail) {
+            if (blockIdx.x == 0 && threadIdx.x == 0) flag(dev_status, CSA_DEV_OOB);
+            n = avail > 0 ? (int)avail : 0;
+        }
     }
     if ((int64_t)blockIdx.x * blockDim.x >= n) return;
     for (int x = threadIdx.x; x < HI * DI; x += blockDim.x)
@@ -49,7 +51,11 @@ __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
     __syncthreads();
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n) return;
-    const int64_t row = ent_off[b] + i;
+    const int64_t row = er.row(b, i);
+    if (row < 0 || row >= ent_rows) {   // a block outside the key store
+        flag(dev_status, CSA_DEV_OOB);
+        return;
+    }
     float kf[DI];
     const uint4* src = reinterpret_cast<const uint4*>(kI + row * DI);
 #pragma unroll
@@ -76,7 +82,7 @@ __global__ void __launch_bounds__(128) indexer_score_simt_kernel(
 cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float* w,
                                 const uint8_t* kI, const float* ks, int64_t ent_rows,
                                 const int64_t* seq_len,
-                                const int64_t* ent_off, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
+                                const EntryRows& er, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
                                 int HI, int dI, int m, int max_n, float* scores, int64_t ld,
                                 int32_t* st, cudaStream_t stream) {
     if (Q == 0 || max_n == 0) return cudaSuccess;
@@ -85,13 +91,13 @@ cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float*
     LaunchScope scope(kKIndexerSimt, stream);
     if (dI == 64) {
         return launch_pdl(indexer_score_simt_kernel<64>, grid, dim3(128), smem, stream, qI, qs, w,
-                          kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n,
+                          kI, ks, ent_rows, seq_len, er, q_seq, q_pos, B, HI, m, max_n,
                           scores, ld, st);
     } else {
         cudaFuncSetAttribute(indexer_score_simt_kernel<128>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         return launch_pdl(indexer_score_simt_kernel<128>, grid, dim3(128), smem, stream, qI, qs,
-                          w, kI, ks, ent_rows, seq_len, ent_off, q_seq, q_pos, B, HI, m, max_n,
+                          w, kI, ks, ent_rows, seq_len, er, q_seq, q_pos, B, HI, m, max_n,
                           scores, ld, st);
     }
     return cudaGetLastError();

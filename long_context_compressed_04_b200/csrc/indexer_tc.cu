@@ -54,7 +54,7 @@ struct IdxArgs {
     const float* w;
     const float* ks;
     const int64_t* seq_len;
-    const int64_t* ent_off;
+    EntryRows er;            // where entry i of sequence b lies (contiguous or block table)
     const int32_t* q_seq;
     const int32_t* q_pos;
     float* scores;
@@ -190,10 +190,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
-                    for (int j = 0; j < gt; j++)
-                        tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k, &full[stage], 0,
-                                    (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows));
+                    if (!a.er.bt) {
+                        mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
+                        for (int j = 0; j < gt; j++)
+                            tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k, &full[stage], 0,
+                                        (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows));
+                    } else {
+                        // block table: each tile in blocks of kPageRows rows (the map's box)
+                        int32_t rows[kGroupTiles][kTilePages];
+                        int nb = 0;
+                        for (int j = 0; j < gt; j++) nb += tile_pages(a, x, x.tile0 + g0 + j, rows[j]);
+                        mbar_arrive_expect_tx(&full[stage], (uint32_t)nb * (kPageRows * kDI));
+                        for (int j = 0; j < gt; j++)
+#pragma unroll
+                            for (int p = 0; p < kTilePages; p++)
+                                if (rows[j][p] >= 0)
+                                    tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes + p * (kPageRows * kDI),
+                                                &tmap_k, &full[stage], 0, rows[j][p]);
+                    }
                     ng++;
                     if (++stage == kStages) {
                         stage = 0;
@@ -289,7 +303,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < kChunkTiles * kTileRows / 32; k++) {
                 const int j = lane + 32 * k;
-                v[k] = (j < nrows && e0 + j < x.n_vis) ? __ldg(a.ks + x.row0 + e0 + j) : 0.f;
+                float vk = 0.f;
+                if (j < nrows && e0 + j < x.n_vis) {
+                    const int64_t r = a.er.bt ? a.er.row(x.b, e0 + j) : x.row0 + e0 + j;
+                    if (r >= 0 && r < a.ent_rows) vk = __ldg(a.ks + r);
+                }
+                v[k] = vk;
             }
 #pragma unroll
             for (int k = 0; k < kChunkTiles * kTileRows / 32; k++)
@@ -440,7 +459,7 @@ template <int HI>
 cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const IdxArgs& args,
                       cudaStream_t stream) {
     CUtensorMap mk, mq;
-    if (!make_rows_map(&mk, kI, (uint64_t)args.ent_rows, kTileRows) ||
+    if (!make_rows_map(&mk, kI, (uint64_t)args.ent_rows, args.er.bt ? kPageRows : kTileRows) ||
         !make_rows_map(&mq, qI, (uint64_t)args.Q * HI, HI))
         return cudaErrorInvalidValue;
     const size_t sm = smem_bytes<HI>();
@@ -461,7 +480,7 @@ bool indexer_tc_supported(int HI, int dI) {
 
 cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w,
                               const uint8_t* kI, const float* ks, int64_t ent_rows,
-                              const int64_t* seq_len, const int64_t* ent_off,
+                              const int64_t* seq_len, const EntryRows& er,
                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
                               int m, int max_n, float* scores, int64_t ld, int32_t* st,
                               cudaStream_t stream, uint32_t* gmax, int64_t ld_g) {
@@ -471,7 +490,7 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
     args.w = w;
     args.ks = ks;
     args.seq_len = seq_len;
-    args.ent_off = ent_off;
+    args.er = er;
     args.q_seq = q_seq;
     args.q_pos = q_pos;
     args.scores = scores;

@@ -59,6 +59,7 @@ enum KernelKind {
     kKCpCandidates,
     kKCpPackRows,
     kKIndexerFp4,
+    kKCacheAppend,
     kKernelKinds
 };
 
@@ -79,10 +80,9 @@ class LaunchScope {
 struct AttnArgs {
     const uint16_t* q;
     const uint8_t* entries;
-    const int64_t* ent_off;
+    EntryRows er;        // where the classical cache holds entry i of sequence b
     const uint16_t* kv;
-    const int64_t* kv_off;
-    const int64_t* kv_pos0;
+    RawRows raw;         // where the state cache holds raw token p of sequence b
     const int32_t* q_seq;
     const int32_t* q_pos;
     const int64_t* seq_len;
@@ -97,28 +97,27 @@ struct AttnArgs {
 };
 
 cudaError_t launch_compress(int span, const void* kv, const void* gate, const float* bias,
-                            const int64_t* seq_len, const int64_t* kv_off, const int64_t* kv_pos0,
-                            const int64_t* ent_off, const int32_t* item_seq,
-                            const int32_t* item_ent, int64_t n_items, int B, int m, int D,
-                            int fmt, float theta, float eps, void* entries, int32_t* st,
-                            cudaStream_t stream);
+                            const int64_t* seq_len, const RawRows& raw, const EntryRows& er,
+                            const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
+                            int B, int m, int D, int fmt, float theta, float eps, void* entries,
+                            int32_t* st, cudaStream_t stream);
 cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float* w,
                                 const uint8_t* kI, const float* ks, int64_t ent_rows,
                                 const int64_t* seq_len,
-                                const int64_t* ent_off, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
+                                const EntryRows& er, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
                                 int HI, int dI, int m, int max_n, float* scores, int64_t ld,
                                 int32_t* st, cudaStream_t stream);
 bool indexer_tc_supported(int HI, int dI);
 cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w,
                               const uint8_t* kI, const float* ks, int64_t ent_rows,
-                              const int64_t* seq_len, const int64_t* ent_off,
+                              const int64_t* seq_len, const EntryRows& er,
                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
                               int m, int max_n, float* scores, int64_t ld, int32_t* st,
                               cudaStream_t stream, uint32_t* gmax = nullptr, int64_t ld_g = 0);
 bool indexer_fp4_supported(int HI, int dI);
 cudaError_t launch_indexer_fp4(const uint8_t* qI, const uint8_t* qI_sf, const float* w,
                                const uint8_t* kI, const uint8_t* kI_sf, int64_t ent_rows,
-                               const int64_t* seq_len, const int64_t* ent_off,
+                               const int64_t* seq_len, const EntryRows& er,
                                const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
                                int m, int max_n, int bf16, float* scores, int64_t ld,
                                int32_t* st, cudaStream_t stream, uint32_t* gmax, int64_t ld_g);
@@ -146,6 +145,13 @@ cudaError_t launch_cp_pack_rows(const int32_t* idx, const int32_t* q_seq, const 
                                 const int64_t* n, const int64_t* ent_off,
                                 const uint8_t* entries, int64_t ent_rows, int row_bytes, int Q,
                                 int B, int k, uint8_t* out, int32_t* local_idx, int32_t* st,
+                                cudaStream_t stream);
+
+cudaError_t launch_cache_append(const uint16_t* kv_new, const uint16_t* gate_new,
+                                const uint8_t* kI_new, const float* ks_new, int64_t* seq_len,
+                                const RawRows& raw, const EntryRows& er, int B, int D, int dI,
+                                int m, int64_t kv_rows, int64_t ent_rows, uint16_t* kv,
+                                uint16_t* gate, uint8_t* kI, float* ks, int32_t* st,
                                 cudaStream_t stream);
 
 // Sets the thread-local message csa_last_error() returns (printf-style).

@@ -49,7 +49,8 @@ extern "C" csa_status_t lightning_indexer_topk_noalloc(
     if (Q <= 0 || scores_out != nullptr || need == 0)
         return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off,
                                       q_seq, q_pos, Q, B, H_I, d_I, m, k, max_n, idx_out,
-                                      scores_out, ld_scores, nullptr, 0, dev_status, stream);
+                                      scores_out, ld_scores, nullptr, 0, nullptr, dev_status,
+                                      stream);
     if (need > (size_t)CSA_NOALLOC_SCRATCH_BYTES) {
         csa::set_error_message("lightning_indexer_topk_noalloc: Q=%d, max_n=%d needs %zu bytes of "
                               "scratch, more than the built-in %zu",
@@ -86,5 +87,6 @@ extern "C" csa_status_t lightning_indexer_topk_noalloc(
     }
     return lightning_indexer_topk(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, ent_off, q_seq, q_pos,
                                   Q, B, H_I, d_I, m, k, max_n, idx_out, scores_out, ld_scores,
-                                  scratch, (size_t)CSA_NOALLOC_SCRATCH_BYTES, dev_status, stream);
+                                  scratch, (size_t)CSA_NOALLOC_SCRATCH_BYTES, nullptr, dev_status,
+                                  stream);
 }

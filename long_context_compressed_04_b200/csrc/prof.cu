@@ -53,7 +53,7 @@ const char* kernel_name(int kind) {
                                               "attn_simt", "indexer_score_tc", "attn_tc",
                                               "attn_combine", "attn576_tc", "topk_merge",
                                               "cp_candidates", "cp_pack_rows",
-                                              "indexer_score_fp4"};
+                                              "indexer_score_fp4", "cache_append"};
     return (kind >= 0 && kind < kKernelKinds) ? names[kind] : "?";
 }
 

@@ -106,8 +106,12 @@ def attend(wl: Workload, buf: Buffers, stream=None):
 
 
 def step(wl: Workload, buf: Buffers, item_seq, item_ent, stream=None):
-    """One pass of the hot path: compress the listed entries, select (CSA), attend."""
+    """One pass of the hot path: compress the listed entries, select (CSA; the MXFP4
+    indexer when the workload carries MXFP4 inputs), attend."""
     compress(wl, buf, item_seq, item_ent, stream)
-    if wl.H_I:
+    if wl.H_I and wl.kI4 is not None:
+        indexer_topk_mxfp4(wl, (wl.qI4, wl.qsf4, wl.kI4, wl.ksf4), buf,
+                           select_bf16=wl.select_bf16, stream=stream)
+    elif wl.H_I:
         indexer_topk(wl, buf, stream=stream)
     attend(wl, buf, stream)

@@ -62,6 +62,12 @@ class Workload:
     qI: Optional[torch.Tensor] = None   # [Q, H_I, d_I] uint8
     qs: Optional[torch.Tensor] = None   # [Q, H_I] fp32
     w: Optional[torch.Tensor] = None    # [Q, H_I] fp32
+    # MXFP4 indexer inputs (instead of kI / ks / qI / qs when set; see mxfp4_indexer)
+    kI4: Optional[torch.Tensor] = None   # [ent_rows, d_I / 2] uint8 (packed e2m1)
+    ksf4: Optional[torch.Tensor] = None  # [ent_rows, d_I / 32] uint8 (UE8M0)
+    qI4: Optional[torch.Tensor] = None   # [Q, H_I, d_I / 2] uint8
+    qsf4: Optional[torch.Tensor] = None  # [Q, H_I, d_I / 32] uint8
+    select_bf16: bool = False            # MXFP4 path: select on BF16-rounded scores
     theta: float = 10000.0
     eps: float = 1e-6
 

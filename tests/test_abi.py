@@ -51,30 +51,30 @@ def test_null_and_unsupported_arguments_fail_on_host():
     fake = P(4096)  # never dereferenced: validation fails before any launch
     # null pointers
     st = lib.csa_compress(None, None, None, None, None, None, None, None, None, 4, 1, 128, 0, 10000.0,
-                          1e-6, None, None, None)
+                          1e-6, None, None, None, None)
     assert st == 1 and b"null" in lib.csa_last_error()
     # n_items = 0 is a no-op even with null pointers
     assert lib.csa_compress(None, None, None, None, None, None, None, None, None, 0, 1, 128, 0,
-                            10000.0, 1e-6, None, None, None) == 0
+                            10000.0, 1e-6, None, None, None, None) == 0
     # unsupported head dim
     st = lib.csa_compress(fake, fake, fake, fake, fake, fake, fake, fake, fake, 4, 1, 96, 0, 10000.0,
-                          1e-6, fake, None, None)
+                          1e-6, fake, None, None, None)
     assert st == 2 and b"head dim" in lib.csa_last_error()
     # misaligned
     st = lib.hca_compress(P(4097), fake, fake, fake, fake, fake, fake, fake, fake, 4, 1, 128, 0,
-                          10000.0, 1e-6, fake, None, None)
+                          10000.0, 1e-6, fake, None, None, None)
     assert st == 1 and b"aligned" in lib.csa_last_error()
     # fp8 format needs D = 576
     st = lib.sparse_mqa_attn(fake, fake, 1, 10, fake, fake, fake, fake, fake, fake, fake, fake, 8, 4, fake,
-                             1, 1, 16, 128, 128, 0.08, 10000.0, 1e-6, fake, None, None)
+                             1, 1, 16, 128, 128, 0.08, 10000.0, 1e-6, fake, None, None, None)
     assert st == 2
     # window above 128
     st = lib.sparse_mqa_attn(fake, fake, 0, 10, fake, fake, fake, fake, fake, fake, fake, fake, 8, 4, fake,
-                             1, 1, 16, 128, 129, 0.08, 10000.0, 1e-6, fake, None, None)
+                             1, 1, 16, 128, 129, 0.08, 10000.0, 1e-6, fake, None, None, None)
     assert st == 1 and b"window" in lib.csa_last_error()
     # unsupported heads
     st = lib.dense_hca_attn(fake, fake, 0, 10, fake, fake, fake, fake, fake, fake, fake, 128, fake, 1, 1, 48,
-                            128, 128, 0.08, 10000.0, 1e-6, 10, fake, fake, 1 << 20, None, None)
+                            128, 128, 0.08, 10000.0, 1e-6, 10, fake, fake, 1 << 20, None, None, None)
     assert st == 2
 
 
@@ -84,11 +84,11 @@ def test_workspace_is_checked_on_host():
     fake = P(4096)
     need = lib.csa_indexer_workspace_size(2, 1000, 64)
     st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, 100, fake, fake, fake, fake, 2, 2, 4, 64,
-                                    4, 64, 1000, fake, None, 0, fake, need - 1, None, None)
+                                    4, 64, 1000, fake, None, 0, fake, need - 1, None, None, None)
     assert st == 4 and b"workspace" in lib.csa_last_error()
     st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, 100, fake, fake, fake, fake, 2, 2, 4, 64,
-                                    4, 4096, 1000, fake, None, 0, fake, need, None, None)
+                                    4, 4096, 1000, fake, None, 0, fake, need, None, None, None)
     assert st == 2 and b"k =" in lib.csa_last_error()
     st = lib.lightning_indexer_topk(fake, fake, fake, fake, fake, 100, fake, fake, fake, fake, 2, 2, 80, 64,
-                                    4, 64, 1000, fake, None, 0, fake, need, None, None)
+                                    4, 64, 1000, fake, None, 0, fake, need, None, None, None)
     assert st == 2
