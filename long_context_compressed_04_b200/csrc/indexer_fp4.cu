@@ -146,7 +146,9 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <int HI>
+// PAGED: the key rows come through the block table (a separate instantiation, so the
+// contiguous kernel carries no block-table code).
+template <int HI, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_fp4_kernel(const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_q, const Fp4Args a) {
@@ -252,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    if (!a.er.bt) {
+                    if constexpr (!PAGED) {
                         mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
                         for (int j = 0; j < gt; j++)
                             tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k,
@@ -383,13 +385,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < gt; j++) {
                     const int64_t e0 = (int64_t)(iss.x.tile0 + iss.g0 + j) * kTileRows;
                     const uint32_t dst = smem_addr(sSfa + (istage * kGroupTiles + j) * kSfBytes) + 16 * lane;
+                    if constexpr (!PAGED) {
 #pragma unroll
-                    for (int r1 = 0; r1 < 4; r1++) {
-                        const int64_t e = e0 + lane + 32 * r1;
-                        int64_t row = iss.x.row0 + e;
-                        if (a.er.bt) row = e < iss.x.n_vis ? a.er.row(iss.x.b, e) : -1;
-                        const bool in = row >= 0 && row < a.ent_rows;
-                        cp_async4(dst + 4 * r1, a.ksf + (in ? row : 0) * 4, in ? 4u : 0u);
+                        for (int r1 = 0; r1 < 4; r1++) {
+                            const int64_t row = iss.x.row0 + e0 + lane + 32 * r1;
+                            const bool in = row < a.ent_rows;
+                            cp_async4(dst + 4 * r1, a.ksf + (in ? row : 0) * 4, in ? 4u : 0u);
+                        }
+                    } else {
+                        int64_t rows[4];
+#pragma unroll
+                        for (int r1 = 0; r1 < 4; r1++) {
+                            const int64_t e = e0 + lane + 32 * r1;
+                            rows[r1] = e < iss.x.n_vis ? a.er.row(iss.x.b, e) : -1;
+                        }
+#pragma unroll
+                        for (int r1 = 0; r1 < 4; r1++) {
+                            const bool in = rows[r1] >= 0 && rows[r1] < a.ent_rows;
+                            cp_async4(dst + 4 * r1, a.ksf + (in ? rows[r1] : 0) * 4, in ? 4u : 0u);
+                        }
                     }
                 }
                 cp_async_commit();
@@ -594,13 +608,14 @@ cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const Fp4Args& args,
         !make_rows64_map(&mq, qI, (uint64_t)args.Q * HI, HI))
         return cudaErrorInvalidValue;
     const size_t sm = smem_bytes<HI>();
-    cudaError_t e = cudaFuncSetAttribute(indexer_fp4_kernel<HI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    auto kernel = args.er.bt ? indexer_fp4_kernel<HI, true> : indexer_fp4_kernel<HI, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sm);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (int64_t)args.Q * args.qtiles;
     const int grid = (int)(tiles < (int64_t)sm_count_fp4() ? tiles : (int64_t)sm_count_fp4());
     LaunchScope scope(kKIndexerFp4, stream);
-    return launch_pdl(indexer_fp4_kernel<HI>, dim3(grid), dim3(kThreads), sm, stream, mk, mq,
+    return launch_pdl(kernel, dim3(grid), dim3(kThreads), sm, stream, mk, mq,
                       args);
 }
 

@@ -84,7 +84,9 @@ __host__ __device__ constexpr int aux_floats() {
     return HI + kChunkTiles * kTileRows;
 }
 
-template <int HI>
+// PAGED: the key rows come through the block table (a separate instantiation, so the
+// contiguous kernel carries no block-table code).
+template <int HI, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_q, const IdxArgs a) {
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         break;
                     }
-                    if (!a.er.bt) {
+                    if constexpr (!PAGED) {
                         mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
                         for (int j = 0; j < gt; j++)
                             tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k, &full[stage], 0,
@@ -300,15 +302,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int64_t e0 = (int64_t)x.tile0 * kTileRows;
             const int nrows = x.ntiles * kTileRows;
             float v[kChunkTiles * kTileRows / 32];
+            if constexpr (!PAGED) {
 #pragma unroll
-            for (int k = 0; k < kChunkTiles * kTileRows / 32; k++) {
-                const int j = lane + 32 * k;
-                float vk = 0.f;
-                if (j < nrows && e0 + j < x.n_vis) {
-                    const int64_t r = a.er.bt ? a.er.row(x.b, e0 + j) : x.row0 + e0 + j;
-                    if (r >= 0 && r < a.ent_rows) vk = __ldg(a.ks + r);
+                for (int k = 0; k < kChunkTiles * kTileRows / 32; k++) {
+                    const int j = lane + 32 * k;
+                    v[k] = (j < nrows && e0 + j < x.n_vis) ? __ldg(a.ks + x.row0 + e0 + j) : 0.f;
                 }
-                v[k] = vk;
+            } else {
+                // block table: the rows of the item's blocks first (one per 32 entries), then
+                // every scale load in flight at once
+                int64_t r[kChunkTiles * kTileRows / 32];
+#pragma unroll
+                for (int k = 0; k < kChunkTiles * kTileRows / 32; k++) {
+                    const int j = lane + 32 * k;
+                    r[k] = (j < nrows && e0 + j < x.n_vis) ? a.er.row(x.b, e0 + j) : -1;
+                }
+#pragma unroll
+                for (int k = 0; k < kChunkTiles * kTileRows / 32; k++)
+                    v[k] = (r[k] >= 0 && r[k] < a.ent_rows) ? __ldg(a.ks + r[k]) : 0.f;
             }
 #pragma unroll
             for (int k = 0; k < kChunkTiles * kTileRows / 32; k++)
@@ -463,13 +474,14 @@ cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const IdxArgs& args,
         !make_rows_map(&mq, qI, (uint64_t)args.Q * HI, HI))
         return cudaErrorInvalidValue;
     const size_t sm = smem_bytes<HI>();
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<HI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    auto kernel = args.er.bt ? indexer_tc_kernel<HI, true> : indexer_tc_kernel<HI, false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sm);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (int64_t)args.Q * args.qtiles;
     const int grid = (int)(tiles < (int64_t)num_sms() ? tiles : (int64_t)num_sms());
     LaunchScope scope(kKIndexerTc, stream);
-    return launch_pdl(indexer_tc_kernel<HI>, dim3(grid), dim3(kThreads), sm, stream, mk, mq, args);
+    return launch_pdl(kernel, dim3(grid), dim3(kThreads), sm, stream, mk, mq, args);
 }
 
 }  // namespace
