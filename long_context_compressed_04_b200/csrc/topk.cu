@@ -254,7 +254,8 @@ __device__ __forceinline__ uint32_t select_kth_raw(const uint32_t* list, uint32_
 // (the group keys and the list of groups reaching the bound, later the selection words),
 // then cap candidate keys and cap candidate entries.
 __host__ __device__ constexpr size_t group_smem_bytes(int max_n, int cap) {
-    return (size_t)((2 * ((max_n + 31) / 32) + 3) / 4) * 16 + (size_t)cap * 8;
+    // group keys and list, candidates (key, entry), then the output words (2 x 2k = cap)
+    return (size_t)((2 * ((max_n + 31) / 32) + 3) / 4) * 16 + (size_t)cap * 12;
 }
 
 // OR / AND of `v` over the CTA into or_and[0] / or_and[1] (initialised by the caller before
@@ -278,10 +279,11 @@ __device__ __forceinline__ void block_or_and(uint32_t o, uint32_t a, uint32_t* o
 // each hold an entry whose key is >= B.  So the top-k are among the entries >= B, and those
 // lie in the groups whose key is >= B (about k of them): only those groups' scores are
 // read.  The entries >= B are listed (at least k of them; the call returns false, with
-// nothing written, when more than cap), the k-th largest key T is selected among them, and
-// the selection -- every entry > T and the lowest-indexed ties -- is written in ascending
-// entry order from bit words of 32 entries.  The result is the unique top-k under the tie
-// order.  All 1024 threads call it (for G >= 2k); dyn holds group_smem_bytes(n, cap) bytes.
+// nothing written, when more than cap, or when more than 2k groups reach B), the k-th
+// largest key T is selected among them, and the selection -- every entry > T and the
+// lowest-indexed ties -- is written in ascending entry order from bit words over the
+// listed groups.  The result is the unique top-k under the tie order.  All 1024 threads
+// call it (for G >= 2k); dyn holds group_smem_bytes(n, cap) bytes.
 __device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
                                const uint32_t* __restrict__ qg, int n, int k, int cap,
                                int32_t* __restrict__ out, uint8_t* dyn, Shared& sh) {
@@ -312,18 +314,40 @@ __device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
     uint32_t krem;
     const uint32_t B = select_kth_raw(gk, (uint32_t)G, (uint32_t)k, sh.cor[0], sh.cor[1], krem,
                                       sh.hist, sh.scan_tmp, &sh.bin, &sh.krem, 2);
-    // 3. the groups reaching B (any order)
-    for (int g0 = 0; g0 < G; g0 += kThreads) {
-        const int g = g0 + tid;
-        const bool pass = g < G && gk[g] >= B;
-        const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-        uint32_t base = 0u;
-        if (lane == 0 && bal) base = atomicAdd(&sh.ngrp, (uint32_t)__popc(bal));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (pass) glist[base + __popc(bal & lanemask_lt())] = (uint32_t)g;
+    // 3. the groups reaching B, in ascending order: each thread a contiguous run of groups,
+    // placed by one block scan (the output below walks them in this order)
+    {
+        // runs of a multiple of 4 groups, read as 16-byte vectors (gk is 16-byte aligned)
+        const int per = ((G + kThreads - 1) / kThreads + 3) & ~3;
+        const int g0 = tid * per, g1 = min(G, g0 + per);
+        uint32_t cnt = 0u;
+        for (int g = g0; g < g1; g += 4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(gk + g);
+            cnt += (v.x >= B) + (g + 1 < g1 && v.y >= B) + (g + 2 < g1 && v.z >= B) +
+                   (g + 3 < g1 && v.w >= B);
+        }
+        unsigned long long tot;
+        uint32_t pos = (uint32_t)block_exclusive_scan64(cnt, sh.scan64, tot);
+        // the list, and in gk (no longer needed) each listed group's position in it
+        for (int g = g0; g < g1; g += 4) {
+            const uint4 v = *reinterpret_cast<const uint4*>(gk + g);
+            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int z = 0; z < 4; z++)
+                if (g + z < g1 && vv[z] >= B) {
+                    glist[pos] = (uint32_t)(g + z);
+                    gk[g + z] = pos++;
+                }
+        }
+        if (tid == 0) sh.ngrp = (uint32_t)tot;
+        __syncthreads();
     }
-    __syncthreads();
     const uint32_t ng = sh.ngrp;
+    // the output words below cover the listed groups only: more than 2k of them (massive
+    // ties among the group keys) take the full row instead
+    if (ng > 2u * (uint32_t)k) return false;
+    if (tid == 0) sh.nsel = 0u;
+    __syncthreads();
     // 4. their entries reaching B: 8 slots of 4 entries per group, up to 4 slots per thread
     // with all of their loads in flight; each thread's passing entries are placed by one
     // warp scan and one shared atomic per warp
@@ -385,50 +409,56 @@ __device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
     block_or_and(kor, kand, sh.cor);
     const uint32_t T = select_kth_raw(ckey, c, (uint32_t)k, sh.cor[0], sh.cor[1], krem,
                                       sh.hist, sh.scan_tmp, &sh.bin, &sh.krem);
-    // 6. selection words over the row (over the group keys and list, no longer needed)
-    const int nw = G;
-    uint32_t* selw = gk;
-    uint32_t* tiew = gk + nw;
-    for (int w = tid; w < 2 * nw; w += kThreads) selw[w] = 0u;
+    // 6. selection words over the listed groups (ascending): bit e & 31 of word gk[e >> 5]
+    // for every candidate > T (selw) or == T (tiew); each thread a contiguous run of words,
+    // placed by one block scan of (selected, tied) counts, every entry > T and the first
+    // krem ties written in ascending entry order
+    uint32_t* selw = cent + cap;
+    uint32_t* tiew = selw + 2 * k;
+    for (uint32_t w = tid; w < ng; w += kThreads) {
+        selw[w] = 0u;
+        tiew[w] = 0u;
+    }
     __syncthreads();
     for (uint32_t i = tid; i < c; i += kThreads) {
         const uint32_t key = ckey[i], e = cent[i];
-        if (key > T) atomicOr(&selw[e >> 5], 1u << (e & 31));
-        else if (key == T) atomicOr(&tiew[e >> 5], 1u << (e & 31));
+        if (key > T) atomicOr(&selw[gk[e >> 5]], 1u << (e & 31));
+        else if (key == T) atomicOr(&tiew[gk[e >> 5]], 1u << (e & 31));
     }
     __syncthreads();
-    // each thread a contiguous run of words: its counts of selected and tied entries; the
-    // CTA's prefix gives its output position and the ties before it
-    const int per = (nw + kThreads - 1) / kThreads;
-    const int w0 = tid * per, w1 = min(nw, w0 + per);
-    uint32_t cs = 0u, ct = 0u;
-    for (int w = w0; w < w1; w++) {
-        cs += __popc(selw[w]);
-        ct += __popc(tiew[w]);
-    }
-    unsigned long long tot;
-    const unsigned long long pre =
-        block_exclusive_scan64(((unsigned long long)cs << 32) | ct, sh.scan64, tot);
-    uint32_t ties = (uint32_t)pre;
-    uint32_t pos = (uint32_t)(pre >> 32) + min(ties, krem);
-    for (int w = w0; w < w1; w++) {
-        const uint32_t sw = selw[w], tw = tiew[w];
-        uint32_t take_t = 0u;
-        if (ties < krem) {
-            uint32_t need = krem - ties, tt = tw;
-            while (need && tt) {
-                take_t |= tt & (0u - tt);
-                tt &= tt - 1u;
-                need--;
-            }
+    {
+        const uint32_t per = (ng + kThreads - 1) / kThreads;
+        const uint32_t w0 = (uint32_t)tid * per, w1 = min(ng, w0 + per);
+        uint32_t cs = 0u, ct = 0u;
+        for (uint32_t w = w0; w < w1; w++) {
+            cs += __popc(selw[w]);
+            ct += __popc(tiew[w]);
         }
-        ties += __popc(tw);
-        uint32_t take = sw | take_t;
-        while (take) {
-            const int bit = __ffs(take) - 1;
-            if (pos < (uint32_t)k) out[pos] = (w << 5) + bit;
-            pos++;
-            take &= take - 1;
+        unsigned long long tot;
+        const unsigned long long pre =
+            block_exclusive_scan64(((unsigned long long)cs << 32) | ct, sh.scan64, tot);
+        uint32_t ties = (uint32_t)pre;
+        uint32_t pos = (uint32_t)(pre >> 32) + min(ties, krem);
+        for (uint32_t w = w0; w < w1; w++) {
+            const uint32_t sw = selw[w], tw = tiew[w];
+            uint32_t take_t = 0u;
+            if (ties < krem) {
+                uint32_t need = krem - ties, tt = tw;
+                while (need && tt) {
+                    take_t |= tt & (0u - tt);
+                    tt &= tt - 1u;
+                    need--;
+                }
+            }
+            ties += __popc(tw);
+            uint32_t take = sw | take_t;
+            const int32_t base = (int32_t)(glist[w] << 5);
+            while (take) {
+                const int bit = __ffs(take) - 1;
+                if (pos < (uint32_t)k) out[pos] = base + bit;
+                pos++;
+                take &= take - 1;
+            }
         }
     }
     return true;
