@@ -53,16 +53,25 @@ WORKLOADS = {
 }
 
 
-# DRAM traffic (read + write, bytes per launch) of the dominant kernel from the ncu capture
-# summarised in profiles/csa_decode_1m_b8_fp8_launch_list.md, valid only while the kernel's
+# DRAM traffic (read + write, bytes per launch) of the dominant kernel from the ncu captures
+# summarised in profiles/ (the launch lists of the two 1M workloads), valid only while the kernel's
 # sources are byte-identical to the ones captured (sha256 of the files, first 16 hex digits).
 MEASURED_TRAFFIC = {
     ("csa_decode_1m_b8_fp8", "indexer_score_tc"): {
-        "bytes": 285_380_352,
+        "bytes": 285_230_336,
         "files": ["long_context_compressed_04_b200/csrc/indexer_tc.cu",
+                  "long_context_compressed_04_b200/csrc/indexer_items.cuh",
                   "long_context_compressed_04_b200/csrc/sm100.cuh",
                   "long_context_compressed_04_b200/csrc/common.cuh"],
-        "sha": "966246eaff27f9b4",
+        "sha": "d2050d6bbec42dc8",
+    },
+    ("csa_decode_1m_b8_mxfp4", "indexer_score_fp4"): {
+        "bytes": 148_762_112,
+        "files": ["long_context_compressed_04_b200/csrc/indexer_fp4.cu",
+                  "long_context_compressed_04_b200/csrc/indexer_items.cuh",
+                  "long_context_compressed_04_b200/csrc/sm100.cuh",
+                  "long_context_compressed_04_b200/csrc/common.cuh"],
+        "sha": "cee81c6696c8ce35",
     },
 }
 
