@@ -534,10 +534,10 @@ def measure(name: str, args, dist, dev, rank: int, world: int, full: bool):
     step_s = ms_max / K / 1e3
     # the dominant kernel is the one that moves the method's dominant bytes: the indexer
     # (every visible key, each step) for CSA decode, the attention (every entry) for HCA
-    alg_of = {"indexer_score_tc": key_bytes, "indexer_score_simt": key_bytes,
+    alg_of = {"indexer_score_tc": key_bytes,
               "indexer_score_fp4": key_bytes,
               "attn_tc": total_bytes - key_bytes, "attn_simt": total_bytes - key_bytes}
-    dom_name = next((n for n in (["indexer_score_tc", "indexer_score_fp4", "indexer_score_simt"]
+    dom_name = next((n for n in (["indexer_score_tc", "indexer_score_fp4"]
                                  if wl.H_I else [])
                      + ["attn_tc", "attn_simt"] if n in per_kernel), None)
     roof = None

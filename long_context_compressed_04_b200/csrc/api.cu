@@ -231,17 +231,11 @@ csa_status_t lightning_indexer_topk(const uint8_t* qI, const float* qI_scale, co
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     uint32_t* gmax = nullptr;
-    if (csa::indexer_tc_supported(H_I, d_I)) {
-        if (workspace && workspace_bytes >= L.gmax_bytes && aligned(workspace, 256))
-            gmax = (uint32_t*)workspace;
-        e = csa::launch_indexer_tc(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, er,
-                                   q_seq, q_pos, Q, B, H_I, m, max_n, scores, ld, dev_status, s,
-                                   gmax, L.ld_g);
-    } else {
-        e = csa::launch_indexer_simt(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, er,
-                                     q_seq, q_pos, Q, B, H_I, d_I, m, max_n, scores, ld,
-                                     dev_status, s);
-    }
+    // every supported shape runs on the tensor cores (head counts padded to 16, 32 or 64)
+    if (workspace && workspace_bytes >= L.gmax_bytes && aligned(workspace, 256))
+        gmax = (uint32_t*)workspace;
+    e = csa::launch_indexer_tc(qI, qI_scale, w, kI, kI_scale, ent_rows, seq_len, er, q_seq, q_pos,
+                               Q, B, H_I, d_I, m, max_n, scores, ld, dev_status, s, gmax, L.ld_g);
     if (e != cudaSuccess) return cuda_status(e, "indexer launch");
     e = csa::launch_topk(scores, ld, q_seq, q_pos, seq_len, Q, B, m, max_n, k, idx_out, dev_status,
                          s, gmax, L.ld_g);

@@ -100,6 +100,7 @@ struct AttnTcArgs {
     // dense only: 0 = the chunks of a query spread over CTAs, combined by
     // attn_combine_kernel; 1 = one CTA takes all chunks of a query and combines them itself
     int single;
+    int hreal;            // query heads of the call (16 or 64): heads >= hreal are zero padding
     float scale_log2;
     float eps;
     double log2_theta;
@@ -618,10 +619,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 pdl_wait();
                 waited_prev = true;
             }
-            for (int u = i; u < kH * (kD / 2); u += 256) {
+            for (int u = i; u < a.hreal * (kD / 2); u += 256) {
                 const int hh = u / (kD / 2), d = 2 * (u % (kD / 2));
                 const float2 o = combine_pair(a, q, t, nch, hh, d);
-                *reinterpret_cast<uint32_t*>(a.out + ((int64_t)q * kH + hh) * kD + d) = pack_bf16x2(o.x, o.y);
+                *reinterpret_cast<uint32_t*>(a.out + ((int64_t)q * a.hreal + hh) * kD + d) = pack_bf16x2(o.x, o.y);
             }
         };
         for (int ii = 0;; ii++) {
@@ -661,11 +662,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 // q head hq, channels u*32 .. u*32+31 (RoPE on the last 64: u = 2, 3)
                 const int hq = i >> 2, u = i & 3;
-                const uint16_t* src = a.q + ((int64_t)x.q * kH + hq) * kD + u * 32;
+                // heads past the call's (16-head calls padded to the 64-head tile) are zero
+                const bool hv = hq < a.hreal;
+                const uint16_t* src = a.q + ((int64_t)x.q * a.hreal + (hv ? hq : 0)) * kD + u * 32;
                 float v[32];
 #pragma unroll
                 for (int c = 0; c < 4; c++) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(src + 8 * c);
+                    const uint4 w = hv ? *reinterpret_cast<const uint4*>(src + 8 * c)
+                                       : make_uint4(0u, 0u, 0u, 0u);
                     const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                     for (int z = 0; z < 4; z++) {
@@ -764,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float sk_mine = -INFINITY;
             if (a.idx) {
                 const int h0 = x.c * kH / a.cluster, h1 = (x.c + 1) * kH / a.cluster;
-                if (i < h1 - h0) sk_mine = a.sink[h0 + i] * kLog2e;
+                if (i < h1 - h0) sk_mine = h0 + i < a.hreal ? a.sink[h0 + i] * kLog2e : -INFINITY;
             }
             // ---- running state of (head h, column-half ch) ----
             // the chunk's own keys only: the sink enters when the partial states are combined.
@@ -999,8 +1003,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             acc = make_float4(acc.x * c0 + acc.y * s0, acc.y * c0 - acc.x * s0,
                                               acc.z * c1 + acc.w * s1, acc.w * c1 - acc.z * s1);
                         }
-                        *reinterpret_cast<uint2*>(a.out + ((int64_t)x.q * kH + h0 + lh) * kD + c4) =
-                            make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+                        if (h0 + lh < a.hreal)
+                            *reinterpret_cast<uint2*>(a.out + ((int64_t)x.q * a.hreal + h0 + lh) * kD + c4) =
+                                make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
                     }
                     // every thread's reads of the receive buffer are done; then it may take
                     // the next query's partials
@@ -1049,9 +1054,9 @@ __global__ void __launch_bounds__(kD / 2) attn_combine_kernel(const AttnTcArgs a
     const int nch = dense_chunks(a, q, t);
     pdl_wait();   // chunk partials come from the attention kernel
     pdl_trigger();
-    if (nch == 0) return;
+    if (nch == 0 || h >= a.hreal) return;
     const float2 o = combine_pair(a, q, t, nch, h, d);
-    *reinterpret_cast<uint32_t*>(a.out + ((int64_t)q * kH + h) * kD + d) = pack_bf16x2(o.x, o.y);
+    *reinterpret_cast<uint32_t*>(a.out + ((int64_t)q * a.hreal + h) * kD + d) = pack_bf16x2(o.x, o.y);
 }
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -1135,7 +1140,10 @@ int dense_chunks_per_q(int max_n) {
 
 }  // namespace
 
-bool attn_tc_supported(int H, int D, int fmt) { return H == kH && D == kD && fmt == CSA_KV_BF16; }
+// 16-head calls run on the 64-head tile, the other heads zero (their outputs are not stored)
+bool attn_tc_supported(int H, int D, int fmt) {
+    return (H == kH || H == 16) && D == kD && fmt == CSA_KV_BF16;
+}
 
 size_t attn_tc_workspace_bytes(int Q, int max_n) {
     return (size_t)Q * dense_chunks_per_q(max_n) * kH * (kD + 2) * sizeof(float);
@@ -1168,6 +1176,7 @@ cudaError_t launch_attn_tc(const AttnArgs& aa, int Q, int max_n, void* workspace
     a.scale_log2 = aa.scale * kLog2e;
     a.eps = aa.eps;
     a.log2_theta = aa.log2_theta;
+    a.hreal = aa.H;
     if (aa.idx) {
         a.cluster = sparse_cluster(aa.k);
         a.chunk_tiles = 0;   // ranks take their tiles by rank

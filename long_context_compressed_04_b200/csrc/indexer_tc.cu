@@ -12,18 +12,22 @@
 // items: the pieces of the range cut at query boundaries and every 8 tiles.  Every entry
 // is always computed in the same tile row by the same instructions whatever the batch.
 // Roles per CTA (11 warps):
-//   warp 0 lane 0  TMA producer: per query the heads (H_I x 128 e4m3, B operand, reused
+//   warp 0 lane 0  TMA producer: per query the heads (H_I x d_I e4m3, B operand, reused
 //                  across consecutive items of the query); per stage a group of up to four
-//                  tiles of 128 key rows (A operand), 128-byte swizzle, 3 x 64 KB ring; it
-//                  decodes its items itself and starts before the others' item table;
+//                  tiles of 128 key rows (A operand), 128-byte swizzle for d_I = 128 and
+//                  64-byte swizzle for d_I = 64, a 3-stage ring; it decodes its items itself
+//                  and starts before the others' item table;
 //   warp 1         TMEM allocation; lane 0 issues tcgen05.mma kind::f8f6f4 (M=128 entries,
-//                  N=H_I heads, 4 x K=32 per tile) into one of two sets of four TMEM
+//                  N=H_I heads, d_I / 32 x K=32 per tile) into one of two sets of four TMEM
 //                  accumulators, the K steps of the group's tiles interleaved;
 //   warp 2         item prefetch: w_h * qs_h of the item's query and the key scales of
 //                  its tiles into a shared-memory ring, ahead of the epilogue;
 //   warps 3-10     epilogue in two groups of four taking alternate tiles of a group:
 //                  tcgen05.ld of one entry row (all heads) per thread, the fixed-order fmaf
 //                  chain, the key scale, a coalesced score store.
+// Head counts below 16, 32 or 64 run on the next of those MMA widths: the padded heads'
+// rows of the B operand are zero and their weights w_h * qs_h are zero, so each adds an
+// exact +0 to the fmaf chain and the scores keep their bits.
 // Barriers are per group of tiles, not per tile: under load every mbarrier operation costs
 // the single issuing thread on the order of a hundred cycles.
 // Every wait is bounded; a timeout aborts the CTA, drains its own copies and MMAs,
@@ -42,9 +46,6 @@ constexpr int kGroupTiles = 4;           // tiles per pipeline stage (one barrie
 constexpr int kStages = 3;               // 3 x 64 KB of key tiles in flight per SM
 constexpr int kAccSets = 2;              // TMEM accumulator sets of kGroupTiles accumulators
 constexpr int kAux = 3;                  // prefetched items
-constexpr int kDI = 128;                 // indexer dim (MMA K total, bytes per key row)
-constexpr int kTileBytes = kTileRows * kDI;
-constexpr int kGroupBytes = kGroupTiles * kTileBytes;
 constexpr int kFirstEpiWarp = 3;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (kFirstEpiWarp + kEpiWarps);
@@ -62,6 +63,7 @@ struct IdxArgs {
     int64_t ent_rows;
     int32_t* st;
     int Q, B, m, max_n;
+    int hreal;               // heads of the call (<= HI; the rest are zero padding)
     int qtiles;              // virtual tiles per query: ceil(max_n / 128)
     int chunks_per_q;        // ceil(qtiles / 8)
     // nullable: per query, the largest score key (order_key) of every group of 32
@@ -84,21 +86,31 @@ __host__ __device__ constexpr int aux_floats() {
     return HI + kChunkTiles * kTileRows;
 }
 
+// Bytes of one tile of 128 key rows of DI e4m3.
+template <int DI>
+__host__ __device__ constexpr int tile_bytes() {
+    return kTileRows * DI;
+}
+
+// HI: MMA width (heads, padded); DI: indexer dim (MMA K total, bytes per key row).
 // PAGED: the key rows come through the block table (a separate instantiation, so the
 // contiguous kernel carries no block-table code).
-template <int HI, bool PAGED>
+template <int HI, int DI, bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                       const __grid_constant__ CUtensorMap tmap_q, const IdxArgs a) {
     using namespace sm100;
-    constexpr int kQBytes = HI * kDI;
+    static_assert(DI == 64 || DI == 128, "indexer dim 64 or 128");
+    constexpr int kTileBytes = tile_bytes<DI>();
+    constexpr int kGroupBytes = kGroupTiles * kTileBytes;
+    constexpr int kQBytes = HI * DI;
     constexpr int kAuxFloats = aux_floats<HI>();
     constexpr uint32_t kIdesc = instr_desc(0, 0, kTileRows, HI);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~uintptr_t(1023));
-    uint8_t* sA = smem;                                  // [kStages][kGroupTiles][128 x 128]
-    uint8_t* sB = sA + kStages * kGroupBytes;            // [2][HI x 128]
+    uint8_t* sA = smem;                                  // [kStages][kGroupTiles][128 x DI]
+    uint8_t* sB = sA + kStages * kGroupBytes;            // [2][HI x DI]
     float* aux = reinterpret_cast<float*>(sB + 2 * kQBytes);   // [kAux][kAuxFloats]
     uint64_t* bars = reinterpret_cast<uint64_t*>(aux + kAux * kAuxFloats);
     uint64_t* full = bars;                               // [kStages]
@@ -153,6 +165,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(tmem_base_smem, tmem_cols<HI>());
         tmem_relinquish();
     }
+    if (a.hreal < HI) {
+        // the padded heads' B rows stay zero: the copies write rows [0, hreal) only.  The
+        // swizzle permutes 16-byte pieces within a row, so rows [hreal, HI) are exactly the
+        // bytes from hreal * DI on in each buffer.
+        for (int u = threadIdx.x; u < 2 * (HI - a.hreal) * DI / 16; u += kThreads) {
+            const int per = (HI - a.hreal) * DI / 16;
+            const int bb = u / per, o = u % per;
+            reinterpret_cast<uint4*>(sB + bb * kQBytes + a.hreal * DI)[o] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -181,8 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (x.q != cur_q) {
                     const int bb = nq & 1;
                     if (!mbar_wait(&bempty[bb], ((nq >> 1) & 1) ^ 1, abort_flag, a.st)) break;
-                    mbar_arrive_expect_tx(&bfull[bb], kQBytes);
-                    tma_load_2d(sB + bb * kQBytes, &tmap_q, &bfull[bb], 0, x.q * HI);
+                    mbar_arrive_expect_tx(&bfull[bb], (uint32_t)(a.hreal * DI));
+                    tma_load_2d(sB + bb * kQBytes, &tmap_q, &bfull[bb], 0, x.q * a.hreal);
                     nq++;
                     cur_q = x.q;
                 }
@@ -202,12 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         int32_t rows[kGroupTiles][kTilePages];
                         int nb = 0;
                         for (int j = 0; j < gt; j++) nb += tile_pages(a, x, x.tile0 + g0 + j, rows[j]);
-                        mbar_arrive_expect_tx(&full[stage], (uint32_t)nb * (kPageRows * kDI));
+                        mbar_arrive_expect_tx(&full[stage], (uint32_t)nb * (kPageRows * DI));
                         for (int j = 0; j < gt; j++)
 #pragma unroll
                             for (int p = 0; p < kTilePages; p++)
                                 if (rows[j][p] >= 0)
-                                    tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes + p * (kPageRows * kDI),
+                                    tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes + p * (kPageRows * DI),
                                                 &tmap_k, &full[stage], 0, rows[j][p]);
                     }
                     ng++;
@@ -248,7 +271,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int bb = nq & 1;
                     if (!mbar_wait(&bfull[bb], (nq >> 1) & 1, abort_flag, a.st)) break;
                     tc_fence_after();
-                    bdesc = smem_desc_k_sw128(sB + bb * kQBytes);
+                    if constexpr (DI == 128)
+                        bdesc = smem_desc_k_sw128(sB + bb * kQBytes);
+                    else
+                        bdesc = smem_desc_k_sw64(sB + bb * kQBytes);
                     nq++;
                     cur_q = x.q;
                 }
@@ -261,10 +287,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t adesc = smem_desc_k_sw128(sA + stage * kGroupBytes);
+                    const uint64_t adesc = DI == 128 ? smem_desc_k_sw128(sA + stage * kGroupBytes)
+                                                     : smem_desc_k_sw64(sA + stage * kGroupBytes);
                     const uint32_t d0 = tmem_base + (uint32_t)(set * kGroupTiles * HI);
 #pragma unroll
-                    for (int kk = 0; kk < kDI / 32; kk++) {   // K = 32 e4m3 = 32 bytes per MMA
+                    for (int kk = 0; kk < DI / 32; kk++) {   // K = 32 e4m3 = 32 bytes per MMA
 #pragma unroll
                         for (int j = 0; j < kGroupTiles; j++)
                             if (j < gt)
@@ -297,7 +324,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             float* ks_s = ws_s + HI;
 #pragma unroll
             for (int h = lane; h < HI; h += 32)
-                ws_s[h] = __ldg(a.w + (int64_t)x.q * HI + h) * __ldg(a.qs + (int64_t)x.q * HI + h);
+                ws_s[h] = h < a.hreal ? __ldg(a.w + (int64_t)x.q * a.hreal + h) *
+                                            __ldg(a.qs + (int64_t)x.q * a.hreal + h)
+                                      : 0.f;
             // all of the item's key scales in flight at once (one memory latency per item)
             const int64_t e0 = (int64_t)x.tile0 * kTileRows;
             const int nrows = x.ntiles * kTileRows;
@@ -416,9 +445,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int HI>
+template <int HI, int DI>
 size_t smem_bytes() {
-    return 1024 + kStages * kGroupBytes + 2 * HI * kDI + kAux * aux_floats<HI>() * sizeof(float) +
+    return 1024 + kStages * kGroupTiles * tile_bytes<DI>() + 2 * HI * DI + kAux * aux_floats<HI>() * sizeof(float) +
            (2 * kStages + 4 + 2 * kAccSets + 2 * kAux + 1) * 8 + 16 + kMaxItems * sizeof(Item);
 }
 
@@ -441,16 +470,18 @@ EncodeFn get_encode_fn() {
     return fn;
 }
 
-// Row-major [rows x 128] byte matrix, boxes of box_rows x 128 bytes, 128-byte swizzle.
-bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows) {
+// Row-major [rows x dI] byte matrix (dI 64 or 128), boxes of box_rows x dI bytes, swizzled
+// by the row width (128- or 64-byte swizzle).
+bool make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows, int dI) {
     EncodeFn enc = get_encode_fn();
     if (!enc) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)kDI};
-    const cuuint32_t box[2] = {(cuuint32_t)kDI, box_rows};
+    const cuuint64_t dims[2] = {(cuuint64_t)dI, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)dI};
+    const cuuint32_t box[2] = {(cuuint32_t)dI, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               dI == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
@@ -466,15 +497,15 @@ int num_sms() {
     return n;
 }
 
-template <int HI>
+template <int HI, int DI>
 cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const IdxArgs& args,
                       cudaStream_t stream) {
     CUtensorMap mk, mq;
-    if (!make_rows_map(&mk, kI, (uint64_t)args.ent_rows, args.er.bt ? kPageRows : kTileRows) ||
-        !make_rows_map(&mq, qI, (uint64_t)args.Q * HI, HI))
+    if (!make_rows_map(&mk, kI, (uint64_t)args.ent_rows, args.er.bt ? kPageRows : kTileRows, DI) ||
+        !make_rows_map(&mq, qI, (uint64_t)args.Q * args.hreal, (uint32_t)args.hreal, DI))
         return cudaErrorInvalidValue;
-    const size_t sm = smem_bytes<HI>();
-    auto kernel = args.er.bt ? indexer_tc_kernel<HI, true> : indexer_tc_kernel<HI, false>;
+    const size_t sm = smem_bytes<HI, DI>();
+    auto kernel = args.er.bt ? indexer_tc_kernel<HI, DI, true> : indexer_tc_kernel<HI, DI, false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)sm);
     if (e != cudaSuccess) return e;
@@ -486,15 +517,16 @@ cudaError_t launch_hi(const uint8_t* qI, const uint8_t* kI, const IdxArgs& args,
 
 }  // namespace
 
+// Any head count 1..64 (run on the MMA width 16, 32 or 64 at or above it), dim 64 or 128.
 bool indexer_tc_supported(int HI, int dI) {
-    return dI == kDI && (HI == 16 || HI == 32 || HI == 64);
+    return (dI == 64 || dI == 128) && HI >= 1 && HI <= 64;
 }
 
 cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w,
                               const uint8_t* kI, const float* ks, int64_t ent_rows,
                               const int64_t* seq_len, const EntryRows& er,
                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
-                              int m, int max_n, float* scores, int64_t ld, int32_t* st,
+                              int dI, int m, int max_n, float* scores, int64_t ld, int32_t* st,
                               cudaStream_t stream, uint32_t* gmax, int64_t ld_g) {
     if (Q == 0 || max_n == 0 || ent_rows == 0) return cudaSuccess;
     IdxArgs args;
@@ -513,15 +545,24 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
     args.B = B;
     args.m = m;
     args.max_n = max_n;
+    args.hreal = HI;
     args.gmax = gmax;
     args.ld_g = ld_g;
     args.qtiles = (max_n + kTileRows - 1) / kTileRows;
     args.chunks_per_q = (args.qtiles + kChunkTiles - 1) / kChunkTiles;
-    switch (HI) {
-        case 64: return launch_hi<64>(qI, kI, args, stream);
-        case 32: return launch_hi<32>(qI, kI, args, stream);
-        case 16: return launch_hi<16>(qI, kI, args, stream);
-        default: return cudaErrorInvalidValue;
+    if (!indexer_tc_supported(HI, dI)) return cudaErrorInvalidValue;
+    const int width = HI <= 16 ? 16 : HI <= 32 ? 32 : 64;   // MMA N
+    if (dI == 128) {
+        switch (width) {
+            case 64: return launch_hi<64, 128>(qI, kI, args, stream);
+            case 32: return launch_hi<32, 128>(qI, kI, args, stream);
+            default: return launch_hi<16, 128>(qI, kI, args, stream);
+        }
+    }
+    switch (width) {
+        case 64: return launch_hi<64, 64>(qI, kI, args, stream);
+        case 32: return launch_hi<32, 64>(qI, kI, args, stream);
+        default: return launch_hi<16, 64>(qI, kI, args, stream);
     }
 }
 

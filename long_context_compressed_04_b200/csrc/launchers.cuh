@@ -48,7 +48,6 @@ cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
 // Kernel kinds for launch accounting (names in prof.cu).
 enum KernelKind {
     kKCompress = 0,
-    kKIndexerSimt,
     kKTopk,
     kKAttnSimt,
     kKIndexerTc,
@@ -101,18 +100,12 @@ cudaError_t launch_compress(int span, const void* kv, const void* gate, const fl
                             const int32_t* item_seq, const int32_t* item_ent, int64_t n_items,
                             int B, int m, int D, int fmt, float theta, float eps, void* entries,
                             int32_t* st, cudaStream_t stream);
-cudaError_t launch_indexer_simt(const uint8_t* qI, const float* qs, const float* w,
-                                const uint8_t* kI, const float* ks, int64_t ent_rows,
-                                const int64_t* seq_len,
-                                const EntryRows& er, const int32_t* q_seq, const int32_t* q_pos, int Q, int B,
-                                int HI, int dI, int m, int max_n, float* scores, int64_t ld,
-                                int32_t* st, cudaStream_t stream);
 bool indexer_tc_supported(int HI, int dI);
 cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w,
                               const uint8_t* kI, const float* ks, int64_t ent_rows,
                               const int64_t* seq_len, const EntryRows& er,
                               const int32_t* q_seq, const int32_t* q_pos, int Q, int B, int HI,
-                              int m, int max_n, float* scores, int64_t ld, int32_t* st,
+                              int dI, int m, int max_n, float* scores, int64_t ld, int32_t* st,
                               cudaStream_t stream, uint32_t* gmax = nullptr, int64_t ld_g = 0);
 bool indexer_fp4_supported(int HI, int dI);
 cudaError_t launch_indexer_fp4(const uint8_t* qI, const uint8_t* qI_sf, const float* w,

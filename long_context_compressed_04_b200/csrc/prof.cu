@@ -49,7 +49,7 @@ cudaEvent_t take_event() {
 }  // namespace
 
 const char* kernel_name(int kind) {
-    static const char* names[kKernelKinds] = {"compress", "indexer_score_simt", "topk_radix",
+    static const char* names[kKernelKinds] = {"compress", "topk_radix",
                                               "attn_simt", "indexer_score_tc", "attn_tc",
                                               "attn_combine", "attn576_tc", "topk_merge",
                                               "cp_candidates", "cp_pack_rows",

@@ -35,6 +35,7 @@ def _random_idx(wl, seed, pad=0):
 
 @pytest.mark.parametrize("H,D,fmt,k,T", [
     (16, 128, 0, 64, [4096]),                      # CSA decode 4K shape
+    (16, 128, 0, 512, [7001, 3000, 2100]),         # 16 heads, clusters of several CTAs
     (64, 128, 0, 512, [7001, 3000, 2100]),         # CSA decode, ragged, k = 512
     (64, 128, 0, 1024, [9001, 4000, 300]),         # k = 1024: one CTA per query combines
     (64, 128, 0, 2048, [20003, 9000]),             # all 64 heads (the prefill kernel shape)
@@ -55,9 +56,11 @@ def test_sparse_attention(H, D, fmt, k, T):
     _orc.assert_out_close(buf.out, ref)
 
 
-@pytest.mark.parametrize("T", [[128 * 40 + 77, 128 * 7], [300], [128 * 2500 + 77, 130]])
-def test_dense_hca_attention(T):
-    wl = synth.make_workload("t", B=len(T), T=T, D=128, H=64, m=128, span=128, seed=32,
+@pytest.mark.parametrize("H,T", [(64, [128 * 40 + 77, 128 * 7]), (64, [300]),
+                                 (64, [128 * 2500 + 77, 130]), (16, [128 * 300 + 5, 1000])])
+def test_dense_hca_attention(H, T):
+    # 16 heads run on the 64-head tile with zero heads added
+    wl = synth.make_workload("t", B=len(T), T=T, D=128, H=H, m=128, span=128, seed=32,
                              device=DEV)
     buf, rows = _with_oracle_entries(wl)
     pipeline.attend(wl, buf)

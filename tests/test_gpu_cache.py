@@ -25,10 +25,11 @@ def _contig_offsets(n):
     return off
 
 
-@pytest.mark.parametrize("D,H,fmt", [(576, 128, 1), (128, 64, 0)])
-def test_paged_ring_decode_matches_contiguous_bitwise(D, H, fmt):
+@pytest.mark.parametrize("D,H,fmt,H_I,d_I", [(576, 128, 1, 64, 128), (128, 64, 0, 64, 128),
+                                             (128, 16, 0, 4, 64)])
+def test_paged_ring_decode_matches_contiguous_bitwise(D, H, fmt, H_I, d_I):
     g = torch.Generator(device=DEV).manual_seed(81)
-    B, S, k, W, H_I, d_I, ring = 4, 70, 64, 128, 64, 128, 128
+    B, S, k, W, ring = 4, 70, 64, 128, 128
     T0 = [3001, 777, 4099, 130]
     Tmax = [t + S for t in T0]
     nEmax = [t // 4 for t in Tmax]

@@ -42,9 +42,11 @@ def test_decode_4k_shape_bit_exact():
     _exact(synth.csa_decode_4k(device=DEV))
 
 
-@pytest.mark.parametrize("HI,dI,k", [(64, 128, 512), (4, 64, 64), (16, 128, 100)])
+@pytest.mark.parametrize("HI,dI,k", [(64, 128, 512), (4, 64, 64), (16, 128, 100), (1, 128, 64),
+                                     (20, 64, 100), (40, 128, 256), (64, 64, 512)])
 def test_ragged_batch_bit_exact(HI, dI, k):
-    # visible counts 1500, 4000, 300 (< k for some shapes: padded with -1), 7
+    # visible counts 1500, 4000, 300 (< k for some shapes: padded with -1), 7.  Head counts
+    # other than 16, 32 and 64 run on the next MMA width with zero heads added.
     wl = synth.make_workload("t", B=4, T=[6003, 16000, 1201, 29], D=128, H=16, m=4, span=8,
                              H_I=HI, d_I=dI, k=k, seed=21, device=DEV)
     idx = _exact(wl)
