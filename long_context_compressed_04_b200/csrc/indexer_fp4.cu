@@ -66,6 +66,7 @@ struct Fp4Args {
     int qtiles;
     int chunks_per_q;
     int bf16;                // round each score to BF16 before storing / selecting
+    int keys_once;           // no more queries than sequences (decode): each key row is read once
     uint32_t* gmax;          // nullable: group maxima, as in the FP8 indexer
     int64_t ld_g;
 };
@@ -237,6 +238,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ephase = 0;
             int nq = 0, cur_q = -1, ng = 0;
             bool ok = true;
+            // key rows read once (decode) take the evict-first policy: the key tiles
+            // leave L2 first, and the score rows and group maxima the top-k reads next stay
+            const uint64_t pol = l2_policy(a.keys_once != 0);
             for (int ii = 0; ii < n_my && ok; ii++) {
                 Item x;
                 if (!get_item(a, v0, v1, ii, x, false)) continue;
@@ -257,9 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (!PAGED) {
                         mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
                         for (int j = 0; j < gt; j++)
-                            tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k,
-                                        &full[stage], 0,
-                                        (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows));
+                            tma_load_2d_hint(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k,
+                                             &full[stage], 0,
+                                             (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows),
+                                             pol);
                     } else {
                         int32_t rows[kGroupTiles][kTilePages];
                         int nb = 0;
@@ -269,9 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int p = 0; p < kTilePages; p++)
                                 if (rows[j][p] >= 0)
-                                    tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes +
-                                                    p * (kPageRows * kRowBytes),
-                                                &tmap_k, &full[stage], 0, rows[j][p]);
+                                    tma_load_2d_hint(sA + stage * kGroupBytes + j * kTileBytes +
+                                                         p * (kPageRows * kRowBytes),
+                                                     &tmap_k, &full[stage], 0, rows[j][p], pol);
                     }
                     ng++;
                     if (++stage == kStages) {
@@ -648,6 +653,7 @@ cudaError_t launch_indexer_fp4(const uint8_t* qI, const uint8_t* qI_sf, const fl
     args.B = B;
     args.m = m;
     args.max_n = max_n;
+    args.keys_once = Q <= B;
     args.bf16 = bf16;
     args.gmax = gmax;
     args.ld_g = ld_g;

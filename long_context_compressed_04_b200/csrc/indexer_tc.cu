@@ -64,6 +64,7 @@ struct IdxArgs {
     int32_t* st;
     int Q, B, m, max_n;
     int hreal;               // heads of the call (<= HI; the rest are zero padding)
+    int keys_once;           // no more queries than sequences (decode): each key row is read once
     int qtiles;              // virtual tiles per query: ceil(max_n / 128)
     int chunks_per_q;        // ceil(qtiles / 8)
     // nullable: per query, the largest score key (order_key) of every group of 32
@@ -198,6 +199,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ephase = 0;
             int nq = 0, cur_q = -1, ng = 0;   // queries and groups issued
             bool ok = true;
+            // key rows read once (decode) take the evict-first policy: the key tiles
+            // leave L2 first, and the score rows and group maxima the top-k reads next stay
+            const uint64_t pol = l2_policy(a.keys_once != 0);
             for (int ii = 0; ii < n_my && ok; ii++) {
                 Item x;
                 if (!get_item(a, v0, v1, ii, x, false)) continue;
@@ -218,8 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if constexpr (!PAGED) {
                         mbar_arrive_expect_tx(&full[stage], gt * kTileBytes);
                         for (int j = 0; j < gt; j++)
-                            tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k, &full[stage], 0,
-                                        (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows));
+                            tma_load_2d_hint(sA + stage * kGroupBytes + j * kTileBytes, &tmap_k, &full[stage], 0,
+                                             (int32_t)(x.row0 + (int64_t)(x.tile0 + g0 + j) * kTileRows), pol);
                     } else {
                         // block table: each tile in blocks of kPageRows rows (the map's box)
                         int32_t rows[kGroupTiles][kTilePages];
@@ -230,8 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                             for (int p = 0; p < kTilePages; p++)
                                 if (rows[j][p] >= 0)
-                                    tma_load_2d(sA + stage * kGroupBytes + j * kTileBytes + p * (kPageRows * DI),
-                                                &tmap_k, &full[stage], 0, rows[j][p]);
+                                    tma_load_2d_hint(sA + stage * kGroupBytes + j * kTileBytes + p * (kPageRows * DI),
+                                                     &tmap_k, &full[stage], 0, rows[j][p], pol);
                     }
                     ng++;
                     if (++stage == kStages) {
@@ -546,6 +550,7 @@ cudaError_t launch_indexer_tc(const uint8_t* qI, const float* qs, const float* w
     args.m = m;
     args.max_n = max_n;
     args.hreal = HI;
+    args.keys_once = Q <= B;
     args.gmax = gmax;
     args.ld_g = ld_g;
     args.qtiles = (max_n + kTileRows - 1) / kTileRows;
