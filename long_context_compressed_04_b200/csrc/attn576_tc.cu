@@ -16,8 +16,7 @@
 // while earlier ones are in the tensor cores.
 //   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once (as
 //              fp16, scaled by 2^-s if needed, see below); the window tile; then, after the
-//              wait, the index row and a bulk L2 prefetch of every entry row this rank
-//              gathers; per tile, 4 threads per key row convert their quarter of the FP8 row
+//              wait, the index row; per tile, 4 threads per key row convert their quarter of the FP8 row
 //              (e4m3 -> fp16 exactly, times the block scale) into a 128-byte-swizzled tile
 //              of 9 blocks of 64 channels; the rows of tile j + 2 are loaded into registers
 //              while tile j is converted (two register sets).
@@ -25,10 +24,11 @@
 //              operands) straight into the TMEM accumulator: channels 0-255 in TMEM lanes
 //              0-15 of each quarter, 256-511 in lanes 16-31, 512-575 in lanes 0-15 again
 //              (N = 256 + 256 + 64), V being the key tile read MN-major.
-//   warps 9-10 lane 0 issues S = Q K^T of the even (warp 9) or odd (warp 10) tiles
-//              (M = 64 heads, N = 32 keys, 36 K steps of 16 channels) into its own S
-//              buffer, as 4 partial accumulators (see s_col): one MMA costs its issuing
-//              thread tens of cycles whatever its shape, so S has two issuers.
+//   warps 9-10 lane 0 issues S = Q K^T of every tile (M = 64 heads, N = 32 keys, 36 K
+//              steps of 16 channels) into S buffer j % 2 as 4 partial accumulators (see
+//              s_col), warp 9 partials 0 and 2, warp 10 partials 1 and 3: one MMA costs its
+//              issuing thread tens of cycles whatever its shape, so S has two issuers, and
+//              both on one tile halve its latency.
 //   warps 5-8  online softmax in the log2 domain, one head row per lane, weights by
 //              ex2.approx of one FMA per key: P as fp16 into shared memory; the running
 //              maximum is a reference that moves only when a tile's maximum exceeds it by
@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             mbar_init(&kfree[i], 1);
         }
         for (int i = 0; i < 2; i++) {
-            mbar_init(&sfull[i], 1);
+            mbar_init(&sfull[i], 2);   // both S issuers commit every tile
             mbar_init(&sfree[i], 4);
             mbar_init(&pfull[i], 4);
             mbar_init(&pfree[i], 1);
@@ -487,9 +487,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         }
         // ---- the index row: the first read of another kernel's output ----
         // Every loader thread waits for the previous grid (the top-k writes the index row,
-        // compression the entries), then the row is staged in shared memory and every entry
-        // row this rank will gather is prefetched into L2 at once (one bulk prefetch per
-        // 656-byte row), so the gathers below meet L2 rather than HBM.
+        // compression the entries), then the row is staged in shared memory.  (Bulk L2
+        // prefetches of the entry rows, one per row through the copy engine, took longer to
+        // issue than the gathers they were to speed up.)
         pdl_wait();
         if (tid == 0) pdl_trigger();
         if (valid) {
@@ -515,24 +515,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             }
         }
         asm volatile("bar.sync 3, 128;" ::: "memory");
-        if (valid) {
-            for (int u = tid; u < nloc * kTK; u += 128) {
-                const int jg = rank + kCl * (u / kTK);
-                const int v = (jg - n_wt) * kTK + u % kTK;
-                if (jg < n_wt || v >= a.k) continue;
-                const int e = sidx[v];
-                if (e >= 0 && e < n_vis) {
-                    const int64_t re = a.er.bt ? a.er.row(b, e) : row0 + e;
-                    if (re >= 0 && re < a.ent_rows)
-                        prefetch_l2_bulk(a.entries + re * (int64_t)kRowBytes, kRowBytes);
-                }
-            }
-        }
         // ---- the selected entries ----
         // Each thread converts its quarter of a key row from registers (e4m3 x scale ->
         // fp16, the bf16 RoPE channels to fp16) into the key buffer.  Two register sets: the
         // loads of tile j + 2 are issued as soon as tile j is converted, so every gather
-        // has two tiles' time to arrive (the rows are also being prefetched into L2).
+        // has two tiles' time to arrive.
         const int j0 = has_win ? 1 : 0;
         EntryQuarter exa, exb;
         exa.valid = exb.valid = false;
@@ -584,19 +571,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         if (lane == 0 && nloc > 0) {
             // ---------------- MMA issuers ----------------
             // One tcgen05.mma costs its issuing thread tens of cycles whatever its shape, and
-            // S takes 36 per tile: the S of even tiles is issued by warp kFirstSWarp, of odd
-            // tiles by warp kFirstSWarp + 1 (each owns one S buffer), and P V by warp 4.
+            // S takes 36 per tile: of every tile, warp kFirstSWarp issues the K steps of
+            // partials 0 and 2, warp kFirstSWarp + 1 those of partials 1 and 3 (a partial's
+            // steps always from one thread, in order), into S buffer j % 2; P V by warp 4.
             // K buffer kb is released by P V's commit: the tile's S was complete before its P
             // (hence its P V) existed.
             bool ok = true;
             if (warp >= kFirstSWarp) {
-                const int e = warp - kFirstSWarp;   // S buffer and tile parity
+                const int e = warp - kFirstSWarp;   // partials e and e + 2 of every tile
                 ok = mbar_wait(qfull, 0, abort_flag, a.st);
                 tc_fence_after();
-                for (int j = e; j < nloc && ok; j += 2) {
-                    const int kb = j % kKBuf;
+                for (int j = 0; j < nloc && ok; j++) {
+                    const int kb = j % kKBuf, sb = j & 1;
                     if (!mbar_wait(&kfull[kb], (j / kKBuf) & 1, abort_flag, a.st) ||
-                        !mbar_wait(&sfree[e], ((j >> 1) & 1) ^ 1, abort_flag, a.st)) {
+                        !mbar_wait(&sfree[sb], ((j >> 1) & 1) ^ 1, abort_flag, a.st)) {
                         ok = false;
                         break;
                     }
@@ -607,11 +595,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                         const uint64_t ad = smem_desc_k_sw128(sQ + cb * kQBlk);
                         const uint64_t bd = smem_desc_k_sw128(tile + cb * kKBlk);
 #pragma unroll
-                        for (int kk = 0; kk < 4; kk++)   // K = 16 fp16 = 32 bytes, partial kk
-                            mma_f16(tmem + s_col(e, kk), ad + 2 * kk, bd + 2 * kk, kIdescS,
+                        for (int kk = e; kk < 4; kk += 2)   // K = 16 fp16 = 32 bytes, partial kk
+                            mma_f16(tmem + s_col(sb, kk), ad + 2 * kk, bd + 2 * kk, kIdescS,
                                     cb ? 1u : 0u);
                     }
-                    mma_commit(&sfull[e]);
+                    mma_commit(&sfull[sb]);
                 }
             } else {
                 for (int j = 0; j < nloc && ok; j++) {
