@@ -16,10 +16,12 @@
 // while earlier ones are in the tensor cores.
 //   warps 0-3  loaders: the query's 64 head rows RoPEd at t into shared memory once (as
 //              fp16, scaled by 2^-s if needed, see below); the window tile; then, after the
-//              wait, the index row; per tile, 4 threads per key row convert their quarter of the FP8 row
-//              (e4m3 -> fp16 exactly, times the block scale) into a 128-byte-swizzled tile
-//              of 9 blocks of 64 channels; the rows of tile j + 2 are loaded into registers
-//              while tile j is converted (two register sets).
+//              wait, the index row; per tile, 4 threads per key row convert their quarter
+//              of the FP8 row (16 channels of every 64, so that a warp load reads 64
+//              contiguous bytes of each of 8 rows; e4m3 -> fp16 exactly, times the block
+//              scale) into a 128-byte-swizzled tile of 9 blocks of 64 channels; the rows of
+//              tile j + 2 are loaded into registers while tile j is converted (two
+//              register sets).
 //   warp 4     TMEM allocation; lane 0 issues O += P V (tcgen05.mma kind::f16, fp16
 //              operands) straight into the TMEM accumulator: channels 0-255 in TMEM lanes
 //              0-15 of each quarter, 256-511 in lanes 16-31, 512-575 in lanes 0-15 again
@@ -192,12 +194,14 @@ __device__ __forceinline__ void dequant16(uint4 c, uint32_t sc2, uint4& lo, uint
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// One loader thread's quarter of a selected entry row, in registers: fp8 channels
-// [128 qt, 128 qt + 128) with their scale, RoPE channels [16 qt, 16 qt + 16).
+// One loader thread's quarter of a selected entry row, in registers: the fp8 channels
+// [64 u + 16 qt, 64 u + 16 qt + 16) for u = 0..7, the row's four block scales, and the RoPE
+// channels [16 qt, 16 qt + 16).  The four threads of a row read 64 contiguous bytes per
+// load, so one warp load touches 8 lines (of the warp's 8 rows) rather than 32.
 struct EntryQuarter {
     uint4 f[8];
     uint4 rope[2];
-    float sc;
+    float4 sc;
     bool valid;
 };
 
@@ -220,11 +224,11 @@ __device__ __forceinline__ void fetch_entry(const A576Args& a, const int32_t* si
     if (x.valid) {
         const uint8_t* er = a.entries + re * (int64_t)kRowBytes;
 #pragma unroll
-        for (int u = 0; u < 8; u++) x.f[u] = *reinterpret_cast<const uint4*>(er + 128 * qt + 16 * u);
+        for (int u = 0; u < 8; u++) x.f[u] = *reinterpret_cast<const uint4*>(er + 64 * u + 16 * qt);
 #pragma unroll
         for (int u = 0; u < 2; u++)
             x.rope[u] = *reinterpret_cast<const uint4*>(er + 528 + 32 * qt + 16 * u);
-        x.sc = *reinterpret_cast<const float*>(er + 512 + 4 * qt);
+        x.sc = *reinterpret_cast<const float4*>(er + 512);
     }
 }
 
@@ -517,7 +521,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         asm volatile("bar.sync 3, 128;" ::: "memory");
         // ---- the selected entries ----
         // Each thread converts its quarter of a key row from registers (e4m3 x scale ->
-        // fp16, the bf16 RoPE channels to fp16) into the key buffer.  Two register sets: the
+        // fp16, the bf16 RoPE channels to fp16) into the key buffer: the 8 lanes of two
+        // rows store to 8 distinct 16-byte columns of the swizzle (no bank conflict).  Two register sets: the
         // loads of tile j + 2 are issued as soon as tile j is converted, so every gather
         // has two tiles' time to arrive.
         const int j0 = has_win ? 1 : 0;
@@ -534,12 +539,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             if (j >= kKBuf && !mbar_wait_warp(&kfree[kb], ((j / kKBuf) & 1) ^ 1, abort_flag, a.st))
                 return false;
             const bool vrow = ex.valid;
-            const uint32_t sc2 = vrow ? pack_f16x2(ex.sc, ex.sc) : 0u;
+            const float scs[4] = {ex.sc.x, ex.sc.y, ex.sc.z, ex.sc.w};
 #pragma unroll
             for (int u = 0; u < 8; u++) {
                 uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
-                if (vrow) dequant16(ex.f[u], sc2, lo, hi);
-                const int d0 = 128 * qt + 16 * u;
+                if (vrow) dequant16(ex.f[u], pack_f16x2(scs[u >> 1], scs[u >> 1]), lo, hi);
+                const int d0 = 64 * u + 16 * qt;
                 *cell8(tile, kKBlk, kr, d0) = lo;
                 *cell8(tile, kKBlk, kr, d0 + 8) = hi;
             }
