@@ -344,7 +344,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
         const int tid = threadIdx.x;
         const int r = tid >> 1, hf = tid & 1;        // key (or head) row, half of it
         bool ok = true;
-        if (valid) {
+        // A rank without tiles needs no Q tile; its softmax warps write its (empty) partial
+        // state over Q / K at once, so nothing else may be written there.
+        if (valid && nloc > 0) {
             // q head row r at t: channels [288 hf, 288 hf + 288), RoPE on 512..575.  Pass 1:
             // the largest |q| of the CTA's 64 heads; if it could leave the fp16 range after
             // the rotation (which grows a pair's component by at most sqrt 2), every q value
@@ -489,51 +491,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
             }
             publish(0, vrow);
         }
-        // ---- the index row: the first read of another kernel's output ----
-        // Every loader thread waits for the previous grid (the top-k writes the index row,
-        // compression the entries), then the row is staged in shared memory.  (Bulk L2
-        // prefetches of the entry rows, one per row through the copy engine, took longer to
-        // issue than the gathers they were to speed up.)
-        pdl_wait();
-        if (tid == 0) pdl_trigger();
-        if (valid) {
-            // all of the row's loads in flight at once (16-byte loads when aligned)
-            const int32_t* src = a.idx + (int64_t)qi * a.k;
-            if ((a.k & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
-                const int n4 = a.k >> 2;   // <= kMaxK / 4 = 4 per thread
-                int4 v[kMaxK / 4 / 128];
-#pragma unroll
-                for (int u = 0; u < kMaxK / 4 / 128; u++)
-                    if (tid + 128 * u < n4) v[u] = reinterpret_cast<const int4*>(src)[tid + 128 * u];
-#pragma unroll
-                for (int u = 0; u < kMaxK / 4 / 128; u++)
-                    if (tid + 128 * u < n4) reinterpret_cast<int4*>(sidx)[tid + 128 * u] = v[u];
-            } else {
-                int v[kMaxK / 128];
-#pragma unroll
-                for (int u = 0; u < kMaxK / 128; u++)
-                    v[u] = tid + 128 * u < a.k ? src[tid + 128 * u] : -1;
-#pragma unroll
-                for (int u = 0; u < kMaxK / 128; u++)
-                    if (tid + 128 * u < a.k) sidx[tid + 128 * u] = v[u];
-            }
-        }
-        asm volatile("bar.sync 3, 128;" ::: "memory");
         // ---- the selected entries ----
         // Each thread converts its quarter of a key row from registers (e4m3 x scale ->
         // fp16, the bf16 RoPE channels to fp16) into the key buffer: the 8 lanes of two
-        // rows store to 8 distinct 16-byte columns of the swizzle (no bank conflict).  Two register sets: the
-        // loads of tile j + 2 are issued as soon as tile j is converted, so every gather
-        // has two tiles' time to arrive.
+        // rows store to 8 distinct 16-byte columns of the swizzle (no bank conflict).  Two
+        // register sets: the loads of tile j + 2 are issued as soon as tile j is converted,
+        // so every gather has two tiles' time to arrive.
+        // When the rank has entry tiles, the loop starts with two dry steps (j = j0 - 2,
+        // j0 - 1), before the wait: they convert zeros through the loop's own code, one per
+        // register set, into the spare key buffers 1 and 2 and publish nothing, so that the
+        // tiles after the wait do not run from a cold instruction cache (the previous
+        // kernels evict the code from L2).  Such a rank writes its partial state over the
+        // buffers only after all of its MMAs, hence after the dry steps.
         const int j0 = has_win ? 1 : 0;
         EntryQuarter exa, exb;
-        exa.valid = exb.valid = false;
+#pragma unroll
+        for (int u = 0; u < 8; u++) exa.f[u] = exb.f[u] = make_uint4(0u, 0u, 0u, 0u);
+        exa.rope[0] = exa.rope[1] = exb.rope[0] = exb.rope[1] = make_uint4(0u, 0u, 0u, 0u);
+        exa.sc = exb.sc = make_float4(0.f, 0.f, 0.f, 0.f);
+        exa.valid = exb.valid = true;
         auto entry_of = [&](int j) { return (rank + kCl * j - n_wt) * kTK + kr; };
-        if (j0 < nloc) fetch_entry(a, sidx, entry_of(j0), n_vis, b, row0, qt, exa);
-        if (j0 + 1 < nloc) fetch_entry(a, sidx, entry_of(j0 + 1), n_vis, b, row0, qt, exb);
         // converts tile j from `ex`, then issues tile j + 2's loads into it
         auto tile_step = [&](int j, EntryQuarter& ex) -> bool {
-            const int kb = j % kKBuf;
+            const bool dry = j < j0;
+            const int kb = dry ? 1 + ((j - j0) & 1) : j % kKBuf;
             uint8_t* tile = sK + kb * kKBytes;
             // this key buffer is free once the P V of the tile kKBuf back has completed
             if (j >= kKBuf && !mbar_wait_warp(&kfree[kb], ((j / kKBuf) & 1) ^ 1, abort_flag, a.st))
@@ -564,12 +545,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn576_tc_kernel(const A576Args 
                 }
                 *cell8(tile, kKBlk, kr, 512 + 16 * qt + 8 * u) = h;
             }
+            if (dry) return true;
             publish(kb, vrow);
             if (j + 2 < nloc) fetch_entry(a, sidx, entry_of(j + 2), n_vis, b, row0, qt, ex);
             return true;
         };
-        for (int j = j0; j < nloc && ok; j += 2) {
-            ok = tile_step(j, exa);
+        const int jend = nloc > j0 ? nloc : j0 + 1;   // the wait below runs in every case
+        for (int j = nloc > j0 ? j0 - 2 : j0; j < jend && ok; j += 2) {
+            if (j == j0) {
+                // ---- the index row: the first read of another kernel's output ----
+                // Every loader thread waits for the previous grid (the top-k writes the
+                // index row, compression the entries), then the row is staged in shared
+                // memory.  (Bulk L2 prefetches of the entry rows, one per row through the
+                // copy engine, took longer to issue than the gathers they were to speed up.)
+                pdl_wait();
+                if (tid == 0) pdl_trigger();
+                if (valid) {
+                    // all of the row's loads in flight at once (16-byte loads when aligned)
+                    const int32_t* src = a.idx + (int64_t)qi * a.k;
+                    if ((a.k & 3) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+                        const int n4 = a.k >> 2;   // <= kMaxK / 4 = 4 per thread
+                        int4 v[kMaxK / 4 / 128];
+#pragma unroll
+                        for (int u = 0; u < kMaxK / 4 / 128; u++)
+                            if (tid + 128 * u < n4) v[u] = reinterpret_cast<const int4*>(src)[tid + 128 * u];
+#pragma unroll
+                        for (int u = 0; u < kMaxK / 4 / 128; u++)
+                            if (tid + 128 * u < n4) reinterpret_cast<int4*>(sidx)[tid + 128 * u] = v[u];
+                    } else {
+                        int v[kMaxK / 128];
+#pragma unroll
+                        for (int u = 0; u < kMaxK / 128; u++)
+                            v[u] = tid + 128 * u < a.k ? src[tid + 128 * u] : -1;
+#pragma unroll
+                        for (int u = 0; u < kMaxK / 128; u++)
+                            if (tid + 128 * u < a.k) sidx[tid + 128 * u] = v[u];
+                    }
+                }
+                asm volatile("bar.sync 3, 128;" ::: "memory");
+                exa.valid = exb.valid = false;
+                if (j0 < nloc) fetch_entry(a, sidx, entry_of(j0), n_vis, b, row0, qt, exa);
+                if (j0 + 1 < nloc) fetch_entry(a, sidx, entry_of(j0 + 1), n_vis, b, row0, qt, exb);
+            }
+            if (j < nloc) ok = tile_step(j, exa);
             if (ok && j + 1 < nloc) ok = tile_step(j + 1, exb);
         }
     } else if (warp == 4 || warp >= kFirstSWarp) {

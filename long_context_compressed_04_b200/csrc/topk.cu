@@ -302,11 +302,22 @@ __device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
     }
     __syncthreads();
     uint32_t kor = 0u, kand = 0xFFFFFFFFu;
-    for (int g = tid; g < G; g += kThreads) {
-        const uint32_t v = qg[g];
-        gk[g] = v;
-        kor |= v;
-        kand &= v;
+    {
+        // 16-byte loads when the row is aligned (all of a thread's loads in flight)
+        const int G4 = (reinterpret_cast<uintptr_t>(qg) & 15) == 0 ? G >> 2 : 0;
+#pragma unroll 4
+        for (int g4 = tid; g4 < G4; g4 += kThreads) {
+            const uint4 v = reinterpret_cast<const uint4*>(qg)[g4];
+            reinterpret_cast<uint4*>(gk)[g4] = v;
+            kor |= v.x | v.y | v.z | v.w;
+            kand &= v.x & v.y & v.z & v.w;
+        }
+        for (int g = 4 * G4 + tid; g < G; g += kThreads) {
+            const uint32_t v = qg[g];
+            gk[g] = v;
+            kor |= v;
+            kand &= v;
+        }
     }
     block_or_and(kor, kand, sh.cor);
     // 2. B: the lower edge of the bin of the k-th largest group key after two 11-bit
@@ -348,22 +359,23 @@ __device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
     if (ng > 2u * (uint32_t)k) return false;
     if (tid == 0) sh.nsel = 0u;
     __syncthreads();
-    // 4. their entries reaching B: 8 slots of 4 entries per group, up to 4 slots per thread
-    // with all of their loads in flight; each thread's passing entries are placed by one
-    // warp scan and one shared atomic per warp
+    // 4. their entries reaching B: 8 slots of 4 entries per group, up to kGatherSlots slots
+    // per thread with all of their loads in flight; each thread's passing entries are
+    // placed by one warp scan and one shared atomic per warp
+    constexpr int kGatherSlots = 4;
     const uint32_t nslots = ng * 8u;
-    for (uint32_t b0 = 0; b0 < nslots; b0 += 4u * kThreads) {
-        uint32_t key[4][4] = {};
-        int e0[4];
+    for (uint32_t b0 = 0; b0 < nslots; b0 += (uint32_t)(kGatherSlots * kThreads)) {
+        uint32_t key[kGatherSlots][4] = {};
+        int e0[kGatherSlots];
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
+        for (int u = 0; u < kGatherSlots; u++) {
             const uint32_t slot = b0 + (uint32_t)tid + (uint32_t)(u * kThreads);
             e0[u] = slot < nslots ? (int)(glist[slot >> 3] * 32u + (slot & 7u) * 4u) : n;
             if (e0[u] < n) load4(s, e0[u], n, vec, key[u]);
         }
         uint32_t pm = 0u;   // bit 4u + z: entry e0[u] + z reaches B
 #pragma unroll
-        for (int u = 0; u < 4; u++)
+        for (int u = 0; u < kGatherSlots; u++)
 #pragma unroll
             for (int z = 0; z < 4; z++)
                 if (e0[u] + z < n && key[u][z] >= B) pm |= 1u << (4 * u + z);
@@ -379,7 +391,7 @@ __device__ bool topk_by_groups(const float* __restrict__ s, bool vec,
         base = __shfl_sync(0xffffffffu, base, 31);
         uint32_t pos = base + inc - cnt;
 #pragma unroll
-        for (int u = 0; u < 4; u++)
+        for (int u = 0; u < kGatherSlots; u++)
 #pragma unroll
             for (int z = 0; z < 4; z++)
                 if ((pm >> (4 * u + z)) & 1u) {
