@@ -58,20 +58,20 @@ WORKLOADS = {
 # sources are byte-identical to the ones captured (sha256 of the files, first 16 hex digits).
 MEASURED_TRAFFIC = {
     ("csa_decode_1m_b8_fp8", "indexer_score_tc"): {
-        "bytes": 285_230_336,
+        "bytes": 281_108_224,
         "files": ["long_context_compressed_04_b200/csrc/indexer_tc.cu",
                   "long_context_compressed_04_b200/csrc/indexer_items.cuh",
                   "long_context_compressed_04_b200/csrc/sm100.cuh",
                   "long_context_compressed_04_b200/csrc/common.cuh"],
-        "sha": "d2050d6bbec42dc8",
+        "sha": "381e8d13a9b6edc5",
     },
     ("csa_decode_1m_b8_mxfp4", "indexer_score_fp4"): {
-        "bytes": 148_762_112,
+        "bytes": 146_638_080,
         "files": ["long_context_compressed_04_b200/csrc/indexer_fp4.cu",
                   "long_context_compressed_04_b200/csrc/indexer_items.cuh",
                   "long_context_compressed_04_b200/csrc/sm100.cuh",
                   "long_context_compressed_04_b200/csrc/common.cuh"],
-        "sha": "cee81c6696c8ce35",
+        "sha": "461b40acd17541e5",
     },
 }
 
